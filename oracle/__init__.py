@@ -1,0 +1,157 @@
+"""Python face of the fp64 CPU oracle (oracle.c).
+
+TEST INFRASTRUCTURE: only tests/, the package smoke entry and bench.py's CPU
+baseline leg import this module.  It shares no code with the CUDA path; inputs
+are numpy arrays of raw 16-bit patterns (np.uint16) plus int32 index arrays.
+Every function cites, in oracle.c, the passage of the pages it follows.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+F16, BF16 = 0, 1
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int, ctypes.c_long
+        L.oracle_decode16.argtypes = [i32, P, i64, P]
+        L.oracle_lora_delta.argtypes = [i32, i32, i32, i32, P, i64, P, P, i64, i32, P, P, P, P,
+                                        P, i32]
+        L.oracle_segments.argtypes = [P, i32, i32, P, P, P, P]
+        L.oracle_merge_requests.argtypes = [P, P, i32, P, P, P]
+        L.oracle_pages_needed.argtypes = [i32, i32, P, P, i64]
+        L.oracle_pages_needed.restype = i64
+        L.oracle_lru_run.argtypes = [i32, P, i64, i32, P, P, P, P, P, P]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def decode16(bits, dtype):
+    bits = _c(bits, np.uint16)
+    out = np.empty(bits.shape, np.float64)
+    rc = lib().oracle_decode16(dtype, _p(bits), bits.size, _p(out))
+    assert rc == 0
+    return out
+
+
+def lora_delta(dtype, x, idx, y_in, ranks, alphas, A_t, B, n_threads=1):
+    """fp64 y_out = y_in + (alpha_a / r_a) * (x_i . A_a) . B_a per token.
+
+    x: (T, d_in) uint16 bits; idx: (T,) int; y_in: (T, d_out) bits or None;
+    ranks: (n_adapters,) int; alphas: (n_adapters,) float; A_t[a]: (r_a, d_in)
+    bits (A transposed, rank-major); B[a]: (r_a, d_out) bits.  A_t[a]/B[a] may
+    be None for adapters no token uses.
+    """
+    x = _c(x, np.uint16)
+    T, d_in = x.shape
+    idx = _c(idx, np.int32)
+    n_ad = len(ranks)
+    d_out = None
+    for b in B:
+        if b is not None and b.size:
+            d_out = b.shape[1]
+            break
+    if y_in is not None:
+        y_in = _c(y_in, np.uint16)
+        d_out = y_in.shape[1]
+    assert d_out is not None, "d_out unknown: pass y_in or one non-empty B"
+    ranks = _c(ranks, np.int32)
+    alphas = _c(alphas, np.float64)
+    keep = []
+    pa = (ctypes.c_void_p * max(n_ad, 1))()
+    pb = (ctypes.c_void_p * max(n_ad, 1))()
+    for a in range(n_ad):
+        if A_t[a] is not None and ranks[a] > 0:
+            at = _c(A_t[a], np.uint16)
+            bb = _c(B[a], np.uint16)
+            assert at.shape == (ranks[a], d_in) and bb.shape == (ranks[a], d_out)
+            keep += [at, bb]
+            pa[a] = at.ctypes.data
+            pb[a] = bb.ctypes.data
+    y_out = np.empty((T, d_out), np.float64)
+    rc = lib().oracle_lora_delta(dtype, T, d_in, d_out, _p(x), d_in, _p(idx),
+                                 _p(y_in) if y_in is not None else None, d_out, n_ad,
+                                 _p(ranks), _p(alphas), ctypes.cast(pa, ctypes.c_void_p),
+                                 ctypes.cast(pb, ctypes.c_void_p), _p(y_out), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_lora_delta: invalid argument")
+    return y_out
+
+
+def segments(idx, max_adapters):
+    """Stable counting sort by adapter: (perm, seg_start, seg_adapter)."""
+    idx = _c(idx, np.int32)
+    T = idx.size
+    perm = np.full(T, -1, np.int32)
+    ss = np.zeros(T + 1, np.int32)
+    sa = np.zeros(max(T, 1), np.int32)
+    S = np.zeros(1, np.int32)
+    rc = lib().oracle_segments(_p(idx), T, max_adapters, _p(perm), _p(ss), _p(sa), _p(S))
+    if rc != 0:
+        raise ValueError("oracle_segments: invalid argument")
+    S = int(S[0])
+    return perm[: ss[S]].copy(), ss[: S + 1].copy(), sa[:S].copy()
+
+
+def merge_requests(req_start, req_adapter):
+    req_start = _c(req_start, np.int32)
+    req_adapter = _c(req_adapter, np.int32)
+    n = req_adapter.size
+    ss = np.zeros(n + 1, np.int32)
+    sa = np.zeros(max(n, 1), np.int32)
+    S = np.zeros(1, np.int32)
+    rc = lib().oracle_merge_requests(_p(req_start), _p(req_adapter), n, _p(ss), _p(sa), _p(S))
+    if rc != 0:
+        raise ValueError("oracle_merge_requests: invalid argument")
+    S = int(S[0])
+    return ss[: S + 1].copy(), sa[:S].copy()
+
+
+def pages_needed(rank, d_in, d_out, page_elems):
+    d_in = _c(d_in, np.int32)
+    d_out = _c(d_out, np.int32)
+    return int(lib().oracle_pages_needed(int(rank), d_in.size, _p(d_in), _p(d_out),
+                                         int(page_elems)))
+
+
+def lru_run(need, capacity, calls):
+    """Run the LRU rules over `calls` (a list of id lists).
+
+    Returns (status[c], resident[c, a] bool, evicted ids per call)."""
+    need = _c(need, np.int64)
+    n_ad = need.size
+    off = np.zeros(len(calls) + 1, np.int32)
+    for c, ids in enumerate(calls):
+        off[c + 1] = off[c] + len(ids)
+    ids = _c(np.concatenate([np.asarray(c, np.int32) for c in calls]) if calls else
+             np.zeros(0, np.int32), np.int32)
+    status = np.zeros(len(calls), np.int32)
+    resident = np.zeros((len(calls), n_ad), np.uint8)
+    evicted = np.zeros(max(n_ad * len(calls), 1), np.int32)
+    eoff = np.zeros(len(calls) + 1, np.int32)
+    lib().oracle_lru_run(n_ad, _p(need), int(capacity), len(calls), _p(off), _p(ids),
+                         _p(status), _p(resident), _p(evicted), _p(eoff))
+    ev = [evicted[eoff[c]:eoff[c + 1]].tolist() for c in range(len(calls))]
+    return status, resident.astype(bool), ev
+
+
+def n_threads_default():
+    return os.cpu_count() or 1

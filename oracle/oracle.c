@@ -1,0 +1,339 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for the heterogeneous-batch paged
+ * LoRA delta.  TEST INFRASTRUCTURE ONLY: nothing in the product path links,
+ * loads or calls this file; only the tests, the package's smoke entry and the
+ * benchmark's CPU-baseline leg do.  It shares no code, header, table or helper
+ * with the CUDA path.
+ *
+ * What it computes (each function cites the passage it follows):
+ *
+ *  oracle_lora_delta   -- y_i <- y_i + (alpha / r_a) * ((x_i . A_a) . B_a) for
+ *                         every token i with adapter a = idx[i] >= 0.
+ *      * the per-token loop with the "adapter id < 0 means skip" rule is the
+ *        Python reference loop of "Paper explainer: S-LoRA" (0h-n0.github.io,
+ *        section "BGMV kernel", bgmv_reference);
+ *      * the scaled, row-vector form Y = X.W0 + (alpha/r).((X.A).B) and the
+ *        order "shrink by A, then expand by B" are from "Multi-LoRA serving:
+ *        S-LoRA, Punica, SGMV, vLLM" (produtoramaxvision.com.br), section on
+ *        how the SGMV kernel executes concurrent adapters.
+ *      The sums are written out in fp64, in ascending index order.  The base
+ *      term X.W0 is outside the path: y_in stands for it.
+ *      Storage: A is held transposed, r rows of d_in (rank-major); B is r rows
+ *      of d_out.  Element values are fp16 or bf16 bit patterns, decoded
+ *      exactly to fp64 by the decoders below.
+ *
+ *  oracle_segments     -- stable counting sort of tokens by adapter id: the
+ *                         segment structure of SGMV ("index vector maps each
+ *                         token to its adapter", same SGMV section).
+ *  oracle_merge_requests -- contiguous request ranges -> segments, merging
+ *                         neighbouring requests that use the same adapter.
+ *  oracle_pages_needed -- pages a rank-r adapter occupies when each of its
+ *                         tensors is laid out flat over fixed-size pages, so that
+ *                         only the last page of each tensor is partly empty
+ *                         (same page's section on the unified paged pool).
+ *  oracle_lru_run      -- least-recently-used residency decisions over a trace
+ *                         of page-in calls ("Paper explainer: S-LoRA", section
+ *                         "Unified Paging", eviction strategy).
+ *
+ * Readings where the pages are silent are listed in the design notes; the ones
+ * that shape this file: rank 0 leaves y unchanged; ties in LRU age go to the
+ * lower adapter id; a page-in call either succeeds whole or changes nothing.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_ERR_ARG 1
+#define OR_ERR_OOM 2
+
+/* ------------------------------------------------------------------------- */
+/* 16-bit float decoding, exact.                                              */
+/* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits.             */
+static double dec_f16(uint16_t h) {
+  int s = (h >> 15) & 1, e = (h >> 10) & 0x1f, f = h & 0x3ff;
+  double v;
+  if (e == 0)
+    v = ldexp((double)f, -24); /* subnormal: f * 2^-14 * 2^-10 */
+  else if (e == 31)
+    v = f ? NAN : INFINITY;
+  else
+    v = ldexp((double)(f + 1024), e - 25); /* (1.f) * 2^(e-15) */
+  return s ? -v : v;
+}
+/* bfloat16: 1 sign, 8 exponent (bias 127), 7 fraction bits. */
+static double dec_bf16(uint16_t b) {
+  int s = (b >> 15) & 1, e = (b >> 7) & 0xff, f = b & 0x7f;
+  double v;
+  if (e == 0)
+    v = ldexp((double)f, -133); /* f * 2^-126 * 2^-7 */
+  else if (e == 255)
+    v = f ? NAN : INFINITY;
+  else
+    v = ldexp((double)(f + 128), e - 134); /* (1.f) * 2^(e-127) */
+  return s ? -v : v;
+}
+static double dec(int dtype, uint16_t v) { return dtype == 1 ? dec_bf16(v) : dec_f16(v); }
+
+/* dtype: 0 = fp16, 1 = bf16 */
+int oracle_decode16(int dtype, const uint16_t* in, long n, double* out) {
+  if (dtype != 0 && dtype != 1) return OR_ERR_ARG;
+  for (long i = 0; i < n; ++i) out[i] = dec(dtype, in[i]);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* The delta.                                                                 */
+typedef struct {
+  int dtype, T, d_in, d_out;
+  const uint16_t* x;
+  long ldx;
+  const int* idx;
+  const uint16_t* y_in;
+  long ldy;
+  int n_adapters;
+  const int* rank;
+  const double* alpha;
+  const uint16_t* const* A_t; /* [adapter] -> rank x d_in   */
+  const uint16_t* const* B;   /* [adapter] -> rank x d_out  */
+  double* y_out;              /* T x d_out                  */
+  int t0, t1;
+} delta_job;
+
+static void* delta_worker(void* arg) {
+  delta_job* J = (delta_job*)arg;
+  double* t = NULL;
+  int tcap = 0;
+  for (int i = J->t0; i < J->t1; ++i) {
+    double* yo = J->y_out + (long)i * J->d_out;
+    const uint16_t* yi = J->y_in ? J->y_in + (long)i * J->ldy : NULL;
+    for (int l = 0; l < J->d_out; ++l) yo[l] = yi ? dec(J->dtype, yi[l]) : 0.0;
+    int a = J->idx[i];
+    if (a < 0) continue; /* "adapter id < 0": row untouched */
+    int r = J->rank[a];
+    if (r == 0) continue; /* rank 0: nothing to add */
+    if (r > tcap) {
+      free(t);
+      t = (double*)malloc(sizeof(double) * r);
+      tcap = r;
+    }
+    const uint16_t* xi = J->x + (long)i * J->ldx;
+    const uint16_t* At = J->A_t[a];
+    const uint16_t* B = J->B[a];
+    /* shrink: t[k] = sum_j x[j] * A[j][k],   A[j][k] = A_t[k][j] */
+    for (int k = 0; k < r; ++k) {
+      double acc = 0.0;
+      for (int j = 0; j < J->d_in; ++j)
+        acc += dec(J->dtype, xi[j]) * dec(J->dtype, At[(long)k * J->d_in + j]);
+      t[k] = acc;
+    }
+    /* expand and scale: y[l] += (alpha / r) * sum_k t[k] * B[k][l] */
+    double s = J->alpha[a] / (double)r;
+    for (int l = 0; l < J->d_out; ++l) {
+      double acc = 0.0;
+      for (int k = 0; k < r; ++k) acc += t[k] * dec(J->dtype, B[(long)k * J->d_out + l]);
+      yo[l] += s * acc;
+    }
+  }
+  free(t);
+  return NULL;
+}
+
+/*
+ * y_out[i][l] (fp64, not rounded) for i < T, l < d_out.  y_in may be NULL
+ * (taken as zero).  idx[i] in [-1, n_adapters).  n_threads >= 1 splits the
+ * token range; the result does not depend on it.
+ */
+int oracle_lora_delta(int dtype, int T, int d_in, int d_out, const uint16_t* x, long ldx,
+                      const int* idx, const uint16_t* y_in, long ldy, int n_adapters,
+                      const int* rank, const double* alpha, const uint16_t* const* A_t,
+                      const uint16_t* const* B, double* y_out, int n_threads) {
+  if ((dtype != 0 && dtype != 1) || T < 0 || d_in <= 0 || d_out <= 0 || ldx < d_in ||
+      (y_in && ldy < d_out) || n_threads < 1)
+    return OR_ERR_ARG;
+  for (int i = 0; i < T; ++i)
+    if (idx[i] < -1 || idx[i] >= n_adapters) return OR_ERR_ARG;
+  for (int i = 0; i < T; ++i)
+    if (idx[i] >= 0 && (rank[idx[i]] < 0 || (rank[idx[i]] > 0 && (!A_t[idx[i]] || !B[idx[i]]))))
+      return OR_ERR_ARG;
+  if (n_threads > T) n_threads = T > 0 ? T : 1;
+  delta_job* jobs = (delta_job*)calloc(n_threads, sizeof(delta_job));
+  pthread_t* th = (pthread_t*)calloc(n_threads, sizeof(pthread_t));
+  for (int w = 0; w < n_threads; ++w) {
+    delta_job j = {dtype, T, d_in, d_out, x, ldx, idx, y_in, ldy, n_adapters, rank, alpha,
+                   A_t, B, y_out, (int)((long)T * w / n_threads),
+                   (int)((long)T * (w + 1) / n_threads)};
+    jobs[w] = j;
+  }
+  for (int w = 1; w < n_threads; ++w) pthread_create(&th[w], NULL, delta_worker, &jobs[w]);
+  delta_worker(&jobs[0]);
+  for (int w = 1; w < n_threads; ++w) pthread_join(th[w], NULL);
+  free(jobs);
+  free(th);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Segments.                                                                  */
+/*
+ * Tokens with idx >= 0, ordered by adapter id ascending and, inside one
+ * adapter, by token position (a stable counting sort).  perm[0..n_valid),
+ * seg_start[0..S], seg_adapter[0..S).  Tokens with idx == -1 are left out.
+ */
+int oracle_segments(const int* idx, int T, int max_adapters, int* perm, int* seg_start,
+                    int* seg_adapter, int* S_out) {
+  if (T < 0 || max_adapters <= 0) return OR_ERR_ARG;
+  for (int i = 0; i < T; ++i)
+    if (idx[i] < -1 || idx[i] >= max_adapters) return OR_ERR_ARG;
+  int* count = (int*)calloc(max_adapters, sizeof(int));
+  for (int i = 0; i < T; ++i)
+    if (idx[i] >= 0) count[idx[i]]++;
+  int* start = (int*)calloc(max_adapters, sizeof(int));
+  int pos = 0, S = 0;
+  for (int a = 0; a < max_adapters; ++a) {
+    start[a] = pos;
+    if (count[a] > 0) {
+      seg_start[S] = pos;
+      seg_adapter[S] = a;
+      S++;
+    }
+    pos += count[a];
+  }
+  seg_start[S] = pos;
+  for (int i = 0; i < T; ++i) /* ascending i keeps the sort stable */
+    if (idx[i] >= 0) perm[start[idx[i]]++] = i;
+  *S_out = S;
+  free(count);
+  free(start);
+  return OR_OK;
+}
+
+/*
+ * Prefill: request q covers tokens [req_start[q], req_start[q+1]) and uses
+ * adapter req_adapter[q] (-1: none).  Neighbouring requests with the same
+ * adapter become one segment; segments partition [req_start[0], req_start[n]).
+ * Empty requests are dropped.
+ */
+int oracle_merge_requests(const int* req_start, const int* req_adapter, int n, int* seg_start,
+                          int* seg_adapter, int* S_out) {
+  if (n < 0) return OR_ERR_ARG;
+  int S = 0;
+  for (int q = 0; q < n; ++q) {
+    if (req_start[q + 1] < req_start[q] || req_adapter[q] < -1) return OR_ERR_ARG;
+    if (req_start[q + 1] == req_start[q]) continue;
+    if (S > 0 && seg_adapter[S - 1] == req_adapter[q]) continue; /* extends the open segment */
+    seg_start[S] = req_start[q];
+    seg_adapter[S] = req_adapter[q];
+    S++;
+  }
+  seg_start[S] = n > 0 ? req_start[n] : 0;
+  *S_out = S;
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Pages.                                                                     */
+static long cdiv(long a, long b) { return (a + b - 1) / b; }
+
+/* Each of the 2*n_proj tensors (r x d_in for A, r x d_out for B) is laid out
+ * flat and cut into pages of page_elems elements. */
+long oracle_pages_needed(int rank, int n_proj, const int* d_in, const int* d_out,
+                         long page_elems) {
+  long n = 0;
+  for (int p = 0; p < n_proj; ++p)
+    n += cdiv((long)rank * d_in[p], page_elems) + cdiv((long)rank * d_out[p], page_elems);
+  return n;
+}
+
+/* ------------------------------------------------------------------------- */
+/* LRU.                                                                       */
+/*
+ * A pool of `capacity` pages and adapters 0..n_adapters-1 needing need[a]
+ * pages each.  Call c asks for ids[call_off[c] .. call_off[c+1]) (duplicates
+ * allowed).  For each call:
+ *   - every asked adapter must end up resident; the asked ones are pinned for
+ *     this call and cannot be evicted by it;
+ *   - while the free pages do not cover the missing adapters, the resident,
+ *     unpinned adapter with the oldest last use is evicted (equal ages: the
+ *     lower id first); never-used counts as oldest;
+ *   - if that cannot make room, the call fails with OOM and nothing changes;
+ *   - on success every asked adapter gets last use = c.
+ * Missing adapters are loaded in the order they first appear in the call.
+ * Outputs: status[c]; resident[c*n_adapters + a] after call c; the evicted ids
+ * of all calls concatenated in eviction order, with evict_off[c] marking where
+ * call c starts (evict_off has n_calls+1 entries).
+ */
+int oracle_lru_run(int n_adapters, const long* need, long capacity, int n_calls,
+                   const int* call_off, const int* ids, int* status, unsigned char* resident,
+                   int* evicted, int* evict_off) {
+  unsigned char* res = (unsigned char*)calloc(n_adapters, 1);
+  long* last = (long*)malloc(sizeof(long) * n_adapters);
+  unsigned char* pin = (unsigned char*)calloc(n_adapters, 1);
+  unsigned char* tmp = (unsigned char*)malloc(n_adapters);
+  int* victims = (int*)malloc(sizeof(int) * (n_adapters + 1));
+  for (int a = 0; a < n_adapters; ++a) last[a] = -1;
+  long used = 0;
+  int ne = 0;
+  for (int c = 0; c < n_calls; ++c) {
+    evict_off[c] = ne;
+    memset(pin, 0, n_adapters);
+    int bad = 0;
+    long missing = 0;
+    for (int q = call_off[c]; q < call_off[c + 1]; ++q) {
+      int a = ids[q];
+      if (a < 0 || a >= n_adapters) {
+        bad = 1;
+        break;
+      }
+      if (!pin[a] && !res[a]) missing += need[a];
+      pin[a] = 1;
+    }
+    if (bad) {
+      status[c] = OR_ERR_ARG;
+    } else {
+      /* plan evictions without changing state */
+      memcpy(tmp, res, n_adapters);
+      long free_pages = capacity - used;
+      int nv = 0;
+      while (free_pages < missing) {
+        int best = -1;
+        for (int a = 0; a < n_adapters; ++a) {
+          if (!tmp[a] || pin[a]) continue;
+          if (best < 0 || last[a] < last[best]) best = a; /* ascending a: ties keep lower id */
+        }
+        if (best < 0) break;
+        tmp[best] = 0;
+        free_pages += need[best];
+        victims[nv++] = best;
+      }
+      if (free_pages < missing) {
+        status[c] = OR_ERR_OOM;
+      } else {
+        for (int v = 0; v < nv; ++v) {
+          res[victims[v]] = 0;
+          used -= need[victims[v]];
+          evicted[ne++] = victims[v];
+        }
+        for (int q = call_off[c]; q < call_off[c + 1]; ++q) {
+          int a = ids[q];
+          if (!res[a]) {
+            res[a] = 1;
+            used += need[a];
+          }
+          last[a] = c;
+        }
+        status[c] = OR_OK;
+      }
+    }
+    memcpy(resident + (long)c * n_adapters, res, n_adapters);
+  }
+  evict_off[n_calls] = ne;
+  free(res);
+  free(last);
+  free(pin);
+  free(tmp);
+  free(victims);
+  return OR_OK;
+}

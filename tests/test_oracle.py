@@ -1,0 +1,261 @@
+"""Pins for the fp64 CPU oracle, against things other than itself.
+
+Each check is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a wrong scale) fails at least one:
+  * a hand-derived worked example (tests/golden/tiny_delta.json);
+  * the exact fp16/bf16 decoders against numpy's own conversions;
+  * brute force with the dense update W_delta = A.B (numpy fp64) on tiny,
+    deliberately non-square shapes;
+  * closed forms: rank 0 / zero A / zero B / adapter -1 leave y unchanged,
+    one shared adapter equals one ordinary GEMM, rank 1 is an outer product,
+    A = I gives y + s.x.B;
+  * invariants: token permutation, linearity in the scale, additivity over a
+    split of the tokens, thread count.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from workloads import BF16, F16, to_bits
+
+
+def _bits(dtype, a):
+    return to_bits(dtype, np.asarray(a, np.float32))
+
+
+def _dec(dtype, bits):
+    bits = np.asarray(bits, np.uint16)
+    if dtype == F16:
+        return bits.view(np.float16).astype(np.float64)
+    with np.errstate(invalid="ignore"):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _rand_case(rng, dtype, T, d_in, d_out, ranks, p_none=0.2):
+    n_ad = len(ranks)
+    x = _bits(dtype, rng.standard_normal((T, d_in)))
+    y = _bits(dtype, rng.standard_normal((T, d_out)))
+    idx = rng.integers(0, n_ad, T).astype(np.int32)
+    idx[rng.random(T) < p_none] = -1
+    A_t = [_bits(dtype, rng.standard_normal((r, d_in)) / np.sqrt(d_in)) for r in ranks]
+    B = [_bits(dtype, rng.standard_normal((r, d_out)) / np.sqrt(max(r, 1))) for r in ranks]
+    return x, y, idx, A_t, B
+
+
+def _dense_ref(dtype, x, y, idx, ranks, alphas, A_t, B):
+    """numpy fp64: y + s_a * x @ (A @ B), with A = A_t.T built explicitly."""
+    X = _dec(dtype, x)
+    Y = _dec(dtype, y).copy()
+    for i, a in enumerate(idx):
+        if a < 0 or ranks[a] == 0:
+            continue
+        A = _dec(dtype, A_t[a]).T          # d_in x r
+        Bm = _dec(dtype, B[a])             # r x d_out
+        W = A @ Bm                         # dense d_in x d_out update
+        Y[i] += (alphas[a] / ranks[a]) * (X[i] @ W)
+    return Y
+
+
+# --------------------------------------------------------------------------
+def test_decoders_match_numpy_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    for dtype in (F16, BF16):
+        ref = _dec(dtype, bits)
+        got = oracle.decode16(bits, dtype)
+        fin = np.isfinite(ref)
+        assert np.array_equal(got[fin], ref[fin])
+        assert np.array_equal(np.isnan(got), np.isnan(ref))
+        assert np.array_equal(got[np.isinf(ref)], ref[np.isinf(ref)])
+
+
+def test_golden_tiny_delta(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "tiny_delta.json")))
+    dt = F16
+    ranks = np.array(g["ranks"], np.int32)
+    A_t = [_bits(dt, np.array(a, np.float32).reshape(r, 3)) for a, r in zip(g["A_t"], ranks)]
+    B = [_bits(dt, np.array(b, np.float32).reshape(r, 2)) for b, r in zip(g["B"], ranks)]
+    y = oracle.lora_delta(dt, _bits(dt, g["x"]), g["idx"], _bits(dt, g["y_in"]), ranks,
+                          np.full(3, g["alpha"]), A_t, B)
+    assert np.array_equal(y, np.array(g["y_out"], np.float64))
+
+
+@pytest.mark.parametrize("dtype", [F16, BF16])
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_bruteforce_dense_update(dtype, seed):
+    rng = np.random.default_rng(seed)
+    ranks = [3, 8, 1, 5]
+    T, d_in, d_out = 13, 24, 40           # non-square on purpose
+    x, y, idx, A_t, B = _rand_case(rng, dtype, T, d_in, d_out, ranks)
+    alphas = np.array([16.0, 16.0, 2.0, 16.0])
+    got = oracle.lora_delta(dtype, x, idx, y, ranks, alphas, A_t, B)
+    ref = _dense_ref(dtype, x, y, idx, ranks, alphas, A_t, B)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_identity_cases():
+    rng = np.random.default_rng(7)
+    dt = F16
+    T, d_in, d_out = 9, 16, 24
+    x, y, idx, A_t, B = _rand_case(rng, dt, T, d_in, d_out, [4, 4, 0, 4], p_none=0.3)
+    A_t[1] = np.zeros_like(A_t[1])       # zero A
+    B[3] = np.zeros_like(B[3])           # zero B
+    got = oracle.lora_delta(dt, x, idx, y, [4, 4, 0, 4], np.full(4, 16.0), A_t, B)
+    Y = _dec(dt, y)
+    for i, a in enumerate(idx):
+        if a in (-1, 1, 2, 3):           # none, zero A, rank 0, zero B
+            assert np.array_equal(got[i], Y[i])
+    assert not np.array_equal(got[idx == 0], Y[idx == 0]) or not np.any(idx == 0)
+
+
+@pytest.mark.parametrize("dtype", [F16, BF16])
+def test_shared_adapter_is_one_gemm(dtype):
+    rng = np.random.default_rng(11)
+    T, d_in, d_out, r = 17, 32, 48, 8
+    x, y, _, A_t, B = _rand_case(rng, dtype, T, d_in, d_out, [r])
+    idx = np.zeros(T, np.int32)
+    got = oracle.lora_delta(dtype, x, idx, y, [r], [16.0], A_t, B)
+    X, Y = _dec(dtype, x), _dec(dtype, y)
+    ref = Y + (16.0 / r) * np.matmul(np.matmul(X, _dec(dtype, A_t[0]).T), _dec(dtype, B[0]))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rank_one_is_outer_product():
+    rng = np.random.default_rng(5)
+    dt = BF16
+    T, d_in, d_out = 6, 20, 12
+    x, y, _, A_t, B = _rand_case(rng, dt, T, d_in, d_out, [1])
+    idx = np.zeros(T, np.int32)
+    got = oracle.lora_delta(dt, x, idx, y, [1], [16.0], A_t, B)
+    X, Y = _dec(dt, x), _dec(dt, y)
+    a, b = _dec(dt, A_t[0])[0], _dec(dt, B[0])[0]
+    ref = Y + 16.0 * np.outer(X @ a, b)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_identity_A_gives_x_B():
+    rng = np.random.default_rng(6)
+    dt = F16
+    T, r, d_out = 5, 8, 16
+    x, y, _, _, B = _rand_case(rng, dt, T, r, d_out, [r])
+    A_t = [_bits(dt, np.eye(r))]
+    got = oracle.lora_delta(dt, x, np.zeros(T, np.int32), y, [r], [16.0], A_t, B)
+    ref = _dec(dt, y) + (16.0 / r) * (_dec(dt, x) @ _dec(dt, B[0]))
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_invariants_permutation_scale_split_threads():
+    rng = np.random.default_rng(21)
+    dt = BF16
+    ranks = [8, 16, 4]
+    T, d_in, d_out = 31, 40, 24
+    x, y, idx, A_t, B = _rand_case(rng, dt, T, d_in, d_out, ranks)
+    al = np.array([16.0, 16.0, 16.0])
+    base = oracle.lora_delta(dt, x, idx, y, ranks, al, A_t, B)
+    # token permutation
+    perm = rng.permutation(T)
+    got = oracle.lora_delta(dt, x[perm], idx[perm], y[perm], ranks, al, A_t, B)
+    assert np.array_equal(got, base[perm])
+    # linear in the scale (x2 is exact in binary)
+    Y = _dec(dt, y)
+    got2 = oracle.lora_delta(dt, x, idx, y, ranks, 2 * al, A_t, B)
+    assert np.array_equal(got2 - Y, 2 * (base - Y))
+    # additivity over a split of the tokens by adapter
+    parts = np.zeros_like(base)
+    for a in [-1, 0, 1, 2]:
+        m = idx == a
+        if m.any():
+            parts[m] = oracle.lora_delta(dt, x[m], idx[m], y[m], ranks, al, A_t, B)
+    assert np.array_equal(parts, base)
+    # thread count does not change the result
+    assert np.array_equal(oracle.lora_delta(dt, x, idx, y, ranks, al, A_t, B, n_threads=4), base)
+
+
+def test_rejects_bad_index():
+    rng = np.random.default_rng(1)
+    x, y, idx, A_t, B = _rand_case(rng, F16, 4, 8, 8, [2])
+    with pytest.raises(ValueError):
+        oracle.lora_delta(F16, x, np.array([0, 1, 0, 0]), y, [2], [16.0], A_t, B)
+
+
+# --------------------------------------------------------------------------
+def test_segments_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "segments.json")))
+    d = g["decode"]
+    perm, ss, sa = oracle.segments(d["idx"], d["max_adapters"])
+    assert perm.tolist() == d["perm"]
+    assert ss.tolist() == d["seg_start"]
+    assert sa.tolist() == d["seg_adapter"]
+    p = g["prefill"]
+    ss, sa = oracle.merge_requests(p["req_start"], p["req_adapter"])
+    assert ss.tolist() == p["seg_start"] and sa.tolist() == p["seg_adapter"]
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_segments_bruteforce(seed):
+    rng = np.random.default_rng(seed)
+    T, n_ad = int(rng.integers(0, 300)), int(rng.integers(1, 50))
+    idx = rng.integers(-1, n_ad, T).astype(np.int32)
+    perm, ss, sa = oracle.segments(idx, n_ad)
+    # brute force: python sort by (adapter, position) over the valid tokens
+    ref = sorted([i for i in range(T) if idx[i] >= 0], key=lambda i: (idx[i], i))
+    assert perm.tolist() == ref
+    assert ss[0] == 0 and ss[-1] == len(ref)
+    for s in range(len(sa)):
+        toks = perm[ss[s]:ss[s + 1]]
+        assert toks.size > 0 and np.all(idx[toks] == sa[s])
+    assert np.all(np.diff(sa) > 0)
+    assert set(sa.tolist()) == set(idx[idx >= 0].tolist())
+
+
+def test_pages_needed_closed_form():
+    # 7B layer, rank 16, 16 KB pages of fp16 (8192 elements):
+    # 4096-wide tensors take 16*4096/8192 = 8 pages, 11008-wide ones ceil(22.5..) = 22
+    d_in = [4096] * 6 + [11008]
+    d_out = [4096] * 4 + [11008] * 2 + [4096]
+    assert oracle.pages_needed(16, d_in, d_out, 8192) == 4 * 16 + 2 * (8 + 22) + (22 + 8)
+    # one row per page (1024-element rows, 1024-element pages): 2*r pages per projection
+    assert oracle.pages_needed(8, [1024], [1024], 1024) == 16
+    assert oracle.pages_needed(0, [1024], [1024], 1024) == 0
+    # a 1024-wide output of rank 8 fits one 8192-element page
+    assert oracle.pages_needed(8, [8192], [1024], 8192) == 8 + 1
+
+
+def test_lru_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "lru_trace.json")))
+    status, res, ev = oracle.lru_run(g["need"], g["capacity"], g["calls"])
+    assert status.tolist() == g["status"]
+    for c in range(len(g["calls"])):
+        assert np.flatnonzero(res[c]).tolist() == g["resident"][c]
+    assert ev == g["evicted"]
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_lru_invariants(seed):
+    rng = np.random.default_rng(seed)
+    n_ad = 30
+    need = rng.integers(1, 6, n_ad)
+    cap = 40
+    calls = [rng.choice(n_ad, size=int(rng.integers(1, 8)), replace=True).tolist()
+             for _ in range(60)]
+    status, res, ev = oracle.lru_run(need, cap, calls)
+    last = {}
+    prev = np.zeros(n_ad, bool)
+    for c, ids in enumerate(calls):
+        if status[c] == 0:
+            assert res[c][ids].all()
+            assert not set(ev[c]) & set(ids)
+            assert need[res[c]].sum() <= cap
+            # each victim was at least as old as every unpinned survivor
+            for v in ev[c]:
+                for a in np.flatnonzero(res[c] & prev):
+                    if a not in ids:
+                        assert (last.get(v, -1), v) <= (last.get(a, -1), a)
+            for a in ids:
+                last[a] = c
+        else:
+            assert status[c] == 2 and ev[c] == []
+            assert np.array_equal(res[c], prev)
+        prev = res[c]
