@@ -1,0 +1,347 @@
+"""Benchmark of the paged multi-adapter LoRA delta on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the page-in call for
+the batch's adapter set (LRU touch; no copies when all are resident), the
+device segment build, the grouped paged shrink and the grouped expand over
+all projections of one layer.  Default workload: the LLaMA-7B decode layer
+(7 projections, 256 tokens, 1000 resident rank-16 adapters, Zipf 1.0, fp16).
+
+Timing: CUDA events that the library records on the compute stream right
+around its own kernels (slora_set_phase_events), so per-kernel and per-step
+device times carry no host gaps.  L2 is flushed (a 256 MiB write) and y reset
+before every step, outside the timed events.  N > 1 (torchrun): every rank
+runs an independent replica (no collective on the data path); the step time
+is the max over ranks (NCCL all-reduce of the timings only).
+
+The reference arm (--impl reference) is the fp64 CPU oracle, timed on the
+host cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "LoRA-delta tokens/s at LLaMA-7B shapes, 1 B200; % of HBM/tensor roofline"
+UNIT = "tokens/s"
+FALLBACK_HBM = 6650.0
+FALLBACK_BF16 = 1590.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, FALLBACK_BF16, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes / flops (each touched adapter and each distinct input read
+# once, y read and written once)
+def algorithmic(w: W.Workload, tokens=None):
+    idx = w.idx if tokens is None else w.idx[tokens]
+    T = idx.size
+    esz = 2
+    touched = np.unique(idx[idx >= 0])
+    r_sum = int(w.ranks[touched].sum())
+    din = sum(p.d_in for p in w.projs)
+    dout = sum(p.d_out for p in w.projs)
+    xin = sum(w.x_dim(n) for n in w.x_names)
+    A_bytes = r_sum * din * esz
+    B_bytes = r_sum * dout * esz
+    x_bytes = T * xin * esz
+    y_bytes = 2 * T * dout * esz
+    r_tok = w.ranks[idx[idx >= 0]].astype(np.int64)
+    flops = int(2 * r_tok.sum() * (din + dout))
+    return dict(shrink_bytes=A_bytes + x_bytes, expand_bytes=B_bytes + y_bytes,
+                total_bytes=A_bytes + B_bytes + x_bytes + y_bytes, flops=flops,
+                touched=int(touched.size))
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.lines = []
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-lms", "100", "-i", str(self.index)],
+                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.p = None
+
+    def _read(self):
+        for line in self.p.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world):
+    import torch
+
+    import gather_lora_paged_b200 as G
+    import harness as H
+
+    dev = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(dev)
+    w = W.config(args.config)
+    if args.config in (3, 4):
+        raise SystemExit("bench.py: configs 3 and 4 are measured by their own paths")
+    pb = H.PoolBuild(w)
+    ten = H.Tensors(w)
+    stream = torch.cuda.current_stream()
+    d_idx = torch.from_numpy(w.idx).cuda()
+    touched = w.touched().tolist()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    G.slora_set_phase_events(pb.h, ev)
+    alg = algorithmic(w)
+
+    def step():
+        G.slora_adapter_page_in(pb.h, touched, stream)
+        G.slora_lora_delta(pb.h, *ten.args(), d_idx, w.T, stream)
+
+    def prep():
+        ten.reset()
+        flush.zero_()
+
+    for _ in range(args.warmup):
+        prep()
+        step()
+    torch.cuda.synchronize()
+    st, code, info = G.slora_check_device(pb.h)
+    assert st == 0, (code, info)
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev)
+    clocks.start()
+    t_step = t_seg = t_shr = t_exp = 0.0
+    for _ in range(args.steps):
+        prep()
+        step()
+        ev[3].synchronize()
+        t_seg += ev[0].elapsed_time(ev[1])
+        t_shr += ev[1].elapsed_time(ev[2])
+        t_exp += ev[2].elapsed_time(ev[3])
+        t_step += ev[0].elapsed_time(ev[3])
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+        t = torch.tensor([t_step], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_step = float(t.item())
+    K = args.steps
+    ms = t_step / K
+    value = world * w.T * K / (t_step / 1e3)
+
+    # end to end through the C ABI with host buffers (pinned), copies timed
+    e2e = None
+    if rank == 0 or True:
+        hx = {n: H.pinned(w.x(n)) for n in w.x_names}
+        hy = [H.pinned(w.y_in(p)) for p in range(len(w.projs))]
+        hout = [torch.empty_like(t).pin_memory() for t in hy]
+        hidx = torch.from_numpy(w.idx).pin_memory()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        G.slora_set_phase_events(pb.h, [])
+        xs = {n: ten.x[n].view(torch.int16) for n in w.x_names}
+        ys = [t.view(torch.int16) for t in ten.y]
+
+        def e2e_step():
+            for n in w.x_names:
+                xs[n].copy_(hx[n], non_blocking=True)
+            for p in range(len(w.projs)):
+                ys[p].copy_(hy[p], non_blocking=True)
+            d_idx.copy_(hidx, non_blocking=True)
+            step()
+            for p in range(len(w.projs)):
+                hout[p].copy_(ys[p], non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        tot = 0.0
+        n_e2e = max(10, min(K, 200))
+        for _ in range(n_e2e):
+            flush.zero_()
+            e0.record()
+            e2e_step()
+            e1.record()
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        h2d = sum(t.numel() * 2 for t in hx.values()) + sum(t.numel() * 2 for t in hy) + hidx.numel() * 4
+        d2h = sum(t.numel() * 2 for t in hout)
+        e2e = {"value": world * w.T * n_e2e / (tot / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": tot / n_e2e}
+
+    hbm, tc, src = peaks()
+    t_exp_l = t_exp / K
+    t_shr_l = t_shr / K
+    dom = ("expand", t_exp_l, alg["expand_bytes"]) if t_exp_l >= t_shr_l else \
+        ("shrink", t_shr_l, alg["shrink_bytes"])
+    achieved = dom[2] / (dom[1] / 1e3) / 1e9
+    step_gbs = alg["total_bytes"] / (ms / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": W.DTYPE_NAME[w.dtype],
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(d_in)) A, N(0,1/sqrt(r)) B; "
+                "Zipf adapter ids)",
+        "config": {"workload": w.name, "tokens_per_step": w.T, "projections": len(w.projs),
+                   "adapters": w.n_adapters, "touched_adapters": alg["touched"],
+                   "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "peak_source": src,
+                     "alg_bytes_per_launch": dom[2]},
+        "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s",
+                          "frac": step_gbs / hbm, "alg_bytes_per_step": alg["total_bytes"],
+                          "flops_per_step": alg["flops"],
+                          "kernel_ms": {"segments": t_seg / K, "shrink": t_shr_l,
+                                        "expand": t_exp_l}},
+        "e2e": e2e,
+        "gpu_launches": 3 * K,
+        "clocks": clk,
+    }
+    pb.close()
+    return out
+
+
+# ---------------------------------------------------------------------------
+def oracle_step(w: W.Workload, tokens, threads):
+    import harness as H
+    import oracle
+    for p in range(len(w.projs)):
+        x, idx, y, A_t, B = H.oracle_inputs(w, p, tokens)
+        oracle.lora_delta(w.dtype, x, idx, y, w.ranks, np.full(w.n_adapters, w.alpha), A_t, B,
+                          n_threads=threads)
+
+
+def cpu_baseline(w: W.Workload, budget_s=10.0):
+    """The oracle, as it stands, on the host cores over a bounded sample of the
+    workload: whole steps when they fit the budget, else a token subset."""
+    threads = os.cpu_count() or 1
+    w.prefetch_adapters(w.touched().tolist())
+    t0 = time.perf_counter()
+    oracle_step(w, None, threads)
+    dt = time.perf_counter() - t0
+    n_steps, toks = 1, w.T
+    while time.perf_counter() - t0 < budget_s and n_steps < 50:
+        oracle_step(w, None, threads)
+        n_steps += 1
+    dt = time.perf_counter() - t0
+    return {"value": n_steps * toks / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n_steps} whole step(s) of {w.name} ({toks} tokens x {len(w.projs)} "
+                      f"projections each), fp64 loops, {threads} threads",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = W.config(args.config)
+    for _ in range(args.warmup):
+        pass
+    cb = cpu_baseline(w, budget_s=max(5.0, min(60.0, 2.0 * args.steps)))
+    return {"metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.T / cb["value"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "tokens_per_step": w.T},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out))
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = run_ours(args, rank, world)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(W.config(args.config))
+        print(json.dumps(out))
+    if world > 1:
+        import torch
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,49 @@
+"""Build the sm_100a CUDA library (libslora.so) in-tree with nvcc.
+
+The library is the product path: kernels in csrc/*.cu, the C-ABI runtime in
+csrc/runtime.cpp, declared by include/slora.h.  The CUDA runtime is linked
+statically so the library does not depend on which libcudart a host process
+(e.g. PyTorch) has loaded.
+"""
+import glob
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+OUT = os.path.join(HERE, "libslora.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def sources():
+    return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")) +
+                  glob.glob(os.path.join(HERE, "csrc", "*.cpp")))
+
+
+def _stale():
+    if not os.path.exists(OUT):
+        return True
+    deps = sources() + glob.glob(os.path.join(HERE, "csrc", "*.h")) + \
+        [os.path.join(ROOT, "include", "slora.h")]
+    t = os.path.getmtime(OUT)
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not _stale():
+        return OUT
+    cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2",
+           "-shared", "-cudart", "static", "-I" + os.path.join(ROOT, "include"),
+           *sources(), "-o", OUT + ".tmp"]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+        print(" ".join(cmd))
+    subprocess.check_call(cmd)
+    os.replace(OUT + ".tmp", OUT)
+    return OUT
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

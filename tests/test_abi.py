@@ -1,0 +1,173 @@
+"""The C-ABI library loads and exports every entry point include/slora.h
+declares; sizing and host-side pool logic (LRU, page accounting, OOM, fault
+injection, batch checks) run without a GPU on a host_only pool and agree with
+the oracle's LRU rules."""
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import gather_lora_paged_b200 as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "slora.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(slora_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = G.lib()
+    names = _declared()
+    assert len(names) >= 20
+    out = subprocess.run(["nm", "-D", "--defined-only", G.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(slora_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(L, n)
+
+
+def test_desc_layout_matches_header():
+    # int32 x 22, then int64 page_elems at byte 88 (see slora_pool_desc)
+    assert G.PoolDesc.page_elems.offset == 88
+    assert G.PoolDesc.dev_pool.offset == 104
+    assert G.PoolDesc.host_only.offset == 136
+    assert __import__("ctypes").sizeof(G.PoolDesc) == 168
+
+
+LAYER7B = ([4096] * 6 + [11008], [4096] * 4 + [11008] * 2 + [4096])
+
+
+def test_sizing_matches_oracle_page_count():
+    d = G.make_desc(G.SLORA_F16, *LAYER7B, 1000, 64, 256, 8192, 10)
+    for r in (0, 8, 16, 24, 64):
+        assert G.slora_pages_for_rank(d, r) == oracle.pages_needed(r, *LAYER7B, 8192)
+    assert G.slora_tables_bytes(d) > 0 and G.slora_scratch_bytes(d) > 0
+
+
+def _host_pool(n_pages=100, max_adapters=40, max_rank=32, page=1024):
+    return G.Pool(G.SLORA_F16, [1024, 2048], [2048, 1024], max_adapters, max_rank, 64, page,
+                  n_pages, host_only=True)
+
+
+def _register_all(pool, ranks):
+    dummy = np.zeros(16, np.uint16)
+    for a, r in enumerate(ranks):
+        pool.register(a, int(r), 16.0, [dummy, dummy], [dummy, dummy])
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_lru_matches_oracle(seed):
+    rng = np.random.default_rng(seed)
+    n_ad = 40
+    ranks = rng.choice([0, 8, 16, 32], n_ad)
+    pool = _host_pool()
+    _register_all(pool, ranks)
+    need = [pool.pages_for_rank(int(r)) for r in ranks]
+    calls = [rng.choice(n_ad, size=int(rng.integers(1, 7))).tolist() for _ in range(80)]
+    calls.insert(10, [n_ad + 3])  # invalid id
+    status, resident, evicted = oracle.lru_run(need, 100, calls)
+    for c, ids in enumerate(calls):
+        st = 0
+        try:
+            pool.page_in(ids)
+        except G.SloraError as e:
+            st = e.status
+        assert st == status[c], (c, ids, st, status[c])
+        got = [G.slora_adapter_is_resident(pool.h, a) for a in range(n_ad)]
+        assert got == resident[c].tolist(), c
+    s = pool.stats()
+    assert s["free_pages"] == 100 - sum(need[a] for a in range(n_ad) if resident[-1][a])
+    assert s["evictions"] == sum(len(e) for e in evicted)
+
+
+def test_lru_golden_trace_through_the_library(golden_dir):
+    import json
+    g = json.load(open(os.path.join(golden_dir, "lru_trace.json")))
+    # pages: d_in 1024, d_out 1024, page 1024 -> 2*rank pages per adapter
+    ranks = [n // 2 for n in g["need"]]
+    pool = G.Pool(G.SLORA_F16, [1024], [1024], len(ranks), 8, 16, 1024, g["capacity"],
+                  host_only=True)
+    _register_all(pool, ranks)
+    assert [pool.pages_for_rank(r) for r in ranks] == g["need"]
+    for c, ids in enumerate(g["calls"]):
+        st = 0
+        try:
+            pool.page_in(ids)
+        except G.SloraError as e:
+            st = e.status
+        assert st == g["status"][c]
+        res = [a for a in range(len(ranks)) if G.slora_adapter_is_resident(pool.h, a)]
+        assert res == g["resident"][c]
+
+
+def test_oom_and_injection_leave_pool_unchanged():
+    pool = _host_pool(n_pages=30)
+    _register_all(pool, [16] * 10)   # 16*(1024+2048)*2/1024 = 96 pages each > 30
+    with pytest.raises(G.SloraError) as e:
+        pool.page_in([0])
+    assert e.value.status == 2
+    pool2 = _host_pool()
+    _register_all(pool2, [8] * 10)   # 48 pages each
+    pool2.page_in([0])
+    before = pool2.stats()
+    G.slora_inject_fault(pool2.h, 0)
+    with pytest.raises(G.SloraError) as e:
+        pool2.page_in([1])
+    assert e.value.status == 8
+    assert pool2.stats() == before
+    pool2.page_in([1])  # disarmed after firing
+    assert G.slora_adapter_is_resident(pool2.h, 1)
+
+
+def test_unregistered_and_batch_checks():
+    pool = _host_pool()
+    _register_all(pool, [8, 8, 8])
+    with pytest.raises(G.SloraError) as e:
+        pool.page_in([5])
+    assert e.value.status == 7
+    pool.page_in([0, 1])
+    G.slora_check_batch(pool.h, [0, 1, -1, 0])
+    with pytest.raises(G.SloraError) as e:
+        G.slora_check_batch(pool.h, [2])
+    assert e.value.status == 3
+    with pytest.raises(G.SloraError) as e:
+        G.slora_check_batch(pool.h, [0, 99])
+    assert e.value.status == 1
+    pool.page_in([1])                   # 0 stays resident but is no longer in the step's set
+    with pytest.raises(G.SloraError):
+        G.slora_check_batch(pool.h, [0])
+    G.slora_adapter_evict(pool.h, 1)
+    assert not G.slora_adapter_is_resident(pool.h, 1)
+
+
+def test_page_order_validation():
+    pool = _host_pool(n_pages=10)
+    with pytest.raises(G.SloraError):
+        G.slora_pool_set_page_order(pool.h, [0, 1, 2])
+    with pytest.raises(G.SloraError):
+        G.slora_pool_set_page_order(pool.h, [0] * 10)
+    G.slora_pool_set_page_order(pool.h, list(range(9, -1, -1)))
+
+
+def test_host_only_pool_refuses_compute():
+    pool = _host_pool()
+    with pytest.raises(G.SloraError) as e:
+        G.slora_lora_delta(pool.h, [0], [0], [1024], [0], [2048], 0, 0)
+    assert e.value.status == 9
+
+
+def test_bad_desc_rejected():
+    d = G.make_desc(G.SLORA_F16, [100], [128], 4, 16, 8, 1024, 4, host_only=True)
+    with pytest.raises(G.SloraError):
+        G.slora_pool_create(d)   # 100 is not a multiple of 64
+    d = G.make_desc(G.SLORA_F16, [128], [128], 4, 16, 8, 1000, 4, host_only=True)
+    with pytest.raises(G.SloraError):
+        G.slora_pool_create(d)   # page size not a power of two
