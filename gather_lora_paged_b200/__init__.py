@@ -83,6 +83,8 @@ def lib():
         "slora_pool_stats": ([P, POINTER(PoolStats)], I32),
         "slora_inject_fault": ([P, I32], I32),
         "slora_set_phase_events": ([P, P, I32], I32),
+        "slora_lora_delta_noalloc": ([P, I32, P, P, P, P, P, P, I32, P], I32),
+        "slora_noalloc_scratch_bytes": ([], c_size_t),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -235,6 +237,18 @@ def slora_lora_delta(pool: int, projs, x, ldx, y, ldy, idx, T: int, stream=None)
     c = lambda a: ctypes.cast(a, c_void_p)  # noqa: E731
     _check(pool, lib().slora_lora_delta(pool, n, c(pp), c(px), c(plx), c(py), c(ply), _ptr(idx),
                                         T, _stream(stream)))
+
+
+def slora_lora_delta_noalloc(pool: int, projs, x, ldx, y, ldy, idx, T: int, stream=None) -> None:
+    """slora_lora_delta with the library's fixed scratch array (no caller scratch)."""
+    n, pp, px, plx, py, ply = _slot_arrays(projs, x, ldx, y, ldy)
+    c = lambda a: ctypes.cast(a, c_void_p)  # noqa: E731
+    _check(pool, lib().slora_lora_delta_noalloc(pool, n, c(pp), c(px), c(plx), c(py), c(ply),
+                                                _ptr(idx), T, _stream(stream)))
+
+
+def slora_noalloc_scratch_bytes() -> int:
+    return lib().slora_noalloc_scratch_bytes()
 
 
 def slora_sgmv(pool: int, projs, x, ldx, y, ldy, seg_start, seg_adapter, S: int, T: int,

@@ -387,6 +387,65 @@ slora_status_t need_device(slora_pool* P) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
+// The fused decode delta on a caller-chosen scratch region instead of the
+// pool's dev_scratch; used by the no-allocation entry point (noalloc.cu).
+// Kernels, launch order and arithmetic are those of slora_lora_delta; only the
+// scratch addresses differ, laid out for this call's T tokens.
+namespace slora {
+slora_status_t lora_delta_on_scratch(slora_pool* P, int32_t n, const int32_t* projs,
+                                     const void* const* x, const int64_t* ldx, void* const* y,
+                                     const int64_t* ldy, const int32_t* idx, int32_t T,
+                                     cudaStream_t st, void* scratch, size_t scratch_cap) {
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  slora_status_t s = need_device(P);
+  if (s) return s;
+  if (T > 0 && !idx) return P->fail(SLORA_ERR_INVALID_ARG, "idx is NULL");
+  BgmvParams bp;
+  base_params(P, bp);
+  s = plan_slots(P, bp, n, projs, x, ldx, y, ldy, T, true, true);
+  if (s) return s;
+  if (T == 0) return SLORA_OK;
+  slora_pool_desc dd = P->d;
+  dd.max_tokens = T;
+  const ScratchLayout L = scratch_layout(dd);
+  const size_t need = L.off_sgmv;  // the decode part of the layout
+  if (need > scratch_cap)
+    return P->fail(SLORA_ERR_INVALID_ARG,
+                   "this call needs " + std::to_string(need) + " bytes of scratch; the static "
+                   "no-allocation scratch holds " + std::to_string(scratch_cap) +
+                   " (fewer tokens, projections or a smaller max_rank fit)");
+  char* b = static_cast<char*>(scratch);
+  bp.max_tokens = T;
+  bp.sc.meta = reinterpret_cast<int32_t*>(b + L.off_meta);
+  bp.sc.perm = reinterpret_cast<int32_t*>(b + L.off_perm);
+  bp.sc.seg_start = reinterpret_cast<int32_t*>(b + L.off_seg_start);
+  bp.sc.seg_adapter = reinterpret_cast<int32_t*>(b + L.off_seg_adapter);
+  bp.sc.shrink_prefix = reinterpret_cast<int32_t*>(b + L.off_shrink_pre);
+  bp.sc.expand_prefix = reinterpret_cast<int32_t*>(b + L.off_expand_pre);
+  bp.sc.ctr_prefix = reinterpret_cast<int32_t*>(b + L.off_ctr_pre);
+  bp.sc.ctr = reinterpret_cast<int32_t*>(b + L.off_ctr);
+  bp.sc.ctr_cap = L.ctr_cap;
+  bp.sc.MS = L.MS;
+  float* tpart = reinterpret_cast<float*>(b + L.off_tpart);
+  float* tfin = reinterpret_cast<float*>(b + L.off_tfin);
+  int64_t off = 0;
+  for (int k = 0; k < bp.n_slots; ++k) {
+    bp.slot[k].tpart = tpart + off;
+    off += (int64_t)bp.slot[k].nck * T * P->d.max_rank;
+    bp.slot[k].tfin = tfin + (int64_t)k * T * P->d.max_rank;
+  }
+  if (off > L.tpart_floats) return P->fail(SLORA_ERR_INVALID_ARG, "too many projections in one call");
+  bp.do_shrink = 1;
+  bp.do_expand = 1;
+  CUDA_TRY(P, launch_segments(bp, idx, T, st));
+  CUDA_TRY(P, launch_shrink(bp, P->d.dtype, P->grid_shrink, st));
+  CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
+  record_epoch(P, st);
+  return SLORA_OK;
+}
+}  // namespace slora
+
+// ---------------------------------------------------------------------------
 // C ABI
 extern "C" {
 

@@ -265,6 +265,36 @@ slora_status_t slora_sgmv(slora_pool* pool, int32_t n, const int32_t* projs,
                           const int64_t* ldy, const int32_t* seg_start,
                           const int32_t* seg_adapter, int32_t S, int32_t T, void* stream);
 
+/* The fused decode delta of slora_lora_delta, for callers that cannot
+ * allocate device memory at the point of the call: a serving loop captured
+ * into a CUDA graph (no device allocation while a stream is captured in the
+ * global capture mode), a plug-in whose host framework owns every device
+ * allocation, or a path that must not risk an allocation blocking the device.
+ * The pages have no counterpart of this entry point; it is an addition of this
+ * library.
+ * Same arguments, semantics and kernels as slora_lora_delta, but the call's
+ * scratch (segments, work plan, counters, fp32 partials and t) is taken from a
+ * fixed device array that the library reserves on every GPU that loads it
+ * (slora_noalloc_scratch_bytes(), 8 MiB) instead of the pool's dev_scratch.
+ * Nothing is allocated or freed by the call.
+ *   - The first call on a device looks up that array's device address (once
+ *     per device, with the device current); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array and it keeps the last call's contents; the
+ *     kernels initialise what must start at zero themselves.  Calls whose
+ *     kernels overlap on the GPU (other streams, other threads) race on it:
+ *     serialise them.
+ *   - A call whose scratch need (it grows with T, the projections named and
+ *     max_rank) exceeds the array fails with SLORA_ERR_INVALID_ARG and a
+ *     message giving both sizes; nothing is enqueued.                         */
+slora_status_t slora_lora_delta_noalloc(slora_pool* pool, int32_t n, const int32_t* projs,
+                                        const void* const* x, const int64_t* ldx,
+                                        void* const* y, const int64_t* ldy, const int32_t* idx,
+                                        int32_t T, void* stream);
+
+/* Size in bytes of the fixed scratch array used by slora_lora_delta_noalloc. */
+size_t slora_noalloc_scratch_bytes(void);
+
 /* ---- diagnostics ---------------------------------------------------------- */
 
 /* Reads back adapter `id`'s weights for projection `proj` from its pages into
