@@ -17,10 +17,13 @@
 //   k_page_in    copies newly resident adapters from pinned host memory into
 //                their scattered pages and updates the page table.
 //
-// All three compute kernels are persistent: a grid of (SMs x resident CTAs)
-// whose warps pull tasks from a device counter.  A task reads one adapter tile
-// once and applies it to every token of its segment that the task covers, so
-// each touched adapter is streamed from HBM about once per step.
+// Shrink and expand are persistent (one CTA of 8 warps per SM).  Every warp
+// runs its own two-slot pipeline: while it computes on one shared-memory slot,
+// the bulk-copy engine fills the other with the next task's page-gathered rows
+// (cp.async.bulk, completion counted on an mbarrier).  A task reads one adapter
+// tile once and applies it to every token of its segment that the task covers,
+// so each touched adapter is streamed from HBM about once per step.  The three
+// kernels are chained with programmatic dependent launch.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -30,21 +33,78 @@ namespace slora {
 
 #define FULL_MASK 0xffffffffu
 
-__device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
+constexpr int kWarps = 8;                 // warps per CTA of shrink / expand
+constexpr int kSlots = 2;                 // pipeline slots per warp
+constexpr int kSlotBytes = 12 * 1024;     // bytes per slot
+constexpr int kSmemBytes = kWarps * kSlots * kSlotBytes;
+constexpr int kExpandRows = 16;           // B rows per expand stage
+constexpr int kLC = 256;                  // outputs per expand task (8 per lane)
+constexpr long long kWaitLimit = 2000000000ll;  // clock cycles before a wait gives up
 
-// Token classes: tasks cover NT tokens of a segment and RW rank rows.
-__device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
-__device__ __forceinline__ int rw_of(int nt) { return nt == 1 ? 8 : 4; }
-// Expand tasks cover at most 4 tokens (8 fp32 accumulators per token per lane).
-__device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
-// Outputs per expand task: about 16 KB of B per task.
-__device__ __forceinline__ int lc_of(int r) {
-  int lc = (8192 / (r > 0 ? r : 1)) & ~255;
-  return lc < 256 ? 256 : lc;
-}
+__host__ __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
+
+// Task shapes.  Shrink tasks cover NT tokens x RW rank rows x kShrinkKC of d_in;
+// expand tasks NTE tokens x kLC outputs.  Slot use: (RW + NT) KiB for shrink,
+// 16 x 512 B + NTE x 512 B for expand; both fit kSlotBytes.
+__host__ __device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
+__host__ __device__ __forceinline__ int rw_of(int nt) { return nt == 1 ? 8 : 4; }
+__host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
 
 __device__ __forceinline__ void record_error(int32_t* err, int code, int info) {
   if (atomicCAS(&err[0], 0, code) == 0) atomicExch(&err[1], info);
+}
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// Bounded wait on an mbarrier phase; false (and a recorded error) if it gives up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
+  const uint32_t a = smem_u32(bar);
+  const long long t0 = clock64();
+  for (;;) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (clock64() - t0 > kWaitLimit) {
+      record_error(err, 4, (int)blockIdx.x);
+      return false;
+    }
+  }
+}
+// Bulk async copy global -> shared, completion counted on `bar`.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 lds128(const unsigned char* p) {
+  return *reinterpret_cast<const uint4*>(p);
 }
 
 // 16-bit -> fp32 for 8 packed elements.
@@ -76,22 +136,29 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   }
 }
 
-__device__ __forceinline__ uint4 ldg_nc(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
 // Address of flat element f of tensor (adapter a, page-list offset lo).
 __device__ __forceinline__ const uint16_t* page_addr(const PoolDev& P, int a, int lo, int64_t f) {
   const int32_t pg = __ldg(P.page_list + (int64_t)a * P.list_stride + lo + (f >> P.page_shift));
   return P.pool + ((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1));
 }
 
+// Copies flat elements [f0, f0 + n) of a paged tensor into dst.  The range
+// crosses at most one page boundary (n <= page size); piece 0 is the part in
+// the first page, piece 1 the rest.  Returns nothing for an empty piece.
+__device__ __forceinline__ void bulk_paged_piece(const PoolDev& P, int a, int lo, int64_t f0, int n,
+                                                 int piece, unsigned char* dst, uint64_t* bar) {
+  const int64_t pb = ((f0 >> P.page_shift) + 1) << P.page_shift;
+  const int64_t f1 = f0 + n;
+  if (piece == 0) {
+    const int64_t e = f1 < pb ? f1 : pb;
+    bulk_g2s(dst, page_addr(P, a, lo, f0), (uint32_t)(2 * (e - f0)), bar);
+  } else if (f1 > pb) {
+    bulk_g2s(dst + 2 * (pb - f0), page_addr(P, a, lo, pb), (uint32_t)(2 * (f1 - pb)), bar);
+  }
+}
+
 // ---------------------------------------------------------------------------
-// Block-wide exclusive scan (blockDim.x threads, multiple of 32).
+// Block-wide exclusive scans (blockDim.x threads, a multiple of 32).
 template <bool kMax>
 __device__ int block_exscan(int v, int* total, int* sh) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -123,16 +190,57 @@ __device__ int block_exscan(int v, int* total, int* sh) {
   return res;
 }
 
+// Exclusive sum-scan of V values per thread at once; v becomes the prefix,
+// tot the block totals.  sh: 32 * kV ints.
+constexpr int kV = 3 * kMaxSlots;
+__device__ void block_multiscan(int (&v)[kV], int (&tot)[kV], int* sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int ex[kV];
+#pragma unroll
+  for (int j = 0; j < kV; ++j) {
+    int x = v[j];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(FULL_MASK, x, o);
+      if (lane >= o) x += y;
+    }
+    ex[j] = x - v[j];
+    if (lane == 31) sh[w * kV + j] = x;
+  }
+  __syncthreads();
+  if (w == 0) {
+#pragma unroll
+    for (int j = 0; j < kV; ++j) {
+      int s = lane < nw ? sh[lane * kV + j] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL_MASK, s, o);
+        if (lane >= o) s += y;
+      }
+      if (lane < nw) sh[lane * kV + j] = s;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kV; ++j) {
+    v[j] = (w ? sh[(w - 1) * kV + j] : 0) + ex[j];
+    tot[j] = sh[(nw - 1) * kV + j];
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
 // k_segments: one CTA of 1024 threads.  Dynamic smem: max_adapters ints.
+constexpr int kMaxAdPerThread = 16;   // max_adapters <= 16384
+
 __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvParams p,
                                                    const int32_t* __restrict__ idx, int T) {
   extern __shared__ int hist[];
-  __shared__ int sh[32];
-  __shared__ int s_tot[4];
+  __shared__ int sh[32 * kV];
   const int tid = threadIdx.x, nth = blockDim.x;
   const int MA = p.pool.max_adapters;
   const ScratchDev& sc = p.sc;
+  griddep_launch();  // the next kernel may start its prologue; it waits for this grid
 
   for (int a = tid; a < MA; a += nth) hist[a] = 0;
   __syncthreads();
@@ -151,31 +259,108 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
   }
   __syncthreads();
 
-  // Per-thread contiguous adapter range -> counts, segment flags -> scans.
+  // Each thread owns a contiguous adapter range; the segments it creates are a
+  // contiguous range of segment indices, which it also plans.
   const int E = (MA + nth - 1) / nth;
   const int a0 = min(tid * E, MA), a1 = min(a0 + E, MA);
+  int segN[kMaxAdPerThread], segR[kMaxAdPerThread];
   int cnt = 0, nseg = 0;
-  for (int a = a0; a < a1; ++a) {
-    cnt += hist[a];
-    nseg += hist[a] > 0;
+#pragma unroll
+  for (int q = 0; q < kMaxAdPerThread; ++q) {
+    const int a = a0 + q;
+    segN[q] = (a < a1) ? hist[a] : 0;
+    segR[q] = (segN[q] > 0) ? p.pool.rank[a] : 0;
+    cnt += segN[q];
+    nseg += segN[q] > 0;
   }
   int n_valid, S;
   int cbase = block_exscan<false>(cnt, &n_valid, sh);
-  int sbase = block_exscan<false>(nseg, &S, sh);
-  for (int a = a0; a < a1; ++a) {
-    const int h = hist[a];
-    if (h > 0) {
-      sc.seg_start[sbase] = cbase;
-      sc.seg_adapter[sbase] = a;
-      ++sbase;
+  const int sbase = block_exscan<false>(nseg, &S, sh);
+  {
+    int sb = sbase;
+#pragma unroll
+    for (int q = 0; q < kMaxAdPerThread; ++q) {
+      const int a = a0 + q;
+      if (segN[q] > 0) {
+        sc.seg_start[sb] = cbase;
+        sc.seg_adapter[sb] = a;
+        ++sb;
+      }
+      if (a < a1) hist[a] = cbase;  // becomes the scatter cursor
+      cbase += segN[q];
     }
-    hist[a] = cbase;  // becomes the scatter cursor
-    cbase += h;
   }
   if (tid == 0) {
     sc.seg_start[S] = n_valid;
     sc.meta[kMetaS] = S;
     sc.meta[kMetaValid] = n_valid;
+  }
+
+  // Work planning: per group shrink tasks and counters, per slot expand tasks.
+  int v[kV], tot[kV];
+#pragma unroll
+  for (int j = 0; j < kV; ++j) v[j] = 0;
+#pragma unroll
+  for (int q = 0; q < kMaxAdPerThread; ++q) {
+    const int n = segN[q], r = segR[q];
+    if (n == 0) continue;
+    const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
+#pragma unroll
+    for (int g = 0; g < kMaxSlots; ++g) {
+      if (g >= p.n_groups || !p.do_shrink) continue;
+      const int nrg = cdiv_i(p.group[g].n * r, rw_of(nt));
+      v[g] += nrg * ntg * cdiv_i(p.group[g].d_in, kShrinkKC);
+      v[kMaxSlots + g] += nrg * ntg;
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxSlots; ++k) {
+      if (k >= p.n_slots || !p.do_expand || r == 0) continue;
+      v[2 * kMaxSlots + k] += nte * cdiv_i(p.slot[k].d_out, kLC);
+    }
+  }
+  block_multiscan(v, tot, sh);
+  int ctr_base[kMaxSlots];
+  int tot_shrink = 0, tot_ctr = 0, tot_expand = 0;
+#pragma unroll
+  for (int g = 0; g < kMaxSlots; ++g) {
+    ctr_base[g] = tot_ctr;
+    tot_shrink += tot[g];
+    tot_ctr += tot[kMaxSlots + g];
+    tot_expand += tot[2 * kMaxSlots + g];
+  }
+  {
+    int sb = sbase;
+#pragma unroll
+    for (int q = 0; q < kMaxAdPerThread; ++q) {
+      const int n = segN[q], r = segR[q];
+      if (n == 0) continue;
+      const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
+#pragma unroll
+      for (int g = 0; g < kMaxSlots; ++g) {
+        if (g >= p.n_groups) continue;
+        sc.shrink_prefix[g * (sc.MS + 1) + sb] = v[g];
+        sc.ctr_prefix[g * (sc.MS + 1) + sb] = ctr_base[g] + v[kMaxSlots + g];
+        if (!p.do_shrink) continue;
+        const int nrg = cdiv_i(p.group[g].n * r, rw_of(nt));
+        v[g] += nrg * ntg * cdiv_i(p.group[g].d_in, kShrinkKC);
+        v[kMaxSlots + g] += nrg * ntg;
+      }
+#pragma unroll
+      for (int k = 0; k < kMaxSlots; ++k) {
+        if (k >= p.n_slots) continue;
+        sc.expand_prefix[k * (sc.MS + 1) + sb] = v[2 * kMaxSlots + k];
+        if (!p.do_expand || r == 0) continue;
+        v[2 * kMaxSlots + k] += nte * cdiv_i(p.slot[k].d_out, kLC);
+      }
+      ++sb;
+    }
+  }
+  if (tid == 0) {
+    for (int g = 0; g < p.n_groups; ++g) {
+      sc.shrink_prefix[g * (sc.MS + 1) + S] = tot[g];
+      sc.ctr_prefix[g * (sc.MS + 1) + S] = ctr_base[g] + tot[kMaxSlots + g];
+    }
+    for (int k = 0; k < p.n_slots; ++k) sc.expand_prefix[k * (sc.MS + 1) + S] = tot[2 * kMaxSlots + k];
   }
   __syncthreads();
 
@@ -183,7 +368,7 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
   const int lane = tid & 31, warp = tid >> 5;
   for (int c0 = 0; c0 < T; c0 += nth) {
     const int i = c0 + tid;
-    int a = i < T ? idx[i] : -1;
+    const int a = i < T ? idx[i] : -1;
     const bool ok = a >= 0 && a < MA && p.pool.rank[a] >= 0;
     const int key = ok ? a : -1;
     const int nw = min(32, (T - c0 + 31) >> 5);
@@ -203,67 +388,7 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
     }
   }
 
-  // Work planning, per group (shrink, counters) and per slot (expand).
-  const int ES = (S + nth - 1) / nth;
-  const int s0 = min(tid * ES, S), s1 = min(s0 + ES, S);
-  int tot_shrink = 0, tot_ctr = 0, tot_expand = 0;
-  for (int g = 0; g < p.n_groups; ++g) {
-    const GroupDev& G = p.group[g];
-    const int n_kc = cdiv_i(G.d_in, kShrinkKC);
-    int lt = 0, lc = 0;
-    for (int s = s0; s < s1; ++s) {
-      const int n = sc.seg_start[s + 1] - sc.seg_start[s];
-      const int r = p.pool.rank[sc.seg_adapter[s]];
-      const int nt = nt_class(n);
-      const int ntg = cdiv_i(n, nt), nrg = cdiv_i(G.n * r, rw_of(nt));
-      lt += p.do_shrink ? nrg * ntg * n_kc : 0;
-      lc += p.do_shrink ? nrg * ntg : 0;
-    }
-    int tt, tc;
-    int bt = block_exscan<false>(lt, &tt, sh);
-    int bc = block_exscan<false>(lc, &tc, sh);
-    int32_t* pt = sc.shrink_prefix + g * (sc.MS + 1);
-    int32_t* pc = sc.ctr_prefix + g * (sc.MS + 1);
-    for (int s = s0; s < s1; ++s) {
-      const int n = sc.seg_start[s + 1] - sc.seg_start[s];
-      const int r = p.pool.rank[sc.seg_adapter[s]];
-      const int nt = nt_class(n);
-      const int ntg = cdiv_i(n, nt), nrg = cdiv_i(G.n * r, rw_of(nt));
-      pt[s] = bt;  // group-local prefix
-      pc[s] = tot_ctr + bc;
-      bt += p.do_shrink ? nrg * ntg * n_kc : 0;
-      bc += p.do_shrink ? nrg * ntg : 0;
-    }
-    if (tid == 0) pt[S] = tt, pc[S] = tot_ctr + tc;
-    tot_shrink += tt;
-    tot_ctr += tc;
-  }
-  for (int k = 0; k < p.n_slots; ++k) {
-    const SlotDev& L = p.slot[k];
-    int le = 0;
-    for (int s = s0; s < s1; ++s) {
-      const int n = sc.seg_start[s + 1] - sc.seg_start[s];
-      const int r = p.pool.rank[sc.seg_adapter[s]];
-      le += (p.do_expand && r > 0) ? cdiv_i(n, nte_class(n)) * cdiv_i(L.d_out, lc_of(r)) : 0;
-    }
-    int te;
-    int be = block_exscan<false>(le, &te, sh);
-    int32_t* pe = sc.expand_prefix + k * (sc.MS + 1);
-    for (int s = s0; s < s1; ++s) {
-      const int n = sc.seg_start[s + 1] - sc.seg_start[s];
-      const int r = p.pool.rank[sc.seg_adapter[s]];
-      pe[s] = be;
-      be += (p.do_expand && r > 0) ? cdiv_i(n, nte_class(n)) * cdiv_i(L.d_out, lc_of(r)) : 0;
-    }
-    if (tid == 0) pe[S] = te;
-    tot_expand += te;
-  }
-  if (tid == 0) {
-    s_tot[0] = tot_shrink;
-    s_tot[1] = tot_ctr;
-  }
-  __syncthreads();
-  int ctr_total = s_tot[1];
+  int ctr_total = tot_ctr;
   if (ctr_total > sc.ctr_cap) {  // cannot happen with the sizing in slora_scratch_bytes
     if (tid == 0) record_error(p.pool.err, 3, ctr_total);
     ctr_total = 0;
@@ -275,12 +400,10 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
     sc.meta[kMetaShrinkTotal] = tot_shrink;
     sc.meta[kMetaExpandTotal] = tot_expand;
     sc.meta[kMetaCtrTotal] = ctr_total;
-    sc.meta[kMetaShrinkWork] = 0;
-    sc.meta[kMetaExpandWork] = 0;
   }
 }
 
-// Largest s with prefix[s] <= q (prefix ascending, prefix[0] = 0).
+// Largest s with prefix[s] <= q (prefix ascending from 0).
 __device__ __forceinline__ int find_seg(const int32_t* prefix, int S, int q) {
   int lo = 0, hi = S - 1;
   while (lo < hi) {
@@ -295,7 +418,6 @@ __device__ __forceinline__ int find_seg(const int32_t* prefix, int S, int q) {
 // holds the total of value L % N.  N is a power of two <= 32.
 template <int N>
 __device__ __forceinline__ float lane_transpose_reduce(float (&v)[N]) {
-  // fold lanes that share an output first
 #pragma unroll
   for (int o = 16; o >= N; o >>= 1) {
 #pragma unroll
@@ -316,254 +438,367 @@ __device__ __forceinline__ float lane_transpose_reduce(float (&v)[N]) {
 }
 
 // ---------------------------------------------------------------------------
-// Shrink task: RW rank rows x NT tokens x one d_in chunk.
-template <int DT, int NT, int RW>
-__device__ __noinline__ void shrink_task(const BgmvParams& p, const GroupDev& G, int a, int r,
-                                            int seg0, int n, int rg, int tg, int kc, int n_kc,
-                                            int ci) {
-  const int lane = threadIdx.x & 31;
-  const PoolDev& P = p.pool;
-  const int R = G.n * r;
-  const int k0 = kc * kShrinkKC, k1 = min(G.d_in, k0 + kShrinkKC);
+// Shrink.
+struct STask {
+  int g, s, a, r, seg0, n, nt, rw, rg, tg, kc, n_kc, ci;
+};
 
-  // rows
-  int row_lo[RW];
-  int64_t row_f[RW];
-  bool row_ok[RW];
-#pragma unroll
-  for (int i = 0; i < RW; ++i) {
-    const int rho = rg * RW + i;
-    row_ok[i] = rho < R;
-    const int j = row_ok[i] ? rho / r : 0, k = row_ok[i] ? rho % r : 0;
-    row_lo[i] = p.slot[G.slot[j]].listA;
-    row_f[i] = (int64_t)k * G.d_in;
+__device__ __forceinline__ bool decode_shrink(const BgmvParams& p, int S, int task, STask& t) {
+  const ScratchDev& sc = p.sc;
+  int g = 0, base = 0;
+  for (; g < p.n_groups; ++g) {
+    const int tg_tot = __ldg(sc.shrink_prefix + g * (sc.MS + 1) + S);
+    if (task < base + tg_tot) break;
+    base += tg_tot;
   }
-  // tokens
-  const uint16_t* xrow[NT];
-  bool tok_ok[NT];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int q = tg * NT + t;
-    tok_ok[t] = q < n;
-    const int token = tok_ok[t] ? __ldg(p.sc.perm + seg0 + q) : 0;
-    xrow[t] = G.x + (int64_t)token * G.ldx;
+  if (g >= p.n_groups) return false;
+  const int32_t* pre = sc.shrink_prefix + g * (sc.MS + 1);
+  const int s = find_seg(pre, S, task - base);
+  int q = task - base - __ldg(pre + s);
+  t.g = g;
+  t.s = s;
+  t.a = __ldg(sc.seg_adapter + s);
+  t.seg0 = __ldg(sc.seg_start + s);
+  t.n = __ldg(sc.seg_start + s + 1) - t.seg0;
+  t.r = __ldg(p.pool.rank + t.a);
+  t.nt = nt_class(t.n);
+  t.rw = rw_of(t.nt);
+  const int n_tg = cdiv_i(t.n, t.nt);
+  t.n_kc = cdiv_i(p.group[g].d_in, kShrinkKC);
+  t.tg = q % n_tg;
+  q /= n_tg;
+  t.kc = q % t.n_kc;
+  t.rg = q / t.n_kc;
+  t.ci = __ldg(sc.ctr_prefix + g * (sc.MS + 1) + s) + t.rg * n_tg + t.tg;
+  return true;
+}
+
+// Slot layout: rank row i at i * 1 KiB, token row t at (rw + t) * 1 KiB.
+__device__ __forceinline__ void issue_shrink(const BgmvParams& p, const STask& t, unsigned char* buf,
+                                             uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  const GroupDev& G = p.group[t.g];
+  const int k0 = t.kc * kShrinkKC;
+  const int L = min(kShrinkKC, G.d_in - k0);
+  const int R = G.n * t.r;
+  const int nrows = min(t.rw, R - t.rg * t.rw);
+  const int ntok = min(t.nt, t.n - t.tg * t.nt);
+  if (lane == 0) mbar_expect_tx(bar, 2u * L * (nrows + ntok));
+  __syncwarp();
+  const int i = lane & 15;
+  if (i < nrows) {
+    const int rho = t.rg * t.rw + i;
+    const int j = rho / t.r, k = rho % t.r;
+    const int lo = p.slot[G.slot[j]].listA;
+    bulk_paged_piece(p.pool, t.a, lo, (int64_t)k * G.d_in + k0, L, lane >> 4, buf + i * 2 * kShrinkKC, bar);
+  } else if (lane < 16 && i >= nrows && i < nrows + ntok) {
+    const int tt = i - nrows;
+    const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
+    bulk_g2s(buf + (t.rw + tt) * 2 * kShrinkKC, G.x + (int64_t)token * G.ldx + k0, 2u * L, bar);
   }
+}
+
+template <int DT, int NT, int RW>
+__device__ __forceinline__ void compute_shrink(const BgmvParams& p, const STask& t,
+                                               const unsigned char* buf) {
+  const int lane = threadIdx.x & 31;
+  const GroupDev& G = p.group[t.g];
+  const PoolDev& P = p.pool;
+  const int k0 = t.kc * kShrinkKC;
+  const int L = min(kShrinkKC, G.d_in - k0);
+  const int R = G.n * t.r;
+  const int nrows = min(RW, R - t.rg * RW);
+  const int ntok = min(NT, t.n - t.tg * NT);
 
   float acc[RW * NT];
 #pragma unroll
   for (int i = 0; i < RW * NT; ++i) acc[i] = 0.f;
-
-#pragma unroll 1
-  for (int e0 = k0 + lane * 8; e0 < k1; e0 += 256) {
+#pragma unroll
+  for (int e = lane * 8; e < kShrinkKC; e += 256) {
+    if (e >= L) break;
     uint4 av[RW], xv[NT];
 #pragma unroll
-    for (int i = 0; i < RW; ++i)
-      av[i] = row_ok[i] ? ldg_nc(page_addr(P, a, row_lo[i], row_f[i] + e0)) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < RW; ++i) av[i] = i < nrows ? lds128(buf + i * 2 * kShrinkKC + 2 * e) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int t = 0; t < NT; ++t)
-      xv[t] = tok_ok[t] ? __ldg(reinterpret_cast<const uint4*>(xrow[t] + e0)) : make_uint4(0, 0, 0, 0);
-    if (NT <= 2) {  // few tokens: unpack x once, stream the rows
+    for (int tt = 0; tt < NT; ++tt)
+      xv[tt] = tt < ntok ? lds128(buf + (RW + tt) * 2 * kShrinkKC + 2 * e) : make_uint4(0, 0, 0, 0);
+    if (NT <= 2) {
       float xf[NT][8];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) unpack8<DT>(xv[t], xf[t]);
+      for (int tt = 0; tt < NT; ++tt) unpack8<DT>(xv[tt], xf[tt]);
 #pragma unroll
       for (int i = 0; i < RW; ++i) {
         float af[8];
         unpack8<DT>(av[i], af);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          float s = acc[i * NT + t];
+        for (int tt = 0; tt < NT; ++tt) {
+          float s = acc[i * NT + tt];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s = fmaf(af[e], xf[t][e], s);
-          acc[i * NT + t] = s;
+          for (int q = 0; q < 8; ++q) s = fmaf(af[q], xf[tt][q], s);
+          acc[i * NT + tt] = s;
         }
       }
-    } else {        // many tokens: unpack the rows once, stream the tokens
+    } else {
       float af[RW][8];
 #pragma unroll
       for (int i = 0; i < RW; ++i) unpack8<DT>(av[i], af[i]);
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
+      for (int tt = 0; tt < NT; ++tt) {
         float xf[8];
-        unpack8<DT>(xv[t], xf);
+        unpack8<DT>(xv[tt], xf);
 #pragma unroll
         for (int i = 0; i < RW; ++i) {
-          float s = acc[i * NT + t];
+          float s = acc[i * NT + tt];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s = fmaf(af[i][e], xf[e], s);
-          acc[i * NT + t] = s;
+          for (int q = 0; q < 8; ++q) s = fmaf(af[i][q], xf[q], s);
+          acc[i * NT + tt] = s;
         }
       }
     }
   }
 
-  const float v = lane_transpose_reduce<RW * NT>(acc);
-  const int L = lane % (RW * NT);
-  const int i = L / NT, t = L % NT;
-  const int rho = rg * RW + i;
-  const int q = tg * NT + t;
-  const bool mine = lane < RW * NT && rho < R && q < n;
-  const int j = rho / r, k = rho % r;
-  const SlotDev& S = p.slot[G.slot[mine ? j : 0]];
-  const int pos = seg0 + q;
-  if (n_kc == 1) {
+  const float val = lane_transpose_reduce<RW * NT>(acc);
+  const int Lx = lane % (RW * NT);
+  const int i = Lx / NT, tt = Lx % NT;
+  const int rho = t.rg * RW + i;
+  const bool mine = lane < RW * NT && i < nrows && tt < ntok;
+  const int j = mine ? rho / t.r : 0, k = mine ? rho % t.r : 0;
+  const SlotDev& S = p.slot[G.slot[j]];
+  const int pos = t.seg0 + t.tg * NT + tt;
+  if (t.n_kc == 1) {
     if (mine) {
       const int64_t row = S.t_by_token ? (int64_t)__ldg(p.sc.perm + pos) : (int64_t)pos;
-      S.tfin[row * S.ldt + k] = v;
+      S.tfin[row * S.ldt + k] = val;
     }
     return;
   }
-  if (mine) S.tpart[((int64_t)kc * p.max_tokens + pos) * P.max_rank + k] = v;
+  if (mine) S.tpart[((int64_t)t.kc * p.max_tokens + pos) * P.max_rank + k] = val;
   __threadfence();
   __syncwarp();
   int old = 0;
-  if (lane == 0) old = atomicAdd(p.sc.ctr + ci, 1);
+  if (lane == 0) old = atomicAdd(p.sc.ctr + t.ci, 1);
   old = __shfl_sync(FULL_MASK, old, 0);
-  if (old != n_kc - 1) return;
+  if (old != t.n_kc - 1) return;
   __threadfence();
   if (mine) {  // last of the n_kc chunk tasks: sum the partials in chunk order
     float s = 0.f;
-    for (int c = 0; c < n_kc; ++c) s += __ldcg(S.tpart + ((int64_t)c * p.max_tokens + pos) * P.max_rank + k);
+    for (int c = 0; c < t.n_kc; ++c)
+      s += __ldcg(S.tpart + ((int64_t)c * p.max_tokens + pos) * P.max_rank + k);
     const int64_t row = S.t_by_token ? (int64_t)__ldg(p.sc.perm + pos) : (int64_t)pos;
     S.tfin[row * S.ldt + k] = s;
   }
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads, 2) k_shrink(const __grid_constant__ BgmvParams p) {
-  const int lane = threadIdx.x & 31;
-  const ScratchDev& sc = p.sc;
-  const int S = sc.meta[kMetaS];
-  const int total = sc.meta[kMetaShrinkTotal];
-  for (;;) {
-    int task = 0;
-    if (lane == 0) task = atomicAdd(sc.meta + kMetaShrinkWork, 1);
-    task = __shfl_sync(FULL_MASK, task, 0);
-    if (task >= total) return;
-    int g = 0, base = 0;
-    for (; g < p.n_groups; ++g) {
-      const int tg_tot = sc.shrink_prefix[g * (sc.MS + 1) + S];
-      if (task < base + tg_tot) break;
-      base += tg_tot;
-    }
-    const GroupDev& G = p.group[g];
-    const int32_t* pre = sc.shrink_prefix + g * (sc.MS + 1);
-    const int s = find_seg(pre, S, task - base);
-    int q = task - base - pre[s];
-    const int a = sc.seg_adapter[s];
-    const int seg0 = sc.seg_start[s], n = sc.seg_start[s + 1] - seg0;
-    const int r = p.pool.rank[a];
-    const int nt = nt_class(n);
-    const int n_tg = cdiv_i(n, nt), n_kc = cdiv_i(G.d_in, kShrinkKC);
-    const int tg = q % n_tg;
-    q /= n_tg;
-    const int kc = q % n_kc, rg = q / n_kc;
-    const int ci = sc.ctr_prefix[g * (sc.MS + 1) + s] + rg * n_tg + tg;
-    switch (nt) {
-      case 1: shrink_task<DT, 1, 8>(p, G, a, r, seg0, n, rg, tg, kc, n_kc, ci); break;
-      case 2: shrink_task<DT, 2, 4>(p, G, a, r, seg0, n, rg, tg, kc, n_kc, ci); break;
-      case 4: shrink_task<DT, 4, 4>(p, G, a, r, seg0, n, rg, tg, kc, n_kc, ci); break;
-      default: shrink_task<DT, 8, 4>(p, G, a, r, seg0, n, rg, tg, kc, n_kc, ci); break;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Expand task: NT tokens x LC outputs of one projection.
-template <int DT, int NT>
-__device__ __forceinline__ void expand_task(const BgmvParams& p, const SlotDev& L, int a, int r,
-                                            int seg0, int n, int tg, int lc) {
-  const int lane = threadIdx.x & 31;
-  const PoolDev& P = p.pool;
-  const float s_a = P.scale[a];
-  const int LC = lc_of(r);
-  int token[NT];
-  bool tok_ok[NT];
-  const float* trow[NT];
-#pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    const int q = tg * NT + t;
-    tok_ok[t] = q < n;
-    const int pos = seg0 + (tok_ok[t] ? q : 0);
-    token[t] = __ldg(p.sc.perm + pos);
-    trow[t] = L.tfin + (L.t_by_token ? (int64_t)token[t] : (int64_t)pos) * L.ldt;
-  }
-  const int l_end = min(L.d_out, (lc + 1) * LC);
-  for (int l = lc * LC + lane * 8; l - lane * 8 < l_end; l += 256) {
-    const bool act = l < l_end;
-    float acc[NT][8];
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[t][e] = 0.f;
-#pragma unroll 1
-    for (int k0 = 0; k0 < r; k0 += 4) {
-      uint4 bv[4];
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        bv[kk] = (act && k0 + kk < r) ? ldg_nc(page_addr(P, a, L.listB, (int64_t)(k0 + kk) * L.d_out + l))
-                                      : make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        float bf[8];
-        unpack8<DT>(bv[kk], bf);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const float tv = (k0 + kk < r) ? __ldg(trow[t] + k0 + kk) : 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[t][e] = fmaf(tv, bf[e], acc[t][e]);
-        }
-      }
-    }
-    if (!act) continue;
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      if (!tok_ok[t]) continue;
-      float yf[8];
-      unpack8<DT>(*reinterpret_cast<const uint4*>(L.y + (int64_t)token[t] * L.ldy + l), yf);
-      uint4 o;
-      o.x = pack2<DT>(fmaf(s_a, acc[t][0], yf[0]), fmaf(s_a, acc[t][1], yf[1]));
-      o.y = pack2<DT>(fmaf(s_a, acc[t][2], yf[2]), fmaf(s_a, acc[t][3], yf[3]));
-      o.z = pack2<DT>(fmaf(s_a, acc[t][4], yf[4]), fmaf(s_a, acc[t][5], yf[5]));
-      o.w = pack2<DT>(fmaf(s_a, acc[t][6], yf[6]), fmaf(s_a, acc[t][7], yf[7]));
-      *reinterpret_cast<uint4*>(L.y + (int64_t)token[t] * L.ldy + l) = o;
-    }
+__device__ __forceinline__ void compute_shrink_any(const BgmvParams& p, const STask& t,
+                                                   const unsigned char* buf) {
+  switch (t.nt) {
+    case 1: compute_shrink<DT, 1, 8>(p, t, buf); break;
+    case 2: compute_shrink<DT, 2, 4>(p, t, buf); break;
+    case 4: compute_shrink<DT, 4, 4>(p, t, buf); break;
+    default: compute_shrink<DT, 8, 4>(p, t, buf); break;
   }
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kThreads, 2) k_expand(const __grid_constant__ BgmvParams p) {
-  const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kWarps * 32, 1) k_shrink(const __grid_constant__ BgmvParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bars[kWarps][kSlots];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* wbuf = smem + warp * kSlots * kSlotBytes;
+  if (lane == 0)
+    for (int s = 0; s < kSlots; ++s) mbar_init(&bars[warp][s], 1);
+  fence_mbar_init();
+  __syncwarp();
+  griddep_wait();
+  const int S = p.sc.meta[kMetaS];
+  const int total = p.sc.meta[kMetaShrinkTotal];
+  const int NW = gridDim.x * kWarps;
+  int task = blockIdx.x * kWarps + warp;
+  STask cur, nxt;
+  bool have = task < total && decode_shrink(p, S, task, cur);
+  if (have) issue_shrink(p, cur, wbuf, &bars[warp][0]);
+  int slot = 0;
+  uint32_t parity = 0;
+  while (have) {
+    const int ntask = task + NW;
+    const bool hn = ntask < total && decode_shrink(p, S, ntask, nxt);
+    if (hn) issue_shrink(p, nxt, wbuf + (slot ^ 1) * kSlotBytes, &bars[warp][slot ^ 1]);
+    if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
+    parity ^= 1u << slot;
+    compute_shrink_any<DT>(p, cur, wbuf + slot * kSlotBytes);
+    __syncwarp();
+    fence_proxy_async();
+    slot ^= 1;
+    task = ntask;
+    cur = nxt;
+    have = hn;
+  }
+  griddep_launch();
+}
+
+// ---------------------------------------------------------------------------
+// Expand.
+struct ETask {
+  int k, s, a, r, seg0, n, nt, tg, lc, nks;
+};
+
+__device__ __forceinline__ bool decode_expand(const BgmvParams& p, int S, int task, ETask& t) {
   const ScratchDev& sc = p.sc;
-  const int S = sc.meta[kMetaS];
-  const int total = sc.meta[kMetaExpandTotal];
-  for (;;) {
-    int task = 0;
-    if (lane == 0) task = atomicAdd(sc.meta + kMetaExpandWork, 1);
-    task = __shfl_sync(FULL_MASK, task, 0);
-    if (task >= total) return;
-    int k = 0, base = 0;
-    for (; k < p.n_slots; ++k) {
-      const int tk = sc.expand_prefix[k * (sc.MS + 1) + S];
-      if (task < base + tk) break;
-      base += tk;
-    }
-    const SlotDev& L = p.slot[k];
-    const int32_t* pre = sc.expand_prefix + k * (sc.MS + 1);
-    const int s = find_seg(pre, S, task - base);
-    const int q = task - base - pre[s];
-    const int a = sc.seg_adapter[s];
-    const int seg0 = sc.seg_start[s], n = sc.seg_start[s + 1] - seg0;
-    const int r = p.pool.rank[a];
-    const int nt = nte_class(n);
-    const int n_tg = cdiv_i(n, nt);
-    const int tg = q % n_tg, lc = q / n_tg;
-    switch (nt) {
-      case 1: expand_task<DT, 1>(p, L, a, r, seg0, n, tg, lc); break;
-      case 2: expand_task<DT, 2>(p, L, a, r, seg0, n, tg, lc); break;
-      default: expand_task<DT, 4>(p, L, a, r, seg0, n, tg, lc); break;
+  int k = 0, base = 0;
+  for (; k < p.n_slots; ++k) {
+    const int tk = __ldg(sc.expand_prefix + k * (sc.MS + 1) + S);
+    if (task < base + tk) break;
+    base += tk;
+  }
+  if (k >= p.n_slots) return false;
+  const int32_t* pre = sc.expand_prefix + k * (sc.MS + 1);
+  const int s = find_seg(pre, S, task - base);
+  const int q = task - base - __ldg(pre + s);
+  t.k = k;
+  t.s = s;
+  t.a = __ldg(sc.seg_adapter + s);
+  t.seg0 = __ldg(sc.seg_start + s);
+  t.n = __ldg(sc.seg_start + s + 1) - t.seg0;
+  t.r = __ldg(p.pool.rank + t.a);
+  t.nt = nte_class(t.n);
+  const int n_tg = cdiv_i(t.n, t.nt);
+  t.tg = q % n_tg;
+  t.lc = q / n_tg;
+  t.nks = cdiv_i(t.r, kExpandRows);
+  return true;
+}
+
+// Slot layout: B row i of this stage at i * 512 B; in the last stage of a
+// task, y row t at (16 + t) * 512 B.
+__device__ __forceinline__ void issue_expand(const BgmvParams& p, const ETask& t, int ks,
+                                             unsigned char* buf, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  const SlotDev& L = p.slot[t.k];
+  const int l0 = t.lc * kLC;
+  const int Lo = min(kLC, L.d_out - l0);
+  const int r0 = ks * kExpandRows;
+  const int nrows = min(kExpandRows, t.r - r0);
+  const bool last = ks == t.nks - 1;
+  const int ntok = last ? min(t.nt, t.n - t.tg * t.nt) : 0;
+  if (lane == 0) mbar_expect_tx(bar, 2u * Lo * (nrows + ntok));
+  __syncwarp();
+  const int i = lane & 15;
+  if (i < nrows)
+    bulk_paged_piece(p.pool, t.a, L.listB, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 4,
+                     buf + i * 2 * kLC, bar);
+  if (lane < ntok) {
+    const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
+    bulk_g2s(buf + (kExpandRows + lane) * 2 * kLC, L.y + (int64_t)token * L.ldy + l0, 2u * Lo, bar);
+  }
+}
+
+template <int DT>
+__device__ __forceinline__ void compute_expand(const BgmvParams& p, const ETask& t, int ks,
+                                               const unsigned char* buf, float (&acc)[4][8]) {
+  const int lane = threadIdx.x & 31;
+  const SlotDev& L = p.slot[t.k];
+  const int l0 = t.lc * kLC;
+  const int Lo = min(kLC, L.d_out - l0);
+  const int r0 = ks * kExpandRows;
+  const int nrows = min(kExpandRows, t.r - r0);
+  const int ntok = min(t.nt, t.n - t.tg * t.nt);
+  const int l = lane * 8;
+  const bool act = l < Lo;
+  const float* trow[4];
+  int token[4];
+#pragma unroll
+  for (int tt = 0; tt < 4; ++tt) {
+    const int pos = t.seg0 + t.tg * t.nt + (tt < ntok ? tt : 0);
+    token[tt] = __ldg(p.sc.perm + pos);
+    trow[tt] = L.tfin + (L.t_by_token ? (int64_t)token[tt] : (int64_t)pos) * L.ldt + r0;
+  }
+  if (act) {
+#pragma unroll 4
+    for (int kk = 0; kk < nrows; ++kk) {
+      float bf[8];
+      unpack8<DT>(lds128(buf + kk * 2 * kLC + 2 * l), bf);
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        if (tt >= ntok) break;
+        const float tv = __ldg(trow[tt] + kk);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tv, bf[e], acc[tt][e]);
+      }
     }
   }
+  if (ks != t.nks - 1) return;
+  const float s_a = __ldg(p.pool.scale + t.a);
+  if (act) {
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+      if (tt >= ntok) break;
+      float yf[8];
+      unpack8<DT>(lds128(buf + (kExpandRows + tt) * 2 * kLC + 2 * l), yf);
+      uint4 o;
+      o.x = pack2<DT>(fmaf(s_a, acc[tt][0], yf[0]), fmaf(s_a, acc[tt][1], yf[1]));
+      o.y = pack2<DT>(fmaf(s_a, acc[tt][2], yf[2]), fmaf(s_a, acc[tt][3], yf[3]));
+      o.z = pack2<DT>(fmaf(s_a, acc[tt][4], yf[4]), fmaf(s_a, acc[tt][5], yf[5]));
+      o.w = pack2<DT>(fmaf(s_a, acc[tt][6], yf[6]), fmaf(s_a, acc[tt][7], yf[7]));
+      *reinterpret_cast<uint4*>(L.y + (int64_t)token[tt] * L.ldy + l0 + l) = o;
+    }
+  }
+#pragma unroll
+  for (int tt = 0; tt < 4; ++tt)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kWarps * 32, 1) k_expand(const __grid_constant__ BgmvParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bars[kWarps][kSlots];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned char* wbuf = smem + warp * kSlots * kSlotBytes;
+  if (lane == 0)
+    for (int s = 0; s < kSlots; ++s) mbar_init(&bars[warp][s], 1);
+  fence_mbar_init();
+  __syncwarp();
+  griddep_wait();
+  const int S = p.sc.meta[kMetaS];
+  const int total = p.sc.meta[kMetaExpandTotal];
+  const int NW = gridDim.x * kWarps;
+  int task = blockIdx.x * kWarps + warp;
+  ETask cur, nxt;
+  bool have = task < total && decode_expand(p, S, task, cur);
+  int ks = 0;
+  if (have) issue_expand(p, cur, 0, wbuf, &bars[warp][0]);
+  float acc[4][8];
+#pragma unroll
+  for (int tt = 0; tt < 4; ++tt)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
+  int slot = 0;
+  uint32_t parity = 0;
+  while (have) {
+    // next stage: the next rank chunk of this task, or the first of the next task
+    int nks = ks + 1, ntask = task;
+    bool hn = true;
+    if (nks >= cur.nks) {
+      nks = 0;
+      ntask = task + NW;
+      hn = ntask < total && decode_expand(p, S, ntask, nxt);
+    } else {
+      nxt = cur;
+    }
+    if (hn) issue_expand(p, nxt, nks, wbuf + (slot ^ 1) * kSlotBytes, &bars[warp][slot ^ 1]);
+    if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
+    parity ^= 1u << slot;
+    compute_expand<DT>(p, cur, ks, wbuf + slot * kSlotBytes, acc);
+    __syncwarp();
+    fence_proxy_async();
+    slot ^= 1;
+    task = ntask;
+    ks = nks;
+    cur = nxt;
+    have = hn;
+  }
+  griddep_launch();
 }
 
 // ---------------------------------------------------------------------------
@@ -695,27 +930,50 @@ __global__ void k_gather_debug(PoolDev P, int id, int d, int list_off, int rank,
 
 // ---------------------------------------------------------------------------
 // Launchers.
+template <typename Kern>
+static cudaError_t launch_dependent(Kern kernel, int grid, int block, size_t smem, cudaStream_t s,
+                                    const BgmvParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+static bool g_attrs_done = false;
+static void set_attrs() {
+  if (g_attrs_done) return;
+  cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(k_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(k_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  g_attrs_done = true;
+}
+
 cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cudaStream_t s) {
+  set_attrs();
   const size_t smem = sizeof(int) * (size_t)p.pool.max_adapters;
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024 + 1024);
-    attr_done = true;
-  }
   k_segments<<<1, 1024, smem, s>>>(p, idx, T);
   return cudaGetLastError();
 }
 
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
-  if (dtype == SLORA_BF16) k_shrink<SLORA_BF16><<<grid, kThreads, 0, s>>>(p);
-  else k_shrink<SLORA_F16><<<grid, kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  set_attrs();
+  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kWarps * 32, kSmemBytes, s, p);
+  return launch_dependent(k_shrink<SLORA_F16>, grid, kWarps * 32, kSmemBytes, s, p);
 }
 
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
-  if (dtype == SLORA_BF16) k_expand<SLORA_BF16><<<grid, kThreads, 0, s>>>(p);
-  else k_expand<SLORA_F16><<<grid, kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  set_attrs();
+  if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kWarps * 32, kSmemBytes, s, p);
+  return launch_dependent(k_expand<SLORA_F16>, grid, kWarps * 32, kSmemBytes, s, p);
 }
 
 cudaError_t launch_merge_requests(const int32_t* req_start, const int32_t* req_adapter, int n,
@@ -749,10 +1007,12 @@ cudaError_t launch_gather_debug(const PoolDev& pool, int id, int d, int list_off
   return cudaGetLastError();
 }
 
+// Resident CTAs per SM of the persistent decode kernels (shared memory bound).
 int occupancy_blocks(int which) {
+  set_attrs();
   int n = 0;
-  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kThreads, 0);
-  else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kThreads, 0);
+  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kWarps * 32, kSmemBytes);
+  else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kWarps * 32, kSmemBytes);
   return n > 0 ? n : 1;
 }
 

@@ -253,8 +253,15 @@ void wait_epoch(slora_pool* P, cudaStream_t s, int64_t epoch) {
   if (P->ev_epoch[slot] >= epoch) cudaStreamWaitEvent(s, P->ev[slot], 0);
 }
 
-void phase(slora_pool* P, int k, cudaStream_t s) {
-  if (P->n_phase >= 4 && k < P->n_phase) cudaEventRecord(P->phase_ev[k], s);
+// Timing hook: with 2 events only the call's start and end are recorded (the
+// kernels stay back to back); with >= 4 also the boundaries between kernels.
+void phase(slora_pool* P, int k, int last, cudaStream_t s) {
+  if (P->n_phase == 2) {
+    if (k == 0) cudaEventRecord(P->phase_ev[0], s);
+    else if (k == last) cudaEventRecord(P->phase_ev[1], s);
+  } else if (P->n_phase >= 4 && k < P->n_phase) {
+    cudaEventRecord(P->phase_ev[k], s);
+  }
 }
 
 void record_epoch(slora_pool* P, cudaStream_t s) {
@@ -876,13 +883,13 @@ slora_status_t slora_lora_delta(slora_pool* P, int32_t n, const int32_t* projs, 
   bp.do_shrink = 1;
   bp.do_expand = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  phase(P, 0, st);
+  phase(P, 0, 3, st);
   CUDA_TRY(P, launch_segments(bp, idx, T, st));
-  phase(P, 1, st);
+  phase(P, 1, 3, st);
   CUDA_TRY(P, launch_shrink(bp, P->d.dtype, P->grid_shrink, st));
-  phase(P, 2, st);
+  phase(P, 2, 3, st);
   CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
-  phase(P, 3, st);
+  phase(P, 3, 3, st);
   record_epoch(P, st);
   return SLORA_OK;
 }
@@ -1011,7 +1018,8 @@ slora_status_t slora_pool_stats(const slora_pool* P, slora_pool_stats_t* out) {
 
 slora_status_t slora_set_phase_events(slora_pool* P, void* const* events, int32_t n) {
   if (!P) return SLORA_ERR_INVALID_ARG;
-  if (n < 0 || n > 8 || (n > 0 && !events)) return P->fail(SLORA_ERR_INVALID_ARG, "events");
+  if (n < 0 || n > 8 || n == 1 || n == 3 || (n > 0 && !events))
+    return P->fail(SLORA_ERR_INVALID_ARG, "events: n must be 0, 2 or 4..8");
   for (int i = 0; i < n; ++i) {
     if (!events[i]) return P->fail(SLORA_ERR_INVALID_ARG, "event is NULL");
     P->phase_ev[i] = static_cast<cudaEvent_t>(events[i]);

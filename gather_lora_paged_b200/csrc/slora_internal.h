@@ -12,7 +12,7 @@ namespace slora {
 // Shrink work split (decode path).  A task covers RW rank rows x NT tokens x
 // KC elements of d_in; KC is fixed so every projection has a fixed number of
 // fp32 partial slices (ceil(d_in / KC)).
-constexpr int kShrinkKC = 1024;
+constexpr int kShrinkKC = 512;
 constexpr int kMaxSlots = SLORA_MAX_PROJ;   // projections per call
 constexpr int kThreads = 256;               // threads per CTA of the decode kernels
 constexpr int kEventRing = 64;

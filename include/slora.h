@@ -311,12 +311,13 @@ slora_status_t slora_check_device(slora_pool* pool, void* stream, int32_t* code,
 
 slora_status_t slora_pool_stats(const slora_pool* pool, slora_pool_stats_t* out);
 
-/* Timing hook: when n >= 4, every following compute call records events[0]
- * on its stream right before its first kernel and events[k] right after its
- * k-th kernel (segment build, shrink, expand for slora_lora_delta; plan,
- * shrink, expand for slora_sgmv).  Events are cudaEvent_t created by the
- * caller with timing enabled; n = 0 switches the hook off.  For measuring
- * per-kernel device time without host gaps.                                   */
+/* Timing hook for measuring device time without host gaps.  n = 2: every
+ * following compute call records events[0] on its stream right before its
+ * first kernel and events[1] right after its last one (the kernels stay back
+ * to back).  n >= 4: events[0] before the first kernel and events[k] right
+ * after its k-th kernel (segment build, shrink, expand for slora_lora_delta;
+ * plan, shrink, expand for slora_sgmv).  Events are cudaEvent_t created by
+ * the caller with timing enabled; n = 0 switches the hook off.                */
 slora_status_t slora_set_phase_events(slora_pool* pool, void* const* events, int32_t n);
 
 /* Fault injection, host side only: the `after`-th next page-in copy submission
