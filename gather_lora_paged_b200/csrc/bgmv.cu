@@ -190,53 +190,30 @@ __device__ int block_exscan(int v, int* total, int* sh) {
   return res;
 }
 
-// Exclusive sum-scan of V values per thread at once; v becomes the prefix,
-// tot the block totals.  sh: 32 * kV ints.
-constexpr int kV = 3 * kMaxSlots;
-__device__ void block_multiscan(int (&v)[kV], int (&tot)[kV], int* sh) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int ex[kV];
-#pragma unroll
-  for (int j = 0; j < kV; ++j) {
-    int x = v[j];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(FULL_MASK, x, o);
-      if (lane >= o) x += y;
-    }
-    ex[j] = x - v[j];
-    if (lane == 31) sh[w * kV + j] = x;
-  }
-  __syncthreads();
-  if (w == 0) {
-#pragma unroll
-    for (int j = 0; j < kV; ++j) {
-      int s = lane < nw ? sh[lane * kV + j] : 0;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(FULL_MASK, s, o);
-        if (lane >= o) s += y;
-      }
-      if (lane < nw) sh[lane * kV + j] = s;
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int j = 0; j < kV; ++j) {
-    v[j] = (w ? sh[(w - 1) * kV + j] : 0) + ex[j];
-    tot[j] = sh[(nw - 1) * kV + j];
-  }
-  __syncthreads();
-}
-
-// ---------------------------------------------------------------------------
 // k_segments: one CTA of 1024 threads.  Dynamic smem: max_adapters ints.
-constexpr int kMaxAdPerThread = 16;   // max_adapters <= 16384
+// Output: perm, segments (start, adapter, rank) and, per segment, the number
+// of shrink tasks, reduction counters and expand tasks before it (prefix sums
+// in segment-major task order).
+
+__device__ __forceinline__ void seg_task_counts(const BgmvParams& p, int n, int r, int& shr, int& ctr,
+                                                int& exp) {
+  shr = ctr = exp = 0;
+  if (n == 0 || r <= 0) return;
+  const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
+  if (p.do_shrink)
+    for (int g = 0; g < p.n_groups; ++g) {
+      const int nrg = cdiv_i(p.group[g].n * r, rw_of(nt));
+      shr += nrg * ntg * cdiv_i(p.group[g].d_in, kShrinkKC);
+      ctr += nrg * ntg;
+    }
+  if (p.do_expand)
+    for (int k = 0; k < p.n_slots; ++k) exp += nte * cdiv_i(p.slot[k].d_out, kLC);
+}
 
 __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvParams p,
                                                    const int32_t* __restrict__ idx, int T) {
   extern __shared__ int hist[];
-  __shared__ int sh[32 * kV];
+  __shared__ int sh[32];
   const int tid = threadIdx.x, nth = blockDim.x;
   const int MA = p.pool.max_adapters;
   const ScratchDev& sc = p.sc;
@@ -259,109 +236,64 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
   }
   __syncthreads();
 
-  // Each thread owns a contiguous adapter range; the segments it creates are a
-  // contiguous range of segment indices, which it also plans.
+  // Each thread owns a contiguous adapter range; the segments it creates form
+  // a contiguous range of segment indices.
   const int E = (MA + nth - 1) / nth;
   const int a0 = min(tid * E, MA), a1 = min(a0 + E, MA);
-  int segN[kMaxAdPerThread], segR[kMaxAdPerThread];
-  int cnt = 0, nseg = 0;
-#pragma unroll
-  for (int q = 0; q < kMaxAdPerThread; ++q) {
-    const int a = a0 + q;
-    segN[q] = (a < a1) ? hist[a] : 0;
-    segR[q] = (segN[q] > 0) ? p.pool.rank[a] : 0;
-    cnt += segN[q];
-    nseg += segN[q] > 0;
+  int cnt = 0, nseg = 0, c_shr = 0, c_ctr = 0, c_exp = 0;
+  for (int a = a0; a < a1; ++a) {
+    const int n = hist[a];
+    if (n == 0) continue;
+    int x, y, z;
+    seg_task_counts(p, n, p.pool.rank[a], x, y, z);
+    cnt += n;
+    nseg += 1;
+    c_shr += x;
+    c_ctr += y;
+    c_exp += z;
   }
-  int n_valid, S;
+  int n_valid, S, t_shr, t_ctr, t_exp;
   int cbase = block_exscan<false>(cnt, &n_valid, sh);
-  const int sbase = block_exscan<false>(nseg, &S, sh);
-  {
-    int sb = sbase;
-#pragma unroll
-    for (int q = 0; q < kMaxAdPerThread; ++q) {
-      const int a = a0 + q;
-      if (segN[q] > 0) {
-        sc.seg_start[sb] = cbase;
-        sc.seg_adapter[sb] = a;
-        ++sb;
-      }
-      if (a < a1) hist[a] = cbase;  // becomes the scatter cursor
-      cbase += segN[q];
-    }
+  int sb = block_exscan<false>(nseg, &S, sh);
+  int b_shr = block_exscan<false>(c_shr, &t_shr, sh);
+  int b_ctr = block_exscan<false>(c_ctr, &t_ctr, sh);
+  int b_exp = block_exscan<false>(c_exp, &t_exp, sh);
+  for (int a = a0; a < a1; ++a) {
+    const int n = hist[a];
+    hist[a] = cbase;  // becomes the scatter cursor
+    if (n == 0) continue;
+    const int r = p.pool.rank[a];
+    int x, y, z;
+    seg_task_counts(p, n, r, x, y, z);
+    sc.seg_start[sb] = cbase;
+    sc.seg_adapter[sb] = a;
+    sc.seg_rank[sb] = r;
+    sc.shrink_prefix[sb] = b_shr;
+    sc.ctr_prefix[sb] = b_ctr;
+    sc.expand_prefix[sb] = b_exp;
+    ++sb;
+    cbase += n;
+    b_shr += x;
+    b_ctr += y;
+    b_exp += z;
+  }
+  int ctr_total = t_ctr;
+  if (ctr_total > sc.ctr_cap) {  // cannot happen with the sizing in slora_scratch_bytes
+    if (tid == 0) record_error(p.pool.err, 3, ctr_total);
+    ctr_total = t_shr = t_exp = 0;
   }
   if (tid == 0) {
     sc.seg_start[S] = n_valid;
+    sc.shrink_prefix[S] = t_shr;
+    sc.ctr_prefix[S] = t_ctr;
+    sc.expand_prefix[S] = t_exp;
     sc.meta[kMetaS] = S;
     sc.meta[kMetaValid] = n_valid;
+    sc.meta[kMetaShrinkTotal] = t_shr;
+    sc.meta[kMetaExpandTotal] = t_exp;
+    sc.meta[kMetaCtrTotal] = ctr_total;
   }
-
-  // Work planning: per group shrink tasks and counters, per slot expand tasks.
-  int v[kV], tot[kV];
-#pragma unroll
-  for (int j = 0; j < kV; ++j) v[j] = 0;
-#pragma unroll
-  for (int q = 0; q < kMaxAdPerThread; ++q) {
-    const int n = segN[q], r = segR[q];
-    if (n == 0) continue;
-    const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
-#pragma unroll
-    for (int g = 0; g < kMaxSlots; ++g) {
-      if (g >= p.n_groups || !p.do_shrink) continue;
-      const int nrg = cdiv_i(p.group[g].n * r, rw_of(nt));
-      v[g] += nrg * ntg * cdiv_i(p.group[g].d_in, kShrinkKC);
-      v[kMaxSlots + g] += nrg * ntg;
-    }
-#pragma unroll
-    for (int k = 0; k < kMaxSlots; ++k) {
-      if (k >= p.n_slots || !p.do_expand || r == 0) continue;
-      v[2 * kMaxSlots + k] += nte * cdiv_i(p.slot[k].d_out, kLC);
-    }
-  }
-  block_multiscan(v, tot, sh);
-  int ctr_base[kMaxSlots];
-  int tot_shrink = 0, tot_ctr = 0, tot_expand = 0;
-#pragma unroll
-  for (int g = 0; g < kMaxSlots; ++g) {
-    ctr_base[g] = tot_ctr;
-    tot_shrink += tot[g];
-    tot_ctr += tot[kMaxSlots + g];
-    tot_expand += tot[2 * kMaxSlots + g];
-  }
-  {
-    int sb = sbase;
-#pragma unroll
-    for (int q = 0; q < kMaxAdPerThread; ++q) {
-      const int n = segN[q], r = segR[q];
-      if (n == 0) continue;
-      const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
-#pragma unroll
-      for (int g = 0; g < kMaxSlots; ++g) {
-        if (g >= p.n_groups) continue;
-        sc.shrink_prefix[g * (sc.MS + 1) + sb] = v[g];
-        sc.ctr_prefix[g * (sc.MS + 1) + sb] = ctr_base[g] + v[kMaxSlots + g];
-        if (!p.do_shrink) continue;
-        const int nrg = cdiv_i(p.group[g].n * r, rw_of(nt));
-        v[g] += nrg * ntg * cdiv_i(p.group[g].d_in, kShrinkKC);
-        v[kMaxSlots + g] += nrg * ntg;
-      }
-#pragma unroll
-      for (int k = 0; k < kMaxSlots; ++k) {
-        if (k >= p.n_slots) continue;
-        sc.expand_prefix[k * (sc.MS + 1) + sb] = v[2 * kMaxSlots + k];
-        if (!p.do_expand || r == 0) continue;
-        v[2 * kMaxSlots + k] += nte * cdiv_i(p.slot[k].d_out, kLC);
-      }
-      ++sb;
-    }
-  }
-  if (tid == 0) {
-    for (int g = 0; g < p.n_groups; ++g) {
-      sc.shrink_prefix[g * (sc.MS + 1) + S] = tot[g];
-      sc.ctr_prefix[g * (sc.MS + 1) + S] = ctr_base[g] + tot[kMaxSlots + g];
-    }
-    for (int k = 0; k < p.n_slots; ++k) sc.expand_prefix[k * (sc.MS + 1) + S] = tot[2 * kMaxSlots + k];
-  }
+  for (int c = tid; c < ctr_total; c += nth) sc.ctr[c] = 0;
   __syncthreads();
 
   // Stable scatter: chunks of 1024 tokens, warps take turns in order.
@@ -387,28 +319,14 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
       __syncthreads();
     }
   }
-
-  int ctr_total = tot_ctr;
-  if (ctr_total > sc.ctr_cap) {  // cannot happen with the sizing in slora_scratch_bytes
-    if (tid == 0) record_error(p.pool.err, 3, ctr_total);
-    ctr_total = 0;
-    tot_shrink = 0;
-    tot_expand = 0;
-  }
-  for (int c = tid; c < ctr_total; c += nth) sc.ctr[c] = 0;
-  if (tid == 0) {
-    sc.meta[kMetaShrinkTotal] = tot_shrink;
-    sc.meta[kMetaExpandTotal] = tot_expand;
-    sc.meta[kMetaCtrTotal] = ctr_total;
-  }
 }
 
-// Largest s with prefix[s] <= q (prefix ascending from 0).
+// Largest s with prefix[s] <= q (prefix ascending from 0, S >= 1).
 __device__ __forceinline__ int find_seg(const int32_t* prefix, int S, int q) {
   int lo = 0, hi = S - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(prefix + mid) <= q) lo = mid;
+    if (prefix[mid] <= q) lo = mid;
     else hi = mid - 1;
   }
   return lo;
@@ -438,39 +356,86 @@ __device__ __forceinline__ float lane_transpose_reduce(float (&v)[N]) {
 }
 
 // ---------------------------------------------------------------------------
-// Shrink.
-struct STask {
-  int g, s, a, r, seg0, n, nt, rw, rg, tg, kc, n_kc, ci;
+// Segment table as seen by the persistent kernels: staged in shared memory
+// when it fits (one round trip per CTA), else read from global memory.
+constexpr int kSegCap = 1024;
+struct SegView {
+  const int32_t* start;   // [S + 1]
+  const int32_t* adapter; // [S]
+  const int32_t* rank;    // [S]
+  const int32_t* prefix;  // [S + 1] tasks before each segment
+  const int32_t* ctr;     // [S + 1] counters before each segment (shrink only)
+  int S;
 };
 
-__device__ __forceinline__ bool decode_shrink(const BgmvParams& p, int S, int task, STask& t) {
-  const ScratchDev& sc = p.sc;
-  int g = 0, base = 0;
-  for (; g < p.n_groups; ++g) {
-    const int tg_tot = __ldg(sc.shrink_prefix + g * (sc.MS + 1) + S);
-    if (task < base + tg_tot) break;
-    base += tg_tot;
+__device__ SegView stage_segments(const ScratchDev& sc, int S, bool shrink, int32_t* sm) {
+  SegView v;
+  v.S = S;
+  const int32_t* pre = shrink ? sc.shrink_prefix : sc.expand_prefix;
+  if (S > kSegCap) {
+    v.start = sc.seg_start;
+    v.adapter = sc.seg_adapter;
+    v.rank = sc.seg_rank;
+    v.prefix = pre;
+    v.ctr = sc.ctr_prefix;
+    return v;
   }
-  if (g >= p.n_groups) return false;
-  const int32_t* pre = sc.shrink_prefix + g * (sc.MS + 1);
-  const int s = find_seg(pre, S, task - base);
-  int q = task - base - __ldg(pre + s);
-  t.g = g;
-  t.s = s;
-  t.a = __ldg(sc.seg_adapter + s);
-  t.seg0 = __ldg(sc.seg_start + s);
-  t.n = __ldg(sc.seg_start + s + 1) - t.seg0;
-  t.r = __ldg(p.pool.rank + t.a);
+  int32_t* st = sm;
+  int32_t* ad = sm + (kSegCap + 1);
+  int32_t* rk = ad + kSegCap;
+  int32_t* pf = rk + kSegCap;
+  int32_t* ct = pf + (kSegCap + 1);
+  for (int i = threadIdx.x; i <= S; i += blockDim.x) {
+    st[i] = sc.seg_start[i];
+    pf[i] = pre[i];
+    if (shrink) ct[i] = sc.ctr_prefix[i];
+    if (i < S) {
+      ad[i] = sc.seg_adapter[i];
+      rk[i] = sc.seg_rank[i];
+    }
+  }
+  __syncthreads();
+  v.start = st;
+  v.adapter = ad;
+  v.rank = rk;
+  v.prefix = pf;
+  v.ctr = ct;
+  return v;
+}
+constexpr int kSegSmemInts = 5 * kSegCap + 3;
+
+// ---------------------------------------------------------------------------
+// Shrink.
+struct STask {
+  int g, a, r, seg0, n, nt, rw, rg, tg, kc, n_kc, ci;
+};
+
+__device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView& V, int task, STask& t) {
+  const int s = find_seg(V.prefix, V.S, task);
+  int q = task - V.prefix[s];
+  t.a = V.adapter[s];
+  t.seg0 = V.start[s];
+  t.n = V.start[s + 1] - t.seg0;
+  t.r = V.rank[s];
   t.nt = nt_class(t.n);
   t.rw = rw_of(t.nt);
   const int n_tg = cdiv_i(t.n, t.nt);
+  int ci = V.ctr[s];
+  int g = 0;
+  for (; g < p.n_groups - 1; ++g) {  // the group owning local task q
+    const int nrg = cdiv_i(p.group[g].n * t.r, t.rw);
+    const int cnt = nrg * n_tg * cdiv_i(p.group[g].d_in, kShrinkKC);
+    if (q < cnt) break;
+    q -= cnt;
+    ci += nrg * n_tg;
+  }
+  t.g = g;
   t.n_kc = cdiv_i(p.group[g].d_in, kShrinkKC);
   t.tg = q % n_tg;
   q /= n_tg;
   t.kc = q % t.n_kc;
   t.rg = q / t.n_kc;
-  t.ci = __ldg(sc.ctr_prefix + g * (sc.MS + 1) + s) + t.rg * n_tg + t.tg;
-  return true;
+  t.ci = ci + t.rg * n_tg + t.tg;
 }
 
 // Slot layout: rank row i at i * 1 KiB, token row t at (rw + t) * 1 KiB.
@@ -491,7 +456,7 @@ __device__ __forceinline__ void issue_shrink(const BgmvParams& p, const STask& t
     const int j = rho / t.r, k = rho % t.r;
     const int lo = p.slot[G.slot[j]].listA;
     bulk_paged_piece(p.pool, t.a, lo, (int64_t)k * G.d_in + k0, L, lane >> 4, buf + i * 2 * kShrinkKC, bar);
-  } else if (lane < 16 && i >= nrows && i < nrows + ntok) {
+  } else if (lane < 16 && i < nrows + ntok) {
     const int tt = i - nrows;
     const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
     bulk_g2s(buf + (t.rw + tt) * 2 * kShrinkKC, G.x + (int64_t)token * G.ldx + k0, 2u * L, bar);
@@ -606,24 +571,31 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_shrink(const __grid_constant
   __shared__ __align__(8) uint64_t bars[kWarps][kSlots];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* wbuf = smem + warp * kSlots * kSlotBytes;
+  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kSmemBytes);
   if (lane == 0)
     for (int s = 0; s < kSlots; ++s) mbar_init(&bars[warp][s], 1);
   fence_mbar_init();
-  __syncwarp();
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaShrinkTotal];
+  const SegView V = stage_segments(p.sc, S, true, segsm);
   const int NW = gridDim.x * kWarps;
   int task = blockIdx.x * kWarps + warp;
   STask cur, nxt;
-  bool have = task < total && decode_shrink(p, S, task, cur);
-  if (have) issue_shrink(p, cur, wbuf, &bars[warp][0]);
+  bool have = task < total;
+  if (have) {
+    decode_shrink(p, V, task, cur);
+    issue_shrink(p, cur, wbuf, &bars[warp][0]);
+  }
   int slot = 0;
   uint32_t parity = 0;
   while (have) {
     const int ntask = task + NW;
-    const bool hn = ntask < total && decode_shrink(p, S, ntask, nxt);
-    if (hn) issue_shrink(p, nxt, wbuf + (slot ^ 1) * kSlotBytes, &bars[warp][slot ^ 1]);
+    const bool hn = ntask < total;
+    if (hn) {
+      decode_shrink(p, V, ntask, nxt);
+      issue_shrink(p, nxt, wbuf + (slot ^ 1) * kSlotBytes, &bars[warp][slot ^ 1]);
+    }
     if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
     parity ^= 1u << slot;
     compute_shrink_any<DT>(p, cur, wbuf + slot * kSlotBytes);
@@ -640,37 +612,36 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_shrink(const __grid_constant
 // ---------------------------------------------------------------------------
 // Expand.
 struct ETask {
-  int k, s, a, r, seg0, n, nt, tg, lc, nks;
+  int k, a, r, seg0, n, nt, tg, lc, nks;
 };
 
-__device__ __forceinline__ bool decode_expand(const BgmvParams& p, int S, int task, ETask& t) {
-  const ScratchDev& sc = p.sc;
-  int k = 0, base = 0;
-  for (; k < p.n_slots; ++k) {
-    const int tk = __ldg(sc.expand_prefix + k * (sc.MS + 1) + S);
-    if (task < base + tk) break;
-    base += tk;
-  }
-  if (k >= p.n_slots) return false;
-  const int32_t* pre = sc.expand_prefix + k * (sc.MS + 1);
-  const int s = find_seg(pre, S, task - base);
-  const int q = task - base - __ldg(pre + s);
-  t.k = k;
-  t.s = s;
-  t.a = __ldg(sc.seg_adapter + s);
-  t.seg0 = __ldg(sc.seg_start + s);
-  t.n = __ldg(sc.seg_start + s + 1) - t.seg0;
-  t.r = __ldg(p.pool.rank + t.a);
+__device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView& V, int task, ETask& t) {
+  const int s = find_seg(V.prefix, V.S, task);
+  int q = task - V.prefix[s];
+  t.a = V.adapter[s];
+  t.seg0 = V.start[s];
+  t.n = V.start[s + 1] - t.seg0;
+  t.r = V.rank[s];
   t.nt = nte_class(t.n);
   const int n_tg = cdiv_i(t.n, t.nt);
+  int k = 0;
+  for (; k < p.n_slots - 1; ++k) {  // the projection owning local task q
+    const int cnt = n_tg * cdiv_i(p.slot[k].d_out, kLC);
+    if (q < cnt) break;
+    q -= cnt;
+  }
+  t.k = k;
   t.tg = q % n_tg;
   t.lc = q / n_tg;
   t.nks = cdiv_i(t.r, kExpandRows);
-  return true;
 }
 
-// Slot layout: B row i of this stage at i * 512 B; in the last stage of a
-// task, y row t at (16 + t) * 512 B.
+// Slot layout: B row i of this stage at i * 512 B; t values of token t for
+// this stage's rank rows at 8 KiB + t * 64 B; in a task's last stage, y row t
+// at 8 KiB + 256 B + t * 512 B.
+constexpr int kExpTOff = kExpandRows * 2 * kLC;
+constexpr int kExpYOff = kExpTOff + 4 * 64;
+
 __device__ __forceinline__ void issue_expand(const BgmvParams& p, const ETask& t, int ks,
                                              unsigned char* buf, uint64_t* bar) {
   const int lane = threadIdx.x & 31;
@@ -679,17 +650,22 @@ __device__ __forceinline__ void issue_expand(const BgmvParams& p, const ETask& t
   const int Lo = min(kLC, L.d_out - l0);
   const int r0 = ks * kExpandRows;
   const int nrows = min(kExpandRows, t.r - r0);
+  const int tcols = (nrows + 3) & ~3;  // t floats copied per token (16-byte multiple)
   const bool last = ks == t.nks - 1;
-  const int ntok = last ? min(t.nt, t.n - t.tg * t.nt) : 0;
-  if (lane == 0) mbar_expect_tx(bar, 2u * Lo * (nrows + ntok));
+  const int ntok = min(t.nt, t.n - t.tg * t.nt);
+  const int nyt = last ? ntok : 0;
+  if (lane == 0) mbar_expect_tx(bar, 2u * Lo * (nrows + nyt) + 4u * tcols * ntok);
   __syncwarp();
   const int i = lane & 15;
   if (i < nrows)
     bulk_paged_piece(p.pool, t.a, L.listB, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 4,
                      buf + i * 2 * kLC, bar);
   if (lane < ntok) {
-    const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
-    bulk_g2s(buf + (kExpandRows + lane) * 2 * kLC, L.y + (int64_t)token * L.ldy + l0, 2u * Lo, bar);
+    const int pos = t.seg0 + t.tg * t.nt + lane;
+    const int token = __ldg(p.sc.perm + pos);
+    const int64_t row = L.t_by_token ? (int64_t)token : (int64_t)pos;
+    bulk_g2s(buf + kExpTOff + lane * 64, L.tfin + row * L.ldt + r0, 4u * tcols, bar);
+    if (last) bulk_g2s(buf + kExpYOff + lane * 2 * kLC, L.y + (int64_t)token * L.ldy + l0, 2u * Lo, bar);
   }
 }
 
@@ -705,14 +681,7 @@ __device__ __forceinline__ void compute_expand(const BgmvParams& p, const ETask&
   const int ntok = min(t.nt, t.n - t.tg * t.nt);
   const int l = lane * 8;
   const bool act = l < Lo;
-  const float* trow[4];
-  int token[4];
-#pragma unroll
-  for (int tt = 0; tt < 4; ++tt) {
-    const int pos = t.seg0 + t.tg * t.nt + (tt < ntok ? tt : 0);
-    token[tt] = __ldg(p.sc.perm + pos);
-    trow[tt] = L.tfin + (L.t_by_token ? (int64_t)token[tt] : (int64_t)pos) * L.ldt + r0;
-  }
+  const float* tv = reinterpret_cast<const float*>(buf + kExpTOff);
   if (act) {
 #pragma unroll 4
     for (int kk = 0; kk < nrows; ++kk) {
@@ -721,9 +690,9 @@ __device__ __forceinline__ void compute_expand(const BgmvParams& p, const ETask&
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt) {
         if (tt >= ntok) break;
-        const float tv = __ldg(trow[tt] + kk);
+        const float tvv = tv[tt * 16 + kk];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tv, bf[e], acc[tt][e]);
+        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tvv, bf[e], acc[tt][e]);
       }
     }
   }
@@ -733,14 +702,15 @@ __device__ __forceinline__ void compute_expand(const BgmvParams& p, const ETask&
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt) {
       if (tt >= ntok) break;
+      const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
       float yf[8];
-      unpack8<DT>(lds128(buf + (kExpandRows + tt) * 2 * kLC + 2 * l), yf);
+      unpack8<DT>(lds128(buf + kExpYOff + tt * 2 * kLC + 2 * l), yf);
       uint4 o;
       o.x = pack2<DT>(fmaf(s_a, acc[tt][0], yf[0]), fmaf(s_a, acc[tt][1], yf[1]));
       o.y = pack2<DT>(fmaf(s_a, acc[tt][2], yf[2]), fmaf(s_a, acc[tt][3], yf[3]));
       o.z = pack2<DT>(fmaf(s_a, acc[tt][4], yf[4]), fmaf(s_a, acc[tt][5], yf[5]));
       o.w = pack2<DT>(fmaf(s_a, acc[tt][6], yf[6]), fmaf(s_a, acc[tt][7], yf[7]));
-      *reinterpret_cast<uint4*>(L.y + (int64_t)token[tt] * L.ldy + l0 + l) = o;
+      *reinterpret_cast<uint4*>(L.y + (int64_t)token * L.ldy + l0 + l) = o;
     }
   }
 #pragma unroll
@@ -755,19 +725,23 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_expand(const __grid_constant
   __shared__ __align__(8) uint64_t bars[kWarps][kSlots];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* wbuf = smem + warp * kSlots * kSlotBytes;
+  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kSmemBytes);
   if (lane == 0)
     for (int s = 0; s < kSlots; ++s) mbar_init(&bars[warp][s], 1);
   fence_mbar_init();
-  __syncwarp();
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaExpandTotal];
+  const SegView V = stage_segments(p.sc, S, false, segsm);
   const int NW = gridDim.x * kWarps;
   int task = blockIdx.x * kWarps + warp;
   ETask cur, nxt;
-  bool have = task < total && decode_expand(p, S, task, cur);
+  bool have = task < total;
   int ks = 0;
-  if (have) issue_expand(p, cur, 0, wbuf, &bars[warp][0]);
+  if (have) {
+    decode_expand(p, V, task, cur);
+    issue_expand(p, cur, 0, wbuf, &bars[warp][0]);
+  }
   float acc[4][8];
 #pragma unroll
   for (int tt = 0; tt < 4; ++tt)
@@ -782,7 +756,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_expand(const __grid_constant
     if (nks >= cur.nks) {
       nks = 0;
       ntask = task + NW;
-      hn = ntask < total && decode_expand(p, S, ntask, nxt);
+      hn = ntask < total;
+      if (hn) decode_expand(p, V, ntask, nxt);
     } else {
       nxt = cur;
     }
@@ -930,6 +905,7 @@ __global__ void k_gather_debug(PoolDev P, int id, int d, int list_off, int rank,
 
 // ---------------------------------------------------------------------------
 // Launchers.
+constexpr int kDynSmem = kSmemBytes + 4 * kSegSmemInts;  // slots + segment table
 template <typename Kern>
 static cudaError_t launch_dependent(Kern kernel, int grid, int block, size_t smem, cudaStream_t s,
                                     const BgmvParams& p) {
@@ -950,10 +926,10 @@ static bool g_attrs_done = false;
 static void set_attrs() {
   if (g_attrs_done) return;
   cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-  cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  cudaFuncSetAttribute(k_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  cudaFuncSetAttribute(k_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  cudaFuncSetAttribute(k_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  cudaFuncSetAttribute(k_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
   g_attrs_done = true;
 }
 
@@ -966,14 +942,14 @@ cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cuda
 
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
   set_attrs();
-  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kWarps * 32, kSmemBytes, s, p);
-  return launch_dependent(k_shrink<SLORA_F16>, grid, kWarps * 32, kSmemBytes, s, p);
+  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kWarps * 32, kDynSmem, s, p);
+  return launch_dependent(k_shrink<SLORA_F16>, grid, kWarps * 32, kDynSmem, s, p);
 }
 
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
   set_attrs();
-  if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kWarps * 32, kSmemBytes, s, p);
-  return launch_dependent(k_expand<SLORA_F16>, grid, kWarps * 32, kSmemBytes, s, p);
+  if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kWarps * 32, kDynSmem, s, p);
+  return launch_dependent(k_expand<SLORA_F16>, grid, kWarps * 32, kDynSmem, s, p);
 }
 
 cudaError_t launch_merge_requests(const int32_t* req_start, const int32_t* req_adapter, int n,
@@ -1011,8 +987,8 @@ cudaError_t launch_gather_debug(const PoolDev& pool, int id, int d, int list_off
 int occupancy_blocks(int which) {
   set_attrs();
   int n = 0;
-  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kWarps * 32, kSmemBytes);
-  else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kWarps * 32, kSmemBytes);
+  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kWarps * 32, kDynSmem);
+  else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kWarps * 32, kDynSmem);
   return n > 0 ? n : 1;
 }
 

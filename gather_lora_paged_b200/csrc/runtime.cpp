@@ -308,6 +308,7 @@ ScratchDev scratch_dev(slora_pool* P) {
   s.shrink_prefix = reinterpret_cast<int32_t*>(b + L.off_shrink_pre);
   s.expand_prefix = reinterpret_cast<int32_t*>(b + L.off_expand_pre);
   s.ctr_prefix = reinterpret_cast<int32_t*>(b + L.off_ctr_pre);
+  s.seg_rank = s.ctr_prefix + (L.MS + 1);
   s.ctr = reinterpret_cast<int32_t*>(b + L.off_ctr);
   s.ctr_cap = L.ctr_cap;
   s.MS = L.MS;
@@ -430,6 +431,7 @@ slora_status_t lora_delta_on_scratch(slora_pool* P, int32_t n, const int32_t* pr
   bp.sc.shrink_prefix = reinterpret_cast<int32_t*>(b + L.off_shrink_pre);
   bp.sc.expand_prefix = reinterpret_cast<int32_t*>(b + L.off_expand_pre);
   bp.sc.ctr_prefix = reinterpret_cast<int32_t*>(b + L.off_ctr_pre);
+  bp.sc.seg_rank = bp.sc.ctr_prefix + (L.MS + 1);
   bp.sc.ctr = reinterpret_cast<int32_t*>(b + L.off_ctr);
   bp.sc.ctr_cap = L.ctr_cap;
   bp.sc.MS = L.MS;

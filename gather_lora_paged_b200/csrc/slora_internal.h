@@ -61,9 +61,10 @@ struct ScratchDev {
   int32_t* seg_start;      // [MS + 1]
   int32_t* seg_adapter;    // [MS]
   int32_t* meta;           // [16]: S, n_valid, shrink total, expand total, ctr total, work counters
-  int32_t* shrink_prefix;  // [kMaxSlots][MS + 1]
-  int32_t* expand_prefix;  // [kMaxSlots][MS + 1]
-  int32_t* ctr_prefix;     // [kMaxSlots][MS + 1]
+  int32_t* shrink_prefix;  // [MS + 1] shrink tasks before each segment (segment-major)
+  int32_t* expand_prefix;  // [MS + 1] expand tasks before each segment
+  int32_t* ctr_prefix;     // [MS + 1] reduction counters before each segment
+  int32_t* seg_rank;       // [MS] rank of each segment's adapter
   int32_t* ctr;            // reduction counters
   int64_t ctr_cap;
   int MS;                  // max segments = min(max_tokens, max_adapters)
