@@ -24,6 +24,8 @@
 // tile once and applies it to every token of its segment that the task covers,
 // so each touched adapter is streamed from HBM about once per step.  The three
 // kernels are chained with programmatic dependent launch.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -37,15 +39,15 @@ constexpr int kWarps = 8;                 // warps per CTA of shrink / expand
 constexpr int kSlots = 2;                 // pipeline slots per warp
 constexpr int kSlotBytes = 12 * 1024;     // bytes per slot
 constexpr int kSmemBytes = kWarps * kSlots * kSlotBytes;
-constexpr int kExpandRows = 16;           // B rows per expand stage
+constexpr int kExpandRows = 8;            // B rows per expand stage
 constexpr int kLC = 256;                  // outputs per expand task (8 per lane)
 constexpr long long kWaitLimit = 2000000000ll;  // clock cycles before a wait gives up
 
 __host__ __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
 
-// Task shapes.  Shrink tasks cover NT tokens x RW rank rows x kShrinkKC of d_in;
-// expand tasks NTE tokens x kLC outputs.  Slot use: (RW + NT) KiB for shrink,
-// 16 x 512 B + NTE x 512 B for expand; both fit kSlotBytes.
+// Task shapes.  Shrink tasks cover NT tokens x RW rank rows x kShrinkKT of
+// d_in; expand tasks NTE tokens x kLC outputs.  Slot use per stage: (RW + NT)
+// KiB for shrink; 8 B rows, the t partials and y rows for expand.
 __host__ __device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
 __host__ __device__ __forceinline__ int rw_of(int nt) { return nt == 1 ? 8 : 4; }
 __host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
@@ -142,21 +144,6 @@ __device__ __forceinline__ const uint16_t* page_addr(const PoolDev& P, int a, in
   return P.pool + ((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1));
 }
 
-// Copies flat elements [f0, f0 + n) of a paged tensor into dst.  The range
-// crosses at most one page boundary (n <= page size); piece 0 is the part in
-// the first page, piece 1 the rest.  Returns nothing for an empty piece.
-__device__ __forceinline__ void bulk_paged_piece(const PoolDev& P, int a, int lo, int64_t f0, int n,
-                                                 int piece, unsigned char* dst, uint64_t* bar) {
-  const int64_t pb = ((f0 >> P.page_shift) + 1) << P.page_shift;
-  const int64_t f1 = f0 + n;
-  if (piece == 0) {
-    const int64_t e = f1 < pb ? f1 : pb;
-    bulk_g2s(dst, page_addr(P, a, lo, f0), (uint32_t)(2 * (e - f0)), bar);
-  } else if (f1 > pb) {
-    bulk_g2s(dst + 2 * (pb - f0), page_addr(P, a, lo, pb), (uint32_t)(2 * (f1 - pb)), bar);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Block-wide exclusive scans (blockDim.x threads, a multiple of 32).
 template <bool kMax>
@@ -192,20 +179,14 @@ __device__ int block_exscan(int v, int* total, int* sh) {
 
 // k_segments: one CTA of 1024 threads.  Dynamic smem: max_adapters ints.
 // Output: perm, segments (start, adapter, rank) and, per segment, the number
-// of shrink tasks, reduction counters and expand tasks before it (prefix sums
-// in segment-major task order).
-
-__device__ __forceinline__ void seg_task_counts(const BgmvParams& p, int n, int r, int& shr, int& ctr,
-                                                int& exp) {
-  shr = ctr = exp = 0;
+// of shrink and expand tasks before it (prefix sums in segment-major order).
+__device__ __forceinline__ void seg_task_counts(const BgmvParams& p, int n, int r, int& shr, int& exp) {
+  shr = exp = 0;
   if (n == 0 || r <= 0) return;
   const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
   if (p.do_shrink)
-    for (int g = 0; g < p.n_groups; ++g) {
-      const int nrg = cdiv_i(p.group[g].n * r, rw_of(nt));
-      shr += nrg * ntg * cdiv_i(p.group[g].d_in, kShrinkKC);
-      ctr += nrg * ntg;
-    }
+    for (int g = 0; g < p.n_groups; ++g)
+      shr += cdiv_i(p.group[g].n * r, rw_of(nt)) * ntg * cdiv_i(p.group[g].d_in, kShrinkKT);
   if (p.do_expand)
     for (int k = 0; k < p.n_slots; ++k) exp += nte * cdiv_i(p.slot[k].d_out, kLC);
 }
@@ -240,60 +221,48 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
   // a contiguous range of segment indices.
   const int E = (MA + nth - 1) / nth;
   const int a0 = min(tid * E, MA), a1 = min(a0 + E, MA);
-  int cnt = 0, nseg = 0, c_shr = 0, c_ctr = 0, c_exp = 0;
+  int cnt = 0, nseg = 0, c_shr = 0, c_exp = 0;
   for (int a = a0; a < a1; ++a) {
     const int n = hist[a];
     if (n == 0) continue;
-    int x, y, z;
-    seg_task_counts(p, n, p.pool.rank[a], x, y, z);
+    int x, z;
+    seg_task_counts(p, n, p.pool.rank[a], x, z);
     cnt += n;
     nseg += 1;
     c_shr += x;
-    c_ctr += y;
     c_exp += z;
   }
-  int n_valid, S, t_shr, t_ctr, t_exp;
+  int n_valid, S, t_shr, t_exp;
   int cbase = block_exscan<false>(cnt, &n_valid, sh);
   int sb = block_exscan<false>(nseg, &S, sh);
   int b_shr = block_exscan<false>(c_shr, &t_shr, sh);
-  int b_ctr = block_exscan<false>(c_ctr, &t_ctr, sh);
   int b_exp = block_exscan<false>(c_exp, &t_exp, sh);
   for (int a = a0; a < a1; ++a) {
     const int n = hist[a];
     hist[a] = cbase;  // becomes the scatter cursor
     if (n == 0) continue;
     const int r = p.pool.rank[a];
-    int x, y, z;
-    seg_task_counts(p, n, r, x, y, z);
+    int x, z;
+    seg_task_counts(p, n, r, x, z);
     sc.seg_start[sb] = cbase;
     sc.seg_adapter[sb] = a;
     sc.seg_rank[sb] = r;
     sc.shrink_prefix[sb] = b_shr;
-    sc.ctr_prefix[sb] = b_ctr;
     sc.expand_prefix[sb] = b_exp;
     ++sb;
     cbase += n;
     b_shr += x;
-    b_ctr += y;
     b_exp += z;
-  }
-  int ctr_total = t_ctr;
-  if (ctr_total > sc.ctr_cap) {  // cannot happen with the sizing in slora_scratch_bytes
-    if (tid == 0) record_error(p.pool.err, 3, ctr_total);
-    ctr_total = t_shr = t_exp = 0;
   }
   if (tid == 0) {
     sc.seg_start[S] = n_valid;
     sc.shrink_prefix[S] = t_shr;
-    sc.ctr_prefix[S] = t_ctr;
     sc.expand_prefix[S] = t_exp;
     sc.meta[kMetaS] = S;
     sc.meta[kMetaValid] = n_valid;
     sc.meta[kMetaShrinkTotal] = t_shr;
     sc.meta[kMetaExpandTotal] = t_exp;
-    sc.meta[kMetaCtrTotal] = ctr_total;
   }
-  for (int c = tid; c < ctr_total; c += nth) sc.ctr[c] = 0;
   __syncthreads();
 
   // Stable scatter: chunks of 1024 tokens, warps take turns in order.
@@ -359,12 +328,12 @@ __device__ __forceinline__ float lane_transpose_reduce(float (&v)[N]) {
 // Segment table as seen by the persistent kernels: staged in shared memory
 // when it fits (one round trip per CTA), else read from global memory.
 constexpr int kSegCap = 1024;
+constexpr int kSegSmemInts = 4 * kSegCap + 2;
 struct SegView {
   const int32_t* start;   // [S + 1]
   const int32_t* adapter; // [S]
   const int32_t* rank;    // [S]
   const int32_t* prefix;  // [S + 1] tasks before each segment
-  const int32_t* ctr;     // [S + 1] counters before each segment (shrink only)
   int S;
 };
 
@@ -377,18 +346,15 @@ __device__ SegView stage_segments(const ScratchDev& sc, int S, bool shrink, int3
     v.adapter = sc.seg_adapter;
     v.rank = sc.seg_rank;
     v.prefix = pre;
-    v.ctr = sc.ctr_prefix;
     return v;
   }
   int32_t* st = sm;
   int32_t* ad = sm + (kSegCap + 1);
   int32_t* rk = ad + kSegCap;
   int32_t* pf = rk + kSegCap;
-  int32_t* ct = pf + (kSegCap + 1);
   for (int i = threadIdx.x; i <= S; i += blockDim.x) {
     st[i] = sc.seg_start[i];
     pf[i] = pre[i];
-    if (shrink) ct[i] = sc.ctr_prefix[i];
     if (i < S) {
       ad[i] = sc.seg_adapter[i];
       rk[i] = sc.seg_rank[i];
@@ -399,15 +365,43 @@ __device__ SegView stage_segments(const ScratchDev& sc, int S, bool shrink, int3
   v.adapter = ad;
   v.rank = rk;
   v.prefix = pf;
-  v.ctr = ct;
   return v;
 }
-constexpr int kSegSmemInts = 5 * kSegCap + 3;
+
+// Page id of flat element f of tensor (adapter a, page-list offset lo).
+__device__ __forceinline__ int32_t page_id(const PoolDev& P, int a, int lo, int64_t f) {
+  return __ldg(P.page_list + (int64_t)a * P.list_stride + lo + (f >> P.page_shift));
+}
+__device__ __forceinline__ const uint16_t* page_ptr(const PoolDev& P, int32_t pg, int64_t f) {
+  return P.pool + ((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1));
+}
+
+// A paged range [f0, f0 + n) (n <= page size) is copied as piece 0 (the part
+// in f0's page) and piece 1 (the rest, if the range crosses a page boundary).
+// aux_page: the page id of the lane's piece, looked up one stage ahead.
+__device__ __forceinline__ int32_t piece_page(const PoolDev& P, int a, int lo, int64_t f0, int n, int piece) {
+  const int64_t pb = ((f0 >> P.page_shift) + 1) << P.page_shift;
+  if (piece == 0) return page_id(P, a, lo, f0);
+  return (f0 + n > pb) ? page_id(P, a, lo, pb) : -1;
+}
+__device__ __forceinline__ void piece_copy(const PoolDev& P, int32_t pg, int64_t f0, int n, int piece,
+                                           unsigned char* dst, uint64_t* bar) {
+  const int64_t pb = ((f0 >> P.page_shift) + 1) << P.page_shift;
+  const int64_t f1 = f0 + n;
+  if (piece == 0) {
+    const int64_t e = f1 < pb ? f1 : pb;
+    bulk_g2s(dst, page_ptr(P, pg, f0), (uint32_t)(2 * (e - f0)), bar);
+  } else if (f1 > pb) {
+    bulk_g2s(dst + 2 * (pb - f0), page_ptr(P, pg, pb), (uint32_t)(2 * (f1 - pb)), bar);
+  }
+}
 
 // ---------------------------------------------------------------------------
-// Shrink.
+// Shrink.  Task = (group g, segment, RW rank rows, NT tokens, kShrinkKT slice
+// of d_in), streamed in stages of kStageK elements.  Slot layout of a stage:
+// rank row i at i * 1 KiB, token row t at (RW + t) * 1 KiB.
 struct STask {
-  int g, a, r, seg0, n, nt, rw, rg, tg, kc, n_kc, ci;
+  int g, a, r, seg0, n, nt, rw, rg, tg, split, nst, nrows, ntok;
 };
 
 __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView& V, int task, STask& t) {
@@ -420,73 +414,75 @@ __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView
   t.nt = nt_class(t.n);
   t.rw = rw_of(t.nt);
   const int n_tg = cdiv_i(t.n, t.nt);
-  int ci = V.ctr[s];
   int g = 0;
   for (; g < p.n_groups - 1; ++g) {  // the group owning local task q
-    const int nrg = cdiv_i(p.group[g].n * t.r, t.rw);
-    const int cnt = nrg * n_tg * cdiv_i(p.group[g].d_in, kShrinkKC);
+    const int cnt = cdiv_i(p.group[g].n * t.r, t.rw) * n_tg * cdiv_i(p.group[g].d_in, kShrinkKT);
     if (q < cnt) break;
     q -= cnt;
-    ci += nrg * n_tg;
   }
   t.g = g;
-  t.n_kc = cdiv_i(p.group[g].d_in, kShrinkKC);
+  const int d_in = p.group[g].d_in;
+  const int n_split = cdiv_i(d_in, kShrinkKT);
   t.tg = q % n_tg;
   q /= n_tg;
-  t.kc = q % t.n_kc;
-  t.rg = q / t.n_kc;
-  t.ci = ci + t.rg * n_tg + t.tg;
+  t.split = q % n_split;
+  t.rg = q / n_split;
+  t.nst = cdiv_i(min(kShrinkKT, d_in - t.split * kShrinkKT), kStageK);
+  t.nrows = min(t.rw, p.group[g].n * t.r - t.rg * t.rw);
+  t.ntok = min(t.nt, t.n - t.tg * t.nt);
 }
 
-// Slot layout: rank row i at i * 1 KiB, token row t at (rw + t) * 1 KiB.
-__device__ __forceinline__ void issue_shrink(const BgmvParams& p, const STask& t, unsigned char* buf,
-                                             uint64_t* bar) {
-  const int lane = threadIdx.x & 31;
+// Lane roles in a shrink stage: lane i < 16 copies piece 0 of rank row i
+// (i < nrows) or token row i - nrows; lane 16 + i copies piece 1 of row i.
+// The per-lane lookup (page id or token id) is done one stage ahead.
+__device__ __forceinline__ int32_t shrink_lookup(const BgmvParams& p, const STask& t, int st) {
+  const int lane = threadIdx.x & 31, i = lane & 15;
   const GroupDev& G = p.group[t.g];
-  const int k0 = t.kc * kShrinkKC;
-  const int L = min(kShrinkKC, G.d_in - k0);
-  const int R = G.n * t.r;
-  const int nrows = min(t.rw, R - t.rg * t.rw);
-  const int ntok = min(t.nt, t.n - t.tg * t.nt);
-  if (lane == 0) mbar_expect_tx(bar, 2u * L * (nrows + ntok));
-  __syncwarp();
-  const int i = lane & 15;
-  if (i < nrows) {
+  const int k0 = t.split * kShrinkKT + st * kStageK;
+  const int L = min(kStageK, G.d_in - k0);
+  if (i < t.nrows) {
     const int rho = t.rg * t.rw + i;
     const int j = rho / t.r, k = rho % t.r;
-    const int lo = p.slot[G.slot[j]].listA;
-    bulk_paged_piece(p.pool, t.a, lo, (int64_t)k * G.d_in + k0, L, lane >> 4, buf + i * 2 * kShrinkKC, bar);
-  } else if (lane < 16 && i < nrows + ntok) {
-    const int tt = i - nrows;
-    const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
-    bulk_g2s(buf + (t.rw + tt) * 2 * kShrinkKC, G.x + (int64_t)token * G.ldx + k0, 2u * L, bar);
+    return piece_page(p.pool, t.a, p.slot[G.slot[j]].listA, (int64_t)k * G.d_in + k0, L, lane >> 4);
+  }
+  if (lane < 16 && i < t.nrows + t.ntok) return __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + (i - t.nrows));
+  return -1;
+}
+
+__device__ __forceinline__ void issue_shrink(const BgmvParams& p, const STask& t, int st, int32_t aux,
+                                             unsigned char* buf, uint64_t* bar) {
+  const int lane = threadIdx.x & 31, i = lane & 15;
+  const GroupDev& G = p.group[t.g];
+  const int k0 = t.split * kShrinkKT + st * kStageK;
+  const int L = min(kStageK, G.d_in - k0);
+  if (lane == 0) mbar_expect_tx(bar, 2u * L * (t.nrows + t.ntok));
+  __syncwarp();
+  if (i < t.nrows) {
+    const int rho = t.rg * t.rw + i;
+    const int k = rho % t.r;
+    piece_copy(p.pool, aux, (int64_t)k * G.d_in + k0, L, lane >> 4, buf + i * 2 * kStageK, bar);
+  } else if (lane < 16 && i < t.nrows + t.ntok) {
+    bulk_g2s(buf + (t.rw + i - t.nrows) * 2 * kStageK, G.x + (int64_t)aux * G.ldx + k0, 2u * L, bar);
   }
 }
 
 template <int DT, int NT, int RW>
-__device__ __forceinline__ void compute_shrink(const BgmvParams& p, const STask& t,
-                                               const unsigned char* buf) {
+__device__ __forceinline__ void shrink_stage(const BgmvParams& p, const STask& t, int st,
+                                             const unsigned char* buf, float (&acc)[32]) {
   const int lane = threadIdx.x & 31;
   const GroupDev& G = p.group[t.g];
-  const PoolDev& P = p.pool;
-  const int k0 = t.kc * kShrinkKC;
-  const int L = min(kShrinkKC, G.d_in - k0);
-  const int R = G.n * t.r;
-  const int nrows = min(RW, R - t.rg * RW);
-  const int ntok = min(NT, t.n - t.tg * NT);
-
-  float acc[RW * NT];
+  const int k0 = t.split * kShrinkKT + st * kStageK;
+  const int L = min(kStageK, G.d_in - k0);
 #pragma unroll
-  for (int i = 0; i < RW * NT; ++i) acc[i] = 0.f;
-#pragma unroll
-  for (int e = lane * 8; e < kShrinkKC; e += 256) {
+  for (int e = lane * 8; e < kStageK; e += 256) {
     if (e >= L) break;
     uint4 av[RW], xv[NT];
 #pragma unroll
-    for (int i = 0; i < RW; ++i) av[i] = i < nrows ? lds128(buf + i * 2 * kShrinkKC + 2 * e) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < RW; ++i)
+      av[i] = i < t.nrows ? lds128(buf + i * 2 * kStageK + 2 * e) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int tt = 0; tt < NT; ++tt)
-      xv[tt] = tt < ntok ? lds128(buf + (RW + tt) * 2 * kShrinkKC + 2 * e) : make_uint4(0, 0, 0, 0);
+      xv[tt] = tt < t.ntok ? lds128(buf + (RW + tt) * 2 * kStageK + 2 * e) : make_uint4(0, 0, 0, 0);
     if (NT <= 2) {
       float xf[NT][8];
 #pragma unroll
@@ -521,47 +517,40 @@ __device__ __forceinline__ void compute_shrink(const BgmvParams& p, const STask&
       }
     }
   }
+}
 
-  const float val = lane_transpose_reduce<RW * NT>(acc);
-  const int Lx = lane % (RW * NT);
+// End of a shrink task: sum over lanes and store the fp32 partial of this
+// d_in slice, t[pos][k][split], for RW rows x NT tokens.
+template <int NT, int RW>
+__device__ __forceinline__ void shrink_finish(const BgmvParams& p, const STask& t, float (&acc)[32]) {
+  constexpr int N = RW * NT;
+  float v[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) v[i] = acc[i];
+  const float val = lane_transpose_reduce<N>(v);
+  const int lane = threadIdx.x & 31;
+  const int Lx = lane % N;
   const int i = Lx / NT, tt = Lx % NT;
-  const int rho = t.rg * RW + i;
-  const bool mine = lane < RW * NT && i < nrows && tt < ntok;
-  const int j = mine ? rho / t.r : 0, k = mine ? rho % t.r : 0;
-  const SlotDev& S = p.slot[G.slot[j]];
-  const int pos = t.seg0 + t.tg * NT + tt;
-  if (t.n_kc == 1) {
-    if (mine) {
-      const int64_t row = S.t_by_token ? (int64_t)__ldg(p.sc.perm + pos) : (int64_t)pos;
-      S.tfin[row * S.ldt + k] = val;
-    }
-    return;
+  if (lane < N && i < t.nrows && tt < t.ntok) {
+    const int rho = t.rg * RW + i;
+    const int j = rho / t.r, k = rho % t.r;
+    const SlotDev& S = p.slot[p.group[t.g].slot[j]];
+    const int pos = t.seg0 + t.tg * NT + tt;
+    S.t[(int64_t)pos * S.t_rs + (int64_t)k * S.t_ns + t.split] = val;
   }
-  if (mine) S.tpart[((int64_t)t.kc * p.max_tokens + pos) * P.max_rank + k] = val;
-  __threadfence();
-  __syncwarp();
-  int old = 0;
-  if (lane == 0) old = atomicAdd(p.sc.ctr + t.ci, 1);
-  old = __shfl_sync(FULL_MASK, old, 0);
-  if (old != t.n_kc - 1) return;
-  __threadfence();
-  if (mine) {  // last of the n_kc chunk tasks: sum the partials in chunk order
-    float s = 0.f;
-    for (int c = 0; c < t.n_kc; ++c)
-      s += __ldcg(S.tpart + ((int64_t)c * p.max_tokens + pos) * P.max_rank + k);
-    const int64_t row = S.t_by_token ? (int64_t)__ldg(p.sc.perm + pos) : (int64_t)pos;
-    S.tfin[row * S.ldt + k] = s;
-  }
+#pragma unroll
+  for (int q = 0; q < 32; ++q) acc[q] = 0.f;
 }
 
 template <int DT>
-__device__ __forceinline__ void compute_shrink_any(const BgmvParams& p, const STask& t,
-                                                   const unsigned char* buf) {
+__device__ __forceinline__ void shrink_stage_any(const BgmvParams& p, const STask& t, int st,
+                                                 const unsigned char* buf, float (&acc)[32]) {
+  const bool last = st == t.nst - 1;
   switch (t.nt) {
-    case 1: compute_shrink<DT, 1, 8>(p, t, buf); break;
-    case 2: compute_shrink<DT, 2, 4>(p, t, buf); break;
-    case 4: compute_shrink<DT, 4, 4>(p, t, buf); break;
-    default: compute_shrink<DT, 8, 4>(p, t, buf); break;
+    case 1: shrink_stage<DT, 1, 8>(p, t, st, buf, acc); if (last) shrink_finish<1, 8>(p, t, acc); break;
+    case 2: shrink_stage<DT, 2, 4>(p, t, st, buf, acc); if (last) shrink_finish<2, 4>(p, t, acc); break;
+    case 4: shrink_stage<DT, 4, 4>(p, t, st, buf, acc); if (last) shrink_finish<4, 4>(p, t, acc); break;
+    default: shrink_stage<DT, 8, 4>(p, t, st, buf, acc); if (last) shrink_finish<8, 4>(p, t, acc); break;
   }
 }
 
@@ -580,39 +569,66 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_shrink(const __grid_constant
   const int total = p.sc.meta[kMetaShrinkTotal];
   const SegView V = stage_segments(p.sc, S, true, segsm);
   const int NW = gridDim.x * kWarps;
-  int task = blockIdx.x * kWarps + warp;
-  STask cur, nxt;
-  bool have = task < total;
-  if (have) {
-    decode_shrink(p, V, task, cur);
-    issue_shrink(p, cur, wbuf, &bars[warp][0]);
+  const int first = blockIdx.x * kWarps + warp;
+  if (first >= total) {
+    griddep_launch();
+    return;
   }
-  int slot = 0;
-  uint32_t parity = 0;
-  while (have) {
-    const int ntask = task + NW;
-    const bool hn = ntask < total;
-    if (hn) {
-      decode_shrink(p, V, ntask, nxt);
-      issue_shrink(p, nxt, wbuf + (slot ^ 1) * kSlotBytes, &bars[warp][slot ^ 1]);
+  // Producer and consumer walk the same (task, stage) sequence; the producer
+  // issues one stage ahead and looks up its page / token ids one more ahead.
+  int ptask = first, pst = 0, pslot = 0;
+  STask pt;
+  decode_shrink(p, V, ptask, pt);
+  bool pvalid = true;
+  int32_t aux = shrink_lookup(p, pt, 0);
+  auto produce = [&]() {
+    issue_shrink(p, pt, pst, aux, wbuf + pslot * kSlotBytes, &bars[warp][pslot]);
+    pslot ^= 1;
+    if (++pst == pt.nst) {
+      pst = 0;
+      ptask += NW;
+      pvalid = ptask < total;
+      if (pvalid) decode_shrink(p, V, ptask, pt);
     }
+    if (pvalid) aux = shrink_lookup(p, pt, pst);
+  };
+  int ctask = first, cst = 0, slot = 0;
+  STask ct = pt;
+  uint32_t parity = 0;
+  float acc[32];
+#pragma unroll
+  for (int q = 0; q < 32; ++q) acc[q] = 0.f;
+  produce();
+  for (;;) {
+    if (pvalid) produce();
     if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
     parity ^= 1u << slot;
-    compute_shrink_any<DT>(p, cur, wbuf + slot * kSlotBytes);
+    shrink_stage_any<DT>(p, ct, cst, wbuf + slot * kSlotBytes, acc);
     __syncwarp();
     fence_proxy_async();
     slot ^= 1;
-    task = ntask;
-    cur = nxt;
-    have = hn;
+    if (++cst == ct.nst) {
+      cst = 0;
+      ctask += NW;
+      if (ctask >= total) break;
+      decode_shrink(p, V, ctask, ct);
+    }
   }
   griddep_launch();
 }
 
 // ---------------------------------------------------------------------------
-// Expand.
+// Expand.  Task = (projection slot k, segment, NTE tokens, kLC outputs),
+// streamed in stages of kExpandRows rank rows.  Slot layout of a stage:
+// B row i at i * 512 B; t partials of token t at kExpT + t * 8 * t_ns * 4 B;
+// y row t (last stage) at kExpY + t * 512 B; t sums at kExpS.
+constexpr int kExpT = kExpandRows * 2 * kLC;
+constexpr int kExpY = 8 * 1024;
+constexpr int kExpS = kExpY + 4 * 2 * kLC;
+static_assert(kExpS + 4 * kExpandRows * 4 <= kSlotBytes, "expand slot overflow");
+
 struct ETask {
-  int k, a, r, seg0, n, nt, tg, lc, nks;
+  int k, a, r, seg0, n, nt, tg, lc, nst, ntok;
 };
 
 __device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView& V, int task, ETask& t) {
@@ -633,78 +649,104 @@ __device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView
   t.k = k;
   t.tg = q % n_tg;
   t.lc = q / n_tg;
-  t.nks = cdiv_i(t.r, kExpandRows);
+  t.nst = cdiv_i(t.r, kExpandRows);
+  t.ntok = min(t.nt, t.n - t.tg * t.nt);
 }
 
-// Slot layout: B row i of this stage at i * 512 B; t values of token t for
-// this stage's rank rows at 8 KiB + t * 64 B; in a task's last stage, y row t
-// at 8 KiB + 256 B + t * 512 B.
-constexpr int kExpTOff = kExpandRows * 2 * kLC;
-constexpr int kExpYOff = kExpTOff + 4 * 64;
+// Lane roles in an expand stage: lanes 0-7 copy piece 0 of B rows 0-7,
+// lanes 8-15 piece 1; lanes 16-19 the t partials of tokens 0-3; lanes 20-23
+// the y rows (last stage).  The lookup (page id / token id) is done a stage ahead.
+__device__ __forceinline__ int32_t expand_lookup(const BgmvParams& p, const ETask& t, int st) {
+  const int lane = threadIdx.x & 31;
+  const SlotDev& L = p.slot[t.k];
+  const int l0 = t.lc * kLC;
+  const int Lo = min(kLC, L.d_out - l0);
+  const int r0 = st * kExpandRows;
+  const int nrows = min(kExpandRows, t.r - r0);
+  if (lane < 16) {
+    const int i = lane & 7;
+    if (i >= nrows) return -1;
+    return piece_page(p.pool, t.a, L.listB, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 3);
+  }
+  const int tt = (lane - 16) & 3;
+  if (lane < 24 && tt < t.ntok) return __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
+  return -1;
+}
 
-__device__ __forceinline__ void issue_expand(const BgmvParams& p, const ETask& t, int ks,
+__device__ __forceinline__ void issue_expand(const BgmvParams& p, const ETask& t, int st, int32_t aux,
                                              unsigned char* buf, uint64_t* bar) {
   const int lane = threadIdx.x & 31;
   const SlotDev& L = p.slot[t.k];
   const int l0 = t.lc * kLC;
   const int Lo = min(kLC, L.d_out - l0);
-  const int r0 = ks * kExpandRows;
+  const int r0 = st * kExpandRows;
   const int nrows = min(kExpandRows, t.r - r0);
-  const int tcols = (nrows + 3) & ~3;  // t floats copied per token (16-byte multiple)
-  const bool last = ks == t.nks - 1;
-  const int ntok = min(t.nt, t.n - t.tg * t.nt);
-  const int nyt = last ? ntok : 0;
-  if (lane == 0) mbar_expect_tx(bar, 2u * Lo * (nrows + nyt) + 4u * tcols * ntok);
+  const bool last = st == t.nst - 1;
+  const uint32_t tbytes = 4u * kExpandRows * L.t_ns;
+  if (lane == 0) mbar_expect_tx(bar, 2u * Lo * (nrows + (last ? t.ntok : 0)) + tbytes * t.ntok);
   __syncwarp();
-  const int i = lane & 15;
-  if (i < nrows)
-    bulk_paged_piece(p.pool, t.a, L.listB, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 4,
-                     buf + i * 2 * kLC, bar);
-  if (lane < ntok) {
-    const int pos = t.seg0 + t.tg * t.nt + lane;
-    const int token = __ldg(p.sc.perm + pos);
-    const int64_t row = L.t_by_token ? (int64_t)token : (int64_t)pos;
-    bulk_g2s(buf + kExpTOff + lane * 64, L.tfin + row * L.ldt + r0, 4u * tcols, bar);
-    if (last) bulk_g2s(buf + kExpYOff + lane * 2 * kLC, L.y + (int64_t)token * L.ldy + l0, 2u * Lo, bar);
+  if (lane < 16) {
+    const int i = lane & 7;
+    if (i < nrows)
+      piece_copy(p.pool, aux, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 3, buf + i * 2 * kLC, bar);
+  } else if (lane < 20) {
+    const int tt = lane - 16;
+    if (tt < t.ntok) {
+      const int64_t row = L.t_by_token ? (int64_t)aux : (int64_t)(t.seg0 + t.tg * t.nt + tt);
+      bulk_g2s(buf + kExpT + tt * tbytes, L.t + row * L.t_rs + (int64_t)r0 * L.t_ns, tbytes, bar);
+    }
+  } else if (lane < 24 && last) {
+    const int tt = lane - 20;
+    if (tt < t.ntok) bulk_g2s(buf + kExpY + tt * 2 * kLC, L.y + (int64_t)aux * L.ldy + l0, 2u * Lo, bar);
   }
 }
 
 template <int DT>
-__device__ __forceinline__ void compute_expand(const BgmvParams& p, const ETask& t, int ks,
-                                               const unsigned char* buf, float (&acc)[4][8]) {
+__device__ __forceinline__ void expand_stage(const BgmvParams& p, const ETask& t, int st, unsigned char* buf,
+                                             float (&acc)[4][8], int32_t ctok) {
   const int lane = threadIdx.x & 31;
   const SlotDev& L = p.slot[t.k];
   const int l0 = t.lc * kLC;
   const int Lo = min(kLC, L.d_out - l0);
-  const int r0 = ks * kExpandRows;
+  const int r0 = st * kExpandRows;
   const int nrows = min(kExpandRows, t.r - r0);
-  const int ntok = min(t.nt, t.n - t.tg * t.nt);
+  // t for this stage: lane (tt, kk) sums the t_ns partials, in order
+  float* tsum = reinterpret_cast<float*>(buf + kExpS);
+  {
+    const int tt = lane >> 3, kk = lane & 7;
+    if (tt < t.ntok && kk < nrows) {
+      const float* src = reinterpret_cast<const float*>(buf + kExpT + tt * 4 * kExpandRows * L.t_ns) + kk * L.t_ns;
+      float s = 0.f;
+      for (int c = 0; c < L.t_ns; ++c) s += src[c];
+      tsum[tt * kExpandRows + kk] = s;
+    }
+  }
+  __syncwarp();
   const int l = lane * 8;
   const bool act = l < Lo;
-  const float* tv = reinterpret_cast<const float*>(buf + kExpTOff);
   if (act) {
-#pragma unroll 4
-    for (int kk = 0; kk < nrows; ++kk) {
+#pragma unroll
+    for (int kk = 0; kk < kExpandRows; ++kk) {
+      if (kk >= nrows) break;
       float bf[8];
       unpack8<DT>(lds128(buf + kk * 2 * kLC + 2 * l), bf);
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt) {
-        if (tt >= ntok) break;
-        const float tvv = tv[tt * 16 + kk];
+        if (tt >= t.ntok) break;
+        const float tv = tsum[tt * kExpandRows + kk];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tvv, bf[e], acc[tt][e]);
+        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tv, bf[e], acc[tt][e]);
       }
     }
   }
-  if (ks != t.nks - 1) return;
+  if (st != t.nst - 1) return;
   const float s_a = __ldg(p.pool.scale + t.a);
-  if (act) {
 #pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-      if (tt >= ntok) break;
-      const int token = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
+  for (int tt = 0; tt < 4; ++tt) {
+    const int token = __shfl_sync(FULL_MASK, ctok, tt);
+    if (act && tt < t.ntok) {
       float yf[8];
-      unpack8<DT>(lds128(buf + kExpYOff + tt * 2 * kLC + 2 * l), yf);
+      unpack8<DT>(lds128(buf + kExpY + tt * 2 * kLC + 2 * l), yf);
       uint4 o;
       o.x = pack2<DT>(fmaf(s_a, acc[tt][0], yf[0]), fmaf(s_a, acc[tt][1], yf[1]));
       o.y = pack2<DT>(fmaf(s_a, acc[tt][2], yf[2]), fmaf(s_a, acc[tt][3], yf[3]));
@@ -712,11 +754,9 @@ __device__ __forceinline__ void compute_expand(const BgmvParams& p, const ETask&
       o.w = pack2<DT>(fmaf(s_a, acc[tt][6], yf[6]), fmaf(s_a, acc[tt][7], yf[7]));
       *reinterpret_cast<uint4*>(L.y + (int64_t)token * L.ldy + l0 + l) = o;
     }
-  }
-#pragma unroll
-  for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
+  }
 }
 
 template <int DT>
@@ -734,46 +774,76 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_expand(const __grid_constant
   const int total = p.sc.meta[kMetaExpandTotal];
   const SegView V = stage_segments(p.sc, S, false, segsm);
   const int NW = gridDim.x * kWarps;
-  int task = blockIdx.x * kWarps + warp;
-  ETask cur, nxt;
-  bool have = task < total;
-  int ks = 0;
-  if (have) {
-    decode_expand(p, V, task, cur);
-    issue_expand(p, cur, 0, wbuf, &bars[warp][0]);
+  const int first = blockIdx.x * kWarps + warp;
+  if (first >= total) {
+    griddep_launch();
+    return;
   }
+  int ptask = first, pst = 0, pslot = 0;
+  ETask pt;
+  decode_expand(p, V, ptask, pt);
+  bool pvalid = true;
+  int32_t aux = expand_lookup(p, pt, 0);
+  auto produce = [&]() {
+    issue_expand(p, pt, pst, aux, wbuf + pslot * kSlotBytes, &bars[warp][pslot]);
+    pslot ^= 1;
+    if (++pst == pt.nst) {
+      pst = 0;
+      ptask += NW;
+      pvalid = ptask < total;
+      if (pvalid) decode_expand(p, V, ptask, pt);
+    }
+    if (pvalid) aux = expand_lookup(p, pt, pst);
+  };
+  int ctask = first, cst = 0, slot = 0;
+  ETask ct = pt;
+  auto ctoken = [&]() {  // token ids of the consumer's task, lane tt holds token tt
+    return lane < ct.ntok ? __ldg(p.sc.perm + ct.seg0 + ct.tg * ct.nt + lane) : 0;
+  };
+  int32_t ctok = ctoken();
+  uint32_t parity = 0;
   float acc[4][8];
 #pragma unroll
   for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
-  int slot = 0;
-  uint32_t parity = 0;
-  while (have) {
-    // next stage: the next rank chunk of this task, or the first of the next task
-    int nks = ks + 1, ntask = task;
-    bool hn = true;
-    if (nks >= cur.nks) {
-      nks = 0;
-      ntask = task + NW;
-      hn = ntask < total;
-      if (hn) decode_expand(p, V, ntask, nxt);
-    } else {
-      nxt = cur;
-    }
-    if (hn) issue_expand(p, nxt, nks, wbuf + (slot ^ 1) * kSlotBytes, &bars[warp][slot ^ 1]);
+  produce();
+  for (;;) {
+    if (pvalid) produce();
     if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
     parity ^= 1u << slot;
-    compute_expand<DT>(p, cur, ks, wbuf + slot * kSlotBytes, acc);
+    expand_stage<DT>(p, ct, cst, wbuf + slot * kSlotBytes, acc, ctok);
     __syncwarp();
     fence_proxy_async();
     slot ^= 1;
-    task = ntask;
-    ks = nks;
-    cur = nxt;
-    have = hn;
+    if (++cst == ct.nst) {
+      cst = 0;
+      ctask += NW;
+      if (ctask >= total) break;
+      decode_expand(p, V, ctask, ct);
+      ctok = ctoken();
+    }
   }
   griddep_launch();
+}
+
+// ---------------------------------------------------------------------------
+// slora_bgmv_shrink's output: t_out[token][k] = sum over the d_in slices.
+__global__ void __launch_bounds__(256) k_reduce_t(const __grid_constant__ BgmvParams p) {
+  griddep_wait();
+  const SlotDev& L = p.slot[0];
+  const int S = p.sc.meta[kMetaS];
+  const int n_valid = p.sc.meta[kMetaValid];
+  const int RK = (int)(L.t_rs / L.t_ns);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < (int64_t)n_valid * RK;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int pos = (int)(e / RK), k = (int)(e % RK);
+    const int s = S > 0 ? find_seg(p.sc.seg_start, S, pos) : 0;
+    if (k >= p.sc.seg_rank[s]) continue;
+    float acc = 0.f;
+    for (int c = 0; c < L.t_ns; ++c) acc += L.t[(int64_t)pos * L.t_rs + (int64_t)k * L.t_ns + c];
+    L.tout[(int64_t)p.sc.perm[pos] * L.ldt_out + k] = acc;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -950,6 +1020,12 @@ cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t
   set_attrs();
   if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kWarps * 32, kDynSmem, s, p);
   return launch_dependent(k_expand<SLORA_F16>, grid, kWarps * 32, kDynSmem, s, p);
+}
+
+cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s) {
+  const int64_t n = (int64_t)T * (p.slot[0].t_rs / p.slot[0].t_ns);
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>((n + 255) / 256, 1), 1184);
+  return launch_dependent(k_reduce_t, grid, 256, 0, s, p);
 }
 
 cudaError_t launch_merge_requests(const int32_t* req_start, const int32_t* req_adapter, int n,

@@ -70,9 +70,9 @@ struct TableLayout {
 
 // Scratch layout inside dev_scratch.
 struct ScratchLayout {
-  size_t off_meta, off_perm, off_seg_start, off_seg_adapter, off_shrink_pre, off_expand_pre,
-      off_ctr_pre, off_ctr, off_tpart, off_tfin, off_sgmv, total;
-  int64_t ctr_cap, tpart_floats;
+  size_t off_meta, off_perm, off_seg_start, off_seg_adapter, off_seg_rank, off_shrink_pre,
+      off_expand_pre, off_tpart, off_sgmv, total;
+  int64_t tpart_floats, rk8;
   int MS;
 };
 
@@ -115,10 +115,10 @@ ScratchLayout scratch_layout(const slora_pool_desc& d) {
   const int64_t T = d.max_tokens;
   L.MS = (int)std::min<int64_t>(T, d.max_adapters);
   if (L.MS < 1) L.MS = 1;
-  int64_t sum_nck = 0;
-  for (int p = 0; p < d.n_proj; ++p) sum_nck += cdiv64(d.d_in[p], kShrinkKC);
-  L.ctr_cap = ((int64_t)d.n_proj * d.max_rank / 4 + d.n_proj) * T + 64;
-  L.tpart_floats = sum_nck * T * d.max_rank;
+  int64_t sum_ns = 0;
+  for (int p = 0; p < d.n_proj; ++p) sum_ns += cdiv64(d.d_in[p], kShrinkKT);
+  L.rk8 = std::max<int64_t>(8, (d.max_rank + 7) / 8 * 8);
+  L.tpart_floats = sum_ns * T * L.rk8;
   size_t o = 0;
   L.off_meta = o;
   o = align_up(o + 4 * kMetaCount, 256);
@@ -128,18 +128,14 @@ ScratchLayout scratch_layout(const slora_pool_desc& d) {
   o = align_up(o + 4 * (size_t)(L.MS + 1), 256);
   L.off_seg_adapter = o;
   o = align_up(o + 4 * (size_t)L.MS, 256);
+  L.off_seg_rank = o;
+  o = align_up(o + 4 * (size_t)L.MS, 256);
   L.off_shrink_pre = o;
-  o = align_up(o + 4 * (size_t)kMaxSlots * (L.MS + 1), 256);
+  o = align_up(o + 4 * (size_t)(L.MS + 1), 256);
   L.off_expand_pre = o;
-  o = align_up(o + 4 * (size_t)kMaxSlots * (L.MS + 1), 256);
-  L.off_ctr_pre = o;
-  o = align_up(o + 4 * (size_t)kMaxSlots * (L.MS + 1), 256);
-  L.off_ctr = o;
-  o = align_up(o + 4 * (size_t)L.ctr_cap, 256);
+  o = align_up(o + 4 * (size_t)(L.MS + 1), 256);
   L.off_tpart = o;
   o = align_up(o + 4 * (size_t)L.tpart_floats, 256);
-  L.off_tfin = o;
-  o = align_up(o + 4 * (size_t)d.n_proj * T * d.max_rank, 256);
   L.off_sgmv = o;
   o = align_up(o + sgmv_scratch_bytes(d), 256);
   L.total = o;
@@ -227,8 +223,9 @@ slora_status_t validate_desc(const slora_pool_desc* d, std::string* why) {
   if (d->dtype != SLORA_F16 && d->dtype != SLORA_BF16) return bad("dtype must be F16 or BF16");
   if (d->n_proj < 1 || d->n_proj > SLORA_MAX_PROJ) return bad("n_proj out of range");
   for (int p = 0; p < d->n_proj; ++p)
-    if (d->d_in[p] <= 0 || d->d_out[p] <= 0 || d->d_in[p] % 64 || d->d_out[p] % 64)
-      return bad("d_in/d_out must be positive multiples of 64");
+    if (d->d_in[p] <= 0 || d->d_out[p] <= 0 || d->d_in[p] % 64 || d->d_out[p] % 64 ||
+        d->d_in[p] > 32768)
+      return bad("d_in/d_out must be positive multiples of 64, d_in <= 32768");
   if (d->max_adapters < 1 || d->max_adapters > 16384) return bad("max_adapters out of [1, 16384]");
   if (d->max_rank < 0 || d->max_rank > 128) return bad("max_rank out of [0, 128]");
   if (d->max_tokens < 1 || d->max_tokens > (1 << 20)) return bad("max_tokens out of [1, 2^20]");
@@ -297,22 +294,36 @@ void fill_pool_dev(slora_pool* P) {
   P->pd.err = reinterpret_cast<int32_t*>(P->tables() + P->tl.off_err);
 }
 
-ScratchDev scratch_dev(slora_pool* P) {
+ScratchDev scratch_at(char* b, const ScratchLayout& L) {
   ScratchDev s{};
-  char* b = P->scratch();
-  const ScratchLayout& L = P->sl;
   s.meta = reinterpret_cast<int32_t*>(b + L.off_meta);
   s.perm = reinterpret_cast<int32_t*>(b + L.off_perm);
   s.seg_start = reinterpret_cast<int32_t*>(b + L.off_seg_start);
   s.seg_adapter = reinterpret_cast<int32_t*>(b + L.off_seg_adapter);
+  s.seg_rank = reinterpret_cast<int32_t*>(b + L.off_seg_rank);
   s.shrink_prefix = reinterpret_cast<int32_t*>(b + L.off_shrink_pre);
   s.expand_prefix = reinterpret_cast<int32_t*>(b + L.off_expand_pre);
-  s.ctr_prefix = reinterpret_cast<int32_t*>(b + L.off_ctr_pre);
-  s.seg_rank = s.ctr_prefix + (L.MS + 1);
-  s.ctr = reinterpret_cast<int32_t*>(b + L.off_ctr);
-  s.ctr_cap = L.ctr_cap;
   s.MS = L.MS;
   return s;
+}
+
+ScratchDev scratch_dev(slora_pool* P) { return scratch_at(P->scratch(), P->sl); }
+
+// Points each slot's t at its share of the fp32 partials region (position-
+// ordered rows of rk8 * nsplit floats for T tokens).  False when they do not fit.
+bool assign_partials(BgmvParams& bp, float* base, int64_t cap_floats, int64_t T, int64_t rk8) {
+  int64_t off = 0;
+  for (int k = 0; k < bp.n_slots; ++k) {
+    SlotDev& S = bp.slot[k];
+    S.t = base + off;
+    S.t_rs = rk8 * S.nsplit;
+    S.t_ns = S.nsplit;
+    S.t_by_token = 0;
+    S.tout = nullptr;
+    S.ldt_out = 0;
+    off += (int64_t)S.nsplit * T * rk8;
+  }
+  return off <= cap_floats;
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
@@ -326,9 +337,6 @@ slora_status_t plan_slots(slora_pool* P, BgmvParams& bp, int n, const int32_t* p
   if (!projs) return P->fail(SLORA_ERR_INVALID_ARG, "projs is NULL");
   bp.n_slots = n;
   bp.n_groups = 0;
-  int64_t tpart_off = 0;
-  float* tpart_base = reinterpret_cast<float*>(P->scratch() + P->sl.off_tpart);
-  float* tfin_base = reinterpret_cast<float*>(P->scratch() + P->sl.off_tfin);
   for (int k = 0; k < n; ++k) {
     const int p = projs[k];
     if (p < 0 || p >= P->d.n_proj) return P->fail(SLORA_ERR_INVALID_ARG, "projection id out of range");
@@ -338,7 +346,7 @@ slora_status_t plan_slots(slora_pool* P, BgmvParams& bp, int n, const int32_t* p
     S.d_out = P->d.d_out[p];
     S.listA = P->listA[p];
     S.listB = P->listB[p];
-    S.nck = (int)cdiv64(S.d_in, kShrinkKC);
+    S.nsplit = (int)cdiv64(S.d_in, kShrinkKT);
     if (need_x) {
       if (!x || !ldx || !x[k]) return P->fail(SLORA_ERR_INVALID_ARG, "x is NULL");
       if (ldx[k] < S.d_in || ldx[k] % 8 || !aligned16(x[k]))
@@ -353,11 +361,6 @@ slora_status_t plan_slots(slora_pool* P, BgmvParams& bp, int n, const int32_t* p
       S.y = static_cast<uint16_t*>(y[k]);
       S.ldy = ldy[k];
     }
-    S.tpart = tpart_base + tpart_off;
-    tpart_off += (int64_t)S.nck * P->d.max_tokens * P->d.max_rank;
-    S.tfin = tfin_base + (int64_t)k * P->d.max_tokens * P->d.max_rank;
-    S.ldt = P->d.max_rank > 0 ? P->d.max_rank : 1;
-    S.t_by_token = 0;
     // x-sharing groups
     int g = -1;
     if (need_x)
@@ -374,7 +377,8 @@ slora_status_t plan_slots(slora_pool* P, BgmvParams& bp, int n, const int32_t* p
     S.gpos = bp.group[g].n;
     bp.group[g].slot[bp.group[g].n++] = k;
   }
-  if (tpart_off > P->sl.tpart_floats)
+  if (!assign_partials(bp, reinterpret_cast<float*>(P->scratch() + P->sl.off_tpart), P->sl.tpart_floats,
+                       P->d.max_tokens, P->sl.rk8))
     return P->fail(SLORA_ERR_INVALID_ARG, "too many projections in one call for the scratch size");
   if (T < 0 || T > P->d.max_tokens) return P->fail(SLORA_ERR_INVALID_ARG, "T out of [0, max_tokens]");
   return SLORA_OK;
@@ -424,26 +428,9 @@ slora_status_t lora_delta_on_scratch(slora_pool* P, int32_t n, const int32_t* pr
                    " (fewer tokens, projections or a smaller max_rank fit)");
   char* b = static_cast<char*>(scratch);
   bp.max_tokens = T;
-  bp.sc.meta = reinterpret_cast<int32_t*>(b + L.off_meta);
-  bp.sc.perm = reinterpret_cast<int32_t*>(b + L.off_perm);
-  bp.sc.seg_start = reinterpret_cast<int32_t*>(b + L.off_seg_start);
-  bp.sc.seg_adapter = reinterpret_cast<int32_t*>(b + L.off_seg_adapter);
-  bp.sc.shrink_prefix = reinterpret_cast<int32_t*>(b + L.off_shrink_pre);
-  bp.sc.expand_prefix = reinterpret_cast<int32_t*>(b + L.off_expand_pre);
-  bp.sc.ctr_prefix = reinterpret_cast<int32_t*>(b + L.off_ctr_pre);
-  bp.sc.seg_rank = bp.sc.ctr_prefix + (L.MS + 1);
-  bp.sc.ctr = reinterpret_cast<int32_t*>(b + L.off_ctr);
-  bp.sc.ctr_cap = L.ctr_cap;
-  bp.sc.MS = L.MS;
-  float* tpart = reinterpret_cast<float*>(b + L.off_tpart);
-  float* tfin = reinterpret_cast<float*>(b + L.off_tfin);
-  int64_t off = 0;
-  for (int k = 0; k < bp.n_slots; ++k) {
-    bp.slot[k].tpart = tpart + off;
-    off += (int64_t)bp.slot[k].nck * T * P->d.max_rank;
-    bp.slot[k].tfin = tfin + (int64_t)k * T * P->d.max_rank;
-  }
-  if (off > L.tpart_floats) return P->fail(SLORA_ERR_INVALID_ARG, "too many projections in one call");
+  bp.sc = scratch_at(b, L);
+  if (!assign_partials(bp, reinterpret_cast<float*>(b + L.off_tpart), L.tpart_floats, T, L.rk8))
+    return P->fail(SLORA_ERR_INVALID_ARG, "too many projections in one call");
   bp.do_shrink = 1;
   bp.do_expand = 1;
   CUDA_TRY(P, launch_segments(bp, idx, T, st));
@@ -902,7 +889,8 @@ slora_status_t slora_bgmv_shrink(slora_pool* P, int32_t proj, const void* x, int
   slora_status_t s = need_device(P);
   if (s) return s;
   if (T > 0 && (!idx || !t)) return P->fail(SLORA_ERR_INVALID_ARG, "idx / t is NULL");
-  if (ldt < P->d.max_rank || ((uintptr_t)t & 15) || ldt % 4) return P->fail(SLORA_ERR_INVALID_ARG, "t: ldt >= max_rank, ldt % 4 == 0, 16-byte aligned");
+  if (ldt < P->d.max_rank || ((uintptr_t)t & 15) || ldt % 8)
+    return P->fail(SLORA_ERR_INVALID_ARG, "t: ldt >= max_rank, ldt % 8 == 0, 16-byte aligned");
   BgmvParams bp;
   base_params(P, bp);
   const void* xs[1] = {x};
@@ -910,15 +898,19 @@ slora_status_t slora_bgmv_shrink(slora_pool* P, int32_t proj, const void* x, int
   s = plan_slots(P, bp, 1, &proj, xs, lx, nullptr, nullptr, T, true, false);
   if (s) return s;
   if (T == 0) return SLORA_OK;
-  bp.slot[0].tfin = t;
-  bp.slot[0].ldt = ldt;
-  bp.slot[0].t_by_token = 1;
+  bp.slot[0].tout = t;
+  bp.slot[0].ldt_out = ldt;
   bp.do_shrink = 1;
   bp.do_expand = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   CUDA_TRY(P, cudaMemsetAsync(t, 0, sizeof(float) * (size_t)T * ldt, st));
+  phase(P, 0, 3, st);
   CUDA_TRY(P, launch_segments(bp, idx, T, st));
+  phase(P, 1, 3, st);
   CUDA_TRY(P, launch_shrink(bp, P->d.dtype, P->grid_shrink, st));
+  phase(P, 2, 3, st);
+  CUDA_TRY(P, launch_reduce_t(bp, T, st));
+  phase(P, 3, 3, st);
   record_epoch(P, st);
   return SLORA_OK;
 }
@@ -929,7 +921,8 @@ slora_status_t slora_bgmv_expand(slora_pool* P, int32_t proj, const float* t, in
   slora_status_t s = need_device(P);
   if (s) return s;
   if (T > 0 && (!idx || !t)) return P->fail(SLORA_ERR_INVALID_ARG, "idx / t is NULL");
-  if (ldt < P->d.max_rank || ((uintptr_t)t & 15) || ldt % 4) return P->fail(SLORA_ERR_INVALID_ARG, "t: ldt >= max_rank, ldt % 4 == 0, 16-byte aligned");
+  if (ldt < P->d.max_rank || ((uintptr_t)t & 15) || ldt % 8)
+    return P->fail(SLORA_ERR_INVALID_ARG, "t: ldt >= max_rank, ldt % 8 == 0, 16-byte aligned");
   BgmvParams bp;
   base_params(P, bp);
   void* ys[1] = {y};
@@ -937,14 +930,18 @@ slora_status_t slora_bgmv_expand(slora_pool* P, int32_t proj, const float* t, in
   s = plan_slots(P, bp, 1, &proj, nullptr, nullptr, ys, ly, T, false, true);
   if (s) return s;
   if (T == 0) return SLORA_OK;
-  bp.slot[0].tfin = const_cast<float*>(t);
-  bp.slot[0].ldt = ldt;
+  bp.slot[0].t = const_cast<float*>(t);
+  bp.slot[0].t_rs = ldt;
+  bp.slot[0].t_ns = 1;
   bp.slot[0].t_by_token = 1;
   bp.do_shrink = 0;
   bp.do_expand = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  phase(P, 0, 2, st);
   CUDA_TRY(P, launch_segments(bp, idx, T, st));
+  phase(P, 1, 2, st);
   CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
+  phase(P, 2, 2, st);
   record_epoch(P, st);
   return SLORA_OK;
 }

@@ -9,10 +9,11 @@
 
 namespace slora {
 
-// Shrink work split (decode path).  A task covers RW rank rows x NT tokens x
-// KC elements of d_in; KC is fixed so every projection has a fixed number of
-// fp32 partial slices (ceil(d_in / KC)).
-constexpr int kShrinkKC = 512;
+// Shrink work split (decode path).  A shrink task covers RW rank rows x NT
+// tokens x kShrinkKT elements of d_in, streamed in stages of kStageK; its
+// fp32 partial (one per kShrinkKT slice of d_in) is summed by the expand.
+constexpr int kShrinkKT = 1024;
+constexpr int kStageK = 512;
 constexpr int kMaxSlots = SLORA_MAX_PROJ;   // projections per call
 constexpr int kThreads = 256;               // threads per CTA of the decode kernels
 constexpr int kEventRing = 64;
@@ -38,13 +39,18 @@ struct SlotDev {
   int64_t ldy;
   int d_in, d_out;
   int listA, listB;        // offsets of this projection's A_t / B page lists in an adapter row
-  int nck;                 // shrink partial slices = ceil(d_in / kShrinkKC)
+  int nsplit;              // shrink partials = ceil(d_in / kShrinkKT)
   int group;               // index of the x-sharing group
   int gpos;                // rank-row block of this slot inside its group
-  float* tpart;            // [nck][max_tokens][max_rank], position-ordered
-  float* tfin;             // final t: position-ordered [max_tokens][ldt] or token-ordered
-  int64_t ldt;
-  int t_by_token;          // 1: tfin row = token id; 0: row = position in perm order
+  // t (rank-r intermediate): element (row, k, c) at t[row * t_rs + k * t_ns + c],
+  // summed over c < t_ns.  row = position in perm order, or the token id when
+  // t_by_token (a caller's dense t, t_ns = 1).
+  float* t;
+  int64_t t_rs;
+  int t_ns;
+  int t_by_token;
+  float* tout;             // slora_bgmv_shrink: reduced t per token (ldt_out), else NULL
+  int64_t ldt_out;
 };
 
 struct GroupDev {
@@ -60,18 +66,15 @@ struct ScratchDev {
   int32_t* perm;           // [max_tokens]
   int32_t* seg_start;      // [MS + 1]
   int32_t* seg_adapter;    // [MS]
-  int32_t* meta;           // [16]: S, n_valid, shrink total, expand total, ctr total, work counters
+  int32_t* meta;           // [16]: S, n_valid, shrink total, expand total
   int32_t* shrink_prefix;  // [MS + 1] shrink tasks before each segment (segment-major)
   int32_t* expand_prefix;  // [MS + 1] expand tasks before each segment
-  int32_t* ctr_prefix;     // [MS + 1] reduction counters before each segment
   int32_t* seg_rank;       // [MS] rank of each segment's adapter
-  int32_t* ctr;            // reduction counters
-  int64_t ctr_cap;
   int MS;                  // max segments = min(max_tokens, max_adapters)
 };
 
 enum MetaIdx { kMetaS = 0, kMetaValid = 1, kMetaShrinkTotal = 2, kMetaExpandTotal = 3,
-               kMetaCtrTotal = 4, kMetaShrinkWork = 5, kMetaExpandWork = 6, kMetaCount = 16 };
+               kMetaCount = 16 };
 
 struct BgmvParams {
   PoolDev pool;
@@ -110,6 +113,7 @@ struct PageInNew {
 cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cudaStream_t s);
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s);
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s);
+cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s);
 cudaError_t launch_merge_requests(const int32_t* req_start, const int32_t* req_adapter, int n,
                                   int32_t* seg_start, int32_t* seg_adapter, int32_t* S_out,
                                   cudaStream_t s);

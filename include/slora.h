@@ -97,7 +97,7 @@ typedef struct slora_pool slora_pool;
 typedef struct {
   int32_t dtype;            /* slora_dtype_t                                         */
   int32_t n_proj;           /* projections per adapter, 1..SLORA_MAX_PROJ            */
-  int32_t d_in[SLORA_MAX_PROJ];  /* multiples of 64                                  */
+  int32_t d_in[SLORA_MAX_PROJ];  /* multiples of 64, at most 32768                   */
   int32_t d_out[SLORA_MAX_PROJ]; /* multiples of 64                                  */
   int32_t max_adapters;     /* adapter ids are 0..max_adapters-1 (<= 16384)          */
   int32_t max_rank;         /* ranks in [0, max_rank], max_rank <= 128               */
@@ -227,7 +227,8 @@ slora_status_t slora_build_sgmv_segments(slora_pool* pool, const int32_t* req_st
 
 /* BGMV shrink for one projection (decode): t[i, k] = sum_j x[i, j] * A_a[j, k]
  * for k < r_a, a = idx[i]; t[i, k] = 0 for k >= r_a and for rows with no
- * adapter.  x: T x d_in[proj] (ldx), t: T x ldt fp32 (ldt >= max_rank), idx: T
+ * adapter.  x: T x d_in[proj] (ldx), t: T x ldt fp32 (ldt >= max_rank, a multiple
+ * of 8, 16-byte aligned), idx: T
  * int32; all device.  [S2 SGMV first phase; S1 BGMV]                           */
 slora_status_t slora_bgmv_shrink(slora_pool* pool, int32_t proj, const void* x, int64_t ldx,
                                  const int32_t* idx, int32_t T, float* t, int64_t ldt,
@@ -235,7 +236,8 @@ slora_status_t slora_bgmv_shrink(slora_pool* pool, int32_t proj, const void* x, 
 
 /* BGMV expand for one projection (decode):
  * y[i, l] <- round(y[i, l] + (alpha_a / r_a) * sum_{k < r_a} t[i, k] * B_a[k, l]).
- * t: T x ldt fp32, y: T x d_out[proj] (ldy); device.  [S2 second phase]        */
+ * t: T x ldt fp32 (as for slora_bgmv_shrink), y: T x d_out[proj] (ldy); device.
+ * [S2 second phase]        */
 slora_status_t slora_bgmv_expand(slora_pool* pool, int32_t proj, const float* t, int64_t ldt,
                                  const int32_t* idx, int32_t T, void* y, int64_t ldy,
                                  void* stream);
