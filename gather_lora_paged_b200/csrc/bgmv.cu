@@ -35,11 +35,11 @@ namespace slora {
 
 #define FULL_MASK 0xffffffffu
 
-constexpr int kWarps = 8;                 // warps per CTA of shrink / expand
+constexpr int kWarps = 16;                // warps per CTA of shrink / expand
 constexpr int kSlots = 2;                 // pipeline slots per warp
-constexpr int kSlotBytes = 12 * 1024;     // bytes per slot
+constexpr int kSlotBytes = 6 * 1024 + 128; // bytes per slot
 constexpr int kSmemBytes = kWarps * kSlots * kSlotBytes;
-constexpr int kExpandRows = 8;            // B rows per expand stage
+constexpr int kExpandRows = 4;            // B rows per expand stage
 constexpr int kLC = 256;                  // outputs per expand task (8 per lane)
 constexpr long long kWaitLimit = 2000000000ll;  // clock cycles before a wait gives up
 
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) k_shrink(const __grid_constant
 // B row i at i * 512 B; t partials of token t at kExpT + t * 8 * t_ns * 4 B;
 // y row t (last stage) at kExpY + t * 512 B; t sums at kExpS.
 constexpr int kExpT = kExpandRows * 2 * kLC;
-constexpr int kExpY = 8 * 1024;
+constexpr int kExpY = 4 * 1024;
 constexpr int kExpS = kExpY + 4 * 2 * kLC;
 static_assert(kExpS + 4 * kExpandRows * 4 <= kSlotBytes, "expand slot overflow");
 
@@ -716,9 +716,16 @@ __device__ __forceinline__ void expand_stage(const BgmvParams& p, const ETask& t
     const int tt = lane >> 3, kk = lane & 7;
     if (tt < t.ntok && kk < nrows) {
       const float* src = reinterpret_cast<const float*>(buf + kExpT + tt * 4 * kExpandRows * L.t_ns) + kk * L.t_ns;
-      float s = 0.f;
-      for (int c = 0; c < L.t_ns; ++c) s += src[c];
-      tsum[tt * kExpandRows + kk] = s;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // four chains; fixed association
+      int c = 0;
+      for (; c + 4 <= L.t_ns; c += 4) {
+        s0 += src[c];
+        s1 += src[c + 1];
+        s2 += src[c + 2];
+        s3 += src[c + 3];
+      }
+      for (; c < L.t_ns; ++c) s0 += src[c];
+      tsum[tt * kExpandRows + kk] = (s0 + s1) + (s2 + s3);
     }
   }
   __syncwarp();

@@ -13,7 +13,7 @@ namespace slora {
 // tokens x kShrinkKT elements of d_in, streamed in stages of kStageK; its
 // fp32 partial (one per kShrinkKT slice of d_in) is summed by the expand.
 constexpr int kShrinkKT = 1024;
-constexpr int kStageK = 512;
+constexpr int kStageK = 256;
 constexpr int kMaxSlots = SLORA_MAX_PROJ;   // projections per call
 constexpr int kThreads = 256;               // threads per CTA of the decode kernels
 constexpr int kEventRing = 64;
