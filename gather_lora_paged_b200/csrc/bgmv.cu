@@ -35,22 +35,24 @@ namespace slora {
 
 #define FULL_MASK 0xffffffffu
 
-constexpr int kWarps = 16;                // warps per CTA of shrink / expand
-constexpr int kSlots = 2;                 // pipeline slots per warp
-constexpr int kSlotBytes = 6 * 1024 + 128; // bytes per slot
-constexpr int kSmemBytes = kWarps * kSlots * kSlotBytes;
-constexpr int kExpandRows = 4;            // B rows per expand stage
-constexpr int kLC = 256;                  // outputs per expand task (8 per lane)
 constexpr long long kWaitLimit = 2000000000ll;  // clock cycles before a wait gives up
 
 __host__ __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
 
-// Task shapes.  Shrink tasks cover NT tokens x RW rank rows x kShrinkKT of
-// d_in; expand tasks NTE tokens x kLC outputs.  Slot use per stage: (RW + NT)
-// KiB for shrink; 8 B rows, the t partials and y rows for expand.
+// Task shapes.  A shrink task covers NT tokens x kRB rank rows x kShrinkKT of
+// d_in; an expand task NTE tokens x kELC outputs (all rank rows).
 __host__ __device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
-__host__ __device__ __forceinline__ int rw_of(int nt) { return nt == 1 ? 8 : 4; }
 __host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
+constexpr int kCW = 8;                        // consumer warps per CTA
+constexpr int kPipeThreads = (kCW + 1) * 32;  // + the producer warp
+constexpr int kNS = 8;                        // ring stages
+constexpr int kStageBytes = 24 * 1024;
+constexpr int kRingBytes = kNS * kStageBytes;
+constexpr int kDescInts = 32;                 // per-stage descriptor (task fields)
+constexpr int kRB = 16;                       // shrink task: rank rows (2 per consumer warp)
+constexpr int kER = 4;                        // expand stage: rank rows
+constexpr int kELC = kCW * 256;               // expand task: outputs (256 per consumer warp)
+constexpr int kMaxPieces = 5;                 // pieces of a 2048-element row over >= 512-element pages
 
 __device__ __forceinline__ void record_error(int32_t* err, int code, int info) {
   if (atomicCAS(&err[0], 0, code) == 0) atomicExch(&err[1], info);
@@ -186,9 +188,9 @@ __device__ __forceinline__ void seg_task_counts(const BgmvParams& p, int n, int 
   const int nt = nt_class(n), ntg = cdiv_i(n, nt), nte = cdiv_i(n, nte_class(n));
   if (p.do_shrink)
     for (int g = 0; g < p.n_groups; ++g)
-      shr += cdiv_i(p.group[g].n * r, rw_of(nt)) * ntg * cdiv_i(p.group[g].d_in, kShrinkKT);
+      shr += cdiv_i(p.group[g].n * r, kRB) * ntg * cdiv_i(p.group[g].d_in, kShrinkKT);
   if (p.do_expand)
-    for (int k = 0; k < p.n_slots; ++k) exp += nte * cdiv_i(p.slot[k].d_out, kLC);
+    for (int k = 0; k < p.n_slots; ++k) exp += nte * cdiv_i(p.slot[k].d_out, kELC);
 }
 
 __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvParams p,
@@ -376,33 +378,34 @@ __device__ __forceinline__ const uint16_t* page_ptr(const PoolDev& P, int32_t pg
   return P.pool + ((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1));
 }
 
-// A paged range [f0, f0 + n) (n <= page size) is copied as piece 0 (the part
-// in f0's page) and piece 1 (the rest, if the range crosses a page boundary).
-// aux_page: the page id of the lane's piece, looked up one stage ahead.
-__device__ __forceinline__ int32_t piece_page(const PoolDev& P, int a, int lo, int64_t f0, int n, int piece) {
-  const int64_t pb = ((f0 >> P.page_shift) + 1) << P.page_shift;
-  if (piece == 0) return page_id(P, a, lo, f0);
-  return (f0 + n > pb) ? page_id(P, a, lo, pb) : -1;
-}
-__device__ __forceinline__ void piece_copy(const PoolDev& P, int32_t pg, int64_t f0, int n, int piece,
-                                           unsigned char* dst, uint64_t* bar) {
-  const int64_t pb = ((f0 >> P.page_shift) + 1) << P.page_shift;
-  const int64_t f1 = f0 + n;
-  if (piece == 0) {
-    const int64_t e = f1 < pb ? f1 : pb;
-    bulk_g2s(dst, page_ptr(P, pg, f0), (uint32_t)(2 * (e - f0)), bar);
-  } else if (f1 > pb) {
-    bulk_g2s(dst + 2 * (pb - f0), page_ptr(P, pg, pb), (uint32_t)(2 * (f1 - pb)), bar);
-  }
+// ---------------------------------------------------------------------------
+// Shrink and expand run as warp-specialised persistent CTAs: one producer warp
+// walks the CTA's (task, stage) sequence and fills a ring of kNS shared-memory
+// stages with page-gathered bulk copies (cp.async.bulk, completion counted on
+// the stage's `full` mbarrier); kCW consumer warps each compute a fixed slice
+// of every stage and release it on the stage's `empty` mbarrier.  Page ids and
+// token ids are looked up two stages before the stage is issued.
+// A paged range [f0, f1) cut at page boundaries: piece q starts at f0 (q = 0)
+// or at the q-th boundary after f0.
+__device__ __forceinline__ bool piece_range(const PoolDev& P, int64_t f0, int64_t f1, int q, int64_t& b,
+                                            int64_t& e) {
+  const int64_t PE = 1ll << P.page_shift;
+  const int64_t pb0 = ((f0 >> P.page_shift) + 1) << P.page_shift;
+  b = q == 0 ? f0 : pb0 + (int64_t)(q - 1) * PE;
+  e = pb0 + (int64_t)q * PE;
+  if (e > f1) e = f1;
+  return b < f1;
 }
 
 // ---------------------------------------------------------------------------
-// Shrink.  Task = (group g, segment, RW rank rows, NT tokens, kShrinkKT slice
-// of d_in), streamed in stages of kStageK elements.  Slot layout of a stage:
-// rank row i at i * 1 KiB, token row t at (RW + t) * 1 KiB.
+// Shrink task = (group g, segment, kRB rank rows, NT tokens, kShrinkKT slice
+// of d_in); stages of kStageK elements.  Stage layout: rank row i at
+// i * 1 KiB, token row t at (kRB + t) * 1 KiB.  Consumer warp w owns rows
+// 2w and 2w + 1 of the task.
 struct STask {
-  int g, a, r, seg0, n, nt, rw, rg, tg, split, nst, nrows, ntok;
+  int g, a, r, seg0, n, nt, rg, tg, split, nst, nrows, ntok;
 };
+static_assert(sizeof(STask) / 4 + 2 <= kDescInts, "descriptor too small");
 
 __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView& V, int task, STask& t) {
   const int s = find_seg(V.prefix, V.S, task);
@@ -412,11 +415,10 @@ __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView
   t.n = V.start[s + 1] - t.seg0;
   t.r = V.rank[s];
   t.nt = nt_class(t.n);
-  t.rw = rw_of(t.nt);
   const int n_tg = cdiv_i(t.n, t.nt);
   int g = 0;
   for (; g < p.n_groups - 1; ++g) {  // the group owning local task q
-    const int cnt = cdiv_i(p.group[g].n * t.r, t.rw) * n_tg * cdiv_i(p.group[g].d_in, kShrinkKT);
+    const int cnt = cdiv_i(p.group[g].n * t.r, kRB) * n_tg * cdiv_i(p.group[g].d_in, kShrinkKT);
     if (q < cnt) break;
     q -= cnt;
   }
@@ -428,208 +430,239 @@ __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView
   t.split = q % n_split;
   t.rg = q / n_split;
   t.nst = cdiv_i(min(kShrinkKT, d_in - t.split * kShrinkKT), kStageK);
-  t.nrows = min(t.rw, p.group[g].n * t.r - t.rg * t.rw);
+  t.nrows = min(kRB, p.group[g].n * t.r - t.rg * kRB);
   t.ntok = min(t.nt, t.n - t.tg * t.nt);
 }
 
-// Lane roles in a shrink stage: lane i < 16 copies piece 0 of rank row i
-// (i < nrows) or token row i - nrows; lane 16 + i copies piece 1 of row i.
-// The per-lane lookup (page id or token id) is done one stage ahead.
-__device__ __forceinline__ int32_t shrink_lookup(const BgmvParams& p, const STask& t, int st) {
+struct SCursor {  // a point of the producer's (task, stage) sequence
+  STask t;
+  int task, st;
+  bool valid;
+};
+
+__device__ __forceinline__ void scursor_next(const BgmvParams& p, const SegView& V, int total, SCursor& c) {
+  if (!c.valid) return;
+  if (++c.st < c.t.nst) return;
+  c.st = 0;
+  c.task += gridDim.x;
+  c.valid = c.task < total;
+  if (c.valid) decode_shrink(p, V, c.task, c.t);
+}
+
+// Per-lane lookups of a shrink stage: lane l copies piece l >> 4 of row l & 15
+// (aux0 = its page id); lane l < ntok also copies token row l (aux1 = token).
+__device__ __forceinline__ void shrink_lookup(const BgmvParams& p, const SCursor& c, int32_t& aux0,
+                                              int32_t& aux1) {
   const int lane = threadIdx.x & 31, i = lane & 15;
+  aux0 = -1;
+  aux1 = -1;
+  if (!c.valid) return;
+  const STask& t = c.t;
   const GroupDev& G = p.group[t.g];
-  const int k0 = t.split * kShrinkKT + st * kStageK;
+  const int k0 = t.split * kShrinkKT + c.st * kStageK;
   const int L = min(kStageK, G.d_in - k0);
   if (i < t.nrows) {
-    const int rho = t.rg * t.rw + i;
+    const int rho = t.rg * kRB + i;
     const int j = rho / t.r, k = rho % t.r;
-    return piece_page(p.pool, t.a, p.slot[G.slot[j]].listA, (int64_t)k * G.d_in + k0, L, lane >> 4);
+    const int64_t f0 = (int64_t)k * G.d_in + k0;
+    int64_t b, e;
+    if (piece_range(p.pool, f0, f0 + L, lane >> 4, b, e))
+      aux0 = page_id(p.pool, t.a, p.slot[G.slot[j]].listA, b);
   }
-  if (lane < 16 && i < t.nrows + t.ntok) return __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + (i - t.nrows));
-  return -1;
+  if (lane < t.ntok) aux1 = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
 }
 
-__device__ __forceinline__ void issue_shrink(const BgmvParams& p, const STask& t, int st, int32_t aux,
-                                             unsigned char* buf, uint64_t* bar) {
+__device__ __forceinline__ void shrink_issue(const BgmvParams& p, const SCursor& c, int32_t aux0, int32_t aux1,
+                                             unsigned char* buf, int32_t* desc, uint64_t* bar) {
   const int lane = threadIdx.x & 31, i = lane & 15;
+  const STask& t = c.t;
   const GroupDev& G = p.group[t.g];
-  const int k0 = t.split * kShrinkKT + st * kStageK;
+  const int k0 = t.split * kShrinkKT + c.st * kStageK;
   const int L = min(kStageK, G.d_in - k0);
-  if (lane == 0) mbar_expect_tx(bar, 2u * L * (t.nrows + t.ntok));
-  __syncwarp();
-  if (i < t.nrows) {
-    const int rho = t.rg * t.rw + i;
-    const int k = rho % t.r;
-    piece_copy(p.pool, aux, (int64_t)k * G.d_in + k0, L, lane >> 4, buf + i * 2 * kStageK, bar);
-  } else if (lane < 16 && i < t.nrows + t.ntok) {
-    bulk_g2s(buf + (t.rw + i - t.nrows) * 2 * kStageK, G.x + (int64_t)aux * G.ldx + k0, 2u * L, bar);
+  if (lane == 0) {
+    const int32_t* src = reinterpret_cast<const int32_t*>(&t);
+    for (int q = 0; q < (int)(sizeof(STask) / 4); ++q) desc[q] = src[q];
+    desc[kDescInts - 2] = c.st;
+    desc[kDescInts - 1] = 1;
+    mbar_expect_tx(bar, 2u * L * (t.nrows + t.ntok));
   }
+  __syncwarp();
+  if (aux0 >= 0) {
+    const int rho = t.rg * kRB + i;
+    const int64_t f0 = (int64_t)(rho % t.r) * G.d_in + k0;
+    int64_t b, e;
+    piece_range(p.pool, f0, f0 + L, lane >> 4, b, e);
+    bulk_g2s(buf + i * 2 * kStageK + 2 * (b - f0), page_ptr(p.pool, aux0, b), (uint32_t)(2 * (e - b)), bar);
+  }
+  if (aux1 >= 0)
+    bulk_g2s(buf + (kRB + lane) * 2 * kStageK, G.x + (int64_t)aux1 * G.ldx + k0, 2u * L, bar);
 }
 
-template <int DT, int NT, int RW>
-__device__ __forceinline__ void shrink_stage(const BgmvParams& p, const STask& t, int st,
-                                             const unsigned char* buf, float (&acc)[32]) {
-  const int lane = threadIdx.x & 31;
+template <int DT, int NT>
+__device__ __forceinline__ void shrink_consume(const BgmvParams& p, const STask& t, int st,
+                                               const unsigned char* buf, float (&acc)[16]) {
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 1;
   const GroupDev& G = p.group[t.g];
   const int k0 = t.split * kShrinkKT + st * kStageK;
   const int L = min(kStageK, G.d_in - k0);
+  const int i0 = 2 * cw;
+  if (i0 < t.nrows) {
+    const bool r1 = i0 + 1 < t.nrows;
 #pragma unroll
-  for (int e = lane * 8; e < kStageK; e += 256) {
-    if (e >= L) break;
-    uint4 av[RW], xv[NT];
+    for (int h = 0; h < kStageK / 256; ++h) {
+      const int e = h * 256 + lane * 8;
+      if (e >= L) break;
+      float a0[8], a1[8];
+      unpack8<DT>(lds128(buf + i0 * 2 * kStageK + 2 * e), a0);
+      if (r1) unpack8<DT>(lds128(buf + (i0 + 1) * 2 * kStageK + 2 * e), a1);
+      else
 #pragma unroll
-    for (int i = 0; i < RW; ++i)
-      av[i] = i < t.nrows ? lds128(buf + i * 2 * kStageK + 2 * e) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt)
-      xv[tt] = tt < t.ntok ? lds128(buf + (RW + tt) * 2 * kStageK + 2 * e) : make_uint4(0, 0, 0, 0);
-    if (NT <= 2) {
-      float xf[NT][8];
-#pragma unroll
-      for (int tt = 0; tt < NT; ++tt) unpack8<DT>(xv[tt], xf[tt]);
-#pragma unroll
-      for (int i = 0; i < RW; ++i) {
-        float af[8];
-        unpack8<DT>(av[i], af);
-#pragma unroll
-        for (int tt = 0; tt < NT; ++tt) {
-          float s = acc[i * NT + tt];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) s = fmaf(af[q], xf[tt][q], s);
-          acc[i * NT + tt] = s;
-        }
-      }
-    } else {
-      float af[RW][8];
-#pragma unroll
-      for (int i = 0; i < RW; ++i) unpack8<DT>(av[i], af[i]);
+        for (int q = 0; q < 8; ++q) a1[q] = 0.f;
 #pragma unroll
       for (int tt = 0; tt < NT; ++tt) {
+        if (tt >= t.ntok) break;
         float xf[8];
-        unpack8<DT>(xv[tt], xf);
+        unpack8<DT>(lds128(buf + (kRB + tt) * 2 * kStageK + 2 * e), xf);
+        float s0 = acc[tt], s1 = acc[NT + tt];
 #pragma unroll
-        for (int i = 0; i < RW; ++i) {
-          float s = acc[i * NT + tt];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) s = fmaf(af[i][q], xf[q], s);
-          acc[i * NT + tt] = s;
+        for (int q = 0; q < 8; ++q) {
+          s0 = fmaf(a0[q], xf[q], s0);
+          s1 = fmaf(a1[q], xf[q], s1);
         }
+        acc[tt] = s0;
+        acc[NT + tt] = s1;
       }
     }
   }
-}
-
-// End of a shrink task: sum over lanes and store the fp32 partial of this
-// d_in slice, t[pos][k][split], for RW rows x NT tokens.
-template <int NT, int RW>
-__device__ __forceinline__ void shrink_finish(const BgmvParams& p, const STask& t, float (&acc)[32]) {
-  constexpr int N = RW * NT;
+  if (st != t.nst - 1) return;
+  // end of the task: sum over lanes, store the fp32 partial of this d_in slice
+  constexpr int N = 2 * NT;
   float v[N];
 #pragma unroll
-  for (int i = 0; i < N; ++i) v[i] = acc[i];
+  for (int q = 0; q < N; ++q) v[q] = acc[q];
   const float val = lane_transpose_reduce<N>(v);
-  const int lane = threadIdx.x & 31;
   const int Lx = lane % N;
-  const int i = Lx / NT, tt = Lx % NT;
+  const int i = i0 + Lx / NT, tt = Lx % NT;
   if (lane < N && i < t.nrows && tt < t.ntok) {
-    const int rho = t.rg * RW + i;
+    const int rho = t.rg * kRB + i;
     const int j = rho / t.r, k = rho % t.r;
-    const SlotDev& S = p.slot[p.group[t.g].slot[j]];
-    const int pos = t.seg0 + t.tg * NT + tt;
+    const SlotDev& S = p.slot[G.slot[j]];
+    const int pos = t.seg0 + t.tg * t.nt + tt;
     S.t[(int64_t)pos * S.t_rs + (int64_t)k * S.t_ns + t.split] = val;
   }
 #pragma unroll
-  for (int q = 0; q < 32; ++q) acc[q] = 0.f;
+  for (int q = 0; q < 16; ++q) acc[q] = 0.f;
 }
 
 template <int DT>
-__device__ __forceinline__ void shrink_stage_any(const BgmvParams& p, const STask& t, int st,
-                                                 const unsigned char* buf, float (&acc)[32]) {
-  const bool last = st == t.nst - 1;
-  switch (t.nt) {
-    case 1: shrink_stage<DT, 1, 8>(p, t, st, buf, acc); if (last) shrink_finish<1, 8>(p, t, acc); break;
-    case 2: shrink_stage<DT, 2, 4>(p, t, st, buf, acc); if (last) shrink_finish<2, 4>(p, t, acc); break;
-    case 4: shrink_stage<DT, 4, 4>(p, t, st, buf, acc); if (last) shrink_finish<4, 4>(p, t, acc); break;
-    default: shrink_stage<DT, 8, 4>(p, t, st, buf, acc); if (last) shrink_finish<8, 4>(p, t, acc); break;
-  }
-}
-
-template <int DT>
-__global__ void __launch_bounds__(kWarps * 32, 1) k_shrink(const __grid_constant__ BgmvParams p) {
+__global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constant__ BgmvParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t bars[kWarps][kSlots];
+  __shared__ __align__(8) uint64_t full[kNS], empty[kNS];
+  __shared__ int32_t desc[kNS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* wbuf = smem + warp * kSlots * kSlotBytes;
-  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kSmemBytes);
-  if (lane == 0)
-    for (int s = 0; s < kSlots; ++s) mbar_init(&bars[warp][s], 1);
-  fence_mbar_init();
+  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kRingBytes);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCW);
+    }
+    fence_mbar_init();
+  }
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaShrinkTotal];
   const SegView V = stage_segments(p.sc, S, true, segsm);
-  const int NW = gridDim.x * kWarps;
-  const int first = blockIdx.x * kWarps + warp;
-  if (first >= total) {
-    griddep_launch();
-    return;
-  }
-  // Producer and consumer walk the same (task, stage) sequence; the producer
-  // issues one stage ahead and looks up its page / token ids one more ahead.
-  int ptask = first, pst = 0, pslot = 0;
-  STask pt;
-  decode_shrink(p, V, ptask, pt);
-  bool pvalid = true;
-  int32_t aux = shrink_lookup(p, pt, 0);
-  auto produce = [&]() {
-    issue_shrink(p, pt, pst, aux, wbuf + pslot * kSlotBytes, &bars[warp][pslot]);
-    pslot ^= 1;
-    if (++pst == pt.nst) {
-      pst = 0;
-      ptask += NW;
-      pvalid = ptask < total;
-      if (pvalid) decode_shrink(p, V, ptask, pt);
+  __syncthreads();
+  if (warp == 0) {
+    // producer
+    SCursor A, B, C;
+    A.task = blockIdx.x;
+    A.st = 0;
+    A.valid = A.task < total;
+    if (A.valid) decode_shrink(p, V, A.task, A.t);
+    B = A;
+    scursor_next(p, V, total, B);
+    C = B;
+    scursor_next(p, V, total, C);
+    int32_t a0, a1, b0, b1;
+    shrink_lookup(p, A, a0, a1);
+    shrink_lookup(p, B, b0, b1);
+    uint32_t eparity = 0;
+    int ring = 0, uses = 0;
+    while (A.valid) {
+      if (uses >= kNS) {
+        if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
+        eparity ^= 1u << ring;
+      }
+      shrink_issue(p, A, a0, a1, smem + ring * kStageBytes, desc[ring], &full[ring]);
+      a0 = b0;
+      a1 = b1;
+      shrink_lookup(p, C, b0, b1);
+      A = B;
+      B = C;
+      scursor_next(p, V, total, C);
+      ring = (ring + 1) % kNS;
+      ++uses;
     }
-    if (pvalid) aux = shrink_lookup(p, pt, pst);
-  };
-  int ctask = first, cst = 0, slot = 0;
-  STask ct = pt;
-  uint32_t parity = 0;
-  float acc[32];
+    // end marker
+    if (uses >= kNS) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
+    if (lane == 0) {
+      desc[ring][kDescInts - 1] = 0;
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[ring])) : "memory");
+    }
+  } else {
+    // consumers
+    float acc[16];
 #pragma unroll
-  for (int q = 0; q < 32; ++q) acc[q] = 0.f;
-  produce();
-  for (;;) {
-    if (pvalid) produce();
-    if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
-    parity ^= 1u << slot;
-    shrink_stage_any<DT>(p, ct, cst, wbuf + slot * kSlotBytes, acc);
-    __syncwarp();
-    fence_proxy_async();
-    slot ^= 1;
-    if (++cst == ct.nst) {
-      cst = 0;
-      ctask += NW;
-      if (ctask >= total) break;
-      decode_shrink(p, V, ctask, ct);
+    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+    uint32_t fparity = 0;
+    int ring = 0;
+    for (;;) {
+      if (!mbar_wait(&full[ring], (fparity >> ring) & 1, p.pool.err)) break;
+      fparity ^= 1u << ring;
+      if (desc[ring][kDescInts - 1] == 0) break;
+      STask t;
+      int32_t* dst = reinterpret_cast<int32_t*>(&t);
+#pragma unroll
+      for (int q = 0; q < (int)(sizeof(STask) / 4); ++q) dst[q] = desc[ring][q];
+      const int st = desc[ring][kDescInts - 2];
+      const unsigned char* buf = smem + ring * kStageBytes;
+      if (DT == SLORA_BF16) {
+        switch (t.nt) {
+          case 1: shrink_consume<SLORA_BF16, 1>(p, t, st, buf, acc); break;
+          case 2: shrink_consume<SLORA_BF16, 2>(p, t, st, buf, acc); break;
+          case 4: shrink_consume<SLORA_BF16, 4>(p, t, st, buf, acc); break;
+          default: shrink_consume<SLORA_BF16, 8>(p, t, st, buf, acc); break;
+        }
+      } else {
+        switch (t.nt) {
+          case 1: shrink_consume<SLORA_F16, 1>(p, t, st, buf, acc); break;
+          case 2: shrink_consume<SLORA_F16, 2>(p, t, st, buf, acc); break;
+          case 4: shrink_consume<SLORA_F16, 4>(p, t, st, buf, acc); break;
+          default: shrink_consume<SLORA_F16, 8>(p, t, st, buf, acc); break;
+        }
+      }
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
+      ring = (ring + 1) % kNS;
     }
   }
   griddep_launch();
 }
 
 // ---------------------------------------------------------------------------
-// Expand.  Task = (projection slot k, segment, NTE tokens, kLC outputs),
-// streamed in stages of kExpandRows rank rows.  Slot layout of a stage:
-// B row i at i * 512 B; t partials of token t at kExpT + t * 8 * t_ns * 4 B;
-// y row t (last stage) at kExpY + t * 512 B; t sums at kExpS.
-constexpr int kExpT = kExpandRows * 2 * kLC;
-constexpr int kExpY = 4 * 1024;
-constexpr int kExpS = kExpY + 4 * 2 * kLC;
-static_assert(kExpS + 4 * kExpandRows * 4 <= kSlotBytes, "expand slot overflow");
+// Expand task = (projection slot k, segment, NTE tokens, kELC outputs); stages
+// of kER rank rows.  Stage layout: B row i at i * 4 KiB; the t partials of
+// token t at kEXT + t * kER * t_ns * 4 B.  Consumer warp w owns outputs
+// [256 w, 256 w + 256) of the task; it loads its y slice when the task starts.
+constexpr int kEXT = kER * 2 * kELC;
+static_assert(kEXT + 4 * kER * 32 * 4 <= kStageBytes, "expand stage overflow");
 
 struct ETask {
-  int k, a, r, seg0, n, nt, tg, lc, nst, ntok;
+  int k, a, r, seg0, n, nt, tg, lc, nst, ntok, tok0, tok1, tok2, tok3;
 };
+static_assert(sizeof(ETask) / 4 + 2 <= kDescInts, "descriptor too small");
 
 __device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView& V, int task, ETask& t) {
   const int s = find_seg(V.prefix, V.S, task);
@@ -642,80 +675,118 @@ __device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView
   const int n_tg = cdiv_i(t.n, t.nt);
   int k = 0;
   for (; k < p.n_slots - 1; ++k) {  // the projection owning local task q
-    const int cnt = n_tg * cdiv_i(p.slot[k].d_out, kLC);
+    const int cnt = n_tg * cdiv_i(p.slot[k].d_out, kELC);
     if (q < cnt) break;
     q -= cnt;
   }
   t.k = k;
   t.tg = q % n_tg;
   t.lc = q / n_tg;
-  t.nst = cdiv_i(t.r, kExpandRows);
+  t.nst = cdiv_i(t.r, kER);
   t.ntok = min(t.nt, t.n - t.tg * t.nt);
+  t.tok0 = t.tok1 = t.tok2 = t.tok3 = 0;
 }
 
-// Lane roles in an expand stage: lanes 0-7 copy piece 0 of B rows 0-7,
-// lanes 8-15 piece 1; lanes 16-19 the t partials of tokens 0-3; lanes 20-23
-// the y rows (last stage).  The lookup (page id / token id) is done a stage ahead.
-__device__ __forceinline__ int32_t expand_lookup(const BgmvParams& p, const ETask& t, int st) {
+struct ECursor {
+  ETask t;
+  int task, st;
+  bool valid;
+};
+
+__device__ __forceinline__ void ecursor_next(const BgmvParams& p, const SegView& V, int total, ECursor& c) {
+  if (!c.valid) return;
+  if (++c.st < c.t.nst) return;
+  c.st = 0;
+  c.task += gridDim.x;
+  c.valid = c.task < total;
+  if (c.valid) decode_expand(p, V, c.task, c.t);
+}
+
+// Per-lane lookups of an expand stage: lane l < kER * kMaxPieces copies piece
+// l % kMaxPieces of row l / kMaxPieces (aux0 = page id); lane l < ntok holds
+// token l (aux1).
+__device__ __forceinline__ void expand_lookup(const BgmvParams& p, const ECursor& c, int32_t& aux0,
+                                              int32_t& aux1) {
   const int lane = threadIdx.x & 31;
+  aux0 = -1;
+  aux1 = -1;
+  if (!c.valid) return;
+  const ETask& t = c.t;
   const SlotDev& L = p.slot[t.k];
-  const int l0 = t.lc * kLC;
-  const int Lo = min(kLC, L.d_out - l0);
-  const int r0 = st * kExpandRows;
-  const int nrows = min(kExpandRows, t.r - r0);
-  if (lane < 16) {
-    const int i = lane & 7;
-    if (i >= nrows) return -1;
-    return piece_page(p.pool, t.a, L.listB, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 3);
+  const int l0 = t.lc * kELC;
+  const int Lo = min(kELC, L.d_out - l0);
+  const int r0 = c.st * kER;
+  const int i = lane / kMaxPieces, q = lane % kMaxPieces;
+  if (lane < kER * kMaxPieces && r0 + i < t.r) {
+    const int64_t f0 = (int64_t)(r0 + i) * L.d_out + l0;
+    int64_t b, e;
+    if (piece_range(p.pool, f0, f0 + Lo, q, b, e)) aux0 = page_id(p.pool, t.a, L.listB, b);
   }
-  const int tt = (lane - 16) & 3;
-  if (lane < 24 && tt < t.ntok) return __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + tt);
-  return -1;
+  if (lane < t.ntok) aux1 = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
 }
 
-__device__ __forceinline__ void issue_expand(const BgmvParams& p, const ETask& t, int st, int32_t aux,
-                                             unsigned char* buf, uint64_t* bar) {
+__device__ __forceinline__ void expand_issue(const BgmvParams& p, const ECursor& c, int32_t aux0, int32_t aux1,
+                                             unsigned char* buf, int32_t* desc, uint64_t* bar) {
   const int lane = threadIdx.x & 31;
+  const ETask& t = c.t;
   const SlotDev& L = p.slot[t.k];
-  const int l0 = t.lc * kLC;
-  const int Lo = min(kLC, L.d_out - l0);
-  const int r0 = st * kExpandRows;
-  const int nrows = min(kExpandRows, t.r - r0);
-  const bool last = st == t.nst - 1;
-  const uint32_t tbytes = 4u * kExpandRows * L.t_ns;
-  if (lane == 0) mbar_expect_tx(bar, 2u * Lo * (nrows + (last ? t.ntok : 0)) + tbytes * t.ntok);
+  const int l0 = t.lc * kELC;
+  const int Lo = min(kELC, L.d_out - l0);
+  const int r0 = c.st * kER;
+  const int nrows = min(kER, t.r - r0);
+  const uint32_t tbytes = 4u * kER * L.t_ns;
+  const int tk0 = __shfl_sync(FULL_MASK, aux1, 0), tk1 = __shfl_sync(FULL_MASK, aux1, 1);
+  const int tk2 = __shfl_sync(FULL_MASK, aux1, 2), tk3 = __shfl_sync(FULL_MASK, aux1, 3);
+  if (lane == 0) {
+    ETask u = t;
+    u.tok0 = tk0;
+    u.tok1 = tk1;
+    u.tok2 = tk2;
+    u.tok3 = tk3;
+    const int32_t* src = reinterpret_cast<const int32_t*>(&u);
+    for (int q = 0; q < (int)(sizeof(ETask) / 4); ++q) desc[q] = src[q];
+    desc[kDescInts - 2] = c.st;
+    desc[kDescInts - 1] = 1;
+    mbar_expect_tx(bar, 2u * Lo * nrows + tbytes * t.ntok);
+  }
   __syncwarp();
-  if (lane < 16) {
-    const int i = lane & 7;
-    if (i < nrows)
-      piece_copy(p.pool, aux, (int64_t)(r0 + i) * L.d_out + l0, Lo, lane >> 3, buf + i * 2 * kLC, bar);
-  } else if (lane < 20) {
-    const int tt = lane - 16;
-    if (tt < t.ntok) {
-      const int64_t row = L.t_by_token ? (int64_t)aux : (int64_t)(t.seg0 + t.tg * t.nt + tt);
-      bulk_g2s(buf + kExpT + tt * tbytes, L.t + row * L.t_rs + (int64_t)r0 * L.t_ns, tbytes, bar);
-    }
-  } else if (lane < 24 && last) {
-    const int tt = lane - 20;
-    if (tt < t.ntok) bulk_g2s(buf + kExpY + tt * 2 * kLC, L.y + (int64_t)aux * L.ldy + l0, 2u * Lo, bar);
+  if (aux0 >= 0) {
+    const int i = lane / kMaxPieces, q = lane % kMaxPieces;
+    const int64_t f0 = (int64_t)(r0 + i) * L.d_out + l0;
+    int64_t b, e;
+    piece_range(p.pool, f0, f0 + Lo, q, b, e);
+    bulk_g2s(buf + i * 2 * kELC + 2 * (b - f0), page_ptr(p.pool, aux0, b), (uint32_t)(2 * (e - b)), bar);
+  }
+  if (lane < t.ntok) {
+    const int64_t row = L.t_by_token ? (int64_t)aux1 : (int64_t)(t.seg0 + t.tg * t.nt + lane);
+    bulk_g2s(buf + kEXT + lane * tbytes, L.t + row * L.t_rs + (int64_t)r0 * L.t_ns, tbytes, bar);
   }
 }
 
 template <int DT>
-__device__ __forceinline__ void expand_stage(const BgmvParams& p, const ETask& t, int st, unsigned char* buf,
-                                             float (&acc)[4][8], int32_t ctok) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask& t, int st,
+                                               const unsigned char* buf, float (&acc)[4][8], uint4 (&yv)[4]) {
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 1;
   const SlotDev& L = p.slot[t.k];
-  const int l0 = t.lc * kLC;
-  const int Lo = min(kLC, L.d_out - l0);
-  const int r0 = st * kExpandRows;
-  const int nrows = min(kExpandRows, t.r - r0);
-  // t for this stage: lane (tt, kk) sums the t_ns partials, in order
-  float* tsum = reinterpret_cast<float*>(buf + kExpS);
+  const int l0 = t.lc * kELC;
+  const int Lo = min(kELC, L.d_out - l0);
+  const int l = cw * 256 + lane * 8;
+  const bool act = l < Lo;
+  const int tokv[4] = {t.tok0, t.tok1, t.tok2, t.tok3};
+  if (st == 0) {  // this warp's y slice, needed at the task's last stage
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt)
+      yv[tt] = (act && tt < t.ntok) ? *reinterpret_cast<const uint4*>(L.y + (int64_t)tokv[tt] * L.ldy + l0 + l)
+                                    : make_uint4(0, 0, 0, 0);
+  }
+  const int r0 = st * kER;
+  const int nrows = min(kER, t.r - r0);
+  // t of (token tt, row kk) summed over the t_ns partials by lane 4 tt + kk
+  float tsum = 0.f;
   {
-    const int tt = lane >> 3, kk = lane & 7;
+    const int tt = lane >> 2, kk = lane & 3;
     if (tt < t.ntok && kk < nrows) {
-      const float* src = reinterpret_cast<const float*>(buf + kExpT + tt * 4 * kExpandRows * L.t_ns) + kk * L.t_ns;
+      const float* src = reinterpret_cast<const float*>(buf + kEXT + tt * 4 * kER * L.t_ns) + kk * L.t_ns;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // four chains; fixed association
       int c = 0;
       for (; c + 4 <= L.t_ns; c += 4) {
@@ -725,41 +796,35 @@ __device__ __forceinline__ void expand_stage(const BgmvParams& p, const ETask& t
         s3 += src[c + 3];
       }
       for (; c < L.t_ns; ++c) s0 += src[c];
-      tsum[tt * kExpandRows + kk] = (s0 + s1) + (s2 + s3);
+      tsum = (s0 + s1) + (s2 + s3);
     }
   }
-  __syncwarp();
-  const int l = lane * 8;
-  const bool act = l < Lo;
-  if (act) {
 #pragma unroll
-    for (int kk = 0; kk < kExpandRows; ++kk) {
-      if (kk >= nrows) break;
-      float bf[8];
-      unpack8<DT>(lds128(buf + kk * 2 * kLC + 2 * l), bf);
+  for (int kk = 0; kk < kER; ++kk) {
+    if (kk >= nrows) break;
+    float bf[8];
+    if (act) unpack8<DT>(lds128(buf + kk * 2 * kELC + 2 * l), bf);
 #pragma unroll
-      for (int tt = 0; tt < 4; ++tt) {
-        if (tt >= t.ntok) break;
-        const float tv = tsum[tt * kExpandRows + kk];
+    for (int tt = 0; tt < 4; ++tt) {
+      const float tv = __shfl_sync(FULL_MASK, tsum, 4 * tt + kk);
+      if (act && tt < t.ntok)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tv, bf[e], acc[tt][e]);
-      }
     }
   }
   if (st != t.nst - 1) return;
   const float s_a = __ldg(p.pool.scale + t.a);
 #pragma unroll
   for (int tt = 0; tt < 4; ++tt) {
-    const int token = __shfl_sync(FULL_MASK, ctok, tt);
     if (act && tt < t.ntok) {
       float yf[8];
-      unpack8<DT>(lds128(buf + kExpY + tt * 2 * kLC + 2 * l), yf);
+      unpack8<DT>(yv[tt], yf);
       uint4 o;
       o.x = pack2<DT>(fmaf(s_a, acc[tt][0], yf[0]), fmaf(s_a, acc[tt][1], yf[1]));
       o.y = pack2<DT>(fmaf(s_a, acc[tt][2], yf[2]), fmaf(s_a, acc[tt][3], yf[3]));
       o.z = pack2<DT>(fmaf(s_a, acc[tt][4], yf[4]), fmaf(s_a, acc[tt][5], yf[5]));
       o.w = pack2<DT>(fmaf(s_a, acc[tt][6], yf[6]), fmaf(s_a, acc[tt][7], yf[7]));
-      *reinterpret_cast<uint4*>(L.y + (int64_t)token * L.ldy + l0 + l) = o;
+      *reinterpret_cast<uint4*>(L.y + (int64_t)tokv[tt] * L.ldy + l0 + l) = o;
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
@@ -767,68 +832,82 @@ __device__ __forceinline__ void expand_stage(const BgmvParams& p, const ETask& t
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kWarps * 32, 1) k_expand(const __grid_constant__ BgmvParams p) {
+__global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constant__ BgmvParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t bars[kWarps][kSlots];
+  __shared__ __align__(8) uint64_t full[kNS], empty[kNS];
+  __shared__ int32_t desc[kNS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  unsigned char* wbuf = smem + warp * kSlots * kSlotBytes;
-  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kSmemBytes);
-  if (lane == 0)
-    for (int s = 0; s < kSlots; ++s) mbar_init(&bars[warp][s], 1);
-  fence_mbar_init();
+  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kRingBytes);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCW);
+    }
+    fence_mbar_init();
+  }
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaExpandTotal];
   const SegView V = stage_segments(p.sc, S, false, segsm);
-  const int NW = gridDim.x * kWarps;
-  const int first = blockIdx.x * kWarps + warp;
-  if (first >= total) {
-    griddep_launch();
-    return;
-  }
-  int ptask = first, pst = 0, pslot = 0;
-  ETask pt;
-  decode_expand(p, V, ptask, pt);
-  bool pvalid = true;
-  int32_t aux = expand_lookup(p, pt, 0);
-  auto produce = [&]() {
-    issue_expand(p, pt, pst, aux, wbuf + pslot * kSlotBytes, &bars[warp][pslot]);
-    pslot ^= 1;
-    if (++pst == pt.nst) {
-      pst = 0;
-      ptask += NW;
-      pvalid = ptask < total;
-      if (pvalid) decode_expand(p, V, ptask, pt);
+  __syncthreads();
+  if (warp == 0) {
+    ECursor A, B, C;
+    A.task = blockIdx.x;
+    A.st = 0;
+    A.valid = A.task < total;
+    if (A.valid) decode_expand(p, V, A.task, A.t);
+    B = A;
+    ecursor_next(p, V, total, B);
+    C = B;
+    ecursor_next(p, V, total, C);
+    int32_t a0, a1, b0, b1;
+    expand_lookup(p, A, a0, a1);
+    expand_lookup(p, B, b0, b1);
+    uint32_t eparity = 0;
+    int ring = 0, uses = 0;
+    while (A.valid) {
+      if (uses >= kNS) {
+        if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
+        eparity ^= 1u << ring;
+      }
+      expand_issue(p, A, a0, a1, smem + ring * kStageBytes, desc[ring], &full[ring]);
+      a0 = b0;
+      a1 = b1;
+      expand_lookup(p, C, b0, b1);
+      A = B;
+      B = C;
+      ecursor_next(p, V, total, C);
+      ring = (ring + 1) % kNS;
+      ++uses;
     }
-    if (pvalid) aux = expand_lookup(p, pt, pst);
-  };
-  int ctask = first, cst = 0, slot = 0;
-  ETask ct = pt;
-  auto ctoken = [&]() {  // token ids of the consumer's task, lane tt holds token tt
-    return lane < ct.ntok ? __ldg(p.sc.perm + ct.seg0 + ct.tg * ct.nt + lane) : 0;
-  };
-  int32_t ctok = ctoken();
-  uint32_t parity = 0;
-  float acc[4][8];
+    if (uses >= kNS) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
+    if (lane == 0) {
+      desc[ring][kDescInts - 1] = 0;
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[ring])) : "memory");
+    }
+  } else {
+    float acc[4][8];
 #pragma unroll
-  for (int tt = 0; tt < 4; ++tt)
+    for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
-  produce();
-  for (;;) {
-    if (pvalid) produce();
-    if (!mbar_wait(&bars[warp][slot], (parity >> slot) & 1, p.pool.err)) break;
-    parity ^= 1u << slot;
-    expand_stage<DT>(p, ct, cst, wbuf + slot * kSlotBytes, acc, ctok);
-    __syncwarp();
-    fence_proxy_async();
-    slot ^= 1;
-    if (++cst == ct.nst) {
-      cst = 0;
-      ctask += NW;
-      if (ctask >= total) break;
-      decode_expand(p, V, ctask, ct);
-      ctok = ctoken();
+      for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
+    uint4 yv[4];
+    uint32_t fparity = 0;
+    int ring = 0;
+    for (;;) {
+      if (!mbar_wait(&full[ring], (fparity >> ring) & 1, p.pool.err)) break;
+      fparity ^= 1u << ring;
+      if (desc[ring][kDescInts - 1] == 0) break;
+      ETask t;
+      int32_t* dst = reinterpret_cast<int32_t*>(&t);
+#pragma unroll
+      for (int q = 0; q < (int)(sizeof(ETask) / 4); ++q) dst[q] = desc[ring][q];
+      const int st = desc[ring][kDescInts - 2];
+      expand_consume<DT>(p, t, st, smem + ring * kStageBytes, acc, yv);
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
+      ring = (ring + 1) % kNS;
     }
   }
   griddep_launch();
@@ -982,7 +1061,7 @@ __global__ void k_gather_debug(PoolDev P, int id, int d, int list_off, int rank,
 
 // ---------------------------------------------------------------------------
 // Launchers.
-constexpr int kDynSmem = kSmemBytes + 4 * kSegSmemInts;  // slots + segment table
+constexpr int kDynSmem = kRingBytes + 4 * kSegSmemInts;  // ring + segment table
 template <typename Kern>
 static cudaError_t launch_dependent(Kern kernel, int grid, int block, size_t smem, cudaStream_t s,
                                     const BgmvParams& p) {
@@ -1019,14 +1098,14 @@ cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cuda
 
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
   set_attrs();
-  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kWarps * 32, kDynSmem, s, p);
-  return launch_dependent(k_shrink<SLORA_F16>, grid, kWarps * 32, kDynSmem, s, p);
+  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kPipeThreads, kDynSmem, s, p);
+  return launch_dependent(k_shrink<SLORA_F16>, grid, kPipeThreads, kDynSmem, s, p);
 }
 
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
   set_attrs();
-  if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kWarps * 32, kDynSmem, s, p);
-  return launch_dependent(k_expand<SLORA_F16>, grid, kWarps * 32, kDynSmem, s, p);
+  if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kPipeThreads, kDynSmem, s, p);
+  return launch_dependent(k_expand<SLORA_F16>, grid, kPipeThreads, kDynSmem, s, p);
 }
 
 cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s) {
@@ -1070,8 +1149,8 @@ cudaError_t launch_gather_debug(const PoolDev& pool, int id, int d, int list_off
 int occupancy_blocks(int which) {
   set_attrs();
   int n = 0;
-  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kWarps * 32, kDynSmem);
-  else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kWarps * 32, kDynSmem);
+  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kPipeThreads, kDynSmem);
+  else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kPipeThreads, kDynSmem);
   return n > 0 ? n : 1;
 }
 

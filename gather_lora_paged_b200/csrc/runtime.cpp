@@ -229,7 +229,7 @@ slora_status_t validate_desc(const slora_pool_desc* d, std::string* why) {
   if (d->max_adapters < 1 || d->max_adapters > 16384) return bad("max_adapters out of [1, 16384]");
   if (d->max_rank < 0 || d->max_rank > 128) return bad("max_rank out of [0, 128]");
   if (d->max_tokens < 1 || d->max_tokens > (1 << 20)) return bad("max_tokens out of [1, 2^20]");
-  if (d->page_elems < 64 || (d->page_elems & (d->page_elems - 1))) return bad("page_elems must be a power of two >= 64");
+  if (d->page_elems < 512 || (d->page_elems & (d->page_elems - 1))) return bad("page_elems must be a power of two >= 512");
   if (d->n_pages < 0 || d->n_pages > (int64_t)INT32_MAX) return bad("n_pages out of range");
   if (d->pagein_mode != SLORA_PAGEIN_KERNEL && d->pagein_mode != SLORA_PAGEIN_MEMCPY)
     return bad("pagein_mode");

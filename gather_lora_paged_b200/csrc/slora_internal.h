@@ -12,8 +12,8 @@ namespace slora {
 // Shrink work split (decode path).  A shrink task covers RW rank rows x NT
 // tokens x kShrinkKT elements of d_in, streamed in stages of kStageK; its
 // fp32 partial (one per kShrinkKT slice of d_in) is summed by the expand.
-constexpr int kShrinkKT = 1024;
-constexpr int kStageK = 256;
+constexpr int kShrinkKT = 2048;
+constexpr int kStageK = 512;
 constexpr int kMaxSlots = SLORA_MAX_PROJ;   // projections per call
 constexpr int kThreads = 256;               // threads per CTA of the decode kernels
 constexpr int kEventRing = 64;

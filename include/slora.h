@@ -103,7 +103,7 @@ typedef struct {
   int32_t max_rank;         /* ranks in [0, max_rank], max_rank <= 128               */
   int32_t max_tokens;       /* largest T of any compute call (<= 1<<20)              */
   int32_t pagein_mode;      /* slora_pagein_mode_t                                   */
-  int64_t page_elems;       /* elements per page: a power of two, >= 64              */
+  int64_t page_elems;       /* elements per page: a power of two, >= 512             */
   int64_t n_pages;          /* pages in dev_pool                                     */
   void* dev_pool;           /* n_pages * page_elems elements, 16-byte aligned        */
   void* dev_tables;         /* slora_tables_bytes(desc) bytes, 256-byte aligned      */
