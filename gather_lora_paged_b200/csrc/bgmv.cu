@@ -44,7 +44,8 @@ __host__ __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1
 __host__ __device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
 __host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
 constexpr int kCW = 8;                        // consumer warps per CTA
-constexpr int kPipeThreads = (kCW + 1) * 32;  // + the producer warp
+constexpr int kProd = 2;                      // producer warps (alternate ring stages)
+constexpr int kPipeThreads = (kCW + kProd) * 32;
 constexpr int kNS = 8;                        // ring stages
 constexpr int kStageBytes = 24 * 1024;
 constexpr int kRingBytes = kNS * kStageBytes;
@@ -78,10 +79,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(1000000u)
         : "memory");
     if (done) return true;
     if (clock64() - t0 > kWaitLimit) {
@@ -501,7 +502,7 @@ __device__ __forceinline__ void shrink_issue(const BgmvParams& p, const SCursor&
 template <int DT, int NT>
 __device__ __forceinline__ void shrink_consume(const BgmvParams& p, const STask& t, int st,
                                                const unsigned char* buf, float (&acc)[16]) {
-  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 1;
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kProd;
   const GroupDev& G = p.group[t.g];
   const int k0 = t.split * kShrinkKT + st * kStageK;
   const int L = min(kStageK, G.d_in - k0);
@@ -573,24 +574,26 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
   const int total = p.sc.meta[kMetaShrinkTotal];
   const SegView V = stage_segments(p.sc, S, true, segsm);
   __syncthreads();
-  if (warp == 0) {
-    // producer
+  if (warp < kProd) {
+    // producer `warp` issues the stages at positions warp, warp + kProd, ...
+    // of the CTA's (task, stage) sequence, into ring slots of the same parity
     SCursor A, B, C;
     A.task = blockIdx.x;
     A.st = 0;
     A.valid = A.task < total;
     if (A.valid) decode_shrink(p, V, A.task, A.t);
+    for (int q = 0; q < warp; ++q) scursor_next(p, V, total, A);
     B = A;
-    scursor_next(p, V, total, B);
+    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, B);
     C = B;
-    scursor_next(p, V, total, C);
+    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, C);
     int32_t a0, a1, b0, b1;
     shrink_lookup(p, A, a0, a1);
     shrink_lookup(p, B, b0, b1);
     uint32_t eparity = 0;
-    int ring = 0, uses = 0;
+    int ring = warp, uses = 0;
     while (A.valid) {
-      if (uses >= kNS) {
+      if (uses >= kNS / kProd) {
         if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
         eparity ^= 1u << ring;
       }
@@ -600,12 +603,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
       shrink_lookup(p, C, b0, b1);
       A = B;
       B = C;
-      scursor_next(p, V, total, C);
-      ring = (ring + 1) % kNS;
+      for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, C);
+      ring = (ring + kProd) % kNS;
       ++uses;
     }
-    // end marker
-    if (uses >= kNS) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
+    // end marker at this producer's next position (the consumers stop at the
+    // first one in sequence order)
+    if (uses >= kNS / kProd) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
     if (lane == 0) {
       desc[ring][kDescInts - 1] = 0;
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[ring])) : "memory");
@@ -766,7 +770,7 @@ __device__ __forceinline__ void expand_issue(const BgmvParams& p, const ECursor&
 template <int DT>
 __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask& t, int st,
                                                const unsigned char* buf, float (&acc)[4][8], uint4 (&yv)[4]) {
-  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - 1;
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kProd;
   const SlotDev& L = p.slot[t.k];
   const int l0 = t.lc * kELC;
   const int Lo = min(kELC, L.d_out - l0);
@@ -850,23 +854,26 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
   const int total = p.sc.meta[kMetaExpandTotal];
   const SegView V = stage_segments(p.sc, S, false, segsm);
   __syncthreads();
-  if (warp == 0) {
+  if (warp < kProd) {
+    // producer `warp` issues the stages at positions warp, warp + kProd, ...
+    // of the CTA's (task, stage) sequence, into ring slots of the same parity
     ECursor A, B, C;
     A.task = blockIdx.x;
     A.st = 0;
     A.valid = A.task < total;
     if (A.valid) decode_expand(p, V, A.task, A.t);
+    for (int q = 0; q < warp; ++q) ecursor_next(p, V, total, A);
     B = A;
-    ecursor_next(p, V, total, B);
+    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, B);
     C = B;
-    ecursor_next(p, V, total, C);
+    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, C);
     int32_t a0, a1, b0, b1;
     expand_lookup(p, A, a0, a1);
     expand_lookup(p, B, b0, b1);
     uint32_t eparity = 0;
-    int ring = 0, uses = 0;
+    int ring = warp, uses = 0;
     while (A.valid) {
-      if (uses >= kNS) {
+      if (uses >= kNS / kProd) {
         if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
         eparity ^= 1u << ring;
       }
@@ -876,11 +883,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
       expand_lookup(p, C, b0, b1);
       A = B;
       B = C;
-      ecursor_next(p, V, total, C);
-      ring = (ring + 1) % kNS;
+      for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, C);
+      ring = (ring + kProd) % kNS;
       ++uses;
     }
-    if (uses >= kNS) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
+    // end marker at this producer's next position (the consumers stop at the
+    // first one in sequence order)
+    if (uses >= kNS / kProd) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
     if (lane == 0) {
       desc[ring][kDescInts - 1] = 0;
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[ring])) : "memory");
