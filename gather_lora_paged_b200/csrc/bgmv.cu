@@ -112,7 +112,16 @@ __device__ __forceinline__ uint4 lds128(const unsigned char* p) {
   return *reinterpret_cast<const uint4*>(p);
 }
 
-// 16-bit -> fp32 for 8 packed elements.
+// 16-bit -> fp32 for 8 packed elements, exact for finite values.  fp16 goes
+// through the integer pipe (exponent/mantissa moved into fp32 position, then
+// an exact multiply by 2^112 rebiases the exponent, subnormals included)
+// instead of the conversion unit; bf16 is the upper half of an fp32.
+__device__ __forceinline__ float h2f_lo(uint32_t w) {
+  return __uint_as_float(((w & 0x7fffu) << 13) | ((w & 0x8000u) << 16)) * 0x1p112f;
+}
+__device__ __forceinline__ float h2f_hi(uint32_t w) {
+  return __uint_as_float(((w >> 3) & 0x0fffe000u) | (w & 0x80000000u)) * 0x1p112f;
+}
 template <int DT>
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -122,14 +131,29 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
       f[2 * i] = __uint_as_float(w[i] << 16);
       f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     } else {
-      __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
-      float2 g = __half22float2(h);
-      f[2 * i] = g.x;
-      f[2 * i + 1] = g.y;
+      f[2 * i] = h2f_lo(w[i]);
+      f[2 * i + 1] = h2f_hi(w[i]);
     }
   }
 }
 
+// acc + a.lo * b.lo + a.hi * b.hi for two packed 16-bit pairs, with the
+// mixed-precision FMA (16-bit sources, fp32 accumulator, one rounding each):
+// the same result as converting exactly and using fp32 FMAs, in order.
+template <int DT>
+__device__ __forceinline__ float fma2_16(uint32_t a, uint32_t b, float acc) {
+  if (DT == SLORA_BF16)
+    asm("{.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;}"
+        : "+f"(acc) : "r"(a), "r"(b));
+  else
+    asm("{.reg .f16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %0;\n\tfma.rn.f32.f16 %0, ah, bh, %0;}"
+        : "+f"(acc) : "r"(a), "r"(b));
+  return acc;
+}
 template <int DT>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   if (DT == SLORA_BF16) {
@@ -513,23 +537,21 @@ __device__ __forceinline__ void shrink_consume(const BgmvParams& p, const STask&
     for (int h = 0; h < kStageK / 256; ++h) {
       const int e = h * 256 + lane * 8;
       if (e >= L) break;
-      float a0[8], a1[8];
-      unpack8<DT>(lds128(buf + i0 * 2 * kStageK + 2 * e), a0);
-      if (r1) unpack8<DT>(lds128(buf + (i0 + 1) * 2 * kStageK + 2 * e), a1);
-      else
-#pragma unroll
-        for (int q = 0; q < 8; ++q) a1[q] = 0.f;
+      const uint4 a0 = lds128(buf + i0 * 2 * kStageK + 2 * e);
+      const uint4 a1 = r1 ? lds128(buf + (i0 + 1) * 2 * kStageK + 2 * e) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int tt = 0; tt < NT; ++tt) {
         if (tt >= t.ntok) break;
-        float xf[8];
-        unpack8<DT>(lds128(buf + (kRB + tt) * 2 * kStageK + 2 * e), xf);
+        const uint4 xv = lds128(buf + (kRB + tt) * 2 * kStageK + 2 * e);
         float s0 = acc[tt], s1 = acc[NT + tt];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          s0 = fmaf(a0[q], xf[q], s0);
-          s1 = fmaf(a1[q], xf[q], s1);
-        }
+        s0 = fma2_16<DT>(a0.x, xv.x, s0);
+        s1 = fma2_16<DT>(a1.x, xv.x, s1);
+        s0 = fma2_16<DT>(a0.y, xv.y, s0);
+        s1 = fma2_16<DT>(a1.y, xv.y, s1);
+        s0 = fma2_16<DT>(a0.z, xv.z, s0);
+        s1 = fma2_16<DT>(a1.z, xv.z, s1);
+        s0 = fma2_16<DT>(a0.w, xv.w, s0);
+        s1 = fma2_16<DT>(a1.w, xv.w, s1);
         acc[tt] = s0;
         acc[NT + tt] = s1;
       }
