@@ -72,10 +72,12 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 // Bounded wait on an mbarrier phase; false (and a recorded error) if it gives up.
+// try_wait suspends the thread for up to the hint; the clock is read only
+// every 64 attempts.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
   const uint32_t a = smem_u32(bar);
-  const long long t0 = clock64();
-  for (;;) {
+  long long t0 = -1;
+  for (uint32_t it = 0;; ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -85,12 +87,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
         : "r"(a), "r"(parity), "r"(1000000u)
         : "memory");
     if (done) return true;
-    if (clock64() - t0 > kWaitLimit) {
-      record_error(err, 4, (int)blockIdx.x);
-      return false;
+    if ((it & 63) == 0) {
+      const long long now = clock64();
+      if (t0 < 0) t0 = now;
+      else if (now - t0 > kWaitLimit) {
+        record_error(err, 4, (int)blockIdx.x);
+        return false;
+      }
     }
   }
 }
+
 // Bulk async copy global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -112,15 +119,14 @@ __device__ __forceinline__ uint4 lds128(const unsigned char* p) {
   return *reinterpret_cast<const uint4*>(p);
 }
 
-// 16-bit -> fp32 for 8 packed elements, exact for finite values.  fp16 goes
-// through the integer pipe (exponent/mantissa moved into fp32 position, then
-// an exact multiply by 2^112 rebiases the exponent, subnormals included)
-// instead of the conversion unit; bf16 is the upper half of an fp32.
-__device__ __forceinline__ float h2f_lo(uint32_t w) {
-  return __uint_as_float(((w & 0x7fffu) << 13) | ((w & 0x8000u) << 16)) * 0x1p112f;
-}
-__device__ __forceinline__ float h2f_hi(uint32_t w) {
-  return __uint_as_float(((w >> 3) & 0x0fffe000u) | (w & 0x80000000u)) * 0x1p112f;
+// 16-bit -> fp32 for 8 packed elements, exact.  fp16 is widened by the
+// mixed-precision FMA x * 1 + (-0) on the FMA pipe (the conversion unit is the
+// scarce one on this part); bf16 is the upper half of an fp32.
+__device__ __forceinline__ void h2x2f(uint32_t w, float& lo, float& hi) {
+  asm("{.reg .f16 l, h, one;\n\t"
+      "mov.b32 {l, h}, %2;\n\tmov.b16 one, 0x3C00;\n\t"
+      "fma.rn.f32.f16 %0, l, one, 0f80000000;\n\tfma.rn.f32.f16 %1, h, one, 0f80000000;}"
+      : "=f"(lo), "=f"(hi) : "r"(w));
 }
 template <int DT>
 __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
@@ -131,8 +137,7 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
       f[2 * i] = __uint_as_float(w[i] << 16);
       f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
     } else {
-      f[2 * i] = h2f_lo(w[i]);
-      f[2 * i + 1] = h2f_hi(w[i]);
+      h2x2f(w[i], f[2 * i], f[2 * i + 1]);
     }
   }
 }
@@ -789,7 +794,7 @@ __device__ __forceinline__ void expand_issue(const BgmvParams& p, const ECursor&
   }
 }
 
-template <int DT>
+template <int DT, int NT>
 __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask& t, int st,
                                                const unsigned char* buf, float (&acc)[4][8], uint4 (&yv)[4]) {
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kProd;
@@ -801,7 +806,7 @@ __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask&
   const int tokv[4] = {t.tok0, t.tok1, t.tok2, t.tok3};
   if (st == 0) {  // this warp's y slice, needed at the task's last stage
 #pragma unroll
-    for (int tt = 0; tt < 4; ++tt)
+    for (int tt = 0; tt < NT; ++tt)
       yv[tt] = (act && tt < t.ntok) ? *reinterpret_cast<const uint4*>(L.y + (int64_t)tokv[tt] * L.ldy + l0 + l)
                                     : make_uint4(0, 0, 0, 0);
   }
@@ -825,23 +830,27 @@ __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask&
       tsum = (s0 + s1) + (s2 + s3);
     }
   }
+  float tv[NT][kER];  // broadcast by every lane, before the lane-dependent part
 #pragma unroll
-  for (int kk = 0; kk < kER; ++kk) {
-    if (kk >= nrows) break;
-    float bf[8];
-    if (act) unpack8<DT>(lds128(buf + kk * 2 * kELC + 2 * l), bf);
+  for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-      const float tv = __shfl_sync(FULL_MASK, tsum, 4 * tt + kk);
-      if (act && tt < t.ntok)
+    for (int kk = 0; kk < kER; ++kk) tv[tt][kk] = __shfl_sync(FULL_MASK, tsum, 4 * tt + kk);
+  if (act) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tv, bf[e], acc[tt][e]);
+    for (int kk = 0; kk < kER; ++kk) {
+      if (kk >= nrows) break;
+      float bf[8];
+      unpack8<DT>(lds128(buf + kk * 2 * kELC + 2 * l), bf);
+#pragma unroll
+      for (int tt = 0; tt < NT; ++tt)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[tt][e] = fmaf(tv[tt][kk], bf[e], acc[tt][e]);
     }
   }
   if (st != t.nst - 1) return;
   const float s_a = __ldg(p.pool.scale + t.a);
 #pragma unroll
-  for (int tt = 0; tt < 4; ++tt) {
+  for (int tt = 0; tt < NT; ++tt) {
     if (act && tt < t.ntok) {
       float yf[8];
       unpack8<DT>(yv[tt], yf);
@@ -934,7 +943,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
 #pragma unroll
       for (int q = 0; q < (int)(sizeof(ETask) / 4); ++q) dst[q] = desc[ring][q];
       const int st = desc[ring][kDescInts - 2];
-      expand_consume<DT>(p, t, st, smem + ring * kStageBytes, acc, yv);
+      const unsigned char* buf = smem + ring * kStageBytes;
+      switch (t.nt) {
+        case 1: expand_consume<DT, 1>(p, t, st, buf, acc, yv); break;
+        case 2: expand_consume<DT, 2>(p, t, st, buf, acc, yv); break;
+        default: expand_consume<DT, 4>(p, t, st, buf, acc, yv); break;
+      }
       __syncwarp();
       if (lane == 0)
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
