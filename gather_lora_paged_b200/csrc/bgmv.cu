@@ -44,7 +44,7 @@ __host__ __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1
 __host__ __device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
 __host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
 constexpr int kCW = 8;                        // consumer warps per CTA
-constexpr int kProd = 2;                      // producer warps (alternate ring stages)
+constexpr int kProd = 4;                      // producer warps (interleaved ring stages)
 constexpr int kPipeThreads = (kCW + kProd) * 32;
 constexpr int kNS = 8;                        // ring stages
 constexpr int kStageBytes = 24 * 1024;
