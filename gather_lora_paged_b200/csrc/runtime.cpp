@@ -26,7 +26,8 @@ using namespace slora;
 
 namespace slora {
 cudaError_t launch_sgmv(const BgmvParams& p, int dtype, const int32_t* seg_start,
-                        const int32_t* seg_adapter, int S, int T, int sm_count, cudaStream_t s);
+                        const int32_t* seg_adapter, int S, int T, int sm_count, cudaStream_t s,
+                        void* scratch, int max_tokens, int64_t n_pages, cudaEvent_t const* ev, int n_ev);
 size_t sgmv_scratch_bytes(const slora_pool_desc& d);
 }  // namespace slora
 
@@ -959,7 +960,10 @@ slora_status_t slora_sgmv(slora_pool* P, int32_t n, const int32_t* projs, const 
   if (s) return s;
   if (S == 0 || T == 0) return SLORA_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_sgmv(bp, P->d.dtype, seg_start, seg_adapter, S, T, P->sm_count, st);
+  if (S > P->d.max_tokens) return P->fail(SLORA_ERR_INVALID_ARG, "more segments than max_tokens");
+  cudaError_t e = launch_sgmv(bp, P->d.dtype, seg_start, seg_adapter, S, T, P->sm_count, st,
+                              P->scratch() + P->sl.off_sgmv, P->d.max_tokens, P->d.n_pages, P->phase_ev,
+                              P->n_phase);
   if (e == cudaErrorNotSupported) return P->fail(SLORA_ERR_UNSUPPORTED, "SGMV shape not supported");
   CUDA_TRY(P, e);
   record_epoch(P, st);

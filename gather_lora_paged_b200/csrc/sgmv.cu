@@ -1,13 +1,740 @@
-// sgmv.cu -- SGMV prefill path (placeholder until the tensor-core kernels land).
+// sgmv.cu -- SGMV prefill path on the 5th-generation tensor cores (sm_100a).
+//
+// Prefill segments are contiguous token ranges that share one adapter
+// ("Multi-LoRA serving: S-LoRA, Punica, SGMV, vLLM", SGMV section: segments of
+// tokens per adapter, dispatched to the Tensor Cores; FAQ: ranks padded into
+// uniform bands to keep tensor-core alignment).  Per segment the delta is two
+// small GEMMs:
+//   shrink  t[128 x R] = X[128 x d_in] . A_t^T      (R = projections x rank)
+//   expand  y[128 x 256] += s * t[128 x r] . B[r x 256]
+// with fp32 accumulators in tensor memory (TMEM).
+//
+// Operands in shared memory use the 128-byte-swizzled canonical layouts:
+//   * X tiles come from an ordinary tiled TMA load (box 64 x 128);
+//   * adapter rows live in scattered pages.  The pool is viewed as a 2-D
+//     tensor of 64-element rows, and TMA tile::gather4 fetches four such rows
+//     (any four pool rows) per instruction, so page-scattered A rows (K-major)
+//     and B rows (MN-major atoms of 8 ranks x 64 outputs) land directly in
+//     the swizzled layout the MMA reads;
+//   * t enters the expand as two 16-bit halves, t = hi + lo with hi = RN(t),
+//     lo = RN(t - hi); both products with B are exact in fp32, so the
+//     intermediate keeps about twice the 16-bit precision.
+// All mbarrier waits are bounded and record an error instead of hanging.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
 #include "slora_internal.h"
 
 namespace slora {
 
-size_t sgmv_scratch_bytes(const slora_pool_desc&) { return 0; }
+namespace {
 
-cudaError_t launch_sgmv(const BgmvParams&, int, const int32_t*, const int32_t*, int, int, int,
-                        cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kBM = 128;             // tokens per tile (MMA M)
+constexpr int kBK = 64;              // K per stage (one 128-byte swizzle atom)
+constexpr int kXTileBytes = kBM * kBK * 2;
+constexpr int kShrinkThreads = 192;  // producer, MMA, 4 epilogue warps
+constexpr int kExpandThreads = 256;
+constexpr int kEN = 256;             // expand outputs per tile (MMA N)
+constexpr long long kWaitLimitS = 2000000000ll;
+
+struct SgmvPlan {      // scratch arrays of one call
+  int32_t* seg_start;  // [S + 1] copy
+  int32_t* seg_adapter;
+  int32_t* seg_rank;   // 0 when the segment is skipped
+  int32_t* shrink_prefix;  // [S + 1]
+  int32_t* expand_prefix;  // [S + 1]
+  int32_t* meta;           // [0] shrink items, [1] expand items
+};
+
+struct SgmvParams {
+  CUtensorMap xmap[kMaxSlots];  // per group: X as (d_in, T) with 64 x 128 boxes
+  CUtensorMap poolmap;          // the pool as (64, rows) with 64 x 1 boxes (gather4)
+  PoolDev pool;
+  int n_groups;
+  GroupDev group[kMaxSlots];
+  int n_slots;
+  SlotDev slot[kMaxSlots];
+  SgmvPlan plan;
+  const int32_t* user_seg_start;
+  const int32_t* user_seg_adapter;
+  int S, T;
+  float* t;             // t of slot k: t + k * t_slot_stride, rows of t_ld floats
+  int64_t t_slot_stride;
+  int t_ld;
+  int64_t pool_rows;    // rows of 64 elements in the pool (out-of-range coordinate)
+  int ntot_max;         // max over groups of round_up(n * max_rank, 16)
+  int stages;           // shrink pipeline depth
+  int dtype;
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers (tcgen05, TMA, mbarrier)
+__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ void bar_init(uint64_t* b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ void bar_expect(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void rec_err(int32_t* err, int code, int info) {
+  if (atomicCAS(&err[0], 0, code) == 0) atomicExch(&err[1], info);
+}
+__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, int32_t* err) {
+  const uint32_t a = su32(b);
+  long long t0 = -1;
+  for (uint32_t it = 0;; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity), "r"(1000000u)
+        : "memory");
+    if (done) return true;
+    if ((it & 63) == 0) {
+      const long long now = clock64();
+      if (t0 < 0) t0 = now;
+      else if (now - t0 > kWaitLimitS) {
+        rec_err(err, 5, (int)blockIdx.x);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_tile_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* b) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          su32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(su32(b))
+      : "memory");
+}
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int r0, int r1, int r2, int r3,
+                                            uint64_t* b) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(su32(dst)),
+      "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(su32(b))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(slot)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* b) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void gd_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void gd_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle.  K-major: rows of 128 B,
+// 8-row atoms 1 KiB apart (SBO).  MN-major: atoms of 8 K-rows x 64 MN
+// elements; lbo = byte distance between MN-adjacent atoms, sbo = between
+// K-adjacent atom rows.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, M = 128.
+__device__ __forceinline__ uint32_t idesc_f16(int dtype, int n, int b_mn_major) {
+  const uint32_t fmt = dtype == SLORA_BF16 ? 1u : 0u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(kBM >> 4) << 24);
+}
+
+__device__ __forceinline__ int find_ge(const int32_t* prefix, int S, int q) {  // largest s, prefix[s] <= q
+  int lo = 0, hi = S - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= q) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int cdiv_d(int a, int b) { return (a + b - 1) / b; }
+
+// Pool row (64 elements) holding flat element f of tensor (adapter a, list offset lo).
+__device__ __forceinline__ int pool_row(const PoolDev& P, int a, int lo, int64_t f) {
+  const int32_t pg = __ldg(P.page_list + (int64_t)a * P.list_stride + lo + (f >> P.page_shift));
+  return (int)((((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1))) >> 6);
+}
+
+// ---------------------------------------------------------------------------
+// Plan: validate segments, per-segment tile counts, prefix sums (one CTA).
+__global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ SgmvParams p) {
+  __shared__ int sh[32];
+  gd_launch();
+  const int S = p.S, tid = threadIdx.x, nth = blockDim.x;
+  const int E = (S + nth - 1) / nth;
+  const int s0 = min(tid * E, S), s1 = min(s0 + E, S);
+  int csh = 0, cex = 0;
+  for (int s = s0; s < s1; ++s) {
+    const int a = p.user_seg_adapter[s];
+    const int b0 = p.user_seg_start[s], b1 = p.user_seg_start[s + 1];
+    const int n = b1 - b0;
+    int r = 0;
+    if (b0 < 0 || b1 > p.T || n < 0) rec_err(p.pool.err, 6, s);  // segment outside [0, T)
+    else if (a >= 0) {
+      if (a >= p.pool.max_adapters) rec_err(p.pool.err, 1, s);
+      else if (p.pool.rank[a] < 0) rec_err(p.pool.err, 2, s);
+      else r = p.pool.rank[a];
+    }
+    const int mt = (r > 0 && n > 0) ? cdiv_d(n, kBM) : 0;
+    csh += mt * p.n_groups;
+    int ex = 0;
+    for (int k = 0; k < p.n_slots; ++k) ex += cdiv_d(p.slot[k].d_out, kEN);
+    cex += mt * ex;
+  }
+  // block exclusive scans (two)
+  auto scan = [&](int v, int* total) {
+    const int lane = tid & 31, w = tid >> 5, nw = nth >> 5;
+    int x = v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sh[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      int q = lane < nw ? sh[lane] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, q, o);
+        if (lane >= o) q += y;
+      }
+      sh[lane] = q;
+    }
+    __syncthreads();
+    const int res = (w ? sh[w - 1] : 0) + x - v;
+    *total = sh[nw - 1];
+    __syncthreads();
+    return res;
+  };
+  int tsh, tex;
+  int bsh = scan(csh, &tsh);
+  int bex = scan(cex, &tex);
+  for (int s = s0; s < s1; ++s) {
+    const int a = p.user_seg_adapter[s];
+    const int b0 = p.user_seg_start[s], b1 = p.user_seg_start[s + 1];
+    const int n = b1 - b0;
+    const bool inb = b0 >= 0 && b1 <= p.T && n >= 0;
+    const int r = (inb && a >= 0 && a < p.pool.max_adapters && p.pool.rank[a] > 0) ? p.pool.rank[a] : 0;
+    const int mt = (r > 0 && n > 0) ? cdiv_d(n, kBM) : 0;
+    p.plan.seg_start[s] = inb ? b0 : 0;
+    p.plan.seg_adapter[s] = a;
+    p.plan.seg_rank[s] = mt > 0 ? r : 0;
+    p.plan.shrink_prefix[s] = bsh;
+    p.plan.expand_prefix[s] = bex;
+    bsh += mt * p.n_groups;
+    int ex = 0;
+    for (int k = 0; k < p.n_slots; ++k) ex += cdiv_d(p.slot[k].d_out, kEN);
+    bex += mt * ex;
+  }
+  if (tid == 0) {
+    p.plan.seg_start[S] = min(max(p.user_seg_start[S], 0), p.T);
+    p.plan.shrink_prefix[S] = tsh;
+    p.plan.expand_prefix[S] = tex;
+    p.plan.meta[0] = tsh;
+    p.plan.meta[1] = tex;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Shrink: one CTA per (segment, group, 128-token tile).
+__global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_constant__ SgmvParams p) {
+  extern __shared__ __align__(1024) unsigned char dsm[];
+  __shared__ __align__(8) uint64_t full[8], empty[8], accb;
+  __shared__ uint32_t tmem_slot;
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  gd_wait();
+  const int total = p.plan.meta[0];
+  const int item = blockIdx.x;
+  if (item >= total) {
+    gd_launch();
+    return;
+  }
+  const int S = p.S;
+  const int s = find_ge(p.plan.shrink_prefix, S, item);
+  const int q = item - p.plan.shrink_prefix[s];
+  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_start[s + 1];
+  const int mt = cdiv_d(seg1 - seg0, kBM);
+  const int g = q / mt, m = q % mt;
+  const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
+  const GroupDev& G = p.group[g];
+  const int R = G.n * r;
+  const int NT = (R + 15) & ~15;
+  const int row0 = seg0 + m * kBM;
+  const int KB = G.d_in / kBK;
+  const int ST = p.stages;
+  const int a_bytes = NT * 128;
+  const int stage_bytes = kXTileBytes + ((p.ntot_max * 128 + 1023) & ~1023);
+  uint32_t ncols = 32;
+  while ((int)ncols < NT) ncols <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ST; ++i) {
+      bar_init(&full[i], 1);
+      bar_init(&empty[i], 1);
+    }
+    bar_init(&accb, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(&tmem_slot, ncols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    // producer: X tile by tiled TMA, A rows by gather4 from the pages
+    for (int kb = 0; kb < KB && ok; ++kb) {
+      const int st = kb % ST;
+      if (kb >= ST) ok = bar_wait(&empty[st], ((kb / ST) - 1) & 1, p.pool.err);
+      if (!ok) break;
+      unsigned char* xs = smem + st * stage_bytes;
+      unsigned char* as = xs + kXTileBytes;
+      if (lane == 0) {
+        bar_expect(&full[st], kXTileBytes + a_bytes);
+        tma_tile_2d(xs, &p.xmap[g], kb * kBK, row0, &full[st]);
+      }
+      __syncwarp();
+      for (int j = lane; j < NT / 4; j += 32) {
+        int rr[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int rho = 4 * j + u;
+          if (rho < R) {
+            const int sj = rho / r, k = rho % r;
+            rr[u] = pool_row(p.pool, a, p.slot[G.slot[sj]].listA, (int64_t)k * G.d_in + (int64_t)kb * kBK);
+          } else {
+            rr[u] = (int)p.pool_rows;  // out of range: TMA fills zeros
+          }
+        }
+        tma_gather4(as + 4 * j * 128, &p.poolmap, rr[0], rr[1], rr[2], rr[3], &full[st]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t lbo = 16, sbo = 1024;
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        const int st = kb % ST;
+        ok = bar_wait(&full[st], (kb / ST) & 1, p.pool.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t xs = su32(smem + st * stage_bytes);
+        const uint32_t as = xs + kXTileBytes;
+        for (int c0 = 0; c0 < NT; c0 += 256) {
+          const int nc = min(256, NT - c0);
+          const uint32_t id = idesc_f16(p.dtype, nc, 0);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t da = sdesc(xs + kk * 32, lbo, sbo);
+            const uint64_t db = sdesc(as + c0 * 128 + kk * 32, lbo, sbo);
+            mma_f16(tmem + c0, da, db, id, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&empty[st]);
+      }
+      mma_commit(&accb);
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps 2..5: TMEM lanes 32 * (warp % 4)
+    ok = bar_wait(&accb, 0, p.pool.err);
+    tc_fence_after();
+    const int quarter = warp & 3;
+    const int mrow = quarter * 32 + lane;
+    const int token = row0 + mrow;
+    const bool valid = token < seg1;
+    for (int c = 0; c < NT; c += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + c, v);
+      if (!valid || !ok) continue;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int rho = c + i;
+        if (rho < R) {
+          const int sj = rho / r, k = rho % r;
+          float* tt = p.t + (int64_t)G.slot[sj] * p.t_slot_stride + (int64_t)token * p.t_ld + k;
+          *tt = __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, ncols);
+  gd_launch();
+}
+
+
+// 16-bit <-> fp32 helpers for the expand epilogue (unpack exact; pack RN).
+template <int DT>
+__device__ __forceinline__ void up2(uint32_t w, float& lo, float& hi) {
+  if (DT == SLORA_BF16) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xffff0000u);
+  } else {
+    asm("{.reg .f16 l, h, one;\n\tmov.b32 {l, h}, %2;\n\tmov.b16 one, 0x3C00;\n\t"
+        "fma.rn.f32.f16 %0, l, one, 0f80000000;\n\tfma.rn.f32.f16 %1, h, one, 0f80000000;}"
+        : "=f"(lo), "=f"(hi) : "r"(w));
+  }
+}
+template <int DT>
+__device__ __forceinline__ uint32_t pk2(float lo, float hi) {
+  uint32_t r;
+  if (DT == SLORA_BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// t = hi + lo in 16-bit halves (hi = RN(t), lo = RN(t - hi)).
+template <int DT>
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pk2<DT>(a, b);
+  float ha, hb;
+  up2<DT>(hi, ha, hb);
+  lo = pk2<DT>(a - ha, b - hb);
+}
+
+// ---------------------------------------------------------------------------
+// Expand: one CTA per (segment, projection slot, 128-token tile, 256 outputs).
+template <int DT>
+__global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_constant__ SgmvParams p) {
+  extern __shared__ __align__(1024) unsigned char dsm[];
+  __shared__ __align__(8) uint64_t bar_b, bar_mma;
+  __shared__ uint32_t tmem_slot;
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  gd_wait();
+  const int total = p.plan.meta[1];
+  const int item = blockIdx.x;
+  if (item >= total) {
+    gd_launch();
+    return;
+  }
+  const int S = p.S;
+  const int s = find_ge(p.plan.expand_prefix, S, item);
+  int q = item - p.plan.expand_prefix[s];
+  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_start[s + 1];
+  const int mt = cdiv_d(seg1 - seg0, kBM);
+  int k = 0;
+  for (; k < p.n_slots - 1; ++k) {
+    const int cnt = mt * cdiv_d(p.slot[k].d_out, kEN);
+    if (q < cnt) break;
+    q -= cnt;
+  }
+  const SlotDev& L = p.slot[k];
+  const int nch = cdiv_d(L.d_out, kEN);
+  const int c = q % nch, m = q / nch;
+  const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
+  const int r16 = (r + 15) & ~15;
+  const int row0 = seg0 + m * kBM;
+  const int n0 = c * kEN, Nc = min(kEN, L.d_out - n0);
+  const int a_bytes = ((r16 + 63) / 64) * (kBM * 128);
+  unsigned char* ahi = smem;
+  unsigned char* alo = smem + a_bytes;
+  unsigned char* bt = smem + 2 * a_bytes;
+
+  if (tid == 0) {
+    bar_init(&bar_b, 1);
+    bar_init(&bar_mma, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // B tile: MN-major atoms (8 ranks x 64 outputs), four pool rows per gather4
+  if (warp == 0) {
+    if (lane == 0) bar_expect(&bar_b, (uint32_t)r16 * 512u);
+    __syncwarp();
+    for (int idx = lane; idx < r16; idx += 32) {  // r16 / 4 rank quads x 4 output atoms
+      const int kq = idx >> 2, cn = idx & 3;
+      int rr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kr = 4 * kq + u, col = n0 + cn * 64;
+        rr[u] = (kr < r && col < L.d_out) ? pool_row(p.pool, a, L.listB, (int64_t)kr * L.d_out + col)
+                                          : (int)p.pool_rows;
+      }
+      tma_gather4(bt + ((4 * kq) >> 3) * 4096 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[0], rr[1], rr[2],
+                  rr[3], &bar_b);
+    }
+  }
+  // t tile as hi / lo halves, K-major 128-byte swizzle (rank columns >= r are 0)
+  const int mrow = tid & 127, part = tid >> 7;
+  const int token = row0 + mrow;
+  const bool valid = token < seg1;
+  {
+    const float* trow = p.t + (int64_t)k * p.t_slot_stride + (int64_t)token * p.t_ld;
+    for (int k0 = part * 8; k0 < r16; k0 += 16) {
+      float v[8];
+      if (valid) {
+        const float4 f0 = *reinterpret_cast<const float4*>(trow + k0);
+        const float4 f1 = *reinterpret_cast<const float4*>(trow + k0 + 4);
+        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (k0 + e >= r) v[e] = 0.f;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      uint4 h, l;
+      split2<DT>(v[0], v[1], h.x, l.x);
+      split2<DT>(v[2], v[3], h.y, l.y);
+      split2<DT>(v[4], v[5], h.z, l.z);
+      split2<DT>(v[6], v[7], h.w, l.w);
+      const int off = (k0 >> 6) * (kBM * 128) + (mrow >> 3) * 1024 + (mrow & 7) * 128 +
+                      ((((k0 & 63) >> 3) ^ (mrow & 7)) << 4);
+      *reinterpret_cast<uint4*>(ahi + off) = h;
+      *reinterpret_cast<uint4*>(alo + off) = l;
+    }
+  }
+  // this thread's y row slice (128 outputs), fetched while the MMAs run
+  uint4 yv[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int col = part * 128 + j * 8;
+    yv[j] = (valid && col < Nc) ? *reinterpret_cast<const uint4*>(L.y + (int64_t)token * L.ldy + n0 + col)
+                                : make_uint4(0, 0, 0, 0);
+  }
+  fence_async_smem();  // the t tiles were written by the generic proxy
+  if (warp == 0) tmem_alloc(&tmem_slot, kEN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  bool ok = true;
+  if (tid == 0) {
+    ok = bar_wait(&bar_b, 0, p.pool.err);
+    tc_fence_after();
+    const uint32_t id = idesc_f16(p.dtype, Nc, 1);
+    const uint32_t sh = su32(ahi), sl = su32(alo), sb = su32(bt);
+    for (int j = 0; j < r16 / 16; ++j)
+      mma_f16(tmem, sdesc(sh + (j >> 2) * (kBM * 128) + (j & 3) * 32, 16, 1024), sdesc(sb + 2 * j * 4096, 1024, 4096),
+              id, j > 0 ? 1u : 0u);
+    for (int j = 0; j < r16 / 16; ++j)
+      mma_f16(tmem, sdesc(sl + (j >> 2) * (kBM * 128) + (j & 3) * 32, 16, 1024), sdesc(sb + 2 * j * 4096, 1024, 4096),
+              id, 1u);
+    mma_commit(&bar_mma);
+  }
+  __syncwarp();
+  ok = bar_wait(&bar_mma, 0, p.pool.err) && ok;
+  tc_fence_after();
+  const float s_a = __ldg(p.pool.scale + a);
+  const int quarter = warp & 3;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int col = part * 128 + j * 16;
+    if (col >= Nc) break;  // warp-uniform
+    uint32_t v[16];
+    tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + col, v);
+    if (!valid || !ok) continue;
+    uint32_t o[8];
+    const uint32_t w[8] = {yv[2 * j].x, yv[2 * j].y, yv[2 * j].z, yv[2 * j].w,
+                           yv[2 * j + 1].x, yv[2 * j + 1].y, yv[2 * j + 1].z, yv[2 * j + 1].w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float y0, y1;
+      up2<DT>(w[e], y0, y1);
+      o[e] = pk2<DT>(fmaf(s_a, __uint_as_float(v[2 * e]), y0), fmaf(s_a, __uint_as_float(v[2 * e + 1]), y1));
+    }
+    uint4* dst = reinterpret_cast<uint4*>(L.y + (int64_t)token * L.ldy + n0 + col);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kEN);
+  gd_launch();
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+               uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dtype == SLORA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int round16(int v) { return (v + 15) & ~15; }
+
+template <typename Kern>
+cudaError_t launch_pdl(Kern kernel, int grid, int block, size_t smem, cudaStream_t s, const SgmvParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+}  // namespace
+
+// Scratch of the prefill path inside dev_scratch: segment plan + t for up to
+// kMaxSlots projection slots of max_tokens rows x round16(max_rank) floats.
+size_t sgmv_scratch_bytes(const slora_pool_desc& d) {
+  const size_t T = (size_t)d.max_tokens;
+  const size_t plan = 4 * (5 * (T + 2) + 16);
+  const size_t t = 4 * (size_t)kMaxSlots * T * (size_t)std::max(16, round16(d.max_rank));
+  return ((plan + 255) / 256) * 256 + t + 256;
+}
+
+static SgmvParams g_sgmv;  // host staging of the (large) parameter block
+
+cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_start, const int32_t* seg_adapter,
+                        int S, int T, int sm_count, cudaStream_t st, void* scratch, int max_tokens,
+                        int64_t n_pages, cudaEvent_t const* ev, int n_ev) {
+  (void)sm_count;
+  SgmvParams& p = g_sgmv;
+  memset(&p, 0, sizeof(p));
+  p.pool = bp.pool;
+  p.dtype = dtype;
+  p.S = S;
+  p.T = T;
+  p.user_seg_start = seg_start;
+  p.user_seg_adapter = seg_adapter;
+  p.n_slots = bp.n_slots;
+  for (int k = 0; k < bp.n_slots; ++k) p.slot[k] = bp.slot[k];
+  // groups: slots sharing x, at most 512 / round16(max_rank) per group (TMEM columns)
+  const int r16max = std::max(16, round16(bp.pool.max_rank));
+  const int per_group = std::max(1, 512 / r16max);
+  p.n_groups = 0;
+  for (int g = 0; g < bp.n_groups; ++g) {
+    const GroupDev& G = bp.group[g];
+    for (int i = 0; i < G.n; i += per_group) {
+      GroupDev& H = p.group[p.n_groups++];
+      H = G;
+      H.n = std::min(per_group, G.n - i);
+      for (int j = 0; j < H.n; ++j) H.slot[j] = G.slot[i + j];
+    }
+  }
+  if (p.n_groups > kMaxSlots) return cudaErrorNotSupported;
+  int ntot = 16;
+  for (int g = 0; g < p.n_groups; ++g) ntot = std::max(ntot, round16(p.group[g].n * bp.pool.max_rank));
+  if (ntot > 512) return cudaErrorNotSupported;
+  p.ntot_max = ntot;
+  const int stage_bytes = kXTileBytes + ((ntot * 128 + 1023) & ~1023);
+  p.stages = std::min(8, (200 * 1024) / stage_bytes);
+  if (p.stages < 2) return cudaErrorNotSupported;
+  // tensor maps
+  const int64_t pool_rows = n_pages * ((int64_t)1 << bp.pool.page_shift) / 64;
+  if (pool_rows <= 0 || pool_rows >= INT32_MAX) return cudaErrorNotSupported;
+  p.pool_rows = pool_rows;
+  if (!encode_2d(&p.poolmap, dtype, bp.pool.pool, 64, (uint64_t)pool_rows, 128, 64, 1)) return cudaErrorNotSupported;
+  for (int g = 0; g < p.n_groups; ++g) {
+    const GroupDev& G = p.group[g];
+    if (!encode_2d(&p.xmap[g], dtype, G.x, (uint64_t)G.d_in, (uint64_t)T, (uint64_t)G.ldx * 2, kBK, kBM))
+      return cudaErrorNotSupported;
+  }
+  // scratch: plan arrays then t
+  int32_t* pl = static_cast<int32_t*>(scratch);
+  const int Tm = max_tokens;
+  p.plan.seg_start = pl;
+  p.plan.seg_adapter = pl + (Tm + 2);
+  p.plan.seg_rank = pl + 2 * (Tm + 2);
+  p.plan.shrink_prefix = pl + 3 * (Tm + 2);
+  p.plan.expand_prefix = pl + 4 * (Tm + 2);
+  p.plan.meta = pl + 5 * (Tm + 2);
+  const size_t plan_bytes = ((4 * (5 * ((size_t)Tm + 2) + 16) + 255) / 256) * 256;
+  p.t = reinterpret_cast<float*>(static_cast<char*>(scratch) + plan_bytes);
+  p.t_ld = r16max;
+  p.t_slot_stride = (int64_t)Tm * r16max;
+  if (S > Tm) return cudaErrorNotSupported;
+
+  static bool attrs = false;
+  const size_t shrink_smem = (size_t)p.stages * stage_bytes + 1024;
+  const size_t expand_smem = 2 * (size_t)((r16max + 63) / 64) * (kBM * 128) + (size_t)r16max * 512 + 1024;
+  if (!attrs) {
+    cudaFuncSetAttribute(k_sgmv_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    cudaFuncSetAttribute(k_sgmv_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    cudaFuncSetAttribute(k_sgmv_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    attrs = true;
+  }
+  const int tiles = (T + kBM - 1) / kBM + S;  // upper bound on 128-token tiles over all segments
+  int nchunks = 0;
+  for (int k = 0; k < p.n_slots; ++k) nchunks += (p.slot[k].d_out + kEN - 1) / kEN;
+  // timing hook: n_ev == 2 brackets the call, n_ev >= 4 also splits it per kernel
+  if (n_ev >= 2) cudaEventRecord(ev[0], st);
+  k_sgmv_plan<<<1, 1024, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (n_ev >= 4) cudaEventRecord(ev[1], st);
+  e = launch_pdl(k_sgmv_shrink, p.n_groups * tiles, kShrinkThreads, shrink_smem, st, p);
+  if (e != cudaSuccess) return e;
+  if (n_ev >= 4) cudaEventRecord(ev[2], st);
+  if (dtype == SLORA_BF16) e = launch_pdl(k_sgmv_expand<SLORA_BF16>, nchunks * tiles, kExpandThreads, expand_smem, st, p);
+  else e = launch_pdl(k_sgmv_expand<SLORA_F16>, nchunks * tiles, kExpandThreads, expand_smem, st, p);
+  if (e != cudaSuccess) return e;
+  if (n_ev >= 4) cudaEventRecord(ev[3], st);
+  else if (n_ev == 2) cudaEventRecord(ev[1], st);
+  return cudaSuccess;
 }
 
 }  // namespace slora

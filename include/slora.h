@@ -260,8 +260,11 @@ slora_status_t slora_lora_delta(slora_pool* pool, int32_t n, const int32_t* proj
  * [seg_start[s], seg_start[s+1]) using seg_adapter[s] (-1: skipped).  Same
  * arithmetic as slora_lora_delta; projections as there.  seg_start (S+1) and
  * seg_adapter (S) are device arrays; S and T (= rows of x and y) host ints.
- * Requires a bf16 or fp16 pool and ranks <= 128.  [S2 SGMV on Tensor Cores,
- * rank bands padded for tensor-core alignment]                                 */
+ * Segment bounds and adapters are checked on the device: a segment outside
+ * [0, T) or with a bad or non-resident adapter is skipped and recorded in the
+ * device error word (codes 6, 1, 2; info = segment index).  Segments may not
+ * overlap.  Ranks are padded to a multiple of 16 for the tensor cores.
+ * [S2 SGMV on Tensor Cores, rank bands padded for tensor-core alignment]      */
 slora_status_t slora_sgmv(slora_pool* pool, int32_t n, const int32_t* projs,
                           const void* const* x, const int64_t* ldx, void* const* y,
                           const int64_t* ldy, const int32_t* seg_start,
