@@ -1124,31 +1124,35 @@ static cudaError_t launch_dependent(Kern kernel, int grid, int block, size_t sme
 }
 
 static bool g_attrs_done = false;
-static void set_attrs() {
-  if (g_attrs_done) return;
-  cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-  cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
-  cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
-  cudaFuncSetAttribute(k_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
-  cudaFuncSetAttribute(k_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
-  g_attrs_done = true;
+static cudaError_t set_attrs() {
+  if (g_attrs_done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  if (e == cudaSuccess) g_attrs_done = true;
+  return e;
 }
 
 cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cudaStream_t s) {
-  set_attrs();
+  cudaError_t ea = set_attrs();
+  if (ea != cudaSuccess) return ea;
   const size_t smem = sizeof(int) * (size_t)p.pool.max_adapters;
   k_segments<<<1, 1024, smem, s>>>(p, idx, T);
   return cudaGetLastError();
 }
 
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
-  set_attrs();
+  cudaError_t ea = set_attrs();
+  if (ea != cudaSuccess) return ea;
   if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kPipeThreads, kDynSmem, s, p);
   return launch_dependent(k_shrink<SLORA_F16>, grid, kPipeThreads, kDynSmem, s, p);
 }
 
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
-  set_attrs();
+  cudaError_t ea = set_attrs();
+  if (ea != cudaSuccess) return ea;
   if (dtype == SLORA_BF16) return launch_dependent(k_expand<SLORA_BF16>, grid, kPipeThreads, kDynSmem, s, p);
   return launch_dependent(k_expand<SLORA_F16>, grid, kPipeThreads, kDynSmem, s, p);
 }

@@ -965,7 +965,7 @@ slora_status_t slora_sgmv(slora_pool* P, int32_t n, const int32_t* projs, const 
                               P->scratch() + P->sl.off_sgmv, P->d.max_tokens, P->d.n_pages, P->phase_ev,
                               P->n_phase);
   if (e == cudaErrorNotSupported) return P->fail(SLORA_ERR_UNSUPPORTED, "SGMV shape not supported");
-  CUDA_TRY(P, e);
+  if (e != cudaSuccess) return P->cuda_fail(e, "SGMV launch");
   record_epoch(P, st);
   return SLORA_OK;
 }

@@ -708,15 +708,13 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   p.t_slot_stride = (int64_t)Tm * r16max;
   if (S > Tm) return cudaErrorNotSupported;
 
-  static bool attrs = false;
   const size_t shrink_smem = (size_t)p.stages * stage_bytes + 1024;
   const size_t expand_smem = 2 * (size_t)((r16max + 63) / 64) * (kBM * 128) + (size_t)r16max * 512 + 1024;
-  if (!attrs) {
-    cudaFuncSetAttribute(k_sgmv_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    cudaFuncSetAttribute(k_sgmv_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    cudaFuncSetAttribute(k_sgmv_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    attrs = true;
-  }
+  cudaError_t ea = cudaFuncSetAttribute(k_sgmv_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shrink_smem);
+  if (ea == cudaSuccess)
+    ea = cudaFuncSetAttribute(dtype == SLORA_BF16 ? k_sgmv_expand<SLORA_BF16> : k_sgmv_expand<SLORA_F16>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)expand_smem);
+  if (ea != cudaSuccess) return ea;
   const int tiles = (T + kBM - 1) / kBM + S;  // upper bound on 128-token tiles over all segments
   int nchunks = 0;
   for (int k = 0; k < p.n_slots; ++k) nchunks += (p.slot[k].d_out + kEN - 1) / kEN;
