@@ -130,56 +130,112 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+class DecodeRun:
+    """Decode step: page-in call for the batch's adapter set (LRU touch), then
+    the fused delta (segment build, grouped shrink, grouped expand)."""
+    phases = ("segments", "shrink", "expand")
+
+    def __init__(self, w):
+        import torch
+
+        import gather_lora_paged_b200 as G
+        import harness as H
+        self.G, self.H, self.w = G, H, w
+        self.pb = H.PoolBuild(w)
+        self.ten = H.Tensors(w)
+        self.d_idx = torch.from_numpy(w.idx).cuda()
+        self.touched = w.touched().tolist()
+
+    def set_events(self, evs):
+        self.G.slora_set_phase_events(self.pb.h, evs)
+
+    def step(self, stream, outer=None):
+        G = self.G
+        G.slora_adapter_page_in(self.pb.h, self.touched, stream)
+        if outer:
+            outer[0].record(stream)
+        G.slora_lora_delta(self.pb.h, *self.ten.args(), self.d_idx, self.w.T, stream)
+        if outer:
+            outer[1].record(stream)
+
+    def inputs(self):  # device tensors refreshed from the host in the e2e run
+        return [self.d_idx]
+
+
+class PrefillRun(DecodeRun):
+    """Prefill step: page-in call, request -> segment merge on the device, and
+    the tensor-core SGMV (plan, shrink, expand) over all projections."""
+    phases = ("plan", "shrink", "expand")
+
+    def __init__(self, w):
+        import torch
+        super().__init__(w)
+        n = w.req_adapter.size
+        self.n = n
+        self.d_rs = torch.from_numpy(w.req_start).cuda()
+        self.d_ra = torch.from_numpy(w.req_adapter).cuda()
+        self.ss = torch.zeros(n + 1, dtype=torch.int32, device="cuda")
+        self.sa = torch.zeros(n, dtype=torch.int32, device="cuda")
+        self.S = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step(self, stream, outer=None):
+        G = self.G
+        G.slora_adapter_page_in(self.pb.h, self.touched, stream)
+        if outer:
+            outer[0].record(stream)
+        G.slora_build_sgmv_segments(self.pb.h, self.d_rs, self.d_ra, self.n, self.ss, self.sa,
+                                    self.S, stream)
+        G.slora_sgmv(self.pb.h, *self.ten.args(), self.ss, self.sa, self.n, self.w.T, stream)
+        if outer:
+            outer[1].record(stream)
+
+    def inputs(self):
+        return [self.d_rs, self.d_ra]
+
+
 def run_ours(args, rank, world):
     import torch
 
-    import gather_lora_paged_b200 as G
     import harness as H
 
     dev = int(os.environ.get("LOCAL_RANK", 0))
     torch.cuda.set_device(dev)
     w = W.config(args.config)
-    if args.config in (3, 4):
-        raise SystemExit("bench.py: configs 3 and 4 are measured by their own paths")
-    pb = H.PoolBuild(w)
-    ten = H.Tensors(w)
+    if args.config == 4:
+        raise SystemExit("bench.py: the mixed workload is measured by --config 4 --mixed (not yet)")
+    R = PrefillRun(w) if args.config == 3 else DecodeRun(w)
     stream = torch.cuda.current_stream()
-    d_idx = torch.from_numpy(w.idx).cuda()
-    touched = w.touched().tolist()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    for e in ev:          # torch creates the CUDA event on first record
+    outer = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for e in ev + outer:  # torch creates the CUDA event on first record
         e.record()
     torch.cuda.synchronize()
-    G.slora_set_phase_events(pb.h, ev)
     alg = algorithmic(w)
 
-    def step():
-        G.slora_adapter_page_in(pb.h, touched, stream)
-        G.slora_lora_delta(pb.h, *ten.args(), d_idx, w.T, stream)
-
     def prep():
-        ten.reset()
+        R.ten.reset()
         flush.zero_()
 
     for _ in range(args.warmup):
         prep()
-        step()
+        R.step(stream)
     torch.cuda.synchronize()
-    st, code, info = G.slora_check_device(pb.h)
+    st, code, info = R.G.slora_check_device(R.pb.h)
     assert st == 0, (code, info)
 
-    # pass 1: per-kernel device times (events between the kernels)
-    t_seg = t_shr = t_exp = 0.0
+    # pass 1: per-kernel device times (library events between its kernels)
+    R.set_events(ev)
+    kt = [0.0, 0.0, 0.0]
     for _ in range(args.steps):
         prep()
-        step()
+        R.step(stream)
         ev[3].synchronize()
-        t_seg += ev[0].elapsed_time(ev[1])
-        t_shr += ev[1].elapsed_time(ev[2])
-        t_exp += ev[2].elapsed_time(ev[3])
-    # pass 2 (the timed region): whole-step device time, kernels back to back
-    G.slora_set_phase_events(pb.h, [ev[0], ev[3]])
+        for i in range(3):
+            kt[i] += ev[i].elapsed_time(ev[i + 1])
+    R.set_events([])
+    # pass 2 (the timed region): whole steps, kernels back to back; the L2
+    # flush ahead of each step keeps the GPU busy while the host enqueues it
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -188,9 +244,9 @@ def run_ours(args, rank, world):
     t_step = 0.0
     for _ in range(args.steps):
         prep()
-        step()
-        ev[3].synchronize()
-        t_step += ev[0].elapsed_time(ev[3])
+        R.step(stream, outer)
+        outer[1].synchronize()
+        t_step += outer[0].elapsed_time(outer[1])
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
@@ -203,76 +259,76 @@ def run_ours(args, rank, world):
     value = world * w.T * K / (t_step / 1e3)
 
     # end to end through the C ABI with host buffers (pinned), copies timed
-    e2e = None
-    if True:
-        hx = {n: H.pinned(w.x(n)) for n in w.x_names}
-        hy = [H.pinned(w.y_in(p)) for p in range(len(w.projs))]
-        hout = [torch.empty_like(t).pin_memory() for t in hy]
-        hidx = torch.from_numpy(w.idx).pin_memory()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        G.slora_set_phase_events(pb.h, [])
-        xs = {n: ten.x[n].view(torch.int16) for n in w.x_names}
-        ys = [t.view(torch.int16) for t in ten.y]
+    hx = {n: H.pinned(w.x(n)) for n in w.x_names}
+    hy = [H.pinned(w.y_in(p)) for p in range(len(w.projs))]
+    hout = [torch.empty_like(t).pin_memory() for t in hy]
+    dins = R.inputs()
+    hins = [t.cpu().pin_memory() for t in dins]
+    xs = {n: R.ten.x[n].view(torch.int16) for n in w.x_names}
+    ys = [t.view(torch.int16) for t in R.ten.y]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-        def e2e_step():
-            for n in w.x_names:
-                xs[n].copy_(hx[n], non_blocking=True)
-            for p in range(len(w.projs)):
-                ys[p].copy_(hy[p], non_blocking=True)
-            d_idx.copy_(hidx, non_blocking=True)
-            step()
-            for p in range(len(w.projs)):
-                hout[p].copy_(ys[p], non_blocking=True)
+    def e2e_step():
+        for n in w.x_names:
+            xs[n].copy_(hx[n], non_blocking=True)
+        for p in range(len(w.projs)):
+            ys[p].copy_(hy[p], non_blocking=True)
+        for d, h in zip(dins, hins):
+            d.copy_(h, non_blocking=True)
+        R.step(stream)
+        for p in range(len(w.projs)):
+            hout[p].copy_(ys[p], non_blocking=True)
 
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        tot = 0.0
-        n_e2e = max(10, min(K, 200))
-        for _ in range(n_e2e):
-            flush.zero_()
-            e0.record()
-            e2e_step()
-            e1.record()
-            e1.synchronize()
-            tot += e0.elapsed_time(e1)
-        h2d = sum(t.numel() * 2 for t in hx.values()) + sum(t.numel() * 2 for t in hy) + hidx.numel() * 4
-        d2h = sum(t.numel() * 2 for t in hout)
-        e2e = {"value": world * w.T * n_e2e / (tot / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": tot / n_e2e}
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    tot = 0.0
+    n_e2e = max(10, min(K, 200))
+    for _ in range(n_e2e):
+        flush.zero_()
+        e0.record()
+        e2e_step()
+        e1.record()
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    h2d = sum(t.numel() * 2 for t in hx.values()) + sum(t.numel() * 2 for t in hy) + \
+        sum(t.numel() * t.element_size() for t in hins)
+    d2h = sum(t.numel() * 2 for t in hout)
+    e2e = {"value": world * w.T * n_e2e / (tot / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "ms_per_step": tot / n_e2e}
 
     hbm, tc, src = peaks()
-    t_exp_l = t_exp / K
-    t_shr_l = t_shr / K
-    dom = ("expand", t_exp_l, alg["expand_bytes"]) if t_exp_l >= t_shr_l else \
-        ("shrink", t_shr_l, alg["shrink_bytes"])
-    achieved = dom[2] / (dom[1] / 1e3) / 1e9
+    kt = [t / K for t in kt]
+    names = R.phases
+    i_dom = 1 if kt[1] >= kt[2] else 2
+    dom_bytes = alg["shrink_bytes"] if i_dom == 1 else alg["expand_bytes"]
+    achieved = dom_bytes / (kt[i_dom] / 1e3) / 1e9
     step_gbs = alg["total_bytes"] / (ms / 1e3) / 1e9
+    tflops = alg["flops"] / (ms / 1e3) / 1e12
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": W.DTYPE_NAME[w.dtype],
         "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(d_in)) A, N(0,1/sqrt(r)) B; "
-                "Zipf adapter ids)",
+                "Zipf or uniform adapter ids)",
         "config": {"workload": w.name, "tokens_per_step": w.T, "projections": len(w.projs),
                    "adapters": w.n_adapters, "touched_adapters": alg["touched"],
                    "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": achieved, "peak": hbm,
+        "roofline": {"bound": "hbm", "kernel": names[i_dom], "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
-                     "peak_source": src,
-                     "alg_bytes_per_launch": dom[2]},
+                     "peak_source": src, "alg_bytes_per_launch": dom_bytes},
         "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": step_gbs / hbm, "alg_bytes_per_step": alg["total_bytes"],
                           "flops_per_step": alg["flops"],
-                          "kernel_ms": {"segments": t_seg / K, "shrink": t_shr_l,
-                                        "expand": t_exp_l}},
+                          "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / tc,
+                          "kernel_ms": dict(zip(names, kt))},
         "e2e": e2e,
-        "gpu_launches": 3 * K,  # segment build + shrink + expand per timed step
+        "gpu_launches": (4 if args.config == 3 else 3) * K,
         "clocks": clk,
     }
-    pb.close()
+    R.pb.close()
     return out
 
 

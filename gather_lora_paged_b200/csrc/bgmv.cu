@@ -1013,9 +1013,15 @@ __global__ void __launch_bounds__(1024) k_merge_requests(const int32_t* __restri
     }
     prev = q;
   }
+  const int end = n > 0 ? req_start[n] : 0;
   if (tid == 0) {
-    seg_start[S] = n > 0 ? req_start[n] : 0;
+    seg_start[S] = end;
     *S_out = S;
+  }
+  // pad to n segments with empty ones, so the arrays can go to slora_sgmv with S = n
+  for (int q = S + tid; q < n; q += nth) {
+    seg_start[q + 1] = end;
+    seg_adapter[q] = -1;
   }
 }
 

@@ -43,7 +43,8 @@ constexpr int kEN = 256;             // expand outputs per tile (MMA N)
 constexpr long long kWaitLimitS = 2000000000ll;
 
 struct SgmvPlan {      // scratch arrays of one call
-  int32_t* seg_start;  // [S + 1] copy
+  int32_t* seg_start;  // [S] first token of each segment (0 when skipped)
+  int32_t* seg_end;    // [S] one past its last token (0 when skipped)
   int32_t* seg_adapter;
   int32_t* seg_rank;   // 0 when the segment is skipped
   int32_t* shrink_prefix;  // [S + 1]
@@ -254,7 +255,8 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
     const bool inb = b0 >= 0 && b1 <= p.T && n >= 0;
     const int r = (inb && a >= 0 && a < p.pool.max_adapters && p.pool.rank[a] > 0) ? p.pool.rank[a] : 0;
     const int mt = (r > 0 && n > 0) ? cdiv_d(n, kBM) : 0;
-    p.plan.seg_start[s] = inb ? b0 : 0;
+    p.plan.seg_start[s] = mt > 0 ? b0 : 0;
+    p.plan.seg_end[s] = mt > 0 ? b1 : 0;
     p.plan.seg_adapter[s] = a;
     p.plan.seg_rank[s] = mt > 0 ? r : 0;
     p.plan.shrink_prefix[s] = bsh;
@@ -265,7 +267,6 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
     bex += mt * ex;
   }
   if (tid == 0) {
-    p.plan.seg_start[S] = min(max(p.user_seg_start[S], 0), p.T);
     p.plan.shrink_prefix[S] = tsh;
     p.plan.expand_prefix[S] = tex;
     p.plan.meta[0] = tsh;
@@ -291,8 +292,13 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   const int S = p.S;
   const int s = find_ge(p.plan.shrink_prefix, S, item);
   const int q = item - p.plan.shrink_prefix[s];
-  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_start[s + 1];
+  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_end[s];
   const int mt = cdiv_d(seg1 - seg0, kBM);
+  if (mt <= 0 || q >= mt * p.n_groups || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
+    if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
+    gd_launch();
+    return;
+  }
   const int g = q / mt, m = q % mt;
   const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
   const GroupDev& G = p.group[g];
@@ -451,13 +457,23 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
   const int S = p.S;
   const int s = find_ge(p.plan.expand_prefix, S, item);
   int q = item - p.plan.expand_prefix[s];
-  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_start[s + 1];
+  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_end[s];
   const int mt = cdiv_d(seg1 - seg0, kBM);
+  if (mt <= 0 || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
+    if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
+    gd_launch();
+    return;
+  }
   int k = 0;
   for (; k < p.n_slots - 1; ++k) {
     const int cnt = mt * cdiv_d(p.slot[k].d_out, kEN);
     if (q < cnt) break;
     q -= cnt;
+  }
+  if (q >= mt * cdiv_d(p.slot[k].d_out, kEN)) {
+    if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
+    gd_launch();
+    return;
   }
   const SlotDev& L = p.slot[k];
   const int nch = cdiv_d(L.d_out, kEN);
@@ -641,7 +657,7 @@ cudaError_t launch_pdl(Kern kernel, int grid, int block, size_t smem, cudaStream
 // kMaxSlots projection slots of max_tokens rows x round16(max_rank) floats.
 size_t sgmv_scratch_bytes(const slora_pool_desc& d) {
   const size_t T = (size_t)d.max_tokens;
-  const size_t plan = 4 * (5 * (T + 2) + 16);
+  const size_t plan = 4 * (6 * (T + 2) + 16);
   const size_t t = 4 * (size_t)kMaxSlots * T * (size_t)std::max(16, round16(d.max_rank));
   return ((plan + 255) / 256) * 256 + t + 256;
 }
@@ -697,12 +713,13 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   int32_t* pl = static_cast<int32_t*>(scratch);
   const int Tm = max_tokens;
   p.plan.seg_start = pl;
-  p.plan.seg_adapter = pl + (Tm + 2);
-  p.plan.seg_rank = pl + 2 * (Tm + 2);
-  p.plan.shrink_prefix = pl + 3 * (Tm + 2);
-  p.plan.expand_prefix = pl + 4 * (Tm + 2);
-  p.plan.meta = pl + 5 * (Tm + 2);
-  const size_t plan_bytes = ((4 * (5 * ((size_t)Tm + 2) + 16) + 255) / 256) * 256;
+  p.plan.seg_end = pl + (Tm + 2);
+  p.plan.seg_adapter = pl + 2 * (Tm + 2);
+  p.plan.seg_rank = pl + 3 * (Tm + 2);
+  p.plan.shrink_prefix = pl + 4 * (Tm + 2);
+  p.plan.expand_prefix = pl + 5 * (Tm + 2);
+  p.plan.meta = pl + 6 * (Tm + 2);
+  const size_t plan_bytes = ((4 * (6 * ((size_t)Tm + 2) + 16) + 255) / 256) * 256;
   p.t = reinterpret_cast<float*>(static_cast<char*>(scratch) + plan_bytes);
   p.t_ld = r16max;
   p.t_slot_stride = (int64_t)Tm * r16max;

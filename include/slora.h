@@ -218,8 +218,10 @@ slora_status_t slora_build_segments(slora_pool* pool, const int32_t* idx, int32_
 /* Prefill segments from requests: request q covers tokens
  * [req_start[q], req_start[q+1]) with adapter req_adapter[q] (-1 = none);
  * neighbouring requests with the same adapter merge into one segment; empty
- * requests are dropped.  All arrays device; seg_start[S+1], seg_adapter[S],
- * *S_out device.                                                              */
+ * requests are dropped.  All arrays device: seg_start has n+1 entries,
+ * seg_adapter n, *S_out one.  Entries after the S-th are filled with empty
+ * segments (adapter -1) so the arrays can be passed to slora_sgmv with S = n
+ * without reading S back to the host.                                         */
 slora_status_t slora_build_sgmv_segments(slora_pool* pool, const int32_t* req_start,
                                          const int32_t* req_adapter, int32_t n,
                                          int32_t* seg_start, int32_t* seg_adapter,
@@ -262,8 +264,8 @@ slora_status_t slora_lora_delta(slora_pool* pool, int32_t n, const int32_t* proj
  * seg_adapter (S) are device arrays; S and T (= rows of x and y) host ints.
  * Segment bounds and adapters are checked on the device: a segment outside
  * [0, T) or with a bad or non-resident adapter is skipped and recorded in the
- * device error word (codes 6, 1, 2; info = segment index).  Segments may not
- * overlap.  Ranks are padded to a multiple of 16 for the tensor cores.
+ * device error word (codes 6, 1, 2; info = segment index; code 7 marks an
+ * inconsistent plan and is never expected).  Segments may not overlap.  Ranks are padded to a multiple of 16 for the tensor cores.
  * [S2 SGMV on Tensor Cores, rank bands padded for tensor-core alignment]      */
 slora_status_t slora_sgmv(slora_pool* pool, int32_t n, const int32_t* projs,
                           const void* const* x, const int64_t* ldx, void* const* y,

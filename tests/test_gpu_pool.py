@@ -145,4 +145,7 @@ def test_merge_requests_bit_exact(seed):
     assert m == len(ref_sa)
     assert np.array_equal(ss.cpu().numpy()[:m + 1], ref_ss)
     assert np.array_equal(sa.cpu().numpy()[:m], ref_sa)
+    # the tail is padded with empty segments (start = end = T, no adapter)
+    assert np.all(ss.cpu().numpy()[m:] == req_start[-1])
+    assert np.all(sa.cpu().numpy()[m:] == -1)
     pb.close()
