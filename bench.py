@@ -52,6 +52,30 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
+# data-parallel replicas: rank k runs workload `config` with its own batch
+# (seeded by k), no collective on the data path; timings are reduced by max.
+def replica_workload(config: int, rank: int) -> W.Workload:
+    return W.config(config, replica=rank)
+
+
+def max_over_ranks(ms: float, world: int, device=None) -> float:
+    """The job's time for a per-rank device time: the max over all ranks."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, tokens_per_step: int, steps: int, t_ms: float) -> float:
+    """Whole-job tokens/s: every rank processed `steps` batches of
+    `tokens_per_step` tokens in (at most) t_ms."""
+    return world * tokens_per_step * steps / (t_ms / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # algorithmic bytes / flops (each touched adapter and each distinct input read
 # once, y read and written once)
 def algorithmic(w: W.Workload, tokens=None):
@@ -200,7 +224,7 @@ def run_ours(args, rank, world):
 
     dev = int(os.environ.get("LOCAL_RANK", 0))
     torch.cuda.set_device(dev)
-    w = W.config(args.config)
+    w = replica_workload(args.config, rank)
     if args.config == 4:
         raise SystemExit("bench.py: the mixed workload is measured by --config 4 --mixed (not yet)")
     R = PrefillRun(w) if args.config == 3 else DecodeRun(w)
@@ -251,12 +275,10 @@ def run_ours(args, rank, world):
     clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
-        t = torch.tensor([t_step], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_step = float(t.item())
+    t_step = max_over_ranks(t_step, world, "cuda")
     K = args.steps
     ms = t_step / K
-    value = world * w.T * K / (t_step / 1e3)
+    value = job_throughput(world, w.T, K, t_step)
 
     # end to end through the C ABI with host buffers (pinned), copies timed
     hx = {n: H.pinned(w.x(n)) for n in w.x_names}
@@ -284,6 +306,8 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     tot = 0.0
     n_e2e = max(10, min(K, 200))
+    if world > 1:
+        torch.distributed.barrier()
     for _ in range(n_e2e):
         flush.zero_()
         e0.record()
@@ -291,10 +315,11 @@ def run_ours(args, rank, world):
         e1.record()
         e1.synchronize()
         tot += e0.elapsed_time(e1)
+    tot = max_over_ranks(tot, world, "cuda")
     h2d = sum(t.numel() * 2 for t in hx.values()) + sum(t.numel() * 2 for t in hy) + \
         sum(t.numel() * t.element_size() for t in hins)
     d2h = sum(t.numel() * 2 for t in hout)
-    e2e = {"value": world * w.T * n_e2e / (tot / 1e3), "unit": UNIT,
+    e2e = {"value": job_throughput(world, w.T, n_e2e, tot), "unit": UNIT,
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
            "ms_per_step": tot / n_e2e}
 

@@ -171,22 +171,19 @@ class Workload:
 # ----------------------------------------------------------------------------
 # The five workloads.  Seeds are 1000 + config index.
 
-def _cfg0(T=8):
-    seed = 1000
+def _cfg0(T=8, seed=1000):
     idx = _rng(seed, _T_IDX).integers(0, 4, size=T).astype(np.int32)
     return Workload(0, "tiny_decode_1proj_d1024_T8_fp16", F16, [Proj("p", 1024, 1024, "x")], T,
                     idx, np.array([8, 8, 16, 16], np.int32), 1024, False, seed, n_decode=T)
 
 
-def _cfg1(T=256, n_adapters=1000):
-    seed = 1001
+def _cfg1(T=256, n_adapters=1000, seed=1001):
     idx = zipf_ids(_rng(seed, _T_IDX), n_adapters, 1.0, T)
     return Workload(1, "llama7b_decode_layer_T256_1000ad_r16_fp16", F16, llama_layer(4096, 11008),
                     T, idx, np.full(n_adapters, 16, np.int32), 8192, False, seed, n_decode=T)
 
 
-def _cfg2(T=512, n_adapters=2000):
-    seed = 1002
+def _cfg2(T=512, n_adapters=2000, seed=1002):
     idx = zipf_ids(_rng(seed, _T_IDX), n_adapters, 1.2, T)
     ranks = _rng(seed, _T_RANK).choice(np.array([8, 16, 32, 64], np.int32), n_adapters)
     return Workload(2, "llama13b_decode_layer_T512_2000ad_r8-64_bf16_shuffled", BF16,
@@ -194,8 +191,7 @@ def _cfg2(T=512, n_adapters=2000):
                     n_decode=T)
 
 
-def _cfg3(n_req=32, n_adapters=64, lo=64, hi=1024):
-    seed = 1003
+def _cfg3(n_req=32, n_adapters=64, lo=64, hi=1024, seed=1003):
     rng = _rng(seed, _T_REQ)
     lens = rng.integers(lo, hi + 1, size=n_req)
     req_ad = rng.integers(0, n_adapters, size=n_req).astype(np.int32)
@@ -208,8 +204,7 @@ def _cfg3(n_req=32, n_adapters=64, lo=64, hi=1024):
                     req_start=req_start, req_adapter=req_ad, n_decode=0)
 
 
-def _cfg4(n_dec=1024, n_req=8, req_len=512, n_adapters=2000):
-    seed = 1004
+def _cfg4(n_dec=1024, n_req=8, req_len=512, n_adapters=2000, seed=1004):
     rng = _rng(seed, _T_IDX)
     dec = zipf_ids(rng, n_adapters, 1.0, n_dec)
     req_ad = zipf_ids(rng, n_adapters, 1.0, n_req)
@@ -225,7 +220,11 @@ def _cfg4(n_dec=1024, n_req=8, req_len=512, n_adapters=2000):
 BUILDERS = {0: _cfg0, 1: _cfg1, 2: _cfg2, 3: _cfg3, 4: _cfg4}
 
 
-def config(i: int, **kw) -> Workload:
+def config(i: int, replica: int = 0, **kw) -> Workload:
+    """Workload i.  Replica k > 0 (one per data-parallel rank) draws its own
+    batch, activations and weights from seed 1000 + i + 10000 k."""
+    if replica:
+        kw["seed"] = 1000 + i + 10000 * int(replica)
     return BUILDERS[i](**kw)
 
 
