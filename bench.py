@@ -23,7 +23,6 @@ from __future__ import annotations
 import argparse
 import json
 import os
-import subprocess
 import sys
 import threading
 import time
@@ -100,57 +99,67 @@ def algorithmic(w: W.Workload, tokens=None):
 
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled every 10 ms through
+    NVML while the timed region runs (read-only queries)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD = 0.01
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap"}
 
     def __init__(self, index: int):
         self.index = index
-        self.lines = []
-        self.p = None
+        self.samples = []
+        self.h = None
+        self.stop_ev = threading.Event()
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(self.index)
+            bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def start(self):
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                       "-lms", "100", "-i", str(self.index)],
-                                      stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            self.nv = pynvml
+            self.h = self._handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         except Exception:
-            self.p = None
+            self.h = None
 
-    def _read(self):
-        for line in self.p.stdout:
-            self.lines.append(line.strip())
+    def _reasons(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(f(self.h))
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)),
+                                     self._reasons()))
+            except Exception:
+                pass
+            self.stop_ev.wait(self.PERIOD)
 
     def stop(self):
-        if self.p is None:
+        if self.h is None:
             return None
-        self.p.terminate()
-        try:
-            self.p.wait(timeout=5)
-        except Exception:
-            self.p.kill()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        self.stop_ev.set()
+        self.t.join(timeout=5)
+        if not self.samples:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = sorted({n for _, m in self.samples for bit, n in self.REASONS.items() if m & bit})
+        return {"sm_mhz": float(np.median([c for c, _ in self.samples])), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 10 ms"}
 
 
 # ---------------------------------------------------------------------------
@@ -226,7 +235,7 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     w = replica_workload(args.config, rank)
     if args.config == 4:
-        raise SystemExit("bench.py: the mixed workload is measured by --config 4 --mixed (not yet)")
+        return run_mixed(args, rank, world, w)
     R = PrefillRun(w) if args.config == 3 else DecodeRun(w)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -358,6 +367,136 @@ def run_ours(args, rank, world):
 
 
 # ---------------------------------------------------------------------------
+def pcie_h2d_peak(nbytes=1 << 30, reps=5):
+    """Measured pinned host -> device copy bandwidth (GB/s), one large copy."""
+    import torch
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    best = 0.0
+    for _ in range(reps):
+        e0.record()
+        d.copy_(h, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        best = max(best, nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    del h, d
+    return best
+
+
+def run_mixed(args, rank, world, w):
+    """The mixed step (decode batch + prefill requests, 30% of the adapters
+    cold): page-in of the cold adapters from pinned host memory on a side
+    stream, then the BGMV and SGMV compute.  Each timed step is preceded,
+    untimed, by the restore of the pool (cold set evicted, fillers back) and
+    an L2 flush."""
+    import torch
+
+    import harness as H
+    mode = {"kernel": H.G.SLORA_PAGEIN_KERNEL, "memcpy": H.G.SLORA_PAGEIN_MEMCPY}[args.pagein]
+    M = H.MixedStep(w, pagein_mode=mode)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    K = min(args.steps, 20)
+    Wm = max(3, min(args.warmup, 5))
+    for _ in range(Wm):
+        M.ten.reset()
+        M.step(stream)
+        M.restore(stream)
+    st, code, info = H.G.slora_check_device(M.h)
+    assert st == 0, (code, info)
+    s0 = H.G.slora_pool_stats(M.h)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", 0)))
+    clocks.start()
+    t_step = t_page = t_comp = 0.0
+    for _ in range(K):
+        M.ten.reset()
+        flush.zero_()
+        M.step(stream, ev[0], ev[1], ev[2])
+        ev[2].synchronize()
+        t_step += ev[0].elapsed_time(ev[2])
+        t_page += ev[0].elapsed_time(ev[1])
+        t_comp += ev[1].elapsed_time(ev[2])
+        M.restore(stream)
+    clk = clocks.stop()
+    s1 = H.G.slora_pool_stats(M.h)
+    paged_steps = (s1["bytes_paged_in"] - s0["bytes_paged_in"]) / K
+    t_step = max_over_ranks(t_step, world, "cuda")
+    ms, ms_page, ms_comp = t_step / K, t_page / K, t_comp / K
+    value = job_throughput(world, w.T, K, t_step)
+
+    # e2e: the same step with x, y and the batch description copied from
+    # pinned host memory and y copied back, all inside the timed region
+    hx = {n: H.pinned(w.x(n)) for n in w.x_names}
+    hy = [H.pinned(w.y_in(p)) for p in range(len(w.projs))]
+    hout = [torch.empty_like(t).pin_memory() for t in hy]
+    dins = [M.d_idx, M.d_rs, M.d_ra]
+    hins = [t.cpu().pin_memory() for t in dins]
+    xs = {n: M.ten.x[n].view(torch.int16) for n in w.x_names}
+    ys = [t.view(torch.int16) for t in M.ten.y]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, min(K, 10))
+    tot = 0.0
+    for _ in range(n_e2e):
+        e0.record(stream)
+        for n in w.x_names:
+            xs[n].copy_(hx[n], non_blocking=True)
+        for p in range(len(w.projs)):
+            ys[p].copy_(hy[p], non_blocking=True)
+        for d, h in zip(dins, hins):
+            d.copy_(h, non_blocking=True)
+        M.step(stream)
+        for p in range(len(w.projs)):
+            hout[p].copy_(ys[p], non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+        M.restore(stream)
+    tot = max_over_ranks(tot, world, "cuda")
+    h2d = sum(t.numel() * 2 for t in hx.values()) + sum(t.numel() * 2 for t in hy) + \
+        sum(t.numel() * t.element_size() for t in hins)
+    d2h = sum(t.numel() * 2 for t in hout)
+
+    peak_pcie = pcie_h2d_peak()
+    hbm, tc, src = peaks()
+    alg = algorithmic(w)
+    comp_gbs = alg["total_bytes"] / (ms_comp / 1e3) / 1e9
+    page_gbs = paged_steps / (ms_page / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": W.DTYPE_NAME[w.dtype],
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(d_in)) A, N(0,1/sqrt(r)) B; "
+                "Zipf adapter ids)",
+        "config": {"workload": w.name, "tokens_per_step": w.T, "decode_tokens": w.n_decode,
+                   "prefill_requests": M.n_req, "projections": len(w.projs),
+                   "adapters": w.n_adapters, "touched_adapters": int(M.U.size),
+                   "cold_adapters": int(M.cold.size), "pool_pages": M.n_pages,
+                   "pagein_mode": args.pagein, "accumulate": "f32",
+                   "l2": "flushed before every step (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "pagein": {"ms": ms_page, "bytes_per_step": int(paged_steps),
+                   "expected_bytes": M.cold_bytes(), "achieved_gbs": page_gbs,
+                   "pcie_h2d_peak_gbs": peak_pcie, "frac": page_gbs / peak_pcie,
+                   "peak_source": "pinned 1 GiB cudaMemcpyAsync, measured in this run"},
+        "roofline": {"bound": "hbm", "kernel": "compute (BGMV decode + SGMV prefill)",
+                     "achieved": comp_gbs, "peak": hbm, "unit": "GB/s", "frac": comp_gbs / hbm,
+                     "traffic": None, "peak_source": src,
+                     "alg_bytes_per_launch": alg["total_bytes"], "compute_ms": ms_comp},
+        "e2e": {"value": job_throughput(world, w.T, n_e2e, tot), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": tot / n_e2e},
+        "gpu_launches": 8 * K,  # page-in gather, segments, shrink, expand, merge, plan, shrink, expand
+        "clocks": clk,
+    }
+    M.close()
+    return out
+
+
+# ---------------------------------------------------------------------------
 def oracle_step(w: W.Workload, tokens, threads):
     import harness as H
     import oracle
@@ -411,6 +550,8 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pagein", default="kernel", choices=["kernel", "memcpy"],
+                    help="page-in mode of the mixed workload (--config 4)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -120,7 +120,12 @@ def _event(e) -> int | None:
         return None
     if isinstance(e, int):
         return e
-    return e.cuda_event
+    h = e.cuda_event
+    if not h:
+        # torch creates the CUDA event on its first record(); passing NULL
+        # would silently drop the completion signal
+        raise ValueError("event has no CUDA handle yet: record it once before passing it")
+    return h
 
 
 def _arr(ctype, vals):

@@ -72,8 +72,8 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 // Bounded wait on an mbarrier phase; false (and a recorded error) if it gives up.
-// try_wait suspends the thread for up to the hint; the clock is read only
-// every 64 attempts.
+// try_wait blocks for a system-dependent time; the clock is read only every
+// 64 attempts.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
   const uint32_t a = smem_u32(bar);
   long long t0 = -1;
@@ -81,10 +81,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(a), "r"(parity), "r"(1000000u)
+        : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
     if ((it & 63) == 0) {

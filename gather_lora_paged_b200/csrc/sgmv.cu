@@ -38,8 +38,10 @@ constexpr int kBM = 128;             // tokens per tile (MMA M)
 constexpr int kBK = 64;              // K per stage (one 128-byte swizzle atom)
 constexpr int kXTileBytes = kBM * kBK * 2;
 constexpr int kShrinkThreads = 192;  // producer, MMA, 4 epilogue warps
-constexpr int kExpandThreads = 256;
-constexpr int kEN = 256;             // expand outputs per tile (MMA N)
+constexpr int kExpandThreads = 192;  // producer, MMA, 4 epilogue warps
+constexpr int kEN = 128;             // expand outputs per item (MMA N)
+constexpr int kAcc = 4;              // expand TMEM accumulators (kAcc x kEN columns)
+constexpr int kYTileBytes = kBM * kEN * 2;
 constexpr long long kWaitLimitS = 2000000000ll;
 
 struct SgmvPlan {      // scratch arrays of one call
@@ -71,6 +73,10 @@ struct SgmvParams {
   int ntot_max;         // max over groups of round_up(n * max_rank, 16)
   int stages;           // shrink pipeline depth
   int dtype;
+  CUtensorMap ymap[kMaxSlots];  // per slot: y as (d_out, T) with 64 x 128 boxes
+  int e_nb, e_ny;       // expand ring depths (B chunks, y tiles)
+  int e_t_half;         // expand: bytes of one t half in shared memory
+  int e_b_stage;        // expand: bytes of one B ring stage
 };
 
 // ---------------------------------------------------------------------------
@@ -92,10 +98,10 @@ __device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, int32_t* 
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(a), "r"(parity), "r"(1000000u)
+        : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
     if ((it & 63) == 0) {
@@ -328,7 +334,34 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   bool ok = true;
 
   if (warp == 0) {
-    // producer: X tile by tiled TMA, A rows by gather4 from the pages
+    // producer: X tile by tiled TMA, A rows by gather4 from the pages.  Lane
+    // j owns rows 4j..4j+3 (+128 per round).  Within a page a row advances one
+    // pool row per stage, so the page table is read only when a row enters a
+    // new page; the next page id is fetched one page ahead.
+    constexpr int kRounds = 4;  // NT <= 512
+    int cur[kRounds][4], left[kRounds][4], nxt[kRounds][4];
+    const int64_t pmask = (1ll << p.pool.page_shift) - 1;
+    const int rows_per_page = (int)((pmask + 1) >> 6);
+#pragma unroll
+    for (int rd = 0; rd < kRounds; ++rd)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int rho = rd * 128 + 4 * lane + u;
+        cur[rd][u] = (int)p.pool_rows;
+        left[rd][u] = 1 << 30;
+        nxt[rd][u] = -1;
+        if (rho < R) {
+          const int sj = rho / r, k = rho % r;
+          const int lo = p.slot[G.slot[sj]].listA;
+          const int64_t f = (int64_t)k * G.d_in;
+          cur[rd][u] = pool_row(p.pool, a, lo, f);
+          left[rd][u] = rows_per_page - (int)((f & pmask) >> 6);
+          const int64_t fn = f + ((int64_t)left[rd][u] << 6);  // first element of the next page
+          nxt[rd][u] = fn < (int64_t)(k + 1) * G.d_in ? __ldg(p.pool.page_list + (int64_t)a * p.pool.list_stride + lo +
+                                                             (fn >> p.pool.page_shift))
+                                                      : -1;
+        }
+      }
     for (int kb = 0; kb < KB && ok; ++kb) {
       const int st = kb % ST;
       if (kb >= ST) ok = bar_wait(&empty[st], ((kb / ST) - 1) & 1, p.pool.err);
@@ -340,19 +373,29 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
         tma_tile_2d(xs, &p.xmap[g], kb * kBK, row0, &full[st]);
       }
       __syncwarp();
-      for (int j = lane; j < NT / 4; j += 32) {
-        int rr[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int rho = 4 * j + u;
-          if (rho < R) {
+      for (int rd = 0; rd < kRounds; ++rd) {
+        if (rd * 128 + 4 * lane < NT)
+          tma_gather4(as + (rd * 128 + 4 * lane) * 128, &p.poolmap, cur[rd][0], cur[rd][1], cur[rd][2], cur[rd][3],
+                      &full[st]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // advance to the next stage's pool row
+          const int rho = rd * 128 + 4 * lane + u;
+          if (rho >= R) continue;
+          if (--left[rd][u] > 0) {
+            ++cur[rd][u];
+          } else if (nxt[rd][u] >= 0) {
             const int sj = rho / r, k = rho % r;
-            rr[u] = pool_row(p.pool, a, p.slot[G.slot[sj]].listA, (int64_t)k * G.d_in + (int64_t)kb * kBK);
-          } else {
-            rr[u] = (int)p.pool_rows;  // out of range: TMA fills zeros
+            const int lo = p.slot[G.slot[sj]].listA;
+            cur[rd][u] = (int)(((int64_t)nxt[rd][u] << p.pool.page_shift) >> 6);
+            left[rd][u] = rows_per_page;
+            const int64_t fstart = (int64_t)k * G.d_in + (int64_t)(kb + 1) * kBK;  // element now loaded
+            const int64_t fn = fstart + ((int64_t)rows_per_page << 6);
+            nxt[rd][u] = fn < (int64_t)(k + 1) * G.d_in ? __ldg(p.pool.page_list + (int64_t)a * p.pool.list_stride +
+                                                               lo + (fn >> p.pool.page_shift))
+                                                        : -1;
           }
         }
-        tma_gather4(as + 4 * j * 128, &p.poolmap, rr[0], rr[1], rr[2], rr[3], &full[st]);
       }
     }
   } else if (warp == 1) {
@@ -422,10 +465,15 @@ __device__ __forceinline__ void up2(uint32_t w, float& lo, float& hi) {
         : "=f"(lo), "=f"(hi) : "r"(w));
   }
 }
+// bf16: round to nearest even on the integer pipe (finite values); fp16: cvt.
+__device__ __forceinline__ uint32_t bf16_rn_bits(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
+}
 template <int DT>
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   uint32_t r;
-  if (DT == SLORA_BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  if (DT == SLORA_BF16) r = bf16_rn_bits(lo) | (bf16_rn_bits(hi) << 16);
   else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
@@ -439,164 +487,326 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 }
 
 // ---------------------------------------------------------------------------
-// Expand: one CTA per (segment, projection slot, 128-token tile, 256 outputs).
+// Expand: persistent CTAs (one per SM) over the item sequence
+//   (segment, 128-token tile m, projection slot k, 128-output chunk c)
+// in that order; CTA b takes the contiguous item range [b N / G, (b+1) N / G).
+// Warp 0 produces: B chunk (r16 ranks x 128 outputs, MN-major atoms, gather4
+// from the pages) into an NB-stage ring and the y tile (128 tokens x 128
+// outputs, two 64 x 128 TMA boxes) into an NY-stage ring.  Warp 1 issues the
+// MMAs into one of kAcc TMEM accumulators of 128 columns.  Warps 2..5 (one
+// token row per thread) convert t to hi/lo halves when a new (tile, slot)
+// unit starts, and drain each accumulator: y <- RN(y + s * acc) in place in
+// shared memory, then 16-byte coalesced stores of the rows inside the segment.
+
+struct ECur {  // a point of the item sequence
+  int s, m, k, c;  // segment, tile, slot, chunk
+  int mt, nch;     // tiles of segment s, chunks of slot k
+  bool valid;
+};
+
+__device__ __forceinline__ int seg_tiles(const SgmvParams& p, int s) {
+  return p.plan.seg_rank[s] > 0 ? cdiv_d(p.plan.seg_end[s] - p.plan.seg_start[s], kBM) : 0;
+}
+
+// First item of the range starting at `item` (< total).
+__device__ __forceinline__ void ecur_init(const SgmvParams& p, int item, ECur& e) {
+  const int s = find_ge(p.plan.expand_prefix, p.S, item);
+  int q = item - p.plan.expand_prefix[s];
+  int tot = 0;
+  for (int k = 0; k < p.n_slots; ++k) tot += cdiv_d(p.slot[k].d_out, kEN);
+  e.s = s;
+  e.mt = seg_tiles(p, s);
+  e.m = q / tot;
+  q -= e.m * tot;
+  int k = 0;
+  for (; k < p.n_slots - 1; ++k) {
+    const int n = cdiv_d(p.slot[k].d_out, kEN);
+    if (q < n) break;
+    q -= n;
+  }
+  e.k = k;
+  e.nch = cdiv_d(p.slot[k].d_out, kEN);
+  e.c = q;
+  e.valid = e.m < e.mt && e.c < e.nch;
+}
+
+// Advances to the next item; returns true when it starts a new (tile, slot) unit.
+__device__ __forceinline__ bool ecur_next(const SgmvParams& p, ECur& e) {
+  if (++e.c < e.nch) return false;
+  e.c = 0;
+  if (++e.k == p.n_slots) {
+    e.k = 0;
+    if (++e.m == e.mt) {
+      e.m = 0;
+      do {
+        ++e.s;
+      } while (e.s < p.S && seg_tiles(p, e.s) == 0);
+      e.valid = e.s < p.S;
+      if (e.valid) e.mt = seg_tiles(p, e.s);
+    }
+  }
+  e.nch = cdiv_d(p.slot[e.k].d_out, kEN);
+  return true;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_constant__ SgmvParams p) {
   extern __shared__ __align__(1024) unsigned char dsm[];
-  __shared__ __align__(8) uint64_t bar_b, bar_mma;
+  __shared__ __align__(8) uint64_t b_full[4], b_empty[4], y_full[4], y_empty[4], a_full[kAcc], a_empty[kAcc];
+  __shared__ __align__(8) uint64_t t_full, fin, e_sync;
   __shared__ uint32_t tmem_slot;
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  gd_wait();
-  const int total = p.plan.meta[1];
-  const int item = blockIdx.x;
-  if (item >= total) {
-    gd_launch();
-    return;
-  }
-  const int S = p.S;
-  const int s = find_ge(p.plan.expand_prefix, S, item);
-  int q = item - p.plan.expand_prefix[s];
-  const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_end[s];
-  const int mt = cdiv_d(seg1 - seg0, kBM);
-  if (mt <= 0 || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
-    if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
-    gd_launch();
-    return;
-  }
-  int k = 0;
-  for (; k < p.n_slots - 1; ++k) {
-    const int cnt = mt * cdiv_d(p.slot[k].d_out, kEN);
-    if (q < cnt) break;
-    q -= cnt;
-  }
-  if (q >= mt * cdiv_d(p.slot[k].d_out, kEN)) {
-    if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
-    gd_launch();
-    return;
-  }
-  const SlotDev& L = p.slot[k];
-  const int nch = cdiv_d(L.d_out, kEN);
-  const int c = q % nch, m = q / nch;
-  const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
-  const int r16 = (r + 15) & ~15;
-  const int row0 = seg0 + m * kBM;
-  const int n0 = c * kEN, Nc = min(kEN, L.d_out - n0);
-  const int a_bytes = ((r16 + 63) / 64) * (kBM * 128);
-  unsigned char* ahi = smem;
-  unsigned char* alo = smem + a_bytes;
-  unsigned char* bt = smem + 2 * a_bytes;
+  const int NB = p.e_nb, NY = p.e_ny;
+  const int t_half = p.e_t_half;   // bytes of one t half (hi or lo)
+  const int b_stage = p.e_b_stage;
+  unsigned char* t_hi = smem;
+  unsigned char* t_lo = smem + t_half;
+  unsigned char* bring = smem + 2 * t_half;
+  unsigned char* yring = bring + NB * b_stage;
 
   if (tid == 0) {
-    bar_init(&bar_b, 1);
-    bar_init(&bar_mma, 1);
+    for (int i = 0; i < NB; ++i) {
+      bar_init(&b_full[i], 1);
+      bar_init(&b_empty[i], 1);
+    }
+    for (int i = 0; i < NY; ++i) {
+      bar_init(&y_full[i], 1);
+      bar_init(&y_empty[i], 4);
+    }
+    for (int i = 0; i < kAcc; ++i) {
+      bar_init(&a_full[i], 1);
+      bar_init(&a_empty[i], 4);
+    }
+    bar_init(&t_full, 4);
+    bar_init(&fin, 1);
+    bar_init(&e_sync, 4);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  __syncthreads();
-  // B tile: MN-major atoms (8 ranks x 64 outputs), four pool rows per gather4
-  if (warp == 0) {
-    if (lane == 0) bar_expect(&bar_b, (uint32_t)r16 * 512u);
-    __syncwarp();
-    for (int idx = lane; idx < r16; idx += 32) {  // r16 / 4 rank quads x 4 output atoms
-      const int kq = idx >> 2, cn = idx & 3;
-      int rr[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kr = 4 * kq + u, col = n0 + cn * 64;
-        rr[u] = (kr < r && col < L.d_out) ? pool_row(p.pool, a, L.listB, (int64_t)kr * L.d_out + col)
-                                          : (int)p.pool_rows;
-      }
-      tma_gather4(bt + ((4 * kq) >> 3) * 4096 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[0], rr[1], rr[2],
-                  rr[3], &bar_b);
-    }
-  }
-  // t tile as hi / lo halves, K-major 128-byte swizzle (rank columns >= r are 0)
-  const int mrow = tid & 127, part = tid >> 7;
-  const int token = row0 + mrow;
-  const bool valid = token < seg1;
-  {
-    const float* trow = p.t + (int64_t)k * p.t_slot_stride + (int64_t)token * p.t_ld;
-    for (int k0 = part * 8; k0 < r16; k0 += 16) {
-      float v[8];
-      if (valid) {
-        const float4 f0 = *reinterpret_cast<const float4*>(trow + k0);
-        const float4 f1 = *reinterpret_cast<const float4*>(trow + k0 + 4);
-        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
-        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (k0 + e >= r) v[e] = 0.f;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      }
-      uint4 h, l;
-      split2<DT>(v[0], v[1], h.x, l.x);
-      split2<DT>(v[2], v[3], h.y, l.y);
-      split2<DT>(v[4], v[5], h.z, l.z);
-      split2<DT>(v[6], v[7], h.w, l.w);
-      const int off = (k0 >> 6) * (kBM * 128) + (mrow >> 3) * 1024 + (mrow & 7) * 128 +
-                      ((((k0 & 63) >> 3) ^ (mrow & 7)) << 4);
-      *reinterpret_cast<uint4*>(ahi + off) = h;
-      *reinterpret_cast<uint4*>(alo + off) = l;
-    }
-  }
-  // this thread's y row slice (128 outputs), fetched while the MMAs run
-  uint4 yv[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int col = part * 128 + j * 8;
-    yv[j] = (valid && col < Nc) ? *reinterpret_cast<const uint4*>(L.y + (int64_t)token * L.ldy + n0 + col)
-                                : make_uint4(0, 0, 0, 0);
-  }
-  fence_async_smem();  // the t tiles were written by the generic proxy
-  if (warp == 0) tmem_alloc(&tmem_slot, kEN);
+  if (warp == 1) tmem_alloc(&tmem_slot, kAcc * kEN);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  gd_wait();
+  const int total = p.plan.meta[1];
+  const int G = gridDim.x;
+  const int i0 = (int)(((int64_t)blockIdx.x * total) / G);
+  const int i1 = (int)(((int64_t)(blockIdx.x + 1) * total) / G);
+  const int n_items = i1 - i0;
   bool ok = true;
-  if (tid == 0) {
-    ok = bar_wait(&bar_b, 0, p.pool.err);
-    tc_fence_after();
-    const uint32_t id = idesc_f16(p.dtype, Nc, 1);
-    const uint32_t sh = su32(ahi), sl = su32(alo), sb = su32(bt);
-    for (int j = 0; j < r16 / 16; ++j)
-      mma_f16(tmem, sdesc(sh + (j >> 2) * (kBM * 128) + (j & 3) * 32, 16, 1024), sdesc(sb + 2 * j * 4096, 1024, 4096),
-              id, j > 0 ? 1u : 0u);
-    for (int j = 0; j < r16 / 16; ++j)
-      mma_f16(tmem, sdesc(sl + (j >> 2) * (kBM * 128) + (j & 3) * 32, 16, 1024), sdesc(sb + 2 * j * 4096, 1024, 4096),
-              id, 1u);
-    mma_commit(&bar_mma);
-  }
-  __syncwarp();
-  ok = bar_wait(&bar_mma, 0, p.pool.err) && ok;
-  tc_fence_after();
-  const float s_a = __ldg(p.pool.scale + a);
-  const int quarter = warp & 3;
+
+  if (n_items > 0 && warp == 0) {
+    // ---------------- producer
+    ECur e;
+    ecur_init(p, i0, e);
+    int issued = 0;
+    for (int j = 0; j < n_items && ok; ++j) {
+      if (!e.valid) {
+        if (lane == 0) rec_err(p.pool.err, 7, i0 + j);
+        ok = false;
+        break;
+      }
+      const SlotDev& L = p.slot[e.k];
+      const int a = p.plan.seg_adapter[e.s], r = p.plan.seg_rank[e.s];
+      const int r16 = (r + 15) & ~15;
+      const int n0 = e.c * kEN;
+      const int row0 = p.plan.seg_start[e.s] + e.m * kBM;
+      // pool rows of this lane's gathers (issued before the waits: latency overlap)
+      int rr[2][4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int col = part * 128 + j * 16;
-    if (col >= Nc) break;  // warp-uniform
-    uint32_t v[16];
-    tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + col, v);
-    if (!valid || !ok) continue;
-    uint32_t o[8];
-    const uint32_t w[8] = {yv[2 * j].x, yv[2 * j].y, yv[2 * j].z, yv[2 * j].w,
-                           yv[2 * j + 1].x, yv[2 * j + 1].y, yv[2 * j + 1].z, yv[2 * j + 1].w};
+      for (int i = 0; i < 2; ++i) {
+        const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float y0, y1;
-      up2<DT>(w[e], y0, y1);
-      o[e] = pk2<DT>(fmaf(s_a, __uint_as_float(v[2 * e]), y0), fmaf(s_a, __uint_as_float(v[2 * e + 1]), y1));
+        for (int u = 0; u < 4; ++u) {
+          const int kr = 4 * kq + u, col = n0 + cn * 64;
+          rr[i][u] = (g < r16 / 2 && kr < r && col < L.d_out)
+                         ? pool_row(p.pool, a, L.listB, (int64_t)kr * L.d_out + col)
+                         : (int)p.pool_rows;
+        }
+      }
+      const int bs = j % NB, ys = j % NY;
+      if (j >= NB) ok = bar_wait(&b_empty[bs], ((j / NB) - 1) & 1, p.pool.err);
+      if (ok && j >= NY) ok = bar_wait(&y_empty[ys], ((j / NY) - 1) & 1, p.pool.err);
+      if (!ok) break;
+      unsigned char* bt = bring + bs * b_stage;
+      unsigned char* yt = yring + ys * kYTileBytes;
+      if (lane == 0) {
+        const bool two = n0 + 64 < L.d_out;  // no box lies wholly past d_out
+        bar_expect(&b_full[bs], (uint32_t)r16 * (kEN * 2));
+        bar_expect(&y_full[ys], (uint32_t)(two ? kYTileBytes : kYTileBytes / 2));
+        tma_tile_2d(yt, &p.ymap[e.k], n0, row0, &y_full[ys]);
+        if (two) tma_tile_2d(yt + kYTileBytes / 2, &p.ymap[e.k], n0 + 64, row0, &y_full[ys]);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
+        if (g < r16 / 2)
+          tma_gather4(bt + ((4 * kq) >> 3) * 2048 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[i][0],
+                      rr[i][1], rr[i][2], rr[i][3], &b_full[bs]);
+      }
+      ++issued;
+      ecur_next(p, e);
     }
-    uint4* dst = reinterpret_cast<uint4*>(L.y + (int64_t)token * L.ldy + n0 + col);
-    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    // every copy issued must land before the CTA may exit (the last phase of
+    // each ring stage is not re-armed, so these waits see their own copies)
+    if (lane == 0) {
+      for (int j = max(0, issued - NB); j < issued; ++j) bar_wait(&b_full[j % NB], (j / NB) & 1, p.pool.err);
+      for (int j = max(0, issued - NY); j < issued; ++j) bar_wait(&y_full[j % NY], (j / NY) & 1, p.pool.err);
+    }
+  } else if (n_items > 0 && warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      ECur e;
+      ecur_init(p, i0, e);
+      int unit = 0;
+      const uint32_t id = idesc_f16(p.dtype, kEN, 1);
+      const uint32_t sh = su32(t_hi), sl = su32(t_lo);
+      for (int j = 0; j < n_items && ok; ++j) {
+        if (!e.valid) break;
+        const int r16 = (p.plan.seg_rank[e.s] + 15) & ~15;
+        const int bs = j % NB, as = j % kAcc;
+        if (j == 0 || e.c == 0) {
+          ok = bar_wait(&t_full, unit & 1, p.pool.err);
+          ++unit;
+        }
+        if (ok) ok = bar_wait(&b_full[bs], (j / NB) & 1, p.pool.err);
+        if (ok && j >= kAcc) ok = bar_wait(&a_empty[as], ((j / kAcc) - 1) & 1, p.pool.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sb = su32(bring + bs * b_stage);
+        const uint32_t acc = tmem + as * kEN;
+        for (int q = 0; q < r16 / 16; ++q)
+          mma_f16(acc, sdesc(sh + (q >> 2) * (kBM * 128) + (q & 3) * 32, 16, 1024), sdesc(sb + q * 4096, 1024, 2048),
+                  id, q > 0 ? 1u : 0u);
+        for (int q = 0; q < r16 / 16; ++q)
+          mma_f16(acc, sdesc(sl + (q >> 2) * (kBM * 128) + (q & 3) * 32, 16, 1024), sdesc(sb + q * 4096, 1024, 2048),
+                  id, 1u);
+        mma_commit(&b_empty[bs]);
+        mma_commit(&a_full[as]);
+        ecur_next(p, e);
+      }
+      // all MMAs complete before TMEM is released
+      mma_commit(&fin);
+      bar_wait(&fin, 0, p.pool.err);
+    }
+    __syncwarp();
+  } else if (n_items > 0) {
+    // ---------------- epilogue warps 2..5: TMEM lanes 32 * (warp % 4)
+    const int quarter = warp & 3;
+    const int mrow = quarter * 32 + lane;
+    const int etid = tid - 64;  // 0..127
+    ECur e;
+    ecur_init(p, i0, e);
+    for (int j = 0; j < n_items && ok; ++j) {
+      if (!e.valid) break;
+      const SlotDev& L = p.slot[e.k];
+      const int s = e.s;
+      const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
+      const int r16 = (r + 15) & ~15;
+      const int seg1 = p.plan.seg_end[s];
+      const int row0 = p.plan.seg_start[s] + e.m * kBM;
+      const int token = row0 + mrow;
+      const bool valid = token < seg1;
+      const int n0 = e.c * kEN;
+      if (j == 0 || e.c == 0) {
+        // new unit: t rows of slot k as hi / lo halves, K-major 128-byte swizzle.
+        // The previous unit's MMAs are complete: this thread waited on the
+        // accumulator of its last item, committed after them.
+        const float* trow = p.t + (int64_t)e.k * p.t_slot_stride + (int64_t)token * p.t_ld;
+        for (int k0 = 0; k0 < r16; k0 += 8) {
+          float v[8];
+          if (valid) {
+            const float4 f0 = *reinterpret_cast<const float4*>(trow + k0);
+            const float4 f1 = *reinterpret_cast<const float4*>(trow + k0 + 4);
+            v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+            v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              if (k0 + q >= r) v[q] = 0.f;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = 0.f;
+          }
+          uint4 h, l;
+          split2<DT>(v[0], v[1], h.x, l.x);
+          split2<DT>(v[2], v[3], h.y, l.y);
+          split2<DT>(v[4], v[5], h.z, l.z);
+          split2<DT>(v[6], v[7], h.w, l.w);
+          const int off = (k0 >> 6) * (kBM * 128) + (mrow >> 3) * 1024 + (mrow & 7) * 128 +
+                          ((((k0 & 63) >> 3) ^ (mrow & 7)) << 4);
+          *reinterpret_cast<uint4*>(t_hi + off) = h;
+          *reinterpret_cast<uint4*>(t_lo + off) = l;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&t_full)) : "memory");
+      }
+      const int as = j % kAcc, ys = j % NY;
+      ok = bar_wait(&a_full[as], (j / kAcc) & 1, p.pool.err);
+      if (ok) ok = bar_wait(&y_full[ys], (j / NY) & 1, p.pool.err);
+      if (!ok) break;
+      tc_fence_after();
+      const float s_a = __ldg(p.pool.scale + a);
+      unsigned char* yt = yring + ys * kYTileBytes;
+#pragma unroll
+      for (int cc = 0; cc < kEN / 16; ++cc) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + as * kEN + cc * 16, v);
+        if (!valid) continue;
+        // 16 outputs = chunks ch, ch + 1 (8 outputs each) of box cc / 4
+        unsigned char* rowp = yt + (cc >> 2) * (kYTileBytes / 2) + mrow * 128;
+        const int ch = (cc & 3) * 2;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint4* pp = reinterpret_cast<uint4*>(rowp + (((ch + h) ^ (mrow & 7)) << 4));
+          const uint4 yv = *pp;
+          const uint32_t w[4] = {yv.x, yv.y, yv.z, yv.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float y0, y1;
+            up2<DT>(w[q], y0, y1);
+            o[q] = pk2<DT>(fmaf(s_a, __uint_as_float(v[h * 8 + 2 * q]), y0),
+                           fmaf(s_a, __uint_as_float(v[h * 8 + 2 * q + 1]), y1));
+          }
+          *pp = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&a_empty[as])) : "memory");
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&e_sync)) : "memory");
+      }
+      // the tile in shared memory is complete once all four warps arrived
+      // (a bounded wait, unlike a named barrier, so a warp that gave up
+      // cannot hang the others)
+      ok = bar_wait(&e_sync, j & 1, p.pool.err);
+      if (!ok) break;
+      // coalesced stores: thread -> (row it * 8 + etid / 16, 16-byte chunk etid % 16)
+      const int q16 = etid & 15, cb = q16 >> 3, cj = q16 & 7;
+      const int col = n0 + q16 * 8;
+#pragma unroll 4
+      for (int it = 0; it < kBM / 8; ++it) {
+        const int row = it * 8 + (etid >> 4);
+        const int tok = row0 + row;
+        if (tok < seg1 && col < L.d_out) {
+          const uint4 v = *reinterpret_cast<const uint4*>(yt + cb * (kYTileBytes / 2) + row * 128 +
+                                                          ((cj ^ (row & 7)) << 4));
+          *reinterpret_cast<uint4*>(L.y + (int64_t)tok * L.ldy + col) = v;
+        }
+      }
+      fence_async_smem();  // generic-proxy writes of the slot before the next TMA fill
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&y_empty[ys])) : "memory");
+      ecur_next(p, e);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kEN);
+  if (warp == 1) tmem_dealloc(tmem, kAcc * kEN);
   gd_launch();
 }
 
@@ -667,7 +877,6 @@ static SgmvParams g_sgmv;  // host staging of the (large) parameter block
 cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_start, const int32_t* seg_adapter,
                         int S, int T, int sm_count, cudaStream_t st, void* scratch, int max_tokens,
                         int64_t n_pages, cudaEvent_t const* ev, int n_ev) {
-  (void)sm_count;
   SgmvParams& p = g_sgmv;
   memset(&p, 0, sizeof(p));
   p.pool = bp.pool;
@@ -725,16 +934,33 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   p.t_slot_stride = (int64_t)Tm * r16max;
   if (S > Tm) return cudaErrorNotSupported;
 
+  for (int k = 0; k < p.n_slots; ++k) {
+    const SlotDev& L = p.slot[k];
+    if (!encode_2d(&p.ymap[k], dtype, L.y, (uint64_t)L.d_out, (uint64_t)T, (uint64_t)L.ldy * 2, 64, kBM))
+      return cudaErrorNotSupported;
+  }
+  // expand shared memory: t hi + lo, NB B stages, NY y tiles (deepest rings that fit)
+  p.e_t_half = ((r16max + 63) / 64) * (kBM * 128);
+  p.e_b_stage = r16max * (kEN * 2);
+  p.e_nb = 4;
+  p.e_ny = 4;
+  const size_t smem_cap = 227 * 1024 - 1024;  // dynamic budget minus static barriers
+  auto esmem = [&] {
+    return 2 * (size_t)p.e_t_half + (size_t)p.e_nb * p.e_b_stage + (size_t)p.e_ny * kYTileBytes + 1024;
+  };
+  while (esmem() > smem_cap && (p.e_nb > 2 || p.e_ny > 2)) {
+    if (p.e_ny > p.e_nb) --p.e_ny;
+    else --p.e_nb;
+  }
+  if (esmem() > smem_cap) return cudaErrorNotSupported;
   const size_t shrink_smem = (size_t)p.stages * stage_bytes + 1024;
-  const size_t expand_smem = 2 * (size_t)((r16max + 63) / 64) * (kBM * 128) + (size_t)r16max * 512 + 1024;
+  const size_t expand_smem = esmem();
   cudaError_t ea = cudaFuncSetAttribute(k_sgmv_shrink, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)shrink_smem);
   if (ea == cudaSuccess)
     ea = cudaFuncSetAttribute(dtype == SLORA_BF16 ? k_sgmv_expand<SLORA_BF16> : k_sgmv_expand<SLORA_F16>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)expand_smem);
   if (ea != cudaSuccess) return ea;
   const int tiles = (T + kBM - 1) / kBM + S;  // upper bound on 128-token tiles over all segments
-  int nchunks = 0;
-  for (int k = 0; k < p.n_slots; ++k) nchunks += (p.slot[k].d_out + kEN - 1) / kEN;
   // timing hook: n_ev == 2 brackets the call, n_ev >= 4 also splits it per kernel
   if (n_ev >= 2) cudaEventRecord(ev[0], st);
   k_sgmv_plan<<<1, 1024, 0, st>>>(p);
@@ -744,8 +970,9 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   e = launch_pdl(k_sgmv_shrink, p.n_groups * tiles, kShrinkThreads, shrink_smem, st, p);
   if (e != cudaSuccess) return e;
   if (n_ev >= 4) cudaEventRecord(ev[2], st);
-  if (dtype == SLORA_BF16) e = launch_pdl(k_sgmv_expand<SLORA_BF16>, nchunks * tiles, kExpandThreads, expand_smem, st, p);
-  else e = launch_pdl(k_sgmv_expand<SLORA_F16>, nchunks * tiles, kExpandThreads, expand_smem, st, p);
+  // persistent expand: one CTA per SM, each a contiguous range of items
+  if (dtype == SLORA_BF16) e = launch_pdl(k_sgmv_expand<SLORA_BF16>, sm_count, kExpandThreads, expand_smem, st, p);
+  else e = launch_pdl(k_sgmv_expand<SLORA_F16>, sm_count, kExpandThreads, expand_smem, st, p);
   if (e != cudaSuccess) return e;
   if (n_ev >= 4) cudaEventRecord(ev[3], st);
   else if (n_ev == 2) cudaEventRecord(ev[1], st);

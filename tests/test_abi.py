@@ -171,3 +171,14 @@ def test_bad_desc_rejected():
     d = G.make_desc(G.SLORA_F16, [128], [128], 4, 16, 8, 1000, 4, host_only=True)
     with pytest.raises(G.SloraError):
         G.slora_pool_create(d)   # page size not a power of two
+
+
+def test_event_without_cuda_handle_is_refused():
+    """A torch event that was never recorded has no CUDA handle (0); passing
+    it as NULL would drop the page-in completion signal, so the binding
+    refuses it."""
+    class Unrecorded:
+        cuda_event = 0
+    with pytest.raises(ValueError):
+        G._event(Unrecorded())
+    assert G._event(None) is None and G._event(1234) == 1234
