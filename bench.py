@@ -406,24 +406,25 @@ def run_mixed(args, rank, world, w):
         M.restore(stream)
     st, code, info = H.G.slora_check_device(M.h)
     assert st == 0, (code, info)
-    s0 = H.G.slora_pool_stats(M.h)
     if world > 1:
         torch.distributed.barrier()
     clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", 0)))
     clocks.start()
     t_step = t_page = t_comp = 0.0
+    paged = 0
     for _ in range(K):
         M.ten.reset()
         flush.zero_()
+        s0 = H.G.slora_pool_stats(M.h)
         M.step(stream, ev[0], ev[1], ev[2])
         ev[2].synchronize()
+        paged += H.G.slora_pool_stats(M.h)["bytes_paged_in"] - s0["bytes_paged_in"]
         t_step += ev[0].elapsed_time(ev[2])
         t_page += ev[0].elapsed_time(ev[1])
         t_comp += ev[1].elapsed_time(ev[2])
         M.restore(stream)
     clk = clocks.stop()
-    s1 = H.G.slora_pool_stats(M.h)
-    paged_steps = (s1["bytes_paged_in"] - s0["bytes_paged_in"]) / K
+    paged_steps = paged / K
     t_step = max_over_ranks(t_step, world, "cuda")
     ms, ms_page, ms_comp = t_step / K, t_page / K, t_comp / K
     value = job_throughput(world, w.T, K, t_step)

@@ -137,3 +137,102 @@ def decode(bits: np.ndarray, dtype) -> np.ndarray:
     if dtype == W.F16:
         return bits.view(np.float16).astype(np.float64)
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+class MixedStep:
+    """The mixed serving step: a decode batch (one adapter per token) and
+    prefill requests (one adapter per request) in one batch, with a share of
+    the step's adapters cold (in pinned host memory only).
+
+    Pool: sized 1.25x the pages of the step's adapter set; filled at build
+    time with the warm adapters plus untouched "filler" adapters until no
+    filler fits, so the cold adapters can only come in by LRU eviction.
+
+    step(): page-in of the whole adapter set on a side stream (the cold ones
+    are copied, evicting fillers), the compute stream waits on its done event,
+    then the fused BGMV delta over the decode tokens and the SGMV over the
+    prefill requests.  restore(): evicts the cold set again and pages the
+    evicted fillers back (outside any timed region), so that every step pays
+    the same page-in."""
+
+    def __init__(self, w: W.Workload, pagein_mode=G.SLORA_PAGEIN_KERNEL, headroom=1.25):
+        import torch
+        self.w = w
+        d_in = [p.d_in for p in w.projs]
+        d_out = [p.d_out for p in w.projs]
+        desc = G.make_desc(w.dtype, d_in, d_out, w.n_adapters, int(w.ranks.max()), 1, w.page_elems, 0)
+        need = np.array([G.slora_pages_for_rank(desc, int(r)) for r in w.ranks], np.int64)
+        self.U = w.touched()
+        self.warm, self.cold = W.cold_split(w)
+        n_pages = int(np.ceil(headroom * need[self.U].sum()))
+        used = int(need[self.warm].sum())
+        touched = set(self.U.tolist())
+        fillers = []
+        for a in range(w.n_adapters):
+            if a not in touched and need[a] > 0 and used + need[a] <= n_pages:
+                fillers.append(a)
+                used += int(need[a])
+        self.fillers = fillers
+        self.n_pages = n_pages
+        self.need = need
+        self.pb = PoolBuild(w, resident=list(self.warm) + fillers, n_pages=n_pages,
+                            pagein_mode=pagein_mode)
+        self.ten = Tensors(w)
+        nd = w.n_decode
+        self.d_idx = torch.from_numpy(w.idx[:nd].copy()).cuda()
+        self.n_req = int(w.req_adapter.size)
+        self.d_rs = torch.from_numpy(w.req_start).cuda()
+        self.d_ra = torch.from_numpy(w.req_adapter).cuda()
+        self.ss = torch.zeros(self.n_req + 1, dtype=torch.int32, device="cuda")
+        self.sa = torch.zeros(self.n_req, dtype=torch.int32, device="cuda")
+        self.S = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.side = torch.cuda.Stream()
+        self.ids = self.U.tolist()
+        self.ev_start = torch.cuda.Event()
+        self.ev_paged = torch.cuda.Event()
+        for e in (self.ev_start, self.ev_paged):
+            e.record()  # torch creates the CUDA event on first record
+        torch.cuda.synchronize()
+
+    @property
+    def h(self):
+        return self.pb.h
+
+    def cold_bytes(self) -> int:
+        """Weight bytes of the cold adapters (what one step copies)."""
+        w = self.w
+        per_rank = sum(p.d_in + p.d_out for p in w.projs) * 2
+        return int(sum(int(w.ranks[a]) * per_rank for a in self.cold))
+
+    def step(self, stream, start=None, paged=None, end=None):
+        """start/end: events recorded on `stream` around the step; paged: the
+        page-in's done event (created by the caller, timing enabled)."""
+        w = self.w
+        start = start or self.ev_start
+        paged = paged or self.ev_paged
+        if not paged.cuda_event:
+            paged.record(self.side)
+        start.record(stream)
+        self.side.wait_event(start)
+        G.slora_adapter_page_in(self.h, self.ids, self.side, paged)
+        stream.wait_event(paged)
+        if w.n_decode:
+            G.slora_lora_delta(self.h, *self.ten.args(), self.d_idx, w.n_decode, stream)
+        if self.n_req:
+            G.slora_build_sgmv_segments(self.h, self.d_rs, self.d_ra, self.n_req, self.ss, self.sa,
+                                        self.S, stream)
+            G.slora_sgmv(self.h, *self.ten.args(), self.ss, self.sa, self.n_req, w.T, stream)
+        if end is not None:
+            end.record(stream)
+
+    def restore(self, stream):
+        for a in self.cold.tolist():
+            G.slora_adapter_evict(self.h, int(a), stream)
+        back = [f for f in self.fillers if not G.slora_adapter_is_resident(self.h, f)]
+        if back:
+            G.slora_adapter_page_in(self.h, back, self.side)
+        self.side.synchronize()
+        stream.synchronize()
+
+    def close(self):
+        self.pb.close()
