@@ -51,6 +51,31 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
+# DRAM traffic per launch from a committed ncu capture (profiles/traffic.json),
+# valid only while the kernel's source file is the one that was captured
+KERNEL_SOURCE = {"shrink": "bgmv.cu", "expand": "bgmv.cu", "segments": "bgmv.cu",
+                 "sgmv_shrink": "sgmv.cu", "sgmv_expand": "sgmv.cu"}
+
+
+def source_sha(name: str) -> str:
+    import hashlib
+    path = os.path.join(ROOT, "gather_lora_paged_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def ncu_traffic(workload: str, kernel: str):
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            e = json.load(f)[workload][kernel]
+        if e["source_sha256"] != source_sha(KERNEL_SOURCE[kernel]):
+            return None  # the kernel changed since the counters were taken
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
 # data-parallel replicas: rank k runs workload `config` with its own batch
 # (seeded by k), no collective on the data path; timings are reduced by max.
 def replica_workload(config: int, rank: int) -> W.Workload:
@@ -167,6 +192,7 @@ class DecodeRun:
     """Decode step: page-in call for the batch's adapter set (LRU touch), then
     the fused delta (segment build, grouped shrink, grouped expand)."""
     phases = ("segments", "shrink", "expand")
+    ncu_names = ("segments", "shrink", "expand")
 
     def __init__(self, w):
         import torch
@@ -199,6 +225,7 @@ class PrefillRun(DecodeRun):
     """Prefill step: page-in call, request -> segment merge on the device, and
     the tensor-core SGMV (plan, shrink, expand) over all projections."""
     phases = ("plan", "shrink", "expand")
+    ncu_names = ("plan", "sgmv_shrink", "sgmv_expand")
 
     def __init__(self, w):
         import torch
@@ -351,7 +378,8 @@ def run_ours(args, rank, world):
                    "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": names[i_dom], "achieved": achieved, "peak": hbm,
-                     "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": ncu_traffic(w.name, R.ncu_names[i_dom]),
                      "peak_source": src, "alg_bytes_per_launch": dom_bytes},
         "step_roofline": {"achieved": step_gbs, "peak": hbm, "unit": "GB/s",
                           "frac": step_gbs / hbm, "alg_bytes_per_step": alg["total_bytes"],

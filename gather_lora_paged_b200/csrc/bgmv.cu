@@ -46,12 +46,8 @@ __host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (
 constexpr int kCW = 8;                        // consumer warps per CTA
 constexpr int kProd = 4;                      // producer warps (interleaved ring stages)
 constexpr int kPipeThreads = (kCW + kProd) * 32;
-constexpr int kNS = 8;                        // ring stages
-constexpr int kStageBytes = 24 * 1024;
-constexpr int kRingBytes = kNS * kStageBytes;
 constexpr int kDescInts = 32;                 // per-stage descriptor (task fields)
 constexpr int kRB = 16;                       // shrink task: rank rows (2 per consumer warp)
-constexpr int kER = 4;                        // expand stage: rank rows
 constexpr int kELC = kCW * 256;               // expand task: outputs (256 per consumer warp)
 constexpr int kMaxPieces = 5;                 // pieces of a 2048-element row over >= 512-element pages
 
@@ -409,12 +405,16 @@ __device__ __forceinline__ const uint16_t* page_ptr(const PoolDev& P, int32_t pg
 }
 
 // ---------------------------------------------------------------------------
-// Shrink and expand run as warp-specialised persistent CTAs: one producer warp
-// walks the CTA's (task, stage) sequence and fills a ring of kNS shared-memory
-// stages with page-gathered bulk copies (cp.async.bulk, completion counted on
-// the stage's `full` mbarrier); kCW consumer warps each compute a fixed slice
-// of every stage and release it on the stage's `empty` mbarrier.  Page ids and
-// token ids are looked up two stages before the stage is issued.
+// Shrink and expand run as warp-specialised persistent CTAs: kProd producer
+// warps take turns along the CTA's (task, stage) sequence and fill a ring of
+// shared-memory stages with page-gathered bulk copies (cp.async.bulk,
+// completion counted on the stage's `full` mbarrier); kCW consumer warps each
+// compute a fixed slice of every stage and release it on the stage's `empty`
+// mbarrier.  Page ids and token ids are looked up two of a producer's stages
+// before the stage is issued.  Stages hold whole 4 KiB row slices: the copy
+// engine's cost per request makes 1 KiB copies top out near 60% of HBM
+// bandwidth, and a consumer warp needs a full row slice per stage to keep its
+// fixed per-stage cost small.
 // A paged range [f0, f1) cut at page boundaries: piece q starts at f0 (q = 0)
 // or at the q-th boundary after f0.
 __device__ __forceinline__ bool piece_range(const PoolDev& P, int64_t f0, int64_t f1, int q, int64_t& b,
@@ -429,11 +429,24 @@ __device__ __forceinline__ bool piece_range(const PoolDev& P, int64_t f0, int64_
 
 // ---------------------------------------------------------------------------
 // Shrink task = (group g, segment, kRB rank rows, NT tokens, kShrinkKT slice
-// of d_in); stages of kStageK elements.  Stage layout: rank row i at
-// i * 1 KiB, token row t at (kRB + t) * 1 KiB.  Consumer warp w owns rows
-// 2w and 2w + 1 of the task.
+// of d_in).  The task's x rows (NT x up to kShrinkKT elements) are copied
+// once, with its first stage, into one of two x buffers (alternating with the
+// CTA's task count); its A rows stream through a kSNS-stage ring kSRows at a
+// time, each stage holding kSRows row slices of up to kShrinkKT elements
+// (4 KiB copies, cut only at page boundaries).  Consumer warp w owns stage row
+// w and writes one fp32 partial per (row, token) of the slice; the expand sums
+// the partials of a row in index order.
+constexpr int kSRows = 8;                        // A rows per shrink stage (one per consumer warp)
+constexpr int kSNS = 4;                          // shrink ring stages
+constexpr int kSStageBytes = kSRows * 2 * kShrinkKT;
+constexpr int kSRingBytes = kSNS * kSStageBytes;
+constexpr int kXBufBytes = 8 * 2 * kShrinkKT;    // up to 8 tokens x kShrinkKT elements
+static_assert(kPartK == kShrinkKT && kCW == kSRows, "shrink stage mapping");
+static_assert(kSRows * kMaxPieces <= 64, "two lookups per lane");
+static_assert(kSNS % kProd == 0 || kProd % kSNS == 0, "ring slots per producer");
+
 struct STask {
-  int g, a, r, seg0, n, nt, rg, tg, split, nst, nrows, ntok;
+  int g, a, r, seg0, n, nt, rg, tg, split, nst, nrows, ntok, xb;
 };
 static_assert(sizeof(STask) / 4 + 2 <= kDescInts, "descriptor too small");
 
@@ -459,9 +472,10 @@ __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView
   q /= n_tg;
   t.split = q % n_split;
   t.rg = q / n_split;
-  t.nst = cdiv_i(min(kShrinkKT, d_in - t.split * kShrinkKT), kStageK);
   t.nrows = min(kRB, p.group[g].n * t.r - t.rg * kRB);
+  t.nst = cdiv_i(t.nrows, kSRows);
   t.ntok = min(t.nt, t.n - t.tg * t.nt);
+  t.xb = ((task - (int)blockIdx.x) / (int)gridDim.x) & 1;  // CTA-local task count parity
 }
 
 struct SCursor {  // a point of the producer's (task, stage) sequence
@@ -479,121 +493,137 @@ __device__ __forceinline__ void scursor_next(const BgmvParams& p, const SegView&
   if (c.valid) decode_shrink(p, V, c.task, c.t);
 }
 
-// Per-lane lookups of a shrink stage: lane l copies piece l >> 4 of row l & 15
-// (aux0 = its page id); lane l < ntok also copies token row l (aux1 = token).
-__device__ __forceinline__ void shrink_lookup(const BgmvParams& p, const SCursor& c, int32_t& aux0,
+// Per-lane lookups of a shrink stage: entry e = lane + 32 u (u = 0, 1),
+// e < kSRows * kMaxPieces, copies piece e % kMaxPieces of stage row
+// e / kMaxPieces (aux0[u] = its page id); on a task's first stage lane
+// l < ntok also copies token row l (aux1 = token).
+__device__ __forceinline__ void shrink_lookup(const BgmvParams& p, const SCursor& c, int32_t (&aux0)[2],
                                               int32_t& aux1) {
-  const int lane = threadIdx.x & 31, i = lane & 15;
-  aux0 = -1;
+  const int lane = threadIdx.x & 31;
+  aux0[0] = aux0[1] = -1;
   aux1 = -1;
   if (!c.valid) return;
   const STask& t = c.t;
   const GroupDev& G = p.group[t.g];
-  const int k0 = t.split * kShrinkKT + c.st * kStageK;
-  const int L = min(kStageK, G.d_in - k0);
-  if (i < t.nrows) {
-    const int rho = t.rg * kRB + i;
-    const int j = rho / t.r, k = rho % t.r;
-    const int64_t f0 = (int64_t)k * G.d_in + k0;
-    int64_t b, e;
-    if (piece_range(p.pool, f0, f0 + L, lane >> 4, b, e))
-      aux0 = page_id(p.pool, t.a, p.slot[G.slot[j]].listA, b);
+  const int k0 = t.split * kShrinkKT;
+  const int L = min(kShrinkKT, G.d_in - k0);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = lane + 32 * u;
+    const int i = e / kMaxPieces, q = e % kMaxPieces;
+    if (i < kSRows && c.st * kSRows + i < t.nrows) {
+      const int rho = t.rg * kRB + c.st * kSRows + i;
+      const int j = rho / t.r, k = rho % t.r;
+      const int64_t f0 = (int64_t)k * G.d_in + k0;
+      int64_t b, en;
+      if (piece_range(p.pool, f0, f0 + L, q, b, en)) aux0[u] = page_id(p.pool, t.a, p.slot[G.slot[j]].listA, b);
+    }
   }
-  if (lane < t.ntok) aux1 = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
+  if (c.st == 0 && lane < t.ntok) aux1 = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
 }
 
-__device__ __forceinline__ void shrink_issue(const BgmvParams& p, const SCursor& c, int32_t aux0, int32_t aux1,
-                                             unsigned char* buf, int32_t* desc, uint64_t* bar) {
-  const int lane = threadIdx.x & 31, i = lane & 15;
+__device__ __forceinline__ void shrink_issue(const BgmvParams& p, const SCursor& c, const int32_t (&aux0)[2],
+                                             int32_t aux1, unsigned char* buf, unsigned char* xbuf, int32_t* desc,
+                                             uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
   const STask& t = c.t;
   const GroupDev& G = p.group[t.g];
-  const int k0 = t.split * kShrinkKT + c.st * kStageK;
-  const int L = min(kStageK, G.d_in - k0);
+  const int k0 = t.split * kShrinkKT;
+  const int L = min(kShrinkKT, G.d_in - k0);
+  const int rows = min(kSRows, t.nrows - c.st * kSRows);
   if (lane == 0) {
     const int32_t* src = reinterpret_cast<const int32_t*>(&t);
     for (int q = 0; q < (int)(sizeof(STask) / 4); ++q) desc[q] = src[q];
     desc[kDescInts - 2] = c.st;
     desc[kDescInts - 1] = 1;
-    mbar_expect_tx(bar, 2u * L * (t.nrows + t.ntok));
+    mbar_expect_tx(bar, 2u * L * (rows + (c.st == 0 ? t.ntok : 0)));
   }
   __syncwarp();
-  if (aux0 >= 0) {
-    const int rho = t.rg * kRB + i;
-    const int64_t f0 = (int64_t)(rho % t.r) * G.d_in + k0;
-    int64_t b, e;
-    piece_range(p.pool, f0, f0 + L, lane >> 4, b, e);
-    bulk_g2s(buf + i * 2 * kStageK + 2 * (b - f0), page_ptr(p.pool, aux0, b), (uint32_t)(2 * (e - b)), bar);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (aux0[u] >= 0) {
+      const int e = lane + 32 * u;
+      const int i = e / kMaxPieces, q = e % kMaxPieces;
+      const int rho = t.rg * kRB + c.st * kSRows + i;
+      const int64_t f0 = (int64_t)(rho % t.r) * G.d_in + k0;
+      int64_t b, en;
+      piece_range(p.pool, f0, f0 + L, q, b, en);
+      bulk_g2s(buf + i * 2 * kShrinkKT + 2 * (b - f0), page_ptr(p.pool, aux0[u], b), (uint32_t)(2 * (en - b)), bar);
+    }
   }
-  if (aux1 >= 0)
-    bulk_g2s(buf + (kRB + lane) * 2 * kStageK, G.x + (int64_t)aux1 * G.ldx + k0, 2u * L, bar);
+  if (aux1 >= 0) bulk_g2s(xbuf + lane * 2 * kShrinkKT, G.x + (int64_t)aux1 * G.ldx + k0, 2u * L, bar);
 }
 
 template <int DT, int NT>
 __device__ __forceinline__ void shrink_consume(const BgmvParams& p, const STask& t, int st,
-                                               const unsigned char* buf, float (&acc)[16]) {
+                                               const unsigned char* buf, const unsigned char* xb) {
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kProd;
+  if (st * kSRows + cw >= t.nrows) return;  // warp-uniform
   const GroupDev& G = p.group[t.g];
-  const int k0 = t.split * kShrinkKT + st * kStageK;
-  const int L = min(kStageK, G.d_in - k0);
-  const int i0 = 2 * cw;
-  if (i0 < t.nrows) {
-    const bool r1 = i0 + 1 < t.nrows;
+  const int L = min(kShrinkKT, G.d_in - t.split * kShrinkKT);
+  // four accumulator chains per token (256-element chunk c feeds chain c % 4),
+  // summed in chain order
+  constexpr int kC = kShrinkKT / 256;
+  float acc[4][NT];
 #pragma unroll
-    for (int h = 0; h < kStageK / 256; ++h) {
-      const int e = h * 256 + lane * 8;
-      if (e >= L) break;
-      const uint4 a0 = lds128(buf + i0 * 2 * kStageK + 2 * e);
-      const uint4 a1 = r1 ? lds128(buf + (i0 + 1) * 2 * kStageK + 2 * e) : make_uint4(0, 0, 0, 0);
+  for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int tt = 0; tt < NT; ++tt) {
-        if (tt >= t.ntok) break;
-        const uint4 xv = lds128(buf + (kRB + tt) * 2 * kStageK + 2 * e);
-        float s0 = acc[tt], s1 = acc[NT + tt];
-        s0 = fma2_16<DT>(a0.x, xv.x, s0);
-        s1 = fma2_16<DT>(a1.x, xv.x, s1);
-        s0 = fma2_16<DT>(a0.y, xv.y, s0);
-        s1 = fma2_16<DT>(a1.y, xv.y, s1);
-        s0 = fma2_16<DT>(a0.z, xv.z, s0);
-        s1 = fma2_16<DT>(a1.z, xv.z, s1);
-        s0 = fma2_16<DT>(a0.w, xv.w, s0);
-        s1 = fma2_16<DT>(a1.w, xv.w, s1);
-        acc[tt] = s0;
-        acc[NT + tt] = s1;
+    for (int tt = 0; tt < NT; ++tt) acc[c][tt] = 0.f;
+  const unsigned char* arow = buf + cw * 2 * kShrinkKT;
+#pragma unroll
+  for (int c0 = 0; c0 < kC; c0 += 4) {
+    const int e0 = c0 * 256 + lane * 8;
+    if (e0 >= L) break;
+    uint4 av[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) av[c] = e0 + c * 256 < L ? lds128(arow + 2 * (e0 + c * 256)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) {
+      if (tt >= t.ntok) break;
+      uint4 xv[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        xv[c] = e0 + c * 256 < L ? lds128(xb + tt * 2 * kShrinkKT + 2 * (e0 + c * 256)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float s0 = acc[c][tt];
+        s0 = fma2_16<DT>(av[c].x, xv[c].x, s0);
+        s0 = fma2_16<DT>(av[c].y, xv[c].y, s0);
+        s0 = fma2_16<DT>(av[c].z, xv[c].z, s0);
+        s0 = fma2_16<DT>(av[c].w, xv[c].w, s0);
+        acc[c][tt] = s0;
       }
     }
   }
-  if (st != t.nst - 1) return;
-  // end of the task: sum over lanes, store the fp32 partial of this d_in slice
-  constexpr int N = 2 * NT;
-  float v[N];
+  float v[NT];
 #pragma unroll
-  for (int q = 0; q < N; ++q) v[q] = acc[q];
-  const float val = lane_transpose_reduce<N>(v);
-  const int Lx = lane % N;
-  const int i = i0 + Lx / NT, tt = Lx % NT;
-  if (lane < N && i < t.nrows && tt < t.ntok) {
-    const int rho = t.rg * kRB + i;
-    const int j = rho / t.r, k = rho % t.r;
-    const SlotDev& S = p.slot[G.slot[j]];
-    const int pos = t.seg0 + t.tg * t.nt + tt;
+  for (int tt = 0; tt < NT; ++tt) v[tt] = (acc[0][tt] + acc[1][tt]) + (acc[2][tt] + acc[3][tt]);
+  // sum over lanes; lane tt < ntok stores the partial of (row, token tt)
+  const float val = lane_transpose_reduce<NT>(v);
+  const int rho = t.rg * kRB + st * kSRows + cw;
+  const int j = rho / t.r, k = rho % t.r;
+  const SlotDev& S = p.slot[G.slot[j]];
+  if (lane < NT && lane < t.ntok) {
+    const int pos = t.seg0 + t.tg * t.nt + lane;
     S.t[(int64_t)pos * S.t_rs + (int64_t)k * S.t_ns + t.split] = val;
   }
-#pragma unroll
-  for (int q = 0; q < 16; ++q) acc[q] = 0.f;
 }
 
 template <int DT>
 __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constant__ BgmvParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full[kNS], empty[kNS];
-  __shared__ int32_t desc[kNS][kDescInts];
+  __shared__ __align__(8) uint64_t full[kSNS], empty[kSNS], xempty[2];
+  __shared__ int32_t desc[kSNS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kRingBytes);
+  unsigned char* xbufs = smem + kSRingBytes;
+  int32_t* segsm = reinterpret_cast<int32_t*>(xbufs + 2 * kXBufBytes);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNS; ++s) {
+    for (int s = 0; s < kSNS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
+    mbar_init(&xempty[0], kCW);
+    mbar_init(&xempty[1], kCW);
     fence_mbar_init();
   }
   griddep_wait();
@@ -614,38 +644,42 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
     for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, B);
     C = B;
     for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, C);
-    int32_t a0, a1, b0, b1;
+    int32_t a0[2], a1, b0[2], b1;
     shrink_lookup(p, A, a0, a1);
     shrink_lookup(p, B, b0, b1);
     uint32_t eparity = 0;
-    int ring = warp, uses = 0;
+    int ring = warp % kSNS, uses = 0;
+    bool ok = true;
     while (A.valid) {
-      if (uses >= kNS / kProd) {
+      if (uses >= kSNS / kProd) {
         if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
         eparity ^= 1u << ring;
       }
-      shrink_issue(p, A, a0, a1, smem + ring * kStageBytes, desc[ring], &full[ring]);
-      a0 = b0;
+      if (A.st == 0) {  // the x buffer of CTA task n is free once task n - 2 is consumed
+        const int n = (A.task - (int)blockIdx.x) / (int)gridDim.x;
+        if (n >= 2) ok = mbar_wait(&xempty[n & 1], ((n >> 1) - 1) & 1, p.pool.err);
+        if (!ok) break;
+      }
+      shrink_issue(p, A, a0, a1, smem + ring * kSStageBytes, xbufs + A.t.xb * kXBufBytes, desc[ring], &full[ring]);
+      a0[0] = b0[0];
+      a0[1] = b0[1];
       a1 = b1;
       shrink_lookup(p, C, b0, b1);
       A = B;
       B = C;
       for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, C);
-      ring = (ring + kProd) % kNS;
+      ring = (ring + kProd) % kSNS;
       ++uses;
     }
     // end marker at this producer's next position (the consumers stop at the
     // first one in sequence order)
-    if (uses >= kNS / kProd) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
+    if (uses >= kSNS / kProd) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
     if (lane == 0) {
       desc[ring][kDescInts - 1] = 0;
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[ring])) : "memory");
     }
   } else {
     // consumers
-    float acc[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) acc[q] = 0.f;
     uint32_t fparity = 0;
     int ring = 0;
     for (;;) {
@@ -657,26 +691,30 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
 #pragma unroll
       for (int q = 0; q < (int)(sizeof(STask) / 4); ++q) dst[q] = desc[ring][q];
       const int st = desc[ring][kDescInts - 2];
-      const unsigned char* buf = smem + ring * kStageBytes;
+      const unsigned char* buf = smem + ring * kSStageBytes;
+      const unsigned char* xb = xbufs + t.xb * kXBufBytes;
       if (DT == SLORA_BF16) {
         switch (t.nt) {
-          case 1: shrink_consume<SLORA_BF16, 1>(p, t, st, buf, acc); break;
-          case 2: shrink_consume<SLORA_BF16, 2>(p, t, st, buf, acc); break;
-          case 4: shrink_consume<SLORA_BF16, 4>(p, t, st, buf, acc); break;
-          default: shrink_consume<SLORA_BF16, 8>(p, t, st, buf, acc); break;
+          case 1: shrink_consume<SLORA_BF16, 1>(p, t, st, buf, xb); break;
+          case 2: shrink_consume<SLORA_BF16, 2>(p, t, st, buf, xb); break;
+          case 4: shrink_consume<SLORA_BF16, 4>(p, t, st, buf, xb); break;
+          default: shrink_consume<SLORA_BF16, 8>(p, t, st, buf, xb); break;
         }
       } else {
         switch (t.nt) {
-          case 1: shrink_consume<SLORA_F16, 1>(p, t, st, buf, acc); break;
-          case 2: shrink_consume<SLORA_F16, 2>(p, t, st, buf, acc); break;
-          case 4: shrink_consume<SLORA_F16, 4>(p, t, st, buf, acc); break;
-          default: shrink_consume<SLORA_F16, 8>(p, t, st, buf, acc); break;
+          case 1: shrink_consume<SLORA_F16, 1>(p, t, st, buf, xb); break;
+          case 2: shrink_consume<SLORA_F16, 2>(p, t, st, buf, xb); break;
+          case 4: shrink_consume<SLORA_F16, 4>(p, t, st, buf, xb); break;
+          default: shrink_consume<SLORA_F16, 8>(p, t, st, buf, xb); break;
         }
       }
       __syncwarp();
-      if (lane == 0)
+      if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
-      ring = (ring + 1) % kNS;
+        if (st == t.nst - 1)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&xempty[t.xb])) : "memory");
+      }
+      ring = (ring + 1) % kSNS;
     }
   }
   griddep_launch();
@@ -684,14 +722,23 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
 
 // ---------------------------------------------------------------------------
 // Expand task = (projection slot k, segment, NTE tokens, kELC outputs); stages
-// of kER rank rows.  Stage layout: B row i at i * 4 KiB; the t partials of
-// token t at kEXT + t * kER * t_ns * 4 B.  Consumer warp w owns outputs
-// [256 w, 256 w + 256) of the task; it loads its y slice when the task starts.
-constexpr int kEXT = kER * 2 * kELC;
-static_assert(kEXT + 4 * kER * 32 * 4 <= kStageBytes, "expand stage overflow");
+// of kER rank rows.  Stage layout: B row i at i * 4 KiB, then the t partials
+// of token t at kEXT + t * kER * t_ns * 4 B.  The task's y rows (NTE x kELC
+// outputs) are copied with its first stage into one of two y buffers
+// (alternating with the CTA's task count) and read back at its last stage.
+// Consumer warp w owns outputs [256 w, 256 w + 256) of the task.
+constexpr int kER = 8;                           // expand stage: rank rows
+constexpr int kEXT = kER * 2 * kELC;             // B rows of a stage
+constexpr int kETMax = 4 * kER * 32 * 4;         // t partials: 4 tokens x kER rows x <= 32 partials
+constexpr int kEStageBytes = kEXT + kETMax;
+constexpr int kENS = 4;                          // expand ring stages
+constexpr int kERingBytes = kENS * kEStageBytes;
+constexpr int kYBufBytes = 4 * 2 * kELC;         // up to 4 tokens x kELC outputs
+static_assert(kER * 4 == 32, "one lane per (token, row) for four tokens");
+static_assert(kER * kMaxPieces <= 64, "two lookups per lane");
 
 struct ETask {
-  int k, a, r, seg0, n, nt, tg, lc, nst, ntok, tok0, tok1, tok2, tok3;
+  int k, a, r, seg0, n, nt, tg, lc, nst, ntok, yb, tok0, tok1, tok2, tok3;
 };
 static_assert(sizeof(ETask) / 4 + 2 <= kDescInts, "descriptor too small");
 
@@ -715,6 +762,7 @@ __device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView
   t.lc = q / n_tg;
   t.nst = cdiv_i(t.r, kER);
   t.ntok = min(t.nt, t.n - t.tg * t.nt);
+  t.yb = ((task - (int)blockIdx.x) / (int)gridDim.x) & 1;  // CTA-local task count parity
   t.tok0 = t.tok1 = t.tok2 = t.tok3 = 0;
 }
 
@@ -733,13 +781,13 @@ __device__ __forceinline__ void ecursor_next(const BgmvParams& p, const SegView&
   if (c.valid) decode_expand(p, V, c.task, c.t);
 }
 
-// Per-lane lookups of an expand stage: lane l < kER * kMaxPieces copies piece
-// l % kMaxPieces of row l / kMaxPieces (aux0 = page id); lane l < ntok holds
-// token l (aux1).
-__device__ __forceinline__ void expand_lookup(const BgmvParams& p, const ECursor& c, int32_t& aux0,
+// Per-lane lookups of an expand stage: entry e = lane + 32 u (u = 0, 1),
+// e < kER * kMaxPieces, copies piece e % kMaxPieces of stage row
+// e / kMaxPieces (aux0[u] = page id); lane l < ntok holds token l (aux1).
+__device__ __forceinline__ void expand_lookup(const BgmvParams& p, const ECursor& c, int32_t (&aux0)[2],
                                               int32_t& aux1) {
   const int lane = threadIdx.x & 31;
-  aux0 = -1;
+  aux0[0] = aux0[1] = -1;
   aux1 = -1;
   if (!c.valid) return;
   const ETask& t = c.t;
@@ -747,17 +795,22 @@ __device__ __forceinline__ void expand_lookup(const BgmvParams& p, const ECursor
   const int l0 = t.lc * kELC;
   const int Lo = min(kELC, L.d_out - l0);
   const int r0 = c.st * kER;
-  const int i = lane / kMaxPieces, q = lane % kMaxPieces;
-  if (lane < kER * kMaxPieces && r0 + i < t.r) {
-    const int64_t f0 = (int64_t)(r0 + i) * L.d_out + l0;
-    int64_t b, e;
-    if (piece_range(p.pool, f0, f0 + Lo, q, b, e)) aux0 = page_id(p.pool, t.a, L.listB, b);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int e = lane + 32 * u;
+    const int i = e / kMaxPieces, q = e % kMaxPieces;
+    if (i < kER && r0 + i < t.r) {
+      const int64_t f0 = (int64_t)(r0 + i) * L.d_out + l0;
+      int64_t b, en;
+      if (piece_range(p.pool, f0, f0 + Lo, q, b, en)) aux0[u] = page_id(p.pool, t.a, L.listB, b);
+    }
   }
   if (lane < t.ntok) aux1 = __ldg(p.sc.perm + t.seg0 + t.tg * t.nt + lane);
 }
 
-__device__ __forceinline__ void expand_issue(const BgmvParams& p, const ECursor& c, int32_t aux0, int32_t aux1,
-                                             unsigned char* buf, int32_t* desc, uint64_t* bar) {
+__device__ __forceinline__ void expand_issue(const BgmvParams& p, const ECursor& c, const int32_t (&aux0)[2],
+                                             int32_t aux1, unsigned char* buf, unsigned char* ybuf, int32_t* desc,
+                                             uint64_t* bar) {
   const int lane = threadIdx.x & 31;
   const ETask& t = c.t;
   const SlotDev& L = p.slot[t.k];
@@ -778,44 +831,43 @@ __device__ __forceinline__ void expand_issue(const BgmvParams& p, const ECursor&
     for (int q = 0; q < (int)(sizeof(ETask) / 4); ++q) desc[q] = src[q];
     desc[kDescInts - 2] = c.st;
     desc[kDescInts - 1] = 1;
-    mbar_expect_tx(bar, 2u * Lo * nrows + tbytes * t.ntok);
+    mbar_expect_tx(bar, 2u * Lo * nrows + tbytes * t.ntok + (c.st == 0 ? 2u * Lo * t.ntok : 0u));
   }
   __syncwarp();
-  if (aux0 >= 0) {
-    const int i = lane / kMaxPieces, q = lane % kMaxPieces;
-    const int64_t f0 = (int64_t)(r0 + i) * L.d_out + l0;
-    int64_t b, e;
-    piece_range(p.pool, f0, f0 + Lo, q, b, e);
-    bulk_g2s(buf + i * 2 * kELC + 2 * (b - f0), page_ptr(p.pool, aux0, b), (uint32_t)(2 * (e - b)), bar);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (aux0[u] >= 0) {
+      const int e = lane + 32 * u;
+      const int i = e / kMaxPieces, q = e % kMaxPieces;
+      const int64_t f0 = (int64_t)(r0 + i) * L.d_out + l0;
+      int64_t b, en;
+      piece_range(p.pool, f0, f0 + Lo, q, b, en);
+      bulk_g2s(buf + i * 2 * kELC + 2 * (b - f0), page_ptr(p.pool, aux0[u], b), (uint32_t)(2 * (en - b)), bar);
+    }
   }
   if (lane < t.ntok) {
     const int64_t row = L.t_by_token ? (int64_t)aux1 : (int64_t)(t.seg0 + t.tg * t.nt + lane);
     bulk_g2s(buf + kEXT + lane * tbytes, L.t + row * L.t_rs + (int64_t)r0 * L.t_ns, tbytes, bar);
+    if (c.st == 0) bulk_g2s(ybuf + lane * 2 * kELC, L.y + (int64_t)aux1 * L.ldy + l0, 2u * Lo, bar);
   }
 }
 
 template <int DT, int NT>
 __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask& t, int st,
-                                               const unsigned char* buf, float (&acc)[4][8], uint4 (&yv)[4]) {
+                                               const unsigned char* buf, const unsigned char* yb,
+                                               float (&acc)[4][8]) {
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - kProd;
   const SlotDev& L = p.slot[t.k];
   const int l0 = t.lc * kELC;
   const int Lo = min(kELC, L.d_out - l0);
   const int l = cw * 256 + lane * 8;
   const bool act = l < Lo;
-  const int tokv[4] = {t.tok0, t.tok1, t.tok2, t.tok3};
-  if (st == 0) {  // this warp's y slice, needed at the task's last stage
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt)
-      yv[tt] = (act && tt < t.ntok) ? *reinterpret_cast<const uint4*>(L.y + (int64_t)tokv[tt] * L.ldy + l0 + l)
-                                    : make_uint4(0, 0, 0, 0);
-  }
   const int r0 = st * kER;
   const int nrows = min(kER, t.r - r0);
-  // t of (token tt, row kk) summed over the t_ns partials by lane 4 tt + kk
+  // t of (token tt, row kk) summed over the t_ns partials by lane kER tt + kk
   float tsum = 0.f;
   {
-    const int tt = lane >> 2, kk = lane & 3;
+    const int tt = lane / kER, kk = lane % kER;
     if (tt < t.ntok && kk < nrows) {
       const float* src = reinterpret_cast<const float*>(buf + kEXT + tt * 4 * kER * L.t_ns) + kk * L.t_ns;
       float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;  // four chains; fixed association
@@ -834,7 +886,7 @@ __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask&
 #pragma unroll
   for (int tt = 0; tt < NT; ++tt)
 #pragma unroll
-    for (int kk = 0; kk < kER; ++kk) tv[tt][kk] = __shfl_sync(FULL_MASK, tsum, 4 * tt + kk);
+    for (int kk = 0; kk < kER; ++kk) tv[tt][kk] = __shfl_sync(FULL_MASK, tsum, kER * tt + kk);
   if (act) {
 #pragma unroll
     for (int kk = 0; kk < kER; ++kk) {
@@ -849,11 +901,12 @@ __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask&
   }
   if (st != t.nst - 1) return;
   const float s_a = __ldg(p.pool.scale + t.a);
+  const int tokv[4] = {t.tok0, t.tok1, t.tok2, t.tok3};
 #pragma unroll
   for (int tt = 0; tt < NT; ++tt) {
     if (act && tt < t.ntok) {
       float yf[8];
-      unpack8<DT>(yv[tt], yf);
+      unpack8<DT>(lds128(yb + tt * 2 * kELC + 2 * l), yf);
       uint4 o;
       o.x = pack2<DT>(fmaf(s_a, acc[tt][0], yf[0]), fmaf(s_a, acc[tt][1], yf[1]));
       o.y = pack2<DT>(fmaf(s_a, acc[tt][2], yf[2]), fmaf(s_a, acc[tt][3], yf[3]));
@@ -869,15 +922,18 @@ __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask&
 template <int DT>
 __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constant__ BgmvParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full[kNS], empty[kNS];
-  __shared__ int32_t desc[kNS][kDescInts];
+  __shared__ __align__(8) uint64_t full[kENS], empty[kENS], yempty[2];
+  __shared__ int32_t desc[kENS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int32_t* segsm = reinterpret_cast<int32_t*>(smem + kRingBytes);
+  unsigned char* ybufs = smem + kERingBytes;
+  int32_t* segsm = reinterpret_cast<int32_t*>(ybufs + 2 * kYBufBytes);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kNS; ++s) {
+    for (int s = 0; s < kENS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
+    mbar_init(&yempty[0], kCW);
+    mbar_init(&yempty[1], kCW);
     fence_mbar_init();
   }
   griddep_wait();
@@ -898,29 +954,35 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
     for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, B);
     C = B;
     for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, C);
-    int32_t a0, a1, b0, b1;
+    int32_t a0[2], a1, b0[2], b1;
     expand_lookup(p, A, a0, a1);
     expand_lookup(p, B, b0, b1);
     uint32_t eparity = 0;
-    int ring = warp, uses = 0;
+    int ring = warp % kENS, uses = 0;
     while (A.valid) {
-      if (uses >= kNS / kProd) {
+      if (uses >= kENS / kProd) {
         if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
         eparity ^= 1u << ring;
       }
-      expand_issue(p, A, a0, a1, smem + ring * kStageBytes, desc[ring], &full[ring]);
-      a0 = b0;
+      if (A.st == 0) {  // the y buffer of CTA task n is free once task n - 2 is consumed
+        const int n = (A.task - (int)blockIdx.x) / (int)gridDim.x;
+        if (n >= 2 && !mbar_wait(&yempty[n & 1], ((n >> 1) - 1) & 1, p.pool.err)) break;
+      }
+      expand_issue(p, A, a0, a1, smem + ring * kEStageBytes, ybufs + A.t.yb * kYBufBytes, desc[ring],
+                   &full[ring]);
+      a0[0] = b0[0];
+      a0[1] = b0[1];
       a1 = b1;
       expand_lookup(p, C, b0, b1);
       A = B;
       B = C;
       for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, C);
-      ring = (ring + kProd) % kNS;
+      ring = (ring + kProd) % kENS;
       ++uses;
     }
     // end marker at this producer's next position (the consumers stop at the
     // first one in sequence order)
-    if (uses >= kNS / kProd) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
+    if (uses >= kENS / kProd) mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err);
     if (lane == 0) {
       desc[ring][kDescInts - 1] = 0;
       asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full[ring])) : "memory");
@@ -931,7 +993,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
     for (int tt = 0; tt < 4; ++tt)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
-    uint4 yv[4];
     uint32_t fparity = 0;
     int ring = 0;
     for (;;) {
@@ -943,16 +1004,20 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
 #pragma unroll
       for (int q = 0; q < (int)(sizeof(ETask) / 4); ++q) dst[q] = desc[ring][q];
       const int st = desc[ring][kDescInts - 2];
-      const unsigned char* buf = smem + ring * kStageBytes;
+      const unsigned char* buf = smem + ring * kEStageBytes;
+      const unsigned char* yb = ybufs + t.yb * kYBufBytes;
       switch (t.nt) {
-        case 1: expand_consume<DT, 1>(p, t, st, buf, acc, yv); break;
-        case 2: expand_consume<DT, 2>(p, t, st, buf, acc, yv); break;
-        default: expand_consume<DT, 4>(p, t, st, buf, acc, yv); break;
+        case 1: expand_consume<DT, 1>(p, t, st, buf, yb, acc); break;
+        case 2: expand_consume<DT, 2>(p, t, st, buf, yb, acc); break;
+        default: expand_consume<DT, 4>(p, t, st, buf, yb, acc); break;
       }
       __syncwarp();
-      if (lane == 0)
+      if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
-      ring = (ring + 1) % kNS;
+        if (st == t.nst - 1)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&yempty[t.yb])) : "memory");
+      }
+      ring = (ring + 1) % kENS;
     }
   }
   griddep_launch();
@@ -1112,7 +1177,9 @@ __global__ void k_gather_debug(PoolDev P, int id, int d, int list_off, int rank,
 
 // ---------------------------------------------------------------------------
 // Launchers.
-constexpr int kDynSmem = kRingBytes + 4 * kSegSmemInts;  // ring + segment table
+constexpr int kDynSmem = kERingBytes + 2 * kYBufBytes + 4 * kSegSmemInts;  // expand: ring, y, segments
+constexpr int kSDynSmem = kSRingBytes + 2 * kXBufBytes + 4 * kSegSmemInts;  // shrink: ring, x, segments
+static_assert(kSDynSmem <= 227 * 1024 - 2048 && kDynSmem <= 227 * 1024 - 2048, "shared memory");
 template <typename Kern>
 static cudaError_t launch_dependent(Kern kernel, int grid, int block, size_t smem, cudaStream_t s,
                                     const BgmvParams& p) {
@@ -1133,8 +1200,8 @@ static bool g_attrs_done = false;
 static cudaError_t set_attrs() {
   if (g_attrs_done) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_shrink<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSDynSmem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_shrink<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSDynSmem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_expand<SLORA_F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_expand<SLORA_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDynSmem);
   if (e == cudaSuccess) g_attrs_done = true;
@@ -1152,8 +1219,8 @@ cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cuda
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
   cudaError_t ea = set_attrs();
   if (ea != cudaSuccess) return ea;
-  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kPipeThreads, kDynSmem, s, p);
-  return launch_dependent(k_shrink<SLORA_F16>, grid, kPipeThreads, kDynSmem, s, p);
+  if (dtype == SLORA_BF16) return launch_dependent(k_shrink<SLORA_BF16>, grid, kPipeThreads, kSDynSmem, s, p);
+  return launch_dependent(k_shrink<SLORA_F16>, grid, kPipeThreads, kSDynSmem, s, p);
 }
 
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s) {
@@ -1204,7 +1271,7 @@ cudaError_t launch_gather_debug(const PoolDev& pool, int id, int d, int list_off
 int occupancy_blocks(int which) {
   set_attrs();
   int n = 0;
-  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kPipeThreads, kDynSmem);
+  if (which == 0) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_shrink<SLORA_F16>, kPipeThreads, kSDynSmem);
   else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_expand<SLORA_F16>, kPipeThreads, kDynSmem);
   return n > 0 ? n : 1;
 }

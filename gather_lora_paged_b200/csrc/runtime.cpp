@@ -117,7 +117,7 @@ ScratchLayout scratch_layout(const slora_pool_desc& d) {
   L.MS = (int)std::min<int64_t>(T, d.max_adapters);
   if (L.MS < 1) L.MS = 1;
   int64_t sum_ns = 0;
-  for (int p = 0; p < d.n_proj; ++p) sum_ns += cdiv64(d.d_in[p], kShrinkKT);
+  for (int p = 0; p < d.n_proj; ++p) sum_ns += cdiv64(d.d_in[p], kPartK);
   L.rk8 = std::max<int64_t>(8, (d.max_rank + 7) / 8 * 8);
   L.tpart_floats = sum_ns * T * L.rk8;
   size_t o = 0;
@@ -347,7 +347,7 @@ slora_status_t plan_slots(slora_pool* P, BgmvParams& bp, int n, const int32_t* p
     S.d_out = P->d.d_out[p];
     S.listA = P->listA[p];
     S.listB = P->listB[p];
-    S.nsplit = (int)cdiv64(S.d_in, kShrinkKT);
+    S.nsplit = (int)cdiv64(S.d_in, kPartK);
     if (need_x) {
       if (!x || !ldx || !x[k]) return P->fail(SLORA_ERR_INVALID_ARG, "x is NULL");
       if (ldx[k] < S.d_in || ldx[k] % 8 || !aligned16(x[k]))

@@ -38,7 +38,8 @@ constexpr int kBM = 128;             // tokens per tile (MMA M)
 constexpr int kBK = 64;              // K per stage (one 128-byte swizzle atom)
 constexpr int kXTileBytes = kBM * kBK * 2;
 constexpr int kShrinkThreads = 192;  // producer, MMA, 4 epilogue warps
-constexpr int kExpandThreads = 192;  // producer, MMA, 4 epilogue warps
+constexpr int kEpiWarps = 8;         // expand epilogue warps (two per TMEM lane quarter)
+constexpr int kExpandThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
 constexpr int kEN = 128;             // expand outputs per item (MMA N)
 constexpr int kAcc = 4;              // expand TMEM accumulators (kAcc x kEN columns)
 constexpr int kYTileBytes = kBM * kEN * 2;
@@ -72,6 +73,7 @@ struct SgmvParams {
   int64_t pool_rows;    // rows of 64 elements in the pool (out-of-range coordinate)
   int ntot_max;         // max over groups of round_up(n * max_rank, 16)
   int stages;           // shrink pipeline depth
+  int s_mq;             // shrink: 128-token tiles per item (share each A stage)
   int dtype;
   CUtensorMap ymap[kMaxSlots];  // per slot: y as (d_out, T) with 64 x 128 boxes
   int e_nb, e_ny;       // expand ring depths (B chunks, y tiles)
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
       else r = p.pool.rank[a];
     }
     const int mt = (r > 0 && n > 0) ? cdiv_d(n, kBM) : 0;
-    csh += mt * p.n_groups;
+    csh += cdiv_d(mt, p.s_mq) * p.n_groups;
     int ex = 0;
     for (int k = 0; k < p.n_slots; ++k) ex += cdiv_d(p.slot[k].d_out, kEN);
     cex += mt * ex;
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
     p.plan.seg_rank[s] = mt > 0 ? r : 0;
     p.plan.shrink_prefix[s] = bsh;
     p.plan.expand_prefix[s] = bex;
-    bsh += mt * p.n_groups;
+    bsh += cdiv_d(mt, p.s_mq) * p.n_groups;
     int ex = 0;
     for (int k = 0; k < p.n_slots; ++k) ex += cdiv_d(p.slot[k].d_out, kEN);
     bex += mt * ex;
@@ -300,12 +302,15 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   const int q = item - p.plan.shrink_prefix[s];
   const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_end[s];
   const int mt = cdiv_d(seg1 - seg0, kBM);
-  if (mt <= 0 || q >= mt * p.n_groups || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
+  const int MQ = p.s_mq;
+  const int mtq = cdiv_d(mt, MQ);
+  if (mt <= 0 || q >= mtq * p.n_groups || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
     if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
     gd_launch();
     return;
   }
-  const int g = q / mt, m = q % mt;
+  const int g = q / mtq, m = (q % mtq) * MQ;  // first tile of this item
+  const int nq = min(MQ, mt - m);             // tiles of this item (share each A stage)
   const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
   const GroupDev& G = p.group[g];
   const int R = G.n * r;
@@ -314,9 +319,9 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   const int KB = G.d_in / kBK;
   const int ST = p.stages;
   const int a_bytes = NT * 128;
-  const int stage_bytes = kXTileBytes + ((p.ntot_max * 128 + 1023) & ~1023);
+  const int stage_bytes = MQ * kXTileBytes + ((p.ntot_max * 128 + 1023) & ~1023);
   uint32_t ncols = 32;
-  while ((int)ncols < NT) ncols <<= 1;
+  while ((int)ncols < nq * NT) ncols <<= 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
@@ -367,10 +372,10 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
       if (kb >= ST) ok = bar_wait(&empty[st], ((kb / ST) - 1) & 1, p.pool.err);
       if (!ok) break;
       unsigned char* xs = smem + st * stage_bytes;
-      unsigned char* as = xs + kXTileBytes;
+      unsigned char* as = xs + MQ * kXTileBytes;
       if (lane == 0) {
-        bar_expect(&full[st], kXTileBytes + a_bytes);
-        tma_tile_2d(xs, &p.xmap[g], kb * kBK, row0, &full[st]);
+        bar_expect(&full[st], nq * kXTileBytes + a_bytes);
+        for (int i = 0; i < nq; ++i) tma_tile_2d(xs + i * kXTileBytes, &p.xmap[g], kb * kBK, row0 + i * kBM, &full[st]);
       }
       __syncwarp();
 #pragma unroll
@@ -407,17 +412,18 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
         if (!ok) break;
         tc_fence_after();
         const uint32_t xs = su32(smem + st * stage_bytes);
-        const uint32_t as = xs + kXTileBytes;
-        for (int c0 = 0; c0 < NT; c0 += 256) {
-          const int nc = min(256, NT - c0);
-          const uint32_t id = idesc_f16(p.dtype, nc, 0);
+        const uint32_t as = xs + MQ * kXTileBytes;
+        for (int i = 0; i < nq; ++i)
+          for (int c0 = 0; c0 < NT; c0 += 256) {
+            const int nc = min(256, NT - c0);
+            const uint32_t id = idesc_f16(p.dtype, nc, 0);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t da = sdesc(xs + kk * 32, lbo, sbo);
-            const uint64_t db = sdesc(as + c0 * 128 + kk * 32, lbo, sbo);
-            mma_f16(tmem + c0, da, db, id, (kb > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t da = sdesc(xs + i * kXTileBytes + kk * 32, lbo, sbo);
+              const uint64_t db = sdesc(as + c0 * 128 + kk * 32, lbo, sbo);
+              mma_f16(tmem + i * NT + c0, da, db, id, (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
-        }
         mma_commit(&empty[st]);
       }
       mma_commit(&accb);
@@ -429,19 +435,30 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
     tc_fence_after();
     const int quarter = warp & 3;
     const int mrow = quarter * 32 + lane;
-    const int token = row0 + mrow;
-    const bool valid = token < seg1;
-    for (int c = 0; c < NT; c += 16) {
+    for (int ci = 0; ci < nq * NT; ci += 16) {
+      const int i = ci / NT, c = ci - i * NT;  // tile, column within it
+      const int token = row0 + i * kBM + mrow;
+      const bool valid = token < seg1;
       uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + c, v);
+      tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + ci, v);
       if (!valid || !ok) continue;
+      const int sj0 = c / r, k0 = c - sj0 * r;
+      if (c + 16 <= R && k0 + 16 <= r && (k0 & 3) == 0) {  // 16 ranks of one slot: vector stores
+        float4* tt = reinterpret_cast<float4*>(p.t + (int64_t)G.slot[sj0] * p.t_slot_stride +
+                                               (int64_t)token * p.t_ld + k0);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int rho = c + i;
+        for (int e = 0; e < 4; ++e)
+          tt[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        continue;
+      }
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int rho = c + e;
         if (rho < R) {
           const int sj = rho / r, k = rho % r;
           float* tt = p.t + (int64_t)G.slot[sj] * p.t_slot_stride + (int64_t)token * p.t_ld + k;
-          *tt = __uint_as_float(v[i]);
+          *tt = __uint_as_float(v[e]);
         }
       }
     }
@@ -465,15 +482,10 @@ __device__ __forceinline__ void up2(uint32_t w, float& lo, float& hi) {
         : "=f"(lo), "=f"(hi) : "r"(w));
   }
 }
-// bf16: round to nearest even on the integer pipe (finite values); fp16: cvt.
-__device__ __forceinline__ uint32_t bf16_rn_bits(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u + 0x7fffu + ((u >> 16) & 1u)) >> 16;
-}
 template <int DT>
 __device__ __forceinline__ uint32_t pk2(float lo, float hi) {
   uint32_t r;
-  if (DT == SLORA_BF16) r = bf16_rn_bits(lo) | (bf16_rn_bits(hi) << 16);
+  if (DT == SLORA_BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
@@ -572,15 +584,15 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
     }
     for (int i = 0; i < NY; ++i) {
       bar_init(&y_full[i], 1);
-      bar_init(&y_empty[i], 4);
+      bar_init(&y_empty[i], kEpiWarps);
     }
     for (int i = 0; i < kAcc; ++i) {
       bar_init(&a_full[i], 1);
-      bar_init(&a_empty[i], 4);
+      bar_init(&a_empty[i], kEpiWarps);
     }
-    bar_init(&t_full, 4);
+    bar_init(&t_full, kEpiWarps);
     bar_init(&fin, 1);
-    bar_init(&e_sync, 4);
+    bar_init(&e_sync, kEpiWarps);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(&tmem_slot, kAcc * kEN);
@@ -693,10 +705,12 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
     }
     __syncwarp();
   } else if (n_items > 0) {
-    // ---------------- epilogue warps 2..5: TMEM lanes 32 * (warp % 4)
+    // ---------------- epilogue warps 2..9: TMEM lanes 32 * (warp % 4), output
+    // columns [64 half, 64 half + 64) of the item with half = (warp - 2) / 4
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int mrow = quarter * 32 + lane;
-    const int etid = tid - 64;  // 0..127
+    const int etid = tid - 64;  // 0 .. 32 * kEpiWarps - 1
     ECur e;
     ecur_init(p, i0, e);
     for (int j = 0; j < n_items && ok; ++j) {
@@ -715,7 +729,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
         // The previous unit's MMAs are complete: this thread waited on the
         // accumulator of its last item, committed after them.
         const float* trow = p.t + (int64_t)e.k * p.t_slot_stride + (int64_t)token * p.t_ld;
-        for (int k0 = 0; k0 < r16; k0 += 8) {
+        for (int k0 = half * 8; k0 < r16; k0 += 16) {
           float v[8];
           if (valid) {
             const float4 f0 = *reinterpret_cast<const float4*>(trow + k0);
@@ -751,7 +765,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
       const float s_a = __ldg(p.pool.scale + a);
       unsigned char* yt = yring + ys * kYTileBytes;
 #pragma unroll
-      for (int cc = 0; cc < kEN / 16; ++cc) {
+      for (int c4 = 0; c4 < kEN / 32; ++c4) {
+        const int cc = half * (kEN / 32) + c4;  // 16-column group of this warp
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + as * kEN + cc * 16, v);
         if (!valid) continue;
@@ -785,12 +800,13 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
       // cannot hang the others)
       ok = bar_wait(&e_sync, j & 1, p.pool.err);
       if (!ok) break;
-      // coalesced stores: thread -> (row it * 8 + etid / 16, 16-byte chunk etid % 16)
+      // coalesced stores: thread -> (row it * R + etid / 16, 16-byte chunk etid % 16)
+      constexpr int kRowsPerIt = 32 * kEpiWarps / 16;
       const int q16 = etid & 15, cb = q16 >> 3, cj = q16 & 7;
       const int col = n0 + q16 * 8;
 #pragma unroll 4
-      for (int it = 0; it < kBM / 8; ++it) {
-        const int row = it * 8 + (etid >> 4);
+      for (int it = 0; it < kBM / kRowsPerIt; ++it) {
+        const int row = it * kRowsPerIt + (etid >> 4);
         const int tok = row0 + row;
         if (tok < seg1 && col < L.d_out) {
           const uint4 v = *reinterpret_cast<const uint4*>(yt + cb * (kYTileBytes / 2) + row * 128 +
@@ -905,8 +921,9 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   for (int g = 0; g < p.n_groups; ++g) ntot = std::max(ntot, round16(p.group[g].n * bp.pool.max_rank));
   if (ntot > 512) return cudaErrorNotSupported;
   p.ntot_max = ntot;
-  const int stage_bytes = kXTileBytes + ((ntot * 128 + 1023) & ~1023);
-  p.stages = std::min(8, (200 * 1024) / stage_bytes);
+  p.s_mq = 2 * ntot <= 512 ? 2 : 1;  // two accumulators of NT columns fit in TMEM
+  const int stage_bytes = p.s_mq * kXTileBytes + ((ntot * 128 + 1023) & ~1023);
+  p.stages = std::min(8, (225 * 1024) / stage_bytes);
   if (p.stages < 2) return cudaErrorNotSupported;
   // tensor maps
   const int64_t pool_rows = n_pages * ((int64_t)1 << bp.pool.page_shift) / 64;
@@ -967,7 +984,8 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (n_ev >= 4) cudaEventRecord(ev[1], st);
-  e = launch_pdl(k_sgmv_shrink, p.n_groups * tiles, kShrinkThreads, shrink_smem, st, p);
+  const int items_ub = (tiles + p.s_mq - 1) / p.s_mq + S;  // >= sum over segments of ceil(tiles / s_mq)
+  e = launch_pdl(k_sgmv_shrink, p.n_groups * items_ub, kShrinkThreads, shrink_smem, st, p);
   if (e != cudaSuccess) return e;
   if (n_ev >= 4) cudaEventRecord(ev[2], st);
   // persistent expand: one CTA per SM, each a contiguous range of items

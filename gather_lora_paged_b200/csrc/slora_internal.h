@@ -9,11 +9,11 @@
 
 namespace slora {
 
-// Shrink work split (decode path).  A shrink task covers RW rank rows x NT
-// tokens x kShrinkKT elements of d_in, streamed in stages of kStageK; its
-// fp32 partial (one per kShrinkKT slice of d_in) is summed by the expand.
+// Shrink work split (decode path).  A shrink task covers a block of rank
+// rows x NT tokens x kShrinkKT elements of d_in; it leaves one fp32 partial
+// per kPartK (= kShrinkKT) slice of d_in, which the expand sums in index order.
 constexpr int kShrinkKT = 2048;
-constexpr int kStageK = 512;
+constexpr int kPartK = 2048;
 constexpr int kMaxSlots = SLORA_MAX_PROJ;   // projections per call
 constexpr int kThreads = 256;               // threads per CTA of the decode kernels
 constexpr int kEventRing = 64;
@@ -39,7 +39,7 @@ struct SlotDev {
   int64_t ldy;
   int d_in, d_out;
   int listA, listB;        // offsets of this projection's A_t / B page lists in an adapter row
-  int nsplit;              // shrink partials = ceil(d_in / kShrinkKT)
+  int nsplit;              // shrink partials = ceil(d_in / kPartK)
   int group;               // index of the x-sharing group
   int gpos;                // rank-row block of this slot inside its group
   // t (rank-r intermediate): element (row, k, c) at t[row * t_rs + k * t_ns + c],
