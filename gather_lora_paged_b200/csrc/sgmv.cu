@@ -37,7 +37,9 @@ namespace {
 constexpr int kBM = 128;             // tokens per tile (MMA M)
 constexpr int kBK = 64;              // K per stage (one 128-byte swizzle atom)
 constexpr int kXTileBytes = kBM * kBK * 2;
-constexpr int kShrinkThreads = 192;  // producer, MMA, 4 epilogue warps
+constexpr int kShrinkThreads = 192;  // X producer, MMA, 4 A-loader / epilogue warps
+constexpr int kALoaders = 128;       // shrink threads copying A rows (warps 2..5)
+constexpr int kALag = 2;             // A copy groups in flight per loader thread (1 or 2)
 constexpr int kEpiWarps = 8;         // expand epilogue warps (two per TMEM lane quarter)
 constexpr int kExpandThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue warps
 constexpr int kEN = 128;             // expand outputs per item (MMA N)
@@ -130,6 +132,39 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
       " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(su32(dst)),
       "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(su32(b))
       : "memory");
+}
+// L2 eviction-priority policies: streamed operands (X, y) go first, adapter
+// rows re-read by every token tile stay.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_tile_2d_hint(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* b,
+                                                 uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(su32(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(su32(b)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_gather4_hint(void* dst, const CUtensorMap* map, int r0, int r1, int r2, int r3,
+                                                 uint64_t* b, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(su32(dst)),
+      "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(su32(b)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w), "l"(pol)
+               : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -325,7 +360,7 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
-      bar_init(&full[i], 1);
+      bar_init(&full[i], 1 + kALoaders);  // X producer (with its bytes) + A loader threads
       bar_init(&empty[i], 1);
     }
     bar_init(&accb, 1);
@@ -339,70 +374,20 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   bool ok = true;
 
   if (warp == 0) {
-    // producer: X tile by tiled TMA, A rows by gather4 from the pages.  Lane
-    // j owns rows 4j..4j+3 (+128 per round).  Within a page a row advances one
-    // pool row per stage, so the page table is read only when a row enters a
-    // new page; the next page id is fetched one page ahead.
-    constexpr int kRounds = 4;  // NT <= 512
-    int cur[kRounds][4], left[kRounds][4], nxt[kRounds][4];
-    const int64_t pmask = (1ll << p.pool.page_shift) - 1;
-    const int rows_per_page = (int)((pmask + 1) >> 6);
-#pragma unroll
-    for (int rd = 0; rd < kRounds; ++rd)
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int rho = rd * 128 + 4 * lane + u;
-        cur[rd][u] = (int)p.pool_rows;
-        left[rd][u] = 1 << 30;
-        nxt[rd][u] = -1;
-        if (rho < R) {
-          const int sj = rho / r, k = rho % r;
-          const int lo = p.slot[G.slot[sj]].listA;
-          const int64_t f = (int64_t)k * G.d_in;
-          cur[rd][u] = pool_row(p.pool, a, lo, f);
-          left[rd][u] = rows_per_page - (int)((f & pmask) >> 6);
-          const int64_t fn = f + ((int64_t)left[rd][u] << 6);  // first element of the next page
-          nxt[rd][u] = fn < (int64_t)(k + 1) * G.d_in ? __ldg(p.pool.page_list + (int64_t)a * p.pool.list_stride + lo +
-                                                             (fn >> p.pool.page_shift))
-                                                      : -1;
-        }
-      }
-    for (int kb = 0; kb < KB && ok; ++kb) {
-      const int st = kb % ST;
-      if (kb >= ST) ok = bar_wait(&empty[st], ((kb / ST) - 1) & 1, p.pool.err);
-      if (!ok) break;
-      unsigned char* xs = smem + st * stage_bytes;
-      unsigned char* as = xs + MQ * kXTileBytes;
-      if (lane == 0) {
-        bar_expect(&full[st], nq * kXTileBytes + a_bytes);
-        for (int i = 0; i < nq; ++i) tma_tile_2d(xs + i * kXTileBytes, &p.xmap[g], kb * kBK, row0 + i * kBM, &full[st]);
-      }
-      __syncwarp();
-#pragma unroll
-      for (int rd = 0; rd < kRounds; ++rd) {
-        if (rd * 128 + 4 * lane < NT)
-          tma_gather4(as + (rd * 128 + 4 * lane) * 128, &p.poolmap, cur[rd][0], cur[rd][1], cur[rd][2], cur[rd][3],
-                      &full[st]);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {  // advance to the next stage's pool row
-          const int rho = rd * 128 + 4 * lane + u;
-          if (rho >= R) continue;
-          if (--left[rd][u] > 0) {
-            ++cur[rd][u];
-          } else if (nxt[rd][u] >= 0) {
-            const int sj = rho / r, k = rho % r;
-            const int lo = p.slot[G.slot[sj]].listA;
-            cur[rd][u] = (int)(((int64_t)nxt[rd][u] << p.pool.page_shift) >> 6);
-            left[rd][u] = rows_per_page;
-            const int64_t fstart = (int64_t)k * G.d_in + (int64_t)(kb + 1) * kBK;  // element now loaded
-            const int64_t fn = fstart + ((int64_t)rows_per_page << 6);
-            nxt[rd][u] = fn < (int64_t)(k + 1) * G.d_in ? __ldg(p.pool.page_list + (int64_t)a * p.pool.list_stride +
-                                                               lo + (fn >> p.pool.page_shift))
-                                                        : -1;
-          }
-        }
+    // X producer: the stage's token tiles by tiled TMA (streamed once: evict first)
+    if (lane == 0) {
+      const uint64_t pol_x = policy_evict_first();
+      for (int kb = 0; kb < KB && ok; ++kb) {
+        const int st = kb % ST;
+        if (kb >= ST) ok = bar_wait(&empty[st], ((kb / ST) - 1) & 1, p.pool.err);
+        if (!ok) break;
+        unsigned char* xs = smem + st * stage_bytes;
+        bar_expect(&full[st], nq * kXTileBytes);
+        for (int i = 0; i < nq; ++i)
+          tma_tile_2d_hint(xs + i * kXTileBytes, &p.xmap[g], kb * kBK, row0 + i * kBM, &full[st], pol_x);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t lbo = 16, sbo = 1024;
@@ -430,8 +415,54 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
     }
     __syncwarp();
   } else {
+    // warps 2..5 first load A: thread t copies 16-byte chunk t % 8 of rows
+    // t / 8 + 16 i of every stage with cp.async into the 128-byte-swizzled
+    // K-major layout (rows past R are zero-filled).  Copies are committed one
+    // group per stage; a stage is released to the MMA kALag stages later,
+    // after its group completed and a proxy fence made it visible to the
+    // tensor cores.
+    {
+      const int et = threadIdx.x - 64, ch = et & 7, r0 = et >> 3;
+      const int32_t* plist = p.pool.page_list + (int64_t)a * p.pool.list_stride;
+      const int64_t pmask = (1ll << p.pool.page_shift) - 1;
+      const uint64_t pol_a = policy_evict_last();  // adapter rows are re-read by every token tile
+      const int lag = min(kALag, ST - 1);           // < ST: a stage is released before its slot is reused
+      int kb = 0;
+      for (; kb < KB && ok; ++kb) {
+        const int st = kb % ST;
+        if (kb >= ST) ok = bar_wait(&empty[st], ((kb / ST) - 1) & 1, p.pool.err);
+        if (!ok) break;
+        const uint32_t as = su32(smem + st * stage_bytes + MQ * kXTileBytes);
+        for (int rho = r0; rho < NT; rho += 16) {
+          const uint32_t dst = as + rho * 128 + ((ch ^ (rho & 7)) << 4);
+          if (rho < R) {
+            const int sj = rho / r, k = rho - sj * r;
+            const int64_t f = (int64_t)k * G.d_in + (int64_t)kb * kBK + ch * 8;
+            const int32_t pg = __ldg(plist + p.slot[G.slot[sj]].listA + (f >> p.pool.page_shift));
+            const uint16_t* src = p.pool.pool + ((int64_t)pg << p.pool.page_shift) + (f & pmask);
+            asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, 16, %2;" ::"r"(dst), "l"(src),
+                         "l"(pol_a)
+                         : "memory");
+          } else {
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(dst), "l"(p.pool.pool) : "memory");
+          }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (kb >= lag) {
+          if (lag == 1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+          else asm volatile("cp.async.wait_group 2;" ::: "memory");
+          fence_async_smem();
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&full[(kb - lag) % ST])) : "memory");
+        }
+      }
+      // release the last stages (every group issued completes before exit)
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      fence_async_smem();
+      for (int k2 = max(0, kb - lag); k2 < kb; ++k2)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&full[k2 % ST])) : "memory");
+    }
     // epilogue warps 2..5: TMEM lanes 32 * (warp % 4)
-    ok = bar_wait(&accb, 0, p.pool.err);
+    ok = bar_wait(&accb, 0, p.pool.err) && ok;
     tc_fence_after();
     const int quarter = warp & 3;
     const int mrow = quarter * 32 + lane;
@@ -613,6 +644,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
     ECur e;
     ecur_init(p, i0, e);
     int issued = 0;
+    const uint64_t pol_y = policy_evict_first(), pol_b = policy_evict_last();
     for (int j = 0; j < n_items && ok; ++j) {
       if (!e.valid) {
         if (lane == 0) rec_err(p.pool.err, 7, i0 + j);
@@ -647,16 +679,16 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
         const bool two = n0 + 64 < L.d_out;  // no box lies wholly past d_out
         bar_expect(&b_full[bs], (uint32_t)r16 * (kEN * 2));
         bar_expect(&y_full[ys], (uint32_t)(two ? kYTileBytes : kYTileBytes / 2));
-        tma_tile_2d(yt, &p.ymap[e.k], n0, row0, &y_full[ys]);
-        if (two) tma_tile_2d(yt + kYTileBytes / 2, &p.ymap[e.k], n0 + 64, row0, &y_full[ys]);
+        tma_tile_2d_hint(yt, &p.ymap[e.k], n0, row0, &y_full[ys], pol_y);
+        if (two) tma_tile_2d_hint(yt + kYTileBytes / 2, &p.ymap[e.k], n0 + 64, row0, &y_full[ys], pol_y);
       }
       __syncwarp();
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
         if (g < r16 / 2)
-          tma_gather4(bt + ((4 * kq) >> 3) * 2048 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[i][0],
-                      rr[i][1], rr[i][2], rr[i][3], &b_full[bs]);
+          tma_gather4_hint(bt + ((4 * kq) >> 3) * 2048 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[i][0],
+                           rr[i][1], rr[i][2], rr[i][3], &b_full[bs], pol_b);
       }
       ++issued;
       ecur_next(p, e);
@@ -711,6 +743,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
     const int half = (warp - 2) >> 2;
     const int mrow = quarter * 32 + lane;
     const int etid = tid - 64;  // 0 .. 32 * kEpiWarps - 1
+    const uint64_t pol_y = policy_evict_first();
     ECur e;
     ecur_init(p, i0, e);
     for (int j = 0; j < n_items && ok; ++j) {
@@ -811,7 +844,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
         if (tok < seg1 && col < L.d_out) {
           const uint4 v = *reinterpret_cast<const uint4*>(yt + cb * (kYTileBytes / 2) + row * 128 +
                                                           ((cj ^ (row & 7)) << 4));
-          *reinterpret_cast<uint4*>(L.y + (int64_t)tok * L.ldy + col) = v;
+          st_global_v4_hint(L.y + (int64_t)tok * L.ldy + col, v, pol_y);
         }
       }
       fence_async_smem();  // generic-proxy writes of the slot before the next TMA fill
