@@ -94,6 +94,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
   }
 }
 
+// Bounded wait until the shared counter *c reaches `target` (a count only ever
+// grows, so unlike an mbarrier phase parity it cannot be misread however far
+// behind the waiter is); false (and a recorded error) if it gives up.
+__device__ __forceinline__ bool counter_wait(const int* c, int target, int32_t* err) {
+  long long t0 = -1;
+  for (uint32_t it = 0;; ++it) {
+    int v;
+    asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(c)) : "memory");
+    if (v >= target) return true;
+    if ((it & 63) == 0) {
+      const long long now = clock64();
+      if (t0 < 0) t0 = now;
+      else if (now - t0 > kWaitLimit) {
+        record_error(err, 4, (int)blockIdx.x);
+        return false;
+      }
+    }
+    __nanosleep(32);
+  }
+}
+
 // Bulk async copy global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -612,7 +633,8 @@ __device__ __forceinline__ void shrink_consume(const BgmvParams& p, const STask&
 template <int DT>
 __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constant__ BgmvParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full[kSNS], empty[kSNS], xempty[2];
+  __shared__ __align__(8) uint64_t full[kSNS], empty[kSNS];
+  __shared__ int xdone[2];  // consumer warps done with each x buffer (kCW per task)
   __shared__ int32_t desc[kSNS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* xbufs = smem + kSRingBytes;
@@ -622,8 +644,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
-    mbar_init(&xempty[0], kCW);
-    mbar_init(&xempty[1], kCW);
+    xdone[0] = xdone[1] = 0;
     fence_mbar_init();
   }
   griddep_wait();
@@ -655,9 +676,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
         if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
         eparity ^= 1u << ring;
       }
-      if (A.st == 0) {  // the x buffer of CTA task n is free once task n - 2 is consumed
+      if (A.st == 0) {  // the x buffer of CTA task n is free once tasks n - 2, n - 4, ... are consumed
         const int n = (A.task - (int)blockIdx.x) / (int)gridDim.x;
-        if (n >= 2) ok = mbar_wait(&xempty[n & 1], ((n >> 1) - 1) & 1, p.pool.err);
+        if (n >= 2) ok = counter_wait(&xdone[n & 1], kCW * (n >> 1), p.pool.err);
         if (!ok) break;
       }
       shrink_issue(p, A, a0, a1, smem + ring * kSStageBytes, xbufs + A.t.xb * kXBufBytes, desc[ring], &full[ring]);
@@ -711,8 +732,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
-        if (st == t.nst - 1)
-          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&xempty[t.xb])) : "memory");
+        if (st == t.nst - 1) atomicAdd(&xdone[t.xb], 1);
       }
       ring = (ring + 1) % kSNS;
     }
@@ -922,7 +942,8 @@ __device__ __forceinline__ void expand_consume(const BgmvParams& p, const ETask&
 template <int DT>
 __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constant__ BgmvParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full[kENS], empty[kENS], yempty[2];
+  __shared__ __align__(8) uint64_t full[kENS], empty[kENS];
+  __shared__ int ydone[2];  // consumer warps done with each y buffer (kCW per task)
   __shared__ int32_t desc[kENS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* ybufs = smem + kERingBytes;
@@ -932,8 +953,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCW);
     }
-    mbar_init(&yempty[0], kCW);
-    mbar_init(&yempty[1], kCW);
+    ydone[0] = ydone[1] = 0;
     fence_mbar_init();
   }
   griddep_wait();
@@ -964,9 +984,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
         if (!mbar_wait(&empty[ring], (eparity >> ring) & 1, p.pool.err)) break;
         eparity ^= 1u << ring;
       }
-      if (A.st == 0) {  // the y buffer of CTA task n is free once task n - 2 is consumed
+      if (A.st == 0) {  // the y buffer of CTA task n is free once tasks n - 2, n - 4, ... are consumed
         const int n = (A.task - (int)blockIdx.x) / (int)gridDim.x;
-        if (n >= 2 && !mbar_wait(&yempty[n & 1], ((n >> 1) - 1) & 1, p.pool.err)) break;
+        if (n >= 2 && !counter_wait(&ydone[n & 1], kCW * (n >> 1), p.pool.err)) break;
       }
       expand_issue(p, A, a0, a1, smem + ring * kEStageBytes, ybufs + A.t.yb * kYBufBytes, desc[ring],
                    &full[ring]);
@@ -1014,8 +1034,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
-        if (st == t.nst - 1)
-          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&yempty[t.yb])) : "memory");
+        if (st == t.nst - 1) atomicAdd(&ydone[t.yb], 1);
       }
       ring = (ring + 1) % kENS;
     }
