@@ -79,6 +79,7 @@ struct SgmvParams {
   int dtype;
   CUtensorMap ymap[kMaxSlots];  // per slot: y as (d_out, T) with 64 x 128 boxes
   int e_nb, e_ny;       // expand ring depths (B chunks, y tiles)
+  int e_pair;           // expand: 128-token tiles per group (one B gather serves them)
   int e_t_half;         // expand: bytes of one t half in shared memory
   int e_b_stage;        // expand: bytes of one B ring stage
 };
@@ -542,8 +543,8 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
 // shared memory, then 16-byte coalesced stores of the rows inside the segment.
 
 struct ECur {  // a point of the item sequence
-  int s, m, k, c;  // segment, tile, slot, chunk
-  int mt, nch;     // tiles of segment s, chunks of slot k
+  int s, g, k, c, i;  // segment, tile group, slot, chunk, tile within the group
+  int mt, nm, nch;    // tiles of segment s, tiles of group g, chunks of slot k
   bool valid;
 };
 
@@ -551,45 +552,72 @@ __device__ __forceinline__ int seg_tiles(const SgmvParams& p, int s) {
   return p.plan.seg_rank[s] > 0 ? cdiv_d(p.plan.seg_end[s] - p.plan.seg_start[s], kBM) : 0;
 }
 
-// First item of the range starting at `item` (< total).
+// Within a segment the items run over groups of PS consecutive 128-token tiles
+// (the last group may be shorter), then slots, then 128-output chunks, then
+// the group's tiles: one B chunk serves the group's tiles, one conversion of
+// the group's t rows serves all its slot's chunks.  First item of the range
+// starting at `item` (< total):
 __device__ __forceinline__ void ecur_init(const SgmvParams& p, int item, ECur& e) {
+  const int PS = p.e_pair;
   const int s = find_ge(p.plan.expand_prefix, p.S, item);
   int q = item - p.plan.expand_prefix[s];
-  int tot = 0;
-  for (int k = 0; k < p.n_slots; ++k) tot += cdiv_d(p.slot[k].d_out, kEN);
+  int NC = 0;
+  for (int k = 0; k < p.n_slots; ++k) NC += cdiv_d(p.slot[k].d_out, kEN);
   e.s = s;
   e.mt = seg_tiles(p, s);
-  e.m = q / tot;
-  q -= e.m * tot;
+  const int full = e.mt / PS;  // complete groups
+  if (q < full * PS * NC) {
+    e.g = q / (PS * NC);
+    q -= e.g * PS * NC;
+    e.nm = PS;
+  } else {
+    e.g = full;
+    q -= full * PS * NC;
+    e.nm = e.mt - full * PS;
+  }
+  const int nm = max(e.nm, 1);
+  int kc = q / nm;
+  e.i = q - kc * nm;
   int k = 0;
   for (; k < p.n_slots - 1; ++k) {
     const int n = cdiv_d(p.slot[k].d_out, kEN);
-    if (q < n) break;
-    q -= n;
+    if (kc < n) break;
+    kc -= n;
   }
   e.k = k;
   e.nch = cdiv_d(p.slot[k].d_out, kEN);
-  e.c = q;
-  e.valid = e.m < e.mt && e.c < e.nch;
+  e.c = kc;
+  e.valid = e.nm > 0 && e.c < e.nch;
 }
 
-// Advances to the next item; returns true when it starts a new (tile, slot) unit.
-__device__ __forceinline__ bool ecur_next(const SgmvParams& p, ECur& e) {
-  if (++e.c < e.nch) return false;
+// Advances to the next item; returns 0 (same B chunk), 1 (new chunk, same
+// t rows) or 2 (new t rows: another slot or tile group).
+__device__ __forceinline__ int ecur_next(const SgmvParams& p, ECur& e) {
+  if (++e.i < e.nm) return 0;
+  e.i = 0;
+  if (++e.c < e.nch) return 1;
   e.c = 0;
-  if (++e.k == p.n_slots) {
-    e.k = 0;
-    if (++e.m == e.mt) {
-      e.m = 0;
-      do {
-        ++e.s;
-      } while (e.s < p.S && seg_tiles(p, e.s) == 0);
-      e.valid = e.s < p.S;
-      if (e.valid) e.mt = seg_tiles(p, e.s);
-    }
+  if (++e.k < p.n_slots) {
+    e.nch = cdiv_d(p.slot[e.k].d_out, kEN);
+    return 2;
   }
-  e.nch = cdiv_d(p.slot[e.k].d_out, kEN);
-  return true;
+  e.k = 0;
+  e.nch = cdiv_d(p.slot[0].d_out, kEN);
+  const int PS = p.e_pair;
+  if ((++e.g) * PS < e.mt) {
+    e.nm = min(PS, e.mt - e.g * PS);
+    return 2;
+  }
+  e.g = 0;
+  do {
+    ++e.s;
+  } while (e.s < p.S && seg_tiles(p, e.s) == 0);
+  e.valid = e.s < p.S;
+  if (e.valid) {
+    e.mt = seg_tiles(p, e.s);
+    e.nm = min(PS, e.mt);
+  }
+  return 2;
 }
 
 template <int DT>
@@ -600,12 +628,11 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
   __shared__ uint32_t tmem_slot;
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NB = p.e_nb, NY = p.e_ny;
+  const int NB = p.e_nb, NY = p.e_ny, PS = p.e_pair;
   const int t_half = p.e_t_half;   // bytes of one t half (hi or lo)
   const int b_stage = p.e_b_stage;
-  unsigned char* t_hi = smem;
-  unsigned char* t_lo = smem + t_half;
-  unsigned char* bring = smem + 2 * t_half;
+  unsigned char* tbuf = smem;      // PS tiles of (hi, lo)
+  unsigned char* bring = smem + PS * 2 * t_half;
   unsigned char* yring = bring + NB * b_stage;
 
   if (tid == 0) {
@@ -640,10 +667,12 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
   bool ok = true;
 
   if (n_items > 0 && warp == 0) {
-    // ---------------- producer
+    // ---------------- producer: a B chunk per run of items (gather4 from the
+    // pages, MN-major atoms of 8 ranks x 64 outputs), a y tile per item (two
+    // tiled TMA boxes)
     ECur e;
     ecur_init(p, i0, e);
-    int issued = 0;
+    int issued = 0, runs = 0, code = 2;
     const uint64_t pol_y = policy_evict_first(), pol_b = policy_evict_last();
     for (int j = 0; j < n_items && ok; ++j) {
       if (!e.valid) {
@@ -652,51 +681,56 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
         break;
       }
       const SlotDev& L = p.slot[e.k];
-      const int a = p.plan.seg_adapter[e.s], r = p.plan.seg_rank[e.s];
-      const int r16 = (r + 15) & ~15;
       const int n0 = e.c * kEN;
-      const int row0 = p.plan.seg_start[e.s] + e.m * kBM;
-      // pool rows of this lane's gathers (issued before the waits: latency overlap)
-      int rr[2][4];
+      if (code > 0) {  // a new B chunk
+        const int a = p.plan.seg_adapter[e.s], r = p.plan.seg_rank[e.s];
+        const int r16 = (r + 15) & ~15;
+        int rr[2][4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
+        for (int i = 0; i < 2; ++i) {
+          const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int kr = 4 * kq + u, col = n0 + cn * 64;
-          rr[i][u] = (g < r16 / 2 && kr < r && col < L.d_out)
-                         ? pool_row(p.pool, a, L.listB, (int64_t)kr * L.d_out + col)
-                         : (int)p.pool_rows;
+          for (int u = 0; u < 4; ++u) {
+            const int kr = 4 * kq + u, col = n0 + cn * 64;
+            rr[i][u] = (g < r16 / 2 && kr < r && col < L.d_out)
+                           ? pool_row(p.pool, a, L.listB, (int64_t)kr * L.d_out + col)
+                           : (int)p.pool_rows;
+          }
         }
+        const int bs = runs % NB;
+        if (runs >= NB) ok = bar_wait(&b_empty[bs], ((runs / NB) - 1) & 1, p.pool.err);
+        if (!ok) break;
+        unsigned char* bt = bring + bs * b_stage;
+        if (lane == 0) bar_expect(&b_full[bs], (uint32_t)r16 * (kEN * 2));
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
+          if (g < r16 / 2)
+            tma_gather4_hint(bt + ((4 * kq) >> 3) * 2048 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[i][0],
+                             rr[i][1], rr[i][2], rr[i][3], &b_full[bs], pol_b);
+        }
+        ++runs;
       }
-      const int bs = j % NB, ys = j % NY;
-      if (j >= NB) ok = bar_wait(&b_empty[bs], ((j / NB) - 1) & 1, p.pool.err);
-      if (ok && j >= NY) ok = bar_wait(&y_empty[ys], ((j / NY) - 1) & 1, p.pool.err);
+      const int ys = j % NY;
+      if (j >= NY) ok = bar_wait(&y_empty[ys], ((j / NY) - 1) & 1, p.pool.err);
       if (!ok) break;
-      unsigned char* bt = bring + bs * b_stage;
-      unsigned char* yt = yring + ys * kYTileBytes;
       if (lane == 0) {
+        unsigned char* yt = yring + ys * kYTileBytes;
+        const int row0 = p.plan.seg_start[e.s] + (e.g * PS + e.i) * kBM;
         const bool two = n0 + 64 < L.d_out;  // no box lies wholly past d_out
-        bar_expect(&b_full[bs], (uint32_t)r16 * (kEN * 2));
         bar_expect(&y_full[ys], (uint32_t)(two ? kYTileBytes : kYTileBytes / 2));
         tma_tile_2d_hint(yt, &p.ymap[e.k], n0, row0, &y_full[ys], pol_y);
         if (two) tma_tile_2d_hint(yt + kYTileBytes / 2, &p.ymap[e.k], n0 + 64, row0, &y_full[ys], pol_y);
       }
       __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int g = lane + 32 * i, kq = g >> 1, cn = g & 1;
-        if (g < r16 / 2)
-          tma_gather4_hint(bt + ((4 * kq) >> 3) * 2048 + cn * 1024 + ((4 * kq) & 7) * 128, &p.poolmap, rr[i][0],
-                           rr[i][1], rr[i][2], rr[i][3], &b_full[bs], pol_b);
-      }
       ++issued;
-      ecur_next(p, e);
+      code = ecur_next(p, e);
     }
     // every copy issued must land before the CTA may exit (the last phase of
     // each ring stage is not re-armed, so these waits see their own copies)
     if (lane == 0) {
-      for (int j = max(0, issued - NB); j < issued; ++j) bar_wait(&b_full[j % NB], (j / NB) & 1, p.pool.err);
+      for (int j = max(0, runs - NB); j < runs; ++j) bar_wait(&b_full[j % NB], (j / NB) & 1, p.pool.err);
       for (int j = max(0, issued - NY); j < issued; ++j) bar_wait(&y_full[j % NY], (j / NY) & 1, p.pool.err);
     }
   } else if (n_items > 0 && warp == 1) {
@@ -704,22 +738,26 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
     if (lane == 0) {
       ECur e;
       ecur_init(p, i0, e);
-      int unit = 0;
+      int unit = 0, runs = 0, bs = 0, code = 2;  // bs: B slot of the current run
       const uint32_t id = idesc_f16(p.dtype, kEN, 1);
-      const uint32_t sh = su32(t_hi), sl = su32(t_lo);
       for (int j = 0; j < n_items && ok; ++j) {
         if (!e.valid) break;
         const int r16 = (p.plan.seg_rank[e.s] + 15) & ~15;
-        const int bs = j % NB, as = j % kAcc;
-        if (j == 0 || e.c == 0) {
+        const int as = j % kAcc;
+        if (code == 2) {  // new t rows
           ok = bar_wait(&t_full, unit & 1, p.pool.err);
           ++unit;
         }
-        if (ok) ok = bar_wait(&b_full[bs], (j / NB) & 1, p.pool.err);
+        if (ok && code > 0) {  // new B chunk
+          bs = runs % NB;
+          ok = bar_wait(&b_full[bs], (runs / NB) & 1, p.pool.err);
+          ++runs;
+        }
         if (ok && j >= kAcc) ok = bar_wait(&a_empty[as], ((j / kAcc) - 1) & 1, p.pool.err);
         if (!ok) break;
         tc_fence_after();
         const uint32_t sb = su32(bring + bs * b_stage);
+        const uint32_t sh = su32(tbuf + e.i * 2 * t_half), sl = sh + t_half;
         const uint32_t acc = tmem + as * kEN;
         for (int q = 0; q < r16 / 16; ++q)
           mma_f16(acc, sdesc(sh + (q >> 2) * (kBM * 128) + (q & 3) * 32, 16, 1024), sdesc(sb + q * 4096, 1024, 2048),
@@ -727,9 +765,9 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
         for (int q = 0; q < r16 / 16; ++q)
           mma_f16(acc, sdesc(sl + (q >> 2) * (kBM * 128) + (q & 3) * 32, 16, 1024), sdesc(sb + q * 4096, 1024, 2048),
                   id, 1u);
-        mma_commit(&b_empty[bs]);
         mma_commit(&a_full[as]);
-        ecur_next(p, e);
+        code = ecur_next(p, e);
+        if (code > 0 || j == n_items - 1) mma_commit(&b_empty[bs]);  // the run's last item
       }
       // all MMAs complete before TMEM is released
       mma_commit(&fin);
@@ -746,6 +784,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
     const uint64_t pol_y = policy_evict_first();
     ECur e;
     ecur_init(p, i0, e);
+    int code = 2;
     for (int j = 0; j < n_items && ok; ++j) {
       if (!e.valid) break;
       const SlotDev& L = p.slot[e.k];
@@ -753,18 +792,22 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
       const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
       const int r16 = (r + 15) & ~15;
       const int seg1 = p.plan.seg_end[s];
-      const int row0 = p.plan.seg_start[s] + e.m * kBM;
-      const int token = row0 + mrow;
-      const bool valid = token < seg1;
+      const int row0 = p.plan.seg_start[s] + (e.g * PS + e.i) * kBM;
+      const bool valid = row0 + mrow < seg1;
       const int n0 = e.c * kEN;
-      if (j == 0 || e.c == 0) {
-        // new unit: t rows of slot k as hi / lo halves, K-major 128-byte swizzle.
-        // The previous unit's MMAs are complete: this thread waited on the
-        // accumulator of its last item, committed after them.
+      // new unit: the t rows of slot k for each tile of the group, as hi / lo
+      // halves, K-major 128-byte swizzle (tile i into t buffer i).  The previous
+      // unit's MMAs are complete: this thread waited on the accumulator of its
+      // last item, committed after them.
+      for (int ti = 0; ti < (code == 2 ? e.nm : 0); ++ti) {
+        unsigned char* t_hi = tbuf + ti * 2 * t_half;
+        unsigned char* t_lo = t_hi + t_half;
+        const int token = p.plan.seg_start[s] + (e.g * PS + ti) * kBM + mrow;
+        const bool tvalid = token < seg1;
         const float* trow = p.t + (int64_t)e.k * p.t_slot_stride + (int64_t)token * p.t_ld;
         for (int k0 = half * 8; k0 < r16; k0 += 16) {
           float v[8];
-          if (valid) {
+          if (tvalid) {
             const float4 f0 = *reinterpret_cast<const float4*>(trow + k0);
             const float4 f1 = *reinterpret_cast<const float4*>(trow + k0 + 4);
             v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
@@ -786,6 +829,8 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
           *reinterpret_cast<uint4*>(t_hi + off) = h;
           *reinterpret_cast<uint4*>(t_lo + off) = l;
         }
+      }
+      if (code == 2) {
         fence_async_smem();
         __syncwarp();
         if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&t_full)) : "memory");
@@ -850,7 +895,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
       fence_async_smem();  // generic-proxy writes of the slot before the next TMA fill
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&y_empty[ys])) : "memory");
-      ecur_next(p, e);
+      code = ecur_next(p, e);
     }
   }
   tc_fence_before();
@@ -992,15 +1037,23 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   // expand shared memory: t hi + lo, NB B stages, NY y tiles (deepest rings that fit)
   p.e_t_half = ((r16max + 63) / 64) * (kBM * 128);
   p.e_b_stage = r16max * (kEN * 2);
-  p.e_nb = 4;
-  p.e_ny = 4;
+  // deepest rings that fit, preferring tile pairs (one B gather for two
+  // tiles) with 4 y tiles, then single tiles with as deep rings as fit
   const size_t smem_cap = 227 * 1024 - 1024;  // dynamic budget minus static barriers
   auto esmem = [&] {
-    return 2 * (size_t)p.e_t_half + (size_t)p.e_nb * p.e_b_stage + (size_t)p.e_ny * kYTileBytes + 1024;
+    return (size_t)p.e_pair * 2 * p.e_t_half + (size_t)p.e_nb * p.e_b_stage + (size_t)p.e_ny * kYTileBytes + 1024;
   };
-  while (esmem() > smem_cap && (p.e_nb > 2 || p.e_ny > 2)) {
-    if (p.e_ny > p.e_nb) --p.e_ny;
-    else --p.e_nb;
+  p.e_pair = 2;
+  p.e_nb = 2;
+  p.e_ny = 4;
+  if (esmem() > smem_cap) {
+    p.e_pair = 1;
+    p.e_nb = 4;
+    p.e_ny = 4;
+    while (esmem() > smem_cap && (p.e_nb > 2 || p.e_ny > 2)) {
+      if (p.e_ny > p.e_nb) --p.e_ny;
+      else --p.e_nb;
+    }
   }
   if (esmem() > smem_cap) return cudaErrorNotSupported;
   const size_t shrink_smem = (size_t)p.stages * stage_bytes + 1024;
