@@ -76,6 +76,7 @@ struct SgmvParams {
   int ntot_max;         // max over groups of round_up(n * max_rank, 16)
   int stages;           // shrink pipeline depth
   int s_mq;             // shrink: 128-token tiles per item (share each A stage)
+  int s_gorder[kMaxSlots];  // shrink: group indices, most expensive first
   int dtype;
   CUtensorMap ymap[kMaxSlots];  // per slot: y as (d_out, T) with 64 x 128 boxes
   int e_nb, e_ny;       // expand ring depths (B chunks, y tiles)
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
       else r = p.pool.rank[a];
     }
     const int mt = (r > 0 && n > 0) ? cdiv_d(n, kBM) : 0;
-    csh += cdiv_d(mt, p.s_mq) * p.n_groups;
+    csh += cdiv_d(mt, p.s_mq);
     int ex = 0;
     for (int k = 0; k < p.n_slots; ++k) ex += cdiv_d(p.slot[k].d_out, kEN);
     cex += mt * ex;
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
     p.plan.seg_rank[s] = mt > 0 ? r : 0;
     p.plan.shrink_prefix[s] = bsh;
     p.plan.expand_prefix[s] = bex;
-    bsh += cdiv_d(mt, p.s_mq) * p.n_groups;
+    bsh += cdiv_d(mt, p.s_mq);
     int ex = 0;
     for (int k = 0; k < p.n_slots; ++k) ex += cdiv_d(p.slot[k].d_out, kEN);
     bex += mt * ex;
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(1024) k_sgmv_plan(const __grid_constant__ Sgmv
   if (tid == 0) {
     p.plan.shrink_prefix[S] = tsh;
     p.plan.expand_prefix[S] = tex;
-    p.plan.meta[0] = tsh;
+    p.plan.meta[0] = tsh * p.n_groups;  // items: groups (most expensive first) x tile pairs
     p.plan.meta[1] = tex;
   }
 }
@@ -333,19 +334,24 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
     gd_launch();
     return;
   }
+  // items run group-major, the groups in descending cost (so the longest items
+  // start first and the last wave is short), then over segments' tile pairs
   const int S = p.S;
-  const int s = find_ge(p.plan.shrink_prefix, S, item);
-  const int q = item - p.plan.shrink_prefix[s];
+  const int per_group = p.plan.shrink_prefix[S];
+  const int g = p.s_gorder[item / per_group];
+  const int qi = item % per_group;
+  const int s = find_ge(p.plan.shrink_prefix, S, qi);
+  const int q = qi - p.plan.shrink_prefix[s];
   const int seg0 = p.plan.seg_start[s], seg1 = p.plan.seg_end[s];
   const int mt = cdiv_d(seg1 - seg0, kBM);
   const int MQ = p.s_mq;
   const int mtq = cdiv_d(mt, MQ);
-  if (mt <= 0 || q >= mtq * p.n_groups || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
+  if (mt <= 0 || q >= mtq || seg0 < 0 || seg1 > p.T) {  // inconsistent plan: record, do nothing
     if (threadIdx.x == 0) rec_err(p.pool.err, 7, item);
     gd_launch();
     return;
   }
-  const int g = q / mtq, m = (q % mtq) * MQ;  // first tile of this item
+  const int m = q * MQ;  // first tile of this item
   const int nq = min(MQ, mt - m);             // tiles of this item (share each A stage)
   const int a = p.plan.seg_adapter[s], r = p.plan.seg_rank[s];
   const GroupDev& G = p.group[g];
@@ -1000,6 +1006,15 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   if (ntot > 512) return cudaErrorNotSupported;
   p.ntot_max = ntot;
   p.s_mq = 2 * ntot <= 512 ? 2 : 1;  // two accumulators of NT columns fit in TMEM
+  {  // shrink group order: descending bytes per item (X tiles + A rows over d_in)
+    int ord[kMaxSlots];
+    for (int g = 0; g < p.n_groups; ++g) ord[g] = g;
+    auto cost = [&](int g) {
+      return (int64_t)p.group[g].d_in * (p.s_mq * kBM + p.group[g].n * bp.pool.max_rank);
+    };
+    std::stable_sort(ord, ord + p.n_groups, [&](int x, int y) { return cost(x) > cost(y); });
+    for (int g = 0; g < p.n_groups; ++g) p.s_gorder[g] = ord[g];
+  }
   const int stage_bytes = p.s_mq * kXTileBytes + ((ntot * 128 + 1023) & ~1023);
   p.stages = std::min(8, (225 * 1024) / stage_bytes);
   if (p.stages < 2) return cudaErrorNotSupported;
