@@ -6,16 +6,17 @@
 // uniform bands to keep tensor-core alignment).  Per segment the delta is two
 // small GEMMs:
 //   shrink  t[128 x R] = X[128 x d_in] . A_t^T      (R = projections x rank)
-//   expand  y[128 x 256] += s * t[128 x r] . B[r x 256]
+//   expand  y[128 x 128] += s * t[128 x r] . B[r x 128]
 // with fp32 accumulators in tensor memory (TMEM).
 //
 // Operands in shared memory use the 128-byte-swizzled canonical layouts:
-//   * X tiles come from an ordinary tiled TMA load (box 64 x 128);
-//   * adapter rows live in scattered pages.  The pool is viewed as a 2-D
-//     tensor of 64-element rows, and TMA tile::gather4 fetches four such rows
-//     (any four pool rows) per instruction, so page-scattered A rows (K-major)
-//     and B rows (MN-major atoms of 8 ranks x 64 outputs) land directly in
-//     the swizzled layout the MMA reads;
+//   * X tiles and y tiles come from ordinary tiled TMA loads (64 x 128 boxes);
+//   * adapter rows live in scattered pages.  Shrink: the A rows of a stage are
+//     copied with per-thread 16-byte cp.async straight into the swizzled
+//     K-major layout (by the warps that later run the epilogue).  Expand: the
+//     pool is viewed as a 2-D tensor of 64-element rows and TMA tile::gather4
+//     fetches four such rows (any four pool rows) per instruction into
+//     MN-major atoms of 8 ranks x 64 outputs;
 //   * t enters the expand as two 16-bit halves, t = hi + lo with hi = RN(t),
 //     lo = RN(t - hi); both products with B are exact in fp32, so the
 //     intermediate keeps about twice the 16-bit precision.
@@ -119,21 +120,6 @@ __device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, int32_t* 
       }
     }
   }
-}
-__device__ __forceinline__ void tma_tile_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* b) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          su32(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(su32(b))
-      : "memory");
-}
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int r0, int r1, int r2, int r3,
-                                            uint64_t* b) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(su32(dst)),
-      "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(su32(b))
-      : "memory");
 }
 // L2 eviction-priority policies: streamed operands (X, y) go first, adapter
 // rows re-read by every token tile stay.
