@@ -307,11 +307,13 @@ def run_ours(args, rank, world):
     clocks = ClockSampler(dev)
     clocks.start()
     t_step = 0.0
+    per_step = []
     for _ in range(args.steps):
         prep()
         R.step(stream, outer)
         outer[1].synchronize()
-        t_step += outer[0].elapsed_time(outer[1])
+        per_step.append(outer[0].elapsed_time(outer[1]))
+        t_step += per_step[-1]
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
@@ -320,6 +322,19 @@ def run_ours(args, rank, world):
     K = args.steps
     ms = t_step / K
     value = job_throughput(world, w.T, K, t_step)
+    ms_median = max_over_ranks(float(np.median(per_step)), world, "cuda")
+
+    # warm L2: the same steps without the flush (y still reset before each)
+    Kw = min(K, 500)
+    t_warm = 0.0
+    for _ in range(Kw):
+        R.ten.reset()
+        R.step(stream, outer)
+        outer[1].synchronize()
+        t_warm += outer[0].elapsed_time(outer[1])
+    t_warm = max_over_ranks(t_warm, world, "cuda")
+    warm = {"value": job_throughput(world, w.T, Kw, t_warm), "ms_per_step": t_warm / Kw, "steps": Kw,
+            "l2": "not flushed between steps"}
 
     # end to end through the C ABI with host buffers (pinned): every step copies
     # its x, y and batch description in from pinned host memory and its y back
@@ -393,7 +408,8 @@ def run_ours(args, rank, world):
     tflops = alg["flops"] / (ms / 1e3) / 1e12
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": ms, "ms_per_step_median": ms_median,
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": W.DTYPE_NAME[w.dtype],
         "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(d_in)) A, N(0,1/sqrt(r)) B; "
                 "Zipf or uniform adapter ids)",
@@ -411,6 +427,7 @@ def run_ours(args, rank, world):
                           "tensor_tflops": tflops, "tensor_frac_of_bf16_peak": tflops / tc,
                           "kernel_ms": dict(zip(names, kt))},
         "e2e": e2e,
+        "warm_l2": warm,
         "gpu_launches": (4 if args.config == 3 else 3) * K,
         "clocks": clk,
     }
@@ -572,10 +589,22 @@ def cpu_baseline(w: W.Workload, budget_s=10.0):
         oracle_step(w, None, threads)
         n_steps += 1
     dt = time.perf_counter() - t0
+    # the same loops on one host thread, over a token subset sized to ~3 s
+    t1 = time.perf_counter()
+    n1 = 0
+    rng = np.random.default_rng(0)
+    while time.perf_counter() - t1 < 3.0 and n1 < w.T:
+        tok = np.sort(rng.choice(w.T, size=min(8, w.T), replace=False))
+        oracle_step(w, tok, 1)
+        n1 += tok.size
+    d1 = time.perf_counter() - t1
     return {"value": n_steps * toks / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{n_steps} whole step(s) of {w.name} ({toks} tokens x {len(w.projs)} "
                       f"projections each), fp64 loops, {threads} threads",
-            "seconds": dt}
+            "seconds": dt,
+            "single_thread": {"value": n1 / d1, "unit": UNIT, "cores": 1,
+                              "sample": f"{n1} tokens of the same workload (all {len(w.projs)} "
+                                        f"projections), fp64 loops, 1 thread", "seconds": d1}}
 
 
 def run_reference(args, rank, world):
