@@ -81,7 +81,7 @@ struct SgmvParams {
   int dtype;
   CUtensorMap ymap[kMaxSlots];  // per slot: y as (d_out, T) with 64 x 128 boxes
   int e_nb, e_ny;       // expand ring depths (B chunks, y tiles)
-  int e_pair;           // expand: 128-token tiles per group (one B gather serves them)
+  int e_pair;           // expand: 128-token tiles per group (1, 2 or 4; one B gather serves them)
   int e_t_half;         // expand: bytes of one t half in shared memory
   int e_b_stage;        // expand: bytes of one B ring stage
 };
@@ -1038,24 +1038,21 @@ cudaError_t launch_sgmv(const BgmvParams& bp, int dtype, const int32_t* seg_star
   // expand shared memory: t hi + lo, NB B stages, NY y tiles (deepest rings that fit)
   p.e_t_half = ((r16max + 63) / 64) * (kBM * 128);
   p.e_b_stage = r16max * (kEN * 2);
-  // deepest rings that fit, preferring tile pairs (one B gather for two
-  // tiles) with 4 y tiles, then single tiles with as deep rings as fit
+  // the largest tile group that fits (one B gather serves the group's tiles;
+  // measured: 4 tiles with 2 y stages beat 2 tiles with 4), then the deepest
+  // y ring that fits
   const size_t smem_cap = 227 * 1024 - 1024;  // dynamic budget minus static barriers
   auto esmem = [&] {
     return (size_t)p.e_pair * 2 * p.e_t_half + (size_t)p.e_nb * p.e_b_stage + (size_t)p.e_ny * kYTileBytes + 1024;
   };
-  p.e_pair = 2;
-  p.e_nb = 2;
-  p.e_ny = 4;
-  if (esmem() > smem_cap) {
-    p.e_pair = 1;
-    p.e_nb = 4;
-    p.e_ny = 4;
-    while (esmem() > smem_cap && (p.e_nb > 2 || p.e_ny > 2)) {
-      if (p.e_ny > p.e_nb) --p.e_ny;
-      else --p.e_nb;
+  bool fits = false;
+  for (int pair = 4; pair >= 1 && !fits; pair >>= 1)
+    for (int ny = 4; ny >= 2 && !fits; --ny) {
+      p.e_pair = pair;
+      p.e_nb = 2;
+      p.e_ny = ny;
+      fits = esmem() <= smem_cap;
     }
-  }
   if (esmem() > smem_cap) return cudaErrorNotSupported;
   const size_t shrink_smem = (size_t)p.stages * stage_bytes + 1024;
   const size_t expand_smem = esmem();
