@@ -115,6 +115,80 @@ __device__ __forceinline__ bool counter_wait(const int* c, int target, int32_t* 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Task schedule of the persistent CTAs.  The first rounds are static: CTA b
+// takes tasks b, b + G, b + 2G, ... (G = gridDim.x) for m_static tasks; the
+// rest, the last tenth of the rounds but at least two, are claimed from a
+// global counter, so that CTAs that drew cheaper tasks take more of them and
+// all finish close together.  The kProd producer warps each walk the CTA's
+// whole (task, stage) sequence: the first warp to reach a dynamic CTA-local
+// ordinal n claims its task with one atomicAdd and publishes the index in
+// slot n % kTix, the others read it there.  The walking cursors stay within
+// 3 kProd stage positions of one another (a producer cannot issue a stage
+// before the ring slot it reuses has been consumed), so a slot is never
+// reused before every warp has read it.
+constexpr int kTix = 32;
+static_assert(3 * kProd < kTix, "claim slots");
+struct TaskClaims {
+  int next;       // next dynamic ordinal to claim
+  int m_static;   // static ordinals per CTA
+  int ord[kTix];  // ordinal published in each slot
+  int id[kTix];   // its task index
+};
+__device__ __forceinline__ int static_rounds(int total) {
+  const int rounds = total / (int)gridDim.x;
+  return max(0, rounds - max(2, rounds / 10));
+}
+// One thread, before the CTA barrier.
+__device__ __forceinline__ void claims_init(TaskClaims& C, int total) {
+  C.m_static = static_rounds(total);
+  C.next = C.m_static;
+  for (int i = 0; i < kTix; ++i) C.ord[i] = -1;
+}
+__device__ __forceinline__ int ld_volatile_s32(const int* a) {
+  int v;
+  asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(a)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_volatile_s32(int* a, int v) {
+  asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
+}
+
+// Task index of CTA-local ordinal n, for every lane of the calling warp (n
+// warp-uniform); -1 if the wait for its publication gave up (error recorded).
+__device__ __forceinline__ int task_of(TaskClaims& C, int n, int* counter, int32_t* err) {
+  if (n < C.m_static) return (int)blockIdx.x + n * (int)gridDim.x;
+  int id = -1;
+  if ((threadIdx.x & 31) == 0) {
+    const int slot = n % kTix;
+    if (atomicCAS(&C.next, n, n + 1) == n) {
+      id = C.m_static * (int)gridDim.x + atomicAdd(counter, 1);
+      st_volatile_s32(&C.id[slot], id);
+      __threadfence_block();
+      st_volatile_s32(&C.ord[slot], n);
+    } else {
+      long long t0 = -1;
+      for (uint32_t it = 0;; ++it) {
+        if (ld_volatile_s32(&C.ord[slot]) == n) {
+          __threadfence_block();
+          id = ld_volatile_s32(&C.id[slot]);
+          break;
+        }
+        if ((it & 63) == 0) {
+          const long long now = clock64();
+          if (t0 < 0) t0 = now;
+          else if (now - t0 > kWaitLimit) {
+            record_error(err, 4, (int)blockIdx.x);
+            break;
+          }
+        }
+        __nanosleep(32);
+      }
+    }
+  }
+  return __shfl_sync(FULL_MASK, id, 0);
+}
+
 // Bulk async copy global -> shared, completion counted on `bar`.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -223,6 +297,52 @@ __device__ int block_exscan(int v, int* total, int* sh) {
   return res;
 }
 
+// Exclusive block-wide prefix sums of four independent values at once; *tot
+// gets the four totals.  sh: 32 int4 of shared memory.
+__device__ int4 block_exscan4(int4 v, int4* tot, int4* sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int4 x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y0 = __shfl_up_sync(FULL_MASK, x.x, o), y1 = __shfl_up_sync(FULL_MASK, x.y, o);
+    const int y2 = __shfl_up_sync(FULL_MASK, x.z, o), y3 = __shfl_up_sync(FULL_MASK, x.w, o);
+    if (lane >= o) x = make_int4(x.x + y0, x.y + y1, x.z + y2, x.w + y3);
+  }
+  int4 ex = make_int4(__shfl_up_sync(FULL_MASK, x.x, 1), __shfl_up_sync(FULL_MASK, x.y, 1),
+                      __shfl_up_sync(FULL_MASK, x.z, 1), __shfl_up_sync(FULL_MASK, x.w, 1));
+  if (lane == 0) ex = make_int4(0, 0, 0, 0);
+  if (lane == 31) sh[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int4 s = lane < nw ? sh[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(FULL_MASK, s.x, o), y1 = __shfl_up_sync(FULL_MASK, s.y, o);
+      const int y2 = __shfl_up_sync(FULL_MASK, s.z, o), y3 = __shfl_up_sync(FULL_MASK, s.w, o);
+      if (lane >= o) s = make_int4(s.x + y0, s.y + y1, s.z + y2, s.w + y3);
+    }
+    sh[lane] = s;
+  }
+  __syncthreads();
+  const int4 wp = w ? sh[w - 1] : make_int4(0, 0, 0, 0);
+  *tot = sh[nw - 1];
+  __syncthreads();
+  return make_int4(wp.x + ex.x, wp.y + ex.y, wp.z + ex.z, wp.w + ex.w);
+}
+
+// Touch every 64-byte line of a kernel's parameter block once, so that the
+// first lookups that index its group and slot tables with runtime values do
+// not each wait on a constant-cache miss.  Runs before the grid dependency
+// resolves (or, in k_segments, beside the histogram reset).
+template <class Params>
+__device__ __forceinline__ void warm_params(const Params& p, int* sink) {
+  constexpr int kLines = (int)((sizeof(Params) + 63) / 64);
+  if ((int)threadIdx.x < kLines) {
+    const int v = reinterpret_cast<const int*>(&p)[threadIdx.x * 16];
+    if (v == 0x5a5a5a5a) *sink = v;  // keeps the load; the value is never used
+  }
+}
+
 // k_segments: one CTA of 1024 threads.  Dynamic smem: max_adapters ints.
 // Output: perm, segments (start, adapter, rank) and, per segment, the number
 // of shrink and expand tasks before it (prefix sums in segment-major order).
@@ -237,17 +357,24 @@ __device__ __forceinline__ void seg_task_counts(const BgmvParams& p, int n, int 
     for (int k = 0; k < p.n_slots; ++k) exp += nte * cdiv_i(p.slot[k].d_out, kELC);
 }
 
-__global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvParams p,
+// Histogram entries pack the adapter's token count (< 2^21) with its rank + 1
+// (bits 21 and up), so that the segment pass needs no second rank lookup.
+constexpr int kHistRankShift = 21;
+
+__global__ void __launch_bounds__(1024, 1) k_segments(const __grid_constant__ BgmvParams p,
                                                    const int32_t* __restrict__ idx, int T) {
   extern __shared__ int hist[];
-  __shared__ int sh[32];
+  __shared__ int4 sh[32];
+  __shared__ int sink;
   const int tid = threadIdx.x, nth = blockDim.x;
   const int MA = p.pool.max_adapters;
   const ScratchDev& sc = p.sc;
   griddep_launch();  // the next kernel may start its prologue; it waits for this grid
+  warm_params(p, &sink);
 
   for (int a = tid; a < MA; a += nth) hist[a] = 0;
   __syncthreads();
+  int key0 = -1;  // adapter of token tid when it is valid (the first scatter chunk)
   for (int i = tid; i < T; i += nth) {
     const int a = idx[i];
     if (a == -1) continue;
@@ -255,11 +382,14 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
       record_error(p.pool.err, 1, i);
       continue;
     }
-    if (p.pool.rank[a] < 0) {
+    const int r = p.pool.rank[a];
+    if (r < 0) {
       record_error(p.pool.err, 2, i);
       continue;
     }
+    atomicOr(&hist[a], (r + 1) << kHistRankShift);
     atomicAdd(&hist[a], 1);
+    if (i == tid) key0 = a;
   }
   __syncthreads();
 
@@ -267,27 +397,27 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
   // a contiguous range of segment indices.
   const int E = (MA + nth - 1) / nth;
   const int a0 = min(tid * E, MA), a1 = min(a0 + E, MA);
-  int cnt = 0, nseg = 0, c_shr = 0, c_exp = 0;
+  int4 c = make_int4(0, 0, 0, 0);  // tokens, segments, shrink tasks, expand tasks
   for (int a = a0; a < a1; ++a) {
-    const int n = hist[a];
-    if (n == 0) continue;
+    const int h = hist[a];
+    if (h == 0) continue;
+    const int n = h & ((1 << kHistRankShift) - 1), r = (h >> kHistRankShift) - 1;
     int x, z;
-    seg_task_counts(p, n, p.pool.rank[a], x, z);
-    cnt += n;
-    nseg += 1;
-    c_shr += x;
-    c_exp += z;
+    seg_task_counts(p, n, r, x, z);
+    c.x += n;
+    c.y += 1;
+    c.z += x;
+    c.w += z;
   }
-  int n_valid, S, t_shr, t_exp;
-  int cbase = block_exscan<false>(cnt, &n_valid, sh);
-  int sb = block_exscan<false>(nseg, &S, sh);
-  int b_shr = block_exscan<false>(c_shr, &t_shr, sh);
-  int b_exp = block_exscan<false>(c_exp, &t_exp, sh);
+  int4 tot;
+  const int4 base = block_exscan4(c, &tot, sh);
+  const int n_valid = tot.x, S = tot.y, t_shr = tot.z, t_exp = tot.w;
+  int cbase = base.x, sb = base.y, b_shr = base.z, b_exp = base.w;
   for (int a = a0; a < a1; ++a) {
-    const int n = hist[a];
+    const int h = hist[a];
     hist[a] = cbase;  // becomes the scatter cursor
-    if (n == 0) continue;
-    const int r = p.pool.rank[a];
+    if (h == 0) continue;
+    const int n = h & ((1 << kHistRankShift) - 1), r = (h >> kHistRankShift) - 1;
     int x, z;
     seg_task_counts(p, n, r, x, z);
     sc.seg_start[sb] = cbase;
@@ -308,6 +438,8 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
     sc.meta[kMetaValid] = n_valid;
     sc.meta[kMetaShrinkTotal] = t_shr;
     sc.meta[kMetaExpandTotal] = t_exp;
+    sc.meta[kMetaShrinkClaim] = 0;
+    sc.meta[kMetaExpandClaim] = 0;
   }
   __syncthreads();
 
@@ -315,13 +447,16 @@ __global__ void __launch_bounds__(1024) k_segments(const __grid_constant__ BgmvP
   const int lane = tid & 31, warp = tid >> 5;
   for (int c0 = 0; c0 < T; c0 += nth) {
     const int i = c0 + tid;
-    const int a = i < T ? idx[i] : -1;
-    const bool ok = a >= 0 && a < MA && p.pool.rank[a] >= 0;
-    const int key = ok ? a : -1;
+    int a = key0;
+    if (c0 > 0) {
+      a = i < T ? idx[i] : -1;
+      if (!(a >= 0 && a < MA && p.pool.rank[a] >= 0)) a = -1;
+    }
+    const bool ok = a >= 0;
     const int nw = min(32, (T - c0 + 31) >> 5);
     for (int w = 0; w < nw; ++w) {
       if (warp == w) {
-        const unsigned m = __match_any_sync(FULL_MASK, key);
+        const unsigned m = __match_any_sync(FULL_MASK, a);
         const int before = __popc(m & ((1u << lane) - 1));
         int cur = 0;
         if (ok) cur = hist[a];
@@ -468,7 +603,7 @@ struct STask {
 };
 static_assert(sizeof(STask) / 4 + 2 <= kDescInts, "descriptor too small");
 
-__device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView& V, int task, STask& t) {
+__device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView& V, int task, int ord, STask& t) {
   const int s = find_seg(V.prefix, V.S, task);
   int q = task - V.prefix[s];
   t.a = V.adapter[s];
@@ -493,22 +628,24 @@ __device__ __forceinline__ void decode_shrink(const BgmvParams& p, const SegView
   t.nrows = min(kRB, p.group[g].n * t.r - t.rg * kRB);
   t.nst = cdiv_i(t.nrows, kSRows);
   t.ntok = min(t.nt, t.n - t.tg * t.nt);
-  t.xb = ((task - (int)blockIdx.x) / (int)gridDim.x) & 1;  // CTA-local task count parity
+  t.xb = ord & 1;  // CTA-local task ordinal parity
 }
 
 struct SCursor {  // a point of the producer's (task, stage) sequence
   STask t;
-  int task, st;
+  int task, ord, st;  // task index, CTA-local task ordinal, stage
   bool valid;
 };
 
-__device__ __forceinline__ void scursor_next(const BgmvParams& p, const SegView& V, int total, SCursor& c) {
+__device__ __forceinline__ void scursor_next(const BgmvParams& p, const SegView& V, int total, TaskClaims& cl,
+                                             SCursor& c) {
   if (!c.valid) return;
   if (++c.st < c.t.nst) return;
   c.st = 0;
-  c.task += gridDim.x;
-  c.valid = c.task < total;
-  if (c.valid) decode_shrink(p, V, c.task, c.t);
+  ++c.ord;
+  c.task = task_of(cl, c.ord, p.sc.meta + kMetaShrinkClaim, p.pool.err);
+  c.valid = c.task >= 0 && c.task < total;
+  if (c.valid) decode_shrink(p, V, c.task, c.ord, c.t);
 }
 
 // Per-lane lookups of a shrink stage: entry e = lane + 32 u (u = 0, 1),
@@ -632,6 +769,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ __align__(8) uint64_t full[kSNS], empty[kSNS];
   __shared__ int xdone[2];  // consumer warps done with each x buffer (kCW per task)
+  __shared__ TaskClaims claims;
+  __shared__ int warm_sink;
   __shared__ int32_t desc[kSNS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* xbufs = smem + kSRingBytes;
@@ -644,24 +783,27 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
     xdone[0] = xdone[1] = 0;
     fence_mbar_init();
   }
+  warm_params(p, &warm_sink);
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaShrinkTotal];
   const SegView V = stage_segments(p.sc, S, true, segsm);
+  if (threadIdx.x == 0) claims_init(claims, total);
   __syncthreads();
   if (warp < kProd) {
     // producer `warp` issues the stages at positions warp, warp + kProd, ...
     // of the CTA's (task, stage) sequence, into ring slots of the same parity
     SCursor A, B, C;
-    A.task = blockIdx.x;
+    A.task = task_of(claims, 0, p.sc.meta + kMetaShrinkClaim, p.pool.err);
+    A.ord = 0;
     A.st = 0;
-    A.valid = A.task < total;
-    if (A.valid) decode_shrink(p, V, A.task, A.t);
-    for (int q = 0; q < warp; ++q) scursor_next(p, V, total, A);
+    A.valid = A.task >= 0 && A.task < total;
+    if (A.valid) decode_shrink(p, V, A.task, 0, A.t);
+    for (int q = 0; q < warp; ++q) scursor_next(p, V, total, claims, A);
     B = A;
-    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, B);
+    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, B);
     C = B;
-    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, C);
+    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, C);
     int32_t a0[2], a1, b0[2], b1;
     shrink_lookup(p, A, a0, a1);
     shrink_lookup(p, B, b0, b1);
@@ -674,7 +816,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
         eparity ^= 1u << ring;
       }
       if (A.st == 0) {  // the x buffer of CTA task n is free once tasks n - 2, n - 4, ... are consumed
-        const int n = (A.task - (int)blockIdx.x) / (int)gridDim.x;
+        const int n = A.ord;
         if (n >= 2) ok = counter_wait(&xdone[n & 1], kCW * (n >> 1), p.pool.err);
         if (!ok) break;
       }
@@ -685,7 +827,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
       shrink_lookup(p, C, b0, b1);
       A = B;
       B = C;
-      for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, C);
+      for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, C);
       ring = (ring + kProd) % kSNS;
       ++uses;
     }
@@ -759,7 +901,7 @@ struct ETask {
 };
 static_assert(sizeof(ETask) / 4 + 2 <= kDescInts, "descriptor too small");
 
-__device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView& V, int task, ETask& t) {
+__device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView& V, int task, int ord, ETask& t) {
   const int s = find_seg(V.prefix, V.S, task);
   int q = task - V.prefix[s];
   t.a = V.adapter[s];
@@ -779,23 +921,25 @@ __device__ __forceinline__ void decode_expand(const BgmvParams& p, const SegView
   t.lc = q / n_tg;
   t.nst = cdiv_i(t.r, kER);
   t.ntok = min(t.nt, t.n - t.tg * t.nt);
-  t.yb = ((task - (int)blockIdx.x) / (int)gridDim.x) & 1;  // CTA-local task count parity
+  t.yb = ord & 1;  // CTA-local task ordinal parity
   t.tok0 = t.tok1 = t.tok2 = t.tok3 = 0;
 }
 
 struct ECursor {
   ETask t;
-  int task, st;
+  int task, ord, st;
   bool valid;
 };
 
-__device__ __forceinline__ void ecursor_next(const BgmvParams& p, const SegView& V, int total, ECursor& c) {
+__device__ __forceinline__ void ecursor_next(const BgmvParams& p, const SegView& V, int total, TaskClaims& cl,
+                                             ECursor& c) {
   if (!c.valid) return;
   if (++c.st < c.t.nst) return;
   c.st = 0;
-  c.task += gridDim.x;
-  c.valid = c.task < total;
-  if (c.valid) decode_expand(p, V, c.task, c.t);
+  ++c.ord;
+  c.task = task_of(cl, c.ord, p.sc.meta + kMetaExpandClaim, p.pool.err);
+  c.valid = c.task >= 0 && c.task < total;
+  if (c.valid) decode_expand(p, V, c.task, c.ord, c.t);
 }
 
 // Per-lane lookups of an expand stage: entry e = lane + 32 u (u = 0, 1),
@@ -941,6 +1085,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ __align__(8) uint64_t full[kENS], empty[kENS];
   __shared__ int ydone[2];  // consumer warps done with each y buffer (kCW per task)
+  __shared__ TaskClaims claims;
+  __shared__ int warm_sink;
   __shared__ int32_t desc[kENS][kDescInts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned char* ybufs = smem + kERingBytes;
@@ -953,24 +1099,27 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
     ydone[0] = ydone[1] = 0;
     fence_mbar_init();
   }
+  warm_params(p, &warm_sink);
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaExpandTotal];
   const SegView V = stage_segments(p.sc, S, false, segsm);
+  if (threadIdx.x == 0) claims_init(claims, total);
   __syncthreads();
   if (warp < kProd) {
     // producer `warp` issues the stages at positions warp, warp + kProd, ...
     // of the CTA's (task, stage) sequence, into ring slots of the same parity
     ECursor A, B, C;
-    A.task = blockIdx.x;
+    A.task = task_of(claims, 0, p.sc.meta + kMetaExpandClaim, p.pool.err);
+    A.ord = 0;
     A.st = 0;
-    A.valid = A.task < total;
-    if (A.valid) decode_expand(p, V, A.task, A.t);
-    for (int q = 0; q < warp; ++q) ecursor_next(p, V, total, A);
+    A.valid = A.task >= 0 && A.task < total;
+    if (A.valid) decode_expand(p, V, A.task, 0, A.t);
+    for (int q = 0; q < warp; ++q) ecursor_next(p, V, total, claims, A);
     B = A;
-    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, B);
+    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, B);
     C = B;
-    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, C);
+    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, C);
     int32_t a0[2], a1, b0[2], b1;
     expand_lookup(p, A, a0, a1);
     expand_lookup(p, B, b0, b1);
@@ -982,7 +1131,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
         eparity ^= 1u << ring;
       }
       if (A.st == 0) {  // the y buffer of CTA task n is free once tasks n - 2, n - 4, ... are consumed
-        const int n = (A.task - (int)blockIdx.x) / (int)gridDim.x;
+        const int n = A.ord;
         if (n >= 2 && !counter_wait(&ydone[n & 1], kCW * (n >> 1), p.pool.err)) break;
       }
       expand_issue(p, A, a0, a1, smem + ring * kEStageBytes, ybufs + A.t.yb * kYBufBytes, desc[ring],
@@ -993,7 +1142,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
       expand_lookup(p, C, b0, b1);
       A = B;
       B = C;
-      for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, C);
+      for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, C);
       ring = (ring + kProd) % kENS;
       ++uses;
     }

@@ -74,6 +74,7 @@ struct ScratchDev {
 };
 
 enum MetaIdx { kMetaS = 0, kMetaValid = 1, kMetaShrinkTotal = 2, kMetaExpandTotal = 3,
+               kMetaShrinkClaim = 4, kMetaExpandClaim = 5,  // dynamic task counters
                kMetaCount = 16 };
 
 struct BgmvParams {
