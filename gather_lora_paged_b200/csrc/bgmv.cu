@@ -357,6 +357,29 @@ __device__ __forceinline__ void seg_task_counts(const BgmvParams& p, int n, int 
     for (int k = 0; k < p.n_slots; ++k) exp += nte * cdiv_i(p.slot[k].d_out, kELC);
 }
 
+// L2 hint for the page lists (A_t and B of every projection of the call) of
+// the adapters of tokens blockIdx.x and blockIdx.x + gridDim.x: warp w < 2
+// takes one token, lane 2k + h the list of projection k, half h.  Runs in a
+// persistent kernel's prologue, while k_segments builds the segment table;
+// idx and the pool tables are final by then (k_segments, which this kernel
+// follows, started only after all earlier work of the stream).
+__device__ __forceinline__ void prefetch_token_page_lists(const BgmvParams& p) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int i = (int)blockIdx.x + w * (int)gridDim.x;
+  if (w >= 2 || p.idx == nullptr || i >= p.T || lane >= 2 * p.n_slots) return;
+  const int a = p.idx[i];
+  if (a < 0 || a >= p.pool.max_adapters) return;
+  const int r = p.pool.rank[a];
+  if (r <= 0) return;
+  const SlotDev& L = p.slot[lane >> 1];
+  const int h = lane & 1;
+  const int64_t np = ((int64_t)r * (h ? L.d_out : L.d_in) + (1ll << p.pool.page_shift) - 1) >> p.pool.page_shift;
+  const int32_t* row = p.pool.page_list + (int64_t)a * p.pool.list_stride + (h ? L.listB : L.listA);
+  const uintptr_t e = reinterpret_cast<uintptr_t>(row + np);
+  for (uintptr_t l = reinterpret_cast<uintptr_t>(row) & ~(uintptr_t)127; l < e; l += 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(l));
+}
+
 // Histogram entries pack the adapter's token count (< 2^21) with its rank + 1
 // (bits 21 and up), so that the segment pass needs no second rank lookup.
 constexpr int kHistRankShift = 21;
@@ -784,6 +807,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
     fence_mbar_init();
   }
   warm_params(p, &warm_sink);
+  prefetch_token_page_lists(p);
   griddep_wait();
   const int S = p.sc.meta[kMetaS];
   const int total = p.sc.meta[kMetaShrinkTotal];
@@ -793,19 +817,19 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
   if (warp < kProd) {
     // producer `warp` issues the stages at positions warp, warp + kProd, ...
     // of the CTA's (task, stage) sequence, into ring slots of the same parity
-    SCursor A, B, C;
+    SCursor A, B;
     A.task = task_of(claims, 0, p.sc.meta + kMetaShrinkClaim, p.pool.err);
     A.ord = 0;
     A.st = 0;
     A.valid = A.task >= 0 && A.task < total;
     if (A.valid) decode_shrink(p, V, A.task, 0, A.t);
     for (int q = 0; q < warp; ++q) scursor_next(p, V, total, claims, A);
-    B = A;
-    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, B);
-    C = B;
-    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, C);
+    // page ids of a position are looked up two of this warp's issues ahead;
+    // A's lookups are in flight while B is walked
     int32_t a0[2], a1, b0[2], b1;
     shrink_lookup(p, A, a0, a1);
+    B = A;
+    for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, B);
     shrink_lookup(p, B, b0, b1);
     uint32_t eparity = 0;
     int ring = warp % kSNS, uses = 0;
@@ -824,10 +848,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
       a0[0] = b0[0];
       a0[1] = b0[1];
       a1 = b1;
-      shrink_lookup(p, C, b0, b1);
       A = B;
-      B = C;
-      for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, C);
+      for (int q = 0; q < kProd; ++q) scursor_next(p, V, total, claims, B);
+      shrink_lookup(p, B, b0, b1);
       ring = (ring + kProd) % kSNS;
       ++uses;
     }
@@ -1109,19 +1132,19 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
   if (warp < kProd) {
     // producer `warp` issues the stages at positions warp, warp + kProd, ...
     // of the CTA's (task, stage) sequence, into ring slots of the same parity
-    ECursor A, B, C;
+    ECursor A, B;
     A.task = task_of(claims, 0, p.sc.meta + kMetaExpandClaim, p.pool.err);
     A.ord = 0;
     A.st = 0;
     A.valid = A.task >= 0 && A.task < total;
     if (A.valid) decode_expand(p, V, A.task, 0, A.t);
     for (int q = 0; q < warp; ++q) ecursor_next(p, V, total, claims, A);
-    B = A;
-    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, B);
-    C = B;
-    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, C);
+    // page ids of a position are looked up two of this warp's issues ahead;
+    // A's lookups are in flight while B is walked
     int32_t a0[2], a1, b0[2], b1;
     expand_lookup(p, A, a0, a1);
+    B = A;
+    for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, B);
     expand_lookup(p, B, b0, b1);
     uint32_t eparity = 0;
     int ring = warp % kENS, uses = 0;
@@ -1139,10 +1162,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
       a0[0] = b0[0];
       a0[1] = b0[1];
       a1 = b1;
-      expand_lookup(p, C, b0, b1);
       A = B;
-      B = C;
-      for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, C);
+      for (int q = 0; q < kProd; ++q) ecursor_next(p, V, total, claims, B);
+      expand_lookup(p, B, b0, b1);
       ring = (ring + kProd) % kENS;
       ++uses;
     }
@@ -1373,7 +1395,9 @@ static cudaError_t set_attrs() {
   return e;
 }
 
-cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cudaStream_t s) {
+cudaError_t launch_segments(BgmvParams& p, const int32_t* idx, int T, cudaStream_t s) {
+  p.idx = idx;
+  p.T = T;
   cudaError_t ea = set_attrs();
   if (ea != cudaSuccess) return ea;
   const size_t smem = sizeof(int) * (size_t)p.pool.max_adapters;

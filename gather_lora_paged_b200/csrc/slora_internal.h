@@ -85,6 +85,8 @@ struct BgmvParams {
   int n_groups;
   GroupDev group[kMaxSlots];
   int max_tokens;
+  const int32_t* idx;       // the call's adapter per token (set by launch_segments)
+  int T;
   int do_shrink, do_expand; // which phases this call plans
 };
 
@@ -111,7 +113,8 @@ struct PageInNew {
 };
 
 // Launchers (kernels.cu).  All return cudaGetLastError() of the launch.
-cudaError_t launch_segments(const BgmvParams& p, const int32_t* idx, int T, cudaStream_t s);
+// Also records idx and T in p, for the kernels launched after it.
+cudaError_t launch_segments(BgmvParams& p, const int32_t* idx, int T, cudaStream_t s);
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s);
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s);
 cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s);
