@@ -388,6 +388,7 @@ __global__ void __launch_bounds__(1024, 1) k_segments(const __grid_constant__ Bg
                                                    const int32_t* __restrict__ idx, int T) {
   extern __shared__ int hist[];
   __shared__ int4 sh[32];
+  __shared__ __align__(16) int ck[1024];  // keys of one scatter chunk
   __shared__ int sink;
   const int tid = threadIdx.x, nth = blockDim.x;
   const int MA = p.pool.max_adapters;
@@ -466,7 +467,10 @@ __global__ void __launch_bounds__(1024, 1) k_segments(const __grid_constant__ Bg
   }
   __syncthreads();
 
-  // Stable scatter: chunks of 1024 tokens, warps take turns in order.
+  // Stable scatter, one chunk of blockDim.x tokens at a time: a token's place
+  // among its adapter's tokens of the chunk is the number of equal keys in
+  // earlier warps (counted from the chunk's keys in shared memory) plus the
+  // number in earlier lanes of its own warp.
   const int lane = tid & 31, warp = tid >> 5;
   for (int c0 = 0; c0 < T; c0 += nth) {
     const int i = c0 + tid;
@@ -475,22 +479,21 @@ __global__ void __launch_bounds__(1024, 1) k_segments(const __grid_constant__ Bg
       a = i < T ? idx[i] : -1;
       if (!(a >= 0 && a < MA && p.pool.rank[a] >= 0)) a = -1;
     }
-    const bool ok = a >= 0;
-    const int nw = min(32, (T - c0 + 31) >> 5);
-    for (int w = 0; w < nw; ++w) {
-      if (warp == w) {
-        const unsigned m = __match_any_sync(FULL_MASK, a);
-        const int before = __popc(m & ((1u << lane) - 1));
-        int cur = 0;
-        if (ok) cur = hist[a];
-        __syncwarp();
-        if (ok) {
-          sc.perm[cur + before] = i;
-          if (before == 0) hist[a] = cur + __popc(m);
-        }
+    ck[tid] = a;
+    __syncthreads();
+    const unsigned m = __match_any_sync(FULL_MASK, a);
+    if (a >= 0) {
+      int before = __popc(m & ((1u << lane) - 1));
+      const int4* k4 = reinterpret_cast<const int4*>(ck);
+      for (int j = 0; j < warp * 8; ++j) {  // the 32 * warp keys of earlier warps
+        const int4 v = k4[j];
+        before += (v.x == a) + (v.y == a) + (v.z == a) + (v.w == a);
       }
-      __syncthreads();
+      sc.perm[hist[a] + before] = i;
     }
+    __syncthreads();  // every cursor read before the chunk's counts are added
+    if (a >= 0 && lane == __ffs(m) - 1) atomicAdd(&hist[a], __popc(m));
+    __syncthreads();
   }
 }
 
