@@ -8,10 +8,14 @@ device segment build, the grouped paged shrink and the grouped expand over
 all projections of one layer.  Default workload: the LLaMA-7B decode layer
 (7 projections, 256 tokens, 1000 resident rank-16 adapters, Zipf 1.0, fp16).
 
-Timing: CUDA events that the library records on the compute stream right
-around its own kernels (slora_set_phase_events), so per-kernel and per-step
-device times carry no host gaps.  L2 is flushed (a 256 MiB write) and y reset
-before every step, outside the timed events.  N > 1 (torchrun): every rank
+Timing: CUDA events on the compute stream right around the library's kernels
+(per kernel: events the library records between them, slora_set_phase_events;
+per step: events around the call).  L2 is flushed (a 256 MiB write) and y reset
+before every step, outside the timed events, and a spin kernel then holds the
+GPU for about 100 us, so that the host has enqueued the whole step before the
+start event is reached: the timed region holds the step's device work back to
+back, without the host's enqueue latency (Python marshalling and the library's
+planning), as when a serving loop runs ahead of the GPU.  N > 1 (torchrun): every rank
 runs an independent replica (no collective on the data path); the step time
 is the max over ranks (NCCL all-reduce of the timings only).
 
@@ -53,6 +57,10 @@ def peaks():
 # ---------------------------------------------------------------------------
 # DRAM traffic per launch from a committed ncu capture (profiles/traffic.json),
 # valid only while the kernel's source file is the one that was captured
+# GPU cycles of the spin kernel ahead of each timed step (about 100 us at the
+# B200's 1.965 GHz): longer than the host takes to enqueue one step.
+HOLD_CYCLES = 200_000
+
 KERNEL_SOURCE = {"shrink": "bgmv.cu", "expand": "bgmv.cu", "segments": "bgmv.cu",
                  "sgmv_shrink": "sgmv.cu", "sgmv_expand": "sgmv.cu"}
 
@@ -281,6 +289,7 @@ def run_ours(args, rank, world):
     def prep():
         R.ten.reset()
         flush.zero_()
+        torch.cuda._sleep(HOLD_CYCLES)
 
     for _ in range(args.warmup):
         prep()
@@ -329,6 +338,7 @@ def run_ours(args, rank, world):
     t_warm = 0.0
     for _ in range(Kw):
         R.ten.reset()
+        torch.cuda._sleep(HOLD_CYCLES)
         R.step(stream, outer)
         outer[1].synchronize()
         t_warm += outer[0].elapsed_time(outer[1])
@@ -416,6 +426,7 @@ def run_ours(args, rank, world):
         "config": {"workload": w.name, "tokens_per_step": w.T, "projections": len(w.projs),
                    "adapters": w.n_adapters, "touched_adapters": alg["touched"],
                    "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
+                   "host_enqueue": "not timed: a ~100 us spin kernel precedes each step's start event",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": names[i_dom], "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm,

@@ -118,7 +118,7 @@ __device__ __forceinline__ bool counter_wait(const int* c, int target, int32_t* 
 // ---------------------------------------------------------------------------
 // Task schedule of the persistent CTAs.  The first rounds are static: CTA b
 // takes tasks b, b + G, b + 2G, ... (G = gridDim.x) for m_static tasks; the
-// rest, the last tenth of the rounds but at least two, are claimed from a
+// rest, the last fifth of the rounds but at least two, are claimed from a
 // global counter, so that CTAs that drew cheaper tasks take more of them and
 // all finish close together.  The kProd producer warps each walk the CTA's
 // whole (task, stage) sequence: the first warp to reach a dynamic CTA-local
@@ -137,7 +137,7 @@ struct TaskClaims {
 };
 __device__ __forceinline__ int static_rounds(int total) {
   const int rounds = total / (int)gridDim.x;
-  return max(0, rounds - max(2, rounds / 10));
+  return max(0, rounds - max(2, rounds / 5));
 }
 // One thread, before the CTA barrier.
 __device__ __forceinline__ void claims_init(TaskClaims& C, int total) {
