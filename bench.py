@@ -541,6 +541,8 @@ def run_mixed(args, rank, world, w):
         sum(t.numel() * t.element_size() for t in hins)
     d2h = sum(t.numel() * 2 for t in hout)
 
+    pre = prefetch_leg(M, w, stream)
+
     peak_pcie = pcie_h2d_peak()
     hbm, tc, src = peaks()
     alg = algorithmic(w)
@@ -572,8 +574,53 @@ def run_mixed(args, rank, world, w):
                 "ms_per_step": tot / n_e2e},
         "gpu_launches": 8 * K,  # page-in gather, segments, shrink, expand, merge, plan, shrink, expand
         "clocks": clk,
+        "prefetch": pre,
     }
     M.close()
+    return out
+
+
+def prefetch_leg(M, w, stream):
+    """Two device-timed measurements of adapter prefetch, after the timed
+    steps (pool restored: cold adapters out, fillers in).
+    rare_adapter: one cold adapter of the largest rank paged in alone on the
+    side stream (its copy time: what a request for a rare adapter waits).
+    prefetched_step: the step with its cold adapters prefetched beforehand
+    (while a step that names only the warm set is current, so the fillers are
+    older and may be evicted); its page-in then finds every adapter resident."""
+    import torch
+
+    import harness as H
+    G = H.G
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for e in (e0, e1):
+        e.record()  # torch creates the CUDA event on its first record
+    torch.cuda.synchronize()
+    a = int(M.cold[np.argmax(w.ranks[M.cold])])
+    e0.record(M.side)
+    G.slora_adapter_page_in(M.h, [a], M.side, e1)
+    e1.synchronize()
+    rare_ms = e0.elapsed_time(e1)
+    rare_bytes = int(w.ranks[a]) * sum(p.d_in + p.d_out for p in w.projs) * 2
+    G.slora_adapter_evict(M.h, a, stream)
+    back = [f for f in M.fillers if not G.slora_adapter_is_resident(M.h, f)]
+    G.slora_adapter_page_in(M.h, list(M.warm) + back, M.side)     # the "current" step
+    M.side.synchronize()
+    n = G.slora_adapter_prefetch(M.h, M.cold.tolist(), 1 << 40, M.side)
+    M.side.synchronize()
+    s0 = G.slora_pool_stats(M.h)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    M.ten.reset()
+    M.step(stream, ev[0], ev[1], ev[2])
+    ev[2].synchronize()
+    s1 = G.slora_pool_stats(M.h)
+    out = {"rare_adapter": {"id": a, "rank": int(w.ranks[a]), "bytes": rare_bytes, "ms": rare_ms,
+                            "gbs": rare_bytes / (rare_ms / 1e3) / 1e9},
+           "prefetched_adapters": n, "cold_adapters": int(M.cold.size),
+           "prefetched_step": {"ms": ev[0].elapsed_time(ev[2]), "pagein_ms": ev[0].elapsed_time(ev[1]),
+                               "hits": s1["hits"] - s0["hits"],
+                               "copied_bytes": s1["bytes_paged_in"] - s0["bytes_paged_in"]}}
+    M.restore(stream)
     return out
 
 

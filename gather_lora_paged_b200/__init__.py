@@ -44,7 +44,8 @@ class PoolDesc(ctypes.Structure):
 
 class PoolStats(ctypes.Structure):
     _fields_ = [(n, c_int64) for n in ("page_ins", "hits", "evictions", "bytes_paged_in",
-                                       "free_pages", "resident", "copy_calls", "epoch")]
+                                       "free_pages", "resident", "copy_calls", "epoch",
+                                       "prefetched", "bytes_prefetched")]
 
 
 _lib = None
@@ -69,6 +70,8 @@ def lib():
         "slora_pool_set_page_order": ([P, P, I64], I32),
         "slora_adapter_register": ([P, I32, I32, c_float, P, P], I32),
         "slora_adapter_page_in": ([P, P, I32, P, P], I32),
+        "slora_adapter_prefetch": ([P, P, I32, I64, P, P, POINTER(c_int32)], I32),
+        "slora_prefetch_candidates": ([P, ctypes.c_double, I32, P, POINTER(c_int32)], I32),
         "slora_adapter_evict": ([P, I32, P], I32),
         "slora_adapter_is_resident": ([P, I32, POINTER(c_int32)], I32),
         "slora_check_batch": ([P, P, I32], I32),
@@ -188,6 +191,24 @@ def slora_adapter_page_in(pool: int, ids, side_stream=None, done_event=None) -> 
     a = _arr(c_int32, [int(i) for i in ids])
     _check(pool, lib().slora_adapter_page_in(pool, ctypes.cast(a, c_void_p), len(ids),
                                              _stream(side_stream), _event(done_event)))
+
+
+def slora_adapter_prefetch(pool: int, ids, max_pages: int, side_stream=None, done_event=None) -> int:
+    """Returns the number of adapters whose copies were enqueued."""
+    a = _arr(c_int32, [int(i) for i in ids])
+    n_done = c_int32(0)
+    _check(pool, lib().slora_adapter_prefetch(pool, ctypes.cast(a, c_void_p), len(ids), int(max_pages),
+                                              _stream(side_stream), _event(done_event),
+                                              ctypes.byref(n_done)))
+    return n_done.value
+
+
+def slora_prefetch_candidates(pool: int, half_life: float, max_n: int) -> list:
+    out = (c_int32 * max(int(max_n), 1))()
+    n = c_int32(0)
+    _check(pool, lib().slora_prefetch_candidates(pool, float(half_life), int(max_n),
+                                                 ctypes.cast(out, c_void_p), ctypes.byref(n)))
+    return [int(out[i]) for i in range(n.value)]
 
 
 def slora_adapter_evict(pool: int, id: int, stream=None) -> None:

@@ -10,6 +10,7 @@
 //   dedicated streams overlapped with compute.
 #include <algorithm>
 #include <chrono>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -39,6 +40,8 @@ constexpr double kWaitSeconds = 30.0;
 int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+constexpr int kUseHistory = 32;  // page_in namings kept per adapter for the prefetch policy
+
 struct Adapter {
   bool registered = false;
   bool resident = false;
@@ -48,7 +51,10 @@ struct Adapter {
   const void* host_B[kMaxSlots] = {};
   const void* map_A[kMaxSlots] = {};  // device-usable addresses of the pinned copies
   const void* map_B[kMaxSlots] = {};
-  int64_t last_use = -1;
+  int64_t last_use = -1;       // LRU age: epoch of the last page_in naming it, or of its prefetch
+  int64_t named = -1;          // epoch of the last page_in naming it (compute may use it iff == epoch)
+  int64_t uses[kUseHistory];   // epochs of its most recent page_in namings (a ring)
+  int n_uses = 0;              // namings recorded so far
   std::vector<int32_t> pages;  // tensor order (p, A), (p, B)
 };
 
@@ -604,10 +610,17 @@ static void evict_one(slora_pool* P, int id) {
   P->st.evictions++;
 }
 
-slora_status_t slora_adapter_page_in(slora_pool* P, const int32_t* ids, int32_t n, void* side_stream,
-                                     void* done_event) {
+// Shared by page_in and prefetch.  page_in (prefetch = false): every id
+// becomes resident, evicting LRU adapters not named; the named set becomes
+// the step's set.  prefetch: the non-resident ids, in order, that fit in
+// max_pages (and in the free pages plus the pages of adapters older than the
+// current step) become resident; nothing the current step or an earlier
+// prefetch of this step holds is evicted, and the step's set is unchanged.
+static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n, void* side_stream,
+                                   void* done_event, bool prefetch, int64_t max_pages, int32_t* n_done) {
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (n < 0 || (n > 0 && !ids)) return P->fail(SLORA_ERR_INVALID_ARG, "ids");
+  if (prefetch && max_pages < 0) return P->fail(SLORA_ERR_INVALID_ARG, "max_pages < 0");
   cudaStream_t side = static_cast<cudaStream_t>(side_stream);
   std::vector<int> uniq;
   std::unordered_set<int> pinned;
@@ -619,21 +632,44 @@ slora_status_t slora_adapter_page_in(slora_pool* P, const int32_t* ids, int32_t 
   }
   std::vector<int> missing;
   int64_t need = 0;
-  for (int a : uniq)
-    if (!P->ad[a].resident) {
-      missing.push_back(a);
-      need += P->pages_for(P->ad[a].rank);
-    }
-  // LRU victims: oldest first, equal ages lower id first (std::set order)
   std::vector<int> victims;
-  int64_t avail = (int64_t)P->free_pages.size();
-  for (auto it = P->lru.begin(); avail < need && it != P->lru.end(); ++it) {
-    if (pinned.count(it->second)) continue;
-    victims.push_back(it->second);
-    avail += (int64_t)P->ad[it->second].pages.size();
+  if (!prefetch) {
+    for (int a : uniq)
+      if (!P->ad[a].resident) {
+        missing.push_back(a);
+        need += P->pages_for(P->ad[a].rank);
+      }
+    // LRU victims: oldest first, equal ages lower id first (std::set order)
+    int64_t avail = (int64_t)P->free_pages.size();
+    for (auto it = P->lru.begin(); avail < need && it != P->lru.end(); ++it) {
+      if (pinned.count(it->second)) continue;
+      victims.push_back(it->second);
+      avail += (int64_t)P->ad[it->second].pages.size();
+    }
+    if (avail < need)
+      return P->fail(SLORA_ERR_OOM, "cannot fit " + std::to_string(need) + " pages with all unpinned adapters evicted");
+  } else {
+    // evictable: resident adapters older than the current step (the step's
+    // set and this step's prefetches have last_use == epoch)
+    int64_t cap = (int64_t)P->free_pages.size();
+    for (const auto& e : P->lru)
+      if (e.first < P->epoch) cap += (int64_t)P->ad[e.second].pages.size();
+    const int64_t limit = std::min(cap, max_pages);
+    for (int a : uniq) {
+      if (P->ad[a].resident) continue;
+      const int64_t np = P->pages_for(P->ad[a].rank);
+      if (need + np > limit) continue;  // does not fit: try the next one
+      missing.push_back(a);
+      need += np;
+    }
+    int64_t avail = (int64_t)P->free_pages.size();
+    for (auto it = P->lru.begin(); avail < need && it != P->lru.end(); ++it) {
+      if (it->first >= P->epoch) break;  // std::set order: the rest are as new
+      victims.push_back(it->second);
+      avail += (int64_t)P->ad[it->second].pages.size();
+    }
   }
-  if (avail < need)
-    return P->fail(SLORA_ERR_OOM, "cannot fit " + std::to_string(need) + " pages with all unpinned adapters evicted");
+  if (n_done) *n_done = (int32_t)missing.size();
   if (P->inject_after >= 0 && !missing.empty()) {
     if (P->inject_after == 0) {
       P->inject_after = -1;
@@ -667,16 +703,30 @@ slora_status_t slora_adapter_page_in(slora_pool* P, const int32_t* ids, int32_t 
     }
     A.resident = true;
     P->st.page_ins++;
-    P->st.bytes_paged_in += 2 * (int64_t)A.rank *
+    (prefetch ? P->st.bytes_prefetched : P->st.bytes_paged_in) += 2 * (int64_t)A.rank *
         [&] { int64_t s = 0; for (int p = 0; p < P->d.n_proj; ++p) s += P->d.d_in[p] + P->d.d_out[p]; return s; }();
   }
-  P->st.hits += (int64_t)(uniq.size() - missing.size());
-  P->epoch++;
-  for (int a : uniq) {
-    Adapter& A = P->ad[a];
-    if (A.resident && A.last_use >= 0) P->lru.erase({A.last_use, a});
-    A.last_use = P->epoch;
-    P->lru.insert({A.last_use, a});
+  if (!prefetch) {
+    P->st.hits += (int64_t)(uniq.size() - missing.size());
+    P->epoch++;
+    for (int a : uniq) {
+      Adapter& A = P->ad[a];
+      if (A.resident && A.last_use >= 0) P->lru.erase({A.last_use, a});
+      A.last_use = P->epoch;
+      A.named = P->epoch;
+      A.uses[A.n_uses % kUseHistory] = P->epoch;
+      A.n_uses++;
+      P->lru.insert({A.last_use, a});
+    }
+  } else {
+    // as recent as the current step's set in the LRU order; usable by a
+    // compute call only once a later page_in names it
+    for (int a : missing) {
+      Adapter& A = P->ad[a];
+      A.last_use = P->epoch;
+      P->lru.insert({A.last_use, a});
+    }
+    P->st.prefetched += (int64_t)missing.size();
   }
   P->st.epoch = P->epoch;
   P->st.free_pages = (int64_t)P->free_pages.size();
@@ -787,7 +837,43 @@ slora_status_t slora_adapter_page_in(slora_pool* P, const int32_t* ids, int32_t 
     CUDA_TRY(P, cudaEventRecord(P->pagein_done, side));
     P->pagein_pending = true;
   }
+  // compute that waits on done_event must also see the copies of an earlier
+  // prefetch (or page-in) of the adapters named here, made on any stream
+  if (missing.empty() && victims.empty() && P->pagein_pending)
+    CUDA_TRY(P, cudaStreamWaitEvent(side, P->pagein_done, 0));
   if (done_event) CUDA_TRY(P, cudaEventRecord(static_cast<cudaEvent_t>(done_event), side));
+  return SLORA_OK;
+}
+
+slora_status_t slora_adapter_page_in(slora_pool* P, const int32_t* ids, int32_t n, void* side_stream,
+                                     void* done_event) {
+  return page_in_impl(P, ids, n, side_stream, done_event, false, 0, nullptr);
+}
+
+slora_status_t slora_adapter_prefetch(slora_pool* P, const int32_t* ids, int32_t n, int64_t max_pages,
+                                      void* side_stream, void* done_event, int32_t* n_done) {
+  return page_in_impl(P, ids, n, side_stream, done_event, true, max_pages, n_done);
+}
+
+slora_status_t slora_prefetch_candidates(const slora_pool* Pc, double half_life, int32_t max_n, int32_t* out,
+                                         int32_t* n_out) {
+  slora_pool* P = const_cast<slora_pool*>(Pc);
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  if (!(half_life > 0) || max_n < 0 || (max_n > 0 && !out) || !n_out)
+    return P->fail(SLORA_ERR_INVALID_ARG, "prefetch_candidates arguments");
+  std::vector<std::pair<double, int>> cand;  // (-score, id)
+  for (int a = 0; a < P->d.max_adapters; ++a) {
+    const Adapter& A = P->ad[a];
+    if (!A.registered || A.resident || A.n_uses == 0) continue;
+    double score = 0.0;
+    const int k = std::min(A.n_uses, kUseHistory);
+    for (int j = 0; j < k; ++j) score += std::exp2(-(double)(P->epoch - A.uses[j]) / half_life);
+    cand.push_back({-score, a});
+  }
+  std::sort(cand.begin(), cand.end());
+  const int m = std::min<int64_t>(max_n, (int64_t)cand.size());
+  for (int i = 0; i < m; ++i) out[i] = cand[i].second;
+  *n_out = m;
   return SLORA_OK;
 }
 
@@ -818,7 +904,7 @@ slora_status_t slora_check_batch(const slora_pool* Pc, const int32_t* idx_host, 
     const int a = idx_host[i];
     if (a == -1) continue;
     if (a < -1 || a >= P->d.max_adapters) return P->fail(SLORA_ERR_INVALID_ARG, "token " + std::to_string(i) + ": adapter id out of range");
-    if (!P->ad[a].resident || P->ad[a].last_use != P->epoch)
+    if (!P->ad[a].resident || P->ad[a].named != P->epoch)
       return P->fail(SLORA_ERR_NOT_RESIDENT, "token " + std::to_string(i) + ": adapter " + std::to_string(a) +
                                                  " is not in the latest page-in set");
   }

@@ -125,6 +125,8 @@ typedef struct {
   int64_t resident;         /* adapters resident now                                 */
   int64_t copy_calls;       /* cudaMemcpyAsync calls (memcpy mode) or gather launches */
   int64_t epoch;            /* page-in calls so far                                  */
+  int64_t prefetched;       /* adapters copied in by slora_adapter_prefetch          */
+  int64_t bytes_prefetched; /* their weight bytes (not counted in bytes_paged_in)    */
 } slora_pool_stats_t;
 
 /* ---- sizing ------------------------------------------------------------- */
@@ -190,6 +192,40 @@ slora_status_t slora_adapter_register(slora_pool* pool, int32_t id, int32_t rank
  * staging ring did not drain), INJECTED, CUDA.                                */
 slora_status_t slora_adapter_page_in(slora_pool* pool, const int32_t* ids, int32_t n,
                                      void* side_stream, void* done_event);
+
+/* Pages in, ahead of the step that will use them, the ids[0..n) that are not
+ * resident, taken in the given order (most wanted first) while they fit:
+ *   - at most max_pages pages in total; an id that does not fit is skipped and
+ *     the next ones are still tried;
+ *   - pages come from the free list, then from resident adapters not named by
+ *     the latest page_in call and not prefetched since it, least recently used
+ *     first: the current step's set is never touched, nor is it changed;
+ *   - copies go on side_stream exactly as page_in's (device-side waits for the
+ *     compute that last read reused pages); done_event (may be NULL) is
+ *     recorded after them.
+ * A prefetched adapter is as recent as the current step's set in the LRU
+ * order, and a compute call may use it only after a later page_in names it
+ * (that call finds it resident, and its done_event orders after these copies)
+ * [S1 implementation notes: with skewed traffic, frequently used adapters are
+ * loaded into VRAM ahead of time to avoid cold-start latency; S2 unified pool
+ * section: the scheduler anticipates requests with asynchronous PCIe loads on
+ * dedicated streams, overlapped with compute].
+ * *n_done (may be NULL) = adapters whose copies were enqueued.
+ * Errors: INVALID_ARG (also max_pages < 0), NOT_REGISTERED, TIMEOUT,
+ * INJECTED, CUDA; never OOM (what does not fit is skipped).                   */
+slora_status_t slora_adapter_prefetch(slora_pool* pool, const int32_t* ids, int32_t n, int64_t max_pages,
+                                      void* side_stream, void* done_event, int32_t* n_done);
+
+/* Prefetch policy: writes to out[0..*n_out) up to max_n registered adapters
+ * that are not resident, most popular first (equal scores: lower id first).
+ * Popularity = sum over the adapter's most recent 32 namings by page_in of
+ * 2^(-age / half_life), age = page_in calls since that naming [S1
+ * implementation notes: pre-load the adapters that skewed traffic uses most;
+ * S2 metrics section: LRU keeps frequent adapters, rare ones come from host].
+ * Adapters never named are not candidates.  Host only.
+ * Errors: INVALID_ARG (half_life <= 0, max_n < 0, NULL out / n_out).          */
+slora_status_t slora_prefetch_candidates(const slora_pool* pool, double half_life, int32_t max_n,
+                                         int32_t* out, int32_t* n_out);
 
 /* Evicts one resident adapter now (its pages become free once the compute that
  * last used it has finished; the device table entry is cleared on `stream`). */

@@ -32,6 +32,7 @@ def lib():
         L.oracle_pages_needed.argtypes = [i32, i32, P, P, i64]
         L.oracle_pages_needed.restype = i64
         L.oracle_lru_run.argtypes = [i32, P, i64, i32, P, P, P, P, P, P]
+        L.oracle_lru_prefetch_run.argtypes = [i32, P, i64, i32, P, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -151,6 +152,27 @@ def lru_run(need, capacity, calls):
                          _p(status), _p(resident), _p(evicted), _p(eoff))
     ev = [evicted[eoff[c]:eoff[c + 1]].tolist() for c in range(len(calls))]
     return status, resident.astype(bool), ev
+
+
+def lru_prefetch_run(need, capacity, calls):
+    """Run the LRU rules with prefetch calls over `calls`, a list of
+    (kind, ids, budget): kind "page_in" or "prefetch" (budget in pages).
+
+    Returns (status[c], resident[c, a] bool)."""
+    need = _c(need, np.int64)
+    n_ad = need.size
+    kind = _c([0 if k == "page_in" else 1 for k, _, _ in calls], np.int32)
+    budget = _c([int(b) for _, _, b in calls], np.int64)
+    off = np.zeros(len(calls) + 1, np.int32)
+    for c, (_, ids, _) in enumerate(calls):
+        off[c + 1] = off[c] + len(ids)
+    ids = _c(np.concatenate([np.asarray(i, np.int32) for _, i, _ in calls]) if calls else
+             np.zeros(0, np.int32), np.int32)
+    status = np.zeros(len(calls), np.int32)
+    resident = np.zeros((len(calls), n_ad), np.uint8)
+    lib().oracle_lru_prefetch_run(n_ad, _p(need), int(capacity), len(calls), _p(kind), _p(budget),
+                                  _p(off), _p(ids), _p(status), _p(resident))
+    return status, resident.astype(bool)
 
 
 def n_threads_default():

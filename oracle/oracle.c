@@ -34,6 +34,12 @@
  *  oracle_lru_run      -- least-recently-used residency decisions over a trace
  *                         of page-in calls ("Paper explainer: S-LoRA", section
  *                         "Unified Paging", eviction strategy).
+ *  oracle_lru_prefetch_run -- the same with prefetch calls interleaved: adapters
+ *                         loaded ahead of the step that uses them, without
+ *                         disturbing the current step ("Paper explainer:
+ *                         S-LoRA", implementation notes on pre-loading frequent
+ *                         adapters; "Multi-LoRA serving", unified pool section:
+ *                         the scheduler anticipates requests).
  *
  * Readings where the pages are silent are listed in the design notes; the ones
  * that shape this file: rank 0 leaves y unchanged; ties in LRU age go to the
@@ -335,5 +341,116 @@ int oracle_lru_run(int n_adapters, const long* need, long capacity, int n_calls,
   free(pin);
   free(tmp);
   free(victims);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* LRU with prefetch.                                                         */
+/*
+ * As oracle_lru_run, with each call c of kind[c]:
+ *   0 (page-in): as above; on success the step counter E grows by one and
+ *     every asked adapter gets age E;
+ *   1 (prefetch, page budget budget[c]): the asked adapters that are not
+ *     resident are taken in the order they first appear; one is chosen when
+ *     the pages chosen so far plus its own stay within min(budget[c], free
+ *     pages + pages of the resident adapters older than E), else it is
+ *     skipped and the next is tried.  Room is made by evicting resident
+ *     adapters older than E, oldest first (equal ages: lower id first).  The
+ *     chosen adapters become resident with age E.  Status OK unless an id is
+ *     out of range (ARG, nothing changes).
+ * Ages start at -1 (never used); E starts at 0.
+ */
+int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int n_calls,
+                            const int* kind, const long* budget, const int* call_off, const int* ids,
+                            int* status, unsigned char* resident) {
+  unsigned char* res = (unsigned char*)calloc(n_adapters, 1);
+  long* age = (long*)malloc(sizeof(long) * n_adapters);
+  unsigned char* mark = (unsigned char*)calloc(n_adapters, 1);
+  unsigned char* tmp = (unsigned char*)malloc(n_adapters);
+  int* order = (int*)malloc(sizeof(int) * (n_adapters + 1));
+  for (int a = 0; a < n_adapters; ++a) age[a] = -1;
+  long used = 0, E = 0;
+  for (int c = 0; c < n_calls; ++c) {
+    int bad = 0;
+    for (int q = call_off[c]; q < call_off[c + 1]; ++q)
+      if (ids[q] < 0 || ids[q] >= n_adapters) bad = 1;
+    memset(mark, 0, n_adapters);
+    if (bad) {
+      status[c] = OR_ERR_ARG;
+    } else if (kind[c] == 0) {
+      long missing = 0;
+      for (int q = call_off[c]; q < call_off[c + 1]; ++q) {
+        int a = ids[q];
+        if (!mark[a] && !res[a]) missing += need[a];
+        mark[a] = 1; /* pinned for this call */
+      }
+      memcpy(tmp, res, n_adapters);
+      long free_pages = capacity - used;
+      while (free_pages < missing) {
+        int best = -1;
+        for (int a = 0; a < n_adapters; ++a)
+          if (tmp[a] && !mark[a] && (best < 0 || age[a] < age[best])) best = a;
+        if (best < 0) break;
+        tmp[best] = 0;
+        free_pages += need[best];
+      }
+      if (free_pages < missing) {
+        status[c] = OR_ERR_OOM;
+      } else {
+        for (int a = 0; a < n_adapters; ++a)
+          if (res[a] && !tmp[a]) {
+            res[a] = 0;
+            used -= need[a];
+          }
+        E += 1;
+        for (int q = call_off[c]; q < call_off[c + 1]; ++q) {
+          int a = ids[q];
+          if (!res[a]) {
+            res[a] = 1;
+            used += need[a];
+          }
+          age[a] = E;
+        }
+        status[c] = OR_OK;
+      }
+    } else {
+      long room = capacity - used;
+      for (int a = 0; a < n_adapters; ++a)
+        if (res[a] && age[a] < E) room += need[a];
+      long limit = budget[c] < room ? budget[c] : room;
+      long chosen = 0;
+      int n_order = 0;
+      for (int q = call_off[c]; q < call_off[c + 1]; ++q) {
+        int a = ids[q];
+        if (res[a] || mark[a]) continue;
+        mark[a] = 1; /* looked at (first occurrence decides) */
+        if (chosen + need[a] > limit) continue;
+        order[n_order++] = a;
+        chosen += need[a];
+      }
+      long free_pages = capacity - used;
+      while (free_pages < chosen) {
+        int best = -1;
+        for (int a = 0; a < n_adapters; ++a)
+          if (res[a] && age[a] < E && (best < 0 || age[a] < age[best])) best = a;
+        if (best < 0) break; /* cannot happen: chosen <= room */
+        res[best] = 0;
+        used -= need[best];
+        free_pages += need[best];
+      }
+      for (int k = 0; k < n_order; ++k) {
+        res[order[k]] = 1;
+        used += need[order[k]];
+        age[order[k]] = E;
+      }
+      status[c] = OR_OK;
+    }
+    memcpy(resident + (long)c * n_adapters, res, n_adapters);
+  }
+  free(res);
+  free(age);
+  free(mark);
+  free(tmp);
+  free(order);
   return OR_OK;
 }

@@ -182,3 +182,115 @@ def test_event_without_cuda_handle_is_refused():
     with pytest.raises(ValueError):
         G._event(Unrecorded())
     assert G._event(None) is None and G._event(1234) == 1234
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefetch_matches_oracle(seed):
+    """page_in and prefetch calls interleaved: the library's residency after
+    every call agrees with the oracle's restatement of the rules."""
+    rng = np.random.default_rng(100 + seed)
+    n_ad = 40
+    ranks = rng.choice([0, 8, 16, 32], n_ad)
+    pool = _host_pool()
+    _register_all(pool, ranks)
+    need = [pool.pages_for_rank(int(r)) for r in ranks]
+    calls = []
+    for _ in range(150):
+        ids = rng.choice(n_ad, size=int(rng.integers(1, 7))).tolist()
+        if rng.random() < 0.4:
+            calls.append(("prefetch", ids, int(rng.integers(0, 160))))
+        else:
+            calls.append(("page_in", ids, 0))
+    calls.insert(7, ("prefetch", [n_ad + 1], 50))     # invalid id
+    status, resident = oracle.lru_prefetch_run(need, 100, calls)
+    n_pre = 0
+    for c, (kind, ids, budget) in enumerate(calls):
+        st = 0
+        try:
+            if kind == "page_in":
+                pool.page_in(ids)
+            else:
+                n_pre += G.slora_adapter_prefetch(pool.h, ids, budget)
+        except G.SloraError as e:
+            st = e.status
+        assert st == status[c], (c, kind, ids, st, status[c])
+        got = [G.slora_adapter_is_resident(pool.h, a) for a in range(n_ad)]
+        assert got == resident[c].tolist(), (c, kind, ids, budget)
+    assert pool.stats()["prefetched"] == n_pre > 0
+
+
+def test_prefetch_keeps_the_step_set_and_needs_a_page_in():
+    pool = _host_pool(n_pages=150)              # rank 8: 48 pages each -> 3 fit
+    _register_all(pool, [8] * 6)
+    pool.page_in([0])
+    pool.page_in([1, 2])                         # the step's set; 0 is older
+    assert G.slora_adapter_prefetch(pool.h, [3, 4], 1000) == 1   # room for one: evicts 0
+    res = [G.slora_adapter_is_resident(pool.h, a) for a in range(6)]
+    assert res == [False, True, True, True, False, False]
+    G.slora_check_batch(pool.h, [1, 2, -1])      # the step's set is unchanged
+    with pytest.raises(G.SloraError) as e:
+        G.slora_check_batch(pool.h, [3])         # prefetched, not yet named
+    assert e.value.status == 3
+    # nothing older than the step is left: a second prefetch cannot evict
+    assert G.slora_adapter_prefetch(pool.h, [4, 5], 1000) == 0
+    before = pool.stats()
+    pool.page_in([3, 1])                         # finds 3 resident: two hits, no copy
+    after = pool.stats()
+    assert after["hits"] - before["hits"] == 2 and after["page_ins"] == before["page_ins"]
+    G.slora_check_batch(pool.h, [3, 1])
+    assert after["bytes_prefetched"] == 2 * 8 * (1024 + 2048 + 2048 + 1024)
+    # a budget smaller than one adapter skips it; rank 0 needs no pages
+    with pytest.raises(G.SloraError) as e:
+        G.slora_adapter_prefetch(pool.h, [4], -1)
+    assert e.value.status == 1
+    assert G.slora_adapter_prefetch(pool.h, [4], 47) == 0
+
+
+def _decayed_scores(trace, n_ad, half_life):
+    """Popularity by its definition: over an adapter's last 32 namings by a
+    page-in call, the sum of 2^(-age / half_life), age in page-in calls."""
+    E = len(trace)
+    scores = {}
+    for a in range(n_ad):
+        epochs = [e + 1 for e, ids in enumerate(trace) if a in ids][-32:]
+        if epochs:
+            scores[a] = sum(2.0 ** (-(E - e) / half_life) for e in epochs)
+    return scores
+
+
+@pytest.mark.parametrize("half_life", [1.0, 4.0, 50.0])
+def test_prefetch_candidates_rank_by_decayed_popularity(half_life):
+    rng = np.random.default_rng(7)
+    n_ad = 12
+    pool = _host_pool(n_pages=100)              # two rank-8 adapters fit
+    _register_all(pool, [8] * n_ad)
+    # skewed traffic: adapter 0 named in most calls (more than 32 times)
+    trace = []
+    for _ in range(60):
+        ids = sorted({int(i) for i in (rng.zipf(1.6, 2) - 1) % n_ad})
+        pool.page_in(ids)
+        trace.append(set(ids))
+    sc = _decayed_scores(trace, n_ad, half_life)
+    want = [a for a in sc if not G.slora_adapter_is_resident(pool.h, a)]
+    got = G.slora_prefetch_candidates(pool.h, half_life, n_ad)
+    assert sorted(got) == sorted(want)
+    for u, v in zip(got, got[1:]):               # most popular first, ties by id
+        assert sc[u] > sc[v] * (1 + 1e-12) or (abs(sc[u] - sc[v]) <= 1e-12 * sc[u] and u < v)
+    assert G.slora_prefetch_candidates(pool.h, half_life, 2) == got[:2]
+    with pytest.raises(G.SloraError):
+        G.slora_prefetch_candidates(pool.h, 0.0, 4)
+
+
+def test_prefetch_hand_trace_through_the_library():
+    from test_oracle import PREFETCH_TRACE as t
+    ranks = [n // 2 for n in t["need"]]          # d_in = d_out = page = 1024: 2 r pages
+    pool = G.Pool(G.SLORA_F16, [1024], [1024], len(ranks), 8, 16, 1024, t["capacity"],
+                  host_only=True)
+    _register_all(pool, ranks)
+    for c, (kind, ids, budget) in enumerate(t["calls"]):
+        if kind == "page_in":
+            pool.page_in(ids)
+        else:
+            G.slora_adapter_prefetch(pool.h, ids, budget)
+        assert [a for a in range(len(ranks)) if G.slora_adapter_is_resident(pool.h, a)] == \
+            t["resident"][c], c

@@ -259,3 +259,42 @@ def test_lru_invariants(seed):
             assert status[c] == 2 and ev[c] == []
             assert np.array_equal(res[c], prev)
         prev = res[c]
+
+
+# A prefetch trace worked by hand from the rules (pages: a0..a2 need 4, a3
+# needs 2, a4 needs 0; capacity 10; E = page-in calls so far):
+#  1 page_in [0]          E=1  {0}
+#  2 page_in [1]          E=2  {0,1}            free 2
+#  3 prefetch [2,3] b=100 room = 2 + 4 (a0, age 1 < 2) = 6: a2 (4) and a3 (2)
+#                         fit; a0 evicted           {1,2,3}
+#  4 prefetch [4,0] b=3   room = 0 (all ages are 2): a4 (0 pages) fits, a0
+#                         does not                  {1,2,3,4}
+#  5 page_in [2,0]   E=3  a0 needs 4, free 0: oldest unpinned of age 2 is a1
+#                         (lowest id)               {0,2,3,4}
+#  6 prefetch [1] b=4     room = 2 (a3) + 0 (a4) < 4: skipped
+#  7 page_in []      E=4
+#  8 prefetch [1] b=10    room = 10; evicts a3, a4 (age 2, ids 3, 4), then a0
+#                         (age 3, before a2 by id)  {1,2}
+PREFETCH_TRACE = dict(
+    need=[4, 4, 4, 2, 0], capacity=10,
+    calls=[("page_in", [0], 0), ("page_in", [1], 0), ("prefetch", [2, 3], 100),
+           ("prefetch", [4, 0], 3), ("page_in", [2, 0], 0), ("prefetch", [1], 4),
+           ("page_in", [], 0), ("prefetch", [1], 10)],
+    resident=[[0], [0, 1], [1, 2, 3], [1, 2, 3, 4], [0, 2, 3, 4], [0, 2, 3, 4], [0, 2, 3, 4],
+              [1, 2]])
+
+
+def test_prefetch_rules_hand_trace():
+    t = PREFETCH_TRACE
+    status, res = oracle.lru_prefetch_run(t["need"], t["capacity"], t["calls"])
+    assert status.tolist() == [0] * len(t["calls"])
+    assert [np.flatnonzero(r).tolist() for r in res] == t["resident"]
+
+
+def test_prefetch_without_prefetch_calls_is_lru():
+    rng = np.random.default_rng(3)
+    need = rng.integers(0, 6, 25)
+    calls = [rng.choice(25, size=int(rng.integers(1, 6))).tolist() for _ in range(50)]
+    s1, r1, _ = oracle.lru_run(need, 30, calls)
+    s2, r2 = oracle.lru_prefetch_run(need, 30, [("page_in", c, 0) for c in calls])
+    assert np.array_equal(s1, s2) and np.array_equal(r1, r2)
