@@ -45,7 +45,7 @@ class PoolDesc(ctypes.Structure):
 class PoolStats(ctypes.Structure):
     _fields_ = [(n, c_int64) for n in ("page_ins", "hits", "evictions", "bytes_paged_in",
                                        "free_pages", "resident", "copy_calls", "epoch",
-                                       "prefetched", "bytes_prefetched")]
+                                       "prefetched", "bytes_prefetched", "kv_pages")]
 
 
 _lib = None
@@ -72,6 +72,8 @@ def lib():
         "slora_adapter_page_in": ([P, P, I32, P, P], I32),
         "slora_adapter_prefetch": ([P, P, I32, I64, P, P, POINTER(c_int32)], I32),
         "slora_prefetch_candidates": ([P, ctypes.c_double, I32, P, POINTER(c_int32)], I32),
+        "slora_kv_alloc": ([P, I64, P, P, P], I32),
+        "slora_kv_free": ([P, P, I64, P], I32),
         "slora_adapter_evict": ([P, I32, P], I32),
         "slora_adapter_is_resident": ([P, I32, POINTER(c_int32)], I32),
         "slora_check_batch": ([P, P, I32], I32),
@@ -209,6 +211,19 @@ def slora_prefetch_candidates(pool: int, half_life: float, max_n: int) -> list:
     _check(pool, lib().slora_prefetch_candidates(pool, float(half_life), int(max_n),
                                                  ctypes.cast(out, c_void_p), ctypes.byref(n)))
     return [int(out[i]) for i in range(n.value)]
+
+
+def slora_kv_alloc(pool: int, n: int, stream=None, done_event=None) -> list:
+    """Returns the page ids taken for KV blocks."""
+    out = (c_int32 * max(int(n), 1))()
+    _check(pool, lib().slora_kv_alloc(pool, int(n), ctypes.cast(out, c_void_p), _stream(stream),
+                                      _event(done_event)))
+    return [int(out[i]) for i in range(int(n))]
+
+
+def slora_kv_free(pool: int, ids, stream=None) -> None:
+    a = _arr(c_int32, [int(i) for i in ids])
+    _check(pool, lib().slora_kv_free(pool, ctypes.cast(a, c_void_p), len(ids), _stream(stream)))
 
 
 def slora_adapter_evict(pool: int, id: int, stream=None) -> None:

@@ -61,7 +61,10 @@ struct Adapter {
 struct FreePage {
   int32_t id;
   int64_t free_epoch;  // compute epoch that last may have read it (-1: none)
+  int rel = -1;        // release event of the KV-block owner that freed it (-1: none)
 };
+
+constexpr int kRelRing = 64;  // events marking the last use of freed KV blocks
 
 struct Staging {
   void* host = nullptr;
@@ -183,6 +186,10 @@ struct slora_pool {
   int next_stg = 0;
   cudaEvent_t pagein_done = nullptr;
   bool pagein_pending = false;
+  std::vector<uint8_t> kv_page;       // 1: the page is held as a KV block
+  int64_t kv_held = 0;
+  cudaEvent_t rel_ev[kRelRing] = {};
+  int64_t n_rel = 0;                  // release events recorded so far
   PoolDev pd{};
   int sm_count = 148;
   int grid_shrink = 0, grid_expand = 0;
@@ -486,7 +493,8 @@ slora_status_t slora_pool_create(const slora_pool_desc* desc, slora_pool** out) 
   P->tl = table_layout(P->d);
   P->sl = scratch_layout(P->d);
   P->ad.resize(P->d.max_adapters);
-  for (int64_t pg = 0; pg < P->d.n_pages; ++pg) P->free_pages.push_back({(int32_t)pg, -1});
+  for (int64_t pg = 0; pg < P->d.n_pages; ++pg) P->free_pages.push_back({(int32_t)pg, -1, -1});
+  P->kv_page.assign((size_t)P->d.n_pages, 0);
   for (int i = 0; i < kEventRing; ++i) P->ev_epoch[i] = -1;
   P->st.free_pages = P->d.n_pages;
   if (!P->d.host_only) {
@@ -498,6 +506,8 @@ slora_status_t slora_pool_create(const slora_pool_desc* desc, slora_pool** out) 
     for (int i = 0; i < kEventRing && e == cudaSuccess; ++i)
       e = cudaEventCreateWithFlags(&P->ev[i], cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&P->pagein_done, cudaEventDisableTiming);
+    for (int i = 0; i < kRelRing && e == cudaSuccess; ++i)
+      e = cudaEventCreateWithFlags(&P->rel_ev[i], cudaEventDisableTiming);
     for (int i = 0; i < kStagingSlots && e == cudaSuccess; ++i)
       e = cudaEventCreateWithFlags(&P->stg[i].done, cudaEventDisableTiming);
     // tables: rank = -1 (0xff bytes), scale = 0, err = 0, page lists = -1
@@ -535,6 +545,8 @@ slora_status_t slora_pool_destroy(slora_pool* P) {
     }
     for (int i = 0; i < kEventRing; ++i)
       if (P->ev[i]) cudaEventDestroy(P->ev[i]);
+    for (int i = 0; i < kRelRing; ++i)
+      if (P->rel_ev[i]) cudaEventDestroy(P->rel_ev[i]);
   }
   delete P;
   return SLORA_OK;
@@ -545,14 +557,14 @@ const char* slora_last_error(const slora_pool* P) { return P ? P->err.c_str() : 
 slora_status_t slora_pool_set_page_order(slora_pool* P, const int32_t* order, int64_t n) {
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (!order || n != P->d.n_pages) return P->fail(SLORA_ERR_INVALID_ARG, "order must list n_pages ids");
-  if (!P->lru.empty()) return P->fail(SLORA_ERR_INVALID_ARG, "only allowed while no adapter is resident");
+  if (!P->lru.empty() || P->kv_held) return P->fail(SLORA_ERR_INVALID_ARG, "only allowed while no page is held");
   std::vector<char> seen(n, 0);
   for (int64_t i = 0; i < n; ++i) {
     if (order[i] < 0 || order[i] >= n || seen[order[i]]) return P->fail(SLORA_ERR_INVALID_ARG, "order is not a permutation");
     seen[order[i]] = 1;
   }
   std::deque<FreePage> fp;
-  for (int64_t i = 0; i < n; ++i) fp.push_back({order[i], -1});
+  for (int64_t i = 0; i < n; ++i) fp.push_back({order[i], -1, -1});
   P->free_pages.swap(fp);
   return SLORA_OK;
 }
@@ -604,7 +616,7 @@ slora_status_t slora_adapter_register(slora_pool* P, int32_t id, int32_t rank, f
 static void evict_one(slora_pool* P, int id) {
   Adapter& A = P->ad[id];
   P->lru.erase({A.last_use, id});
-  for (int32_t pg : A.pages) P->free_pages.push_back({pg, A.last_use});
+  for (int32_t pg : A.pages) P->free_pages.push_back({pg, A.last_use, -1});
   A.pages.clear();
   A.resident = false;
   P->st.evictions++;
@@ -688,6 +700,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     }
   }
   // ---- commit host state
+  std::set<int> rel_wait;  // release events of freed KV blocks among the pages taken
   for (int v : victims) evict_one(P, v);
   int64_t wait_ep = -1;
   for (int v : victims) wait_ep = std::max(wait_ep, P->ad[v].last_use);
@@ -700,6 +713,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
       P->free_pages.pop_front();
       A.pages[i] = f.id;
       wait_ep = std::max(wait_ep, f.free_epoch);
+      if (f.rel >= 0) rel_wait.insert(f.rel);
     }
     A.resident = true;
     P->st.page_ins++;
@@ -801,6 +815,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     // compute that last read the pages being reused
     if (P->pagein_pending) CUDA_TRY(P, cudaStreamWaitEvent(side, P->pagein_done, 0));
     wait_epoch(P, side, wait_ep);
+    for (int r : rel_wait) CUDA_TRY(P, cudaStreamWaitEvent(side, P->rel_ev[r], 0));
     char* desc_dev = P->tables() + P->tl.off_desc;
     CUDA_TRY(P, cudaMemcpyAsync(desc_dev, h, bytes, cudaMemcpyHostToDevice, side));
     CUDA_TRY(P, cudaEventRecord(stg->done, side));
@@ -877,12 +892,91 @@ slora_status_t slora_prefetch_candidates(const slora_pool* Pc, double half_life,
   return SLORA_OK;
 }
 
+slora_status_t slora_kv_alloc(slora_pool* P, int64_t n, int32_t* ids_out, void* stream, void* done_event) {
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  if (n < 0 || (n > 0 && !ids_out)) return P->fail(SLORA_ERR_INVALID_ARG, "kv_alloc arguments");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // room: free pages, then adapters older than the current step, LRU first
+  std::vector<int> victims;
+  int64_t avail = (int64_t)P->free_pages.size();
+  for (auto it = P->lru.begin(); avail < n && it != P->lru.end(); ++it) {
+    if (it->first >= P->epoch) break;  // std::set order: the rest are as new
+    victims.push_back(it->second);
+    avail += (int64_t)P->ad[it->second].pages.size();
+  }
+  if (avail < n)
+    return P->fail(SLORA_ERR_OOM, "cannot take " + std::to_string(n) + " pages for KV blocks");
+  int64_t wait_ep = -1;
+  for (int v : victims) {
+    wait_ep = std::max(wait_ep, P->ad[v].last_use);
+    evict_one(P, v);
+  }
+  std::set<int> rel_wait;
+  for (int64_t i = 0; i < n; ++i) {
+    FreePage f = P->free_pages.front();
+    P->free_pages.pop_front();
+    ids_out[i] = f.id;
+    P->kv_page[f.id] = 1;
+    wait_ep = std::max(wait_ep, f.free_epoch);
+    if (f.rel >= 0) rel_wait.insert(f.rel);
+  }
+  P->kv_held += n;
+  P->st.free_pages = (int64_t)P->free_pages.size();
+  P->st.resident = (int64_t)P->lru.size();
+  if (P->d.host_only) return SLORA_OK;
+  // the evicted adapters leave the device table; the pages are the caller's
+  // once the compute, page-in copies and KV owners that last touched them are done
+  // (table writes join the page-in chain, so a later page-in of the same
+  // adapter on another stream lands after them)
+  if (P->pagein_pending) CUDA_TRY(P, cudaStreamWaitEvent(st, P->pagein_done, 0));
+  for (int v : victims) CUDA_TRY(P, cudaMemsetAsync(P->pd.rank + v, 0xff, 4, st));
+  if (!victims.empty()) {
+    CUDA_TRY(P, cudaEventRecord(P->pagein_done, st));
+    P->pagein_pending = true;
+  }
+  wait_epoch(P, st, wait_ep);
+  for (int r : rel_wait) CUDA_TRY(P, cudaStreamWaitEvent(st, P->rel_ev[r], 0));
+  if (done_event) CUDA_TRY(P, cudaEventRecord(static_cast<cudaEvent_t>(done_event), st));
+  return SLORA_OK;
+}
+
+slora_status_t slora_kv_free(slora_pool* P, const int32_t* ids, int64_t n, void* stream) {
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  if (n < 0 || (n > 0 && !ids)) return P->fail(SLORA_ERR_INVALID_ARG, "kv_free arguments");
+  std::unordered_set<int32_t> seen;
+  for (int64_t i = 0; i < n; ++i)
+    if (ids[i] < 0 || ids[i] >= P->d.n_pages || !P->kv_page[ids[i]] || !seen.insert(ids[i]).second)
+      return P->fail(SLORA_ERR_INVALID_ARG, "page " + std::to_string(ids[i]) + " is not a held KV page");
+  int rel = -1;
+  if (!P->d.host_only && stream && n > 0) {
+    // reusing a slot: the work it marked is long done (64 releases ago); make sure
+    rel = (int)(P->n_rel % kRelRing);
+    if (P->n_rel >= kRelRing) {
+      slora_status_t ws = wait_event_bounded(P, P->rel_ev[rel]);
+      if (ws != SLORA_OK) return ws;
+    }
+    CUDA_TRY(P, cudaEventRecord(P->rel_ev[rel], static_cast<cudaStream_t>(stream)));
+    P->n_rel++;
+  }
+  for (int64_t i = 0; i < n; ++i) {
+    P->kv_page[ids[i]] = 0;
+    P->free_pages.push_back({ids[i], -1, rel});
+  }
+  P->kv_held -= n;
+  P->st.free_pages = (int64_t)P->free_pages.size();
+  return SLORA_OK;
+}
+
 slora_status_t slora_adapter_evict(slora_pool* P, int32_t id, void* stream) {
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (id < 0 || id >= P->d.max_adapters) return P->fail(SLORA_ERR_INVALID_ARG, "adapter id out of range");
   if (!P->ad[id].resident) return P->fail(SLORA_ERR_NOT_RESIDENT, "adapter " + std::to_string(id));
   if (!P->d.host_only) {
-    CUDA_TRY(P, cudaMemsetAsync(P->pd.rank + id, 0xff, 4, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (P->pagein_pending) CUDA_TRY(P, cudaStreamWaitEvent(st, P->pagein_done, 0));
+    CUDA_TRY(P, cudaMemsetAsync(P->pd.rank + id, 0xff, 4, st));
+    CUDA_TRY(P, cudaEventRecord(P->pagein_done, st));  // a later page-in lands after it
+    P->pagein_pending = true;
   }
   evict_one(P, id);
   P->st.free_pages = (int64_t)P->free_pages.size();
@@ -1102,6 +1196,7 @@ slora_status_t slora_pool_stats(const slora_pool* P, slora_pool_stats_t* out) {
   out->free_pages = (int64_t)P->free_pages.size();
   out->resident = (int64_t)P->lru.size();
   out->epoch = P->epoch;
+  out->kv_pages = P->kv_held;
   return SLORA_OK;
 }
 

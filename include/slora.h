@@ -127,6 +127,7 @@ typedef struct {
   int64_t epoch;            /* page-in calls so far                                  */
   int64_t prefetched;       /* adapters copied in by slora_adapter_prefetch          */
   int64_t bytes_prefetched; /* their weight bytes (not counted in bytes_paged_in)    */
+  int64_t kv_pages;         /* pages held as KV blocks (slora_kv_alloc)              */
 } slora_pool_stats_t;
 
 /* ---- sizing ------------------------------------------------------------- */
@@ -226,6 +227,33 @@ slora_status_t slora_adapter_prefetch(slora_pool* pool, const int32_t* ids, int3
  * Errors: INVALID_ARG (half_life <= 0, max_n < 0, NULL out / n_out).          */
 slora_status_t slora_prefetch_candidates(const slora_pool* pool, double half_life, int32_t max_n,
                                          int32_t* out, int32_t* n_out);
+
+/* ---- KV-cache blocks in the same pool ------------------------------------- */
+
+/* Takes n pages of the pool for KV-cache blocks (or any other page-granular
+ * owner), so that adapters and the KV cache share one pool of one page size
+ * [S1 Unified Paging: one unified pool for the KV cache and adapter weights;
+ * S2 unified pool section: adapter memory and the KV cache under one paged
+ * abstraction]:
+ *   - free pages first; when too few are free, resident adapters older than
+ *     the current step (not named by the latest page_in, not prefetched since)
+ *     are evicted, least recently used first (equal ages: lower id first);
+ *   - ids_out[0..n) = the page ids; page g is elements [g*page_elems,
+ *     (g+1)*page_elems) of dev_pool, in the pool's 16-bit element type;
+ *   - the caller may write the pages after done_event (may be NULL; then use
+ *     `stream` itself): it is recorded on `stream` after the evicted adapters'
+ *     table entries are cleared and after the compute, page-in copies and KV
+ *     owners that last touched those pages.
+ * KV pages are never evicted: they stay the caller's until slora_kv_free.
+ * Errors: INVALID_ARG, OOM (nothing changed), CUDA.                           */
+slora_status_t slora_kv_alloc(slora_pool* pool, int64_t n, int32_t* ids_out, void* stream, void* done_event);
+
+/* Returns KV pages to the pool.  stream: where the last kernels that use these
+ * pages were enqueued (an event recorded there orders later adapter copies
+ * into the pages after them); NULL: that work has completed.
+ * Errors: INVALID_ARG (an id not held as a KV page, or repeated; nothing
+ * changed), TIMEOUT, CUDA.                                                    */
+slora_status_t slora_kv_free(slora_pool* pool, const int32_t* ids, int64_t n, void* stream);
 
 /* Evicts one resident adapter now (its pages become free once the compute that
  * last used it has finished; the device table entry is cleared on `stream`). */

@@ -155,13 +155,15 @@ def lru_run(need, capacity, calls):
 
 
 def lru_prefetch_run(need, capacity, calls):
-    """Run the LRU rules with prefetch calls over `calls`, a list of
-    (kind, ids, budget): kind "page_in" or "prefetch" (budget in pages).
+    """Run the LRU rules with prefetch and KV-block calls over `calls`, a
+    list of (kind, ids, n): kind "page_in", "prefetch" (n = page budget),
+    "kv_alloc" or "kv_free" (n pages; ids unused).
 
     Returns (status[c], resident[c, a] bool)."""
     need = _c(need, np.int64)
     n_ad = need.size
-    kind = _c([0 if k == "page_in" else 1 for k, _, _ in calls], np.int32)
+    kinds = {"page_in": 0, "prefetch": 1, "kv_alloc": 2, "kv_free": 3}
+    kind = _c([kinds[k] for k, _, _ in calls], np.int32)
     budget = _c([int(b) for _, _, b in calls], np.int64)
     off = np.zeros(len(calls) + 1, np.int32)
     for c, (_, ids, _) in enumerate(calls):

@@ -39,7 +39,9 @@
  *                         disturbing the current step ("Paper explainer:
  *                         S-LoRA", implementation notes on pre-loading frequent
  *                         adapters; "Multi-LoRA serving", unified pool section:
- *                         the scheduler anticipates requests).
+ *                         the scheduler anticipates requests), and with KV-cache
+ *                         blocks taking and returning pages of the same pool
+ *                         ("Paper explainer: S-LoRA", section "Unified Paging").
  *
  * Readings where the pages are silent are listed in the design notes; the ones
  * that shape this file: rank 0 leaves y unchanged; ties in LRU age go to the
@@ -357,7 +359,13 @@ int oracle_lru_run(int n_adapters, const long* need, long capacity, int n_calls,
  *     skipped and the next is tried.  Room is made by evicting resident
  *     adapters older than E, oldest first (equal ages: lower id first).  The
  *     chosen adapters become resident with age E.  Status OK unless an id is
- *     out of range (ARG, nothing changes).
+ *     out of range (ARG, nothing changes);
+ *   2 (KV blocks take budget[c] pages): when the free pages do not cover them,
+ *     resident adapters older than E are evicted, oldest first (equal ages:
+ *     lower id first); if even all of those cannot make room: OOM, nothing
+ *     changes;
+ *   3 (KV blocks return budget[c] pages).
+ * Pages held by KV blocks are neither free nor evictable.
  * Ages start at -1 (never used); E starts at 0.
  */
 int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int n_calls,
@@ -369,8 +377,33 @@ int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int
   unsigned char* tmp = (unsigned char*)malloc(n_adapters);
   int* order = (int*)malloc(sizeof(int) * (n_adapters + 1));
   for (int a = 0; a < n_adapters; ++a) age[a] = -1;
-  long used = 0, E = 0;
+  long used = 0, kv = 0, E = 0;
   for (int c = 0; c < n_calls; ++c) {
+    if (kind[c] == 2 || kind[c] == 3) {
+      if (kind[c] == 3) {
+        kv -= budget[c];
+        status[c] = OR_OK;
+      } else {
+        long room = capacity - used - kv;
+        for (int a = 0; a < n_adapters; ++a)
+          if (res[a] && age[a] < E) room += need[a];
+        if (room < budget[c]) {
+          status[c] = OR_ERR_OOM;
+        } else {
+          while (capacity - used - kv < budget[c]) {
+            int best = -1;
+            for (int a = 0; a < n_adapters; ++a)
+              if (res[a] && age[a] < E && (best < 0 || age[a] < age[best])) best = a;
+            res[best] = 0;
+            used -= need[best];
+          }
+          kv += budget[c];
+          status[c] = OR_OK;
+        }
+      }
+      memcpy(resident + (long)c * n_adapters, res, n_adapters);
+      continue;
+    }
     int bad = 0;
     for (int q = call_off[c]; q < call_off[c + 1]; ++q)
       if (ids[q] < 0 || ids[q] >= n_adapters) bad = 1;
@@ -385,7 +418,7 @@ int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int
         mark[a] = 1; /* pinned for this call */
       }
       memcpy(tmp, res, n_adapters);
-      long free_pages = capacity - used;
+      long free_pages = capacity - used - kv;
       while (free_pages < missing) {
         int best = -1;
         for (int a = 0; a < n_adapters; ++a)
@@ -414,7 +447,7 @@ int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int
         status[c] = OR_OK;
       }
     } else {
-      long room = capacity - used;
+      long room = capacity - used - kv;
       for (int a = 0; a < n_adapters; ++a)
         if (res[a] && age[a] < E) room += need[a];
       long limit = budget[c] < room ? budget[c] : room;
@@ -428,7 +461,7 @@ int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int
         order[n_order++] = a;
         chosen += need[a];
       }
-      long free_pages = capacity - used;
+      long free_pages = capacity - used - kv;
       while (free_pages < chosen) {
         int best = -1;
         for (int a = 0; a < n_adapters; ++a)

@@ -294,3 +294,98 @@ def test_prefetch_hand_trace_through_the_library():
             G.slora_adapter_prefetch(pool.h, ids, budget)
         assert [a for a in range(len(ranks)) if G.slora_adapter_is_resident(pool.h, a)] == \
             t["resident"][c], c
+
+
+def test_kv_hand_trace_through_the_library():
+    from test_oracle import KV_TRACE as t
+    ranks = [n // 2 for n in t["need"]]
+    pool = G.Pool(G.SLORA_F16, [1024], [1024], len(ranks), 8, 16, 1024, t["capacity"],
+                  host_only=True)
+    _register_all(pool, ranks)
+    held = []
+    for c, (kind, ids, n) in enumerate(t["calls"]):
+        st = 0
+        try:
+            if kind == "page_in":
+                pool.page_in(ids)
+            elif kind == "kv_alloc":
+                held += G.slora_kv_alloc(pool.h, n)
+            else:
+                G.slora_kv_free(pool.h, held[:n])
+                held = held[n:]
+        except G.SloraError as e:
+            st = e.status
+        assert st == t["status"][c], c
+        assert [a for a in range(len(ranks)) if G.slora_adapter_is_resident(pool.h, a)] == \
+            t["resident"][c], c
+    assert pool.stats()["kv_pages"] == len(held) == 2
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_kv_blocks_and_prefetch_match_oracle(seed):
+    rng = np.random.default_rng(200 + seed)
+    n_ad = 30
+    ranks = rng.choice([0, 8, 16], n_ad)
+    pool = _host_pool(n_pages=160)
+    _register_all(pool, ranks)
+    need = [pool.pages_for_rank(int(r)) for r in ranks]
+    held, calls, got_status, got_res = [], [], [], []
+    for _ in range(160):
+        u = rng.random()
+        if u < 0.45:
+            call = ("page_in", rng.choice(n_ad, size=int(rng.integers(1, 5))).tolist(), 0)
+        elif u < 0.6:
+            call = ("prefetch", rng.choice(n_ad, size=int(rng.integers(1, 5))).tolist(),
+                    int(rng.integers(0, 120)))
+        elif u < 0.8:
+            call = ("kv_alloc", [], int(rng.integers(0, 60)))
+        else:
+            call = ("kv_free", [], int(rng.integers(0, len(held) + 1)))
+        kind, ids, n = call
+        st = 0
+        try:
+            if kind == "page_in":
+                pool.page_in(ids)
+            elif kind == "prefetch":
+                G.slora_adapter_prefetch(pool.h, ids, n)
+            elif kind == "kv_alloc":
+                held += G.slora_kv_alloc(pool.h, n)
+            else:
+                pick = set(rng.choice(len(held), size=n, replace=False).tolist())
+                G.slora_kv_free(pool.h, [held[i] for i in sorted(pick)])
+                held = [h for i, h in enumerate(held) if i not in pick]
+        except G.SloraError as e:
+            st = e.status
+        calls.append(call)
+        got_status.append(st)
+        got_res.append([G.slora_adapter_is_resident(pool.h, a) for a in range(n_ad)])
+        assert len(set(held)) == len(held)
+        s = pool.stats()
+        assert s["kv_pages"] == len(held)
+        assert s["free_pages"] + len(held) + sum(need[a] for a in range(n_ad) if got_res[-1][a]) == 160
+    status, res = oracle.lru_prefetch_run(need, 160, calls)
+    assert got_status == status.tolist()
+    assert got_res == res.tolist()
+    assert 2 in got_status                       # the trace reached an OOM
+
+
+def test_kv_free_checks_ids_and_pages_are_never_evicted():
+    pool = _host_pool(n_pages=100)
+    _register_all(pool, [8, 8])                  # 48 pages each
+    kv = G.slora_kv_alloc(pool.h, 40)
+    assert len(set(kv)) == 40 and pool.stats()["kv_pages"] == 40
+    with pytest.raises(G.SloraError) as e:       # 96 pages needed, only 60 are not KV
+        pool.page_in([0, 1])
+    assert e.value.status == 2
+    pool.page_in([0])
+    for bad in ([kv[0], kv[0]], [kv[0], 10 ** 6], [i for i in range(100) if i not in kv][:1]):
+        with pytest.raises(G.SloraError) as e:
+            G.slora_kv_free(pool.h, bad)
+        assert e.value.status == 1
+    assert pool.stats()["kv_pages"] == 40        # nothing changed
+    with pytest.raises(G.SloraError):
+        G.slora_pool_set_page_order(pool.h, list(range(100)))
+    G.slora_kv_free(pool.h, kv[:36])
+    pool.page_in([0, 1])                         # 12 free + 36 returned = 48
+    assert G.slora_adapter_is_resident(pool.h, 0) and G.slora_adapter_is_resident(pool.h, 1)
+    assert pool.stats()["free_pages"] == 0

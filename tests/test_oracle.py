@@ -298,3 +298,28 @@ def test_prefetch_without_prefetch_calls_is_lru():
     s1, r1, _ = oracle.lru_run(need, 30, calls)
     s2, r2 = oracle.lru_prefetch_run(need, 30, [("page_in", c, 0) for c in calls])
     assert np.array_equal(s1, s2) and np.array_equal(r1, r2)
+
+
+# KV blocks sharing the pool, worked by hand (a0, a1 need 4 pages, a2 needs 2;
+# capacity 10):
+#  1 page_in [0]   E=1  {0}              used 4
+#  2 kv_alloc 4         free 6 -> kv 4   {0}
+#  3 page_in [1]   E=2  free 2 < 4: a0 (oldest) evicted   {1}
+#  4 kv_alloc 4         free 2; a1 has age 2 = E, not evictable: OOM
+#  5 page_in [2]   E=3  free 2 fits a2   {1,2}
+#  6 kv_alloc 4         free 0; a1 (age 2 < 3) evicted -> kv 8   {2}
+#  7 kv_free 6          kv 2
+#  8 page_in [0,1] E=4  free 6 < 8: a2 evicted   {0,1}
+KV_TRACE = dict(
+    need=[4, 4, 2], capacity=10,
+    calls=[("page_in", [0], 0), ("kv_alloc", [], 4), ("page_in", [1], 0), ("kv_alloc", [], 4),
+           ("page_in", [2], 0), ("kv_alloc", [], 4), ("kv_free", [], 6), ("page_in", [0, 1], 0)],
+    status=[0, 0, 0, 2, 0, 0, 0, 0],
+    resident=[[0], [0], [1], [1], [1, 2], [2], [2], [0, 1]])
+
+
+def test_kv_blocks_hand_trace():
+    t = KV_TRACE
+    status, res = oracle.lru_prefetch_run(t["need"], t["capacity"], t["calls"])
+    assert status.tolist() == t["status"]
+    assert [np.flatnonzero(r).tolist() for r in res] == t["resident"]
