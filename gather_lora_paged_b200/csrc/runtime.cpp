@@ -681,7 +681,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
       avail += (int64_t)P->ad[it->second].pages.size();
     }
   }
-  if (n_done) *n_done = (int32_t)missing.size();
+  if (n_done) *n_done = 0;
   if (P->inject_after >= 0 && !missing.empty()) {
     if (P->inject_after == 0) {
       P->inject_after = -1;
@@ -745,6 +745,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
   P->st.epoch = P->epoch;
   P->st.free_pages = (int64_t)P->free_pages.size();
   P->st.resident = (int64_t)P->lru.size();
+  if (n_done) *n_done = (int32_t)missing.size();
   if (P->d.host_only) return SLORA_OK;
 
   // ---- device work on the side stream
