@@ -716,7 +716,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
       if (f.rel >= 0) rel_wait.insert(f.rel);
     }
     A.resident = true;
-    P->st.page_ins++;
+    if (!prefetch) P->st.page_ins++;
     (prefetch ? P->st.bytes_prefetched : P->st.bytes_paged_in) += 2 * (int64_t)A.rank *
         [&] { int64_t s = 0; for (int p = 0; p < P->d.n_proj; ++p) s += P->d.d_in[p] + P->d.d_out[p]; return s; }();
   }

@@ -117,7 +117,7 @@ typedef struct {
 } slora_pool_desc;
 
 typedef struct {
-  int64_t page_ins;         /* adapters copied host -> device                        */
+  int64_t page_ins;         /* adapters copied host -> device by page_in             */
   int64_t hits;             /* page-in requests that found the adapter resident      */
   int64_t evictions;        /* adapters evicted by LRU or slora_adapter_evict        */
   int64_t bytes_paged_in;   /* weight bytes copied host -> device                    */
