@@ -33,6 +33,10 @@ def lib():
         L.oracle_pages_needed.restype = i64
         L.oracle_lru_run.argtypes = [i32, P, i64, i32, P, P, P, P, P, P]
         L.oracle_lru_prefetch_run.argtypes = [i32, P, i64, i32, P, P, P, P, P, P]
+        L.oracle_decode_e4m3.argtypes = [P, i64, P]
+        L.oracle_quantize_e4m3.argtypes = [P, i64, ctypes.c_double, P]
+        L.oracle_lora_delta_q8.argtypes = [i32, i32, i32, i32, P, i64, P, P, i64, i32, P, P, P, P,
+                                           P, P, P, i32]
         _lib = L
     return _lib
 
@@ -94,6 +98,67 @@ def lora_delta(dtype, x, idx, y_in, ranks, alphas, A_t, B, n_threads=1):
                                  ctypes.cast(pb, ctypes.c_void_p), _p(y_out), int(n_threads))
     if rc != 0:
         raise ValueError("oracle_lora_delta: invalid argument")
+    return y_out
+
+
+def decode_e4m3(codes):
+    """e4m3 codes (uint8) -> exact fp64 values (NaN for 0x7f / 0xff)."""
+    codes = _c(codes, np.uint8)
+    out = np.empty(codes.shape, np.float64)
+    lib().oracle_decode_e4m3(_p(codes), codes.size, _p(out))
+    return out
+
+
+def quantize_e4m3(values, scale):
+    """Nearest e4m3 codes of values / scale (ties: even fraction; saturating
+    at +-448); all zero codes when scale == 0."""
+    v = _c(values, np.float64)
+    out = np.empty(v.shape, np.uint8)
+    if lib().oracle_quantize_e4m3(_p(v), v.size, float(scale), _p(out)) != 0:
+        raise ValueError("oracle_quantize_e4m3: invalid argument")
+    return out
+
+
+def quantize_rows_e4m3(values):
+    """Per-row quantisation of a (rows, n) fp64 array: scale = max|row| / 448
+    stored as fp32, codes = nearest e4m3 of row / scale.  Returns (codes,
+    scales)."""
+    values = np.asarray(values, np.float64)
+    scales = (np.abs(values).max(axis=1, initial=0.0) / 448.0).astype(np.float32)
+    codes = np.stack([quantize_e4m3(row, float(s)) for row, s in zip(values, scales)]) \
+        if values.shape[0] else np.zeros(values.shape, np.uint8)
+    return codes, scales
+
+
+def lora_delta_q8(dtype, x, idx, y_in, ranks, alphas, qA_t, sA, qB, sB, n_threads=1):
+    """As lora_delta, with adapter a's weights as e4m3 codes qA_t[a] (r_a,
+    d_in), qB[a] (r_a, d_out) and fp32 row scales sA[a], sB[a] (r_a,)."""
+    x = _c(x, np.uint16)
+    T, d_in = x.shape
+    idx = _c(idx, np.int32)
+    n_ad = len(ranks)
+    y_in = _c(y_in, np.uint16)
+    d_out = y_in.shape[1]
+    ranks = _c(ranks, np.int32)
+    alphas = _c(alphas, np.float64)
+    keep = []
+    ptr = [(ctypes.c_void_p * max(n_ad, 1))() for _ in range(4)]
+    for a in range(n_ad):
+        if qA_t[a] is not None and ranks[a] > 0:
+            arrs = [_c(qA_t[a], np.uint8), _c(sA[a], np.float32), _c(qB[a], np.uint8),
+                    _c(sB[a], np.float32)]
+            assert arrs[0].shape == (ranks[a], d_in) and arrs[2].shape == (ranks[a], d_out)
+            assert arrs[1].shape == arrs[3].shape == (ranks[a],)
+            keep += arrs
+            for q in range(4):
+                ptr[q][a] = arrs[q].ctypes.data
+    y_out = np.empty((T, d_out), np.float64)
+    rc = lib().oracle_lora_delta_q8(dtype, T, d_in, d_out, _p(x), d_in, _p(idx), _p(y_in), d_out,
+                                    n_ad, _p(ranks), _p(alphas),
+                                    *[ctypes.cast(q, ctypes.c_void_p) for q in ptr], _p(y_out),
+                                    int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_lora_delta_q8: invalid argument")
     return y_out
 
 

@@ -31,6 +31,14 @@
  *                         tensors is laid out flat over fixed-size pages, so that
  *                         only the last page of each tensor is partly empty
  *                         (same page's section on the unified paged pool).
+ *  oracle_decode_e4m3, oracle_quantize_e4m3, oracle_lora_delta_q8 -- the delta
+ *                         with 8-bit adapter weights (e4m3, one fp32 scale per
+ *                         rank row): "Multi-LoRA serving", trade-offs section
+ *                         (adapters quantised to FP8 or INT4 halve their PCIe
+ *                         traffic and let more of them stay resident) and SGMV
+ *                         section (the segmented kernels exist in FP8 form).  The
+ *                         per-row scale is a reading: the page gives none.  Test
+ *                         infrastructure ahead of the kernels for that format.
  *  oracle_lru_run      -- least-recently-used residency decisions over a trace
  *                         of page-in calls ("Paper explainer: S-LoRA", section
  *                         "Unified Paging", eviction strategy).
@@ -485,5 +493,144 @@ int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int
   free(mark);
   free(tmp);
   free(order);
+  return OR_OK;
+}
+
+/* ------------------------------------------------------------------------- */
+/* 8-bit adapter weights.                                                     */
+/* e4m3 in its "fn" form: 1 sign, 4 exponent (bias 7), 3 fraction bits, no
+ * infinities; exponent 15 with fraction 7 is NaN; the largest finite value is
+ * 448 (exponent 15, fraction 6). */
+static double dec_e4m3(uint8_t b) {
+  int s = (b >> 7) & 1, e = (b >> 3) & 0xf, f = b & 7;
+  double v;
+  if (e == 15 && f == 7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)f, -9); /* subnormal: f * 2^-3 * 2^-6 */
+  else
+    v = ldexp((double)(f + 8), e - 10); /* (1.f) * 2^(e-7) */
+  return s ? -v : v;
+}
+
+int oracle_decode_e4m3(const uint8_t* in, long n, double* out) {
+  for (long i = 0; i < n; ++i) out[i] = dec_e4m3(in[i]);
+  return OR_OK;
+}
+
+/* The finite e4m3 value nearest to v, found by trying every non-negative
+ * finite code; a tie goes to the code with an even fraction; beyond 448 the
+ * result saturates at +-448.  v must not be NaN. */
+static uint8_t enc_e4m3(double v) {
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const double a = fabs(v);
+  int best = 0;
+  double best_d = INFINITY;
+  for (int c = 0; c <= 0x7e; ++c) {
+    const double d = fabs(a - dec_e4m3((uint8_t)c));
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* out[i] = the e4m3 code nearest to in[i] / scale (scale > 0), or 0 when
+ * scale == 0 (an all-zero row). */
+int oracle_quantize_e4m3(const double* in, long n, double scale, uint8_t* out) {
+  if (!(scale >= 0)) return OR_ERR_ARG;
+  for (long i = 0; i < n; ++i) {
+    if (isnan(in[i])) return OR_ERR_ARG;
+    out[i] = scale == 0 ? 0 : enc_e4m3(in[i] / scale);
+  }
+  return OR_OK;
+}
+
+typedef struct {
+  int dtype, T, d_in, d_out;
+  const uint16_t* x;
+  long ldx;
+  const int* idx;
+  const uint16_t* y_in;
+  long ldy;
+  const int* rank;
+  const double* alpha;
+  const uint8_t* const* qA; /* [adapter] -> rank x d_in codes  */
+  const float* const* sA;   /* [adapter] -> rank row scales    */
+  const uint8_t* const* qB; /* [adapter] -> rank x d_out codes */
+  const float* const* sB;
+  double* y_out;
+  int t0, t1;
+} q8_job;
+
+static void* q8_worker(void* arg) {
+  q8_job* J = (q8_job*)arg;
+  double* t = NULL;
+  int tcap = 0;
+  for (int i = J->t0; i < J->t1; ++i) {
+    double* yo = J->y_out + (long)i * J->d_out;
+    const uint16_t* yi = J->y_in ? J->y_in + (long)i * J->ldy : NULL;
+    for (int l = 0; l < J->d_out; ++l) yo[l] = yi ? dec(J->dtype, yi[l]) : 0.0;
+    int a = J->idx[i];
+    if (a < 0) continue;
+    int r = J->rank[a];
+    if (r == 0) continue;
+    if (r > tcap) {
+      free(t);
+      t = (double*)malloc(sizeof(double) * r);
+      tcap = r;
+    }
+    const uint16_t* xi = J->x + (long)i * J->ldx;
+    /* shrink: t[k] = sA[k] * sum_j x[j] * qA[k][j] */
+    for (int k = 0; k < r; ++k) {
+      double acc = 0.0;
+      for (int j = 0; j < J->d_in; ++j)
+        acc += dec(J->dtype, xi[j]) * dec_e4m3(J->qA[a][(long)k * J->d_in + j]);
+      t[k] = (double)J->sA[a][k] * acc;
+    }
+    /* expand and scale: y[l] += (alpha / r) * sum_k t[k] * (sB[k] * qB[k][l]) */
+    double s = J->alpha[a] / (double)r;
+    for (int l = 0; l < J->d_out; ++l) {
+      double acc = 0.0;
+      for (int k = 0; k < r; ++k)
+        acc += t[k] * ((double)J->sB[a][k] * dec_e4m3(J->qB[a][(long)k * J->d_out + l]));
+      yo[l] += s * acc;
+    }
+  }
+  free(t);
+  return NULL;
+}
+
+/* As oracle_lora_delta, with adapter a's weights given as e4m3 codes and one
+ * fp32 scale per rank row: A[j][k] = sA[k] * e4m3(qA[k][j]) (A held
+ * transposed, rank-major), B[k][l] = sB[k] * e4m3(qB[k][l]). */
+int oracle_lora_delta_q8(int dtype, int T, int d_in, int d_out, const uint16_t* x, long ldx,
+                         const int* idx, const uint16_t* y_in, long ldy, int n_adapters,
+                         const int* rank, const double* alpha, const uint8_t* const* qA,
+                         const float* const* sA, const uint8_t* const* qB, const float* const* sB,
+                         double* y_out, int n_threads) {
+  if ((dtype != 0 && dtype != 1) || T < 0 || d_in <= 0 || d_out <= 0 || ldx < d_in ||
+      (y_in && ldy < d_out) || n_threads < 1)
+    return OR_ERR_ARG;
+  for (int i = 0; i < T; ++i) {
+    const int a = idx[i];
+    if (a < -1 || a >= n_adapters) return OR_ERR_ARG;
+    if (a >= 0 && (rank[a] < 0 || (rank[a] > 0 && (!qA[a] || !sA[a] || !qB[a] || !sB[a]))))
+      return OR_ERR_ARG;
+  }
+  if (n_threads > T) n_threads = T > 0 ? T : 1;
+  q8_job* jobs = (q8_job*)calloc(n_threads, sizeof(q8_job));
+  pthread_t* th = (pthread_t*)calloc(n_threads, sizeof(pthread_t));
+  for (int w = 0; w < n_threads; ++w) {
+    q8_job j = {dtype, T, d_in, d_out, x, ldx, idx, y_in, ldy, rank, alpha, qA, sA, qB, sB,
+                y_out, (int)((long)T * w / n_threads), (int)((long)T * (w + 1) / n_threads)};
+    jobs[w] = j;
+  }
+  for (int w = 1; w < n_threads; ++w) pthread_create(&th[w], NULL, q8_worker, &jobs[w]);
+  q8_worker(&jobs[0]);
+  for (int w = 1; w < n_threads; ++w) pthread_join(th[w], NULL);
+  free(jobs);
+  free(th);
   return OR_OK;
 }

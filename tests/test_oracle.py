@@ -323,3 +323,93 @@ def test_kv_blocks_hand_trace():
     status, res = oracle.lru_prefetch_run(t["need"], t["capacity"], t["calls"])
     assert status.tolist() == t["status"]
     assert [np.flatnonzero(r).tolist() for r in res] == t["resident"]
+
+
+# ---------------------------------------------------------------------------
+# 8-bit adapter weights (e4m3 codes with one fp32 scale per rank row)
+
+def test_e4m3_decoder_matches_torch_for_all_codes():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.decode_e4m3(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert got[0x7e] == 448.0 and got[0x01] == 2.0 ** -9 and np.isnan(got[0x7f])
+
+
+def test_e4m3_quantizer_round_trip_ties_and_torch():
+    import torch
+    finite = np.array([c for c in range(256) if c not in (0x7f, 0xff)], np.uint8)
+    vals = oracle.decode_e4m3(finite)
+    assert np.array_equal(oracle.quantize_e4m3(vals, 1.0), finite)      # exact values map back
+    # midpoints of neighbouring positive codes go to the even code
+    pos = np.arange(0, 0x7e, dtype=np.uint8)
+    lo, hi = oracle.decode_e4m3(pos), oracle.decode_e4m3(pos + 1)
+    mids = oracle.quantize_e4m3((lo + hi) / 2, 1.0)
+    assert np.array_equal(mids, np.where(pos % 2 == 0, pos, pos + 1).astype(np.uint8))
+    # random fp32 inputs: torch's float -> e4m3 conversion rounds to nearest even too
+    rng = np.random.default_rng(0)
+    v = (rng.standard_normal(20000) * rng.choice([1e-3, 0.1, 1, 30, 200], 20000)).astype(np.float32)
+    v = np.clip(v, -448, 448)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.quantize_e4m3(v.astype(np.float64), 1.0), ref)
+    assert oracle.quantize_e4m3([1e6, -1e6], 1.0).tolist() == [0x7e, 0xfe]   # saturates
+    assert oracle.quantize_e4m3([3.0, -2.0], 0.0).tolist() == [0, 0]
+
+
+def test_e4m3_row_quantisation_error_bound():
+    rng = np.random.default_rng(1)
+    rows = rng.standard_normal((16, 300)) * rng.uniform(1e-3, 10, (16, 1))
+    rows[3] = 0.0
+    codes, scales = oracle.quantize_rows_e4m3(rows)
+    deq = oracle.decode_e4m3(codes) * scales[:, None].astype(np.float64)
+    s = scales[:, None].astype(np.float64)
+    # half an ulp: 2^-4 of the magnitude for normals, 2^-10 of the scale below them
+    bound = np.maximum(np.abs(rows) * 2.0 ** -4, s * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(deq - rows) <= bound)
+    assert np.all(deq[3] == 0) and scales[3] == 0
+    assert np.all(np.abs(oracle.decode_e4m3(codes)).max(axis=1)[scales > 0] <= 448)
+
+
+def _q8_case(seed, T=9, d_in=96, d_out=80, ranks=(4, 8, 0)):
+    rng = np.random.default_rng(seed)
+    x = to_bits(F16, rng.standard_normal((T, d_in)).astype(np.float32))
+    y = to_bits(F16, rng.standard_normal((T, d_out)).astype(np.float32))
+    idx = rng.integers(-1, len(ranks), T).astype(np.int32)
+    finite = np.array([c for c in range(256) if c not in (0x7f, 0xff)], np.uint8)
+    qA = [rng.choice(finite, (r, d_in)) for r in ranks]
+    qB = [rng.choice(finite, (r, d_out)) for r in ranks]
+    return x, y, idx, np.array(ranks, np.int32), qA, qB
+
+
+def test_q8_delta_with_unit_scales_is_the_16bit_delta():
+    """e4m3 values are exact in fp16: with scales 1 the 8-bit delta must equal
+    the 16-bit oracle on the decoded weights, bit for bit."""
+    x, y, idx, ranks, qA, qB = _q8_case(2)
+    ones = [np.ones(r, np.float32) for r in ranks]
+    got = oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0), qA, ones, qB, ones)
+    to16 = lambda q: oracle.decode_e4m3(q).astype(np.float16).view(np.uint16)
+    ref = oracle.lora_delta(F16, x, idx, y, ranks, np.full(3, 16.0), [to16(q) for q in qA],
+                            [to16(q) for q in qB])
+    assert np.array_equal(got, ref)
+
+
+def test_q8_delta_scales_enter_per_row():
+    x, y, idx, ranks, qA, qB = _q8_case(3)
+    ones = [np.ones(r, np.float32) for r in ranks]
+    base = oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0), qA, ones, qB, ones)
+    # powers of two cancel exactly: (2 sA) with (sB / 2)
+    two = [np.full(r, 2.0, np.float32) for r in ranks]
+    half = [np.full(r, 0.5, np.float32) for r in ranks]
+    assert np.array_equal(base, oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0),
+                                                     qA, two, qB, half))
+    # zeroing one row's scale removes exactly that rank row's contribution
+    sA = [np.ones(r, np.float32) for r in ranks]
+    sA[1][5] = 0.0
+    qA2 = [q.copy() for q in qA]
+    qA2[1][5] = 0
+    a = oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0), qA, sA, qB, ones)
+    b = oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0), qA2, ones, qB, ones)
+    assert np.array_equal(a, b)
