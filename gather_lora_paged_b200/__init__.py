@@ -72,6 +72,7 @@ def lib():
         "slora_adapter_page_in": ([P, P, I32, P, P], I32),
         "slora_adapter_prefetch": ([P, P, I32, I64, P, P, POINTER(c_int32)], I32),
         "slora_prefetch_candidates": ([P, ctypes.c_double, I32, P, POINTER(c_int32)], I32),
+        "slora_quantize_e4m3_rows": ([I32, P, I64, I64, P, P], I32),
         "slora_kv_alloc": ([P, I64, P, P, P], I32),
         "slora_kv_free": ([P, P, I64, P], I32),
         "slora_adapter_evict": ([P, I32, P], I32),
@@ -211,6 +212,18 @@ def slora_prefetch_candidates(pool: int, half_life: float, max_n: int) -> list:
     _check(pool, lib().slora_prefetch_candidates(pool, float(half_life), int(max_n),
                                                  ctypes.cast(out, c_void_p), ctypes.byref(n)))
     return [int(out[i]) for i in range(n.value)]
+
+
+def slora_quantize_e4m3_rows(dtype: int, bits):
+    """(rows, n) 16-bit host values -> (codes uint8 (rows, n), scales float32 (rows,))."""
+    import numpy as np
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    rows, n = bits.shape
+    codes = np.empty((rows, n), np.uint8)
+    scales = np.empty(max(rows, 1), np.float32)
+    _check(None, lib().slora_quantize_e4m3_rows(dtype, bits.ctypes.data, rows, n, codes.ctypes.data,
+                                                scales.ctypes.data))
+    return codes, scales[:rows]
 
 
 def slora_kv_alloc(pool: int, n: int, stream=None, done_event=None) -> list:

@@ -1191,6 +1191,65 @@ slora_status_t slora_check_device(slora_pool* P, void* stream, int32_t* code, in
   return P->fail(SLORA_ERR_DEVICE_CHECK, "kernel recorded code " + std::to_string(w[0]) + " at " + std::to_string(w[1]));
 }
 
+// ---------------------------------------------------------------------------
+// Host-side quantisation of adapter rows to e4m3 (the registration step of
+// 8-bit adapter pages).
+
+// Exact value of a 16-bit element: fp16 (1/5/10) or bf16 (1/8/7).
+static double value16(int dtype, uint16_t h) {
+  if (dtype == SLORA_BF16) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+  }
+  const int s = h >> 15, e = (h >> 10) & 31, m = h & 1023;
+  double v = e == 0 ? std::ldexp((double)m, -24)
+                    : e == 31 ? (m ? NAN : INFINITY) : std::ldexp((double)(m | 1024), e - 25);
+  return s ? -v : v;
+}
+
+// e4m3 code of a finite q, rounded to nearest with ties to an even fraction,
+// saturating at +-448: the exponent from frexp, the 3 fraction bits by one
+// rint (the current rounding mode, nearest-even) of the exactly scaled value.
+static uint8_t e4m3_of(double q) {
+  const uint8_t sign = std::signbit(q) ? 0x80 : 0x00;
+  const double a = std::fabs(q);
+  if (a >= 448.0) return sign | 0x7e;
+  int e;
+  std::frexp(a, &e);  // a = m * 2^e, m in [0.5, 1)
+  int code;
+  if (a < 0.015625) {  // below 2^-6: subnormal steps of 2^-9
+    code = (int)std::rint(std::ldexp(a, 9));  // 8 carries into the first normal code
+  } else {
+    const int E = e - 1;                                     // a in [2^E, 2^(E+1))
+    const int f = (int)std::rint(std::ldexp(a, 3 - E)) - 8;  // 0..8
+    code = ((E + 7) << 3) + f;                               // f = 8 carries into the exponent
+  }
+  return sign | (uint8_t)std::min(code, 0x7e);
+}
+
+slora_status_t slora_quantize_e4m3_rows(int32_t dtype, const uint16_t* in, int64_t rows, int64_t n,
+                                        uint8_t* codes, float* scales) {
+  if ((dtype != SLORA_F16 && dtype != SLORA_BF16) || rows < 0 || n < 0 ||
+      (rows > 0 && n > 0 && (!in || !codes)) || (rows > 0 && !scales))
+    return SLORA_ERR_INVALID_ARG;
+  for (int64_t r = 0; r < rows; ++r) {
+    const uint16_t* row = in + r * n;
+    double amax = 0.0;
+    for (int64_t j = 0; j < n; ++j) {
+      const double v = value16(dtype, row[j]);
+      if (!std::isfinite(v)) return SLORA_ERR_INVALID_ARG;
+      amax = std::max(amax, std::fabs(v));
+    }
+    const float sc = (float)(amax / 448.0);
+    scales[r] = sc;
+    for (int64_t j = 0; j < n; ++j)
+      codes[r * n + j] = sc == 0.0f ? 0 : e4m3_of(value16(dtype, row[j]) / (double)sc);
+  }
+  return SLORA_OK;
+}
+
 slora_status_t slora_pool_stats(const slora_pool* P, slora_pool_stats_t* out) {
   if (!P || !out) return SLORA_ERR_INVALID_ARG;
   *out = P->st;

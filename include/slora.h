@@ -382,6 +382,19 @@ slora_status_t slora_check_device(slora_pool* pool, void* stream, int32_t* code,
 
 slora_status_t slora_pool_stats(const slora_pool* pool, slora_pool_stats_t* out);
 
+/* Quantises `rows` rows of n 16-bit values (in, row-major, fp16 or bf16 per
+ * dtype; host memory) to e4m3 codes with one fp32 scale per row, the storage
+ * of 8-bit adapter pages [S2 trade-offs section: adapters quantised to FP8
+ * halve their PCIe traffic]: scales[r] = max|row r| / 448 (computed in fp64,
+ * stored as fp32); codes[r*n + j] = the e4m3 value nearest to in / scales[r]
+ * (fp64 quotient; ties to the even fraction; saturating at +-448; e4m3 in its
+ * finite-only form, 4 exponent bits with bias 7 and 3 fraction bits).  An
+ * all-zero row gets scale 0 and zero codes.  Host work only.
+ * Errors: INVALID_ARG (bad dtype or sizes, NULL buffers, a NaN or infinite
+ * input).                                                                    */
+slora_status_t slora_quantize_e4m3_rows(int32_t dtype, const uint16_t* in, int64_t rows, int64_t n,
+                                        uint8_t* codes, float* scales);
+
 /* Timing hook for measuring device time without host gaps.  n = 2: every
  * following compute call records events[0] on its stream right before its
  * first kernel and events[1] right after its last one (the kernels stay back

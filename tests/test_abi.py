@@ -389,3 +389,28 @@ def test_kv_free_checks_ids_and_pages_are_never_evicted():
     pool.page_in([0, 1])                         # 12 free + 36 returned = 48
     assert G.slora_adapter_is_resident(pool.h, 0) and G.slora_adapter_is_resident(pool.h, 1)
     assert pool.stats()["free_pages"] == 0
+
+
+@pytest.mark.parametrize("dtype", [G.SLORA_F16, G.SLORA_BF16])
+def test_e4m3_row_quantiser_matches_oracle(dtype):
+    """The library's host quantiser (frexp / rint) against the oracle's
+    (nearest code by trying every code), codes and scales bit for bit."""
+    rng = np.random.default_rng(dtype)
+    rows = rng.standard_normal((40, 257)) * rng.choice([1e-6, 1e-3, 1.0, 50.0, 3e3], (40, 1))
+    rows = np.clip(rows, -6e4, 6e4)         # finite in fp16
+    rows[5] = 0.0
+    rows[6, :] = 0.0
+    rows[6, 3] = -0.0
+    rows[7, 10] = 1e-7                       # lone tiny value: subnormal codes
+    bits = __import__("workloads").to_bits(dtype, rows.astype(np.float32))
+    codes, scales = G.slora_quantize_e4m3_rows(dtype, bits)
+    vals = oracle.decode16(bits, dtype)
+    ref_codes, ref_scales = oracle.quantize_rows_e4m3(vals)
+    assert np.array_equal(scales.view(np.uint32), ref_scales.view(np.uint32))
+    assert np.array_equal(codes, ref_codes)
+    assert scales[5] == 0 and not codes[5].any()
+    nan = bits.copy()
+    nan[2, 2] = 0x7E00 if dtype == G.SLORA_F16 else 0x7FC0
+    with pytest.raises(G.SloraError) as e:
+        G.slora_quantize_e4m3_rows(dtype, nan)
+    assert e.value.status == 1
