@@ -82,8 +82,8 @@ def test_reference_arm_runs_on_rank0_only():
 
 @pytest.mark.timeout(300)
 def test_reference_arm_under_torchrun_two_ranks():
-    """`bench.py --impl reference` launched like the driver's N=2 run: rank 0
-    prints one JSON line, rank 1 exits 0 without work."""
+    """`bench.py --impl reference` launched as a two-process torchrun job:
+    rank 0 prints one JSON line, rank 1 exits 0 without work."""
     port = _free_port()
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
            "--master-addr", "127.0.0.1", "--master-port", str(port),
