@@ -222,12 +222,12 @@ def lru_run(need, capacity, calls):
 def lru_prefetch_run(need, capacity, calls):
     """Run the LRU rules with prefetch and KV-block calls over `calls`, a
     list of (kind, ids, n): kind "page_in", "prefetch" (n = page budget),
-    "kv_alloc" or "kv_free" (n pages; ids unused).
+    "kv_alloc" or "kv_free" (n pages; ids unused), "evict" (ids = [one id]).
 
     Returns (status[c], resident[c, a] bool)."""
     need = _c(need, np.int64)
     n_ad = need.size
-    kinds = {"page_in": 0, "prefetch": 1, "kv_alloc": 2, "kv_free": 3}
+    kinds = {"page_in": 0, "prefetch": 1, "kv_alloc": 2, "kv_free": 3, "evict": 4}
     kind = _c([kinds[k] for k, _, _ in calls], np.int32)
     budget = _c([int(b) for _, _, b in calls], np.int64)
     off = np.zeros(len(calls) + 1, np.int32)

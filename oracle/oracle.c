@@ -372,7 +372,10 @@ int oracle_lru_run(int n_adapters, const long* need, long capacity, int n_calls,
  *     resident adapters older than E are evicted, oldest first (equal ages:
  *     lower id first); if even all of those cannot make room: OOM, nothing
  *     changes;
- *   3 (KV blocks return budget[c] pages).
+ *   3 (KV blocks return budget[c] pages);
+ *   4 (explicit eviction of the one adapter ids[call_off[c]]): ARG if it is
+ *     out of range, NOT_RESIDENT (3) if it is not resident, else it leaves the
+ *     pool (ages and E unchanged).
  * Pages held by KV blocks are neither free nor evictable.
  * Ages start at -1 (never used); E starts at 0.
  */
@@ -387,6 +390,20 @@ int oracle_lru_prefetch_run(int n_adapters, const long* need, long capacity, int
   for (int a = 0; a < n_adapters; ++a) age[a] = -1;
   long used = 0, kv = 0, E = 0;
   for (int c = 0; c < n_calls; ++c) {
+    if (kind[c] == 4) {
+      const int a = call_off[c + 1] > call_off[c] ? ids[call_off[c]] : -1;
+      if (a < 0 || a >= n_adapters) {
+        status[c] = OR_ERR_ARG;
+      } else if (!res[a]) {
+        status[c] = 3;
+      } else {
+        res[a] = 0;
+        used -= need[a];
+        status[c] = OR_OK;
+      }
+      memcpy(resident + (long)c * n_adapters, res, n_adapters);
+      continue;
+    }
     if (kind[c] == 2 || kind[c] == 3) {
       if (kind[c] == 3) {
         kv -= budget[c];

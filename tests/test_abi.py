@@ -337,10 +337,12 @@ def test_kv_blocks_and_prefetch_match_oracle(seed):
         elif u < 0.6:
             call = ("prefetch", rng.choice(n_ad, size=int(rng.integers(1, 5))).tolist(),
                     int(rng.integers(0, 120)))
-        elif u < 0.8:
+        elif u < 0.75:
             call = ("kv_alloc", [], int(rng.integers(0, 60)))
-        else:
+        elif u < 0.9:
             call = ("kv_free", [], int(rng.integers(0, len(held) + 1)))
+        else:
+            call = ("evict", [int(rng.integers(0, n_ad))], 0)
         kind, ids, n = call
         st = 0
         try:
@@ -350,6 +352,8 @@ def test_kv_blocks_and_prefetch_match_oracle(seed):
                 G.slora_adapter_prefetch(pool.h, ids, n)
             elif kind == "kv_alloc":
                 held += G.slora_kv_alloc(pool.h, n)
+            elif kind == "evict":
+                G.slora_adapter_evict(pool.h, ids[0])
             else:
                 pick = set(rng.choice(len(held), size=n, replace=False).tolist())
                 G.slora_kv_free(pool.h, [held[i] for i in sorted(pick)])
