@@ -636,30 +636,49 @@ def oracle_step(w: W.Workload, tokens, threads):
 
 def cpu_baseline(w: W.Workload, budget_s=10.0):
     """The oracle, as it stands, on the host cores over a bounded sample of the
-    workload: whole steps when they fit the budget, else a token subset."""
+    workload: whole steps when one fits the budget, else seeded uniform token
+    subsets (all projections of each sampled token) for about the budget."""
     threads = os.cpu_count() or 1
     w.prefetch_adapters(w.touched().tolist())
+    rng = np.random.default_rng(0)
+    # cost of one token, from a small subset after a warm-up call (neither counted)
+    oracle_step(w, np.arange(min(w.T, 2)), threads)
+    probe = np.sort(rng.choice(w.T, size=min(w.T, 2 * threads), replace=False))
     t0 = time.perf_counter()
-    oracle_step(w, None, threads)
-    dt = time.perf_counter() - t0
-    n_steps, toks = 1, w.T
-    while time.perf_counter() - t0 < budget_s and n_steps < 50:
+    oracle_step(w, probe, threads)
+    per_tok = (time.perf_counter() - t0) / probe.size
+    if per_tok * w.T <= budget_s:
+        t0 = time.perf_counter()
         oracle_step(w, None, threads)
-        n_steps += 1
-    dt = time.perf_counter() - t0
+        n_steps = 1
+        while time.perf_counter() - t0 < budget_s and n_steps < 50:
+            oracle_step(w, None, threads)
+            n_steps += 1
+        dt = time.perf_counter() - t0
+        n_tok = n_steps * w.T
+        sample = (f"{n_steps} whole step(s) of {w.name} ({w.T} tokens x {len(w.projs)} "
+                  f"projections each), fp64 loops, {threads} threads")
+    else:
+        chunk = min(w.T, 4 * threads)
+        t0 = time.perf_counter()
+        n_tok = 0
+        while n_tok == 0 or time.perf_counter() - t0 < budget_s:
+            oracle_step(w, np.sort(rng.choice(w.T, size=chunk, replace=False)), threads)
+            n_tok += chunk
+        dt = time.perf_counter() - t0
+        sample = (f"{n_tok} tokens of {w.name} drawn uniformly in subsets of {chunk} (all "
+                  f"{len(w.projs)} projections of each; a whole step of {w.T} tokens would "
+                  f"take about {per_tok * w.T:.0f} s), fp64 loops, {threads} threads")
     # the same loops on one host thread, over a token subset sized to ~3 s
     t1 = time.perf_counter()
     n1 = 0
-    rng = np.random.default_rng(0)
     while time.perf_counter() - t1 < 3.0 and n1 < w.T:
         tok = np.sort(rng.choice(w.T, size=min(8, w.T), replace=False))
         oracle_step(w, tok, 1)
         n1 += tok.size
     d1 = time.perf_counter() - t1
-    return {"value": n_steps * toks / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{n_steps} whole step(s) of {w.name} ({toks} tokens x {len(w.projs)} "
-                      f"projections each), fp64 loops, {threads} threads",
-            "seconds": dt,
+    return {"value": n_tok / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": sample, "seconds": dt,
             "single_thread": {"value": n1 / d1, "unit": UNIT, "cores": 1,
                               "sample": f"{n1} tokens of the same workload (all {len(w.projs)} "
                                         f"projections), fp64 loops, 1 thread", "seconds": d1}}
