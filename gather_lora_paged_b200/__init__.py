@@ -416,5 +416,17 @@ class Pool:
     def page_in(self, ids, side_stream=None, done_event=None):
         slora_adapter_page_in(self.h, list(ids), side_stream, done_event)
 
+    def prefetch(self, ids, max_pages, side_stream=None, done_event=None) -> int:
+        return slora_adapter_prefetch(self.h, list(ids), max_pages, side_stream, done_event)
+
+    def prefetch_candidates(self, half_life, max_n) -> list:
+        return slora_prefetch_candidates(self.h, half_life, max_n)
+
+    def kv_alloc(self, n, stream=None, done_event=None) -> list:
+        return slora_kv_alloc(self.h, n, stream, done_event)
+
+    def kv_free(self, ids, stream=None) -> None:
+        slora_kv_free(self.h, list(ids), stream)
+
     def stats(self):
         return slora_pool_stats(self.h)

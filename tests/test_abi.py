@@ -418,3 +418,15 @@ def test_e4m3_row_quantiser_matches_oracle(dtype):
     with pytest.raises(G.SloraError) as e:
         G.slora_quantize_e4m3_rows(dtype, nan)
     assert e.value.status == 1
+
+
+def test_pool_convenience_methods():
+    pool = _host_pool(n_pages=100)
+    _register_all(pool, [8, 8, 8])
+    pool.page_in([0])
+    assert pool.prefetch([1, 2], 1000) == 1            # 52 free pages: one rank-8 adapter
+    kv = pool.kv_alloc(4)
+    assert pool.stats()["kv_pages"] == 4
+    pool.kv_free(kv)
+    pool.page_in([0])
+    assert pool.prefetch_candidates(2.0, 5) == []      # only adapter 0 was ever named, and it is resident
