@@ -17,6 +17,7 @@
 // stand-in); the device address is looked up with cudaGetSymbolAddress once per
 // device, on the first call made while that device is current.
 #include <mutex>
+#include <nvtx3/nvToolsExt.h>
 #include <string>
 
 #include "slora_internal.h"
@@ -65,10 +66,13 @@ extern "C" slora_status_t slora_lora_delta_noalloc(slora_pool* pool, int32_t n,
                                                    const int64_t* ldy, const int32_t* idx,
                                                    int32_t T, void* stream) {
   if (!pool) return SLORA_ERR_INVALID_ARG;
+  nvtxRangePushA("slora_lora_delta_noalloc");
   void* scratch = nullptr;
-  cudaError_t e = scratch_address(&scratch);
-  if (e != cudaSuccess) return SLORA_ERR_CUDA;
-  return slora::lora_delta_on_scratch(pool, n, projs, x, ldx, y, ldy, idx, T,
+  slora_status_t st = SLORA_ERR_CUDA;
+  if (scratch_address(&scratch) == cudaSuccess)
+    st = slora::lora_delta_on_scratch(pool, n, projs, x, ldx, y, ldy, idx, T,
                                       static_cast<cudaStream_t>(stream), scratch,
                                       kNoAllocScratchBytes);
+  nvtxRangePop();
+  return st;
 }

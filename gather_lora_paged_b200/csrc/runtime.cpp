@@ -21,6 +21,8 @@
 #include <unordered_set>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "slora_internal.h"
 
 using namespace slora;
@@ -39,6 +41,16 @@ constexpr double kWaitSeconds = 30.0;
 
 int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// An NVTX range around each C-ABI call that enqueues work or changes the pool,
+// so that profilers show the library's calls on the timeline (no cost when no
+// tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kUseHistory = 32;  // page_in namings kept per adapter for the prefetch policy
 
@@ -201,6 +213,7 @@ struct slora_pool {
 
   slora_status_t fail(slora_status_t s, const std::string& m) {
     err = std::string(status_name(s)) + ": " + m;
+    if (getenv("SLORA_LOG")) fprintf(stderr, "slora: %s\n", err.c_str());
     return s;
   }
   slora_status_t cuda_fail(cudaError_t e, const char* where) {
@@ -479,6 +492,7 @@ int64_t slora_pages_for_rank(const slora_pool_desc* d, int32_t rank) {
 }
 
 slora_status_t slora_pool_create(const slora_pool_desc* desc, slora_pool** out) {
+  NvtxRange nvtx_("slora_pool_create");
   if (!out) return SLORA_ERR_INVALID_ARG;
   *out = nullptr;
   std::string why;
@@ -530,6 +544,7 @@ slora_status_t slora_pool_create(const slora_pool_desc* desc, slora_pool** out) 
 }
 
 slora_status_t slora_pool_destroy(slora_pool* P) {
+  NvtxRange nvtx_("slora_pool_destroy");
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (!P->d.host_only) {
     if (P->pagein_done) {
@@ -571,6 +586,7 @@ slora_status_t slora_pool_set_page_order(slora_pool* P, const int32_t* order, in
 
 slora_status_t slora_adapter_register(slora_pool* P, int32_t id, int32_t rank, float alpha,
                                       const void* const* host_A_t, const void* const* host_B) {
+  NvtxRange nvtx_("slora_adapter_register");
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (id < 0 || id >= P->d.max_adapters) return P->fail(SLORA_ERR_INVALID_ARG, "adapter id out of range");
   if (rank < 0 || rank > P->d.max_rank) return P->fail(SLORA_ERR_INVALID_ARG, "rank out of [0, max_rank]");
@@ -863,11 +879,13 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
 
 slora_status_t slora_adapter_page_in(slora_pool* P, const int32_t* ids, int32_t n, void* side_stream,
                                      void* done_event) {
+  NvtxRange nvtx_("slora_adapter_page_in");
   return page_in_impl(P, ids, n, side_stream, done_event, false, 0, nullptr);
 }
 
 slora_status_t slora_adapter_prefetch(slora_pool* P, const int32_t* ids, int32_t n, int64_t max_pages,
                                       void* side_stream, void* done_event, int32_t* n_done) {
+  NvtxRange nvtx_("slora_adapter_prefetch");
   return page_in_impl(P, ids, n, side_stream, done_event, true, max_pages, n_done);
 }
 
@@ -894,6 +912,7 @@ slora_status_t slora_prefetch_candidates(const slora_pool* Pc, double half_life,
 }
 
 slora_status_t slora_kv_alloc(slora_pool* P, int64_t n, int32_t* ids_out, void* stream, void* done_event) {
+  NvtxRange nvtx_("slora_kv_alloc");
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (n < 0 || (n > 0 && !ids_out)) return P->fail(SLORA_ERR_INVALID_ARG, "kv_alloc arguments");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -942,6 +961,7 @@ slora_status_t slora_kv_alloc(slora_pool* P, int64_t n, int32_t* ids_out, void* 
 }
 
 slora_status_t slora_kv_free(slora_pool* P, const int32_t* ids, int64_t n, void* stream) {
+  NvtxRange nvtx_("slora_kv_free");
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (n < 0 || (n > 0 && !ids)) return P->fail(SLORA_ERR_INVALID_ARG, "kv_free arguments");
   std::unordered_set<int32_t> seen;
@@ -969,6 +989,7 @@ slora_status_t slora_kv_free(slora_pool* P, const int32_t* ids, int64_t n, void*
 }
 
 slora_status_t slora_adapter_evict(slora_pool* P, int32_t id, void* stream) {
+  NvtxRange nvtx_("slora_adapter_evict");
   if (!P) return SLORA_ERR_INVALID_ARG;
   if (id < 0 || id >= P->d.max_adapters) return P->fail(SLORA_ERR_INVALID_ARG, "adapter id out of range");
   if (!P->ad[id].resident) return P->fail(SLORA_ERR_NOT_RESIDENT, "adapter " + std::to_string(id));
@@ -1008,6 +1029,7 @@ slora_status_t slora_check_batch(const slora_pool* Pc, const int32_t* idx_host, 
 
 slora_status_t slora_build_segments(slora_pool* P, const int32_t* idx, int32_t T, int32_t* perm,
                                     int32_t* seg_start, int32_t* seg_adapter, int32_t* S_out, void* stream) {
+  NvtxRange nvtx_("slora_build_segments");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
@@ -1029,6 +1051,7 @@ slora_status_t slora_build_segments(slora_pool* P, const int32_t* idx, int32_t T
 slora_status_t slora_build_sgmv_segments(slora_pool* P, const int32_t* req_start, const int32_t* req_adapter,
                                          int32_t n, int32_t* seg_start, int32_t* seg_adapter, int32_t* S_out,
                                          void* stream) {
+  NvtxRange nvtx_("slora_build_sgmv_segments");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
@@ -1042,6 +1065,7 @@ slora_status_t slora_build_sgmv_segments(slora_pool* P, const int32_t* req_start
 slora_status_t slora_lora_delta(slora_pool* P, int32_t n, const int32_t* projs, const void* const* x,
                                 const int64_t* ldx, void* const* y, const int64_t* ldy, const int32_t* idx,
                                 int32_t T, void* stream) {
+  NvtxRange nvtx_("slora_lora_delta");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
@@ -1067,6 +1091,7 @@ slora_status_t slora_lora_delta(slora_pool* P, int32_t n, const int32_t* projs, 
 
 slora_status_t slora_bgmv_shrink(slora_pool* P, int32_t proj, const void* x, int64_t ldx, const int32_t* idx,
                                  int32_t T, float* t, int64_t ldt, void* stream) {
+  NvtxRange nvtx_("slora_bgmv_shrink");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
@@ -1099,6 +1124,7 @@ slora_status_t slora_bgmv_shrink(slora_pool* P, int32_t proj, const void* x, int
 
 slora_status_t slora_bgmv_expand(slora_pool* P, int32_t proj, const float* t, int64_t ldt, const int32_t* idx,
                                  int32_t T, void* y, int64_t ldy, void* stream) {
+  NvtxRange nvtx_("slora_bgmv_expand");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
@@ -1131,6 +1157,7 @@ slora_status_t slora_bgmv_expand(slora_pool* P, int32_t proj, const float* t, in
 slora_status_t slora_sgmv(slora_pool* P, int32_t n, const int32_t* projs, const void* const* x,
                           const int64_t* ldx, void* const* y, const int64_t* ldy, const int32_t* seg_start,
                           const int32_t* seg_adapter, int32_t S, int32_t T, void* stream) {
+  NvtxRange nvtx_("slora_sgmv");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
@@ -1177,6 +1204,7 @@ slora_status_t slora_debug_gather(slora_pool* P, int32_t id, int32_t proj, void*
 }
 
 slora_status_t slora_check_device(slora_pool* P, void* stream, int32_t* code, int32_t* info) {
+  NvtxRange nvtx_("slora_check_device");
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
