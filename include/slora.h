@@ -137,7 +137,9 @@ typedef struct {
 size_t slora_tables_bytes(const slora_pool_desc* desc);
 
 /* Bytes of device scratch for compute calls with up to max_tokens tokens:
- * segment arrays, work counters and the fp32 shrink partials. */
+ * segment arrays, work counters and the fp32 shrink partials.  All compute
+ * calls of a pool use this one scratch, so their kernels must not overlap on
+ * the GPU: issue them on one stream, or order streams with events. */
 size_t slora_scratch_bytes(const slora_pool_desc* desc);
 
 /* Pages one adapter of rank `rank` occupies: sum over projections of
