@@ -321,6 +321,28 @@ def test_kv_hand_trace_through_the_library():
     assert pool.stats()["kv_pages"] == len(held) == 2
 
 
+def test_evict_hand_trace_through_the_library():
+    from test_oracle import EVICT_TRACE as t
+    ranks = [n // 2 for n in t["need"]]          # d_in = d_out = page = 1024: 2 r pages
+    pool = G.Pool(G.SLORA_F16, [1024], [1024], len(ranks), 8, 16, 1024, t["capacity"],
+                  host_only=True)
+    _register_all(pool, ranks)
+    for c, (kind, ids, budget) in enumerate(t["calls"]):
+        st = 0
+        try:
+            if kind == "page_in":
+                pool.page_in(ids)
+            elif kind == "prefetch":
+                G.slora_adapter_prefetch(pool.h, ids, budget)
+            else:
+                G.slora_adapter_evict(pool.h, ids[0])
+        except G.SloraError as e:
+            st = e.status
+        assert st == t["status"][c], c
+        assert [a for a in range(len(ranks)) if G.slora_adapter_is_resident(pool.h, a)] == \
+            t["resident"][c], c
+
+
 @pytest.mark.parametrize("seed", range(4))
 def test_kv_blocks_and_prefetch_match_oracle(seed):
     rng = np.random.default_rng(200 + seed)

@@ -318,6 +318,43 @@ KV_TRACE = dict(
     resident=[[0], [0], [1], [1], [1, 2], [2], [2], [0, 1]])
 
 
+# Explicit eviction, worked by hand from the rules (a0..a2 need 4 pages, a3
+# needs 2; capacity 10; E = page-in calls so far):
+#  1 page_in [0]      E=1  {0}        used 4   age a0=1
+#  2 page_in [1]      E=2  {0,1}      used 8   a1=2
+#  3 evict [2]        a2 is not resident: NOT_RESIDENT (3), nothing changes
+#  4 evict [0]        {1}, used 4; E stays 2, no age moves
+#  5 prefetch [2,3,0] b=100
+#                     room = free 6 + adapters older than E (none: a1's age is
+#                     E) = 6: a2 (4) and a3 (2) fit, a0 does not   {1,2,3}
+#                     (had the evict bumped E, a1 would count as older and a0
+#                     would fit; had it kept a0's pages, only a3 would fit)
+#  6 evict [3]        {1,2}, used 8 (between a prefetch and a page-in)
+#  7 page_in [0] E=3  needs 4, free 2 (a3's pages): oldest unpinned of age 2
+#                     are a1 and a2, lower id first: a1 evicted   {0,2}  a0=3
+#  8 page_in [3] E=4  a3 fits the 2 free pages   {0,2,3}  a3=4
+#  9 evict [3]        {0,2}; ages stay a0=3, a2=2
+# 10 page_in [1] E=5  needs 4, free 2: a2 (age 2) goes before a0 (age 3)
+#                     {0,1}  (had the evict refreshed the residents' ages,
+#                     a0 and a2 would tie and a0 would go)
+# 11 evict [7]        id out of range: ARG (1), nothing changes
+EVICT_TRACE = dict(
+    need=[4, 4, 4, 2], capacity=10,
+    calls=[("page_in", [0], 0), ("page_in", [1], 0), ("evict", [2], 0), ("evict", [0], 0),
+           ("prefetch", [2, 3, 0], 100), ("evict", [3], 0), ("page_in", [0], 0),
+           ("page_in", [3], 0), ("evict", [3], 0), ("page_in", [1], 0), ("evict", [7], 0)],
+    status=[0, 0, 3, 0, 0, 0, 0, 0, 0, 0, 1],
+    resident=[[0], [0, 1], [0, 1], [1], [1, 2, 3], [1, 2], [0, 2], [0, 2, 3], [0, 2], [0, 1],
+              [0, 1]])
+
+
+def test_evict_hand_trace():
+    t = EVICT_TRACE
+    status, res = oracle.lru_prefetch_run(t["need"], t["capacity"], t["calls"])
+    assert status.tolist() == t["status"]
+    assert [np.flatnonzero(r).tolist() for r in res] == t["resident"]
+
+
 def test_kv_blocks_hand_trace():
     t = KV_TRACE
     status, res = oracle.lru_prefetch_run(t["need"], t["capacity"], t["calls"])
