@@ -3,9 +3,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch: the page-in call for
-the batch's adapter set (LRU touch; no copies when all are resident), the
-device segment build, the grouped paged shrink and the grouped expand over
-all projections of one layer.  Default workload: the LLaMA-7B decode layer
+the batch's adapter set (LRU touch; no copies when all are resident), then the
+segment build, the grouped paged shrink and the grouped expand over all
+projections of one layer (decode batches of up to 1024 tokens: all three in one
+persistent kernel).  Default workload: the LLaMA-7B decode layer
 (7 projections, 256 tokens, 1000 resident rank-16 adapters, Zipf 1.0, fp16).
 
 Timing: CUDA events on the compute stream right around the library's kernels
@@ -61,7 +62,7 @@ def peaks():
 # B200's 1.965 GHz): longer than the host takes to enqueue one step.
 HOLD_CYCLES = 200_000
 
-KERNEL_SOURCE = {"shrink": "bgmv.cu", "expand": "bgmv.cu", "segments": "bgmv.cu",
+KERNEL_SOURCE = {"delta": "fused.cu", "shrink": "bgmv.cu", "expand": "bgmv.cu", "segments": "bgmv.cu",
                  "sgmv_shrink": "sgmv.cu", "sgmv_expand": "sgmv.cu"}
 
 
@@ -110,7 +111,9 @@ def job_throughput(world: int, tokens_per_step: int, steps: int, t_ms: float) ->
 # ---------------------------------------------------------------------------
 # algorithmic bytes / flops (each touched adapter and each distinct input read
 # once, y read and written once)
-def algorithmic(w: W.Workload, tokens=None):
+def algorithmic(w: W.Workload, tokens=None, wbytes=2):
+    """wbytes: bytes per adapter weight (2: 16-bit pages, 1: e4m3 codes; the
+    per-row scales add r floats per tensor, counted too)."""
     idx = w.idx if tokens is None else w.idx[tokens]
     T = idx.size
     esz = 2
@@ -119,8 +122,9 @@ def algorithmic(w: W.Workload, tokens=None):
     din = sum(p.d_in for p in w.projs)
     dout = sum(p.d_out for p in w.projs)
     xin = sum(w.x_dim(n) for n in w.x_names)
-    A_bytes = r_sum * din * esz
-    B_bytes = r_sum * dout * esz
+    n_t = len(w.projs)
+    A_bytes = r_sum * din * wbytes + (4 * r_sum * n_t if wbytes == 1 else 0)
+    B_bytes = r_sum * dout * wbytes + (4 * r_sum * n_t if wbytes == 1 else 0)
     x_bytes = T * xin * esz
     y_bytes = 2 * T * dout * esz
     r_tok = w.ranks[idx[idx >= 0]].astype(np.int64)
@@ -132,10 +136,10 @@ def algorithmic(w: W.Workload, tokens=None):
 
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    """SM clock and clock-event (throttle) reasons sampled every 10 ms through
-    NVML while the timed region runs (read-only queries)."""
+    """SM clock and clock-event (throttle) reasons sampled every 2 ms through
+    NVML while the timed passes run (read-only queries)."""
 
-    PERIOD = 0.01
+    PERIOD = 0.002
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap"}
 
@@ -192,23 +196,31 @@ class ClockSampler:
             return None
         reasons = sorted({n for _, m in self.samples for bit, n in self.REASONS.items() if m & bit})
         return {"sm_mhz": float(np.median([c for c, _ in self.samples])), "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(self.samples), "source": "nvml, 10 ms"}
+                "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml, every 2 ms across the per-kernel, timed and warm-L2 passes"}
 
 
 # ---------------------------------------------------------------------------
 class DecodeRun:
     """Decode step: page-in call for the batch's adapter set (LRU touch), then
-    the fused delta (segment build, grouped shrink, grouped expand)."""
-    phases = ("segments", "shrink", "expand")
-    ncu_names = ("segments", "shrink", "expand")
+    the delta over all projections: one persistent kernel for batches of up to
+    1024 tokens, else (or with split=True) segment build, grouped shrink and
+    grouped expand."""
+    FUSED_MAX_T = 1024
 
-    def __init__(self, w):
+    def __init__(self, w, path="auto", weights="16"):
         import torch
 
         import gather_lora_paged_b200 as G
         import harness as H
         self.G, self.H, self.w = G, H, w
-        self.pb = H.PoolBuild(w)
+        self.wbytes = 1 if weights == "e4m3" else 2
+        dp = {"auto": G.SLORA_DECODE_AUTO, "split": G.SLORA_DECODE_SPLIT, "fused": G.SLORA_DECODE_FUSED}[path]
+        self.pb = H.PoolBuild(w, decode_path=dp,
+                              weight_format=G.SLORA_WEIGHTS_E4M3 if weights == "e4m3" else G.SLORA_WEIGHTS_16)
+        fused = G.slora_decode_kernels(self.pb.h, w.T) == 1
+        self.phases = ("delta",) if fused else ("segments", "shrink", "expand")
+        self.ncu_names = self.phases
         self.ten = H.Tensors(w)
         self.d_idx = torch.from_numpy(w.idx).cuda()
         self.touched = w.touched().tolist()
@@ -236,12 +248,11 @@ class DecodeRun:
 class PrefillRun(DecodeRun):
     """Prefill step: page-in call, request -> segment merge on the device, and
     the tensor-core SGMV (plan, shrink, expand) over all projections."""
-    phases = ("plan", "shrink", "expand")
-    ncu_names = ("plan", "sgmv_shrink", "sgmv_expand")
-
     def __init__(self, w):
         import torch
         super().__init__(w)
+        self.phases = ("plan", "shrink", "expand")
+        self.ncu_names = ("plan", "sgmv_shrink", "sgmv_expand")
         n = w.req_adapter.size
         self.n = n
         self.d_rs = torch.from_numpy(w.req_start).cuda()
@@ -276,7 +287,7 @@ def run_ours(args, rank, world):
     w = replica_workload(args.config, rank)
     if args.config == 4:
         return run_mixed(args, rank, world, w)
-    R = PrefillRun(w) if args.config == 3 else DecodeRun(w)
+    R = PrefillRun(w) if args.config == 3 else DecodeRun(w, path=args.path, weights=args.weights)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -284,7 +295,7 @@ def run_ours(args, rank, world):
     for e in ev + outer:  # torch creates the CUDA event on first record
         e.record()
     torch.cuda.synchronize()
-    alg = algorithmic(w)
+    alg = algorithmic(w, wbytes=getattr(R, "wbytes", 2))
 
     def prep():
         R.ten.reset()
@@ -299,22 +310,24 @@ def run_ours(args, rank, world):
     assert st == 0, (code, info)
 
     # pass 1: per-kernel device times (library events between its kernels)
-    R.set_events(ev)
-    kt = [0.0, 0.0, 0.0]
+    nk = len(R.phases)
+    pev = ev[:2] if nk == 1 else ev
+    clocks = ClockSampler(dev)
+    clocks.start()
+    R.set_events(pev)
+    kt = [0.0] * nk
     for _ in range(args.steps):
         prep()
         R.step(stream)
-        ev[3].synchronize()
-        for i in range(3):
-            kt[i] += ev[i].elapsed_time(ev[i + 1])
+        pev[-1].synchronize()
+        for i in range(nk):
+            kt[i] += pev[i].elapsed_time(pev[i + 1])
     R.set_events([])
     # pass 2 (the timed region): whole steps, kernels back to back; the L2
     # flush ahead of each step keeps the GPU busy while the host enqueues it
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(dev)
-    clocks.start()
     t_step = 0.0
     per_step = []
     for _ in range(args.steps):
@@ -324,7 +337,6 @@ def run_ours(args, rank, world):
         per_step.append(outer[0].elapsed_time(outer[1]))
         t_step += per_step[-1]
     torch.cuda.synchronize()
-    clk = clocks.stop()
     if world > 1:
         torch.distributed.barrier()
     t_step = max_over_ranks(t_step, world, "cuda")
@@ -342,6 +354,7 @@ def run_ours(args, rank, world):
         R.step(stream, outer)
         outer[1].synchronize()
         t_warm += outer[0].elapsed_time(outer[1])
+    clk = clocks.stop()
     t_warm = max_over_ranks(t_warm, world, "cuda")
     warm = {"value": job_throughput(world, w.T, Kw, t_warm), "ms_per_step": t_warm / Kw, "steps": Kw,
             "l2": "not flushed between steps"}
@@ -411,8 +424,11 @@ def run_ours(args, rank, world):
     hbm, tc, src = peaks()
     kt = [t / K for t in kt]
     names = R.phases
-    i_dom = 1 if kt[1] >= kt[2] else 2
-    dom_bytes = alg["shrink_bytes"] if i_dom == 1 else alg["expand_bytes"]
+    if nk == 1:  # one kernel runs the whole step
+        i_dom, dom_bytes = 0, alg["total_bytes"]
+    else:
+        i_dom = 1 if kt[1] >= kt[2] else 2
+        dom_bytes = alg["shrink_bytes"] if i_dom == 1 else alg["expand_bytes"]
     achieved = dom_bytes / (kt[i_dom] / 1e3) / 1e9
     step_gbs = alg["total_bytes"] / (ms / 1e3) / 1e9
     tflops = alg["flops"] / (ms / 1e3) / 1e12
@@ -423,8 +439,11 @@ def run_ours(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": W.DTYPE_NAME[w.dtype],
         "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(d_in)) A, N(0,1/sqrt(r)) B; "
                 "Zipf or uniform adapter ids)",
-        "config": {"workload": w.name, "tokens_per_step": w.T, "projections": len(w.projs),
+        "config": {"workload": w.name + ("_e4m3pages" if getattr(R, "wbytes", 2) == 1 else ""),
+                   "tokens_per_step": w.T, "projections": len(w.projs),
                    "adapters": w.n_adapters, "touched_adapters": alg["touched"],
+                   "adapter_weights": "e4m3 codes + fp32 row scales" if getattr(R, "wbytes", 2) == 1
+                   else W.DTYPE_NAME[w.dtype],
                    "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
                    "host_enqueue": "not timed: a ~100 us spin kernel precedes each step's start event",
                    "parallelism": f"replicas x{world}"},
@@ -439,7 +458,7 @@ def run_ours(args, rank, world):
                           "kernel_ms": dict(zip(names, kt))},
         "e2e": e2e,
         "warm_l2": warm,
-        "gpu_launches": (4 if args.config == 3 else 3) * K,
+        "gpu_launches": (4 if args.config == 3 else len(R.phases)) * K,
         "clocks": clk,
     }
     R.pb.close()
@@ -572,7 +591,9 @@ def run_mixed(args, rank, world, w):
         "e2e": {"value": job_throughput(world, w.T, n_e2e, tot), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": tot / n_e2e},
-        "gpu_launches": 8 * K,  # page-in gather, segments, shrink, expand, merge, plan, shrink, expand
+        # page-in gather, the decode delta (one or three kernels), request
+        # merge, SGMV plan, shrink, expand
+        "gpu_launches": (5 + H.G.slora_decode_kernels(M.h, w.n_decode)) * K,
         "clocks": clk,
         "prefetch": pre,
     }
@@ -709,6 +730,11 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", default="auto", choices=["auto", "split", "fused"],
+                    help="decode kernels: the library's choice, the three-kernel path (segment "
+                         "build, shrink, expand) or the one persistent kernel")
+    ap.add_argument("--weights", default="16", choices=["16", "e4m3"],
+                    help="decode: adapter pages in the pool's 16-bit dtype or as e4m3 codes")
     ap.add_argument("--pagein", default="kernel", choices=["kernel", "memcpy"],
                     help="page-in mode of the mixed workload (--config 4)")
     args = ap.parse_args()

@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(_HERE, "libslora.so")
 
 SLORA_F16, SLORA_BF16 = 0, 1
 SLORA_PAGEIN_KERNEL, SLORA_PAGEIN_MEMCPY = 0, 1
+SLORA_DECODE_AUTO, SLORA_DECODE_SPLIT, SLORA_DECODE_FUSED = 0, 1, 2
+SLORA_WEIGHTS_16, SLORA_WEIGHTS_E4M3 = 0, 1
 MAX_PROJ = 8
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "OOM", 3: "NOT_RESIDENT", 4: "CUDA", 5: "TIMEOUT",
@@ -39,7 +41,7 @@ class PoolDesc(ctypes.Structure):
                 ("max_tokens", c_int32), ("pagein_mode", c_int32), ("page_elems", c_int64),
                 ("n_pages", c_int64), ("dev_pool", c_void_p), ("dev_tables", c_void_p),
                 ("dev_scratch", c_void_p), ("scratch_bytes", c_size_t), ("host_only", c_int32),
-                ("reserved", c_int32 * 7)]
+                ("decode_path", c_int32), ("weight_format", c_int32), ("reserved", c_int32 * 5)]
 
 
 class PoolStats(ctypes.Structure):
@@ -69,6 +71,7 @@ def lib():
         "slora_last_error": ([P], ctypes.c_char_p),
         "slora_pool_set_page_order": ([P, P, I64], I32),
         "slora_adapter_register": ([P, I32, I32, c_float, P, P], I32),
+        "slora_adapter_register_e4m3": ([P, I32, I32, c_float, P, P, P, P], I32),
         "slora_adapter_page_in": ([P, P, I32, P, P], I32),
         "slora_adapter_prefetch": ([P, P, I32, I64, P, P, POINTER(c_int32)], I32),
         "slora_prefetch_candidates": ([P, ctypes.c_double, I32, P, POINTER(c_int32)], I32),
@@ -91,6 +94,7 @@ def lib():
         "slora_set_phase_events": ([P, P, I32], I32),
         "slora_lora_delta_noalloc": ([P, I32, P, P, P, P, P, P, I32, P], I32),
         "slora_noalloc_scratch_bytes": ([], c_size_t),
+        "slora_decode_kernels": ([P, I32], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -188,6 +192,18 @@ def slora_adapter_register(pool: int, id: int, rank: int, alpha: float, host_A_t
     pb = _arr(c_void_p, [_ptr(t) for t in host_B])
     _check(pool, lib().slora_adapter_register(pool, id, rank, alpha, ctypes.cast(pa, c_void_p),
                                               ctypes.cast(pb, c_void_p)))
+
+
+def slora_adapter_register_e4m3(pool: int, id: int, rank: int, alpha: float, codes_A_t, scales_A_t,
+                                codes_B, scales_B) -> None:
+    """codes_*: pinned host tensors (uint8); scales_*: host float32 arrays (one per rank row)."""
+    ca = _arr(c_void_p, [_ptr(t) for t in codes_A_t])
+    sa = _arr(c_void_p, [_ptr(t) for t in scales_A_t])
+    cb = _arr(c_void_p, [_ptr(t) for t in codes_B])
+    sb = _arr(c_void_p, [_ptr(t) for t in scales_B])
+    _check(pool, lib().slora_adapter_register_e4m3(pool, id, rank, alpha, ctypes.cast(ca, c_void_p),
+                                                   ctypes.cast(sa, c_void_p), ctypes.cast(cb, c_void_p),
+                                                   ctypes.cast(sb, c_void_p)))
 
 
 def slora_adapter_page_in(pool: int, ids, side_stream=None, done_event=None) -> None:
@@ -331,6 +347,11 @@ def slora_pool_stats(pool: int) -> dict:
     return {f: getattr(s, f) for f, _ in PoolStats._fields_}
 
 
+def slora_decode_kernels(pool: int, T: int) -> int:
+    """Kernels slora_lora_delta launches for T tokens on this pool (1 or 3)."""
+    return int(lib().slora_decode_kernels(pool, int(T)))
+
+
 def slora_set_phase_events(pool: int, events) -> None:
     a = _arr(c_void_p, [_event(e) for e in events])
     _check(pool, lib().slora_set_phase_events(pool, ctypes.cast(a, c_void_p), len(events)))
@@ -342,7 +363,8 @@ def slora_inject_fault(pool: int, after: int) -> None:
 
 # ---------------------------------------------------------------------------
 def make_desc(dtype, d_in, d_out, max_adapters, max_rank, max_tokens, page_elems, n_pages,
-              pagein_mode=SLORA_PAGEIN_KERNEL, host_only=False) -> PoolDesc:
+              pagein_mode=SLORA_PAGEIN_KERNEL, host_only=False,
+              decode_path=SLORA_DECODE_AUTO, weight_format=SLORA_WEIGHTS_16) -> PoolDesc:
     d = PoolDesc()
     d.dtype = dtype
     d.n_proj = len(d_in)
@@ -356,6 +378,8 @@ def make_desc(dtype, d_in, d_out, max_adapters, max_rank, max_tokens, page_elems
     d.page_elems = page_elems
     d.n_pages = n_pages
     d.host_only = 1 if host_only else 0
+    d.decode_path = decode_path
+    d.weight_format = weight_format
     return d
 
 
@@ -364,9 +388,10 @@ class Pool:
     as torch tensors) and the pinned host copies of registered adapters."""
 
     def __init__(self, dtype, d_in, d_out, max_adapters, max_rank, max_tokens, page_elems,
-                 n_pages, pagein_mode=SLORA_PAGEIN_KERNEL, host_only=False, device="cuda"):
+                 n_pages, pagein_mode=SLORA_PAGEIN_KERNEL, host_only=False, device="cuda",
+                 decode_path=SLORA_DECODE_AUTO, weight_format=SLORA_WEIGHTS_16):
         self.desc = make_desc(dtype, d_in, d_out, max_adapters, max_rank, max_tokens, page_elems,
-                              n_pages, pagein_mode, host_only)
+                              n_pages, pagein_mode, host_only, decode_path, weight_format)
         self.host_only = host_only
         self.keep = {}
         if not host_only:

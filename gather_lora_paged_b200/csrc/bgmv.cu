@@ -26,94 +26,18 @@
 // kernels are chained with programmatic dependent launch.
 #include <algorithm>
 
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-
-#include "slora_internal.h"
+#include "dev_common.cuh"
 
 namespace slora {
 
-#define FULL_MASK 0xffffffffu
-
-constexpr long long kWaitLimit = 2000000000ll;  // clock cycles before a wait gives up
-
-__host__ __device__ __forceinline__ int cdiv_i(int a, int b) { return (a + b - 1) / b; }
-
 // Task shapes.  A shrink task covers NT tokens x kRB rank rows x kShrinkKT of
 // d_in; an expand task NTE tokens x kELC outputs (all rank rows).
-__host__ __device__ __forceinline__ int nt_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : (n <= 4 ? 4 : 8)); }
-__host__ __device__ __forceinline__ int nte_class(int n) { return n <= 1 ? 1 : (n == 2 ? 2 : 4); }
 constexpr int kCW = 8;                        // consumer warps per CTA
 constexpr int kProd = 4;                      // producer warps (interleaved ring stages)
 constexpr int kPipeThreads = (kCW + kProd) * 32;
 constexpr int kDescInts = 32;                 // per-stage descriptor (task fields)
 constexpr int kRB = 16;                       // shrink task: rank rows (2 per consumer warp)
 constexpr int kELC = kCW * 256;               // expand task: outputs (256 per consumer warp)
-constexpr int kMaxPieces = 5;                 // pieces of a 2048-element row over >= 512-element pages
-
-__device__ __forceinline__ void record_error(int32_t* err, int code, int info) {
-  if (atomicCAS(&err[0], 0, code) == 0) atomicExch(&err[1], info);
-}
-
-// ---------------------------------------------------------------------------
-// PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-// Bounded wait on an mbarrier phase; false (and a recorded error) if it gives up.
-// try_wait blocks for a system-dependent time; the clock is read only every
-// 64 attempts.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err) {
-  const uint32_t a = smem_u32(bar);
-  long long t0 = -1;
-  for (uint32_t it = 0;; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((it & 63) == 0) {
-      const long long now = clock64();
-      if (t0 < 0) t0 = now;
-      else if (now - t0 > kWaitLimit) {
-        record_error(err, 4, (int)blockIdx.x);
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait until the shared counter *c reaches `target` (a count only ever
-// grows, so unlike an mbarrier phase parity it cannot be misread however far
-// behind the waiter is); false (and a recorded error) if it gives up.
-__device__ __forceinline__ bool counter_wait(const int* c, int target, int32_t* err) {
-  long long t0 = -1;
-  for (uint32_t it = 0;; ++it) {
-    int v;
-    asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(c)) : "memory");
-    if (v >= target) return true;
-    if ((it & 63) == 0) {
-      const long long now = clock64();
-      if (t0 < 0) t0 = now;
-      else if (now - t0 > kWaitLimit) {
-        record_error(err, 4, (int)blockIdx.x);
-        return false;
-      }
-    }
-    __nanosleep(32);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Task schedule of the persistent CTAs.  The first rounds are static: CTA b
@@ -145,15 +69,6 @@ __device__ __forceinline__ void claims_init(TaskClaims& C, int total) {
   C.next = C.m_static;
   for (int i = 0; i < kTix; ++i) C.ord[i] = -1;
 }
-__device__ __forceinline__ int ld_volatile_s32(const int* a) {
-  int v;
-  asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(smem_u32(a)) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_volatile_s32(int* a, int v) {
-  asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
-}
-
 // Task index of CTA-local ordinal n, for every lane of the calling warp (n
 // warp-uniform); -1 if the wait for its publication gave up (error recorded).
 __device__ __forceinline__ int task_of(TaskClaims& C, int n, int* counter, int32_t* err) {
@@ -187,147 +102,6 @@ __device__ __forceinline__ int task_of(TaskClaims& C, int n, int* counter, int32
     }
   }
   return __shfl_sync(FULL_MASK, id, 0);
-}
-
-// Bulk async copy global -> shared, completion counted on `bar`.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-__device__ __forceinline__ uint4 lds128(const unsigned char* p) {
-  return *reinterpret_cast<const uint4*>(p);
-}
-
-// 16-bit -> fp32 for 8 packed elements, exact.  fp16 is widened by the
-// mixed-precision FMA x * 1 + (-0) on the FMA pipe (the conversion unit is the
-// scarce one on this part); bf16 is the upper half of an fp32.
-__device__ __forceinline__ void h2x2f(uint32_t w, float& lo, float& hi) {
-  asm("{.reg .f16 l, h, one;\n\t"
-      "mov.b32 {l, h}, %2;\n\tmov.b16 one, 0x3C00;\n\t"
-      "fma.rn.f32.f16 %0, l, one, 0f80000000;\n\tfma.rn.f32.f16 %1, h, one, 0f80000000;}"
-      : "=f"(lo), "=f"(hi) : "r"(w));
-}
-template <int DT>
-__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (DT == SLORA_BF16) {
-      f[2 * i] = __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    } else {
-      h2x2f(w[i], f[2 * i], f[2 * i + 1]);
-    }
-  }
-}
-
-// acc + a.lo * b.lo + a.hi * b.hi for two packed 16-bit pairs, with the
-// mixed-precision FMA (16-bit sources, fp32 accumulator, one rounding each):
-// the same result as converting exactly and using fp32 FMAs, in order.
-template <int DT>
-__device__ __forceinline__ float fma2_16(uint32_t a, uint32_t b, float acc) {
-  if (DT == SLORA_BF16)
-    asm("{.reg .b16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, al, bl, %0;\n\tfma.rn.f32.bf16 %0, ah, bh, %0;}"
-        : "+f"(acc) : "r"(a), "r"(b));
-  else
-    asm("{.reg .f16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.f16 %0, al, bl, %0;\n\tfma.rn.f32.f16 %0, ah, bh, %0;}"
-        : "+f"(acc) : "r"(a), "r"(b));
-  return acc;
-}
-template <int DT>
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  if (DT == SLORA_BF16) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-  } else {
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
-  }
-}
-
-// Address of flat element f of tensor (adapter a, page-list offset lo).
-__device__ __forceinline__ const uint16_t* page_addr(const PoolDev& P, int a, int lo, int64_t f) {
-  const int32_t pg = __ldg(P.page_list + (int64_t)a * P.list_stride + lo + (f >> P.page_shift));
-  return P.pool + ((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1));
-}
-
-// ---------------------------------------------------------------------------
-// Block-wide exclusive scans (blockDim.x threads, a multiple of 32).
-template <bool kMax>
-__device__ int block_exscan(int v, int* total, int* sh) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int ident = kMax ? -1 : 0;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(FULL_MASK, x, o);
-    if (lane >= o) x = kMax ? max(x, y) : x + y;
-  }
-  int ex = __shfl_up_sync(FULL_MASK, x, 1);
-  if (lane == 0) ex = ident;
-  if (lane == 31) sh[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    int s = lane < nw ? sh[lane] : ident;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(FULL_MASK, s, o);
-      if (lane >= o) s = kMax ? max(s, y) : s + y;
-    }
-    sh[lane] = s;
-  }
-  __syncthreads();
-  const int wp = w ? sh[w - 1] : ident;
-  const int res = kMax ? max(wp, ex) : wp + ex;
-  if (total) *total = sh[nw - 1];
-  __syncthreads();
-  return res;
-}
-
-// Exclusive block-wide prefix sums of four independent values at once; *tot
-// gets the four totals.  sh: 32 int4 of shared memory.
-__device__ int4 block_exscan4(int4 v, int4* tot, int4* sh) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int4 x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y0 = __shfl_up_sync(FULL_MASK, x.x, o), y1 = __shfl_up_sync(FULL_MASK, x.y, o);
-    const int y2 = __shfl_up_sync(FULL_MASK, x.z, o), y3 = __shfl_up_sync(FULL_MASK, x.w, o);
-    if (lane >= o) x = make_int4(x.x + y0, x.y + y1, x.z + y2, x.w + y3);
-  }
-  int4 ex = make_int4(__shfl_up_sync(FULL_MASK, x.x, 1), __shfl_up_sync(FULL_MASK, x.y, 1),
-                      __shfl_up_sync(FULL_MASK, x.z, 1), __shfl_up_sync(FULL_MASK, x.w, 1));
-  if (lane == 0) ex = make_int4(0, 0, 0, 0);
-  if (lane == 31) sh[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    int4 s = lane < nw ? sh[lane] : make_int4(0, 0, 0, 0);
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y0 = __shfl_up_sync(FULL_MASK, s.x, o), y1 = __shfl_up_sync(FULL_MASK, s.y, o);
-      const int y2 = __shfl_up_sync(FULL_MASK, s.z, o), y3 = __shfl_up_sync(FULL_MASK, s.w, o);
-      if (lane >= o) s = make_int4(s.x + y0, s.y + y1, s.z + y2, s.w + y3);
-    }
-    sh[lane] = s;
-  }
-  __syncthreads();
-  const int4 wp = w ? sh[w - 1] : make_int4(0, 0, 0, 0);
-  *tot = sh[nw - 1];
-  __syncthreads();
-  return make_int4(wp.x + ex.x, wp.y + ex.y, wp.z + ex.z, wp.w + ex.w);
 }
 
 // Touch every 64-byte line of a kernel's parameter block once, so that the
@@ -497,40 +271,6 @@ __global__ void __launch_bounds__(1024, 1) k_segments(const __grid_constant__ Bg
   }
 }
 
-// Largest s with prefix[s] <= q (prefix ascending from 0, S >= 1).
-__device__ __forceinline__ int find_seg(const int32_t* prefix, int S, int q) {
-  int lo = 0, hi = S - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= q) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
-// Sum over the 32 lanes of each of the N values v[0..N); afterwards lane L
-// holds the total of value L % N.  N is a power of two <= 32.
-template <int N>
-__device__ __forceinline__ float lane_transpose_reduce(float (&v)[N]) {
-#pragma unroll
-  for (int o = 16; o >= N; o >>= 1) {
-#pragma unroll
-    for (int i = 0; i < N; ++i) v[i] += __shfl_xor_sync(FULL_MASK, v[i], o);
-  }
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = N / 2; o >= 1; o >>= 1) {
-    const bool up = lane & o;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float send = up ? v[i] : v[i + o];
-      const float keep = up ? v[i + o] : v[i];
-      v[i] = keep + __shfl_xor_sync(FULL_MASK, send, o);
-    }
-  }
-  return v[0];
-}
-
 // ---------------------------------------------------------------------------
 // Segment table as seen by the persistent kernels: staged in shared memory
 // when it fits (one round trip per CTA), else read from global memory.
@@ -575,14 +315,6 @@ __device__ SegView stage_segments(const ScratchDev& sc, int S, bool shrink, int3
   return v;
 }
 
-// Page id of flat element f of tensor (adapter a, page-list offset lo).
-__device__ __forceinline__ int32_t page_id(const PoolDev& P, int a, int lo, int64_t f) {
-  return __ldg(P.page_list + (int64_t)a * P.list_stride + lo + (f >> P.page_shift));
-}
-__device__ __forceinline__ const uint16_t* page_ptr(const PoolDev& P, int32_t pg, int64_t f) {
-  return P.pool + ((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1));
-}
-
 // ---------------------------------------------------------------------------
 // Shrink and expand run as warp-specialised persistent CTAs: kProd producer
 // warps take turns along the CTA's (task, stage) sequence and fill a ring of
@@ -594,18 +326,6 @@ __device__ __forceinline__ const uint16_t* page_ptr(const PoolDev& P, int32_t pg
 // engine's cost per request makes 1 KiB copies top out near 60% of HBM
 // bandwidth, and a consumer warp needs a full row slice per stage to keep its
 // fixed per-stage cost small.
-// A paged range [f0, f1) cut at page boundaries: piece q starts at f0 (q = 0)
-// or at the q-th boundary after f0.
-__device__ __forceinline__ bool piece_range(const PoolDev& P, int64_t f0, int64_t f1, int q, int64_t& b,
-                                            int64_t& e) {
-  const int64_t PE = 1ll << P.page_shift;
-  const int64_t pb0 = ((f0 >> P.page_shift) + 1) << P.page_shift;
-  b = q == 0 ? f0 : pb0 + (int64_t)(q - 1) * PE;
-  e = pb0 + (int64_t)q * PE;
-  if (e > f1) e = f1;
-  return b < f1;
-}
-
 // ---------------------------------------------------------------------------
 // Shrink task = (group g, segment, kRB rank rows, NT tokens, kShrinkKT slice
 // of d_in).  The task's x rows (NT x up to kShrinkKT elements) are copied
@@ -619,7 +339,7 @@ constexpr int kSRows = 8;                        // A rows per shrink stage (one
 constexpr int kSNS = 4;                          // shrink ring stages
 constexpr int kSStageBytes = kSRows * 2 * kShrinkKT;
 constexpr int kSRingBytes = kSNS * kSStageBytes;
-constexpr int kXBufBytes = 8 * 2 * kShrinkKT;    // up to 8 tokens x kShrinkKT elements
+constexpr int kXBufBytes = 4 * 2 * kShrinkKT;    // up to 4 tokens x kShrinkKT elements
 static_assert(kPartK == kShrinkKT && kCW == kSRows, "shrink stage mapping");
 static_assert(kSRows * kMaxPieces <= 64, "two lookups per lane");
 static_assert(kSNS % kProd == 0 || kProd % kSNS == 0, "ring slots per producer");
@@ -883,15 +603,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
         switch (t.nt) {
           case 1: shrink_consume<SLORA_BF16, 1>(p, t, st, buf, xb); break;
           case 2: shrink_consume<SLORA_BF16, 2>(p, t, st, buf, xb); break;
-          case 4: shrink_consume<SLORA_BF16, 4>(p, t, st, buf, xb); break;
-          default: shrink_consume<SLORA_BF16, 8>(p, t, st, buf, xb); break;
+          default: shrink_consume<SLORA_BF16, 4>(p, t, st, buf, xb); break;
         }
       } else {
         switch (t.nt) {
           case 1: shrink_consume<SLORA_F16, 1>(p, t, st, buf, xb); break;
           case 2: shrink_consume<SLORA_F16, 2>(p, t, st, buf, xb); break;
-          case 4: shrink_consume<SLORA_F16, 4>(p, t, st, buf, xb); break;
-          default: shrink_consume<SLORA_F16, 8>(p, t, st, buf, xb); break;
+          default: shrink_consume<SLORA_F16, 4>(p, t, st, buf, xb); break;
         }
       }
       __syncwarp();
@@ -1305,6 +1023,13 @@ __global__ void __launch_bounds__(256) k_page_in(PoolDev P, PageInConst C, const
     if (threadIdx.x == 0) {
       P.rank[w.id] = w.rank;
       P.scale[w.id] = w.scale;
+    }
+    if (w.qs_off >= 0) {  // e4m3 row scales into the adapter's table row
+      const float* qs = reinterpret_cast<const float*>(desc + w.qs_off);
+      for (int e = threadIdx.x; e < n_proj * 2 * w.rank; e += blockDim.x) {
+        const int t = e / w.rank, k = e % w.rank;
+        P.qscale[((int64_t)w.id * n_proj * 2 + t) * P.max_rank + k] = qs[e];
+      }
     }
   }
   if (!H->copy_data) return;

@@ -1,21 +1,21 @@
-// noalloc.cu -- slora_lora_delta_noalloc: the fused decode delta with its
-// scratch in a fixed device array that the library owns, so the caller does
-// not have to provide (or allocate) any scratch memory for the call.
+// noalloc.cu -- slora_lora_delta_noalloc: the decode delta with its scratch in
+// a fixed device array that the library owns, so the caller does not have to
+// provide (or allocate) any scratch memory for the call.
 //
-// Who needs this: code that must not allocate device memory at the point where
-// it runs the delta -- for instance a serving loop that is being captured into
-// a CUDA graph (device allocation is not allowed while a stream is captured in
-// the global capture mode), a plug-in whose host framework owns every device
-// allocation and gives it only its inputs and outputs, or a latency-critical
-// path where an allocation could block on the device.  Such a caller still
-// passes the pool, x, y and the index vector; everything else the kernels need
-// comes from the array below.
+// Who needs this: code that cannot allocate device memory at the point where
+// it runs the delta -- for instance a plug-in whose host framework owns every
+// device allocation and hands it only its inputs and outputs, or a
+// latency-critical serving loop that must not risk an allocation blocking on
+// the device.  Such a caller still passes the pool, x, y and the index vector;
+// everything else the kernels need comes from the array below.
 //
 // The array is a file-scope __device__ object: every GPU that loads this
 // library reserves kNoAllocScratchBytes for it until the process exits.  Host
 // code must not pass the symbol itself to a kernel (on the host it is only a
 // stand-in); the device address is looked up with cudaGetSymbolAddress once per
-// device, on the first call made while that device is current.
+// device, on the first call made while that device is current, and kept for the
+// life of the process: resetting a device (cudaDeviceReset) while the library
+// is loaded is not supported.
 #include <mutex>
 #include <nvtx3/nvToolsExt.h>
 #include <string>

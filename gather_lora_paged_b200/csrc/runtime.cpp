@@ -40,6 +40,12 @@ constexpr int kStagingSlots = 4;
 constexpr double kWaitSeconds = 30.0;
 
 int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Size of a rank x dim weight tensor in the pool's 16-bit units: one element
+// each, or (e4m3 weights) two codes each.
+int64_t tensor_units(const slora_pool_desc& d, int64_t rank, int64_t dim) {
+  return d.weight_format == SLORA_WEIGHTS_E4M3 ? rank * dim / 2 : rank * dim;
+}
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // An NVTX range around each C-ABI call that enqueues work or changes the pool,
@@ -68,6 +74,7 @@ struct Adapter {
   int64_t uses[kUseHistory];   // epochs of its most recent page_in namings (a ring)
   int n_uses = 0;              // namings recorded so far
   std::vector<int32_t> pages;  // tensor order (p, A), (p, B)
+  std::vector<float> qs;       // e4m3 weights: row scales [projection][A_t, B][rank]
 };
 
 struct FreePage {
@@ -87,12 +94,17 @@ struct Staging {
 
 // Table layout inside dev_tables.
 struct TableLayout {
-  size_t off_rank, off_scale, off_err, off_list, off_desc, desc_cap, total;
+  size_t off_rank, off_scale, off_err, off_list, off_qscale, off_desc, desc_cap, total;
 };
+
+// Row scales of e4m3 weights, per adapter: [projection][A_t, B][max_rank] floats.
+size_t qscale_floats(const slora_pool_desc& d) {
+  return d.weight_format == SLORA_WEIGHTS_E4M3 ? (size_t)d.n_proj * 2 * (size_t)d.max_rank : 0;
+}
 
 // Scratch layout inside dev_scratch.
 struct ScratchLayout {
-  size_t off_meta, off_perm, off_seg_start, off_seg_adapter, off_seg_rank, off_shrink_pre,
+  size_t off_ready, off_meta, off_perm, off_seg_start, off_seg_adapter, off_seg_rank, off_shrink_pre,
       off_expand_pre, off_tpart, off_sgmv, total;
   int64_t tpart_floats, rk8;
   int MS;
@@ -102,9 +114,9 @@ int64_t list_stride_of(const slora_pool_desc& d, int* listA, int* listB) {
   int64_t off = 0;
   for (int p = 0; p < d.n_proj; ++p) {
     listA[p] = (int)off;
-    off += cdiv64((int64_t)d.max_rank * d.d_in[p], d.page_elems);
+    off += cdiv64(tensor_units(d, d.max_rank, d.d_in[p]), d.page_elems);
     listB[p] = (int)off;
-    off += cdiv64((int64_t)d.max_rank * d.d_out[p], d.page_elems);
+    off += cdiv64(tensor_units(d, d.max_rank, d.d_out[p]), d.page_elems);
   }
   for (int p = d.n_proj; p < kMaxSlots; ++p) listA[p] = listB[p] = 0;
   return off > 0 ? off : 1;
@@ -123,9 +135,12 @@ TableLayout table_layout(const slora_pool_desc& d) {
   o = align_up(o + 16, 256);
   L.off_list = o;
   o = align_up(o + 4 * (size_t)d.max_adapters * stride, 256);
+  L.off_qscale = o;
+  o = align_up(o + 4 * (size_t)d.max_adapters * qscale_floats(d), 256);
   L.off_desc = o;
   L.desc_cap = align_up(sizeof(PageInHeader) + 4 * (size_t)d.max_adapters +
-                            (sizeof(PageInNew) + 4 * (size_t)stride + 16) * (size_t)d.max_adapters,
+                            (sizeof(PageInNew) + 4 * (size_t)stride + 4 * qscale_floats(d) + 32) *
+                                (size_t)d.max_adapters,
                         256);
   o += L.desc_cap;
   L.total = o;
@@ -142,6 +157,8 @@ ScratchLayout scratch_layout(const slora_pool_desc& d) {
   L.rk8 = std::max<int64_t>(8, (d.max_rank + 7) / 8 * 8);
   L.tpart_floats = sum_ns * T * L.rk8;
   size_t o = 0;
+  L.off_ready = o;  // first in every layout: zero between calls (see kFReadyCap)
+  o = align_up(o + kFReadyBytes, 256);
   L.off_meta = o;
   o = align_up(o + 4 * kMetaCount, 256);
   L.off_perm = o;
@@ -218,15 +235,18 @@ struct slora_pool {
   }
   slora_status_t cuda_fail(cudaError_t e, const char* where) {
     err = std::string("CUDA error in ") + where + ": " + cudaGetErrorString(e);
+    if (getenv("SLORA_LOG")) fprintf(stderr, "slora: %s\n", err.c_str());
+    cudaGetLastError();  // a non-sticky error must not resurface at the next launch check
     return SLORA_ERR_CUDA;
   }
   int64_t pages_for(int rank) const {
     int64_t n = 0;
     for (int p = 0; p < d.n_proj; ++p)
-      n += cdiv64((int64_t)rank * d.d_in[p], d.page_elems) +
-           cdiv64((int64_t)rank * d.d_out[p], d.page_elems);
+      n += cdiv64(tensor_units(d, rank, d.d_in[p]), d.page_elems) +
+           cdiv64(tensor_units(d, rank, d.d_out[p]), d.page_elems);
     return n;
   }
+  bool e4m3() const { return d.weight_format == SLORA_WEIGHTS_E4M3; }
   char* tables() const { return static_cast<char*>(d.dev_tables); }
   char* scratch() const { return static_cast<char*>(d.dev_scratch); }
 };
@@ -260,6 +280,8 @@ slora_status_t validate_desc(const slora_pool_desc* d, std::string* why) {
   if (d->n_pages < 0 || d->n_pages > (int64_t)INT32_MAX) return bad("n_pages out of range");
   if (d->pagein_mode != SLORA_PAGEIN_KERNEL && d->pagein_mode != SLORA_PAGEIN_MEMCPY)
     return bad("pagein_mode");
+  if (d->decode_path < SLORA_DECODE_AUTO || d->decode_path > SLORA_DECODE_FUSED) return bad("decode_path");
+  if (d->weight_format != SLORA_WEIGHTS_16 && d->weight_format != SLORA_WEIGHTS_E4M3) return bad("weight_format");
   if (!d->host_only) {
     if (!d->dev_pool && d->n_pages > 0) return bad("dev_pool is NULL");
     if (!d->dev_tables || !d->dev_scratch) return bad("dev_tables/dev_scratch is NULL");
@@ -271,10 +293,11 @@ slora_status_t validate_desc(const slora_pool_desc* d, std::string* why) {
 }
 
 // Device-side wait (no host block) for the compute of `epoch` to finish.
-void wait_epoch(slora_pool* P, cudaStream_t s, int64_t epoch) {
-  if (epoch < 0) return;
+cudaError_t wait_epoch(slora_pool* P, cudaStream_t s, int64_t epoch) {
+  if (epoch < 0) return cudaSuccess;
   const int slot = (int)(epoch % kEventRing);
-  if (P->ev_epoch[slot] >= epoch) cudaStreamWaitEvent(s, P->ev[slot], 0);
+  if (P->ev_epoch[slot] >= epoch) return cudaStreamWaitEvent(s, P->ev[slot], 0);
+  return cudaSuccess;
 }
 
 // Timing hook: with 2 events only the call's start and end are recorded (the
@@ -288,10 +311,11 @@ void phase(slora_pool* P, int k, int last, cudaStream_t s) {
   }
 }
 
-void record_epoch(slora_pool* P, cudaStream_t s) {
+cudaError_t record_epoch(slora_pool* P, cudaStream_t s) {
   const int slot = (int)(P->epoch % kEventRing);
-  cudaEventRecord(P->ev[slot], s);
-  P->ev_epoch[slot] = P->epoch;
+  const cudaError_t e = cudaEventRecord(P->ev[slot], s);
+  if (e == cudaSuccess) P->ev_epoch[slot] = P->epoch;
+  return e;
 }
 
 // Bounded host wait on an event.
@@ -319,6 +343,9 @@ void fill_pool_dev(slora_pool* P) {
   P->pd.scale = reinterpret_cast<float*>(P->tables() + P->tl.off_scale);
   P->pd.page_list = reinterpret_cast<int32_t*>(P->tables() + P->tl.off_list);
   P->pd.err = reinterpret_cast<int32_t*>(P->tables() + P->tl.off_err);
+  P->pd.qscale = P->e4m3() ? reinterpret_cast<float*>(P->tables() + P->tl.off_qscale) : nullptr;
+  P->pd.wfmt = P->d.weight_format;
+  P->pd.n_proj = P->d.n_proj;
 }
 
 ScratchDev scratch_at(char* b, const ScratchLayout& L) {
@@ -328,6 +355,7 @@ ScratchDev scratch_at(char* b, const ScratchLayout& L) {
   s.seg_start = reinterpret_cast<int32_t*>(b + L.off_seg_start);
   s.seg_adapter = reinterpret_cast<int32_t*>(b + L.off_seg_adapter);
   s.seg_rank = reinterpret_cast<int32_t*>(b + L.off_seg_rank);
+  s.ready = reinterpret_cast<int32_t*>(b + L.off_ready);
   s.shrink_prefix = reinterpret_cast<int32_t*>(b + L.off_shrink_pre);
   s.expand_prefix = reinterpret_cast<int32_t*>(b + L.off_expand_pre);
   s.MS = L.MS;
@@ -373,6 +401,7 @@ slora_status_t plan_slots(slora_pool* P, BgmvParams& bp, int n, const int32_t* p
     S.d_out = P->d.d_out[p];
     S.listA = P->listA[p];
     S.listB = P->listB[p];
+    S.proj = p;
     S.nsplit = (int)cdiv64(S.d_in, kPartK);
     if (need_x) {
       if (!x || !ldx || !x[k]) return P->fail(SLORA_ERR_INVALID_ARG, "x is NULL");
@@ -423,6 +452,39 @@ slora_status_t need_device(slora_pool* P) {
   return SLORA_OK;
 }
 
+// Whether a decode call of T tokens runs as the one persistent kernel.
+bool fused_path(const slora_pool* P, int T) {
+  if (T > kFMaxT) return false;
+  if (P->d.decode_path == SLORA_DECODE_FUSED) return true;
+  return P->d.decode_path == SLORA_DECODE_AUTO && P->d.weight_format == SLORA_WEIGHTS_E4M3;
+}
+
+// The decode delta's kernels for a planned call (both phases): the one
+// persistent kernel or the three-kernel path (fused_path); timing events
+// (slora_set_phase_events) bracket each kernel when `timed`.
+slora_status_t enqueue_delta(slora_pool* P, BgmvParams& bp, const int32_t* idx, int T, cudaStream_t st,
+                             bool timed) {
+  bp.do_shrink = 1;
+  bp.do_expand = 1;
+  if (P->e4m3() && !fused_path(P, T))
+    return P->fail(SLORA_ERR_UNSUPPORTED, "e4m3 weights: decode calls of up to 1024 tokens on the one-kernel path");
+  if (fused_path(P, T)) {
+    const int grid = std::max(1, std::min(P->sm_count, fused_grid_bound(bp, T)));
+    if (timed) phase(P, 0, 1, st);
+    CUDA_TRY(P, launch_fused(bp, P->d.dtype, idx, T, grid, st));
+    if (timed) phase(P, 1, 1, st);
+    return SLORA_OK;
+  }
+  if (timed) phase(P, 0, 3, st);
+  CUDA_TRY(P, launch_segments(bp, idx, T, st));
+  if (timed) phase(P, 1, 3, st);
+  CUDA_TRY(P, launch_shrink(bp, P->d.dtype, P->grid_shrink, st));
+  if (timed) phase(P, 2, 3, st);
+  CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
+  if (timed) phase(P, 3, 3, st);
+  return SLORA_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -447,7 +509,11 @@ slora_status_t lora_delta_on_scratch(slora_pool* P, int32_t n, const int32_t* pr
   slora_pool_desc dd = P->d;
   dd.max_tokens = T;
   const ScratchLayout L = scratch_layout(dd);
-  const size_t need = L.off_sgmv;  // the decode part of the layout
+  // the decode part of the layout: tables, then the fp32 partials of the
+  // projections this call names (not of every projection of the pool)
+  int64_t part_floats = 0;
+  for (int k = 0; k < bp.n_slots; ++k) part_floats += (int64_t)bp.slot[k].nsplit * T * L.rk8;
+  const size_t need = L.off_tpart + 4 * (size_t)part_floats;
   if (need > scratch_cap)
     return P->fail(SLORA_ERR_INVALID_ARG,
                    "this call needs " + std::to_string(need) + " bytes of scratch; the static "
@@ -456,14 +522,11 @@ slora_status_t lora_delta_on_scratch(slora_pool* P, int32_t n, const int32_t* pr
   char* b = static_cast<char*>(scratch);
   bp.max_tokens = T;
   bp.sc = scratch_at(b, L);
-  if (!assign_partials(bp, reinterpret_cast<float*>(b + L.off_tpart), L.tpart_floats, T, L.rk8))
+  if (!assign_partials(bp, reinterpret_cast<float*>(b + L.off_tpart), part_floats, T, L.rk8))
     return P->fail(SLORA_ERR_INVALID_ARG, "too many projections in one call");
-  bp.do_shrink = 1;
-  bp.do_expand = 1;
-  CUDA_TRY(P, launch_segments(bp, idx, T, st));
-  CUDA_TRY(P, launch_shrink(bp, P->d.dtype, P->grid_shrink, st));
-  CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
-  record_epoch(P, st);
+  s = enqueue_delta(P, bp, idx, T, st, false);
+  if (s) return s;
+  CUDA_TRY(P, record_epoch(P, st));
   return SLORA_OK;
 }
 }  // namespace slora
@@ -487,7 +550,8 @@ int64_t slora_pages_for_rank(const slora_pool_desc* d, int32_t rank) {
   if (!d || rank < 0 || d->page_elems < 1) return -1;
   int64_t n = 0;
   for (int p = 0; p < d->n_proj && p < SLORA_MAX_PROJ; ++p)
-    n += cdiv64((int64_t)rank * d->d_in[p], d->page_elems) + cdiv64((int64_t)rank * d->d_out[p], d->page_elems);
+    n += cdiv64(tensor_units(*d, rank, d->d_in[p]), d->page_elems) +
+         cdiv64(tensor_units(*d, rank, d->d_out[p]), d->page_elems);
   return n;
 }
 
@@ -584,24 +648,36 @@ slora_status_t slora_pool_set_page_order(slora_pool* P, const int32_t* order, in
   return SLORA_OK;
 }
 
-slora_status_t slora_adapter_register(slora_pool* P, int32_t id, int32_t rank, float alpha,
-                                      const void* const* host_A_t, const void* const* host_B) {
-  NvtxRange nvtx_("slora_adapter_register");
-  if (!P) return SLORA_ERR_INVALID_ARG;
+static slora_status_t register_impl(slora_pool* P, int32_t id, int32_t rank, float alpha,
+                                    const void* const* host_A_t, const void* const* host_B,
+                                    const float* const* scales_A_t, const float* const* scales_B) {
   if (id < 0 || id >= P->d.max_adapters) return P->fail(SLORA_ERR_INVALID_ARG, "adapter id out of range");
   if (rank < 0 || rank > P->d.max_rank) return P->fail(SLORA_ERR_INVALID_ARG, "rank out of [0, max_rank]");
   Adapter& A = P->ad[id];
   if (A.resident) return P->fail(SLORA_ERR_INVALID_ARG, "adapter is resident; evict it first");
   if (rank > 0 && (!host_A_t || !host_B)) return P->fail(SLORA_ERR_INVALID_ARG, "weight pointers are NULL");
+  const bool q8 = P->e4m3();
+  if (q8 && rank > 0 && (!scales_A_t || !scales_B)) return P->fail(SLORA_ERR_INVALID_ARG, "scale pointers are NULL");
   Adapter N;
   N.registered = true;
   N.rank = rank;
   N.alpha = alpha;
   N.last_use = A.last_use;
+  if (q8) N.qs.assign((size_t)P->d.n_proj * 2 * rank, 0.f);
   for (int p = 0; p < P->d.n_proj && rank > 0; ++p) {
     if (!host_A_t[p] || !host_B[p]) return P->fail(SLORA_ERR_INVALID_ARG, "weight pointer is NULL");
     if (!aligned16(host_A_t[p]) || !aligned16(host_B[p]))
       return P->fail(SLORA_ERR_INVALID_ARG, "weights must be 16-byte aligned");
+    if (q8) {
+      if (!scales_A_t[p] || !scales_B[p]) return P->fail(SLORA_ERR_INVALID_ARG, "scale pointer is NULL");
+      for (int k = 0; k < rank; ++k) {
+        const float a = scales_A_t[p][k], b = scales_B[p][k];
+        if (!(a >= 0.f) || !(b >= 0.f) || !std::isfinite(a) || !std::isfinite(b))
+          return P->fail(SLORA_ERR_INVALID_ARG, "scales must be finite and non-negative");
+        N.qs[((size_t)p * 2 + 0) * rank + k] = a;
+        N.qs[((size_t)p * 2 + 1) * rank + k] = b;
+      }
+    }
     N.host_A[p] = host_A_t[p];
     N.host_B[p] = host_B[p];
     N.map_A[p] = host_A_t[p];
@@ -627,6 +703,23 @@ slora_status_t slora_adapter_register(slora_pool* P, int32_t id, int32_t rank, f
   }
   A = N;
   return SLORA_OK;
+}
+
+slora_status_t slora_adapter_register(slora_pool* P, int32_t id, int32_t rank, float alpha,
+                                      const void* const* host_A_t, const void* const* host_B) {
+  NvtxRange nvtx_("slora_adapter_register");
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  if (P->e4m3()) return P->fail(SLORA_ERR_INVALID_ARG, "the pool holds e4m3 weights: use slora_adapter_register_e4m3");
+  return register_impl(P, id, rank, alpha, host_A_t, host_B, nullptr, nullptr);
+}
+
+slora_status_t slora_adapter_register_e4m3(slora_pool* P, int32_t id, int32_t rank, float alpha,
+                                           const void* const* codes_A_t, const float* const* scales_A_t,
+                                           const void* const* codes_B, const float* const* scales_B) {
+  NvtxRange nvtx_("slora_adapter_register_e4m3");
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  if (!P->e4m3()) return P->fail(SLORA_ERR_INVALID_ARG, "the pool holds 16-bit weights: use slora_adapter_register");
+  return register_impl(P, id, rank, alpha, codes_A_t, codes_B, scales_A_t, scales_B);
 }
 
 static void evict_one(slora_pool* P, int id) {
@@ -733,8 +826,10 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     }
     A.resident = true;
     if (!prefetch) P->st.page_ins++;
-    (prefetch ? P->st.bytes_prefetched : P->st.bytes_paged_in) += 2 * (int64_t)A.rank *
-        [&] { int64_t s = 0; for (int p = 0; p < P->d.n_proj; ++p) s += P->d.d_in[p] + P->d.d_out[p]; return s; }();
+    (prefetch ? P->st.bytes_prefetched : P->st.bytes_paged_in) +=
+        [&] { int64_t s = 0; for (int p = 0; p < P->d.n_proj; ++p)
+                s += 2 * (tensor_units(P->d, A.rank, P->d.d_in[p]) + tensor_units(P->d, A.rank, P->d.d_out[p]));
+              return s; }();
   }
   if (!prefetch) {
     P->st.hits += (int64_t)(uniq.size() - missing.size());
@@ -771,7 +866,9 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     size_t off_evict = align_up(sizeof(PageInHeader), 16);
     size_t off_new = align_up(off_evict + 4 * victims.size(), 16);
     size_t off_lists = align_up(off_new + sizeof(PageInNew) * missing.size(), 16);
-    size_t bytes = off_lists + 4 * (size_t)stride * missing.size();
+    size_t off_qs = align_up(off_lists + 4 * (size_t)stride * missing.size(), 16);
+    size_t bytes = off_qs;
+    for (int a : missing) bytes += 4 * P->ad[a].qs.size();
     if (!stg) {
       stg = &P->stg[P->next_stg];
       if (stg->pending) {
@@ -802,6 +899,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     for (size_t i = 0; i < victims.size(); ++i) ev[i] = victims[i];
     PageInNew* nw = reinterpret_cast<PageInNew*>(h + off_new);
     int64_t units = 0;
+    size_t qs_at = off_qs;
     for (size_t i = 0; i < missing.size(); ++i) {
       const Adapter& A = P->ad[missing[i]];
       PageInNew& w = nw[i];
@@ -813,6 +911,11 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
       w.unit_base = units;
       units += (int64_t)A.pages.size();
       w.list_off = (int64_t)(off_lists + 4 * (size_t)stride * i);
+      w.qs_off = A.qs.empty() ? -1 : (int64_t)qs_at;
+      if (!A.qs.empty()) {
+        memcpy(h + qs_at, A.qs.data(), 4 * A.qs.size());
+        qs_at += 4 * A.qs.size();
+      }
       for (int p = 0; p < P->d.n_proj; ++p) {
         w.host[p][0] = static_cast<const uint16_t*>(A.map_A[p]);
         w.host[p][1] = static_cast<const uint16_t*>(A.map_B[p]);
@@ -821,9 +924,9 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
       for (int64_t e = 0; e < stride; ++e) row[e] = -1;
       int64_t c = 0;
       for (int p = 0; p < P->d.n_proj; ++p) {
-        const int64_t na = cdiv64((int64_t)A.rank * P->d.d_in[p], P->d.page_elems);
+        const int64_t na = cdiv64(tensor_units(P->d, A.rank, P->d.d_in[p]), P->d.page_elems);
         for (int64_t j = 0; j < na; ++j) row[P->listA[p] + j] = A.pages[c++];
-        const int64_t nb = cdiv64((int64_t)A.rank * P->d.d_out[p], P->d.page_elems);
+        const int64_t nb = cdiv64(tensor_units(P->d, A.rank, P->d.d_out[p]), P->d.page_elems);
         for (int64_t j = 0; j < nb; ++j) row[P->listB[p] + j] = A.pages[c++];
       }
     }
@@ -831,7 +934,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     // device-side ordering: previous page-in done (descriptor area), and the
     // compute that last read the pages being reused
     if (P->pagein_pending) CUDA_TRY(P, cudaStreamWaitEvent(side, P->pagein_done, 0));
-    wait_epoch(P, side, wait_ep);
+    CUDA_TRY(P, wait_epoch(P, side, wait_ep));
     for (int r : rel_wait) CUDA_TRY(P, cudaStreamWaitEvent(side, P->rel_ev[r], 0));
     char* desc_dev = P->tables() + P->tl.off_desc;
     CUDA_TRY(P, cudaMemcpyAsync(desc_dev, h, bytes, cudaMemcpyHostToDevice, side));
@@ -840,7 +943,12 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
     P->next_stg = (P->next_stg + 1) % kStagingSlots;
     int grid = (int)std::min<int64_t>(std::max<int64_t>(units, 1), 2 * (int64_t)P->sm_count);
     if (missing.size() > (size_t)grid) grid = (int)std::min<size_t>(missing.size(), 4096);
-    CUDA_TRY(P, launch_page_in(P->pd, P->d.d_in, P->d.d_out, P->listA, P->listB, desc_dev, units, grid, side));
+    int u_in[kMaxSlots], u_out[kMaxSlots];  // tensor widths in 16-bit units
+    for (int q = 0; q < kMaxSlots; ++q) {
+      u_in[q] = P->e4m3() ? P->d.d_in[q] / 2 : P->d.d_in[q];
+      u_out[q] = P->e4m3() ? P->d.d_out[q] / 2 : P->d.d_out[q];
+    }
+    CUDA_TRY(P, launch_page_in(P->pd, u_in, u_out, P->listA, P->listB, desc_dev, units, grid, side));
     P->st.copy_calls++;
     if (P->d.pagein_mode == SLORA_PAGEIN_MEMCPY) {
       const int64_t Pb = P->d.page_elems * 2;
@@ -849,7 +957,7 @@ static slora_status_t page_in_impl(slora_pool* P, const int32_t* ids, int32_t n,
         int64_t c = 0;
         for (int t = 0; t < 2 * P->d.n_proj; ++t) {
           const int p = t >> 1;
-          const int64_t nel = (int64_t)A.rank * ((t & 1) ? P->d.d_out[p] : P->d.d_in[p]);
+          const int64_t nel = tensor_units(P->d, A.rank, (t & 1) ? P->d.d_out[p] : P->d.d_in[p]);
           const int64_t np = cdiv64(nel, P->d.page_elems);
           const char* src = static_cast<const char*>((t & 1) ? A.host_B[p] : A.host_A[p]);
           int64_t j = 0;
@@ -954,7 +1062,7 @@ slora_status_t slora_kv_alloc(slora_pool* P, int64_t n, int32_t* ids_out, void* 
     CUDA_TRY(P, cudaEventRecord(P->pagein_done, st));
     P->pagein_pending = true;
   }
-  wait_epoch(P, st, wait_ep);
+  CUDA_TRY(P, wait_epoch(P, st, wait_ep));
   for (int r : rel_wait) CUDA_TRY(P, cudaStreamWaitEvent(st, P->rel_ev[r], 0));
   if (done_event) CUDA_TRY(P, cudaEventRecord(static_cast<cudaEvent_t>(done_event), st));
   return SLORA_OK;
@@ -1010,6 +1118,11 @@ slora_status_t slora_adapter_is_resident(const slora_pool* P, int32_t id, int32_
   if (!P || !out || id < 0 || id >= P->d.max_adapters) return SLORA_ERR_INVALID_ARG;
   *out = P->ad[id].resident ? 1 : 0;
   return SLORA_OK;
+}
+
+int32_t slora_decode_kernels(const slora_pool* P, int32_t T) {
+  if (!P || T <= 0) return 0;
+  return fused_path(P, T) ? 1 : 3;
 }
 
 slora_status_t slora_check_batch(const slora_pool* Pc, const int32_t* idx_host, int32_t T) {
@@ -1075,17 +1188,10 @@ slora_status_t slora_lora_delta(slora_pool* P, int32_t n, const int32_t* projs, 
   s = plan_slots(P, bp, n, projs, x, ldx, y, ldy, T, true, true);
   if (s) return s;
   if (T == 0) return SLORA_OK;
-  bp.do_shrink = 1;
-  bp.do_expand = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  phase(P, 0, 3, st);
-  CUDA_TRY(P, launch_segments(bp, idx, T, st));
-  phase(P, 1, 3, st);
-  CUDA_TRY(P, launch_shrink(bp, P->d.dtype, P->grid_shrink, st));
-  phase(P, 2, 3, st);
-  CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
-  phase(P, 3, 3, st);
-  record_epoch(P, st);
+  s = enqueue_delta(P, bp, idx, T, st, true);
+  if (s) return s;
+  CUDA_TRY(P, record_epoch(P, st));
   return SLORA_OK;
 }
 
@@ -1095,6 +1201,7 @@ slora_status_t slora_bgmv_shrink(slora_pool* P, int32_t proj, const void* x, int
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
+  if (P->e4m3()) return P->fail(SLORA_ERR_UNSUPPORTED, "slora_bgmv_shrink takes 16-bit weights only");
   if (T > 0 && (!idx || !t)) return P->fail(SLORA_ERR_INVALID_ARG, "idx / t is NULL");
   if (ldt < P->d.max_rank || ((uintptr_t)t & 15) || ldt % 8)
     return P->fail(SLORA_ERR_INVALID_ARG, "t: ldt >= max_rank, ldt % 8 == 0, 16-byte aligned");
@@ -1118,7 +1225,7 @@ slora_status_t slora_bgmv_shrink(slora_pool* P, int32_t proj, const void* x, int
   phase(P, 2, 3, st);
   CUDA_TRY(P, launch_reduce_t(bp, T, st));
   phase(P, 3, 3, st);
-  record_epoch(P, st);
+  CUDA_TRY(P, record_epoch(P, st));
   return SLORA_OK;
 }
 
@@ -1128,6 +1235,7 @@ slora_status_t slora_bgmv_expand(slora_pool* P, int32_t proj, const float* t, in
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
+  if (P->e4m3()) return P->fail(SLORA_ERR_UNSUPPORTED, "slora_bgmv_expand takes 16-bit weights only");
   if (T > 0 && (!idx || !t)) return P->fail(SLORA_ERR_INVALID_ARG, "idx / t is NULL");
   if (ldt < P->d.max_rank || ((uintptr_t)t & 15) || ldt % 8)
     return P->fail(SLORA_ERR_INVALID_ARG, "t: ldt >= max_rank, ldt % 8 == 0, 16-byte aligned");
@@ -1150,7 +1258,7 @@ slora_status_t slora_bgmv_expand(slora_pool* P, int32_t proj, const float* t, in
   phase(P, 1, 2, st);
   CUDA_TRY(P, launch_expand(bp, P->d.dtype, P->grid_expand, st));
   phase(P, 2, 2, st);
-  record_epoch(P, st);
+  CUDA_TRY(P, record_epoch(P, st));
   return SLORA_OK;
 }
 
@@ -1161,6 +1269,7 @@ slora_status_t slora_sgmv(slora_pool* P, int32_t n, const int32_t* projs, const 
   if (!P) return SLORA_ERR_INVALID_ARG;
   slora_status_t s = need_device(P);
   if (s) return s;
+  if (P->e4m3()) return P->fail(SLORA_ERR_UNSUPPORTED, "slora_sgmv takes 16-bit weights only");
   if (S < 0 || (S > 0 && (!seg_start || !seg_adapter))) return P->fail(SLORA_ERR_INVALID_ARG, "segments");
   BgmvParams bp;
   base_params(P, bp);
@@ -1174,7 +1283,7 @@ slora_status_t slora_sgmv(slora_pool* P, int32_t n, const int32_t* projs, const 
                               P->n_phase);
   if (e == cudaErrorNotSupported) return P->fail(SLORA_ERR_UNSUPPORTED, "SGMV shape not supported");
   if (e != cudaSuccess) return P->cuda_fail(e, "SGMV launch");
-  record_epoch(P, st);
+  CUDA_TRY(P, record_epoch(P, st));
   return SLORA_OK;
 }
 
@@ -1187,13 +1296,15 @@ slora_status_t slora_debug_gather(slora_pool* P, int32_t id, int32_t proj, void*
   if (!P->ad[id].resident) return P->fail(SLORA_ERR_NOT_RESIDENT, "adapter " + std::to_string(id));
   const int r = P->ad[id].rank;
   if (r == 0) return SLORA_OK;
-  // Debug path: uses its own temporary device buffer.
-  const size_t na = (size_t)r * P->d.d_in[proj] * 2, nb = (size_t)r * P->d.d_out[proj] * 2;
+  // Debug path: uses its own temporary device buffer.  Widths in 16-bit units.
+  const int w_in = P->e4m3() ? P->d.d_in[proj] / 2 : P->d.d_in[proj];
+  const int w_out = P->e4m3() ? P->d.d_out[proj] / 2 : P->d.d_out[proj];
+  const size_t na = (size_t)r * w_in * 2, nb = (size_t)r * w_out * 2;
   void* buf = nullptr;
   CUDA_TRY(P, cudaMalloc(&buf, na + nb));
-  cudaError_t e = launch_gather_debug(P->pd, id, P->d.d_in[proj], P->listA[proj], r, static_cast<uint16_t*>(buf), 0);
+  cudaError_t e = launch_gather_debug(P->pd, id, w_in, P->listA[proj], r, static_cast<uint16_t*>(buf), 0);
   if (e == cudaSuccess)
-    e = launch_gather_debug(P->pd, id, P->d.d_out[proj], P->listB[proj], r,
+    e = launch_gather_debug(P->pd, id, w_out, P->listB[proj], r,
                             reinterpret_cast<uint16_t*>(static_cast<char*>(buf) + na), 0);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e == cudaSuccess && host_A_t) e = cudaMemcpy(host_A_t, buf, na, cudaMemcpyDeviceToHost);

@@ -18,6 +18,17 @@ constexpr int kMaxSlots = SLORA_MAX_PROJ;   // projections per call
 constexpr int kThreads = 256;               // threads per CTA of the decode kernels
 constexpr int kEventRing = 64;
 
+// One-kernel decode path (fused.cu): every CTA keeps the batch's token order
+// and segment table in shared memory, which bounds the tokens per call; larger
+// calls take the three-kernel path (bgmv.cu).
+constexpr int kFMaxT = 1024;                // tokens per call
+constexpr int kFSegCap = kFMaxT;            // segments per call (<= tokens)
+// Ready counters of the fused path, one per (segment, x group), then a count
+// of finished CTAs; all zero between calls (the last CTA of a call clears
+// them).  They sit at the start of every scratch layout.
+constexpr int kFReadyCap = kFSegCap * kMaxSlots;
+constexpr size_t kFReadyBytes = 4 * (kFReadyCap + 64);
+
 // Device view of the pool and its tables.
 struct PoolDev {
   uint16_t* pool;          // page storage
@@ -29,6 +40,9 @@ struct PoolDev {
   float* scale;            // [max_adapters], alpha / rank
   int32_t* page_list;      // [max_adapters * list_stride]
   int32_t* err;            // [2]: first error code, its token
+  float* qscale;           // e4m3 weights: [max_adapters][n_proj][A_t, B][max_rank] row scales
+  int wfmt;                // slora_weight_format_t
+  int n_proj;              // projections per adapter
 };
 
 // One projection entry of a compute call.
@@ -39,6 +53,7 @@ struct SlotDev {
   int64_t ldy;
   int d_in, d_out;
   int listA, listB;        // offsets of this projection's A_t / B page lists in an adapter row
+  int proj;                // the pool's projection index
   int nsplit;              // shrink partials = ceil(d_in / kPartK)
   int group;               // index of the x-sharing group
   int gpos;                // rank-row block of this slot inside its group
@@ -70,6 +85,7 @@ struct ScratchDev {
   int32_t* shrink_prefix;  // [MS + 1] shrink tasks before each segment (segment-major)
   int32_t* expand_prefix;  // [MS + 1] expand tasks before each segment
   int32_t* seg_rank;       // [MS] rank of each segment's adapter
+  int32_t* ready;          // [kFReadyCap + 1] fused path: ready counters, then finished CTAs
   int MS;                  // max segments = min(max_tokens, max_adapters)
 };
 
@@ -109,6 +125,7 @@ struct PageInNew {
   int32_t n_units;         // pages of this adapter
   int64_t unit_base;       // prefix of units over previous adapters
   int64_t list_off;        // byte offset of its page-list row in the descriptor
+  int64_t qs_off;          // byte offset of its e4m3 row scales ([proj][A_t, B][rank]), -1: none
   const uint16_t* host[kMaxSlots][2];   // device-usable pointers to pinned host weights
 };
 
@@ -118,6 +135,9 @@ cudaError_t launch_segments(BgmvParams& p, const int32_t* idx, int T, cudaStream
 cudaError_t launch_shrink(const BgmvParams& p, int dtype, int grid, cudaStream_t s);
 cudaError_t launch_expand(const BgmvParams& p, int dtype, int grid, cudaStream_t s);
 cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s);
+// The one-kernel decode delta (fused.cu): T <= kFMaxT, both phases.
+cudaError_t launch_fused(BgmvParams& p, int dtype, const int32_t* idx, int T, int grid, cudaStream_t s);
+int fused_grid_bound(const BgmvParams& p, int T);  // CTAs worth launching for T tokens
 cudaError_t launch_merge_requests(const int32_t* req_start, const int32_t* req_adapter, int n,
                                   int32_t* seg_start, int32_t* seg_adapter, int32_t* S_out,
                                   cudaStream_t s);

@@ -33,6 +33,11 @@ def pinned(bits: np.ndarray):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).pin_memory()
 
 
+def pinned_bytes(codes: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).pin_memory()
+
+
 class PoolBuild:
     """A pool holding a workload's adapters.
 
@@ -40,18 +45,22 @@ class PoolBuild:
     n_pages: pool size (default: exactly the pages of all adapters)."""
 
     def __init__(self, w: W.Workload, resident=None, n_pages=None, max_tokens=None,
-                 pagein_mode=G.SLORA_PAGEIN_KERNEL, threads=8, chunk=256):
+                 pagein_mode=G.SLORA_PAGEIN_KERNEL, threads=8, chunk=256,
+                 decode_path=G.SLORA_DECODE_AUTO, weight_format=G.SLORA_WEIGHTS_16):
         import torch
         self.w = w
+        self.q8 = weight_format == G.SLORA_WEIGHTS_E4M3
         d_in = [p.d_in for p in w.projs]
         d_out = [p.d_out for p in w.projs]
         max_rank = int(w.ranks.max())
-        desc = G.make_desc(w.dtype, d_in, d_out, w.n_adapters, max_rank, 1, w.page_elems, 0)
+        desc = G.make_desc(w.dtype, d_in, d_out, w.n_adapters, max_rank, 1, w.page_elems, 0,
+                           weight_format=weight_format)
         self.need = np.array([G.slora_pages_for_rank(desc, int(r)) for r in w.ranks], np.int64)
         if n_pages is None:
             n_pages = int(self.need.sum())
         self.pool = G.Pool(w.dtype, d_in, d_out, w.n_adapters, max_rank,
-                           max_tokens or max(w.T, 1), w.page_elems, n_pages, pagein_mode)
+                           max_tokens or max(w.T, 1), w.page_elems, n_pages, pagein_mode,
+                           decode_path=decode_path, weight_format=weight_format)
         if w.shuffle_pages:
             G.slora_pool_set_page_order(self.pool.h, W.page_order(n_pages, w.seed))
         # host weights: own data for touched adapters, one pinned filler per rank
@@ -59,18 +68,29 @@ class PoolBuild:
         w.prefetch_adapters(sorted(touched), threads)
         self.host = {}
         fill = {}
+        self.q8w = {}  # e4m3 pools: adapter -> (codes A_t, scales A_t, codes B, scales B) per projection
+        store, qstore = {}, {}
         for a in range(w.n_adapters):
             r = int(w.ranks[a])
-            if a in touched:
+            key = a if a in touched else ("fill", r)
+            if key not in store:
                 A_t, B = w.adapter(a)
-                self.host[a] = ([pinned(x) for x in A_t], [pinned(x) for x in B])
+                if self.q8:
+                    qa = [G.slora_quantize_e4m3_rows(w.dtype, x) for x in A_t]
+                    qb = [G.slora_quantize_e4m3_rows(w.dtype, x) for x in B]
+                    qstore[key] = ([c for c, _ in qa], [s for _, s in qa], [c for c, _ in qb],
+                                   [s for _, s in qb])
+                    store[key] = ([pinned_bytes(c) for c, _ in qa], [pinned_bytes(c) for c, _ in qb])
+                else:
+                    store[key] = ([pinned(x) for x in A_t], [pinned(x) for x in B])
+            self.host[a] = store[key]
+            hA, hB = store[key]
+            if self.q8:
+                self.q8w[a] = qstore[key]
+                cA, sA, cB, sB = self.q8w[a]
+                G.slora_adapter_register_e4m3(self.pool.h, a, r, w.alpha, hA, sA, hB, sB)
             else:
-                if r not in fill:
-                    A_t, B = w.adapter(a)
-                    fill[r] = ([pinned(x) for x in A_t], [pinned(x) for x in B])
-                self.host[a] = fill[r]
-            hA, hB = self.host[a]
-            G.slora_adapter_register(self.pool.h, a, r, w.alpha, hA, hB)
+                G.slora_adapter_register(self.pool.h, a, r, w.alpha, hA, hB)
         ids = list(range(w.n_adapters)) if resident is None else [int(a) for a in resident]
         side = torch.cuda.Stream()
         for i in range(0, len(ids), chunk):
@@ -105,6 +125,20 @@ class Tensors:
         return (projs, xs, [x.stride(0) for x in xs], ys, [y.stride(0) for y in ys])
 
 
+def oracle_inputs_q8(pb: PoolBuild, p: int, tokens=None):
+    """(x bits, idx, y_in bits, codes A_t, scales A_t, codes B, scales B) of
+    projection p for the 8-bit oracle, with the codes and scales the pool
+    holds; restricted to `tokens` when given."""
+    w = pb.w
+    x, idx, y, _, _ = oracle_inputs(w, p, tokens)
+    n = w.n_adapters
+    qa, sa, qb, sb = [None] * n, [None] * n, [None] * n, [None] * n
+    for a in set(np.unique(idx[idx >= 0]).tolist()):
+        cA, sA, cB, sB = pb.q8w[a]
+        qa[a], sa[a], qb[a], sb[a] = cA[p], sA[p], cB[p], sB[p]
+    return x, idx, y, qa, sa, qb, sb
+
+
 def oracle_inputs(w: W.Workload, p: int, tokens=None):
     """(x bits, idx, y_in bits, A_t list, B list) of projection p for the oracle,
     restricted to `tokens` (row indices) when given."""
@@ -121,6 +155,35 @@ def oracle_inputs(w: W.Workload, p: int, tokens=None):
         At_all, B_all = w.adapter(a)
         A_t[a], B[a] = At_all[p], B_all[p]
     return x, idx, y, A_t, B
+
+
+def tile_tokens(req_start, req_adapter, tile=128, per_tile=1, seed=0, offset=0):
+    """Token indices that touch every tile the prefill path computes: for each
+    request and for each merged segment (neighbouring requests on one adapter),
+    its first and last token and `per_tile` random tokens of every `tile`-token
+    tile counted from its start; plus one random token of every `tile`-token
+    window of the whole range.  `offset` is added to every index."""
+    rng = np.random.default_rng(seed)
+    rs = np.asarray(req_start, np.int64)
+    ra = np.asarray(req_adapter)
+    spans = [(int(rs[q]), int(rs[q + 1])) for q in range(ra.size) if rs[q + 1] > rs[q]]
+    q = 0
+    while q < ra.size:  # merged segments
+        e = q
+        while e + 1 < ra.size and ra[e + 1] == ra[q]:
+            e += 1
+        if rs[e + 1] > rs[q]:
+            spans.append((int(rs[q]), int(rs[e + 1])))
+        q = e + 1
+    lo, hi = int(rs[0]), int(rs[-1])
+    spans += [(b, min(b + tile, hi)) for b in range(lo, hi, tile)]
+    out = set()
+    for b, e in spans:
+        out.update((b, e - 1))
+        for t0 in range(b, e, tile):
+            t1 = min(t0 + tile, e)
+            out.update(int(v) for v in rng.integers(t0, t1, size=per_tile))
+    return np.array(sorted(out), np.int64) + offset
 
 
 def tolerance_check(got_bits: np.ndarray, ref: np.ndarray, dtype):

@@ -90,6 +90,41 @@ typedef enum {
   SLORA_PAGEIN_MEMCPY = 1      /* one cudaMemcpyAsync per run of consecutive pages */
 } slora_pagein_mode_t;
 
+/* Kernels that run slora_lora_delta (and slora_lora_delta_noalloc).  Both give
+ * the same arithmetic (fp32 partials per 2048-element slice of d_in, summed in
+ * slice order, one rounding of y); they differ in launches and scheduling.
+ * slora_decode_kernels() tells which one a call takes. */
+typedef enum {
+  SLORA_DECODE_AUTO = 0,       /* the library's choice: the one-kernel path for
+                                  e4m3 pools, the three-kernel path for 16-bit
+                                  pools (the faster one on B200 at the shapes
+                                  measured so far)                              */
+  SLORA_DECODE_SPLIT = 1,      /* always three kernels: segment build, shrink,
+                                  expand                                         */
+  SLORA_DECODE_FUSED = 2       /* one persistent kernel for calls of up to 1024
+                                  tokens (every CTA builds the segment table, then
+                                  the shrink and expand tasks in one launch); the
+                                  three kernels above that                       */
+} slora_decode_path_t;
+
+/* How a pool stores adapter weights in its pages. */
+typedef enum {
+  SLORA_WEIGHTS_16 = 0,        /* the pool's 16-bit dtype (fp16 / bf16)             */
+  SLORA_WEIGHTS_E4M3 = 1       /* 8-bit e4m3 codes (finite-only form: 4 exponent bits,
+                                  bias 7, 3 fraction bits, max 448) with one fp32
+                                  scale per rank row of each tensor: weight =
+                                  scale[row] * value(code).  A page holds
+                                  2 * page_elems codes, so an adapter takes about half
+                                  the pages and half the HBM and PCIe bytes
+                                  [S2 trade-offs section: adapters quantised to FP8
+                                  halve PCIe traffic and keep more of them warm].
+                                  x and y stay 16-bit; accumulation is fp32.  Decode
+                                  calls of up to 1024 tokens (slora_lora_delta and
+                                  slora_lora_delta_noalloc on the one-kernel path) take
+                                  such pools; the other compute calls return
+                                  SLORA_ERR_UNSUPPORTED.                           */
+} slora_weight_format_t;
+
 #define SLORA_MAX_PROJ 8
 
 typedef struct slora_pool slora_pool;
@@ -113,7 +148,9 @@ typedef struct {
                                (LRU, page accounting and validation run; compute
                                calls return SLORA_ERR_UNSUPPORTED).  For tests on
                                machines without a GPU.                               */
-  int32_t reserved[7];
+  int32_t decode_path;      /* slora_decode_path_t: kernels of slora_lora_delta     */
+  int32_t weight_format;    /* slora_weight_format_t of every adapter in the pool    */
+  int32_t reserved[5];
 } slora_pool_desc;
 
 typedef struct {
@@ -143,7 +180,8 @@ size_t slora_tables_bytes(const slora_pool_desc* desc);
 size_t slora_scratch_bytes(const slora_pool_desc* desc);
 
 /* Pages one adapter of rank `rank` occupies: sum over projections of
- * ceil(rank*d_in/page_elems) + ceil(rank*d_out/page_elems) [S2 paged pool]. */
+ * ceil(rank*d_in/page_elems) + ceil(rank*d_out/page_elems) [S2 paged pool];
+ * with e4m3 weights, of ceil(rank*d/(2*page_elems)) (two codes per element). */
 int64_t slora_pages_for_rank(const slora_pool_desc* desc, int32_t rank);
 
 /* ---- pool lifetime -------------------------------------------------------- */
@@ -176,6 +214,20 @@ slora_status_t slora_pool_set_page_order(slora_pool* pool, const int32_t* order,
  * adapter is INVALID_ARG; a non-resident one is replaced.                     */
 slora_status_t slora_adapter_register(slora_pool* pool, int32_t id, int32_t rank, float alpha,
                                       const void* const* host_A_t, const void* const* host_B);
+
+/* As slora_adapter_register, for a pool whose weight_format is
+ * SLORA_WEIGHTS_E4M3: codes_A_t[p] (rank x d_in[p] bytes) and codes_B[p]
+ * (rank x d_out[p] bytes) are e4m3 codes, row-major, in PINNED host memory,
+ * 16-byte aligned, valid until the adapter is unregistered; scales_A_t[p] and
+ * scales_B[p] hold one fp32 scale per rank row (host memory, copied by this
+ * call).  slora_quantize_e4m3_rows produces both from 16-bit rows.  Weight
+ * (k, j) of A_t is scales_A_t[p][k] * value(codes_A_t[p][k * d_in + j]).
+ * Errors: as slora_adapter_register; INVALID_ARG on a 16-bit pool (and
+ * slora_adapter_register is INVALID_ARG on an e4m3 pool), or for a scale that
+ * is negative or not finite.                                                  */
+slora_status_t slora_adapter_register_e4m3(slora_pool* pool, int32_t id, int32_t rank, float alpha,
+                                           const void* const* codes_A_t, const float* const* scales_A_t,
+                                           const void* const* codes_B, const float* const* scales_B);
 
 /* Makes every adapter in ids[0..n) resident and pins them for the compute
  * calls that follow, until the next page_in call [S1 Unified Paging: on-demand
@@ -338,32 +390,39 @@ slora_status_t slora_sgmv(slora_pool* pool, int32_t n, const int32_t* projs,
                           const int64_t* ldy, const int32_t* seg_start,
                           const int32_t* seg_adapter, int32_t S, int32_t T, void* stream);
 
-/* The fused decode delta of slora_lora_delta, for callers that cannot
- * allocate device memory at the point of the call: a serving loop captured
- * into a CUDA graph (no device allocation while a stream is captured in the
- * global capture mode), a plug-in whose host framework owns every device
- * allocation, or a path that must not risk an allocation blocking the device.
+/* The decode delta of slora_lora_delta, for callers that cannot allocate
+ * device memory at the point of the call: a plug-in whose host framework owns
+ * every device allocation and hands it only inputs and outputs, or a serving
+ * loop that must not risk an allocation blocking the device.
  * The pages have no counterpart of this entry point; it is an addition of this
  * library.
  * Same arguments, semantics and kernels as slora_lora_delta, but the call's
- * scratch (segments, work plan, counters, fp32 partials and t) is taken from a
- * fixed device array that the library reserves on every GPU that loads it
+ * scratch (segments, work plan, counters, fp32 partials) is taken from a fixed
+ * device array that the library reserves on every GPU that loads it
  * (slora_noalloc_scratch_bytes(), 8 MiB) instead of the pool's dev_scratch.
  * Nothing is allocated or freed by the call.
  *   - The first call on a device looks up that array's device address (once
- *     per device, with the device current); make that first call before any
- *     stream capture.
+ *     per device, with the device current) and keeps it for the life of the
+ *     process; make that first call before any stream capture.  Resetting the
+ *     device while the library is loaded is not supported.
  *   - All calls share the one array and it keeps the last call's contents; the
- *     kernels initialise what must start at zero themselves.  Calls whose
- *     kernels overlap on the GPU (other streams, other threads) race on it:
- *     serialise them.
- *   - A call whose scratch need (it grows with T, the projections named and
- *     max_rank) exceeds the array fails with SLORA_ERR_INVALID_ARG and a
- *     message giving both sizes; nothing is enqueued.                         */
+ *     kernels clear what must start at zero themselves.  Calls whose kernels
+ *     overlap on the GPU (other streams, other threads) race on it: serialise
+ *     them.
+ *   - A call whose scratch need exceeds the array fails with
+ *     SLORA_ERR_INVALID_ARG and a message giving both sizes; nothing is
+ *     enqueued.  The need grows with T, max_rank and the projections the call
+ *     names (their fp32 partials: ceil(d_in / 2048) x T x round8(max_rank)
+ *     floats each), plus about 40 KB of tables.                               */
 slora_status_t slora_lora_delta_noalloc(slora_pool* pool, int32_t n, const int32_t* projs,
                                         const void* const* x, const int64_t* ldx,
                                         void* const* y, const int64_t* ldy, const int32_t* idx,
                                         int32_t T, void* stream);
+
+/* Number of kernels slora_lora_delta launches for a call of T tokens on this
+ * pool (1: the one-kernel path, 3: segment build, shrink, expand); 0 for T <= 0
+ * or a NULL pool.  Host only. */
+int32_t slora_decode_kernels(const slora_pool* pool, int32_t T);
 
 /* Size in bytes of the fixed scratch array used by slora_lora_delta_noalloc. */
 size_t slora_noalloc_scratch_bytes(void);
@@ -371,8 +430,9 @@ size_t slora_noalloc_scratch_bytes(void);
 /* ---- diagnostics ---------------------------------------------------------- */
 
 /* Reads back adapter `id`'s weights for projection `proj` from its pages into
- * host_A_t (rank x d_in) and host_B (rank x d_out), synchronously.  For tests of
- * the page-table gather (bit-exact).                                           */
+ * host_A_t (rank x d_in) and host_B (rank x d_out), synchronously: 16-bit
+ * elements, or e4m3 codes (one byte each) in an e4m3 pool.  For tests of the
+ * page-table gather (bit-exact).                                               */
 slora_status_t slora_debug_gather(slora_pool* pool, int32_t id, int32_t proj, void* host_A_t,
                                   void* host_B);
 

@@ -50,6 +50,37 @@ def test_sizing_matches_oracle_page_count():
     for r in (0, 8, 16, 24, 64):
         assert G.slora_pages_for_rank(d, r) == oracle.pages_needed(r, *LAYER7B, 8192)
     assert G.slora_tables_bytes(d) > 0 and G.slora_scratch_bytes(d) > 0
+    # e4m3 weights: a page of page_elems 16-bit units holds 2 * page_elems codes
+    d8 = G.make_desc(G.SLORA_F16, *LAYER7B, 1000, 64, 256, 8192, 10, weight_format=G.SLORA_WEIGHTS_E4M3)
+    for r in (0, 3, 8, 16, 24, 64):
+        assert G.slora_pages_for_rank(d8, r) == oracle.pages_needed(r, *LAYER7B, 2 * 8192)
+    # the tables grow by the row-scale table of every adapter
+    assert G.slora_tables_bytes(d8) >= G.slora_tables_bytes(d) + 4 * 1000 * 7 * 2 * 64
+
+
+def test_e4m3_pool_registration_and_lru():
+    """A host-only e4m3 pool: registration needs codes and scales (and the
+    16-bit call is refused), pages are counted at two codes per unit, LRU as
+    for 16-bit pools."""
+    pool = G.Pool(G.SLORA_F16, [1024, 2048], [2048, 1024], 8, 32, 64, 1024, 192, host_only=True,
+                  weight_format=G.SLORA_WEIGHTS_E4M3)
+    codes = np.zeros(16, np.uint8)
+    sc = np.ones(32, np.float32)
+    with pytest.raises(G.SloraError) as e:
+        G.slora_adapter_register(pool.h, 0, 8, 16.0, [codes, codes], [codes, codes])
+    assert e.value.status == 1
+    with pytest.raises(G.SloraError) as e:   # a negative scale
+        G.slora_adapter_register_e4m3(pool.h, 0, 8, 16.0, [codes, codes], [-sc, sc], [codes, codes],
+                                      [sc, sc])
+    assert e.value.status == 1
+    for a in range(4):
+        G.slora_adapter_register_e4m3(pool.h, a, 32, 16.0, [codes, codes], [sc, sc], [codes, codes],
+                                      [sc, sc])
+    need = pool.pages_for_rank(32)
+    assert need == 2 * (32 * 1024 // 2048 + 32 * 2048 // 2048)      # 96: half of the 16-bit count
+    pool.page_in([0, 1])
+    pool.page_in([2])                  # 192 pages hold two adapters: the oldest (0) goes
+    assert [G.slora_adapter_is_resident(pool.h, a) for a in range(4)] == [0, 1, 1, 0]
 
 
 def _host_pool(n_pages=100, max_adapters=40, max_rank=32, page=1024):

@@ -1,5 +1,9 @@
 """GPU parity of the decode path (segment build + paged shrink + expand) with
-the fp64 oracle, on the same seeded inputs.
+the fp64 oracle, on the same seeded inputs.  Both decode paths are checked:
+the one persistent kernel (pools created with SLORA_DECODE_FUSED, batches of
+up to 1024 tokens) and the three-kernel path (SLORA_DECODE_SPLIT, the default
+for 16-bit pools, and every batch above 1024 tokens); the two must agree bit
+for bit (same fp32 partials, same summation order).
 
 Acceptance bound, per projection output y_out:
     |gpu - oracle| <= 1e-2 * max|oracle| + 1e-3   (elementwise)
@@ -65,8 +69,12 @@ def test_tiny_config():
     pb.close()
 
 
+PATHS = [G.SLORA_DECODE_FUSED, G.SLORA_DECODE_SPLIT]
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["fused", "split"])
 @pytest.mark.parametrize("dtype", [W.F16, W.BF16])
-def test_ragged_mixed(dtype):
+def test_ragged_mixed(dtype, path):
     """Ragged everything: d_in not a multiple of the 1024-element chunk nor of
     256, ranks not multiples of 8, rank 0, tokens without adapter, segments of
     1, 2, 3, 4, 5..40 tokens (all token classes), shared x across projections."""
@@ -78,7 +86,7 @@ def test_ragged_mixed(dtype):
     idx = np.concatenate([np.full(c, a) for a, c in enumerate(counts)] + [np.full(5, -1)])
     idx = idx[rng.permutation(idx.size)].astype(np.int32)
     w = _custom(dtype, projs, ranks, idx, page_elems=512)
-    pb = H.PoolBuild(w)
+    pb = H.PoolBuild(w, decode_path=path)
     ten = H.Tensors(w)
     _run_delta(pb, ten, w)
     _check_all(w, ten, tight=True)
@@ -176,13 +184,48 @@ def test_bad_token_is_skipped_and_reported():
 def test_full_size_configs(cfg):
     """LLaMA-7B (fp16, 1000 adapters r=16, Zipf 1.0, T=256) and LLaMA-13B (bf16,
     2000 adapters r in {8..64}, Zipf 1.2, shuffled pool, T=512) decode layers,
-    in the launch configuration bench.py times, every output element compared."""
+    on the one-kernel path, every output element compared; then the
+    three-kernel path on the same pool layout must give the same bits."""
     w = W.config(cfg)
-    pb = H.PoolBuild(w)
+    pb = H.PoolBuild(w, decode_path=G.SLORA_DECODE_FUSED)
     ten = H.Tensors(w)
     _run_delta(pb, ten, w)
     _check_all(w, ten, threads=16)
+    fused = [H.from_device(t) for t in ten.y]
     pb.close()
+    pb = H.PoolBuild(w, decode_path=G.SLORA_DECODE_SPLIT)
+    ten.reset()
+    _run_delta(pb, ten, w)
+    for p in range(len(w.projs)):
+        assert np.array_equal(fused[p], H.from_device(ten.y[p])), w.projs[p].name
+    pb.close()
+
+
+@pytest.mark.parametrize("T", [1, 2, 33, 1024])
+def test_fused_matches_split_bitwise(T):
+    """Token counts at the edges of the one-kernel path (1 token, 2, a ragged
+    33, the 1024-token limit) with Zipf-skewed ids over mixed ranks: the fused
+    kernel and the three-kernel path give identical bits, and both match the
+    oracle on sampled tokens."""
+    rng = np.random.default_rng(100 + T)
+    projs = [W.Proj("q", 2048, 2048, "a"), W.Proj("v", 2048, 512, "a"), W.Proj("d", 5504, 2048, "c")]
+    n_ad = 64
+    ranks = rng.choice(np.array([8, 16, 32, 64, 128, 24], np.int32), n_ad)
+    idx = W.zipf_ids(rng, n_ad, 1.1, T)
+    if T > 2:
+        idx[rng.random(T) < 0.1] = -1
+    w = _custom(W.BF16, projs, ranks, idx, page_elems=8192, shuffle=True, seed=31)
+    outs = []
+    for path in PATHS:
+        pb = H.PoolBuild(w, decode_path=path)
+        ten = H.Tensors(w)
+        _run_delta(pb, ten, w)
+        outs.append([H.from_device(t) for t in ten.y])
+        pb.close()
+    for p in range(len(projs)):
+        assert np.array_equal(outs[0][p], outs[1][p]), projs[p].name
+    tokens = np.arange(T) if T <= 64 else np.sort(rng.choice(T, 96, replace=False))
+    _check_all(w, ten, tokens=tokens, tight=True, threads=16)
 
 
 def test_many_single_stage_tasks_repeatable():

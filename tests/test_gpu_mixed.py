@@ -4,7 +4,8 @@ adapters of ranks 8..128, 30% of the step's adapters cold.
 
 The cold adapters come in from pinned host memory on a side stream and take
 their pages from untouched adapters by LRU eviction; the step's output is
-checked against the fp64 oracle on sampled tokens of both parts, the cold
+checked against the fp64 oracle on every decode token and on tokens covering
+every 128-token tile of the prefill requests, the cold
 adapters' pages against their host bytes (bit-exact), and a second step,
 after the pool has been put back, must give bit-identical output.
 """
@@ -19,11 +20,14 @@ import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def _sample(w, n_dec=128, n_pre=128, seed=11):
-    rng = np.random.default_rng(seed)
-    dec = rng.choice(w.n_decode, size=n_dec, replace=False)
-    pre = w.n_decode + rng.choice(w.T - w.n_decode, size=n_pre, replace=False)
-    return np.sort(np.concatenate([dec, pre]))
+def _sample(w, seed=11):
+    """Every decode token (the decode batch is one kernel's whole work), and on
+    the prefill side every 128-token tile of every request (two random tokens
+    per tile plus each request's first and last token)."""
+    dec = np.arange(w.n_decode)
+    pre = H.tile_tokens(w.req_start - w.n_decode, w.req_adapter, per_tile=2, seed=seed,
+                        offset=w.n_decode)
+    return np.unique(np.concatenate([dec, pre]))
 
 
 @pytest.mark.parametrize("mode", [G.SLORA_PAGEIN_KERNEL, G.SLORA_PAGEIN_MEMCPY])

@@ -124,15 +124,17 @@ def test_sgmv_bad_segment_is_skipped():
     pb.close()
 
 
-def test_sgmv_prefill_config_sampled():
+def test_sgmv_prefill_config_every_tile():
     """The LLaMA-7B prefill workload (32 requests of 64..1024 tokens, 64
     adapters of rank 16/32/64, bf16) in the launch configuration bench.py
-    times; 256 sampled tokens, every projection, against the oracle."""
+    times; every projection against the oracle on tokens that touch every
+    128-token tile of every request and merged segment (two random tokens per
+    tile, plus each one's first and last token) and every 128-token window."""
     w = W.config(3)
     pb = H.PoolBuild(w)
     ten = H.Tensors(w)
     _run_sgmv(pb, ten, w, w.req_start, w.req_adapter)
-    rng = np.random.default_rng(7)
-    tokens = np.sort(rng.choice(w.T, size=256, replace=False))
-    _check(w, ten, tokens=tokens, tight=True)
+    tokens = H.tile_tokens(w.req_start, w.req_adapter, per_tile=2, seed=7)
+    assert tokens.size > 300
+    _check(w, ten, tokens=tokens, tight=True, threads=32)
     pb.close()
