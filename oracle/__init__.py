@@ -35,6 +35,7 @@ def lib():
         L.oracle_lru_prefetch_run.argtypes = [i32, P, i64, i32, P, P, P, P, P, P]
         L.oracle_decode_e4m3.argtypes = [P, i64, P]
         L.oracle_quantize_e4m3.argtypes = [P, i64, ctypes.c_double, P]
+        L.oracle_linear.argtypes = [i32, i32, i32, i32, P, i64, P, i64, P, i32]
         L.oracle_lora_delta_q8.argtypes = [i32, i32, i32, i32, P, i64, P, P, i64, i32, P, P, P, P,
                                            P, P, P, i32]
         _lib = L
@@ -128,6 +129,29 @@ def quantize_rows_e4m3(values):
     codes = np.stack([quantize_e4m3(row, float(s)) for row, s in zip(values, scales)]) \
         if values.shape[0] else np.zeros(values.shape, np.uint8)
     return codes, scales
+
+
+def linear(dtype, x, w0, n_threads=1):
+    """fp64 y = x . W0 for x (T, d_in) bits and w0 (d_out, d_in) bits (the
+    layout of a linear layer's weight)."""
+    x = _c(x, np.uint16)
+    w0 = _c(w0, np.uint16)
+    T, d_in = x.shape
+    d_out = w0.shape[0]
+    assert w0.shape[1] == d_in
+    y = np.empty((T, d_out), np.float64)
+    if lib().oracle_linear(dtype, T, d_in, d_out, _p(x), d_in, _p(w0), d_in, _p(y), int(n_threads)) != 0:
+        raise ValueError("oracle_linear: invalid argument")
+    return y
+
+
+def linear_lora(dtype, x, w0, idx, ranks, alphas, A_t, B, n_threads=1):
+    """fp64 Y = X.W0 + (alpha_a / r_a) (x_i . A_a) . B_a per token: the base
+    linear map plus the delta (the delta starts from zero)."""
+    x = _c(x, np.uint16)
+    zero = np.zeros((x.shape[0], np.asarray(w0).shape[0]), np.uint16)
+    return linear(dtype, x, w0, n_threads) + lora_delta(dtype, x, idx, zero, ranks, alphas, A_t, B,
+                                                         n_threads)
 
 
 def lora_delta_q8(dtype, x, idx, y_in, ranks, alphas, qA_t, sA, qB, sB, n_threads=1):

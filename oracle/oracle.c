@@ -22,6 +22,14 @@
  *      of d_out.  Element values are fp16 or bf16 bit patterns, decoded
  *      exactly to fp64 by the decoders below.
  *
+ *  oracle_linear       -- the base term of the same page's scaled form,
+ *                         y = X.W0 (W0 stored as d_out rows of d_in, the
+ *                         layout of a linear layer's weight), fp64 sums in
+ *                         ascending index order.  With oracle_lora_delta it
+ *                         gives the whole linear layer with its LoRA delta,
+ *                         Y = X.W0 + (alpha/r).((X.A).B) -- the output that the
+ *                         "residual add fused into the linear layer's output"
+ *                         remark of the page's metrics section refers to.
  *  oracle_segments     -- stable counting sort of tokens by adapter id: the
  *                         segment structure of SGMV ("index vector maps each
  *                         token to its adapter", same SGMV section).
@@ -261,6 +269,55 @@ long oracle_pages_needed(int rank, int n_proj, const int* d_in, const int* d_out
   for (int p = 0; p < n_proj; ++p)
     n += cdiv((long)rank * d_in[p], page_elems) + cdiv((long)rank * d_out[p], page_elems);
   return n;
+}
+
+/* ------------------------------------------------------------------------- */
+/* The base linear map y = x . W0 (W0 given as d_out rows of d_in).          */
+typedef struct {
+  int dtype, d_in, d_out;
+  const uint16_t* x;
+  long ldx;
+  const uint16_t* w;
+  long ldw;
+  double* y;
+  int t0, t1;
+} linear_job;
+
+static void* linear_worker(void* arg) {
+  linear_job* J = (linear_job*)arg;
+  double* xr = (double*)malloc(sizeof(double) * J->d_in);
+  for (int i = J->t0; i < J->t1; ++i) {
+    for (int j = 0; j < J->d_in; ++j) xr[j] = dec(J->dtype, J->x[(long)i * J->ldx + j]);
+    for (int l = 0; l < J->d_out; ++l) {
+      const uint16_t* wl = J->w + (long)l * J->ldw;
+      double acc = 0.0;
+      for (int j = 0; j < J->d_in; ++j) acc += xr[j] * dec(J->dtype, wl[j]);
+      J->y[(long)i * J->d_out + l] = acc;
+    }
+  }
+  free(xr);
+  return NULL;
+}
+
+int oracle_linear(int dtype, int T, int d_in, int d_out, const uint16_t* x, long ldx, const uint16_t* w,
+                  long ldw, double* y_out, int n_threads) {
+  if ((dtype != 0 && dtype != 1) || T < 0 || d_in <= 0 || d_out <= 0 || ldx < d_in || ldw < d_in ||
+      n_threads < 1)
+    return OR_ERR_ARG;
+  if (n_threads > T) n_threads = T > 0 ? T : 1;
+  linear_job* jobs = (linear_job*)calloc(n_threads, sizeof(linear_job));
+  pthread_t* th = (pthread_t*)calloc(n_threads, sizeof(pthread_t));
+  for (int k = 0; k < n_threads; ++k) {
+    linear_job j = {dtype, d_in, d_out, x, ldx, w, ldw, y_out, (int)((long)T * k / n_threads),
+                    (int)((long)T * (k + 1) / n_threads)};
+    jobs[k] = j;
+  }
+  for (int k = 1; k < n_threads; ++k) pthread_create(&th[k], NULL, linear_worker, &jobs[k]);
+  linear_worker(&jobs[0]);
+  for (int k = 1; k < n_threads; ++k) pthread_join(th[k], NULL);
+  free(jobs);
+  free(th);
+  return OR_OK;
 }
 
 /* ------------------------------------------------------------------------- */

@@ -20,6 +20,7 @@ import pytest
 
 import oracle
 from workloads import BF16, F16, to_bits
+import workloads as W
 
 
 def _bits(dtype, a):
@@ -450,3 +451,69 @@ def test_q8_delta_scales_enter_per_row():
     a = oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0), qA, sA, qB, ones)
     b = oracle.lora_delta_q8(F16, x, idx, y, ranks, np.full(3, 16.0), qA2, ones, qB, ones)
     assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------------------
+# The base linear map and the whole layer Y = X.W0 + (alpha/r).((X.A).B)
+
+def test_linear_lora_hand_example():
+    """Worked by hand: x = [[1, 2, 3], [0.5, -1, 2]], W0 (2 x 3, a linear
+    layer's weight) = [[1, 0, -1], [2, 1, 0.5]] gives X.W0 = [[-2, 5.5],
+    [-1.5, 1]]; token 0 uses a rank-1 adapter with alpha 2 (scale 2),
+    A_t = [[1, 1, 0]] (t = 3) and B = [[0.5, -1]] (delta [3, -6]); token 1 has
+    no adapter.  Y = [[1, -0.5], [-1.5, 1]]."""
+    f = lambda a: W.to_bits(W.F16, np.asarray(a, np.float32))
+    x = f([[1, 2, 3], [0.5, -1, 2]])
+    w0 = f([[1, 0, -1], [2, 1, 0.5]])
+    y = oracle.linear_lora(W.F16, x, w0, np.array([0, -1]), [1], [2.0], [f([[1, 1, 0]])], [f([[0.5, -1]])])
+    assert np.array_equal(y, [[1.0, -0.5], [-1.5, 1.0]])
+    assert np.array_equal(oracle.linear(W.F16, x, w0), [[-2.0, 5.5], [-1.5, 1.0]])
+
+
+def _layer_inputs(seed, dtype=W.BF16, T=9, d_in=96, d_out=80):
+    rng = np.random.default_rng(seed)
+    x = W.to_bits(dtype, rng.standard_normal((T, d_in)).astype(np.float32))
+    w0 = W.to_bits(dtype, (rng.standard_normal((d_out, d_in)) / np.sqrt(d_in)).astype(np.float32))
+    ranks = [4, 8]
+    A_t = [W.to_bits(dtype, rng.standard_normal((r, d_in)).astype(np.float32)) for r in ranks]
+    B = [W.to_bits(dtype, rng.standard_normal((r, d_out)).astype(np.float32)) for r in ranks]
+    idx = rng.integers(-1, 2, T).astype(np.int32)
+    return x, w0, idx, ranks, A_t, B
+
+
+def test_linear_lora_with_zero_base_is_the_delta():
+    x, w0, idx, ranks, A_t, B = _layer_inputs(1)
+    zero_w = np.zeros_like(w0)
+    y = oracle.linear_lora(W.BF16, x, zero_w, idx, ranks, [16.0, 16.0], A_t, B)
+    ref = oracle.lora_delta(W.BF16, x, idx, np.zeros((x.shape[0], w0.shape[0]), np.uint16), ranks,
+                            [16.0, 16.0], A_t, B)
+    assert np.array_equal(y, ref)          # 0 + delta: bit for bit
+
+
+def test_linear_lora_without_adapters_is_a_matmul():
+    x, w0, idx, ranks, A_t, B = _layer_inputs(2)
+    X = H_decode(x, W.BF16)
+    Wm = H_decode(w0, W.BF16)
+    ref = X @ Wm.T                          # numpy's fp64 matmul (another summation order)
+    for ids in (np.full(x.shape[0], -1, np.int32), idx):
+        zA = [np.zeros_like(a) for a in A_t] if ids is idx else A_t
+        y = oracle.linear_lora(W.BF16, x, w0, ids, ranks, [16.0, 16.0], zA, B)
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_linear_is_linear_in_the_weight():
+    x, w0, _, _, _, _ = _layer_inputs(3, dtype=W.F16)
+    rng = np.random.default_rng(4)
+    # two weights whose sum is exact in fp16 (small integers)
+    w1 = W.to_bits(W.F16, rng.integers(-4, 5, w0.shape).astype(np.float32))
+    w2 = W.to_bits(W.F16, rng.integers(-4, 5, w0.shape).astype(np.float32))
+    ws = W.to_bits(W.F16, (H_decode(w1, W.F16) + H_decode(w2, W.F16)).astype(np.float32))
+    a, b, c = (oracle.linear(W.F16, x, w) for w in (w1, w2, ws))
+    assert np.allclose(a + b, c, rtol=1e-13, atol=1e-13 * np.abs(c).max())
+
+
+def H_decode(bits, dtype):
+    bits = np.asarray(bits, np.uint16)
+    if dtype == W.F16:
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
