@@ -46,6 +46,9 @@ FALLBACK_HBM = 6650.0
 FALLBACK_BF16 = 1590.0
 
 
+FALLBACK_BF16_SUSTAINED = 1400.0
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -53,6 +56,17 @@ def peaks():
         return float(m["hbm_gbs"]), float(m["bf16_tflops"]), "measured"
     except Exception:
         return FALLBACK_HBM, FALLBACK_BF16, "fallback"
+
+
+def bf16_sustained():
+    """The bf16 peak for a kernel timed inside a long step (the power-capped
+    loop figure), else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m.get("bf16_tflops_sustained", m["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_BF16_SUSTAINED, "fallback"
 
 
 # ---------------------------------------------------------------------------
@@ -287,6 +301,8 @@ def run_ours(args, rank, world):
     w = replica_workload(args.config, rank)
     if args.config == 4:
         return run_mixed(args, rank, world, w)
+    if args.linear:
+        return run_linear(args, rank, world, w)
     R = PrefillRun(w) if args.config == 3 else DecodeRun(w, path=args.path, weights=args.weights)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -462,6 +478,94 @@ def run_ours(args, rank, world):
         "clocks": clk,
     }
     R.pb.close()
+    return out
+
+
+# ---------------------------------------------------------------------------
+def run_linear(args, rank, world, w):
+    """The prefill linear layer with its delta in one tensor-core kernel
+    (slora_sgmv_linear): y = x . W0 + delta for the 7 projections of the
+    layer, with random-init base weights.  Timed with L2 flushed before each
+    step, and once more with every segment's adapter set to -1 (the base
+    GEMM alone, same kernel) to give the delta's overhead."""
+    import torch
+
+    import gather_lora_paged_b200 as G
+    import harness as H
+    dev = int(os.environ.get("LOCAL_RANK", 0))
+    pb = H.PoolBuild(w)
+    ten = H.Tensors(w)
+    w0s = [H.to_device(w.w0(p), w.dtype) for p in range(len(w.projs))]
+    rs, ra = w.req_start, w.req_adapter
+    ss, sa = [0], []
+    for q in range(ra.size):  # merged segments covering [0, T)
+        if sa and sa[-1] == ra[q]:
+            ss[-1] = int(rs[q + 1])
+        else:
+            sa.append(int(ra[q]))
+            ss.append(int(rs[q + 1]))
+    d_ss = torch.tensor(ss, dtype=torch.int32, device="cuda")
+    d_sa = torch.tensor(sa, dtype=torch.int32, device="cuda")
+    d_none = torch.full_like(d_sa, -1)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    projs, xs, ldx, ys, ldy = ten.args()
+    ldw = [t.stride(0) for t in w0s]
+
+    def step(ads):
+        G.slora_sgmv_linear(pb.h, projs, xs, ldx, w0s, ldw, ys, ldy, d_ss, ads, len(sa), w.T, stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(d_sa)
+    torch.cuda.synchronize()
+    st, code, info = G.slora_check_device(pb.h)
+    assert st == 0, (code, info)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    res = {}
+    for name, ads in (("lora", d_sa), ("base", d_none)):
+        if world > 1:
+            torch.distributed.barrier()
+        t = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            e0.record(stream)
+            step(ads)
+            e1.record(stream)
+            e1.synchronize()
+            t += e0.elapsed_time(e1)
+        res[name] = max_over_ranks(t, world, "cuda") / args.steps
+    clk = clocks.stop()
+    K = args.steps
+    ms = res["lora"]
+    din = [p.d_in for p in w.projs]
+    dout = [p.d_out for p in w.projs]
+    base_flops = 2 * w.T * sum(a * b for a, b in zip(din, dout))
+    alg = algorithmic(w)
+    flops = base_flops + alg["flops"]
+    tflops = flops / (ms / 1e3) / 1e12
+    peak, src = bf16_sustained()
+    out = {
+        "metric": METRIC, "value": job_throughput(world, w.T, K, ms * K), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": W.DTYPE_NAME[w.dtype],
+        "data": "synthetic (seeded N(0,1) activations; N(0,1/sqrt(d_in)) base weights and A; "
+                "N(0,1/sqrt(r)) B)",
+        "config": {"workload": w.name + "_linear_layer", "tokens_per_step": w.T, "projections": len(w.projs),
+                   "segments": len(sa), "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
+                   "what": "y = x.W0 + (alpha/r)(x.A).B in one tcgen05 kernel per layer (base GEMM fused "
+                           "with the delta)", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "linear", "achieved": tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None, "peak_source": src,
+                     "flops_per_step": flops},
+        "lora_overhead": {"base_only_ms": res["base"], "with_delta_ms": ms,
+                          "overhead_frac": ms / res["base"] - 1.0},
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    pb.close()
     return out
 
 
@@ -733,6 +837,8 @@ def main():
     ap.add_argument("--path", default="auto", choices=["auto", "split", "fused"],
                     help="decode kernels: the library's choice, the three-kernel path (segment "
                          "build, shrink, expand) or the one persistent kernel")
+    ap.add_argument("--linear", action="store_true",
+                    help="--config 3: the whole linear layer (base GEMM + delta) in one kernel")
     ap.add_argument("--weights", default="16", choices=["16", "e4m3"],
                     help="decode: adapter pages in the pool's 16-bit dtype or as e4m3 codes")
     ap.add_argument("--pagein", default="kernel", choices=["kernel", "memcpy"],

@@ -87,6 +87,7 @@ def lib():
         "slora_bgmv_expand": ([P, I32, P, I64, P, I32, P, I64, P], I32),
         "slora_lora_delta": ([P, I32, P, P, P, P, P, P, I32, P], I32),
         "slora_sgmv": ([P, I32, P, P, P, P, P, P, P, I32, I32, P], I32),
+        "slora_sgmv_linear": ([P, I32, P, P, P, P, P, P, P, P, P, I32, I32, P], I32),
         "slora_debug_gather": ([P, I32, I32, P, P], I32),
         "slora_check_device": ([P, P, POINTER(c_int32), POINTER(c_int32)], I32),
         "slora_pool_stats": ([P, POINTER(PoolStats)], I32),
@@ -327,6 +328,17 @@ def slora_sgmv(pool: int, projs, x, ldx, y, ldy, seg_start, seg_adapter, S: int,
     c = lambda a: ctypes.cast(a, c_void_p)  # noqa: E731
     _check(pool, lib().slora_sgmv(pool, n, c(pp), c(px), c(plx), c(py), c(ply), _ptr(seg_start),
                                   _ptr(seg_adapter), S, T, _stream(stream)))
+
+
+def slora_sgmv_linear(pool: int, projs, x, ldx, w0, ldw, y, ldy, seg_start, seg_adapter, S: int, T: int,
+                      stream=None) -> None:
+    """y = x . W0 + delta per projection (w0[k]: d_out x d_in device tensors)."""
+    n, pp, px, plx, py, ply = _slot_arrays(projs, x, ldx, y, ldy)
+    pw = _arr(c_void_p, [_ptr(t) for t in w0])
+    plw = _arr(c_int64, [int(v) for v in ldw])
+    c = lambda a: ctypes.cast(a, c_void_p)  # noqa: E731
+    _check(pool, lib().slora_sgmv_linear(pool, n, c(pp), c(px), c(plx), c(pw), c(plw), c(py), c(ply),
+                                         _ptr(seg_start), _ptr(seg_adapter), S, T, _stream(stream)))
 
 
 def slora_debug_gather(pool: int, id: int, proj: int, host_A_t, host_B) -> None:

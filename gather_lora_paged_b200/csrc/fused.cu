@@ -128,8 +128,9 @@ __device__ bool ready_wait(const int32_t* c, int target, int32_t* err) {
 }
 
 // Task counts and byte cost (256-byte units) of one segment of n tokens on a
-// rank-r adapter.  Cost: adapter bytes, re-reads of a later token group counted
-// at half weight (they mostly hit L2), activations, and 2 KB per stage.
+// rank-r adapter.  Cost: the bytes each task streams through the copy ring
+// (a token group after the first re-reads the rows, from L2 mostly, but its
+// stages take the ring just the same), activations, and 2 KB per stage.
 __device__ void seg_costs(const BgmvParams& p, int n, int r, int& n_s, int& n_e, int& c_s, int& c_e) {
   n_s = n_e = c_s = c_e = 0;
   if (n <= 0 || r <= 0) return;
@@ -140,13 +141,13 @@ __device__ void seg_costs(const BgmvParams& p, int n, int r, int& n_s, int& n_e,
     const int rows = G.n * r, ns = cdiv_i(G.d_in, kFKT);
     const int tasks = cdiv_i(rows, kFRB) * ntg * ns;
     n_s += tasks;
-    bs += 2ll * G.d_in * ((int64_t)rows * (ntg + 1) / 2 + n) + 2048ll * 2 * tasks;
+    bs += 2ll * G.d_in * ((int64_t)rows * ntg + n) + 2048ll * 2 * tasks;
   }
   for (int k = 0; k < p.n_slots; ++k) {
     const SlotDev& L = p.slot[k];
     const int tasks = nte * cdiv_i(L.d_out, kFELC);
     n_e += tasks;
-    be += 2ll * L.d_out * ((int64_t)r * (nte + 1) / 2 + 2 * n) + 2048ll * cdiv_i(r, kFRows) * tasks;
+    be += 2ll * L.d_out * ((int64_t)r * nte + 2 * n) + 2048ll * cdiv_i(r, kFRows) * tasks;
   }
   c_s = (int)(bs >> 8);
   c_e = (int)(be >> 8);
@@ -532,7 +533,7 @@ __global__ void __launch_bounds__(kFThreads, 1) k_delta(const __grid_constant__ 
   __shared__ FLook look[kFLook];
   __shared__ FDesc desc[kFNS];
   __shared__ float dqs[kFNS][8];  // e4m3: row scales of each ring stage
-  __shared__ int resolved, issued, xydone[kFXYBufs];
+  __shared__ int resolved, issued, xydone[kFXYBufs], warm_sink;
   __shared__ int sigq[kFSigQ], sig_n, sig_done;
   __shared__ FRanges R;
   unsigned char* ring = smem;
@@ -547,6 +548,14 @@ __global__ void __launch_bounds__(kFThreads, 1) k_delta(const __grid_constant__ 
   const int T = p.T, MA = p.pool.max_adapters;
   int32_t* err = p.pool.err;
 
+  {  // touch every 64-byte line of the parameter block once, so that later
+     // lookups with runtime indices (groups, slots) hit the constant cache
+    constexpr int kLines = (int)((sizeof(BgmvParams) + 63) / 64);
+    if (tid < kLines) {
+      const int v = reinterpret_cast<const int*>(&p)[tid * 16];
+      if (v == 0x5a5a5a5a) warm_sink = v;  // keeps the load; the value is never used
+    }
+  }
   if (tid == 0) {
     for (int s = 0; s < kFNS; ++s) {
       mbar_init(&full[s], 1);

@@ -32,6 +32,9 @@ cudaError_t launch_sgmv(const BgmvParams& p, int dtype, const int32_t* seg_start
                         const int32_t* seg_adapter, int S, int T, int sm_count, cudaStream_t s,
                         void* scratch, int max_tokens, int64_t n_pages, cudaEvent_t const* ev, int n_ev);
 size_t sgmv_scratch_bytes(const slora_pool_desc& d);
+cudaError_t launch_linear(const BgmvParams& bp, int dtype, const void* const* w0, const int64_t* ldw,
+                          const int32_t* seg_start, const int32_t* seg_adapter, int S, int T, int sm_count,
+                          cudaStream_t st, void* scratch, int max_tokens, int64_t n_pages);
 }  // namespace slora
 
 namespace {
@@ -452,6 +455,12 @@ slora_status_t need_device(slora_pool* P) {
   return SLORA_OK;
 }
 
+// Whether a decode call of T tokens runs as one CTA per token (AUTO, 16-bit
+// weights, at most kTokenMaxT tokens: a latency-bound batch).
+bool token_path(const slora_pool* P, int T) {
+  return P->d.decode_path == SLORA_DECODE_AUTO && P->d.weight_format == SLORA_WEIGHTS_16 && T <= kTokenMaxT;
+}
+
 // Whether a decode call of T tokens runs as the one persistent kernel.
 bool fused_path(const slora_pool* P, int T) {
   if (T > kFMaxT) return false;
@@ -468,6 +477,12 @@ slora_status_t enqueue_delta(slora_pool* P, BgmvParams& bp, const int32_t* idx, 
   bp.do_expand = 1;
   if (P->e4m3() && !fused_path(P, T))
     return P->fail(SLORA_ERR_UNSUPPORTED, "e4m3 weights: decode calls of up to 1024 tokens on the one-kernel path");
+  if (token_path(P, T)) {
+    if (timed) phase(P, 0, 1, st);
+    CUDA_TRY(P, launch_token(bp, P->d.dtype, idx, T, st));
+    if (timed) phase(P, 1, 1, st);
+    return SLORA_OK;
+  }
   if (fused_path(P, T)) {
     const int grid = std::max(1, std::min(P->sm_count, fused_grid_bound(bp, T)));
     if (timed) phase(P, 0, 1, st);
@@ -1122,7 +1137,7 @@ slora_status_t slora_adapter_is_resident(const slora_pool* P, int32_t id, int32_
 
 int32_t slora_decode_kernels(const slora_pool* P, int32_t T) {
   if (!P || T <= 0) return 0;
-  return fused_path(P, T) ? 1 : 3;
+  return token_path(P, T) || fused_path(P, T) ? 1 : 3;
 }
 
 slora_status_t slora_check_batch(const slora_pool* Pc, const int32_t* idx_host, int32_t T) {
@@ -1283,6 +1298,38 @@ slora_status_t slora_sgmv(slora_pool* P, int32_t n, const int32_t* projs, const 
                               P->n_phase);
   if (e == cudaErrorNotSupported) return P->fail(SLORA_ERR_UNSUPPORTED, "SGMV shape not supported");
   if (e != cudaSuccess) return P->cuda_fail(e, "SGMV launch");
+  CUDA_TRY(P, record_epoch(P, st));
+  return SLORA_OK;
+}
+
+slora_status_t slora_sgmv_linear(slora_pool* P, int32_t n, const int32_t* projs, const void* const* x,
+                                 const int64_t* ldx, const void* const* w0, const int64_t* ldw, void* const* y,
+                                 const int64_t* ldy, const int32_t* seg_start, const int32_t* seg_adapter,
+                                 int32_t S, int32_t T, void* stream) {
+  NvtxRange nvtx_("slora_sgmv_linear");
+  if (!P) return SLORA_ERR_INVALID_ARG;
+  slora_status_t s = need_device(P);
+  if (s) return s;
+  if (P->e4m3()) return P->fail(SLORA_ERR_UNSUPPORTED, "slora_sgmv_linear takes 16-bit weights only");
+  if (P->d.max_rank > 64) return P->fail(SLORA_ERR_UNSUPPORTED, "slora_sgmv_linear: max_rank above 64");
+  if (S < 1 || !seg_start || !seg_adapter) return P->fail(SLORA_ERR_INVALID_ARG, "segments");
+  if (T < 1) return P->fail(SLORA_ERR_INVALID_ARG, "T must be positive");
+  BgmvParams bp;
+  base_params(P, bp);
+  s = plan_slots(P, bp, n, projs, x, ldx, y, ldy, T, true, true);
+  if (s) return s;
+  if (!w0 || !ldw) return P->fail(SLORA_ERR_INVALID_ARG, "w0 is NULL");
+  for (int k = 0; k < n; ++k)
+    if (!w0[k] || !aligned16(w0[k]) || ldw[k] < bp.slot[k].d_in || ldw[k] % 8)
+      return P->fail(SLORA_ERR_INVALID_ARG, "w0 must be 16-byte aligned with ldw >= d_in, ldw % 8 == 0");
+  if (S > P->d.max_tokens) return P->fail(SLORA_ERR_INVALID_ARG, "more segments than max_tokens");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  phase(P, 0, 1, st);
+  cudaError_t e = launch_linear(bp, P->d.dtype, w0, ldw, seg_start, seg_adapter, S, T, P->sm_count, st,
+                                P->scratch() + P->sl.off_sgmv, P->d.max_tokens, P->d.n_pages);
+  if (e == cudaErrorNotSupported) return P->fail(SLORA_ERR_UNSUPPORTED, "linear layer shape not supported");
+  if (e != cudaSuccess) return P->cuda_fail(e, "linear layer launch");
+  phase(P, 1, 1, st);
   CUDA_TRY(P, record_epoch(P, st));
   return SLORA_OK;
 }

@@ -29,13 +29,13 @@
 #include <cstring>
 #include <mutex>
 
-#include "slora_internal.h"
+#include "tc_common.cuh"
 
 namespace slora {
 
 namespace {
 
-constexpr int kBM = 128;             // tokens per tile (MMA M)
+using namespace tc;
 constexpr int kBK = 64;              // K per stage (one 128-byte swizzle atom)
 constexpr int kXTileBytes = kBM * kBK * 2;
 constexpr int kShrinkThreads = 192;  // X producer, MMA, 4 A-loader / epilogue warps
@@ -46,7 +46,6 @@ constexpr int kExpandThreads = 64 + 32 * kEpiWarps;  // producer, MMA, epilogue 
 constexpr int kEN = 128;             // expand outputs per item (MMA N)
 constexpr int kAcc = 4;              // expand TMEM accumulators (kAcc x kEN columns)
 constexpr int kYTileBytes = kBM * kEN * 2;
-constexpr long long kWaitLimitS = 2000000000ll;
 
 struct SgmvPlan {      // scratch arrays of one call
   int32_t* seg_start;  // [S] first token of each segment (0 when skipped)
@@ -85,146 +84,6 @@ struct SgmvParams {
   int e_t_half;         // expand: bytes of one t half in shared memory
   int e_b_stage;        // expand: bytes of one B ring stage
 };
-
-// ---------------------------------------------------------------------------
-// PTX helpers (tcgen05, TMA, mbarrier)
-__device__ __forceinline__ uint32_t su32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-__device__ __forceinline__ void bar_init(uint64_t* b, uint32_t n) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
-}
-__device__ __forceinline__ void bar_expect(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void rec_err(int32_t* err, int code, int info) {
-  if (atomicCAS(&err[0], 0, code) == 0) atomicExch(&err[1], info);
-}
-__device__ __forceinline__ bool bar_wait(uint64_t* b, uint32_t parity, int32_t* err) {
-  const uint32_t a = su32(b);
-  long long t0 = -1;
-  for (uint32_t it = 0;; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((it & 63) == 0) {
-      const long long now = clock64();
-      if (t0 < 0) t0 = now;
-      else if (now - t0 > kWaitLimitS) {
-        rec_err(err, 5, (int)blockIdx.x);
-        return false;
-      }
-    }
-  }
-}
-// L2 eviction-priority policies: streamed operands (X, y) go first, adapter
-// rows re-read by every token tile stay.
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ void tma_tile_2d_hint(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* b,
-                                                 uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(su32(dst)),
-      "l"(map), "r"(c0), "r"(c1), "r"(su32(b)), "l"(pol)
-      : "memory");
-}
-__device__ __forceinline__ void tma_gather4_hint(void* dst, const CUtensorMap* map, int r0, int r1, int r2, int r3,
-                                                 uint64_t* b, uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(su32(dst)),
-      "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(su32(b)), "l"(pol)
-      : "memory");
-}
-__device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w), "l"(pol)
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(slot)), "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* b) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(b))
-               : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void gd_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void gd_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle.  K-major: rows of 128 B,
-// 8-row atoms 1 KiB apart (SBO).  MN-major: atoms of 8 K-rows x 64 MN
-// elements; lbo = byte distance between MN-adjacent atoms, sbo = between
-// K-adjacent atom rows.
-__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFF);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-  return d;
-}
-// Instruction descriptor, kind::f16: fp32 accumulator, M = 128.
-__device__ __forceinline__ uint32_t idesc_f16(int dtype, int n, int b_mn_major) {
-  const uint32_t fmt = dtype == SLORA_BF16 ? 1u : 0u;
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(kBM >> 4) << 24);
-}
-
-__device__ __forceinline__ int find_ge(const int32_t* prefix, int S, int q) {  // largest s, prefix[s] <= q
-  int lo = 0, hi = S - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= q) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
-__device__ __forceinline__ int cdiv_d(int a, int b) { return (a + b - 1) / b; }
-
-// Pool row (64 elements) holding flat element f of tensor (adapter a, list offset lo).
-__device__ __forceinline__ int pool_row(const PoolDev& P, int a, int lo, int64_t f) {
-  const int32_t pg = __ldg(P.page_list + (int64_t)a * P.list_stride + lo + (f >> P.page_shift));
-  return (int)((((int64_t)pg << P.page_shift) + (f & ((1ll << P.page_shift) - 1))) >> 6);
-}
 
 // ---------------------------------------------------------------------------
 // Plan: validate segments, per-segment tile counts, prefix sums (one CTA).
@@ -493,34 +352,6 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   gd_launch();
 }
 
-
-// 16-bit <-> fp32 helpers for the expand epilogue (unpack exact; pack RN).
-template <int DT>
-__device__ __forceinline__ void up2(uint32_t w, float& lo, float& hi) {
-  if (DT == SLORA_BF16) {
-    lo = __uint_as_float(w << 16);
-    hi = __uint_as_float(w & 0xffff0000u);
-  } else {
-    asm("{.reg .f16 l, h, one;\n\tmov.b32 {l, h}, %2;\n\tmov.b16 one, 0x3C00;\n\t"
-        "fma.rn.f32.f16 %0, l, one, 0f80000000;\n\tfma.rn.f32.f16 %1, h, one, 0f80000000;}"
-        : "=f"(lo), "=f"(hi) : "r"(w));
-  }
-}
-template <int DT>
-__device__ __forceinline__ uint32_t pk2(float lo, float hi) {
-  uint32_t r;
-  if (DT == SLORA_BF16) asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  else asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-// t = hi + lo in 16-bit halves (hi = RN(t), lo = RN(t - hi)).
-template <int DT>
-__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  hi = pk2<DT>(a, b);
-  float ha, hb;
-  up2<DT>(hi, ha, hb);
-  lo = pk2<DT>(a - ha, b - hb);
-}
 
 // ---------------------------------------------------------------------------
 // Expand: persistent CTAs (one per SM) over the item sequence
@@ -898,38 +729,6 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
 
 // ---------------------------------------------------------------------------
 // Host side.
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  });
-  return fn;
-}
-
-bool encode_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-               uint32_t box_inner, uint32_t box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, dtype == SLORA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                        2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 int round16(int v) { return (v + 15) & ~15; }
 
 template <typename Kern>

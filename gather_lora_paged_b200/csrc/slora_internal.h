@@ -138,6 +138,9 @@ cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s);
 // The one-kernel decode delta (fused.cu): T <= kFMaxT, both phases.
 cudaError_t launch_fused(BgmvParams& p, int dtype, const int32_t* idx, int T, int grid, cudaStream_t s);
 int fused_grid_bound(const BgmvParams& p, int T);  // CTAs worth launching for T tokens
+// The small-batch decode delta (token.cu): one CTA per token, no scratch.
+constexpr int kTokenMaxT = 16;
+cudaError_t launch_token(const BgmvParams& p, int dtype, const int32_t* idx, int T, cudaStream_t s);
 cudaError_t launch_merge_requests(const int32_t* req_start, const int32_t* req_adapter, int n,
                                   int32_t* seg_start, int32_t* seg_adapter, int32_t* S_out,
                                   cudaStream_t s);

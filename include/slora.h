@@ -95,10 +95,12 @@ typedef enum {
  * slice order, one rounding of y); they differ in launches and scheduling.
  * slora_decode_kernels() tells which one a call takes. */
 typedef enum {
-  SLORA_DECODE_AUTO = 0,       /* the library's choice: the one-kernel path for
-                                  e4m3 pools, the three-kernel path for 16-bit
-                                  pools (the faster one on B200 at the shapes
-                                  measured so far)                              */
+  SLORA_DECODE_AUTO = 0,       /* the library's choice: 16-bit pools run calls of
+                                  up to 16 tokens as one CTA per token (plain
+                                  loads, no scratch: a latency-bound batch) and
+                                  larger calls on the three-kernel path (the
+                                  faster one on B200 at the shapes measured so
+                                  far); e4m3 pools take the one-kernel path    */
   SLORA_DECODE_SPLIT = 1,      /* always three kernels: segment build, shrink,
                                   expand                                         */
   SLORA_DECODE_FUSED = 2       /* one persistent kernel for calls of up to 1024
@@ -390,6 +392,30 @@ slora_status_t slora_sgmv(slora_pool* pool, int32_t n, const int32_t* projs,
                           const int64_t* ldy, const int32_t* seg_start,
                           const int32_t* seg_adapter, int32_t S, int32_t T, void* stream);
 
+/* The whole linear layer with its LoRA delta, for prefill segments, in one
+ * tensor-core kernel:
+ *     y[i, :] = x[i, :] . W0 + (alpha_a / r_a) (x[i, :] . A_a) . B_a
+ * for the tokens i of a segment whose adapter is a, and y[i, :] = x[i, :] . W0
+ * for a segment without one (seg_adapter -1).  y is written, not accumulated.
+ * [S2 SGMV section: Y = X.W0 + (alpha/r).((X.A).B); metrics section: the delta
+ * fused into the linear layer's output]
+ * Per projection k: x[k] (T x d_in, ldx), w0[k] (d_out rows of d_in: the
+ * layout of a linear layer's weight, leading dimension ldw[k] >= d_in, a
+ * multiple of 8, 16-byte aligned), y[k] (T x d_out, ldy).  seg_start (S + 1)
+ * and seg_adapter (S) are device arrays; the segments must cover [0, T) in
+ * order (seg_start[0] = 0, seg_start[S] = T), checked on the device (code 6,
+ * info = segment; a bad adapter: codes 1, 2, and the segment gets the base map
+ * only).  The shrink X.A is computed in the same K loop as X.W0 (the A rows as
+ * extra output columns), t enters the tensor cores as two 16-bit halves, and
+ * t.B is accumulated into X.W0's accumulator before y is stored once.
+ * Errors: INVALID_ARG (also S < 1, T < 1); UNSUPPORTED for max_rank > 64 and
+ * for e4m3 pools.                                                             */
+slora_status_t slora_sgmv_linear(slora_pool* pool, int32_t n, const int32_t* projs,
+                                 const void* const* x, const int64_t* ldx, const void* const* w0,
+                                 const int64_t* ldw, void* const* y, const int64_t* ldy,
+                                 const int32_t* seg_start, const int32_t* seg_adapter, int32_t S,
+                                 int32_t T, void* stream);
+
 /* The decode delta of slora_lora_delta, for callers that cannot allocate
  * device memory at the point of the call: a plug-in whose host framework owns
  * every device allocation and hands it only inputs and outputs, or a serving
@@ -420,8 +446,8 @@ slora_status_t slora_lora_delta_noalloc(slora_pool* pool, int32_t n, const int32
                                         int32_t T, void* stream);
 
 /* Number of kernels slora_lora_delta launches for a call of T tokens on this
- * pool (1: the one-kernel path, 3: segment build, shrink, expand); 0 for T <= 0
- * or a NULL pool.  Host only. */
+ * pool (1: the one-kernel path or one CTA per token, 3: segment build,
+ * shrink, expand); 0 for T <= 0 or a NULL pool.  Host only. */
 int32_t slora_decode_kernels(const slora_pool* pool, int32_t T);
 
 /* Size in bytes of the fixed scratch array used by slora_lora_delta_noalloc. */

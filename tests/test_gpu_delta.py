@@ -128,6 +128,28 @@ def test_unfused_shrink_expand():
     pb.close()
 
 
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_small_batch_token_path(T):
+    """Batches of up to 16 tokens run as one CTA per token on 16-bit pools
+    (the default path): ranks up to 128, rank 0, tokens without adapter and
+    tokens sharing one, projections sharing x, rows across 512-element pages;
+    every element against the oracle at the tight bound."""
+    import torch
+    rng = np.random.default_rng(300 + T)
+    projs = [W.Proj("q", 1088, 2112, "a"), W.Proj("k", 1088, 192, "a"), W.Proj("d", 3136, 1024, "c")]
+    ranks = [8, 128, 0, 24, 3]
+    idx = rng.integers(-1, len(ranks), T).astype(np.int32)
+    if T > 2:
+        idx[1] = idx[0] = 1                      # two tokens on the rank-128 adapter
+    w = _custom(W.BF16, projs, ranks, idx, page_elems=512)
+    pb = H.PoolBuild(w)
+    assert G.slora_decode_kernels(pb.h, T) == 1
+    ten = H.Tensors(w)
+    _run_delta(pb, ten, w)
+    _check_all(w, ten, tight=True)
+    pb.close()
+
+
 def test_degenerate_batches():
     import torch
     projs = [W.Proj("q", 1024, 1024, "a")]

@@ -8,6 +8,8 @@ Value recipe (the pages publish no datasets for this op; these stand in for
 the serving traces the pages evaluate on):
   * x ~ N(0, 1), y_in ~ N(0, 1) (y_in stands for the base output X.W0);
   * A ~ N(0, std = 1/sqrt(d_in)), B ~ N(0, std = 1/sqrt(r)), alpha = 16;
+  * the base weight of a projection (for the whole linear layer) W0 ~
+    N(0, std = 1/sqrt(d_in)), stored as d_out rows of d_in;
   * values are drawn in fp32 and rounded to nearest-even into fp16 or bf16;
   * adapter per token: uniform (the tiny case) or a finite Zipf law
     P(id = j) ~ (j + 1)^(-s) over j in [0, N), drawn by inverse CDF.
@@ -30,7 +32,7 @@ DTYPE_NAME = {F16: "f16", BF16: "bf16"}
 ALPHA = 16.0
 
 # stream tags
-_T_IDX, _T_RANK, _T_X, _T_Y, _T_AD, _T_FILL, _T_REQ, _T_COLD = range(8)
+_T_IDX, _T_RANK, _T_X, _T_Y, _T_AD, _T_FILL, _T_REQ, _T_COLD, _T_W0 = range(9)
 
 
 def _rng(*key):
@@ -129,6 +131,17 @@ class Workload:
         if key not in self._cache:
             self._cache[key] = normal_bits(_rng(self.seed, _T_Y, p),
                                            (self.T, self.projs[p].d_out), 1.0, self.dtype)
+        return self._cache[key]
+
+    def w0(self, p: int) -> np.ndarray:
+        """The base weight of projection p as a linear layer stores it: d_out
+        rows of d_in, N(0, std = 1/sqrt(d_in)) (random-init stand-in for the
+        model's weight)."""
+        key = ("w0", p)
+        if key not in self._cache:
+            pr = self.projs[p]
+            self._cache[key] = normal_bits(_rng(self.seed, _T_W0, p), (pr.d_out, pr.d_in),
+                                           1.0 / np.sqrt(pr.d_in), self.dtype)
         return self._cache[key]
 
     def _draw_adapter(self, key_rng, r):
