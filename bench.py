@@ -229,7 +229,8 @@ class DecodeRun:
         import harness as H
         self.G, self.H, self.w = G, H, w
         self.wbytes = 1 if weights == "e4m3" else 2
-        dp = {"auto": G.SLORA_DECODE_AUTO, "split": G.SLORA_DECODE_SPLIT, "fused": G.SLORA_DECODE_FUSED}[path]
+        dp = {"auto": G.SLORA_DECODE_AUTO, "split": G.SLORA_DECODE_SPLIT, "fused": G.SLORA_DECODE_FUSED,
+              "stream": G.SLORA_DECODE_STREAM}[path]
         self.pb = H.PoolBuild(w, decode_path=dp,
                               weight_format=G.SLORA_WEIGHTS_E4M3 if weights == "e4m3" else G.SLORA_WEIGHTS_16)
         fused = G.slora_decode_kernels(self.pb.h, w.T) == 1
@@ -834,7 +835,7 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--path", default="auto", choices=["auto", "split", "fused"],
+    ap.add_argument("--path", default="auto", choices=["auto", "split", "fused", "stream"],
                     help="decode kernels: the library's choice, the three-kernel path (segment "
                          "build, shrink, expand) or the one persistent kernel")
     ap.add_argument("--linear", action="store_true",

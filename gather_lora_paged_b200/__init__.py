@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "libslora.so")
 
 SLORA_F16, SLORA_BF16 = 0, 1
 SLORA_PAGEIN_KERNEL, SLORA_PAGEIN_MEMCPY = 0, 1
-SLORA_DECODE_AUTO, SLORA_DECODE_SPLIT, SLORA_DECODE_FUSED = 0, 1, 2
+SLORA_DECODE_AUTO, SLORA_DECODE_SPLIT, SLORA_DECODE_FUSED, SLORA_DECODE_STREAM = 0, 1, 2, 3
 SLORA_WEIGHTS_16, SLORA_WEIGHTS_E4M3 = 0, 1
 MAX_PROJ = 8
 

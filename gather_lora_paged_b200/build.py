@@ -26,7 +26,7 @@ def _stale():
     if not os.path.exists(OUT):
         return True
     deps = sources() + glob.glob(os.path.join(HERE, "csrc", "*.h")) + \
-        [os.path.join(ROOT, "include", "slora.h")]
+        glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + [os.path.join(ROOT, "include", "slora.h")]
     t = os.path.getmtime(OUT)
     return any(os.path.getmtime(d) > t for d in deps)
 

@@ -224,7 +224,7 @@ struct slora_pool {
   int64_t n_rel = 0;                  // release events recorded so far
   PoolDev pd{};
   int sm_count = 148;
-  int grid_shrink = 0, grid_expand = 0;
+  int grid_shrink = 0, grid_expand = 0, grid_stream = 0;
   int inject_after = -1;
   cudaEvent_t phase_ev[8] = {};
   int n_phase = 0;
@@ -283,7 +283,7 @@ slora_status_t validate_desc(const slora_pool_desc* d, std::string* why) {
   if (d->n_pages < 0 || d->n_pages > (int64_t)INT32_MAX) return bad("n_pages out of range");
   if (d->pagein_mode != SLORA_PAGEIN_KERNEL && d->pagein_mode != SLORA_PAGEIN_MEMCPY)
     return bad("pagein_mode");
-  if (d->decode_path < SLORA_DECODE_AUTO || d->decode_path > SLORA_DECODE_FUSED) return bad("decode_path");
+  if (d->decode_path < SLORA_DECODE_AUTO || d->decode_path > SLORA_DECODE_STREAM) return bad("decode_path");
   if (d->weight_format != SLORA_WEIGHTS_16 && d->weight_format != SLORA_WEIGHTS_E4M3) return bad("weight_format");
   if (!d->host_only) {
     if (!d->dev_pool && d->n_pages > 0) return bad("dev_pool is NULL");
@@ -463,9 +463,14 @@ bool token_path(const slora_pool* P, int T) {
 
 // Whether a decode call of T tokens runs as the one persistent kernel.
 bool fused_path(const slora_pool* P, int T) {
+  return T <= kFMaxT && P->d.decode_path == SLORA_DECODE_FUSED;
+}
+
+// Whether a decode call of T tokens runs as the one kernel of streaming tasks.
+bool stream_path(const slora_pool* P, int T) {
   if (T > kFMaxT) return false;
-  if (P->d.decode_path == SLORA_DECODE_FUSED) return true;
-  return P->d.decode_path == SLORA_DECODE_AUTO && P->d.weight_format == SLORA_WEIGHTS_E4M3;
+  if (P->d.decode_path == SLORA_DECODE_STREAM) return true;
+  return P->d.decode_path == SLORA_DECODE_AUTO && !token_path(P, T);
 }
 
 // The decode delta's kernels for a planned call (both phases): the one
@@ -475,11 +480,17 @@ slora_status_t enqueue_delta(slora_pool* P, BgmvParams& bp, const int32_t* idx, 
                              bool timed) {
   bp.do_shrink = 1;
   bp.do_expand = 1;
-  if (P->e4m3() && !fused_path(P, T))
-    return P->fail(SLORA_ERR_UNSUPPORTED, "e4m3 weights: decode calls of up to 1024 tokens on the one-kernel path");
+  if (P->e4m3() && !fused_path(P, T) && !stream_path(P, T))
+    return P->fail(SLORA_ERR_UNSUPPORTED, "e4m3 weights: decode calls of up to 1024 tokens on a one-kernel path");
   if (token_path(P, T)) {
     if (timed) phase(P, 0, 1, st);
     CUDA_TRY(P, launch_token(bp, P->d.dtype, idx, T, st));
+    if (timed) phase(P, 1, 1, st);
+    return SLORA_OK;
+  }
+  if (stream_path(P, T)) {
+    if (timed) phase(P, 0, 1, st);
+    CUDA_TRY(P, launch_stream(bp, P->d.dtype, idx, T, P->grid_stream, st));
     if (timed) phase(P, 1, 1, st);
     return SLORA_OK;
   }
@@ -617,6 +628,7 @@ slora_status_t slora_pool_create(const slora_pool_desc* desc, slora_pool** out) 
     }
     P->grid_shrink = P->sm_count * occupancy_blocks(0);
     P->grid_expand = P->sm_count * occupancy_blocks(1);
+    P->grid_stream = P->sm_count * stream_blocks_per_sm(P->d.max_adapters);
   }
   *out = P;
   return SLORA_OK;
@@ -1137,7 +1149,7 @@ slora_status_t slora_adapter_is_resident(const slora_pool* P, int32_t id, int32_
 
 int32_t slora_decode_kernels(const slora_pool* P, int32_t T) {
   if (!P || T <= 0) return 0;
-  return token_path(P, T) || fused_path(P, T) ? 1 : 3;
+  return token_path(P, T) || fused_path(P, T) || stream_path(P, T) ? 1 : 3;
 }
 
 slora_status_t slora_check_batch(const slora_pool* Pc, const int32_t* idx_host, int32_t T) {

@@ -138,6 +138,10 @@ cudaError_t launch_reduce_t(const BgmvParams& p, int T, cudaStream_t s);
 // The one-kernel decode delta (fused.cu): T <= kFMaxT, both phases.
 cudaError_t launch_fused(BgmvParams& p, int dtype, const int32_t* idx, int T, int grid, cudaStream_t s);
 int fused_grid_bound(const BgmvParams& p, int T);  // CTAs worth launching for T tokens
+// The decode delta as one kernel of streaming tasks (stream.cu): T <= kFMaxT,
+// both phases; grid = SMs x stream_blocks_per_sm (any size works).
+cudaError_t launch_stream(BgmvParams& p, int dtype, const int32_t* idx, int T, int grid, cudaStream_t s);
+int stream_blocks_per_sm(int max_adapters);
 // The small-batch decode delta (token.cu): one CTA per token, no scratch.
 constexpr int kTokenMaxT = 16;
 cudaError_t launch_token(const BgmvParams& p, int dtype, const int32_t* idx, int T, cudaStream_t s);

@@ -1,0 +1,733 @@
+// stream.cu -- the decode delta as one kernel of streaming stages (sm_100a).
+//
+// Every CTA plans the call on its own: a stable counting sort of the batch's
+// tokens by adapter gives the segments (one per adapter with tokens: "Multi-
+// LoRA serving: S-LoRA, Punica, SGMV, vLLM", SGMV section, and "Paper
+// explainer: S-LoRA", BGMV kernel section: tokens of one batch use different
+// adapters, fetched from paged memory by id) and each segment's task counts.
+// CTA b then takes an equal share of the shrink tasks and, after them, an
+// equal share (by stages) of the expand tasks:
+//
+//   shrink (segment, x group, 8 rank rows, 2048 of d_in, up to 8 tokens):
+//       t_c[i, k] = sum_{j in chunk c} x[i, j] * A_a[j, k]
+//     The 8 rows arrive in shared memory by bulk copies (one per page piece
+//     of a row).  The 8 consumer warps split the chunk: lane l reads 8
+//     consecutive elements of row l / 4 and the same 8 columns of the x row
+//     of token l / 4, and the warp multiplies them on the tensor cores
+//     (mma.sync m16n8k16, fp32 accumulate).  Inside a 32-column step the
+//     contraction order is permuted in the same way for both operands, which
+//     is what lets 16-byte reads fill the fragments directly.  The warps'
+//     sums are added in warp order; chunk c of d_in leaves partial t_c.
+//   expand (segment, projection, 2048 outputs, up to 4 tokens), as stages of
+//   8 rank rows:
+//       y[i, l] <- RN(y[i, l] + (alpha_a / r_a) * sum_k t[i, k] * B_a[k, l]),
+//       t[i, k] = sum_c t_c[i, k] (chunk order)
+//     Lane l owns 8 consecutive outputs and accumulates on the FMA pipe in
+//     fp32, rank rows in order, then rounds y once.
+//
+// A producer warp walks the CTA's stages: page ids one stage ahead, the bulk
+// copies of the next stage into the other of two slots (a full / empty
+// mbarrier pair each), L2 prefetches of the x and y rows the consumers will
+// read.  The phases meet at one grid barrier (cooperative launch): expand
+// stages read the t partials of every CTA.  The last CTA to finish clears the
+// barrier count.  e4m3 pages: codes are widened exactly (every e4m3 value is
+// a 16-bit value of either type), and the per-rank-row scales multiply the
+// partials of A and the t entering the expand.
+#include "dev_common.cuh"
+
+namespace slora {
+
+namespace {
+
+constexpr int kQThreads = 256;                // 8 warps
+constexpr int kQWarps = kQThreads / 32;
+constexpr int kQRB = 8;                       // rank rows per shrink task (the mma's N)
+constexpr int kQKT = kPartK;                  // d_in per shrink task: 256 per warp
+constexpr int kQSTok = 8;                     // tokens per shrink task (mma rows 0..7)
+constexpr int kQECols = 2048;                 // outputs per expand task: 256 per warp
+constexpr int kQETok = 4;                     // tokens per expand task
+constexpr int kQMaxR = 128;
+static_assert(kQKT == kQWarps * 256 && kQECols == kQWarps * 256, "task shapes");
+constexpr int kQBar = kFReadyCap + 1;         // ready[]: finished CTAs at kFReadyCap, then the phase barrier
+
+// The call's plan, identical in every CTA.
+struct QPlan {
+  int S;
+  int seg_start[kFSegCap + 1];  // positions in perm order
+  int seg_adapter[kFSegCap];
+  int seg_rank[kFSegCap];
+  int shr_pre[kFSegCap + 1];    // shrink tasks before each segment
+  int exp_pre[kFSegCap + 1];    // expand tasks before each segment
+  int exp_spre[kFSegCap + 1];   // expand stages before each segment (ceil(r / 8) per task)
+  int perm[kFMaxT];             // token of each position
+};
+
+// Reads of data written earlier in this kernel by other CTAs (L2, not L1).
+__device__ __forceinline__ float ld_cg_f32(const float* p) {
+  float v;
+  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_acquire_s32(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+template <int DT>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  if (DT == SLORA_BF16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// e4m3 pair -> 16-bit pair of type DT, exactly.
+template <int DT>
+__device__ __forceinline__ uint32_t e4m3x2_to_16(uint32_t two) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((unsigned short)two));
+  if (DT == SLORA_F16) return h;
+  float lo, hi;
+  h2x2f(h, lo, hi);
+  return pack2<SLORA_BF16>(lo, hi);
+}
+__device__ __forceinline__ void unpack8_q8(const uint2& v, float* f) {
+  const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    h2x2f(e4m3x2_to_16<SLORA_F16>(w[i] & 0xffffu), f[4 * i], f[4 * i + 1]);
+    h2x2f(e4m3x2_to_16<SLORA_F16>(w[i] >> 16), f[4 * i + 2], f[4 * i + 3]);
+  }
+}
+
+__device__ __forceinline__ int shrink_tasks(const BgmvParams& p, int n, int r) {
+  int c = 0;
+  const int ntt = cdiv_i(n, kQSTok);
+  for (int g = 0; g < p.n_groups; ++g)
+    c += cdiv_i(p.group[g].n * r, kQRB) * cdiv_i(p.group[g].d_in, kQKT) * ntt;
+  return c;
+}
+__device__ __forceinline__ int expand_tasks(const BgmvParams& p, int n) {
+  int c = 0;
+  const int ntg = cdiv_i(n, kQETok);
+  for (int k = 0; k < p.n_slots; ++k) c += cdiv_i(p.slot[k].d_out, kQECols) * ntg;
+  return c;
+}
+
+// ---------------------------------------------------------------------------
+// The plan: histogram over adapter ids (count | rank << 21), segments in
+// adapter order, stable scatter of the tokens into perm.  Invalid tokens are
+// reported by CTA 0 and, like rank-0 adapters and id -1, leave y unchanged.
+constexpr int kRankShift = 21;
+
+__device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int4* sh4, int* sh1) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool worker = tid < kQThreads;  // token work: the first kQThreads threads
+  const int T = p.T, MA = p.pool.max_adapters;
+  for (int a = tid; a < MA; a += blockDim.x) hist[a] = 0;
+  __syncthreads();
+  int key[kFMaxT / kQThreads];
+#pragma unroll
+  for (int u = 0; u < kFMaxT / kQThreads; ++u) {
+    const int i = tid + u * kQThreads;
+    int a = -1;
+    if (worker && i < T) {
+      a = p.idx[i];
+      if (a < -1 || a >= MA) {
+        if (blockIdx.x == 0) record_error(p.pool.err, 1, i);
+        a = -1;
+      } else if (a >= 0) {
+        const int r = p.pool.rank[a];
+        if (r < 0 && blockIdx.x == 0) record_error(p.pool.err, 2, i);
+        if (r <= 0) {
+          a = -1;
+        } else {
+          atomicOr(&hist[a], r << kRankShift);
+          atomicAdd(&hist[a], 1);
+        }
+      }
+    }
+    key[u] = a;
+  }
+  __syncthreads();
+  // each worker owns a contiguous adapter range; its segments are contiguous
+  const int E = cdiv_i(MA, kQThreads);
+  const int a0 = worker ? min(tid * E, MA) : MA, a1 = min(a0 + E, MA);
+  int4 c = make_int4(0, 0, 0, 0);  // tokens, segments, shrink tasks, expand tasks
+  int cs = 0;                      // expand stages
+  for (int a = a0; a < a1; ++a) {
+    const int h = hist[a];
+    if (h == 0) continue;
+    const int n = h & ((1 << kRankShift) - 1), r = h >> kRankShift;
+    const int ne = expand_tasks(p, n);
+    c.x += n;
+    c.y += 1;
+    c.z += shrink_tasks(p, n, r);
+    c.w += ne;
+    cs += ne * cdiv_i(r, 8);
+  }
+  int4 tot;
+  const int4 base = block_exscan4(c, &tot, sh4);
+  int tot_s;
+  int bst = block_exscan<false>(cs, &tot_s, sh1);
+  int cb = base.x, sb = base.y, bs = base.z, be = base.w;
+  for (int a = a0; a < a1; ++a) {
+    const int h = hist[a];
+    hist[a] = cb;  // becomes the scatter cursor
+    if (h == 0) continue;
+    const int n = h & ((1 << kRankShift) - 1), r = h >> kRankShift;
+    const int ne = expand_tasks(p, n);
+    P.seg_start[sb] = cb;
+    P.seg_adapter[sb] = a;
+    P.seg_rank[sb] = r;
+    P.shr_pre[sb] = bs;
+    P.exp_pre[sb] = be;
+    P.exp_spre[sb] = bst;
+    ++sb;
+    cb += n;
+    bs += shrink_tasks(p, n, r);
+    be += ne;
+    bst += ne * cdiv_i(r, 8);
+  }
+  if (tid == 0) {
+    P.S = tot.y;
+    P.seg_start[tot.y] = tot.x;
+    P.shr_pre[tot.y] = tot.z;
+    P.exp_pre[tot.y] = tot.w;
+    P.exp_spre[tot.y] = tot_s;
+  }
+  __syncthreads();
+  // Stable scatter, one chunk of kQThreads tokens at a time: a token's place
+  // among its adapter's tokens of the chunk is the number of equal keys in
+  // earlier warps plus the number in earlier lanes of its own warp.
+#pragma unroll
+  for (int u = 0; u < kFMaxT / kQThreads; ++u) {
+    if (u * kQThreads >= T) break;
+    const int a = key[u];
+    if (worker) ck[tid] = a;
+    __syncthreads();
+    const unsigned m = __match_any_sync(FULL_MASK, a);
+    if (a >= 0) {
+      int before = __popc(m & ((1u << lane) - 1));
+      const int4* k4 = reinterpret_cast<const int4*>(ck);
+      for (int j = 0; j < warp * 8; ++j) {
+        const int4 v = k4[j];
+        before += (v.x == a) + (v.y == a) + (v.z == a) + (v.w == a);
+      }
+      P.perm[hist[a] + before] = tid + u * kQThreads;
+    }
+    __syncthreads();  // every cursor read before the chunk's counts are added
+    if (a >= 0 && lane == __ffs(m) - 1) atomicAdd(&hist[a], __popc(m));
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// A task, decoded from its index: shrink (segment s, x group u, rank-row
+// block v, d_in chunk c, token tile w) or expand (segment s, slot u, output
+// chunk v, token group w).  An expand task runs as ceil(r / 8) stages of 8
+// rank rows (sub = 0, 1, ...), a shrink task as one stage.
+struct QTask {
+  int shrink;  // 1: shrink, 0: expand, -1: none (the end of the CTA's stages)
+  int s, u, v, c, w;
+  int sub;
+};
+
+__device__ __forceinline__ QTask decode_task(const BgmvParams& p, const QPlan& P, int task, int n_shr, int total) {
+  QTask t{-1, 0, 0, 0, 0, 0, 0};
+  if (task >= total) return t;
+  const int S = P.S;
+  if (task < n_shr) {
+    const int s = find_seg(P.shr_pre, S, task);
+    int q = task - P.shr_pre[s];
+    const int n = P.seg_start[s + 1] - P.seg_start[s], r = P.seg_rank[s], ntt = cdiv_i(n, kQSTok);
+    int g = 0;
+    for (; g < p.n_groups - 1; ++g) {
+      const int cnt = cdiv_i(p.group[g].n * r, kQRB) * cdiv_i(p.group[g].d_in, kQKT) * ntt;
+      if (q < cnt) break;
+      q -= cnt;
+    }
+    const int nb = cdiv_i(p.group[g].n * r, kQRB);
+    const int c = q / (nb * ntt), rem = q - c * nb * ntt;
+    t = QTask{1, s, g, rem / ntt, c, rem % ntt, 0};
+  } else {
+    const int te = task - n_shr;
+    const int s = find_seg(P.exp_pre, S, te);
+    int q = te - P.exp_pre[s];
+    const int n = P.seg_start[s + 1] - P.seg_start[s], ntg = cdiv_i(n, kQETok);
+    int ks = 0;
+    for (; ks < p.n_slots - 1; ++ks) {
+      const int cnt = cdiv_i(p.slot[ks].d_out, kQECols) * ntg;
+      if (q < cnt) break;
+      q -= cnt;
+    }
+    t = QTask{0, s, ks, q / ntg, 0, q % ntg, 0};
+  }
+  return t;
+}
+
+// Stage slots: 8 rows (rank rows of the stage) of 2048 elements each, rows
+// 4160 bytes apart: the 64-byte pad puts the 8 rows a lane quad reads in
+// distinct bank groups.  Stage bytes land by bulk copies (one per page piece
+// of a row), counted on the slot's `full` mbarrier.
+constexpr int kQRowBytes = 2 * kQKT + 64;
+constexpr int kQSlotBytes = kQRB * kQRowBytes;
+constexpr int kQCons = 8;                          // consumer warps
+constexpr int kQAll = (kQCons + 1) * 32;           // + the producer warp
+static_assert(kQCons * 32 == kQThreads, "consumers");
+
+__device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, %0;" ::"n"(kQThreads) : "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// The 8 rows of a stage: weight tensor page list, first element f0 of row 0,
+// element stride between rows, row length L (elements), rows present.
+struct QRows {
+  const int32_t* list[kQRB];
+  int64_t f0[kQRB];
+  int L, nrows;
+};
+
+__device__ __forceinline__ void stage_rows(const BgmvParams& p, const QPlan& P, const QTask& t, int i,
+                                           const int32_t*& list, int64_t& f0, int& L, bool& ok) {
+  const int a = P.seg_adapter[t.s], r = P.seg_rank[t.s];
+  const int32_t* row = p.pool.page_list + (int64_t)a * p.pool.list_stride;
+  ok = false;
+  if (t.shrink > 0) {
+    const GroupDev& G = p.group[t.u];
+    const int rho = t.v * kQRB + i;
+    L = min(kQKT, G.d_in - t.c * kQKT);
+    if (rho < G.n * r) {
+      const int js = rho / r, k = rho - js * r;
+      list = row + p.slot[G.slot[js]].listA;
+      f0 = (int64_t)k * G.d_in + t.c * kQKT;
+      ok = true;
+    }
+  } else if (t.shrink == 0) {
+    const SlotDev& S = p.slot[t.u];
+    const int k = t.sub * kQRB + i;
+    L = min(kQECols, S.d_out - t.v * kQECols);
+    if (k < r) {
+      list = row + S.listB;
+      f0 = (int64_t)k * S.d_out + t.v * kQECols;
+      ok = true;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Shrink stage (segment s, x group g, rank-row block b, d_in chunk c, token
+// tile of up to 8 tokens).  Lane l reads rank row l / 4 of the stage (zero
+// past the group's rows) and token l / 4 of the tile (zero past the segment).
+template <int DT, int WF>
+__device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, const QTask& t,
+                             const unsigned char* slot) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, q = lane & 3, gr = lane >> 2;
+  const int s = t.s, g = t.u, b = t.v, c = t.c;
+  const int a = P.seg_adapter[s], r = P.seg_rank[s];
+  const int pos0 = P.seg_start[s] + t.w * kQSTok;
+  const int nt = min(kQSTok, P.seg_start[s + 1] - pos0);
+  const GroupDev& G = p.group[g];
+  const int d_in = G.d_in, nrows = G.n * r;
+  const bool rv = b * kQRB + gr < nrows, xv = gr < nt;
+  const int j0 = w * 256 + q * 8;  // in the chunk; step u adds 32
+  const int jw = c * kQKT + j0;
+  const uint16_t* xr = G.x + (int64_t)P.perm[pos0 + min(gr, nt - 1)] * G.ldx;
+  uint4 xc[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) xc[u] = __ldg(reinterpret_cast<const uint4*>(xr + min(jw + 32 * u, d_in - 8)));
+  const unsigned char* arow = slot + gr * kQRowBytes;
+  float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // two chains: steps u even / odd
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    float (&acc)[4] = acc2[u & 1];
+    const bool in = jw + 32 * u < d_in;
+    const uint4 xu = (xv && in) ? xc[u] : make_uint4(0, 0, 0, 0);
+    uint32_t bw[4] = {0u, 0u, 0u, 0u};
+    if (rv && in) {
+      if (WF == 0) {
+        const uint4 v = *reinterpret_cast<const uint4*>(arow + 2 * (j0 + 32 * u));
+        bw[0] = v.x; bw[1] = v.y; bw[2] = v.z; bw[3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(arow + (j0 + 32 * u));
+        bw[0] = e4m3x2_to_16<DT>(v.x & 0xffffu);
+        bw[1] = e4m3x2_to_16<DT>(v.x >> 16);
+        bw[2] = e4m3x2_to_16<DT>(v.y & 0xffffu);
+        bw[3] = e4m3x2_to_16<DT>(v.y >> 16);
+      }
+    }
+    // contraction slots 2q, 2q+1 <- elements 0, 1; 2q+8, 2q+9 <- 2, 3 (then
+    // 4..7); mma rows 8..15 (no tokens) stay zero
+    mma16816<DT>(acc, xu.x, 0u, xu.y, 0u, bw[0], bw[1]);
+    mma16816<DT>(acc, xu.z, 0u, xu.w, 0u, bw[2], bw[3]);
+  }
+  // warp partials: red[w][token][row]; D row gr, columns 2q, 2q + 1
+  red[w * 64 + gr * 8 + 2 * q] = acc2[0][0] + acc2[1][0];
+  red[w * 64 + gr * 8 + 2 * q + 1] = acc2[0][1] + acc2[1][1];
+  bar_consumers();
+  if (tid < 64) {
+    const int m = tid >> 3, nn = tid & 7, row = b * kQRB + nn;
+    if (m < nt && row < nrows) {
+      float sum = red[tid];
+#pragma unroll
+      for (int w2 = 1; w2 < kQCons; ++w2) sum += red[w2 * 64 + tid];
+      const int j2 = row / r, k2 = row - j2 * r;
+      const SlotDev& S2 = p.slot[G.slot[j2]];
+      if (WF == 1) sum *= p.pool.qscale[(((int64_t)a * p.pool.n_proj + S2.proj) * 2) * p.pool.max_rank + k2];
+      S2.t[(int64_t)(pos0 + m) * S2.t_rs + (int64_t)k2 * S2.t_ns + c] = sum;
+    }
+  }
+  bar_consumers();  // red is rewritten by the next shrink stage
+}
+
+// ---------------------------------------------------------------------------
+// Expand stage: rank rows 8 sub .. 8 sub + 7 of task (segment s, slot ks,
+// output chunk e, token group tg).  The first stage fills tS with t = sum of
+// the chunk partials (every shrink task has finished: the phases are split by
+// a grid barrier); the last one adds s_a * acc to y (prefetched to L2 by the
+// producer) and rounds.
+template <int DT, int WF, int NT>
+__device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, const QTask& t,
+                             const unsigned char* slot, float (&acc)[kQETok][8]) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int s = t.s, a = P.seg_adapter[s], r = P.seg_rank[s];
+  const int pos0 = P.seg_start[s] + t.w * kQETok;
+  const int nt = min(kQETok, P.seg_start[s + 1] - pos0);
+  const SlotDev& L = p.slot[t.u];
+  const int jl = w * 256 + lane * 8;  // in the chunk
+  const int col = t.v * kQECols + jl;
+  const bool act = col < L.d_out;
+  if (t.sub == 0) {
+#pragma unroll
+    for (int m = 0; m < NT; ++m)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
+    bar_consumers();  // the previous expand task's reads of tS are done
+    for (int v = tid; v < nt * r; v += kQThreads) {
+      const int m = v / r, kk = v - m * r;
+      const float* src = L.t + (int64_t)(pos0 + m) * L.t_rs + (int64_t)kk * L.t_ns;
+      float sum = ld_cg_f32(src);
+      for (int c = 1; c < L.t_ns; ++c) sum += ld_cg_f32(src + c);
+      if (WF == 1) sum *= p.pool.qscale[(((int64_t)a * p.pool.n_proj + L.proj) * 2 + 1) * p.pool.max_rank + kk];
+      tS[m * kQMaxR + kk] = sum;
+    }
+    bar_consumers();
+  }
+  if (act) {
+#pragma unroll
+    for (int kk = 0; kk < kQRB; ++kk) {
+      const int k = t.sub * kQRB + kk;
+      if (k >= r) break;  // warp-uniform
+      float bf[8];
+      const unsigned char* br = slot + kk * kQRowBytes;
+      if (WF == 0) unpack8<DT>(*reinterpret_cast<const uint4*>(br + 2 * jl), bf);
+      else unpack8_q8(*reinterpret_cast<const uint2*>(br + jl), bf);
+#pragma unroll
+      for (int m = 0; m < NT; ++m) {
+        const float tk = tS[m * kQMaxR + k];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[m][i] = fmaf(tk, bf[i], acc[m][i]);
+      }
+    }
+    if (t.sub == cdiv_i(r, kQRB) - 1) {
+      const float sa = p.pool.scale[a];
+#pragma unroll
+      for (int m = 0; m < NT; ++m) {
+        if (m >= nt) break;
+        uint16_t* yp = L.y + (int64_t)P.perm[pos0 + m] * L.ldy + col;
+        float yf[8];
+        unpack8<DT>(*reinterpret_cast<const uint4*>(yp), yf);
+        uint4 o;
+        o.x = pack2<DT>(fmaf(sa, acc[m][0], yf[0]), fmaf(sa, acc[m][1], yf[1]));
+        o.y = pack2<DT>(fmaf(sa, acc[m][2], yf[2]), fmaf(sa, acc[m][3], yf[3]));
+        o.z = pack2<DT>(fmaf(sa, acc[m][4], yf[4]), fmaf(sa, acc[m][5], yf[5]));
+        o.w = pack2<DT>(fmaf(sa, acc[m][6], yf[6]), fmaf(sa, acc[m][7], yf[7]));
+        *reinterpret_cast<uint4*>(yp) = o;
+      }
+    }
+  }
+}
+
+// Grid barrier between the phases (all CTAs are resident: cooperative launch).
+__device__ __forceinline__ void grid_arrive(int* bar) {
+  bar_consumers();  // every t partial of this CTA is written
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(bar, 1);
+  }
+}
+__device__ __forceinline__ void grid_wait(const int* bar, int32_t* err) {
+  if (threadIdx.x == 0) {
+    long long t0 = -1;
+    for (uint32_t it = 0; ld_acquire_s32(bar) < (int)gridDim.x; ++it) {
+      if ((it & 15) == 0) {
+        const long long now = clock64();
+        if (t0 < 0) t0 = now;
+        else if (now - t0 > kWaitLimit) {
+          record_error(err, 4, (int)blockIdx.x);
+          break;
+        }
+      }
+      __nanosleep(64);
+    }
+  }
+  bar_consumers();
+}
+
+// The CTA's stages: its shrink tasks [sh0, sh1) (an equal share of the count),
+// then the expand tasks whose first stage falls in its equal share of all
+// expand stages.
+struct QSeq {
+  int task, sub;     // current task index (shrink < n_shr <= expand) and stage within it
+  int sh1, e1;       // end of the shrink share; end (in expand stages) of the expand share
+};
+
+__device__ __forceinline__ int first_expand_task(const QPlan& P, const BgmvParams& p, int e0) {
+  const int S = P.S;
+  if (S == 0 || e0 >= P.exp_spre[S]) return P.exp_pre[S];
+  const int s = find_seg(P.exp_spre, S, e0);
+  const int ns = cdiv_i(P.seg_rank[s], kQRB);
+  const int loc = cdiv_i(e0 - P.exp_spre[s], ns);
+  return P.exp_pre[s] + loc;  // loc may equal the segment's task count: the next segment's first
+}
+__device__ __forceinline__ int expand_first_stage(const QPlan& P, int te) {
+  const int s = find_seg(P.exp_pre, P.S, te);
+  return P.exp_spre[s] + (te - P.exp_pre[s]) * cdiv_i(P.seg_rank[s], kQRB);
+}
+
+template <int DT, int WF>
+__global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ BgmvParams p) {
+  __shared__ QPlan P;
+  __shared__ __align__(16) float red[kQCons * 64];
+  __shared__ __align__(16) float tS[kQETok * kQMaxR];
+  __shared__ __align__(16) int ck[kQThreads];
+  __shared__ int4 sh4[32];
+  __shared__ int sh1[32];
+  __shared__ QTask sdesc[2];
+  __shared__ __align__(8) uint64_t full[2], empty[2];
+  __shared__ int warm_sink;
+  extern __shared__ __align__(128) unsigned char ring[];  // 2 stage slots; the plan's histogram first
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* ready = p.sc.ready;
+  int* gbar = ready + kQBar;
+  {  // every 64-byte line of the parameter block at once: the plan's first
+     // lookups into the group and slot tables would otherwise each wait on a
+     // cold constant-cache miss
+    constexpr int kLines = (int)((sizeof(BgmvParams) + 63) / 64);
+    static_assert(kLines <= kQAll, "parameter lines");
+    if (tid < kLines) {
+      const int v = reinterpret_cast<const int*>(&p)[tid * 16];
+      if (v == 0x5a5a5a5a) warm_sink = v;  // keeps the load; the value is never used
+    }
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kQCons);
+    }
+    fence_mbar_init();
+  }
+  plan_call(p, P, reinterpret_cast<int*>(ring), ck, sh4, sh1);  // ends with a barrier
+  const int S = P.S, n_shr = P.shr_pre[S], total = n_shr + P.exp_pre[S];
+  if (warp == kQCons) {
+    // ---- producer warp: the CTA's stage sequence, page ids one stage ahead,
+    // one bulk copy per page piece of a stage row (lane: row lane / 4, pieces
+    // lane % 4 and lane % 4 + 4 of it)
+    const int G = gridDim.x, bx = blockIdx.x;
+    const int sh0 = (int)((int64_t)bx * n_shr / G), sh_end = (int)((int64_t)(bx + 1) * n_shr / G);
+    const int n_es = P.exp_spre[S];
+    const int e0 = (int)((int64_t)bx * n_es / G), e_end = (int)((int64_t)(bx + 1) * n_es / G);
+    auto valid = [&](int tk) {
+      if (tk < n_shr) return tk < sh_end;
+      return tk < total && expand_first_stage(P, tk - n_shr) < e_end;
+    };
+    auto at = [&](int tk) -> QTask {
+      return valid(tk) ? decode_task(p, P, tk, n_shr, total) : QTask{-1, 0, 0, 0, 0, 0, 0};
+    };
+    int task = sh0 < sh_end ? sh0 : n_shr + first_expand_task(P, p, e0);
+    QTask t = at(task);
+    const int i = lane >> 2, qp = lane & 3;
+    const int sh = p.pool.page_shift + WF;
+    int32_t pg[2];
+    int ipo[2], dso[2], nb[2];  // in-page byte offset, destination offset in the slot, bytes
+    auto resolve = [&](const QTask& tt) {
+      const int32_t* list = nullptr;
+      int64_t f0 = 0;
+      int L = 0;
+      bool ok = false;
+      if (tt.shrink >= 0) stage_rows(p, P, tt, i, list, f0, L, ok);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int pq = qp + 4 * h;  // the row's pieces: [f0, next page boundary), then page by page
+        const int64_t fb = pq == 0 ? f0 : ((f0 >> sh) + pq) << sh;
+        const int64_t fe = min(f0 + L, ((f0 >> sh) + pq + 1) << sh);
+        const bool has = ok && fb < fe;
+        nb[h] = has ? (int)(fe - fb) << (1 - WF) : 0;
+        ipo[h] = (int)(fb & ((1ll << sh) - 1)) << (1 - WF);
+        dso[h] = i * kQRowBytes + ((int)(fb - f0) << (1 - WF));
+        pg[h] = has ? __ldg(list + (fb >> sh)) : 0;
+      }
+    };
+    // L2 prefetch of what the consumers read besides the slot: a shrink
+    // stage's x rows, an expand task's y rows (with its first stage)
+    auto prefetch_xy = [&](const QTask& tt) {
+      if (tt.shrink < 0 || (tt.shrink == 0 && tt.sub > 0)) return;
+      const int pos0 = P.seg_start[tt.s] + tt.w * (tt.shrink ? kQSTok : kQETok);
+      const int nt = min(tt.shrink ? kQSTok : kQETok, P.seg_start[tt.s + 1] - pos0);
+      const uint16_t* base;
+      int64_t ld;
+      int c0, len;
+      if (tt.shrink) {
+        const GroupDev& Gx = p.group[tt.u];
+        base = Gx.x;
+        ld = Gx.ldx;
+        c0 = tt.c * kQKT;
+        len = min(kQKT, Gx.d_in - c0);
+      } else {
+        const SlotDev& Sy = p.slot[tt.u];
+        base = Sy.y;
+        ld = Sy.ldy;
+        c0 = tt.v * kQECols;
+        len = min(kQECols, Sy.d_out - c0);
+      }
+      for (int v = lane; v < nt * (kQKT / 64); v += 32) {
+        const int m = v / (kQKT / 64), col = (v - m * (kQKT / 64)) * 64;
+        if (col < len)
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (int64_t)P.perm[pos0 + m] * ld + c0 + col));
+      }
+    };
+    resolve(t);
+    prefetch_xy(t);
+    const unsigned char* pool = reinterpret_cast<const unsigned char*>(p.pool.pool);
+    for (int n = 0;; ++n) {
+      const int slot = n & 1;
+      if (n >= 2) mbar_wait(&empty[slot], ((n >> 1) - 1) & 1, p.pool.err);
+      if (lane == 0) sdesc[slot] = t;
+      if (t.shrink < 0) {  // the end: the consumers read the descriptor and stop
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[slot]);
+        break;
+      }
+      int bytes = nb[0] + nb[1];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) bytes += __shfl_xor_sync(FULL_MASK, bytes, o);
+      __syncwarp();  // the descriptor is written before the arrival that publishes it
+      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)bytes);
+      __syncwarp();
+      unsigned char* dst = ring + slot * kQSlotBytes;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (nb[h] > 0)
+          bulk_g2s(dst + dso[h], pool + ((int64_t)pg[h] << (p.pool.page_shift + 1)) + ipo[h], (uint32_t)nb[h],
+                   &full[slot]);
+      // the next stage: the task's next rank-row block, or the next task of the share
+      if (t.shrink == 0 && t.sub + 1 < cdiv_i(P.seg_rank[t.s], kQRB)) {
+        ++t.sub;
+      } else {
+        ++task;
+        if (task == sh_end && task <= n_shr) task = n_shr + first_expand_task(P, p, e0);
+        t = at(task);
+      }
+      resolve(t);
+      prefetch_xy(t);
+    }
+  } else {
+    // ---- consumer warps
+    float acc[kQETok][8];
+    bool arrived = false, passed = false;
+    for (int n = 0;; ++n) {
+      const int slot = n & 1;
+      mbar_wait(&full[slot], (n >> 1) & 1, p.pool.err);
+      const QTask t = sdesc[slot];
+      if (t.shrink != 1 && !arrived) {  // this CTA's shrink stages are done
+        grid_arrive(gbar);
+        arrived = true;
+      }
+      if (t.shrink < 0) break;
+      if (t.shrink == 0 && !passed) {
+        grid_wait(gbar, p.pool.err);
+        passed = true;
+      }
+      const unsigned char* sl = ring + slot * kQSlotBytes;
+      if (t.shrink) {
+        shrink_stage<DT, WF>(p, P, red, t, sl);
+      } else {
+        const int nt = min(kQETok, P.seg_start[t.s + 1] - P.seg_start[t.s] - t.w * kQETok);
+        if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, acc);
+        else if (nt == 2) expand_stage<DT, WF, 2>(p, P, tS, t, sl, acc);
+        else expand_stage<DT, WF, 4>(p, P, tS, t, sl, acc);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+  }
+  // the last CTA to finish clears the counters for the next call
+  __shared__ int last_cta;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    last_cta = atomicAdd(ready + kFReadyCap, 1) == (int)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (last_cta && tid == 0) {
+    ready[kQBar] = 0;
+    ready[kFReadyCap] = 0;
+  }
+}
+
+// Dynamic shared memory: the two stage slots, which also hold the plan's
+// histogram (max_adapters <= 16384 ints) before the first stage.
+constexpr int kQDyn = 2 * kQSlotBytes;
+static_assert(4 * 16384 <= kQDyn, "histogram");
+
+template <int DT, int WF>
+cudaError_t launch_one(const BgmvParams& p, int grid, cudaStream_t s) {
+  static bool granted = false;
+  if (!granted) {
+    const cudaError_t e = cudaFuncSetAttribute(k_stream<DT, WF>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQDyn);
+    if (e != cudaSuccess) return e;
+    granted = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kQAll);
+  cfg.dynamicSmemBytes = kQDyn;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeCooperative;  // the phases meet at a grid barrier
+  at[0].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_stream<DT, WF>, p);
+}
+
+}  // namespace
+
+int stream_blocks_per_sm(int /*max_adapters*/) {
+  int n = 0;
+  if (cudaFuncSetAttribute(k_stream<SLORA_F16, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kQDyn) != cudaSuccess)
+    return 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_stream<SLORA_F16, 0>, kQAll, kQDyn) != cudaSuccess)
+    return 1;
+  return n < 1 ? 1 : n;
+}
+
+cudaError_t launch_stream(BgmvParams& p, int dtype, const int32_t* idx, int T, int grid, cudaStream_t s) {
+  p.idx = idx;
+  p.T = T;
+  if (T > kFMaxT || p.sc.ready == nullptr || p.n_groups * kFSegCap > kFReadyCap) return cudaErrorInvalidValue;
+  const int wf = p.pool.wfmt == SLORA_WEIGHTS_E4M3 ? 1 : 0;
+  if (dtype == SLORA_BF16) return wf ? launch_one<SLORA_BF16, 1>(p, grid, s) : launch_one<SLORA_BF16, 0>(p, grid, s);
+  return wf ? launch_one<SLORA_F16, 1>(p, grid, s) : launch_one<SLORA_F16, 0>(p, grid, s);
+}
+
+}  // namespace slora

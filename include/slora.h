@@ -90,23 +90,31 @@ typedef enum {
   SLORA_PAGEIN_MEMCPY = 1      /* one cudaMemcpyAsync per run of consecutive pages */
 } slora_pagein_mode_t;
 
-/* Kernels that run slora_lora_delta (and slora_lora_delta_noalloc).  Both give
- * the same arithmetic (fp32 partials per 2048-element slice of d_in, summed in
- * slice order, one rounding of y); they differ in launches and scheduling.
- * slora_decode_kernels() tells which one a call takes. */
+/* Kernels that run slora_lora_delta (and slora_lora_delta_noalloc).  All give
+ * fp32 partials per 2048-element slice of d_in, summed in slice order, and one
+ * rounding of y; they differ in launches, scheduling and the summation order
+ * inside a slice (the FMA pipe for SPLIT and FUSED, the tensor cores' fp32
+ * accumulation for STREAM's shrink); the one-CTA-per-token kernel of small
+ * AUTO calls sums each rank row in one pass.  slora_decode_kernels() tells
+ * how many kernels a call launches. */
 typedef enum {
   SLORA_DECODE_AUTO = 0,       /* the library's choice: 16-bit pools run calls of
                                   up to 16 tokens as one CTA per token (plain
-                                  loads, no scratch: a latency-bound batch) and
-                                  larger calls on the three-kernel path (the
-                                  faster one on B200 at the shapes measured so
-                                  far); e4m3 pools take the one-kernel path    */
+                                  loads, no scratch: a latency-bound batch);
+                                  other calls of up to 1024 tokens take STREAM,
+                                  larger ones SPLIT                              */
   SLORA_DECODE_SPLIT = 1,      /* always three kernels: segment build, shrink,
                                   expand                                         */
-  SLORA_DECODE_FUSED = 2       /* one persistent kernel for calls of up to 1024
-                                  tokens (every CTA builds the segment table, then
-                                  the shrink and expand tasks in one launch); the
-                                  three kernels above that                       */
+  SLORA_DECODE_FUSED = 2,      /* one persistent kernel with a bulk-copy ring for
+                                  calls of up to 1024 tokens (every CTA builds the
+                                  segment table, then the shrink and expand tasks
+                                  in one launch); SPLIT above that               */
+  SLORA_DECODE_STREAM = 3      /* one kernel of independent tasks for calls of up
+                                  to 1024 tokens: every CTA plans the call, then
+                                  claims shrink tasks and, after them, expand
+                                  tasks from one counter; weights stream from the
+                                  pages into registers with plain 16-byte loads.
+                                  SPLIT above 1024 tokens                        */
 } slora_decode_path_t;
 
 /* How a pool stores adapter weights in its pages. */
@@ -446,8 +454,8 @@ slora_status_t slora_lora_delta_noalloc(slora_pool* pool, int32_t n, const int32
                                         int32_t T, void* stream);
 
 /* Number of kernels slora_lora_delta launches for a call of T tokens on this
- * pool (1: the one-kernel path or one CTA per token, 3: segment build,
- * shrink, expand); 0 for T <= 0 or a NULL pool.  Host only. */
+ * pool (1: one kernel -- one CTA per token, FUSED or STREAM; 3: segment
+ * build, shrink, expand); 0 for T <= 0 or a NULL pool.  Host only. */
 int32_t slora_decode_kernels(const slora_pool* pool, int32_t T);
 
 /* Size in bytes of the fixed scratch array used by slora_lora_delta_noalloc. */

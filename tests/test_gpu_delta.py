@@ -1,9 +1,10 @@
 """GPU parity of the decode path (segment build + paged shrink + expand) with
-the fp64 oracle, on the same seeded inputs.  Both decode paths are checked:
-the one persistent kernel (pools created with SLORA_DECODE_FUSED, batches of
-up to 1024 tokens) and the three-kernel path (SLORA_DECODE_SPLIT, the default
-for 16-bit pools, and every batch above 1024 tokens); the two must agree bit
-for bit (same fp32 partials, same summation order).
+the fp64 oracle, on the same seeded inputs.  Every decode path is checked: the
+one kernel of streaming tasks (SLORA_DECODE_STREAM, the default for 17..1024
+tokens), the persistent bulk-copy kernel (SLORA_DECODE_FUSED) and the
+three-kernel path (SLORA_DECODE_SPLIT, every batch above 1024 tokens); the
+last two must agree bit for bit (same fp32 partials, same summation order),
+and every path must give the same bits on a repeated call.
 
 Acceptance bound, per projection output y_out:
     |gpu - oracle| <= 1e-2 * max|oracle| + 1e-3   (elementwise)
@@ -70,9 +71,11 @@ def test_tiny_config():
 
 
 PATHS = [G.SLORA_DECODE_FUSED, G.SLORA_DECODE_SPLIT]
+ALL_PATHS = [G.SLORA_DECODE_STREAM, G.SLORA_DECODE_FUSED, G.SLORA_DECODE_SPLIT]
+ALL_IDS = ["stream", "fused", "split"]
 
 
-@pytest.mark.parametrize("path", PATHS, ids=["fused", "split"])
+@pytest.mark.parametrize("path", ALL_PATHS, ids=ALL_IDS)
 @pytest.mark.parametrize("dtype", [W.F16, W.BF16])
 def test_ragged_mixed(dtype, path):
     """Ragged everything: d_in not a multiple of the 1024-element chunk nor of
@@ -150,14 +153,18 @@ def test_small_batch_token_path(T):
     pb.close()
 
 
-def test_degenerate_batches():
+@pytest.mark.parametrize("path", [G.SLORA_DECODE_AUTO] + ALL_PATHS, ids=["auto"] + ALL_IDS)
+@pytest.mark.parametrize("T", [4, 40])
+def test_degenerate_batches(T, path):
     import torch
     projs = [W.Proj("q", 1024, 1024, "a")]
-    w = _custom(W.F16, projs, [16, 0], [-1, -1, 1, -1])
-    pb = H.PoolBuild(w)
+    idx = np.resize(np.array([-1, -1, 1, -1], np.int32), T)
+    w = _custom(W.F16, projs, [16, 0], idx)
+    pb = H.PoolBuild(w, decode_path=path)
     ten = H.Tensors(w)
-    _run_delta(pb, ten, w)           # no adapter / rank 0 only: y unchanged
-    assert np.array_equal(H.from_device(ten.y[0]), w.y_in(0))
+    for _ in range(2):               # no adapter / rank 0 only: y unchanged
+        _run_delta(pb, ten, w)
+        assert np.array_equal(H.from_device(ten.y[0]), w.y_in(0))
     idx = torch.zeros(1, dtype=torch.int32, device="cuda")
     G.slora_lora_delta(pb.h, *ten.args(), idx, 0)     # T = 0 is a no-op
     torch.cuda.synchronize()
@@ -183,22 +190,42 @@ def test_single_shared_adapter_is_a_gemm():
     pb.close()
 
 
-def test_bad_token_is_skipped_and_reported():
+@pytest.mark.parametrize("T", [4, 24])
+def test_bad_token_is_skipped_and_reported(T):
     import torch
     projs = [W.Proj("q", 1024, 1024, "a")]
-    idx = np.array([0, 1, 7, 0], np.int32)
-    w = _custom(W.F16, projs, [16, 8], np.array([0, 1, 1, 0], np.int32))
+    idx = np.resize(np.array([0, 1, 1, 0], np.int32), T)
+    idx[2] = 7                                        # the one bad id
+    w = _custom(W.F16, projs, [16, 8], np.where(idx == 7, 1, idx).astype(np.int32))
     pb = H.PoolBuild(w)
     ten = H.Tensors(w)
-    G.slora_lora_delta(pb.h, *ten.args(), torch.from_numpy(idx).cuda(), 4)
+    G.slora_lora_delta(pb.h, *ten.args(), torch.from_numpy(idx).cuda(), T)
     st, code, info = G.slora_check_device(pb.h)
     assert st == 6 and code == 1 and info == 2
     got = H.from_device(ten.y[0])
     assert np.array_equal(got[2], w.y_in(0)[2])       # bad token untouched
-    ok_idx = np.array([0, 1, -1, 0], np.int32)
+    ok_idx = np.where(idx == 7, -1, idx).astype(np.int32)
     x, _, y, A_t, B = H.oracle_inputs(w, 0)
     ref = oracle.lora_delta(w.dtype, x, ok_idx, y, w.ranks, [16.0, 16.0], A_t, B)
     assert H.tolerance_check(got, ref, w.dtype)[0]
+    pb.close()
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_full_size_configs_stream(cfg):
+    """The LLaMA-7B and LLaMA-13B decode layers on the default path (one kernel
+    of streaming tasks), every output element against the oracle, and a
+    repeated call bit-identical."""
+    w = W.config(cfg)
+    pb = H.PoolBuild(w)
+    assert G.slora_decode_kernels(pb.h, w.T) == 1
+    ten = H.Tensors(w)
+    _run_delta(pb, ten, w)
+    _check_all(w, ten, threads=16)
+    first = [H.from_device(t) for t in ten.y]
+    ten.reset()
+    _run_delta(pb, ten, w)
+    assert all(np.array_equal(a, H.from_device(b)) for a, b in zip(first, ten.y))
     pb.close()
 
 
@@ -248,6 +275,35 @@ def test_fused_matches_split_bitwise(T):
         assert np.array_equal(outs[0][p], outs[1][p]), projs[p].name
     tokens = np.arange(T) if T <= 64 else np.sort(rng.choice(T, 96, replace=False))
     _check_all(w, ten, tokens=tokens, tight=True, threads=16)
+
+
+@pytest.mark.parametrize("T", [17, 33, 700, 1024])
+def test_stream_edges(T):
+    """The streaming-task kernel at the edges of its range (17 tokens, a ragged
+    33, 700, the 1024-token limit) with Zipf-skewed ids over mixed ranks up to
+    128, one hot adapter holding more than one shrink token tile, and rows
+    across 8192-element pages: sampled tokens against the oracle at the tight
+    bound, and a repeated call bit-identical."""
+    rng = np.random.default_rng(500 + T)
+    projs = [W.Proj("q", 2048, 2048, "a"), W.Proj("v", 2048, 512, "a"), W.Proj("d", 5504, 2048, "c")]
+    n_ad = 64
+    ranks = rng.choice(np.array([8, 16, 32, 64, 128, 24, 5], np.int32), n_ad)
+    idx = W.zipf_ids(rng, n_ad, 1.1, T)
+    idx[: T // 3] = 7                            # a hot adapter: tokens spread over the batch
+    idx = idx[rng.permutation(T)]
+    if T > 2:
+        idx[rng.random(T) < 0.1] = -1
+    w = _custom(W.BF16, projs, ranks, idx, page_elems=8192, shuffle=True, seed=37)
+    pb = H.PoolBuild(w, decode_path=G.SLORA_DECODE_STREAM)
+    ten = H.Tensors(w)
+    _run_delta(pb, ten, w)
+    first = [H.from_device(t) for t in ten.y]
+    tokens = np.arange(T) if T <= 64 else np.sort(rng.choice(T, 96, replace=False))
+    _check_all(w, ten, tokens=tokens, tight=True, threads=16)
+    ten.reset()
+    _run_delta(pb, ten, w)
+    assert all(np.array_equal(a, H.from_device(b)) for a, b in zip(first, ten.y))
+    pb.close()
 
 
 def test_many_single_stage_tasks_repeatable():

@@ -27,9 +27,9 @@ def _tight_ok(got_bits, ref, dtype):
     return bool(np.all(np.abs(got - ref) <= bound))
 
 
-def _run_and_check(w, tokens=None, tight=True, threads=16):
+def _run_and_check(w, tokens=None, tight=True, threads=16, path=G.SLORA_DECODE_AUTO):
     import torch
-    pb = H.PoolBuild(w, weight_format=G.SLORA_WEIGHTS_E4M3)
+    pb = H.PoolBuild(w, weight_format=G.SLORA_WEIGHTS_E4M3, decode_path=path)
     ten = H.Tensors(w)
     idx = torch.from_numpy(w.idx).cuda()
     G.slora_lora_delta(pb.h, *ten.args(), idx, w.T)
@@ -67,13 +67,14 @@ def test_q8_tiny():
     pb.close()
 
 
+@pytest.mark.parametrize("path", [G.SLORA_DECODE_STREAM, G.SLORA_DECODE_FUSED], ids=["stream", "fused"])
 @pytest.mark.parametrize("dtype", [W.F16, W.BF16])
-def test_q8_ragged(dtype):
+def test_q8_ragged(dtype, path):
     """Ranks not multiples of 8, rank 0, tokens without adapter, rows that
-    straddle 512-element pages (1024 codes), shared x across projections; the
-    pages hold exactly the registered codes."""
+    straddle 512-element pages (1024 codes), shared x across projections, on
+    both one-kernel paths; the pages hold exactly the registered codes."""
     w = _ragged(dtype)
-    pb, ten = _run_and_check(w)
+    pb, ten = _run_and_check(w, path=path)
     for a in (2, 5, 8):
         cA, _, cB, _ = pb.q8w[a]
         for p in range(len(w.projs)):

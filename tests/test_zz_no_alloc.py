@@ -4,8 +4,8 @@ where they run the delta, such as a plug-in whose host framework owns every
 device allocation), checked on two calls in a row against the fp64 oracle
 (the acceptance bound and the tighter arithmetic bound) and against
 slora_lora_delta on the same inputs; a call whose scratch need exceeds the
-array is refused.  Both decode paths (one persistent kernel, three kernels)
-run through it.
+array is refused.  Every decode path (the streaming-task kernel, the
+persistent kernel, three kernels) runs through it.
 
 Kept in its own file, named to be collected last, so that a run stopping at the
 first failure has already run every other test.  It builds its own pools, so
@@ -41,7 +41,8 @@ def _tight_ok(got_bits, ref, dtype):
     return bool(np.all(np.abs(got - ref) <= bound))
 
 
-@pytest.mark.parametrize("path", [G.SLORA_DECODE_FUSED, G.SLORA_DECODE_SPLIT], ids=["fused", "split"])
+@pytest.mark.parametrize("path", [G.SLORA_DECODE_STREAM, G.SLORA_DECODE_FUSED, G.SLORA_DECODE_SPLIT],
+                         ids=["stream", "fused", "split"])
 @pytest.mark.parametrize("make", [lambda: W.config(0), _ragged_workload], ids=["tiny", "ragged"])
 def test_noalloc_matches_oracle_twice(make, path):
     import torch
