@@ -48,7 +48,8 @@ constexpr int kQECols = 2048;                 // outputs per expand task: 256 pe
 constexpr int kQETok = 4;                     // tokens per expand task
 constexpr int kQMaxR = 128;
 static_assert(kQKT == kQWarps * 256 && kQECols == kQWarps * 256, "task shapes");
-constexpr int kQBar = kFReadyCap + 1;         // ready[]: finished CTAs at kFReadyCap, then the phase barrier
+// ready[] (scratch, zero between calls): per (segment, x group) counts of
+// finished shrink tasks, then at kFReadyCap the count of finished CTAs
 
 // The call's plan, identical in every CTA.
 struct QPlan {
@@ -280,6 +281,9 @@ __device__ __forceinline__ QTask decode_task(const BgmvParams& p, const QPlan& P
 // of a row), counted on the slot's `full` mbarrier.
 constexpr int kQRowBytes = 2 * kQKT + 64;
 constexpr int kQSlotBytes = kQRB * kQRowBytes;
+constexpr int kQNS = 2;                            // stage slots (copies run up to kQNS - 1 stages ahead)
+constexpr int kQND = 2 * kQNS;                     // descriptor ring
+constexpr int kQCTAs = kQNS <= 2 ? 2 : 1;          // resident CTAs per SM
 constexpr int kQCons = 8;                          // consumer warps
 constexpr int kQAll = (kQCons + 1) * 32;           // + the producer warp
 static_assert(kQCons * 32 == kQThreads, "consumers");
@@ -328,9 +332,25 @@ __device__ __forceinline__ void stage_rows(const BgmvParams& p, const QPlan& P, 
 // Shrink stage (segment s, x group g, rank-row block b, d_in chunk c, token
 // tile of up to 8 tokens).  Lane l reads rank row l / 4 of the stage (zero
 // past the group's rows) and token l / 4 of the tile (zero past the segment).
+// A shrink stage's x pieces for lane l: token l / 4 of the tile, the lane's 8
+// columns of each 32-column step (clamped to the tile's last token and the
+// row's last 8 columns; the stage zeroes what lies outside).  Loaded one stage
+// ahead, so that the stage finds them in registers.
+__device__ __forceinline__ void load_x(const BgmvParams& p, const QPlan& P, const QTask& t, uint4 (&xc)[8]) {
+  if (t.shrink != 1) return;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const GroupDev& G = p.group[t.u];
+  const int pos0 = P.seg_start[t.s] + t.w * kQSTok;
+  const int nt = min(kQSTok, P.seg_start[t.s + 1] - pos0);
+  const int jw = t.c * kQKT + w * 256 + (lane & 3) * 8;
+  const uint16_t* xr = G.x + (int64_t)P.perm[pos0 + min(lane >> 2, nt - 1)] * G.ldx;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) xc[u] = __ldg(reinterpret_cast<const uint4*>(xr + min(jw + 32 * u, G.d_in - 8)));
+}
+
 template <int DT, int WF>
 __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, const QTask& t,
-                             const unsigned char* slot) {
+                             const unsigned char* slot, const uint4 (&xc)[8]) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, q = lane & 3, gr = lane >> 2;
   const int s = t.s, g = t.u, b = t.v, c = t.c;
   const int a = P.seg_adapter[s], r = P.seg_rank[s];
@@ -341,10 +361,6 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
   const bool rv = b * kQRB + gr < nrows, xv = gr < nt;
   const int j0 = w * 256 + q * 8;  // in the chunk; step u adds 32
   const int jw = c * kQKT + j0;
-  const uint16_t* xr = G.x + (int64_t)P.perm[pos0 + min(gr, nt - 1)] * G.ldx;
-  uint4 xc[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) xc[u] = __ldg(reinterpret_cast<const uint4*>(xr + min(jw + 32 * u, d_in - 8)));
   const unsigned char* arow = slot + gr * kQRowBytes;
   float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // two chains: steps u even / odd
 #pragma unroll
@@ -391,10 +407,10 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
 
 // ---------------------------------------------------------------------------
 // Expand stage: rank rows 8 sub .. 8 sub + 7 of task (segment s, slot ks,
-// output chunk e, token group tg).  The first stage fills tS with t = sum of
-// the chunk partials (every shrink task has finished: the phases are split by
-// a grid barrier); the last one adds s_a * acc to y (prefetched to L2 by the
-// producer) and rounds.
+// output chunk e, token group tg).  The first stage waits until every shrink
+// task of (s, the slot's x group) has been counted, then fills tS with t =
+// sum of the chunk partials; the last one adds s_a * acc to y (prefetched to
+// L2 by the producer) and rounds.
 template <int DT, int WF, int NT>
 __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, const QTask& t,
                              const unsigned char* slot, float (&acc)[kQETok][8]) {
@@ -411,7 +427,25 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
     for (int m = 0; m < NT; ++m)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
-    bar_consumers();  // the previous expand task's reads of tS are done
+    if (tid == 0) {  // bounded wait for the shrink tasks of (s, x group)
+      const GroupDev& G = p.group[L.group];
+      const int need = cdiv_i(G.n * r, kQRB) * cdiv_i(G.d_in, kQKT) *
+                       cdiv_i(P.seg_start[s + 1] - P.seg_start[s], kQSTok);
+      const int* cnt = p.sc.ready + s * p.n_groups + L.group;
+      long long t0 = -1;
+      for (uint32_t it = 0; ld_acquire_s32(cnt) < need; ++it) {
+        if ((it & 15) == 0) {
+          const long long now = clock64();
+          if (t0 < 0) t0 = now;
+          else if (now - t0 > kWaitLimit) {
+            record_error(p.pool.err, 4, (int)blockIdx.x);
+            break;
+          }
+        }
+        __nanosleep(32);
+      }
+    }
+    bar_consumers();  // the count is seen; the previous expand task's reads of tS are done
     for (int v = tid; v < nt * r; v += kQThreads) {
       const int m = v / r, kk = v - m * r;
       const float* src = L.t + (int64_t)(pos0 + m) * L.t_rs + (int64_t)kk * L.t_ns;
@@ -457,40 +491,9 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
   }
 }
 
-// Grid barrier between the phases (all CTAs are resident: cooperative launch).
-__device__ __forceinline__ void grid_arrive(int* bar) {
-  bar_consumers();  // every t partial of this CTA is written
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(bar, 1);
-  }
-}
-__device__ __forceinline__ void grid_wait(const int* bar, int32_t* err) {
-  if (threadIdx.x == 0) {
-    long long t0 = -1;
-    for (uint32_t it = 0; ld_acquire_s32(bar) < (int)gridDim.x; ++it) {
-      if ((it & 15) == 0) {
-        const long long now = clock64();
-        if (t0 < 0) t0 = now;
-        else if (now - t0 > kWaitLimit) {
-          record_error(err, 4, (int)blockIdx.x);
-          break;
-        }
-      }
-      __nanosleep(64);
-    }
-  }
-  bar_consumers();
-}
-
-// The CTA's stages: its shrink tasks [sh0, sh1) (an equal share of the count),
-// then the expand tasks whose first stage falls in its equal share of all
-// expand stages.
-struct QSeq {
-  int task, sub;     // current task index (shrink < n_shr <= expand) and stage within it
-  int sh1, e1;       // end of the shrink share; end (in expand stages) of the expand share
-};
-
+// The CTA's stages: its shrink tasks [sh0, sh_end) (an equal share of the
+// count), then the expand tasks whose first stage falls in its equal share of
+// all expand stages.
 __device__ __forceinline__ int first_expand_task(const QPlan& P, const BgmvParams& p, int e0) {
   const int S = P.S;
   if (S == 0 || e0 >= P.exp_spre[S]) return P.exp_pre[S];
@@ -504,21 +507,112 @@ __device__ __forceinline__ int expand_first_stage(const QPlan& P, int te) {
   return P.exp_spre[s] + (te - P.exp_pre[s]) * cdiv_i(P.seg_rank[s], kQRB);
 }
 
+// The producer's walk over the CTA's tasks: the current task's fields kept
+// alongside the counts they run through, so that the next task follows with
+// a few increments (the same order decode_task assigns: shrink tasks by
+// segment, x group, d_in chunk, rank-row block, token tile; expand tasks by
+// segment, slot, output chunk, token group; an expand task's stages by sub).
+struct QCursor {
+  QTask t;
+  int task;   // global task index (shrink < n_shr <= expand)
+  int stage;  // expand: index of the task's first stage among all expand stages
+  int n, r;   // the segment's tokens and rank
+  int nb, nc, ntt;  // shrink: row blocks and chunks of the group, token tiles
+  int ne, ntg, ns;  // expand: output chunks of the slot, token groups, stages per task
+
+  __device__ void seg_fields(const BgmvParams& p, const QPlan& P) {
+    n = P.seg_start[t.s + 1] - P.seg_start[t.s];
+    r = P.seg_rank[t.s];
+    ntt = cdiv_i(n, kQSTok);
+    ntg = cdiv_i(n, kQETok);
+    ns = cdiv_i(r, kQRB);
+  }
+  __device__ void sub_fields(const BgmvParams& p) {
+    if (t.shrink > 0) {
+      nb = cdiv_i(p.group[t.u].n * r, kQRB);
+      nc = cdiv_i(p.group[t.u].d_in, kQKT);
+    } else if (t.shrink == 0) {
+      ne = cdiv_i(p.slot[t.u].d_out, kQECols);
+    }
+  }
+  __device__ void start(const BgmvParams& p, const QPlan& P, int tk, int n_shr, int total) {
+    task = tk;
+    t = decode_task(p, P, tk, n_shr, total);
+    if (t.shrink < 0) return;
+    seg_fields(p, P);
+    sub_fields(p);
+    if (t.shrink == 0) stage = expand_first_stage(P, tk - n_shr);
+  }
+  // the next stage; false past the end of the plan
+  __device__ bool next(const BgmvParams& p, const QPlan& P) {
+    if (t.shrink == 0) {
+      if (++t.sub < ns) return true;
+      t.sub = 0;
+      stage += ns;
+      ++task;
+      if (++t.w < ntg) return true;
+      t.w = 0;
+      if (++t.v < ne) return true;
+      t.v = 0;
+      if (++t.u < p.n_slots) {
+        sub_fields(p);
+        return true;
+      }
+      t.u = 0;
+      if (++t.s >= P.S) return false;
+      seg_fields(p, P);
+      sub_fields(p);
+      return true;
+    }
+    ++task;
+    if (++t.w < ntt) return true;
+    t.w = 0;
+    if (++t.v < nb) return true;
+    t.v = 0;
+    if (++t.c < nc) return true;
+    t.c = 0;
+    if (++t.u < p.n_groups) {
+      sub_fields(p);
+      return true;
+    }
+    t.u = 0;
+    if (++t.s >= P.S) return false;
+    seg_fields(p, P);
+    sub_fields(p);
+    return true;
+  }
+};
+
+// Bytes of a stage's rows.
+template <int WF>
+__device__ __forceinline__ int stage_bytes(const BgmvParams& p, const QPlan& P, const QTask& t) {
+  const int r = P.seg_rank[t.s];
+  int rows, L;
+  if (t.shrink > 0) {
+    rows = min(kQRB, p.group[t.u].n * r - t.v * kQRB);
+    L = min(kQKT, p.group[t.u].d_in - t.c * kQKT);
+  } else {
+    rows = min(kQRB, r - t.sub * kQRB);
+    L = min(kQECols, p.slot[t.u].d_out - t.v * kQECols);
+  }
+  return (rows * L) << (1 - WF);
+}
+
 template <int DT, int WF>
-__global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ BgmvParams p) {
+__global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant__ BgmvParams p) {
   __shared__ QPlan P;
   __shared__ __align__(16) float red[kQCons * 64];
   __shared__ __align__(16) float tS[kQETok * kQMaxR];
   __shared__ __align__(16) int ck[kQThreads];
   __shared__ int4 sh4[32];
   __shared__ int sh1[32];
-  __shared__ QTask sdesc[2];
-  __shared__ __align__(8) uint64_t full[2], empty[2];
+  __shared__ QTask sdesc[kQND];  // stage n's descriptor at n % kQND (written with dready[n % kQND])
+  // per slot: bytes landed (full), consumed (empty)
+  __shared__ __align__(8) uint64_t dready[kQND], full[kQNS], empty[kQNS];
   __shared__ int warm_sink;
   extern __shared__ __align__(128) unsigned char ring[];  // 2 stage slots; the plan's histogram first
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* ready = p.sc.ready;
-  int* gbar = ready + kQBar;
   {  // every 64-byte line of the parameter block at once: the plan's first
      // lookups into the group and slot tables would otherwise each wait on a
      // cold constant-cache miss
@@ -530,7 +624,8 @@ __global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ Bgm
     }
   }
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kQND; ++i) mbar_init(&dready[i], 1);
+    for (int i = 0; i < kQNS; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kQCons);
     }
@@ -546,20 +641,22 @@ __global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ Bgm
     const int sh0 = (int)((int64_t)bx * n_shr / G), sh_end = (int)((int64_t)(bx + 1) * n_shr / G);
     const int n_es = P.exp_spre[S];
     const int e0 = (int)((int64_t)bx * n_es / G), e_end = (int)((int64_t)(bx + 1) * n_es / G);
-    auto valid = [&](int tk) {
-      if (tk < n_shr) return tk < sh_end;
-      return tk < total && expand_first_stage(P, tk - n_shr) < e_end;
+    QCursor cur;
+    bool in_shrink = sh0 < sh_end;
+    cur.start(p, P, in_shrink ? sh0 : n_shr + first_expand_task(P, p, e0), n_shr, total);
+    auto in_share = [&]() {
+      if (cur.t.shrink < 0) return false;
+      return cur.t.shrink ? cur.task < sh_end : cur.stage < e_end;
     };
-    auto at = [&](int tk) -> QTask {
-      return valid(tk) ? decode_task(p, P, tk, n_shr, total) : QTask{-1, 0, 0, 0, 0, 0, 0};
-    };
-    int task = sh0 < sh_end ? sh0 : n_shr + first_expand_task(P, p, e0);
-    QTask t = at(task);
+    if (!in_share()) cur.t.shrink = -1;
+    QTask& t = cur.t;
     const int i = lane >> 2, qp = lane & 3;
     const int sh = p.pool.page_shift + WF;
-    int32_t pg[2];
-    int ipo[2], dso[2], nb[2];  // in-page byte offset, destination offset in the slot, bytes
-    auto resolve = [&](const QTask& tt) {
+    struct Pieces {
+      int32_t pg[2];
+      int ipo[2], dso[2], nb[2];  // in-page byte offset, destination offset in the slot, bytes
+    };
+    auto resolve = [&](const QTask& tt, Pieces& pc) {
       const int32_t* list = nullptr;
       int64_t f0 = 0;
       int L = 0;
@@ -571,10 +668,12 @@ __global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ Bgm
         const int64_t fb = pq == 0 ? f0 : ((f0 >> sh) + pq) << sh;
         const int64_t fe = min(f0 + L, ((f0 >> sh) + pq + 1) << sh);
         const bool has = ok && fb < fe;
-        nb[h] = has ? (int)(fe - fb) << (1 - WF) : 0;
-        ipo[h] = (int)(fb & ((1ll << sh) - 1)) << (1 - WF);
-        dso[h] = i * kQRowBytes + ((int)(fb - f0) << (1 - WF));
-        pg[h] = has ? __ldg(list + (fb >> sh)) : 0;
+        pc.nb[h] = has ? (int)(fe - fb) << (1 - WF) : 0;
+        pc.ipo[h] = (int)(fb & ((1ll << sh) - 1)) << (1 - WF);
+        pc.dso[h] = i * kQRowBytes + ((int)(fb - f0) << (1 - WF));
+        // unconditional (an absent piece re-reads the table's first entry), so
+        // that nothing consumes the load before the copies are issued
+        pc.pg[h] = __ldg(has ? list + (fb >> sh) : p.pool.page_list);
       }
     };
     // L2 prefetch of what the consumers read besides the slot: a shrink
@@ -605,67 +704,97 @@ __global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ Bgm
           asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (int64_t)P.perm[pos0 + m] * ld + c0 + col));
       }
     };
-    resolve(t);
-    prefetch_xy(t);
     const unsigned char* pool = reinterpret_cast<const unsigned char*>(p.pool.pool);
-    for (int n = 0;; ++n) {
-      const int slot = n & 1;
-      if (n >= 2) mbar_wait(&empty[slot], ((n >> 1) - 1) & 1, p.pool.err);
-      if (lane == 0) sdesc[slot] = t;
-      if (t.shrink < 0) {  // the end: the consumers read the descriptor and stop
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[slot]);
-        break;
+    // Descriptors go to a ring of 4 as soon as a stage is known (the consumers
+    // load its x from it); copies go to the stage's slot once the stage two
+    // before it has released the slot.
+    auto publish = [&](int n, const QTask& tt) {
+      if (lane == 0) sdesc[n % kQND] = tt;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dready[n % kQND]);
+    };
+    // Counts of finished shrink stages per (segment, x group): a stage is
+    // finished once its slot is released.  A pair's stages are consecutive in
+    // the CTA's sequence; their count is added (lane 0, after a fence) when
+    // the last of them is released, which never waits on a later stage.
+    int run_n = 0;
+    auto count = [&](const QTask& done, const QTask& after) {
+      if (done.shrink != 1) return;
+      const int key = done.s * p.n_groups + done.u;
+      ++run_n;
+      if (after.shrink != 1 || after.s * p.n_groups + after.u != key) {
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(ready + key, run_n);
+        }
+        run_n = 0;
       }
-      int bytes = nb[0] + nb[1];
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) bytes += __shfl_xor_sync(FULL_MASK, bytes, o);
-      __syncwarp();  // the descriptor is written before the arrival that publishes it
-      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)bytes);
+    };
+    Pieces pc_cur, pc_next;
+    resolve(t, pc_cur);
+    prefetch_xy(t);
+    publish(0, t);
+    int n = 0;
+    for (;; ++n) {
+      const int slot = n % kQNS;
+      const QTask tn = t;  // stage n
+      if (tn.shrink >= 0) {  // stage n + 1: known, published, its page ids on the way
+        const bool more = cur.next(p, P);
+        if (in_shrink && (!more || cur.task >= sh_end)) {  // the shrink share is done: the expand share
+          in_shrink = false;
+          cur.start(p, P, n_shr + first_expand_task(P, p, e0), n_shr, total);
+        } else if (!more) {
+          t.shrink = -1;
+        }
+        if (!in_share()) t.shrink = -1;
+        publish(n + 1, t);
+        resolve(t, pc_next);
+        prefetch_xy(t);
+      }
+      if (n >= kQNS) {  // stage n - kQNS has released the slot (its descriptor is still in the ring)
+        mbar_wait(&empty[slot], (n / kQNS - 1) & 1, p.pool.err);
+        count(sdesc[(n - kQNS) % kQND], sdesc[(n - kQNS + 1) % kQND]);
+      }
+      if (tn.shrink < 0) break;
+      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)stage_bytes<WF>(p, P, tn));
       __syncwarp();
       unsigned char* dst = ring + slot * kQSlotBytes;
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        if (nb[h] > 0)
-          bulk_g2s(dst + dso[h], pool + ((int64_t)pg[h] << (p.pool.page_shift + 1)) + ipo[h], (uint32_t)nb[h],
-                   &full[slot]);
-      // the next stage: the task's next rank-row block, or the next task of the share
-      if (t.shrink == 0 && t.sub + 1 < cdiv_i(P.seg_rank[t.s], kQRB)) {
-        ++t.sub;
-      } else {
-        ++task;
-        if (task == sh_end && task <= n_shr) task = n_shr + first_expand_task(P, p, e0);
-        t = at(task);
-      }
-      resolve(t);
-      prefetch_xy(t);
+        if (pc_cur.nb[h] > 0)
+          bulk_g2s(dst + pc_cur.dso[h], pool + ((int64_t)pc_cur.pg[h] << (p.pool.page_shift + 1)) + pc_cur.ipo[h],
+                   (uint32_t)pc_cur.nb[h], &full[slot]);
+      pc_cur = pc_next;
+    }
+    // the last stages are counted once released (stage n is the end marker)
+    for (int k = max(0, n - kQNS + 1); k < n; ++k) {
+      mbar_wait(&empty[k % kQNS], (k / kQNS) & 1, p.pool.err);
+      count(sdesc[k % kQND], sdesc[(k + 1) % kQND]);
     }
   } else {
     // ---- consumer warps
     float acc[kQETok][8];
-    bool arrived = false, passed = false;
+    uint4 xq[8];
+    mbar_wait(&dready[0], 0, p.pool.err);
+    QTask t = sdesc[0];
+    load_x(p, P, t, xq);
     for (int n = 0;; ++n) {
-      const int slot = n & 1;
-      mbar_wait(&full[slot], (n >> 1) & 1, p.pool.err);
-      const QTask t = sdesc[slot];
-      if (t.shrink != 1 && !arrived) {  // this CTA's shrink stages are done
-        grid_arrive(gbar);
-        arrived = true;
-      }
+      const int slot = n % kQNS;
       if (t.shrink < 0) break;
-      if (t.shrink == 0 && !passed) {
-        grid_wait(gbar, p.pool.err);
-        passed = true;
-      }
+      mbar_wait(&full[slot], (n / kQNS) & 1, p.pool.err);
       const unsigned char* sl = ring + slot * kQSlotBytes;
       if (t.shrink) {
-        shrink_stage<DT, WF>(p, P, red, t, sl);
+        shrink_stage<DT, WF>(p, P, red, t, sl, xq);
       } else {
         const int nt = min(kQETok, P.seg_start[t.s + 1] - P.seg_start[t.s] - t.w * kQETok);
         if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, acc);
         else if (nt == 2) expand_stage<DT, WF, 2>(p, P, tS, t, sl, acc);
         else expand_stage<DT, WF, 4>(p, P, tS, t, sl, acc);
       }
+      // the next stage's descriptor (and x) before this slot is released
+      mbar_wait(&dready[(n + 1) % kQND], ((n + 1) / kQND) & 1, p.pool.err);
+      t = sdesc[(n + 1) % kQND];
+      load_x(p, P, t, xq);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
@@ -678,15 +807,15 @@ __global__ void __launch_bounds__(kQAll, 2) k_stream(const __grid_constant__ Bgm
     last_cta = atomicAdd(ready + kFReadyCap, 1) == (int)gridDim.x - 1;
   }
   __syncthreads();
-  if (last_cta && tid == 0) {
-    ready[kQBar] = 0;
-    ready[kFReadyCap] = 0;
+  if (last_cta) {
+    for (int i = tid; i < S * p.n_groups; i += kQAll) ready[i] = 0;
+    if (tid == 0) ready[kFReadyCap] = 0;
   }
 }
 
 // Dynamic shared memory: the two stage slots, which also hold the plan's
 // histogram (max_adapters <= 16384 ints) before the first stage.
-constexpr int kQDyn = 2 * kQSlotBytes;
+constexpr int kQDyn = kQNS * kQSlotBytes;
 static_assert(4 * 16384 <= kQDyn, "histogram");
 
 template <int DT, int WF>
