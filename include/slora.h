@@ -100,21 +100,23 @@ typedef enum {
 typedef enum {
   SLORA_DECODE_AUTO = 0,       /* the library's choice: 16-bit pools run calls of
                                   up to 16 tokens as one CTA per token (plain
-                                  loads, no scratch: a latency-bound batch);
-                                  other calls of up to 1024 tokens take STREAM,
-                                  larger ones SPLIT                              */
+                                  loads, no scratch: a latency-bound batch),
+                                  17..256 tokens on STREAM and larger calls on
+                                  SPLIT; e4m3 pools take STREAM up to 1024
+                                  tokens                                         */
   SLORA_DECODE_SPLIT = 1,      /* always three kernels: segment build, shrink,
                                   expand                                         */
   SLORA_DECODE_FUSED = 2,      /* one persistent kernel with a bulk-copy ring for
                                   calls of up to 1024 tokens (every CTA builds the
                                   segment table, then the shrink and expand tasks
                                   in one launch); SPLIT above that               */
-  SLORA_DECODE_STREAM = 3      /* one kernel of independent tasks for calls of up
-                                  to 1024 tokens: every CTA plans the call, then
-                                  claims shrink tasks and, after them, expand
-                                  tasks from one counter; weights stream from the
-                                  pages into registers with plain 16-byte loads.
-                                  SPLIT above 1024 tokens                        */
+  SLORA_DECODE_STREAM = 3      /* one kernel of streaming stages for calls of up
+                                  to 1024 tokens: every CTA plans the call and
+                                  takes an equal share of the shrink tasks, then
+                                  of the expand stages; a producer warp moves each
+                                  stage's rank rows from the pages by bulk copies,
+                                  the shrink runs on mma.sync.  SPLIT above 1024
+                                  tokens                                         */
 } slora_decode_path_t;
 
 /* How a pool stores adapter weights in its pages. */

@@ -213,11 +213,11 @@ def test_bad_token_is_skipped_and_reported(T):
 
 @pytest.mark.parametrize("cfg", [1, 2])
 def test_full_size_configs_stream(cfg):
-    """The LLaMA-7B and LLaMA-13B decode layers on the default path (one kernel
-    of streaming tasks), every output element against the oracle, and a
-    repeated call bit-identical."""
+    """The LLaMA-7B and LLaMA-13B decode layers on the streaming-stage kernel
+    (the default for the 256-token layer), every output element against the
+    oracle, and a repeated call bit-identical."""
     w = W.config(cfg)
-    pb = H.PoolBuild(w)
+    pb = H.PoolBuild(w, decode_path=G.SLORA_DECODE_STREAM)
     assert G.slora_decode_kernels(pb.h, w.T) == 1
     ten = H.Tensors(w)
     _run_delta(pb, ten, w)
