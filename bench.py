@@ -76,8 +76,9 @@ def bf16_sustained():
 # B200's 1.965 GHz): longer than the host takes to enqueue one step.
 HOLD_CYCLES = 200_000
 
-KERNEL_SOURCE = {"delta": "fused.cu", "shrink": "bgmv.cu", "expand": "bgmv.cu", "segments": "bgmv.cu",
-                 "sgmv_shrink": "sgmv.cu", "sgmv_expand": "sgmv.cu"}
+KERNEL_SOURCE = {"stream": "stream.cu", "fused": "fused.cu", "token": "token.cu", "shrink": "bgmv.cu",
+                 "expand": "bgmv.cu", "segments": "bgmv.cu", "sgmv_shrink": "sgmv.cu", "sgmv_expand": "sgmv.cu",
+                 "linear": "linear.cu"}
 
 
 def source_sha(name: str) -> str:
@@ -222,7 +223,7 @@ class DecodeRun:
     grouped expand."""
     FUSED_MAX_T = 1024
 
-    def __init__(self, w, path="auto", weights="16"):
+    def __init__(self, w, path="auto", weights="16", pool="all"):
         import torch
 
         import gather_lora_paged_b200 as G
@@ -231,10 +232,17 @@ class DecodeRun:
         self.wbytes = 1 if weights == "e4m3" else 2
         dp = {"auto": G.SLORA_DECODE_AUTO, "split": G.SLORA_DECODE_SPLIT, "fused": G.SLORA_DECODE_FUSED,
               "stream": G.SLORA_DECODE_STREAM}[path]
-        self.pb = H.PoolBuild(w, decode_path=dp,
-                              weight_format=G.SLORA_WEIGHTS_E4M3 if weights == "e4m3" else G.SLORA_WEIGHTS_16)
-        fused = G.slora_decode_kernels(self.pb.h, w.T) == 1
-        self.phases = ("delta",) if fused else ("segments", "shrink", "expand")
+        wf = G.SLORA_WEIGHTS_E4M3 if weights == "e4m3" else G.SLORA_WEIGHTS_16
+        kw = {}
+        if pool == "touched":  # only the batch's adapters: the same kernel work in a smaller pool
+            t = sorted(set(w.touched().tolist()))
+            d = G.make_desc(w.dtype, [p.d_in for p in w.projs], [p.d_out for p in w.projs], w.n_adapters,
+                            int(w.ranks.max()), 1, w.page_elems, 0, weight_format=wf)
+            kw = {"resident": t, "n_pages": int(sum(G.slora_pages_for_rank(d, int(w.ranks[a])) for a in t))}
+        self.pb = H.PoolBuild(w, decode_path=dp, weight_format=wf, **kw)
+        kind = G.slora_decode_kind(self.pb.h, w.T)
+        self.phases = {G.SLORA_KIND_TOKEN: ("token",), G.SLORA_KIND_STREAM: ("stream",),
+                       G.SLORA_KIND_FUSED: ("fused",)}.get(kind, ("segments", "shrink", "expand"))
         self.ncu_names = self.phases
         self.ten = H.Tensors(w)
         self.d_idx = torch.from_numpy(w.idx).cuda()
@@ -304,7 +312,7 @@ def run_ours(args, rank, world):
         return run_mixed(args, rank, world, w)
     if args.linear:
         return run_linear(args, rank, world, w)
-    R = PrefillRun(w) if args.config == 3 else DecodeRun(w, path=args.path, weights=args.weights)
+    R = PrefillRun(w) if args.config == 3 else DecodeRun(w, path=args.path, weights=args.weights, pool=args.pool)
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -463,6 +471,8 @@ def run_ours(args, rank, world):
                    else W.DTYPE_NAME[w.dtype],
                    "accumulate": "f32", "l2": "flushed before every step (256 MiB write)",
                    "host_enqueue": "not timed: a ~100 us spin kernel precedes each step's start event",
+                   "pool": "the batch's adapters only" if getattr(args, "pool", "all") == "touched"
+                   else "every adapter of the workload",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": names[i_dom], "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm,
@@ -559,8 +569,8 @@ def run_linear(args, rank, world, w):
                    "what": "y = x.W0 + (alpha/r)(x.A).B in one tcgen05 kernel per layer (base GEMM fused "
                            "with the delta)", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "linear", "achieved": tflops, "peak": peak,
-                     "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None, "peak_source": src,
-                     "flops_per_step": flops},
+                     "unit": "TFLOP/s", "frac": tflops / peak, "traffic": ncu_traffic(w.name, "linear"),
+                     "peak_source": src, "flops_per_step": flops},
         "lora_overhead": {"base_only_ms": res["base"], "with_delta_ms": ms,
                           "overhead_frac": ms / res["base"] - 1.0},
         "gpu_launches": 2 * K,
@@ -840,6 +850,9 @@ def main():
                          "build, shrink, expand) or the one persistent kernel")
     ap.add_argument("--linear", action="store_true",
                     help="--config 3: the whole linear layer (base GEMM + delta) in one kernel")
+    ap.add_argument("--pool", default="all", choices=["all", "touched"],
+                    help="decode: a pool of every adapter of the workload, or of the batch's adapters only "
+                         "(the same kernel work; smaller device footprint for profiler captures)")
     ap.add_argument("--weights", default="16", choices=["16", "e4m3"],
                     help="decode: adapter pages in the pool's 16-bit dtype or as e4m3 codes")
     ap.add_argument("--pagein", default="kernel", choices=["kernel", "memcpy"],

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libslora.so")
 SLORA_F16, SLORA_BF16 = 0, 1
 SLORA_PAGEIN_KERNEL, SLORA_PAGEIN_MEMCPY = 0, 1
 SLORA_DECODE_AUTO, SLORA_DECODE_SPLIT, SLORA_DECODE_FUSED, SLORA_DECODE_STREAM = 0, 1, 2, 3
+SLORA_KIND_NONE, SLORA_KIND_TOKEN, SLORA_KIND_STREAM, SLORA_KIND_FUSED, SLORA_KIND_SPLIT = 0, 1, 2, 3, 4
 SLORA_WEIGHTS_16, SLORA_WEIGHTS_E4M3 = 0, 1
 MAX_PROJ = 8
 
@@ -96,6 +97,7 @@ def lib():
         "slora_lora_delta_noalloc": ([P, I32, P, P, P, P, P, P, I32, P], I32),
         "slora_noalloc_scratch_bytes": ([], c_size_t),
         "slora_decode_kernels": ([P, I32], I32),
+        "slora_decode_kind": ([P, I32], I32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -362,6 +364,11 @@ def slora_pool_stats(pool: int) -> dict:
 def slora_decode_kernels(pool: int, T: int) -> int:
     """Kernels slora_lora_delta launches for T tokens on this pool (1 or 3)."""
     return int(lib().slora_decode_kernels(pool, int(T)))
+
+
+def slora_decode_kind(pool: int, T: int) -> int:
+    """SLORA_KIND_* of the kernels a decode call of T tokens takes."""
+    return int(lib().slora_decode_kind(pool, int(T)))
 
 
 def slora_set_phase_events(pool: int, events) -> None:

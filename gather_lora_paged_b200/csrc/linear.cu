@@ -75,8 +75,14 @@ struct LUnit {
   int row0, seg_end, a, r, k, c0, nc;
 };
 
+// Units run in groups of kLGroup token tiles x every (projection, chunk group):
+// the CTAs of one wave then share a few x tiles and W0 chunk groups, which
+// stay in L2 while each unit re-reads its x tile once per chunk.
+constexpr int kLGroup = 32;
 __device__ __forceinline__ void lunit(const LinParams& p, int n_tiles, int u, LUnit& U) {
-  const int tile = u % n_tiles, sgi = u / n_tiles;
+  const int g = u / (kLGroup * p.n_sg), base = g * kLGroup;
+  const int gm = min(kLGroup, n_tiles - base), i = u - base * p.n_sg;
+  const int tile = base + i % gm, sgi = i / gm;
   const int s = find_ge(p.tile_prefix, p.S, tile);
   U.row0 = p.seg_start[s] + (tile - p.tile_prefix[s]) * kBM;
   U.seg_end = p.seg_start[s + 1];

@@ -1158,6 +1158,14 @@ int32_t slora_decode_kernels(const slora_pool* P, int32_t T) {
   return token_path(P, T) || fused_path(P, T) || stream_path(P, T) ? 1 : 3;
 }
 
+int32_t slora_decode_kind(const slora_pool* P, int32_t T) {
+  if (!P || T <= 0) return SLORA_KIND_NONE;
+  if (token_path(P, T)) return SLORA_KIND_TOKEN;
+  if (stream_path(P, T)) return SLORA_KIND_STREAM;
+  if (fused_path(P, T)) return SLORA_KIND_FUSED;
+  return SLORA_KIND_SPLIT;
+}
+
 slora_status_t slora_check_batch(const slora_pool* Pc, const int32_t* idx_host, int32_t T) {
   slora_pool* P = const_cast<slora_pool*>(Pc);
   if (!P) return SLORA_ERR_INVALID_ARG;

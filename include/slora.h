@@ -460,6 +460,19 @@ slora_status_t slora_lora_delta_noalloc(slora_pool* pool, int32_t n, const int32
  * build, shrink, expand); 0 for T <= 0 or a NULL pool.  Host only. */
 int32_t slora_decode_kernels(const slora_pool* pool, int32_t T);
 
+/* Which kernels slora_lora_delta launches for a call of T tokens on this pool
+ * (the AUTO choice resolved): one CTA per token, the streaming-stage kernel,
+ * the persistent bulk-copy kernel, or segment build + shrink + expand; NONE
+ * for T <= 0 or a NULL pool.  Host only. */
+typedef enum {
+  SLORA_KIND_NONE = 0,
+  SLORA_KIND_TOKEN = 1,
+  SLORA_KIND_STREAM = 2,
+  SLORA_KIND_FUSED = 3,
+  SLORA_KIND_SPLIT = 4
+} slora_decode_kind_t;
+int32_t slora_decode_kind(const slora_pool* pool, int32_t T);
+
 /* Size in bytes of the fixed scratch array used by slora_lora_delta_noalloc. */
 size_t slora_noalloc_scratch_bytes(void);
 

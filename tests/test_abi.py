@@ -504,5 +504,14 @@ def test_decode_path_policy(fmt):
                       decode_path=path, weight_format=fmt)
         for T, k in cases.items():
             assert G.slora_decode_kernels(pool.h, T) == k, (path, T)
+            kind = G.slora_decode_kind(pool.h, T)
+            assert (kind == G.SLORA_KIND_SPLIT) == (k == 3), (path, T, kind)
+            if path == G.SLORA_DECODE_STREAM and T <= 1024:
+                assert kind == G.SLORA_KIND_STREAM
+            if path == G.SLORA_DECODE_FUSED and T <= 1024:
+                assert kind == G.SLORA_KIND_FUSED
+            if path == G.SLORA_DECODE_AUTO and T <= 16 and fmt == G.SLORA_WEIGHTS_16:
+                assert kind == G.SLORA_KIND_TOKEN
         assert G.slora_decode_kernels(pool.h, 0) == 0
+        assert G.slora_decode_kind(pool.h, 0) == G.SLORA_KIND_NONE
         pool.close()
