@@ -59,7 +59,7 @@ struct QPlan {
   int seg_rank[kFSegCap];
   int shr_pre[kFSegCap + 1];    // shrink tasks before each segment
   int exp_pre[kFSegCap + 1];    // expand tasks before each segment
-  int exp_spre[kFSegCap + 1];   // expand stages before each segment (ceil(r / 8) per task)
+  int exp_cpre[kFSegCap + 1];   // expand cost units before each segment (expand_task_cost)
   int perm[kFMaxT];             // token of each position
 };
 
@@ -116,6 +116,16 @@ __device__ __forceinline__ int shrink_tasks(const BgmvParams& p, int n, int r) {
     c += cdiv_i(p.group[g].n * r, kQRB) * cdiv_i(p.group[g].d_in, kQKT) * ntt;
   return c;
 }
+// Cost of an expand task in units for balancing the CTAs' shares: per stage
+// (ceil(r / 8) of them) a fixed part kQEW plus the task's token class (1, 2 or
+// 4: its FMA work).  Only a segment's last token group can be partial, so all
+// (slot, output chunk) blocks of a segment cost the same.
+constexpr int kQEW = 2;
+__device__ __forceinline__ int etok_class(int nt) { return nt <= 1 ? 1 : (nt == 2 ? 2 : 4); }
+__device__ __forceinline__ int expand_block_cost(int n, int r) {
+  const int full = n / kQETok, rem = n - full * kQETok;
+  return cdiv_i(r, 8) * (full * (kQEW + 4) + (rem ? kQEW + etok_class(rem) : 0));
+}
 __device__ __forceinline__ int expand_tasks(const BgmvParams& p, int n) {
   int c = 0;
   const int ntg = cdiv_i(n, kQETok);
@@ -163,7 +173,7 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
   const int E = cdiv_i(MA, kQThreads);
   const int a0 = worker ? min(tid * E, MA) : MA, a1 = min(a0 + E, MA);
   int4 c = make_int4(0, 0, 0, 0);  // tokens, segments, shrink tasks, expand tasks
-  int cs = 0;                      // expand stages
+  int cs = 0;                      // expand cost units
   for (int a = a0; a < a1; ++a) {
     const int h = hist[a];
     if (h == 0) continue;
@@ -173,7 +183,7 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     c.y += 1;
     c.z += shrink_tasks(p, n, r);
     c.w += ne;
-    cs += ne * cdiv_i(r, 8);
+    cs += ne / cdiv_i(n, kQETok) * expand_block_cost(n, r);
   }
   int4 tot;
   const int4 base = block_exscan4(c, &tot, sh4);
@@ -191,19 +201,19 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     P.seg_rank[sb] = r;
     P.shr_pre[sb] = bs;
     P.exp_pre[sb] = be;
-    P.exp_spre[sb] = bst;
+    P.exp_cpre[sb] = bst;
     ++sb;
     cb += n;
     bs += shrink_tasks(p, n, r);
     be += ne;
-    bst += ne * cdiv_i(r, 8);
+    bst += ne / cdiv_i(n, kQETok) * expand_block_cost(n, r);
   }
   if (tid == 0) {
     P.S = tot.y;
     P.seg_start[tot.y] = tot.x;
     P.shr_pre[tot.y] = tot.z;
     P.exp_pre[tot.y] = tot.w;
-    P.exp_spre[tot.y] = tot_s;
+    P.exp_cpre[tot.y] = tot_s;
   }
   __syncthreads();
   // Stable scatter, one chunk of kQThreads tokens at a time: a token's place
@@ -492,19 +502,24 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
 }
 
 // The CTA's stages: its shrink tasks [sh0, sh_end) (an equal share of the
-// count), then the expand tasks whose first stage falls in its equal share of
-// all expand stages.
+// count), then the expand tasks whose cost position (expand cost units before
+// the task) falls in its equal share of all expand cost.
 __device__ __forceinline__ int first_expand_task(const QPlan& P, const BgmvParams& p, int e0) {
   const int S = P.S;
-  if (S == 0 || e0 >= P.exp_spre[S]) return P.exp_pre[S];
-  const int s = find_seg(P.exp_spre, S, e0);
-  const int ns = cdiv_i(P.seg_rank[s], kQRB);
-  const int loc = cdiv_i(e0 - P.exp_spre[s], ns);
-  return P.exp_pre[s] + loc;  // loc may equal the segment's task count: the next segment's first
+  if (S == 0 || e0 >= P.exp_cpre[S]) return P.exp_pre[S];
+  const int s = find_seg(P.exp_cpre, S, e0);
+  const int n = P.seg_start[s + 1] - P.seg_start[s], r = P.seg_rank[s], ntg = cdiv_i(n, kQETok);
+  const int bc = expand_block_cost(n, r), full = cdiv_i(r, 8) * (kQEW + 4);
+  const int off = e0 - P.exp_cpre[s], blk = off / bc;
+  const int tg = cdiv_i(off - blk * bc, full);  // task tg of a block starts tg full groups in
+  // tg may equal ntg: the next block's first task (or the next segment's)
+  return P.exp_pre[s] + blk * ntg + tg;
 }
 __device__ __forceinline__ int expand_first_stage(const QPlan& P, int te) {
   const int s = find_seg(P.exp_pre, P.S, te);
-  return P.exp_spre[s] + (te - P.exp_pre[s]) * cdiv_i(P.seg_rank[s], kQRB);
+  const int n = P.seg_start[s + 1] - P.seg_start[s], r = P.seg_rank[s], ntg = cdiv_i(n, kQETok);
+  const int q = te - P.exp_pre[s], blk = q / ntg, tg = q - blk * ntg;
+  return P.exp_cpre[s] + blk * expand_block_cost(n, r) + tg * cdiv_i(r, 8) * (kQEW + 4);
 }
 
 // The producer's walk over the CTA's tasks: the current task's fields kept
@@ -515,7 +530,7 @@ __device__ __forceinline__ int expand_first_stage(const QPlan& P, int te) {
 struct QCursor {
   QTask t;
   int task;   // global task index (shrink < n_shr <= expand)
-  int stage;  // expand: index of the task's first stage among all expand stages
+  int stage;  // expand: the task's cost position (expand cost units before it)
   int n, r;   // the segment's tokens and rank
   int nb, nc, ntt;  // shrink: row blocks and chunks of the group, token tiles
   int ne, ntg, ns;  // expand: output chunks of the slot, token groups, stages per task
@@ -548,7 +563,7 @@ struct QCursor {
     if (t.shrink == 0) {
       if (++t.sub < ns) return true;
       t.sub = 0;
-      stage += ns;
+      stage += ns * (kQEW + etok_class(min(kQETok, n - t.w * kQETok)));
       ++task;
       if (++t.w < ntg) return true;
       t.w = 0;
@@ -639,7 +654,7 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     // lane % 4 and lane % 4 + 4 of it)
     const int G = gridDim.x, bx = blockIdx.x;
     const int sh0 = (int)((int64_t)bx * n_shr / G), sh_end = (int)((int64_t)(bx + 1) * n_shr / G);
-    const int n_es = P.exp_spre[S];
+    const int n_es = P.exp_cpre[S];
     const int e0 = (int)((int64_t)bx * n_es / G), e_end = (int)((int64_t)(bx + 1) * n_es / G);
     QCursor cur;
     bool in_shrink = sh0 < sh_end;
