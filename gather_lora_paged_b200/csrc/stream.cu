@@ -61,6 +61,8 @@ struct QPlan {
   int exp_pre[kFSegCap + 1];    // expand tasks before each segment
   int exp_cpre[kFSegCap + 1];   // expand cost units before each segment (expand_task_cost)
   int perm[kFMaxT];             // token of each position
+  int stab[kQMaxR + 1];         // shrink tasks per token tile of an adapter of rank r
+  int sum_ne;                   // output chunks over the call's slots
 };
 
 // Reads of data written earlier in this kernel by other CTAs (L2, not L1).
@@ -109,13 +111,6 @@ __device__ __forceinline__ void unpack8_q8(const uint2& v, float* f) {
   }
 }
 
-__device__ __forceinline__ int shrink_tasks(const BgmvParams& p, int n, int r) {
-  int c = 0;
-  const int ntt = cdiv_i(n, kQSTok);
-  for (int g = 0; g < p.n_groups; ++g)
-    c += cdiv_i(p.group[g].n * r, kQRB) * cdiv_i(p.group[g].d_in, kQKT) * ntt;
-  return c;
-}
 // Cost of an expand task in units for balancing the CTAs' shares: per stage
 // (ceil(r / 8) of them) a fixed part kQEW plus the task's token class (1, 2 or
 // 4: its FMA work).  Only a segment's last token group can be partial, so all
@@ -125,12 +120,6 @@ __device__ __forceinline__ int etok_class(int nt) { return nt <= 1 ? 1 : (nt == 
 __device__ __forceinline__ int expand_block_cost(int n, int r) {
   const int full = n / kQETok, rem = n - full * kQETok;
   return cdiv_i(r, 8) * (full * (kQEW + 4) + (rem ? kQEW + etok_class(rem) : 0));
-}
-__device__ __forceinline__ int expand_tasks(const BgmvParams& p, int n) {
-  int c = 0;
-  const int ntg = cdiv_i(n, kQETok);
-  for (int k = 0; k < p.n_slots; ++k) c += cdiv_i(p.slot[k].d_out, kQECols) * ntg;
-  return c;
 }
 
 // ---------------------------------------------------------------------------
@@ -144,6 +133,16 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
   const bool worker = tid < kQThreads;  // token work: the first kQThreads threads
   const int T = p.T, MA = p.pool.max_adapters;
   for (int a = tid; a < MA; a += blockDim.x) hist[a] = 0;
+  if (tid <= kQMaxR) {  // per-call constants of the task counts
+    int c = 0;
+    for (int g = 0; g < p.n_groups; ++g) c += cdiv_i(p.group[g].n * tid, kQRB) * cdiv_i(p.group[g].d_in, kQKT);
+    P.stab[tid] = c;
+  }
+  if (tid == kQMaxR + 1) {
+    int c = 0;
+    for (int k = 0; k < p.n_slots; ++k) c += cdiv_i(p.slot[k].d_out, kQECols);
+    P.sum_ne = c;
+  }
   __syncthreads();
   int key[kFMaxT / kQThreads];
 #pragma unroll
@@ -174,16 +173,16 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
   const int a0 = worker ? min(tid * E, MA) : MA, a1 = min(a0 + E, MA);
   int4 c = make_int4(0, 0, 0, 0);  // tokens, segments, shrink tasks, expand tasks
   int cs = 0;                      // expand cost units
+  const int sum_ne = P.sum_ne;
   for (int a = a0; a < a1; ++a) {
     const int h = hist[a];
     if (h == 0) continue;
     const int n = h & ((1 << kRankShift) - 1), r = h >> kRankShift;
-    const int ne = expand_tasks(p, n);
     c.x += n;
     c.y += 1;
-    c.z += shrink_tasks(p, n, r);
-    c.w += ne;
-    cs += ne / cdiv_i(n, kQETok) * expand_block_cost(n, r);
+    c.z += P.stab[r] * cdiv_i(n, kQSTok);
+    c.w += sum_ne * cdiv_i(n, kQETok);
+    cs += sum_ne * expand_block_cost(n, r);
   }
   int4 tot;
   const int4 base = block_exscan4(c, &tot, sh4);
@@ -195,7 +194,6 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     hist[a] = cb;  // becomes the scatter cursor
     if (h == 0) continue;
     const int n = h & ((1 << kRankShift) - 1), r = h >> kRankShift;
-    const int ne = expand_tasks(p, n);
     P.seg_start[sb] = cb;
     P.seg_adapter[sb] = a;
     P.seg_rank[sb] = r;
@@ -204,9 +202,9 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     P.exp_cpre[sb] = bst;
     ++sb;
     cb += n;
-    bs += shrink_tasks(p, n, r);
-    be += ne;
-    bst += ne / cdiv_i(n, kQETok) * expand_block_cost(n, r);
+    bs += P.stab[r] * cdiv_i(n, kQSTok);
+    be += sum_ne * cdiv_i(n, kQETok);
+    bst += sum_ne * expand_block_cost(n, r);
   }
   if (tid == 0) {
     P.S = tot.y;
