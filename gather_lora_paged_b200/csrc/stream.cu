@@ -290,7 +290,7 @@ __device__ __forceinline__ QTask decode_task(const BgmvParams& p, const QPlan& P
 constexpr int kQRowBytes = 2 * kQKT + 64;
 constexpr int kQSlotBytes = kQRB * kQRowBytes;
 constexpr int kQNS = 2;                            // stage slots (copies run up to kQNS - 1 stages ahead)
-constexpr int kQND = 2 * kQNS;                     // descriptor ring
+constexpr int kQND = 8;                            // descriptor ring (published two stages ahead)
 constexpr int kQCTAs = kQNS <= 2 ? 2 : 1;          // resident CTAs per SM
 constexpr int kQCons = 8;                          // consumer warps
 constexpr int kQAll = (kQCons + 1) * 32;           // + the producer warp
@@ -410,7 +410,6 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
       S2.t[(int64_t)(pos0 + m) * S2.t_rs + (int64_t)k2 * S2.t_ns + c] = sum;
     }
   }
-  bar_consumers();  // red is rewritten by the next shrink stage
 }
 
 // ---------------------------------------------------------------------------
@@ -614,7 +613,7 @@ __device__ __forceinline__ int stage_bytes(const BgmvParams& p, const QPlan& P, 
 template <int DT, int WF>
 __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant__ BgmvParams p) {
   __shared__ QPlan P;
-  __shared__ __align__(16) float red[kQCons * 64];
+  __shared__ __align__(16) float red[2][kQCons * 64];  // by shrink-stage parity: one barrier a stage
   __shared__ __align__(16) float tS[kQETok * kQMaxR];
   __shared__ __align__(16) int ck[kQThreads];
   __shared__ int4 sh4[32];
@@ -718,9 +717,9 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
       }
     };
     const unsigned char* pool = reinterpret_cast<const unsigned char*>(p.pool.pool);
-    // Descriptors go to a ring of 4 as soon as a stage is known (the consumers
-    // load its x from it); copies go to the stage's slot once the stage two
-    // before it has released the slot.
+    // Descriptors go to a ring of kQND two stages before their stage (the
+    // consumers load x from them); copies go to the stage's slot once the stage
+    // kQNS before it has released the slot.
     auto publish = [&](int n, const QTask& tt) {
       if (lane == 0) sdesc[n % kQND] = tt;
       __syncwarp();
@@ -743,33 +742,42 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
         run_n = 0;
       }
     };
+    // the cursor runs two stages ahead of the copies: stage n + 2 is published
+    // while stage n's copies wait for their slot
+    auto advance = [&]() {
+      if (t.shrink < 0) return;
+      const bool more = cur.next(p, P);
+      if (in_shrink && (!more || cur.task >= sh_end)) {  // the shrink share is done: the expand share
+        in_shrink = false;
+        cur.start(p, P, n_shr + first_expand_task(P, p, e0), n_shr, total);
+      } else if (!more) {
+        t.shrink = -1;
+      }
+      if (!in_share()) t.shrink = -1;
+    };
+    QTask q0 = t;  // stage n
+    publish(0, q0);
+    advance();
+    QTask q1 = t;  // stage n + 1
+    publish(1, q1);
+    advance();     // the cursor: stage n + 2
     Pieces pc_cur, pc_next;
-    resolve(t, pc_cur);
-    prefetch_xy(t);
-    publish(0, t);
+    resolve(q0, pc_cur);
+    prefetch_xy(q0);
     int n = 0;
     for (;; ++n) {
       const int slot = n % kQNS;
-      const QTask tn = t;  // stage n
-      if (tn.shrink >= 0) {  // stage n + 1: known, published, its page ids on the way
-        const bool more = cur.next(p, P);
-        if (in_shrink && (!more || cur.task >= sh_end)) {  // the shrink share is done: the expand share
-          in_shrink = false;
-          cur.start(p, P, n_shr + first_expand_task(P, p, e0), n_shr, total);
-        } else if (!more) {
-          t.shrink = -1;
-        }
-        if (!in_share()) t.shrink = -1;
-        publish(n + 1, t);
-        resolve(t, pc_next);
-        prefetch_xy(t);
+      if (q0.shrink >= 0) {
+        publish(n + 2, t);
+        resolve(q1, pc_next);  // stage n + 1: its page ids on the way, its x / y rows to L2
+        prefetch_xy(q1);
       }
       if (n >= kQNS) {  // stage n - kQNS has released the slot (its descriptor is still in the ring)
         mbar_wait(&empty[slot], (n / kQNS - 1) & 1, p.pool.err);
         count(sdesc[(n - kQNS) % kQND], sdesc[(n - kQNS + 1) % kQND]);
       }
-      if (tn.shrink < 0) break;
-      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)stage_bytes<WF>(p, P, tn));
+      if (q0.shrink < 0) break;
+      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)stage_bytes<WF>(p, P, q0));
       __syncwarp();
       unsigned char* dst = ring + slot * kQSlotBytes;
 #pragma unroll
@@ -778,6 +786,9 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
           bulk_g2s(dst + pc_cur.dso[h], pool + ((int64_t)pc_cur.pg[h] << (p.pool.page_shift + 1)) + pc_cur.ipo[h],
                    (uint32_t)pc_cur.nb[h], &full[slot]);
       pc_cur = pc_next;
+      q0 = q1;
+      q1 = t;
+      advance();
     }
     // the last stages are counted once released (stage n is the end marker)
     for (int k = max(0, n - kQNS + 1); k < n; ++k) {
@@ -788,6 +799,7 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     // ---- consumer warps
     float acc[kQETok][8];
     uint4 xq[8];
+    int nsh = 0;  // shrink stages so far
     mbar_wait(&dready[0], 0, p.pool.err);
     QTask t = sdesc[0];
     load_x(p, P, t, xq);
@@ -797,7 +809,7 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
       mbar_wait(&full[slot], (n / kQNS) & 1, p.pool.err);
       const unsigned char* sl = ring + slot * kQSlotBytes;
       if (t.shrink) {
-        shrink_stage<DT, WF>(p, P, red, t, sl, xq);
+        shrink_stage<DT, WF>(p, P, red[nsh++ & 1], t, sl, xq);
       } else {
         const int nt = min(kQETok, P.seg_start[t.s + 1] - P.seg_start[t.s] - t.w * kQETok);
         if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, acc);
