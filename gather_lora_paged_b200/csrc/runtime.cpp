@@ -469,9 +469,10 @@ bool fused_path(const slora_pool* P, int T) {
 // Whether a decode call of T tokens runs as the one kernel of streaming stages.
 // AUTO takes it for 17..kStreamAutoMaxT tokens (16-bit) and for every call of
 // an e4m3 pool up to kFMaxT; above kStreamAutoMaxT 16-bit calls take the
-// three-kernel path, the faster of the two on B200 at 512 tokens (LLaMA-13B
-// layer, Zipf 1.2 ids) while the streaming kernel is the faster at 256.
-constexpr int kStreamAutoMaxT = 256;
+// three-kernel path, the faster of the two on B200 at 1024 tokens (LLaMA-70B
+// layer, ranks up to 128) while the streaming kernel is the faster at 256 and
+// 512 (LLaMA-7B and -13B layers).
+constexpr int kStreamAutoMaxT = 512;
 bool stream_path(const slora_pool* P, int T) {
   if (T > kFMaxT) return false;
   if (P->d.decode_path == SLORA_DECODE_STREAM) return true;

@@ -101,7 +101,7 @@ typedef enum {
   SLORA_DECODE_AUTO = 0,       /* the library's choice: 16-bit pools run calls of
                                   up to 16 tokens as one CTA per token (plain
                                   loads, no scratch: a latency-bound batch),
-                                  17..256 tokens on STREAM and larger calls on
+                                  17..512 tokens on STREAM and larger calls on
                                   SPLIT; e4m3 pools take STREAM up to 1024
                                   tokens                                         */
   SLORA_DECODE_SPLIT = 1,      /* always three kernels: segment build, shrink,
