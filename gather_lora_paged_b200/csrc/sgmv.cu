@@ -691,6 +691,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
         }
       }
       tc_fence_before();
+      fence_async_smem();  // the tile's new y values, for a TMA store
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(&a_empty[as])) : "memory");
@@ -701,18 +702,31 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
       // cannot hang the others)
       ok = bar_wait(&e_sync, j & 1, p.pool.err);
       if (!ok) break;
-      // coalesced stores: thread -> (row it * R + etid / 16, 16-byte chunk etid % 16)
-      constexpr int kRowsPerIt = 32 * kEpiWarps / 16;
-      const int q16 = etid & 15, cb = q16 >> 3, cj = q16 & 7;
-      const int col = n0 + q16 * 8;
+      if (row0 + kBM <= seg1) {
+        // the whole tile belongs to the segment: one TMA store per box (clipped
+        // at d_out); the slot is released once the copy has read it
+        if (etid == 0) {
+          tma_store_2d_hint(&p.ymap[e.k], n0, row0, yt, pol_y);
+          if (n0 + 64 < L.d_out) tma_store_2d_hint(&p.ymap[e.k], n0 + 64, row0, yt + kYTileBytes / 2, pol_y);
+          bulk_commit();
+          bulk_wait_read();
+        }
+      } else {
+        // the segment ends inside the tile (its other rows are another
+        // segment's): coalesced stores of this segment's rows, thread ->
+        // (row it * R + etid / 16, 16-byte chunk etid % 16)
+        constexpr int kRowsPerIt = 32 * kEpiWarps / 16;
+        const int q16 = etid & 15, cb = q16 >> 3, cj = q16 & 7;
+        const int col = n0 + q16 * 8;
 #pragma unroll 4
-      for (int it = 0; it < kBM / kRowsPerIt; ++it) {
-        const int row = it * kRowsPerIt + (etid >> 4);
-        const int tok = row0 + row;
-        if (tok < seg1 && col < L.d_out) {
-          const uint4 v = *reinterpret_cast<const uint4*>(yt + cb * (kYTileBytes / 2) + row * 128 +
-                                                          ((cj ^ (row & 7)) << 4));
-          st_global_v4_hint(L.y + (int64_t)tok * L.ldy + col, v, pol_y);
+        for (int it = 0; it < kBM / kRowsPerIt; ++it) {
+          const int row = it * kRowsPerIt + (etid >> 4);
+          const int tok = row0 + row;
+          if (tok < seg1 && col < L.d_out) {
+            const uint4 v = *reinterpret_cast<const uint4*>(yt + cb * (kYTileBytes / 2) + row * 128 +
+                                                            ((cj ^ (row & 7)) << 4));
+            st_global_v4_hint(L.y + (int64_t)tok * L.ldy + col, v, pol_y);
+          }
         }
       }
       fence_async_smem();  // generic-proxy writes of the slot before the next TMA fill
@@ -721,6 +735,7 @@ __global__ void __launch_bounds__(kExpandThreads, 1) k_sgmv_expand(const __grid_
       code = ecur_next(p, e);
     }
   }
+  if (tid == 64) bulk_wait_all();  // the epilogue's TMA stores are complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, kAcc * kEN);

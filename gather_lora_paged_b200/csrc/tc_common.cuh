@@ -81,6 +81,21 @@ __device__ __forceinline__ void tma_gather4_hint(void* dst, const CUtensorMap* m
       "l"(map), "r"(0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(su32(b)), "l"(pol)
       : "memory");
 }
+// Tiled TMA store of one box from shared memory (bulk-group completion): the
+// writes are done once the issuing thread's bulk_wait_read / bulk_wait_all
+// returns; coordinates are never negative here.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, int c0, int c1, const void* src,
+                                                  uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(map),
+      "r"(c0), "r"(c1), "r"(su32(src)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of every committed store have been read
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// every committed store is complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void st_global_v4_hint(void* ptr, uint4 v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w), "l"(pol)
