@@ -115,7 +115,7 @@ __device__ __forceinline__ void unpack8_q8(const uint2& v, float* f) {
 // (ceil(r / 8) of them) a fixed part kQEW plus the task's token class (1, 2 or
 // 4: its FMA work).  Only a segment's last token group can be partial, so all
 // (slot, output chunk) blocks of a segment cost the same.
-constexpr int kQEW = 2;
+constexpr int kQEW = 1;
 __device__ __forceinline__ int etok_class(int nt) { return nt <= 1 ? 1 : (nt == 2 ? 2 : 4); }
 __device__ __forceinline__ int expand_block_cost(int n, int r) {
   const int full = n / kQETok, rem = n - full * kQETok;
@@ -420,7 +420,7 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
 // L2 by the producer) and rounds.
 template <int DT, int WF, int NT>
 __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, const QTask& t,
-                             const unsigned char* slot, float (&acc)[kQETok][8]) {
+                             const unsigned char* slot, float (&acc)[kQETok][8], int& tkey) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int s = t.s, a = P.seg_adapter[s], r = P.seg_rank[s];
   const int pos0 = P.seg_start[s] + t.w * kQETok;
@@ -434,6 +434,13 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
     for (int m = 0; m < NT; ++m)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[m][i] = 0.f;
+  }
+  // t of (segment, projection, token group) is the same for all of the
+  // projection's output chunks, which run back to back: filled once for them
+  // (key: segment < 1024, token group < 256, projection < 8; CTA-uniform)
+  const int key = (s * 256 + t.w) * 8 + t.u;
+  if (t.sub == 0 && key != tkey) {
+    tkey = key;
     if (tid == 0) {  // bounded wait for the shrink tasks of (s, x group)
       const GroupDev& G = p.group[L.group];
       const int need = cdiv_i(G.n * r, kQRB) * cdiv_i(G.d_in, kQKT) *
@@ -796,30 +803,51 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
       count(sdesc[k % kQND], sdesc[(k + 1) % kQND]);
     }
   } else {
-    // ---- consumer warps
-    float acc[kQETok][8];
-    uint4 xq[8];
-    int nsh = 0;  // shrink stages so far
+    // ---- consumer warps.  A CTA's stages are its shrink tasks, then its
+    // expand tasks: two loops, so that the x pieces (shrink) and the output
+    // accumulators (expand) never hold registers at the same time.
+    int n = 0;
     mbar_wait(&dready[0], 0, p.pool.err);
     QTask t = sdesc[0];
-    load_x(p, P, t, xq);
-    for (int n = 0;; ++n) {
+    {
+      uint4 xq[8];
+      // x pieces are the same for the rank-row blocks of one (segment, x group,
+      // d_in chunk, token tile), which run back to back: loaded once for them
+      // (key: segment < 1024, tile < 128, chunk < 16, group < 8)
+      int xkey = -1;
+      auto x_for = [&](const QTask& tk) {
+        if (tk.shrink != 1) return;
+        const int k = ((tk.s * 128 + tk.w) * 16 + tk.c) * 8 + tk.u;
+        if (k != xkey) {
+          load_x(p, P, tk, xq);
+          xkey = k;
+        }
+      };
+      x_for(t);
+      for (; t.shrink == 1; ++n) {
+        const int slot = n % kQNS;
+        mbar_wait(&full[slot], (n / kQNS) & 1, p.pool.err);
+        shrink_stage<DT, WF>(p, P, red[n & 1], t, ring + slot * kQSlotBytes, xq);
+        // the next stage's descriptor (and x) before this slot is released
+        mbar_wait(&dready[(n + 1) % kQND], ((n + 1) / kQND) & 1, p.pool.err);
+        t = sdesc[(n + 1) % kQND];
+        x_for(t);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+    }
+    float acc[kQETok][8];
+    int tkey = -1;
+    for (; t.shrink == 0; ++n) {
       const int slot = n % kQNS;
-      if (t.shrink < 0) break;
       mbar_wait(&full[slot], (n / kQNS) & 1, p.pool.err);
       const unsigned char* sl = ring + slot * kQSlotBytes;
-      if (t.shrink) {
-        shrink_stage<DT, WF>(p, P, red[nsh++ & 1], t, sl, xq);
-      } else {
-        const int nt = min(kQETok, P.seg_start[t.s + 1] - P.seg_start[t.s] - t.w * kQETok);
-        if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, acc);
-        else if (nt == 2) expand_stage<DT, WF, 2>(p, P, tS, t, sl, acc);
-        else expand_stage<DT, WF, 4>(p, P, tS, t, sl, acc);
-      }
-      // the next stage's descriptor (and x) before this slot is released
+      const int nt = min(kQETok, P.seg_start[t.s + 1] - P.seg_start[t.s] - t.w * kQETok);
+      if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, acc, tkey);
+      else if (nt == 2) expand_stage<DT, WF, 2>(p, P, tS, t, sl, acc, tkey);
+      else expand_stage<DT, WF, 4>(p, P, tS, t, sl, acc, tkey);
       mbar_wait(&dready[(n + 1) % kQND], ((n + 1) / kQND) & 1, p.pool.err);
       t = sdesc[(n + 1) % kQND];
-      load_x(p, P, t, xq);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
     }
