@@ -467,17 +467,14 @@ bool fused_path(const slora_pool* P, int T) {
 }
 
 // Whether a decode call of T tokens runs as the one kernel of streaming stages.
-// AUTO takes it for 17..kStreamAutoMaxT tokens (16-bit) and for every call of
-// an e4m3 pool up to kFMaxT; above kStreamAutoMaxT 16-bit calls take the
-// three-kernel path, the faster of the two on B200 at 1024 tokens (LLaMA-70B
-// layer, ranks up to 128) while the streaming kernel is the faster at 256 and
-// 512 (LLaMA-7B and -13B layers).
-constexpr int kStreamAutoMaxT = 512;
+// AUTO takes it for 17..kFMaxT tokens (16-bit) and for every call of an e4m3
+// pool up to kFMaxT: on B200 it is the faster of the measured kernels at 256,
+// 512 and 1024 tokens (LLaMA-7B, -13B and -70B layers); larger 16-bit calls
+// take the three-kernel path, which has no token limit.
 bool stream_path(const slora_pool* P, int T) {
   if (T > kFMaxT) return false;
   if (P->d.decode_path == SLORA_DECODE_STREAM) return true;
-  if (P->d.decode_path != SLORA_DECODE_AUTO || token_path(P, T)) return false;
-  return P->e4m3() || T <= kStreamAutoMaxT;
+  return P->d.decode_path == SLORA_DECODE_AUTO && !token_path(P, T);
 }
 
 // The decode delta's kernels for a planned call (both phases): the one

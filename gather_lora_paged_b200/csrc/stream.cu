@@ -47,9 +47,11 @@ constexpr int kQSTok = 8;                     // tokens per shrink task (mma row
 constexpr int kQECols = 2048;                 // outputs per expand task: 256 per warp
 constexpr int kQETok = 4;                     // tokens per expand task
 constexpr int kQMaxR = 128;
+constexpr int kQExpChunk = 2;                 // expand tasks per claimed chunk
 static_assert(kQKT == kQWarps * 256 && kQECols == kQWarps * 256, "task shapes");
 // ready[] (scratch, zero between calls): per (segment, x group) counts of
-// finished shrink tasks, then at kFReadyCap the count of finished CTAs
+// finished shrink tasks, then at kFReadyCap the count of finished CTAs and at
+// kFReadyCap + 1 the counter the CTAs claim task chunks from
 
 // The call's plan, identical in every CTA.
 struct QPlan {
@@ -59,7 +61,6 @@ struct QPlan {
   int seg_rank[kFSegCap];
   int shr_pre[kFSegCap + 1];    // shrink tasks before each segment
   int exp_pre[kFSegCap + 1];    // expand tasks before each segment
-  int exp_cpre[kFSegCap + 1];   // expand cost units before each segment (expand_task_cost)
   int perm[kFMaxT];             // token of each position
   int stab[kQMaxR + 1];         // shrink tasks per token tile of an adapter of rank r
   int sum_ne;                   // output chunks over the call's slots
@@ -109,17 +110,6 @@ __device__ __forceinline__ void unpack8_q8(const uint2& v, float* f) {
     h2x2f(e4m3x2_to_16<SLORA_F16>(w[i] & 0xffffu), f[4 * i], f[4 * i + 1]);
     h2x2f(e4m3x2_to_16<SLORA_F16>(w[i] >> 16), f[4 * i + 2], f[4 * i + 3]);
   }
-}
-
-// Cost of an expand task in units for balancing the CTAs' shares: per stage
-// (ceil(r / 8) of them) a fixed part kQEW plus the task's token class (1, 2 or
-// 4: its FMA work).  Only a segment's last token group can be partial, so all
-// (slot, output chunk) blocks of a segment cost the same.
-constexpr int kQEW = 1;
-__device__ __forceinline__ int etok_class(int nt) { return nt <= 1 ? 1 : (nt == 2 ? 2 : 4); }
-__device__ __forceinline__ int expand_block_cost(int n, int r) {
-  const int full = n / kQETok, rem = n - full * kQETok;
-  return cdiv_i(r, 8) * (full * (kQEW + 4) + (rem ? kQEW + etok_class(rem) : 0));
 }
 
 // ---------------------------------------------------------------------------
@@ -172,7 +162,6 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
   const int E = cdiv_i(MA, kQThreads);
   const int a0 = worker ? min(tid * E, MA) : MA, a1 = min(a0 + E, MA);
   int4 c = make_int4(0, 0, 0, 0);  // tokens, segments, shrink tasks, expand tasks
-  int cs = 0;                      // expand cost units
   const int sum_ne = P.sum_ne;
   for (int a = a0; a < a1; ++a) {
     const int h = hist[a];
@@ -182,12 +171,9 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     c.y += 1;
     c.z += P.stab[r] * cdiv_i(n, kQSTok);
     c.w += sum_ne * cdiv_i(n, kQETok);
-    cs += sum_ne * expand_block_cost(n, r);
   }
   int4 tot;
   const int4 base = block_exscan4(c, &tot, sh4);
-  int tot_s;
-  int bst = block_exscan<false>(cs, &tot_s, sh1);
   int cb = base.x, sb = base.y, bs = base.z, be = base.w;
   for (int a = a0; a < a1; ++a) {
     const int h = hist[a];
@@ -199,19 +185,16 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     P.seg_rank[sb] = r;
     P.shr_pre[sb] = bs;
     P.exp_pre[sb] = be;
-    P.exp_cpre[sb] = bst;
     ++sb;
     cb += n;
     bs += P.stab[r] * cdiv_i(n, kQSTok);
     be += sum_ne * cdiv_i(n, kQETok);
-    bst += sum_ne * expand_block_cost(n, r);
   }
   if (tid == 0) {
     P.S = tot.y;
     P.seg_start[tot.y] = tot.x;
     P.shr_pre[tot.y] = tot.z;
     P.exp_pre[tot.y] = tot.w;
-    P.exp_cpre[tot.y] = tot_s;
   }
   __syncthreads();
   // Stable scatter, one chunk of kQThreads tokens at a time: a token's place
@@ -505,28 +488,7 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
   }
 }
 
-// The CTA's stages: its shrink tasks [sh0, sh_end) (an equal share of the
-// count), then the expand tasks whose cost position (expand cost units before
-// the task) falls in its equal share of all expand cost.
-__device__ __forceinline__ int first_expand_task(const QPlan& P, const BgmvParams& p, int e0) {
-  const int S = P.S;
-  if (S == 0 || e0 >= P.exp_cpre[S]) return P.exp_pre[S];
-  const int s = find_seg(P.exp_cpre, S, e0);
-  const int n = P.seg_start[s + 1] - P.seg_start[s], r = P.seg_rank[s], ntg = cdiv_i(n, kQETok);
-  const int bc = expand_block_cost(n, r), full = cdiv_i(r, 8) * (kQEW + 4);
-  const int off = e0 - P.exp_cpre[s], blk = off / bc;
-  const int tg = cdiv_i(off - blk * bc, full);  // task tg of a block starts tg full groups in
-  // tg may equal ntg: the next block's first task (or the next segment's)
-  return P.exp_pre[s] + blk * ntg + tg;
-}
-__device__ __forceinline__ int expand_first_stage(const QPlan& P, int te) {
-  const int s = find_seg(P.exp_pre, P.S, te);
-  const int n = P.seg_start[s + 1] - P.seg_start[s], r = P.seg_rank[s], ntg = cdiv_i(n, kQETok);
-  const int q = te - P.exp_pre[s], blk = q / ntg, tg = q - blk * ntg;
-  return P.exp_cpre[s] + blk * expand_block_cost(n, r) + tg * cdiv_i(r, 8) * (kQEW + 4);
-}
-
-// The producer's walk over the CTA's tasks: the current task's fields kept
+// The producer's walk over a chunk of tasks: the current task's fields kept
 // alongside the counts they run through, so that the next task follows with
 // a few increments (the same order decode_task assigns: shrink tasks by
 // segment, x group, d_in chunk, rank-row block, token tile; expand tasks by
@@ -534,7 +496,6 @@ __device__ __forceinline__ int expand_first_stage(const QPlan& P, int te) {
 struct QCursor {
   QTask t;
   int task;   // global task index (shrink < n_shr <= expand)
-  int stage;  // expand: the task's cost position (expand cost units before it)
   int n, r;   // the segment's tokens and rank
   int nb, nc, ntt;  // shrink: row blocks and chunks of the group, token tiles
   int ne, ntg, ns;  // expand: output chunks of the slot, token groups, stages per task
@@ -560,14 +521,12 @@ struct QCursor {
     if (t.shrink < 0) return;
     seg_fields(p, P);
     sub_fields(p);
-    if (t.shrink == 0) stage = expand_first_stage(P, tk - n_shr);
   }
   // the next stage; false past the end of the plan
   __device__ bool next(const BgmvParams& p, const QPlan& P) {
     if (t.shrink == 0) {
       if (++t.sub < ns) return true;
       t.sub = 0;
-      stage += ns * (kQEW + etok_class(min(kQETok, n - t.w * kQETok)));
       ++task;
       if (++t.w < ntg) return true;
       t.w = 0;
@@ -656,18 +615,32 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     // ---- producer warp: the CTA's stage sequence, page ids one stage ahead,
     // one bulk copy per page piece of a stage row (lane: row lane / 4, pieces
     // lane % 4 and lane % 4 + 4 of it)
-    const int G = gridDim.x, bx = blockIdx.x;
-    const int sh0 = (int)((int64_t)bx * n_shr / G), sh_end = (int)((int64_t)(bx + 1) * n_shr / G);
-    const int n_es = P.exp_cpre[S];
-    const int e0 = (int)((int64_t)bx * n_es / G), e_end = (int)((int64_t)(bx + 1) * n_es / G);
+    //
+    // The tasks are handed out in chunks of consecutive tasks: ksc shrink
+    // tasks (about two chunks per CTA, a multiple of 4 up to 16) or kQExpChunk
+    // expand tasks, all shrink chunks first.  CTA b
+    // takes chunk b, then chunks claimed from a counter, each claim made when
+    // the chunk before it starts, so that its answer is there when needed.
+    // Claims only grow, so a CTA runs all its shrink chunks before any expand
+    // chunk, and an expand task never waits on a shrink task queued behind it.
+    const int ksc = min(16, max(4, (n_shr / (2 * (int)gridDim.x) + 2) / 4 * 4));
+    const int n_sc = cdiv_i(n_shr, ksc);
+    const int n_chunks = n_sc + cdiv_i(total - n_shr, kQExpChunk);
+    int* claim = ready + kFReadyCap + 1;
+    int claimed = 0;  // lane 0: the chunk after the current one
+    int cend = 0;     // the current chunk's end (task index)
     QCursor cur;
-    bool in_shrink = sh0 < sh_end;
-    cur.start(p, P, in_shrink ? sh0 : n_shr + first_expand_task(P, p, e0), n_shr, total);
-    auto in_share = [&]() {
-      if (cur.t.shrink < 0) return false;
-      return cur.t.shrink ? cur.task < sh_end : cur.stage < e_end;
+    auto take = [&](int c) {
+      if (c >= n_chunks) {
+        cur.t.shrink = -1;
+        return;
+      }
+      const int f = c < n_sc ? c * ksc : n_shr + (c - n_sc) * kQExpChunk;
+      cend = c < n_sc ? min(f + ksc, n_shr) : min(f + kQExpChunk, total);
+      cur.start(p, P, f, n_shr, total);
+      if (lane == 0) claimed = (int)gridDim.x + atomicAdd(claim, 1);
     };
-    if (!in_share()) cur.t.shrink = -1;
+    take(blockIdx.x);
     QTask& t = cur.t;
     const int i = lane >> 2, qp = lane & 3;
     const int sh = p.pool.page_shift + WF;
@@ -754,13 +727,7 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     auto advance = [&]() {
       if (t.shrink < 0) return;
       const bool more = cur.next(p, P);
-      if (in_shrink && (!more || cur.task >= sh_end)) {  // the shrink share is done: the expand share
-        in_shrink = false;
-        cur.start(p, P, n_shr + first_expand_task(P, p, e0), n_shr, total);
-      } else if (!more) {
-        t.shrink = -1;
-      }
-      if (!in_share()) t.shrink = -1;
+      if (!more || cur.task >= cend) take(__shfl_sync(FULL_MASK, claimed, 0));
     };
     QTask q0 = t;  // stage n
     publish(0, q0);
@@ -862,7 +829,10 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
   __syncthreads();
   if (last_cta) {
     for (int i = tid; i < S * p.n_groups; i += kQAll) ready[i] = 0;
-    if (tid == 0) ready[kFReadyCap] = 0;
+    if (tid == 0) {
+      ready[kFReadyCap] = 0;
+      ready[kFReadyCap + 1] = 0;
+    }
   }
 }
 

@@ -101,7 +101,7 @@ typedef enum {
   SLORA_DECODE_AUTO = 0,       /* the library's choice: 16-bit pools run calls of
                                   up to 16 tokens as one CTA per token (plain
                                   loads, no scratch: a latency-bound batch),
-                                  17..512 tokens on STREAM and larger calls on
+                                  17..1024 tokens on STREAM and larger calls on
                                   SPLIT; e4m3 pools take STREAM up to 1024
                                   tokens                                         */
   SLORA_DECODE_SPLIT = 1,      /* always three kernels: segment build, shrink,
@@ -112,8 +112,8 @@ typedef enum {
                                   in one launch); SPLIT above that               */
   SLORA_DECODE_STREAM = 3      /* one kernel of streaming stages for calls of up
                                   to 1024 tokens: every CTA plans the call and
-                                  takes an equal share of the shrink tasks, then
-                                  of the expand stages; a producer warp moves each
+                                  claims chunks of shrink tasks, then of expand
+                                  tasks, from a counter; a producer warp moves each
                                   stage's rank rows from the pages by bulk copies,
                                   the shrink runs on mma.sync.  SPLIT above 1024
                                   tokens                                         */

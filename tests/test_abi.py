@@ -488,13 +488,12 @@ def test_pool_convenience_methods():
 @pytest.mark.parametrize("fmt", [G.SLORA_WEIGHTS_16, G.SLORA_WEIGHTS_E4M3], ids=["16bit", "e4m3"])
 def test_decode_path_policy(fmt):
     """Kernels a decode call launches, per path and token count (host logic):
-    AUTO runs up to 16 tokens of a 16-bit pool as one CTA per token, 17..512
+    AUTO runs up to 16 tokens of a 16-bit pool as one CTA per token, 17..1024
     on the streaming-stage kernel and more on the three-kernel path; an e4m3
     pool takes the streaming kernel up to 1024 tokens; the one-kernel paths
     hand calls above 1024 tokens to the three-kernel path."""
     want = {
-        G.SLORA_DECODE_AUTO: {1: 1, 16: 1, 17: 1, 512: 1, 513: 3 if fmt == G.SLORA_WEIGHTS_16 else 1,
-                              1024: 3 if fmt == G.SLORA_WEIGHTS_16 else 1, 1025: 3},
+        G.SLORA_DECODE_AUTO: {1: 1, 16: 1, 17: 1, 512: 1, 513: 1, 1024: 1, 1025: 3},
         G.SLORA_DECODE_SPLIT: {1: 3, 256: 3, 1025: 3},
         G.SLORA_DECODE_FUSED: {1: 1, 1024: 1, 1025: 3},
         G.SLORA_DECODE_STREAM: {1: 1, 1024: 1, 1025: 3},
@@ -512,6 +511,8 @@ def test_decode_path_policy(fmt):
                 assert kind == G.SLORA_KIND_FUSED
             if path == G.SLORA_DECODE_AUTO and T <= 16 and fmt == G.SLORA_WEIGHTS_16:
                 assert kind == G.SLORA_KIND_TOKEN
+            if path == G.SLORA_DECODE_AUTO and (T > 16 or fmt != G.SLORA_WEIGHTS_16) and T <= 1024:
+                assert kind == G.SLORA_KIND_STREAM
         assert G.slora_decode_kernels(pool.h, 0) == 0
         assert G.slora_decode_kind(pool.h, 0) == G.SLORA_KIND_NONE
         pool.close()
