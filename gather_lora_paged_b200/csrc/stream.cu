@@ -5,8 +5,9 @@
 // LoRA serving: S-LoRA, Punica, SGMV, vLLM", SGMV section, and "Paper
 // explainer: S-LoRA", BGMV kernel section: tokens of one batch use different
 // adapters, fetched from paged memory by id) and each segment's task counts.
-// CTA b then takes an equal share of the shrink tasks and, after them, an
-// equal share (by stages) of the expand tasks:
+// The tasks -- all shrink tasks, then all expand tasks -- go out in chunks of
+// consecutive tasks: CTA b takes chunk b, then chunks it claims from a counter,
+// so that CTAs that run faster take more:
 //
 //   shrink (segment, x group, 8 rank rows, 2048 of d_in, up to 8 tokens):
 //       t_c[i, k] = sum_{j in chunk c} x[i, j] * A_a[j, k]
@@ -28,9 +29,10 @@
 // A producer warp walks the CTA's stages: page ids one stage ahead, the bulk
 // copies of the next stage into the other of two slots (a full / empty
 // mbarrier pair each), L2 prefetches of the x and y rows the consumers will
-// read.  The phases meet at one grid barrier (cooperative launch): expand
-// stages read the t partials of every CTA.  The last CTA to finish clears the
-// barrier count.  e4m3 pages: codes are widened exactly (every e4m3 value is
+// read.  An expand task reads the t partials that other CTAs wrote: it starts
+// once a count per (segment, x group), which producers add to as shrink
+// stages finish, shows them all (a bounded wait; the grid is co-resident by
+// cooperative launch).  The last CTA to finish clears the counts.  e4m3 pages: codes are widened exactly (every e4m3 value is
 // a 16-bit value of either type), and the per-rank-row scales multiply the
 // partials of A and the t entering the expand.
 #include "dev_common.cuh"
