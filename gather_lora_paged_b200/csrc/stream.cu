@@ -26,14 +26,18 @@
 //     Lane l owns 8 consecutive outputs and accumulates on the FMA pipe in
 //     fp32, rank rows in order, then rounds y once.
 //
-// A producer warp walks the CTA's stages: page ids one stage ahead, the bulk
-// copies of the next stage into the other of two slots (a full / empty
-// mbarrier pair each), L2 prefetches of the x and y rows the consumers will
-// read.  An expand task reads the t partials that other CTAs wrote: it starts
-// once a count per (segment, x group), which producers add to as shrink
-// stages finish, shows them all (a bounded wait; the grid is co-resident by
-// cooperative launch).  The last CTA to finish clears the counts.  e4m3 pages: codes are widened exactly (every e4m3 value is
-// a 16-bit value of either type), and the per-rank-row scales multiply the
+// Two producer warps feed the stages.  A planner warp walks the CTA's stage
+// sequence: it publishes each stage's descriptor, resolves the page ids of the
+// stage's rows and hands the bulk-copy pieces to an issuer warp, and prefetches
+// the x and y rows the consumers will read to L2.  The issuer copies each
+// stage into one of two slots (a full / empty mbarrier pair each) as soon as
+// the stage two before it has released the slot; consumers release a slot once
+// their share of it is in registers.  An expand task reads the t partials that
+// other CTAs wrote: it starts once a count per (segment, x group), which the
+// consumers add to as shrink stages finish, shows them all (a bounded wait;
+// the grid is co-resident by cooperative launch).  The last CTA to finish
+// clears the counts.  e4m3 pages: codes are widened exactly (every e4m3 value
+// is a 16-bit value of either type), and the per-rank-row scales multiply the
 // partials of A and the t entering the expand.
 #include "dev_common.cuh"
 
@@ -275,10 +279,11 @@ __device__ __forceinline__ QTask decode_task(const BgmvParams& p, const QPlan& P
 constexpr int kQRowBytes = 2 * kQKT + 64;
 constexpr int kQSlotBytes = kQRB * kQRowBytes;
 constexpr int kQNS = 2;                            // stage slots (copies run up to kQNS - 1 stages ahead)
-constexpr int kQND = 8;                            // descriptor ring (published two stages ahead)
+constexpr int kQND = 8;                            // descriptor ring (published up to kQNP + 1 stages ahead)
 constexpr int kQCTAs = kQNS <= 2 ? 2 : 1;          // resident CTAs per SM
+constexpr int kQNP = 3;                            // copy-piece records (planner -> issuer)
 constexpr int kQCons = 8;                          // consumer warps
-constexpr int kQAll = (kQCons + 1) * 32;           // + the producer warp
+constexpr int kQAll = (kQCons + 2) * 32;           // + the planner and issuer warps
 static_assert(kQCons * 32 == kQThreads, "consumers");
 
 __device__ __forceinline__ void bar_consumers() { asm volatile("bar.sync 1, %0;" ::"n"(kQThreads) : "memory"); }
@@ -343,7 +348,8 @@ __device__ __forceinline__ void load_x(const BgmvParams& p, const QPlan& P, cons
 
 template <int DT, int WF>
 __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, const QTask& t,
-                             const unsigned char* slot, const uint4 (&xc)[8]) {
+                             const unsigned char* slot, uint64_t* empty, const uint4 (&xc)[8],
+                             int flush_key, int flush_n) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, q = lane & 3, gr = lane >> 2;
   const int s = t.s, g = t.u, b = t.v, c = t.c;
   const int a = P.seg_adapter[s], r = P.seg_rank[s];
@@ -355,24 +361,38 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
   const int j0 = w * 256 + q * 8;  // in the chunk; step u adds 32
   const int jw = c * kQKT + j0;
   const unsigned char* arow = slot + gr * kQRowBytes;
+  // the warp's share of the slot into registers, then the slot is released
+  // (the issuer's next copy into it overlaps the arithmetic)
+  uint4 av[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    av[u] = make_uint4(0, 0, 0, 0);
+    if (rv && jw + 32 * u < d_in) {
+      if (WF == 0) {
+        av[u] = *reinterpret_cast<const uint4*>(arow + 2 * (j0 + 32 * u));
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(arow + (j0 + 32 * u));
+        av[u].x = v.x;
+        av[u].y = v.y;
+      }
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty);
   float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // two chains: steps u even / odd
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     float (&acc)[4] = acc2[u & 1];
     const bool in = jw + 32 * u < d_in;
     const uint4 xu = (xv && in) ? xc[u] : make_uint4(0, 0, 0, 0);
-    uint32_t bw[4] = {0u, 0u, 0u, 0u};
-    if (rv && in) {
-      if (WF == 0) {
-        const uint4 v = *reinterpret_cast<const uint4*>(arow + 2 * (j0 + 32 * u));
-        bw[0] = v.x; bw[1] = v.y; bw[2] = v.z; bw[3] = v.w;
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(arow + (j0 + 32 * u));
-        bw[0] = e4m3x2_to_16<DT>(v.x & 0xffffu);
-        bw[1] = e4m3x2_to_16<DT>(v.x >> 16);
-        bw[2] = e4m3x2_to_16<DT>(v.y & 0xffffu);
-        bw[3] = e4m3x2_to_16<DT>(v.y >> 16);
-      }
+    uint32_t bw[4];
+    if (WF == 0) {
+      bw[0] = av[u].x; bw[1] = av[u].y; bw[2] = av[u].z; bw[3] = av[u].w;
+    } else {
+      bw[0] = e4m3x2_to_16<DT>(av[u].x & 0xffffu);
+      bw[1] = e4m3x2_to_16<DT>(av[u].x >> 16);
+      bw[2] = e4m3x2_to_16<DT>(av[u].y & 0xffffu);
+      bw[3] = e4m3x2_to_16<DT>(av[u].y >> 16);
     }
     // contraction slots 2q, 2q+1 <- elements 0, 1; 2q+8, 2q+9 <- 2, 3 (then
     // 4..7); mma rows 8..15 (no tokens) stay zero
@@ -383,6 +403,12 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
   red[w * 64 + gr * 8 + 2 * q] = acc2[0][0] + acc2[1][0];
   red[w * 64 + gr * 8 + 2 * q + 1] = acc2[0][1] + acc2[1][1];
   bar_consumers();
+  // every consumer has passed the barrier, so the t partials of the earlier
+  // stages are written: a finished run of them is counted now
+  if (tid == 0 && flush_n > 0) {
+    __threadfence();
+    atomicAdd(p.sc.ready + flush_key, flush_n);
+  }
   if (tid < 64) {
     const int m = tid >> 3, nn = tid & 7, row = b * kQRB + nn;
     if (m < nt && row < nrows) {
@@ -402,10 +428,10 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
 // output chunk e, token group tg).  The first stage waits until every shrink
 // task of (s, the slot's x group) has been counted, then fills tS with t =
 // sum of the chunk partials; the last one adds s_a * acc to y (prefetched to
-// L2 by the producer) and rounds.
+// L2 by the planner) and rounds.
 template <int DT, int WF, int NT>
 __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, const QTask& t,
-                             const unsigned char* slot, float (&acc)[kQETok][8], int& tkey) {
+                             const unsigned char* slot, uint64_t* empty, float (&acc)[kQETok][8], int& tkey) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int s = t.s, a = P.seg_adapter[s], r = P.seg_rank[s];
   const int pos0 = P.seg_start[s] + t.w * kQETok;
@@ -414,6 +440,25 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
   const int jl = w * 256 + lane * 8;  // in the chunk
   const int col = t.v * kQECols + jl;
   const bool act = col < L.d_out;
+  // the thread's 8 outputs of the stage's rank rows into registers, then the
+  // slot is released (the issuer's next copy into it overlaps the rest)
+  uint4 bv[kQRB];
+#pragma unroll
+  for (int kk = 0; kk < kQRB; ++kk) {
+    bv[kk] = make_uint4(0, 0, 0, 0);
+    if (act && t.sub * kQRB + kk < r) {
+      const unsigned char* br = slot + kk * kQRowBytes;
+      if (WF == 0) {
+        bv[kk] = *reinterpret_cast<const uint4*>(br + 2 * jl);
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(br + jl);
+        bv[kk].x = v.x;
+        bv[kk].y = v.y;
+      }
+    }
+  }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(empty);
   if (t.sub == 0) {
 #pragma unroll
     for (int m = 0; m < NT; ++m)
@@ -461,9 +506,8 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
       const int k = t.sub * kQRB + kk;
       if (k >= r) break;  // warp-uniform
       float bf[8];
-      const unsigned char* br = slot + kk * kQRowBytes;
-      if (WF == 0) unpack8<DT>(*reinterpret_cast<const uint4*>(br + 2 * jl), bf);
-      else unpack8_q8(*reinterpret_cast<const uint2*>(br + jl), bf);
+      if (WF == 0) unpack8<DT>(bv[kk], bf);
+      else unpack8_q8(make_uint2(bv[kk].x, bv[kk].y), bf);
 #pragma unroll
       for (int m = 0; m < NT; ++m) {
         const float tk = tS[m * kQMaxR + k];
@@ -490,7 +534,7 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
   }
 }
 
-// The producer's walk over a chunk of tasks: the current task's fields kept
+// The planner's walk over a chunk of tasks: the current task's fields kept
 // alongside the counts they run through, so that the next task follows with
 // a few increments (the same order decode_task assigns: shrink tasks by
 // segment, x group, d_in chunk, rank-row block, token tile; expand tasks by
@@ -563,6 +607,13 @@ struct QCursor {
   }
 };
 
+// A lane's bulk copies of a stage: page ids, in-page byte offsets, offsets
+// in the slot, bytes (0: none).
+struct QPieces {
+  int32_t pg[2];
+  int ipo[2], dso[2], nb[2];
+};
+
 // Bytes of a stage's rows.
 template <int WF>
 __device__ __forceinline__ int stage_bytes(const BgmvParams& p, const QPlan& P, const QTask& t) {
@@ -589,6 +640,10 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
   __shared__ QTask sdesc[kQND];  // stage n's descriptor at n % kQND (written with dready[n % kQND])
   // per slot: bytes landed (full), consumed (empty)
   __shared__ __align__(8) uint64_t dready[kQND], full[kQNS], empty[kQNS];
+  // planner -> issuer: the copy pieces of stage n in record n % kQNP
+  __shared__ __align__(16) QPieces precs[kQNP][32];
+  __shared__ int pbytes[kQNP];
+  __shared__ __align__(8) uint64_t pready[kQNP], pfree[kQNP];
   __shared__ int warm_sink;
   extern __shared__ __align__(128) unsigned char ring[];  // 2 stage slots; the plan's histogram first
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -609,27 +664,34 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kQCons);
     }
+    for (int i = 0; i < kQNP; ++i) {
+      mbar_init(&pready[i], 1);
+      mbar_init(&pfree[i], 1);
+    }
     fence_mbar_init();
   }
   plan_call(p, P, reinterpret_cast<int*>(ring), ck, sh4, sh1);  // ends with a barrier
   const int S = P.S, n_shr = P.shr_pre[S], total = n_shr + P.exp_pre[S];
   if (warp == kQCons) {
-    // ---- producer warp: the CTA's stage sequence, page ids one stage ahead,
-    // one bulk copy per page piece of a stage row (lane: row lane / 4, pieces
-    // lane % 4 and lane % 4 + 4 of it)
+    // ---- planner warp: the CTA's stage sequence.  For stage m it publishes
+    // the descriptor (the consumers read it before the stage), resolves the
+    // page ids of the stage's rows and writes the bulk-copy pieces to record
+    // m % kQNP for the issuer (lane: row lane / 4, pieces lane % 4 and
+    // lane % 4 + 4 of it), and prefetches the x / y rows the consumers will
+    // read to L2.  A record is written one stage after its page-id loads were
+    // issued, so that their latency overlaps the next stage's work.
     //
     // The tasks are handed out in chunks of consecutive tasks: ksc shrink
     // tasks (about two chunks per CTA, a multiple of 4 up to 16) or kQExpChunk
-    // expand tasks, all shrink chunks first.  CTA b
-    // takes chunk b, then chunks claimed from a counter, each claim made when
-    // the chunk before it starts, so that its answer is there when needed.
+    // expand tasks, all shrink chunks first.  CTA b takes chunk b, then chunks
+    // claimed from a counter when the one before is used up (the planner runs
+    // up to kQNP stages ahead of the copies, which hides the claim's latency).
     // Claims only grow, so a CTA runs all its shrink chunks before any expand
     // chunk, and an expand task never waits on a shrink task queued behind it.
     const int ksc = min(16, max(4, (n_shr / (2 * (int)gridDim.x) + 2) / 4 * 4));
     const int n_sc = cdiv_i(n_shr, ksc);
     const int n_chunks = n_sc + cdiv_i(total - n_shr, kQExpChunk);
     int* claim = ready + kFReadyCap + 1;
-    int claimed = 0;  // lane 0: the chunk after the current one
     int cend = 0;     // the current chunk's end (task index)
     QCursor cur;
     auto take = [&](int c) {
@@ -640,17 +702,12 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
       const int f = c < n_sc ? c * ksc : n_shr + (c - n_sc) * kQExpChunk;
       cend = c < n_sc ? min(f + ksc, n_shr) : min(f + kQExpChunk, total);
       cur.start(p, P, f, n_shr, total);
-      if (lane == 0) claimed = (int)gridDim.x + atomicAdd(claim, 1);
     };
     take(blockIdx.x);
     QTask& t = cur.t;
     const int i = lane >> 2, qp = lane & 3;
     const int sh = p.pool.page_shift + WF;
-    struct Pieces {
-      int32_t pg[2];
-      int ipo[2], dso[2], nb[2];  // in-page byte offset, destination offset in the slot, bytes
-    };
-    auto resolve = [&](const QTask& tt, Pieces& pc) {
+    auto resolve = [&](const QTask& tt, QPieces& pc) {
       const int32_t* list = nullptr;
       int64_t f0 = 0;
       int L = 0;
@@ -672,8 +729,14 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     };
     // L2 prefetch of what the consumers read besides the slot: a shrink
     // stage's x rows, an expand task's y rows (with its first stage)
+    int xkey = -1;  // the x pieces last prefetched: consecutive rank-row blocks share them
     auto prefetch_xy = [&](const QTask& tt) {
       if (tt.shrink < 0 || (tt.shrink == 0 && tt.sub > 0)) return;
+      if (tt.shrink) {
+        const int k = ((tt.s * 128 + tt.w) * 16 + tt.c) * 8 + tt.u;
+        if (k == xkey) return;
+        xkey = k;
+      }
       const int pos0 = P.seg_start[tt.s] + tt.w * (tt.shrink ? kQSTok : kQETok);
       const int nt = min(tt.shrink ? kQSTok : kQETok, P.seg_start[tt.s + 1] - pos0);
       const uint16_t* base;
@@ -698,79 +761,76 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
           asm volatile("prefetch.global.L2 [%0];" ::"l"(base + (int64_t)P.perm[pos0 + m] * ld + c0 + col));
       }
     };
-    const unsigned char* pool = reinterpret_cast<const unsigned char*>(p.pool.pool);
-    // Descriptors go to a ring of kQND two stages before their stage (the
-    // consumers load x from them); copies go to the stage's slot once the stage
-    // kQNS before it has released the slot.
     auto publish = [&](int n, const QTask& tt) {
       if (lane == 0) sdesc[n % kQND] = tt;
       __syncwarp();
       if (lane == 0) mbar_arrive(&dready[n % kQND]);
     };
-    // Counts of finished shrink stages per (segment, x group): a stage is
-    // finished once its slot is released.  A pair's stages are consecutive in
-    // the CTA's sequence; their count is added (lane 0, after a fence) when
-    // the last of them is released, which never waits on a later stage.
-    int run_n = 0;
-    auto count = [&](const QTask& done, const QTask& after) {
-      if (done.shrink != 1) return;
-      const int key = done.s * p.n_groups + done.u;
-      ++run_n;
-      if (after.shrink != 1 || after.s * p.n_groups + after.u != key) {
-        if (lane == 0) {
-          __threadfence();
-          atomicAdd(ready + key, run_n);
-        }
-        run_n = 0;
-      }
-    };
-    // the cursor runs two stages ahead of the copies: stage n + 2 is published
-    // while stage n's copies wait for their slot
     auto advance = [&]() {
       if (t.shrink < 0) return;
       const bool more = cur.next(p, P);
-      if (!more || cur.task >= cend) take(__shfl_sync(FULL_MASK, claimed, 0));
+      if (!more || cur.task >= cend) {
+        int c = 0;
+        if (lane == 0) c = (int)gridDim.x + atomicAdd(claim, 1);
+        take(__shfl_sync(FULL_MASK, c, 0));
+      }
     };
-    QTask q0 = t;  // stage n
-    publish(0, q0);
-    advance();
-    QTask q1 = t;  // stage n + 1
-    publish(1, q1);
-    advance();     // the cursor: stage n + 2
-    Pieces pc_cur, pc_next;
-    resolve(q0, pc_cur);
-    prefetch_xy(q0);
+    auto write = [&](int mm, const QPieces& pc, int bytes) {
+      precs[mm % kQNP][lane] = pc;
+      if (lane == 0) pbytes[mm % kQNP] = bytes;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pready[mm % kQNP]);
+    };
+    // Two piece sets alternate between the stage being resolved and the one
+    // being written (the loop body runs twice per pass).
+    QPieces pcA{}, pcB{};
+    int byA = 0, byB = 0;
+    int m = 0;
+    auto step = [&](QPieces& pc_new, int& by_new, const QPieces& pc_prev, int by_prev) -> bool {
+      if (m >= kQNP) mbar_wait(&pfree[m % kQNP], (m / kQNP - 1) & 1, p.pool.err);
+      publish(m, t);
+      by_new = -1;  // -1: the end of the CTA's stages
+      if (t.shrink >= 0) {
+        resolve(t, pc_new);
+        by_new = stage_bytes<WF>(p, P, t);
+      }
+      if (m >= 1) write(m - 1, pc_prev, by_prev);
+      if (t.shrink < 0) {
+        write(m, pc_prev, -1);
+        return false;
+      }
+      prefetch_xy(t);
+      advance();
+      ++m;
+      return true;
+    };
+    while (step(pcA, byA, pcB, byB) && step(pcB, byB, pcA, byA)) {
+    }
+  } else if (warp == kQCons + 1) {
+    // ---- issuer warp: record n's copies into slot n % kQNS once stage
+    // n - kQNS has released it, then record n back to the planner
+    const unsigned char* pool = reinterpret_cast<const unsigned char*>(p.pool.pool);
     int n = 0;
     for (;; ++n) {
-      const int slot = n % kQNS;
-      if (q0.shrink >= 0) {
-        publish(n + 2, t);
-        resolve(q1, pc_next);  // stage n + 1: its page ids on the way, its x / y rows to L2
-        prefetch_xy(q1);
-      }
-      if (n >= kQNS) {  // stage n - kQNS has released the slot (its descriptor is still in the ring)
-        mbar_wait(&empty[slot], (n / kQNS - 1) & 1, p.pool.err);
-        count(sdesc[(n - kQNS) % kQND], sdesc[(n - kQNS + 1) % kQND]);
-      }
-      if (q0.shrink < 0) break;
-      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)stage_bytes<WF>(p, P, q0));
+      const int rq = n % kQNP, slot = n % kQNS;
+      mbar_wait(&pready[rq], (n / kQNP) & 1, p.pool.err);
+      const int bytes = pbytes[rq];
+      if (bytes < 0) break;
+      const QPieces pc = precs[rq][lane];
+      if (n >= kQNS) mbar_wait(&empty[slot], (n / kQNS - 1) & 1, p.pool.err);
+      if (lane == 0) mbar_expect_tx(&full[slot], (uint32_t)bytes);
       __syncwarp();
       unsigned char* dst = ring + slot * kQSlotBytes;
 #pragma unroll
       for (int h = 0; h < 2; ++h)
-        if (pc_cur.nb[h] > 0)
-          bulk_g2s(dst + pc_cur.dso[h], pool + ((int64_t)pc_cur.pg[h] << (p.pool.page_shift + 1)) + pc_cur.ipo[h],
-                   (uint32_t)pc_cur.nb[h], &full[slot]);
-      pc_cur = pc_next;
-      q0 = q1;
-      q1 = t;
-      advance();
+        if (pc.nb[h] > 0)
+          bulk_g2s(dst + pc.dso[h], pool + ((int64_t)pc.pg[h] << (p.pool.page_shift + 1)) + pc.ipo[h],
+                   (uint32_t)pc.nb[h], &full[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pfree[rq]);
     }
-    // the last stages are counted once released (stage n is the end marker)
-    for (int k = max(0, n - kQNS + 1); k < n; ++k) {
-      mbar_wait(&empty[k % kQNS], (k / kQNS) & 1, p.pool.err);
-      count(sdesc[k % kQND], sdesc[(k + 1) % kQND]);
-    }
+    // the last stages' slots released (stage n is the end marker)
+    for (int k = max(0, n - kQNS + 1); k < n; ++k) mbar_wait(&empty[k % kQNS], (k / kQNS) & 1, p.pool.err);
   } else {
     // ---- consumer warps.  A CTA's stages are its shrink tasks, then its
     // expand tasks: two loops, so that the x pieces (shrink) and the output
@@ -793,16 +853,34 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
         }
       };
       x_for(t);
+      // Counts of finished shrink stages per (segment, x group), which the
+      // expand tasks wait on: a run of consecutive stages with one key is
+      // added once, at the next shrink stage's reduction barrier, or after
+      // the last shrink stage (before any expand stage, which may wait on it).
+      int run_key = 0, run_n = 0;
       for (; t.shrink == 1; ++n) {
         const int slot = n % kQNS;
+        const int key = t.s * p.n_groups + t.u;
+        int fk = 0, fn = 0;
+        if (key != run_key) {
+          fk = run_key;
+          fn = run_n;
+          run_key = key;
+          run_n = 0;
+        }
+        ++run_n;
         mbar_wait(&full[slot], (n / kQNS) & 1, p.pool.err);
-        shrink_stage<DT, WF>(p, P, red[n & 1], t, ring + slot * kQSlotBytes, xq);
-        // the next stage's descriptor (and x) before this slot is released
+        shrink_stage<DT, WF>(p, P, red[n & 1], t, ring + slot * kQSlotBytes, &empty[slot], xq, fk, fn);
         mbar_wait(&dready[(n + 1) % kQND], ((n + 1) / kQND) & 1, p.pool.err);
         t = sdesc[(n + 1) % kQND];
         x_for(t);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
+      }
+      if (run_n > 0) {
+        bar_consumers();
+        if (tid == 0) {
+          __threadfence();
+          atomicAdd(ready + run_key, run_n);
+        }
       }
     }
     float acc[kQETok][8];
@@ -812,13 +890,11 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
       mbar_wait(&full[slot], (n / kQNS) & 1, p.pool.err);
       const unsigned char* sl = ring + slot * kQSlotBytes;
       const int nt = min(kQETok, P.seg_start[t.s + 1] - P.seg_start[t.s] - t.w * kQETok);
-      if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, acc, tkey);
-      else if (nt == 2) expand_stage<DT, WF, 2>(p, P, tS, t, sl, acc, tkey);
-      else expand_stage<DT, WF, 4>(p, P, tS, t, sl, acc, tkey);
+      if (nt == 1) expand_stage<DT, WF, 1>(p, P, tS, t, sl, &empty[slot], acc, tkey);
+      else if (nt == 2) expand_stage<DT, WF, 2>(p, P, tS, t, sl, &empty[slot], acc, tkey);
+      else expand_stage<DT, WF, 4>(p, P, tS, t, sl, &empty[slot], acc, tkey);
       mbar_wait(&dready[(n + 1) % kQND], ((n + 1) / kQND) & 1, p.pool.err);
       t = sdesc[(n + 1) % kQND];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
     }
   }
   // the last CTA to finish clears the counters for the next call
