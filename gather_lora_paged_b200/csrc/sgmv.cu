@@ -205,7 +205,6 @@ __global__ void __launch_bounds__(kShrinkThreads, 1) k_sgmv_shrink(const __grid_
   const int row0 = seg0 + m * kBM;
   const int KB = G.d_in / kBK;
   const int ST = p.stages;
-  const int a_bytes = NT * 128;
   const int stage_bytes = MQ * kXTileBytes + ((p.ntot_max * 128 + 1023) & ~1023);
   uint32_t ncols = 32;
   while ((int)ncols < nq * NT) ncols <<= 1;

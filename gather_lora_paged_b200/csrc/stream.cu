@@ -72,12 +72,8 @@ struct QPlan {
   int sum_ne;                   // output chunks over the call's slots
 };
 
-// Reads of data written earlier in this kernel by other CTAs (L2, not L1).
-__device__ __forceinline__ float ld_cg_f32(const float* p) {
-  float v;
-  asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
-  return v;
-}
+// A count that other CTAs add to in this kernel (acquire: the data it
+// counts is visible once the count is).
 __device__ __forceinline__ int ld_acquire_s32(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -493,13 +489,24 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
     for (int v = tid; v < nt * r; v += kQThreads) {
       const int m = v / r, kk = v - m * r;
       const float* src = L.t + (int64_t)(pos0 + m) * L.t_rs + (int64_t)kk * L.t_ns;
-      float sum = ld_cg_f32(src);
-      for (int c = 1; c < L.t_ns; ++c) sum += ld_cg_f32(src + c);
+      // the chunk partials of (token, k) are contiguous: up to 4 loads in
+      // flight at once (from L2: other CTAs wrote them in this kernel),
+      // summed in chunk order
+      float sum = 0.f;
+      for (int c0 = 0; c0 < L.t_ns; c0 += 4) {
+        float v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] = c0 + c < L.t_ns ? __ldcg(src + c0 + c) : 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c0 + c < L.t_ns) sum = c0 + c == 0 ? v[c] : sum + v[c];
+      }
       if (WF == 1) sum *= p.pool.qscale[(((int64_t)a * p.pool.n_proj + L.proj) * 2 + 1) * p.pool.max_rank + kk];
       tS[m * kQMaxR + kk] = sum;
     }
     bar_consumers();
   }
+  const bool last = t.sub == cdiv_i(r, kQRB) - 1;
   if (act) {
 #pragma unroll
     for (int kk = 0; kk < kQRB; ++kk) {
@@ -515,7 +522,7 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
         for (int i = 0; i < 8; ++i) acc[m][i] = fmaf(tk, bf[i], acc[m][i]);
       }
     }
-    if (t.sub == cdiv_i(r, kQRB) - 1) {
+    if (last) {
       const float sa = p.pool.scale[a];
 #pragma unroll
       for (int m = 0; m < NT; ++m) {
