@@ -690,14 +690,18 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     //
     // The tasks are handed out in chunks of consecutive tasks: ksc shrink
     // tasks (about two chunks per CTA, a multiple of 4 up to 16) or kQExpChunk
-    // expand tasks, all shrink chunks first.  CTA b takes chunk b, then chunks
+    // expand tasks (single tasks at the end), all shrink chunks first.  CTA b takes chunk b, then chunks
     // claimed from a counter when the one before is used up (the planner runs
     // up to kQNP stages ahead of the copies, which hides the claim's latency).
     // Claims only grow, so a CTA runs all its shrink chunks before any expand
     // chunk, and an expand task never waits on a shrink task queued behind it.
     const int ksc = min(16, max(4, (n_shr / (2 * (int)gridDim.x) + 2) / 4 * 4));
     const int n_sc = cdiv_i(n_shr, ksc);
-    const int n_chunks = n_sc + cdiv_i(total - n_shr, kQExpChunk);
+    // expand: chunks of kQExpChunk tasks, then single tasks for the last
+    // n_tail (two per CTA: the end of the kernel balances finer)
+    const int n_exp = total - n_shr, n_tail = min(n_exp, 2 * (int)gridDim.x);
+    const int n_ec = cdiv_i(n_exp - n_tail, kQExpChunk);
+    const int n_chunks = n_sc + n_ec + n_tail;
     int* claim = ready + kFReadyCap + 1;
     int cend = 0;     // the current chunk's end (task index)
     QCursor cur;
@@ -706,8 +710,17 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
         cur.t.shrink = -1;
         return;
       }
-      const int f = c < n_sc ? c * ksc : n_shr + (c - n_sc) * kQExpChunk;
-      cend = c < n_sc ? min(f + ksc, n_shr) : min(f + kQExpChunk, total);
+      int f;
+      if (c < n_sc) {
+        f = c * ksc;
+        cend = min(f + ksc, n_shr);
+      } else if (c < n_sc + n_ec) {
+        f = n_shr + (c - n_sc) * kQExpChunk;
+        cend = min(f + kQExpChunk, total - n_tail);
+      } else {
+        f = total - n_tail + (c - n_sc - n_ec);
+        cend = f + 1;
+      }
       cur.start(p, P, f, n_shr, total);
     };
     take(blockIdx.x);
