@@ -120,7 +120,22 @@ __device__ __forceinline__ void unpack8_q8(const uint2& v, float* f) {
 // reported by CTA 0 and, like rank-0 adapters and id -1, leave y unchanged.
 constexpr int kRankShift = 21;
 
-__device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int4* sh4, int* sh1) {
+// The batch's adapter ids and their ranks, loaded at the kernel's entry so
+// that the two dependent loads overlap the rest of the prologue.
+constexpr int kQTokU = kFMaxT / kQThreads;  // tokens per worker thread
+__device__ __forceinline__ void plan_load(const BgmvParams& p, int (&key)[kQTokU], int (&rk)[kQTokU]) {
+  const int tid = threadIdx.x, MA = p.pool.max_adapters;
+#pragma unroll
+  for (int u = 0; u < kQTokU; ++u) {
+    const int i = tid + u * kQThreads;
+    key[u] = tid < kQThreads && i < p.T ? p.idx[i] : -1;
+  }
+#pragma unroll
+  for (int u = 0; u < kQTokU; ++u) rk[u] = key[u] >= 0 && key[u] < MA ? p.pool.rank[key[u]] : 0;
+}
+
+__device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int4* sh4, int* sh1,
+                          int (&key)[kQTokU], const int (&rk)[kQTokU]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool worker = tid < kQThreads;  // token work: the first kQThreads threads
   const int T = p.T, MA = p.pool.max_adapters;
@@ -136,18 +151,17 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     P.sum_ne = c;
   }
   __syncthreads();
-  int key[kFMaxT / kQThreads];
 #pragma unroll
-  for (int u = 0; u < kFMaxT / kQThreads; ++u) {
+  for (int u = 0; u < kQTokU; ++u) {
     const int i = tid + u * kQThreads;
     int a = -1;
     if (worker && i < T) {
-      a = p.idx[i];
+      a = key[u];
       if (a < -1 || a >= MA) {
         if (blockIdx.x == 0) record_error(p.pool.err, 1, i);
         a = -1;
       } else if (a >= 0) {
-        const int r = p.pool.rank[a];
+        const int r = rk[u];
         if (r < 0 && blockIdx.x == 0) record_error(p.pool.err, 2, i);
         if (r <= 0) {
           a = -1;
@@ -203,7 +217,7 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
   // among its adapter's tokens of the chunk is the number of equal keys in
   // earlier warps plus the number in earlier lanes of its own warp.
 #pragma unroll
-  for (int u = 0; u < kFMaxT / kQThreads; ++u) {
+  for (int u = 0; u < kQTokU; ++u) {
     if (u * kQThreads >= T) break;
     const int a = key[u];
     if (worker) ck[tid] = a;
@@ -655,6 +669,8 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
   extern __shared__ __align__(128) unsigned char ring[];  // 2 stage slots; the plan's histogram first
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* ready = p.sc.ready;
+  int key[kQTokU], rk[kQTokU];
+  plan_load(p, key, rk);
   {  // every 64-byte line of the parameter block at once: the plan's first
      // lookups into the group and slot tables would otherwise each wait on a
      // cold constant-cache miss
@@ -677,7 +693,7 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     }
     fence_mbar_init();
   }
-  plan_call(p, P, reinterpret_cast<int*>(ring), ck, sh4, sh1);  // ends with a barrier
+  plan_call(p, P, reinterpret_cast<int*>(ring), ck, sh4, sh1, key, rk);  // ends with a barrier
   const int S = P.S, n_shr = P.shr_pre[S], total = n_shr + P.exp_pre[S];
   if (warp == kQCons) {
     // ---- planner warp: the CTA's stage sequence.  For stage m it publishes
@@ -686,7 +702,8 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
     // m % kQNP for the issuer (lane: row lane / 4, pieces lane % 4 and
     // lane % 4 + 4 of it), and prefetches the x / y rows the consumers will
     // read to L2.  A record is written one stage after its page-id loads were
-    // issued, so that their latency overlaps the next stage's work.
+    // issued, so that their latency overlaps the next stage's work (the first
+    // stage's record at once).
     //
     // The tasks are handed out in chunks of consecutive tasks: ksc shrink
     // tasks (about two chunks per CTA, a multiple of 4 up to 16) or kQExpChunk
@@ -814,7 +831,8 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
         resolve(t, pc_new);
         by_new = stage_bytes<WF>(p, P, t);
       }
-      if (m >= 1) write(m - 1, pc_prev, by_prev);
+      if (m >= 2) write(m - 1, pc_prev, by_prev);
+      if (m == 0 && t.shrink >= 0) write(0, pc_new, by_new);  // the first stage at once
       if (t.shrink < 0) {
         write(m, pc_prev, -1);
         return false;
