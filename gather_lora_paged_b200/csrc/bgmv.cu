@@ -612,6 +612,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_shrink(const __grid_constan
           default: shrink_consume<SLORA_F16, 4>(p, t, st, buf, xb); break;
         }
       }
+      // the slot's generic-proxy reads before the next bulk copy into it
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");
@@ -920,6 +922,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_expand(const __grid_constan
         case 2: expand_consume<DT, 2>(p, t, st, buf, yb, acc); break;
         default: expand_consume<DT, 4>(p, t, st, buf, yb, acc); break;
       }
+      // the slot's generic-proxy reads before the next bulk copy into it
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring])) : "memory");

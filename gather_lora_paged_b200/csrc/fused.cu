@@ -946,6 +946,8 @@ __global__ void __launch_bounds__(kFThreads, 1) k_delta(const __grid_constant__ 
           default: f_expand<DT, 4, WF>(p, t, cw, buf, xyb, qs, acc); break;
         }
       }
+      // the slot's generic-proxy reads before the next bulk copy into it
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring_i])) : "memory");

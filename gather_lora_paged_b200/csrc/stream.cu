@@ -236,6 +236,10 @@ __device__ void plan_call(const BgmvParams& p, QPlan& P, int* hist, int* ck, int
     if (a >= 0 && lane == __ffs(m) - 1) atomicAdd(&hist[a], __popc(m));
     __syncthreads();
   }
+  // the histogram lives in the stage slots, which bulk copies (async proxy)
+  // fill next: its generic-proxy accesses are ordered before them
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -372,7 +376,10 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
   const int jw = c * kQKT + j0;
   const unsigned char* arow = slot + gr * kQRowBytes;
   // the warp's share of the slot into registers, then the slot is released
-  // (the issuer's next copy into it overlaps the arithmetic)
+  // (the issuer's next copy into it overlaps the arithmetic).  The proxy
+  // fence orders these generic-proxy reads before the bulk copy (async
+  // proxy) that will overwrite the slot: without it, a copy issued right
+  // after the release could land before a read had taken its value.
   uint4 av[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
@@ -387,6 +394,7 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
       }
     }
   }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
   if (lane == 0) mbar_arrive(empty);
   float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // two chains: steps u even / odd
@@ -412,13 +420,12 @@ __device__ void shrink_stage(const BgmvParams& p, const QPlan& P, float* red, co
   // warp partials: red[w][token][row]; D row gr, columns 2q, 2q + 1
   red[w * 64 + gr * 8 + 2 * q] = acc2[0][0] + acc2[1][0];
   red[w * 64 + gr * 8 + 2 * q + 1] = acc2[0][1] + acc2[1][1];
+  // A run of stages that ended with the previous one is counted at this
+  // barrier: the threads that wrote its t partials (tid < 64) make them
+  // visible to the whole GPU first, then one thread adds the count.
+  if (flush_n > 0 && tid < 64) __threadfence();
   bar_consumers();
-  // every consumer has passed the barrier, so the t partials of the earlier
-  // stages are written: a finished run of them is counted now
-  if (tid == 0 && flush_n > 0) {
-    __threadfence();
-    atomicAdd(p.sc.ready + flush_key, flush_n);
-  }
+  if (tid == 0 && flush_n > 0) atomicAdd(p.sc.ready + flush_key, flush_n);
   if (tid < 64) {
     const int m = tid >> 3, nn = tid & 7, row = b * kQRB + nn;
     if (m < nt && row < nrows) {
@@ -451,7 +458,8 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
   const int col = t.v * kQECols + jl;
   const bool act = col < L.d_out;
   // the thread's 8 outputs of the stage's rank rows into registers, then the
-  // slot is released (the issuer's next copy into it overlaps the rest)
+  // slot is released (the issuer's next copy into it overlaps the rest; the
+  // proxy fence as in the shrink stage)
   uint4 bv[kQRB];
 #pragma unroll
   for (int kk = 0; kk < kQRB; ++kk) {
@@ -467,6 +475,7 @@ __device__ void expand_stage(const BgmvParams& p, const QPlan& P, float* tS, con
       }
     }
   }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
   if (lane == 0) mbar_arrive(empty);
   if (t.sub == 0) {
@@ -914,11 +923,9 @@ __global__ void __launch_bounds__(kQAll, kQCTAs) k_stream(const __grid_constant_
         x_for(t);
       }
       if (run_n > 0) {
+        if (tid < 64) __threadfence();  // the writers' t partials, as at a stage's barrier
         bar_consumers();
-        if (tid == 0) {
-          __threadfence();
-          atomicAdd(ready + run_key, run_n);
-        }
+        if (tid == 0) atomicAdd(ready + run_key, run_n);
       }
     }
     float acc[kQETok][8];

@@ -230,6 +230,36 @@ def test_full_size_configs_stream(cfg):
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
+def test_stream_many_calls_bit_identical(cfg):
+    """Forty calls of the streaming-stage kernel on one pool, L2 flushed before
+    each, give the same bits every time.  The schedule (which CTA takes which
+    chunk of tasks, when a stage's copy lands) differs from call to call while
+    the arithmetic order does not, so a difference can only come from a race:
+    an expand task reading t partials before they are visible, or a bulk copy
+    overwriting a stage slot before every read of it has taken its value."""
+    import hashlib
+    import torch
+    w = W.config(cfg)
+    pb = H.PoolBuild(w, decode_path=G.SLORA_DECODE_STREAM)
+    ten = H.Tensors(w)
+    idx = torch.from_numpy(w.idx).cuda()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    digests = []
+    for _ in range(40):
+        ten.reset()
+        flush.zero_()
+        G.slora_lora_delta(pb.h, *ten.args(), idx, w.T)
+        torch.cuda.synchronize()
+        assert G.slora_check_device(pb.h)[0] == 0
+        h = hashlib.sha1()
+        for t in ten.y:
+            h.update(H.from_device(t).tobytes())
+        digests.append(h.hexdigest())
+    assert len(set(digests)) == 1, [i for i, d in enumerate(digests) if d != digests[0]]
+    pb.close()
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
 def test_full_size_configs(cfg):
     """LLaMA-7B (fp16, 1000 adapters r=16, Zipf 1.0, T=256) and LLaMA-13B (bf16,
     2000 adapters r in {8..64}, Zipf 1.2, shuffled pool, T=512) decode layers,
