@@ -229,9 +229,10 @@ def test_full_size_configs_stream(cfg):
     pb.close()
 
 
+@pytest.mark.parametrize("path", [G.SLORA_DECODE_STREAM, G.SLORA_DECODE_FUSED], ids=["stream", "fused"])
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_stream_many_calls_bit_identical(cfg):
-    """Forty calls of the streaming-stage kernel on one pool, L2 flushed before
+def test_one_kernel_many_calls_bit_identical(cfg, path):
+    """Forty calls of a one-kernel decode path on one pool, L2 flushed before
     each, give the same bits every time.  The schedule (which CTA takes which
     chunk of tasks, when a stage's copy lands) differs from call to call while
     the arithmetic order does not, so a difference can only come from a race:
@@ -240,7 +241,7 @@ def test_stream_many_calls_bit_identical(cfg):
     import hashlib
     import torch
     w = W.config(cfg)
-    pb = H.PoolBuild(w, decode_path=G.SLORA_DECODE_STREAM)
+    pb = H.PoolBuild(w, decode_path=path)
     ten = H.Tensors(w)
     idx = torch.from_numpy(w.idx).cuda()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
