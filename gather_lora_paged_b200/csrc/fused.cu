@@ -948,6 +948,10 @@ __global__ void __launch_bounds__(kFThreads, 1) k_delta(const __grid_constant__ 
       }
       // the slot's generic-proxy reads before the next bulk copy into it
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // a shrink task's t partials, stored by every lane, visible to the whole
+      // GPU before the signaller counts the task (another warp's fence alone
+      // does not order this warp's stores)
+      if (last && t.kind == 1) __threadfence();
       __syncwarp();
       if (lane == 0) {
         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[ring_i])) : "memory");
