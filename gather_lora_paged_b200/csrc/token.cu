@@ -16,7 +16,7 @@ namespace slora {
 
 namespace {
 
-constexpr int kTThreads = 256;  // 8 warps
+constexpr int kTThreads = 512;  // 16 warps
 constexpr int kTMaxR = 128;
 constexpr int kTMaxList = 4096; // page-list entries staged in shared memory
 
