@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kTThreads) k_token(const __grid_constant__ Bgm
     for (int64_t f = (int64_t)tid * 64; f < n; f += kTThreads * 64)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(page_ptr(p.pool, list[L.listB + (f >> p.pool.page_shift)], f)));
   }
-  // shrink: warp w takes the (slot, rank row) pairs w, w + 8, ...; lane l the
+  // shrink: warp w takes the (slot, rank row) pairs w, w + 16, ...; lane l the
   // 8-element pieces l, l + 32, ... of the row; four chains per lane
   const int pairs = p.n_slots * r;
   for (int q = warp; q < pairs; q += kTThreads / 32) {
